@@ -1,0 +1,505 @@
+#!/usr/bin/env python
+"""Benchmark of the DSA hot path on B200: indexer -> top-k -> sparse attention (+ gate).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config c2] [--impl reference]
+
+One step is one pass of the whole path over one batch of the workload, with inputs resident
+in HBM.  Times are CUDA events on the launching stream around each library call; L2 is
+flushed (a 512 MB write) between steps, outside the timed events.  Prints one JSON line.
+
+Multi-GPU: one process per GPU (torchrun); each rank runs its own copy of the workload
+(the path has no exchange step: weak scaling), the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from workloads import dsa_inputs, get_config, swa_inputs  # noqa: E402
+
+METRIC = "query-tokens/s (indexer+top-k+sparse attn) and % of tensor/HBM roofline"
+UNIT = "query-tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# float32 FMA peak of the CUDA cores: 148 SMs x 128 FMA/clk x 2 flop x 1.965 GHz.
+F32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+# DRAM traffic per launch from committed ncu captures: (kernel, config) -> (bytes,
+# sha256 of the kernel source when captured).  Reported as null when the source changed.
+NCU_TRAFFIC = {}
+
+
+# ----------------------------------------------------------------------------- helpers
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS if k in d}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def src_sha(name):
+    p = os.path.join(ROOT, "sparse_attention_15_b200", "csrc", name)
+    with open(p, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def causal_pairs(S, T, B, q_off):
+    # number of (query, key) pairs with t <= s + q_off, over all batch rows
+    n = np.minimum(np.arange(S, dtype=np.int64) + q_off + 1, T)
+    return int(B * n.sum())
+
+
+def selected_pairs(S, T, B, q_off, K):
+    n = np.minimum(np.arange(S, dtype=np.int64) + q_off + 1, T)
+    return int(B * np.minimum(n, K).sum())
+
+
+class ClockSampler:
+    """nvidia-smi sampling (200 ms) of the GPU this process uses, during the timed region."""
+
+    FIELDS = ("pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.samples = []
+        self.proc = None
+        self.t_start = self.t_stop = None
+        try:
+            pci = torch.cuda.get_device_properties(device).pci_bus_id.lower()
+        except Exception:
+            pci = None
+        self.pci = pci
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), [x.strip() for x in line.split(",")]))
+
+    def mark(self, which):
+        setattr(self, which, time.time())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = [(t, f) for t, f in self.samples if len(f) >= 9 and
+                (self.pci is None or self.pci.endswith(f[0].lower()[-12:]) or
+                 f[0].lower().endswith(self.pci[-12:]))]
+        if not rows:
+            return None
+        win = [f for t, f in rows if self.t_start and self.t_stop and
+               self.t_start - 0.2 <= t <= self.t_stop + 0.2] or [f for _, f in rows]
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return float("nan")
+
+        sm = [num(f[1]) for f in win]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for f in win:
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": num(win[0][2]),
+                "reasons": sorted(reasons), "samples": len(win),
+                "power_w_max": max(num(f[3]) for f in win)}
+
+
+# ----------------------------------------------------------------------------- workloads
+class Workload:
+    """Device buffers and the library calls of one step of config `name`."""
+
+    def __init__(self, name, device, seed_offset=0):
+        import sparse_attention_15_b200 as dsa
+
+        self.dsa = dsa
+        self.cfg = cfg = get_config(name)
+        self.device = device
+        B = cfg.B
+        if name == "c4":  # 174 GB of expanded K/V cache: shrink the batch only if it cannot fit
+            free, _ = torch.cuda.mem_get_info(device)
+            per_row = cfg.T * (cfg.DI + cfg.H * (cfg.dqk + cfg.dv)) * 2
+            B = min(cfg.B, int((free - (6 << 30)) // per_row))
+            if B < 1:
+                raise RuntimeError("not enough device memory for one decode batch row")
+        self.B = B
+        x = dsa_inputs(cfg, device=device, B=B, seed=cfg.seed + seed_offset)
+        self.x = x
+        self.K = cfg.k_eff
+        self.scores = torch.empty((B, cfg.S, cfg.T), dtype=torch.float32, device=device)
+        self.idx = torch.empty((B, cfg.S, self.K), dtype=torch.int32, device=device)
+        self.out = torch.empty((B, cfg.S, cfg.H, cfg.dv), dtype=x["q"].dtype, device=device)
+        nb = dsa.dsa_sparse_attn_workspace_bytes(B, cfg.S, cfg.T, cfg.H, cfg.dv, self.K)
+        self.ws = torch.empty(max(nb, 16), dtype=torch.uint8, device=device)
+        self.ws_bytes = nb
+        self.swa = []
+        for layer in range(1, cfg.swa_layers + 1):
+            s = swa_inputs(cfg, layer, device=device, seed=cfg.seed + seed_offset)
+            s["out"] = torch.empty((B, cfg.S, cfg.H, cfg.dv), dtype=x["q"].dtype, device=device)
+            self.swa.append(s)
+        self.stages = ["indexer", "topk", "attention"] + [f"swa{i + 1}" for i in
+                                                          range(len(self.swa))]
+        self.launches_per_step = 3 + (1 if nb > 0 else 0) + len(self.swa)
+
+    def step(self, ev):
+        """Run one step; ev is a list of len(stages)+1 CUDA events recorded between calls."""
+        c, x, d = self.cfg, self.x, self.dsa
+        ev[0].record()
+        d.dsa_index_scores(x["q_idx"], x["k_idx"], x["w"], c.scale, scores=self.scores)
+        ev[1].record()
+        d.dsa_topk(self.scores, self.K, idx=self.idx)
+        ev[2].record()
+        d.dsa_sparse_attn(x["q"], x["k"], x["v"], self.idx, gate=x["gate"], out=self.out,
+                          ws=self.ws)
+        ev[3].record()
+        for i, s in enumerate(self.swa):
+            d.dsa_window_attn(s["q"], s["k"], s["v"], c.window, gate=s["gate"], out=s["out"])
+            ev[4 + i].record()
+
+    # algorithmic work per launch of each stage
+    def work(self):
+        c, B = self.cfg, self.B
+        es = 4 if c.dtype == "f32" else 2
+        pairs = causal_pairs(c.S, c.T, B, c.q_off)
+        sel = selected_pairs(c.S, c.T, B, c.q_off, self.K)
+        rows = B * c.S
+        w = {
+            "indexer": ("tensor" if c.dtype == "bf16" else "alu", 2.0 * c.HI * c.DI * pairs,
+                        "TFLOP/s"),
+            "topk": ("hbm", 4.0 * pairs + 4.0 * rows * self.K, "GB/s"),
+            "attention": ("hbm", sel * c.H * (c.dqk + c.dv) * es +
+                          rows * c.H * (c.dqk + c.dv) * es, "GB/s"),
+        }
+        for i in range(len(self.swa)):
+            band = selected_pairs(c.S, c.T, B, c.q_off, c.window)
+            w[f"swa{i + 1}"] = ("hbm", band * c.swa_kv_heads * (c.dqk + c.dv) * es +
+                                rows * c.H * (c.dqk + c.dv) * es, "GB/s")
+        return w
+
+    def host_copy(self):
+        """Pinned host copies of every input of the DSA layer (for the end-to-end leg)."""
+        return {k: (None if v is None else v.cpu().pin_memory()) for k, v in self.x.items()}
+
+    def e2e_step(self, host, dev_bufs, out_host):
+        """Host inputs -> device -> dsa_forward -> result back to the host."""
+        for k, v in host.items():
+            if v is not None:
+                dev_bufs[k].copy_(v, non_blocking=True)
+        x = dev_bufs
+        c = self.cfg
+        self.dsa.dsa_forward(x["q_idx"], x["k_idx"], x["w"], c.scale, c.K, x["q"], x["k"],
+                             x["v"], gate=x["gate"], out=self.out, idx_out=self.idx,
+                             ws=self.fwd_ws, ws_bytes=self.fwd_ws_bytes)
+        out_host.copy_(self.out, non_blocking=True)
+
+
+# ----------------------------------------------------------------------------- oracle timing
+def oracle_rows_per_s(cfg, x_host, rows, budget_s):
+    """The CPU oracle as it stands, on sampled query rows of batch row 0: returns
+    (rows done, seconds).  Each row runs scores -> top-k -> dense masked attention."""
+    from oracle import dsa_oracle as O
+
+    q_off = cfg.q_off
+    done = 0
+    t0 = time.perf_counter()
+    for s in rows:
+        sl = slice(s, s + 1)
+        sc = O.index_scores(x_host["q_idx"][:1, sl], x_host["k_idx"][:1], x_host["w"][:1, sl],
+                            cfg.scale, q_off=s + q_off)
+        idx = O.topk_indices(sc, cfg.k_eff, q_off=s + q_off)
+        g = None if x_host["gate"] is None else x_host["gate"][:1, sl]
+        O.sparse_attention(x_host["q"][:1, sl], x_host["k"][:1], x_host["v"][:1], idx,
+                           gate=g, gate_mode=cfg.gate, q_off=s + q_off)
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    return done, time.perf_counter() - t0
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def sample_rows(S, n):
+    return sorted(set(int(r) for r in np.linspace(0, S - 1, n)))
+
+
+def host_inputs(cfg, x, B_rows=1):
+    return {k: (None if v is None else v[:B_rows].cpu()) for k, v in x.items()}
+
+
+# ----------------------------------------------------------------------------- main
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        if world == 1 and args.gpus > 1:
+            sys.exit("bench.py --gpus N>1 must be launched with torchrun (one process per GPU)")
+    return world, rank, local
+
+
+def run_reference(args, world, rank):
+    """The reference arm: the CPU oracle, timed on bounded samples of the workload."""
+    if rank != 0:
+        return
+    cfg = get_config(args.config)
+    x = dsa_inputs(cfg, device="cpu", B=1)
+    per_step = {"c1": 16, "c2": 4, "c3": 1, "c4": 1, "c5": 1}[cfg.name]
+    rows_all = sample_rows(cfg.S, max(per_step * (args.steps + args.warmup), 1))
+    rng = np.random.default_rng(0)
+    rng.shuffle(rows_all)
+    it = iter(rows_all * 2)
+    for _ in range(args.warmup):
+        oracle_rows_per_s(cfg, x, [next(it) for _ in range(per_step)], 1e9)
+    total_rows, total_s = 0, 0.0
+    for _ in range(args.steps):
+        n, dt = oracle_rows_per_s(cfg, x, [next(it) for _ in range(per_step)], 1e9)
+        total_rows += n
+        total_s += dt
+    value = total_rows / total_s
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total_s / max(args.steps, 1), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(cfg, cfg.B if cfg.name != "c4" else cfg.B),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{per_step} query row(s) per step of batch row 0, spread "
+                                   f"over the {cfg.S} queries; float64 numpy oracle"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(cfg, B):
+    return {"workload": f"{cfg.name}: {cfg.description}", "B": B, "S": cfg.S, "T": cfg.T,
+            "indexer": f"{cfg.HI}x{cfg.DI}", "top_k": cfg.K, "heads": cfg.H,
+            "qk_dim": f"{cfg.d_nope}+{cfg.d_rope}", "v_dim": cfg.dv, "gate": cfg.gate,
+            "swa_layers": cfg.swa_layers, "window": cfg.window,
+            "l2": "flushed between steps (512 MB write outside the timed events)"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="c2", choices=["c1", "c2", "c3", "c4", "c5"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    world, rank, local = dist_setup(args)
+
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+
+    from sparse_attention_15_b200 import build as _build
+
+    _build.build_if_needed()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist
+
+    wl = Workload(args.config, dev, seed_offset=rank)
+    cfg = wl.cfg
+    nst = len(wl.stages)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def barrier():
+        if pg is not None:
+            pg.barrier()
+        torch.cuda.synchronize(dev)
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)]
+          for _ in range(args.steps)]
+    wev = [torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)]
+    for _ in range(args.warmup):
+        flush.zero_()
+        wl.step(wev)
+    torch.cuda.synchronize(dev)
+    wl.dsa.dsa_device_status(reset=True)
+
+    clocks = ClockSampler(dev)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    clocks.mark("t_start")
+    t_wall = time.perf_counter()
+    for i in range(args.steps):
+        flush.zero_()
+        wl.step(ev[i])
+    barrier()
+    t_wall = time.perf_counter() - t_wall
+    clocks.mark("t_stop")
+    clk = clocks.stop()
+    wl.dsa.dsa_device_status(reset=True)  # raises if any wait timed out
+
+    stage_ms = np.zeros(nst)
+    for i in range(args.steps):
+        for j in range(nst):
+            stage_ms[j] += ev[i][j].elapsed_time(ev[i][j + 1])
+    stage_ms /= args.steps
+    step_ms = float(stage_ms.sum())
+    if pg is not None:
+        t = torch.tensor([step_ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        step_ms = float(t.item())
+    units = wl.B * cfg.S * world
+    value = units / (step_ms / 1e3)
+
+    # roofline of the dominant stage
+    peaks, peak_src = load_peaks()
+    work = wl.work()
+    kernels = {}
+    for j, name in enumerate(wl.stages):
+        bound, amount, unit = work[name]
+        sec = stage_ms[j] / 1e3
+        if bound == "tensor":
+            ach, peak = amount / sec / 1e12, peaks["bf16_tflops"]
+        elif bound == "alu":
+            ach, peak = amount / sec / 1e12, F32_SIMT_TFLOPS
+        else:
+            ach, peak = amount / sec / 1e9, peaks["hbm_gbs"]
+        kernels[name] = {"ms": round(float(stage_ms[j]), 5), "bound": bound,
+                         "achieved": round(ach, 2), "peak": peak, "unit": unit,
+                         "frac": round(ach / peak, 4),
+                         "share": round(float(stage_ms[j]) / float(stage_ms.sum()), 4)}
+    dom = max(kernels, key=lambda k: kernels[k]["ms"])
+    kname = {"indexer": "index_scores", "topk": "topk", "attention": "gather_attn"}.get(
+        dom, "gather_attn")
+    tr = NCU_TRAFFIC.get((kname, cfg.name))
+    srcfile = {"index_scores": "indexer_tc.cu", "topk": "topk.cu",
+               "gather_attn": "gather_attn.cu"}[kname]
+    traffic = tr[0] if tr and tr[1] == src_sha(srcfile) else None
+    roof = dict(kernels[dom])
+    roof.pop("ms")
+    roof.pop("share")
+    roof.update({"kernel": dom, "traffic": traffic,
+                 "peak_source": f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'profiling recipe fallback'})"})
+
+    # end-to-end through the public call with host buffers
+    e2e = None
+    if not args.no_e2e:
+        host = wl.host_copy()
+        dev_bufs = {k: (None if v is None else torch.empty_like(v, device=dev))
+                    for k, v in host.items()}
+        out_host = torch.empty(wl.out.shape, dtype=wl.out.dtype).pin_memory()
+        import sparse_attention_15_b200 as dsa
+
+        a = dsa._forward_args(dev_bufs["q_idx"], dev_bufs["k_idx"], dev_bufs["w"], cfg.scale,
+                              cfg.K, dev_bufs["q"], dev_bufs["k"], dev_bufs["v"],
+                              dev_bufs["gate"], None, "none", 0.0, "auto", wl.out, None, wl.idx)
+        wl.fwd_ws_bytes = dsa.dsa_forward_workspace_bytes(a)
+        wl.fwd_ws = torch.empty(max(wl.fwd_ws_bytes, 16), dtype=torch.uint8, device=dev)
+        for _ in range(args.warmup):
+            wl.e2e_step(host, dev_bufs, out_host)
+        torch.cuda.synchronize(dev)
+        n_e2e = max(3, min(args.steps, 50))
+        e0 = [torch.cuda.Event(enable_timing=True) for _ in range(n_e2e)]
+        e1 = [torch.cuda.Event(enable_timing=True) for _ in range(n_e2e)]
+        barrier()
+        for i in range(n_e2e):
+            flush.zero_()
+            e0[i].record()
+            wl.e2e_step(host, dev_bufs, out_host)
+            e1[i].record()
+        barrier()
+        e2e_ms = sum(e0[i].elapsed_time(e1[i]) for i in range(n_e2e)) / n_e2e
+        if pg is not None:
+            t = torch.tensor([e2e_ms], device=dev)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
+        e2e = {"value": units / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(out_host.numel() * out_host.element_size()),
+               "ms_per_step": round(e2e_ms, 4), "steps": n_e2e}
+        wl.dsa.dsa_device_status(reset=True)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        xh = host_inputs(cfg, wl.x, 1)
+        rows = sample_rows(cfg.S, 4096)
+        rng = np.random.default_rng(0)
+        rng.shuffle(rows)
+        n, sec = oracle_rows_per_s(cfg, xh, rows, args.cpu_budget)
+        cpu = {"value": n / sec, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{n} query rows of batch row 0 drawn evenly over the {cfg.S} "
+                         f"queries, {sec:.1f} s of float64 numpy oracle work "
+                         f"(scores -> top-k -> dense masked attention per row)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32" if cfg.dtype == "f32" else "bf16", "data": "synthetic",
+            "config": workload_config(cfg, wl.B),
+            "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+            "clocks": clk, "gpu_launches": wl.launches_per_step * args.steps,
+            "wall_ms_per_step_incl_flush": round(1e3 * t_wall / args.steps, 4),
+        }
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,214 @@
+/*
+ * dsa.h -- C ABI of libdsa, the B200 (sm_100a) DeepSeek-style sparse attention hot path.
+ *
+ * The path has four steps, each a call below:
+ *   1. dsa_index_scores   lightning-indexer scores with the causal mask
+ *   2. dsa_topk           per-query top-k of those scores
+ *   3. dsa_sparse_attn    attention over the selected rows of the expanded K/V
+ *   4. (fused into 3)     optional headwise sigmoid / silu output gate
+ * plus dsa_forward, which runs 1-4 in one call, and dsa_window_attn, the sliding-window
+ * layer of the DSA-SWA-SWA hybrid block.
+ *
+ * Sources (web pages, cited by title and section):
+ *   [AXK2]  "Transformers 中的 AXK2 架构解析：SK Telecom A.X-K2 稀疏注意力 MoE 大模型集成指南",
+ *           sections "注意力前向的骨架：MLA + 显式稀疏掩码", "SK Telecom 三大改进 / 1. Sparse
+ *           Gated Attention（SGA）", "AXK2Config：核心配置与默认值", "使用注意事项小结".
+ *   [SPARK] Spark-X2.5-1.7B-Base headwise attention output gate walkthrough, sections
+ *           "在 Spark-X2.5-1.7B-Base 中如何开启？", "前向流程：从 gate_score 计算到相乘".
+ *   [DSV2]  DeepSeek-V2 attention parameter guide ("参数详解", items 4-6).
+ *   [PANGU] openPangu-2.0 technical-report reading, §3.2 (SWA), §3.3 (Lightning Indexer,
+ *           fixed K), §3.5 Table 1 (cost model).
+ *
+ * Conventions shared by every call
+ *   - Every tensor is dense, row-major, last index fastest, and lives in device memory
+ *     of the current CUDA device, allocated and owned by the caller.  The library never
+ *     allocates, frees or synchronises; inputs are read-only; outputs are overwritten in
+ *     full (including the -inf / -1 / zero padding described per call).
+ *   - Calls are asynchronous: they validate their arguments on the host, enqueue kernels
+ *     on `stream` and return.  Argument errors are reported before anything is launched
+ *     (DSA_ERR_INVALID_ARG / DSA_ERR_UNSUPPORTED) and leave the outputs untouched.
+ *     A launch failure returns DSA_ERR_CUDA.  Waits inside kernels are bounded (about
+ *     2 s); a wait that gives up records DSA_ERR_TIMEOUT in a per-device status word that
+ *     dsa_device_status() reads after the stream has been synchronised.  While a timeout
+ *     is recorded, later in-kernel waits give up at once; dsa_device_status(1) clears it.
+ *   - Base pointers must be 16-byte aligned.  bf16 head dimensions must be multiples of
+ *     8, float32 ones multiples of 4.
+ *   - q_off = T - S throughout: query s of a batch row sits at key position s + q_off,
+ *     i.e. the queries are the last S of the T positions (prefill: S == T; decode: S == 1).
+ *   - No C++ exception crosses this boundary.  Calls on distinct streams are thread-safe.
+ *     dsa_last_error() returns a thread-local text for the last failed call.
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* dsa_stream_t;
+
+typedef enum {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = 1, /* a null pointer, a non-positive size, an impossible shape   */
+  DSA_ERR_UNSUPPORTED = 2, /* a valid shape this build has no kernel for, misalignment  */
+  DSA_ERR_CUDA = 3,        /* a CUDA runtime / launch error                             */
+  DSA_ERR_TIMEOUT = 4,     /* a bounded in-kernel wait gave up (see dsa_device_status)  */
+  DSA_ERR_INTERNAL = 5     /* an in-kernel consistency check failed                     */
+} dsa_status;
+
+typedef enum { DSA_F32 = 0, DSA_BF16 = 1 } dsa_dtype;
+
+/* Where the indexer applies ReLU.  [AXK2] SGA prints the score as a plain weighted sum
+ * (DSA_RELU_NONE, the default reading); its prose adds "then ReLU" after the weighted sum
+ * (DSA_RELU_POST_SUM); DSA_RELU_PER_HEAD applies ReLU to each head's dot product before
+ * weighting, the upstream DeepSeek form, offered as an option. */
+typedef enum { DSA_RELU_NONE = 0, DSA_RELU_POST_SUM = 1, DSA_RELU_PER_HEAD = 2 } dsa_relu_mode;
+
+/* Headwise output gate, [SPARK] "前向流程" step 3: sigmoid or silu of one logit per
+ * (token, head), evaluated in float32; any other mode is rejected (the page's ValueError). */
+typedef enum { DSA_GATE_OFF = 0, DSA_GATE_SIGMOID = 1, DSA_GATE_SILU = 2 } dsa_gate_mode;
+
+/* Attention algorithm for dsa_forward / dsa_sparse_attn_ex. */
+typedef enum {
+  DSA_ATTN_AUTO = 0,      /* pick by the cost model (bytes gathered vs. dense tile work)  */
+  DSA_ATTN_GATHER = 1,    /* gather the selected K/V rows per query (decode-shaped work) */
+  DSA_ATTN_MASKED_TILE = 2 /* dense tensor-core tiles under the selection bitmask         */
+} dsa_attn_algo;
+
+/* ---------------------------------------------------------------------------------
+ * 1. Lightning-indexer scores.  [AXK2] SGA: index_score[b,s,t] =
+ *    sum_h weight[b,s,h] * softmax_scale * (q[b,s,h,:] . k[b,t,:]); causality is imposed
+ *    while scoring.  [PANGU] §3.5 Table 1: this is the quadratic prefill term,
+ *    S^2 * N_head^I * D^I.
+ *
+ *   q_idx   [B,S,HI,DI]  dtype       indexer queries (after their projection and RoPE)
+ *   k_idx   [B,T,DI]     dtype       indexer key cache (one head, shared by all HI heads)
+ *   w       [B,S,HI]     float32     per-head weights (the weights_proj output)
+ *   scale   > 0, finite              softmax_scale
+ *   scores  [B,S,T]      float32     out: the score for t <= s + q_off, -inf for t > s+q_off
+ *
+ *   Arithmetic: each head's dot product is accumulated in float32 from the dtype inputs;
+ *   the score is scale * sum_h w[h] * dot_h (float32).  With integer-valued inputs and a
+ *   power-of-two scale (the synthetic workloads) every intermediate is exact.
+ *   Requires 1 <= HI <= 256, 1 <= DI <= 128, T >= S.
+ * --------------------------------------------------------------------------------- */
+dsa_status dsa_index_scores(dsa_dtype dtype, const void* q_idx, const void* k_idx,
+                            const float* w, float scale, dsa_relu_mode relu, int B, int S,
+                            int T, int HI, int DI, float* scores, dsa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * 2. Per-query top-k.  [AXK2] SGA: the indexer returns int32 indices [B,S,topk];
+ *    "AXK2Config" (index_topk): topk = min(index_topk, number of keys).  [PANGU] §3.3:
+ *    the number of selected keys is a fixed K.
+ *
+ *   scores  [B,S,T]  float32   (as written by dsa_index_scores; only t <= s+q_off is read)
+ *   K       >= 1               columns of idx (callers pass min(index_topk, T))
+ *   idx     [B,S,K]  int32     out: the min(K, n) valid keys that come first in the order
+ *                              (higher score, then lower index), n = min(T, s+q_off+1),
+ *                              written in ascending key order, then -1 padding.
+ *   -0.0 and +0.0 compare equal.  NaN scores give an unspecified (but in-range) selection.
+ *   Exact and deterministic: a radix select on the float bit patterns, no float math.
+ * --------------------------------------------------------------------------------- */
+dsa_status dsa_topk(const float* scores, int B, int S, int T, int K, int32_t* idx,
+                    dsa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * 3+4. Sparse attention over the selected keys, with the optional headwise gate.
+ *    [AXK2] "注意力前向的骨架": the selected positions form an additive mask folded with
+ *    the causal mask, all other positions are -inf; the cache holds the expanded per-head
+ *    K/V.  [DSV2] items 4-6: q/k heads are qk_nope + qk_rope wide, v heads v_head_dim.
+ *    [SPARK] "前向流程": out[b,s,h,:] *= act(gate[b,s,h]) (act in float32).
+ *
+ *   q     [B,S,H,DQK]  dtype      k [B,T,H,DQK] dtype      v [B,T,H,DV] dtype
+ *   idx   [B,S,K]      int32      selected keys; -1, values outside [0,T) and keys in the
+ *                                 future of the query (t > s+q_off) are skipped.  A row's
+ *                                 valid entries must be distinct.
+ *   gate  [B,S,H]      dtype      gate logits, or NULL when gate_mode == DSA_GATE_OFF
+ *   sm_scale                      softmax scale; <= 0 selects 1/sqrt(DQK)
+ *   out   [B,S,H,DV]   dtype      out: softmax-weighted sum of the selected v rows (float32
+ *                                 accumulation, one rounding to dtype, gate applied before
+ *                                 that rounding); a row with no valid key gets zeros.
+ *   ws / ws_bytes                 scratch for split-key partial results; the size comes
+ *                                 from dsa_sparse_attn_workspace_bytes (may be 0 -> NULL ok).
+ *   Requires DQK <= 256, DV <= 256, H <= 64 (H a multiple of 2 above 16, of 4 above 32),
+ *   and H*DQK, H*DV rows that are multiples of 16 bytes.
+ * --------------------------------------------------------------------------------- */
+size_t dsa_sparse_attn_workspace_bytes(int B, int S, int T, int H, int DV, int K);
+dsa_status dsa_sparse_attn(dsa_dtype dtype, const void* q, const void* k, const void* v,
+                           const int32_t* idx, int K, const void* gate,
+                           dsa_gate_mode gate_mode, float sm_scale, int B, int S, int T,
+                           int H, int DQK, int DV, void* out, void* ws, size_t ws_bytes,
+                           dsa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * The whole DSA step: 1 -> 2 -> 3+4.  [AXK2] "注意力前向的骨架" steps 4-5.
+ * Scores and indices go to the caller's buffers when scores_out / idx_out are given,
+ * else to the workspace.  Without scores_out the score buffer may be smaller than
+ * B*S*T floats: the queries are then processed in row blocks that fit.
+ * --------------------------------------------------------------------------------- */
+typedef struct {
+  dsa_dtype dtype;
+  int B, S, T;             /* q_off = T - S                                              */
+  int HI, DI;              /* indexer heads / head dim                                   */
+  float index_scale;       /* indexer softmax_scale (> 0)                                */
+  dsa_relu_mode relu;
+  int K;                   /* index_topk; the path uses K_eff = min(K, T)                */
+  int H, DQK, DV;          /* attention heads, qk_nope+qk_rope, v_head_dim               */
+  float sm_scale;          /* <= 0 selects 1/sqrt(DQK)                                   */
+  dsa_gate_mode gate_mode;
+  dsa_attn_algo attn_algo;
+  const void* q_idx;       /* [B,S,HI,DI]                                                */
+  const void* k_idx;       /* [B,T,DI]                                                   */
+  const float* w;          /* [B,S,HI]                                                   */
+  const void* q;           /* [B,S,H,DQK]                                                */
+  const void* k;           /* [B,T,H,DQK]                                                */
+  const void* v;           /* [B,T,H,DV]                                                 */
+  const void* gate;        /* [B,S,H] or NULL                                            */
+  void* out;               /* [B,S,H,DV] out                                             */
+  float* scores_out;       /* optional [B,S,T] out                                       */
+  int32_t* idx_out;        /* optional [B,S,K_eff] out                                   */
+} dsa_forward_args;
+
+/* Bytes of workspace dsa_forward needs to run without row blocking. */
+size_t dsa_forward_workspace_bytes(const dsa_forward_args* a);
+/* Smallest workspace dsa_forward accepts (one row block). */
+size_t dsa_forward_min_workspace_bytes(const dsa_forward_args* a);
+dsa_status dsa_forward(const dsa_forward_args* a, void* ws, size_t ws_bytes,
+                       dsa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * Sliding-window causal attention with grouped KV heads: the SWA layers of the
+ * DSA-SWA-SWA hybrid.  [PANGU] §3.2: window fixed at 512 tokens, SWA:DSA layers 2:1.
+ * [SPARK] "为什么 Spark-X2.5 要加这一层门控？": window 512, GQA, headwise gate.
+ *
+ *   q [B,S,H,DQK], k [B,T,HKV,DQK], v [B,T,HKV,DV], gate [B,S,H] or NULL, out [B,S,H,DV];
+ *   query head h reads KV head h / (H/HKV); query s sees keys
+ *   s+q_off-window < t <= s+q_off.  Same arithmetic contract as dsa_sparse_attn.
+ * --------------------------------------------------------------------------------- */
+dsa_status dsa_window_attn(dsa_dtype dtype, const void* q, const void* k, const void* v,
+                           const void* gate, dsa_gate_mode gate_mode, float sm_scale,
+                           int window, int B, int S, int T, int H, int HKV, int DQK, int DV,
+                           void* out, dsa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * Status and introspection.
+ * --------------------------------------------------------------------------------- */
+const char* dsa_status_string(dsa_status s);
+/* Thread-local description of the last failed call on this thread ("" if none). */
+const char* dsa_last_error(void);
+/* Reads and (if reset != 0) clears the current device's in-kernel status word.
+ * Synchronous with respect to the device: call it after synchronising the streams used.
+ * Returns DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_INTERNAL (or DSA_ERR_CUDA if it cannot read). */
+dsa_status dsa_device_status(int reset);
+/* Library version, e.g. "dsa-b200 0.1.0 sm_100a". */
+const char* dsa_version(void);
+
+#ifdef __cplusplus
+} /* extern "C" */
+#endif
+
+#endif /* DSA_H_ */

@@ -76,11 +76,11 @@ def index_scores(q_idx, k_idx, w, scale, relu="none", q_off=None):
     if q_off is None:
         q_off = T - S
     # per-head dot products d[b,s,h,t] = q[b,s,h,:] . k[b,t,:]   (a plain matmul)
-    dots = np.einsum("bshd,btd->bsht", q, k)
+    dots = np.matmul(q, np.swapaxes(k, 1, 2)[:, None])
     if relu == "per_head":
         dots = np.maximum(dots, 0.0)
     # weighted sum over heads, each head term carrying the softmax_scale factor
-    score = np.einsum("bsh,bsht->bst", wt * float(scale), dots)
+    score = np.matmul((wt * float(scale))[:, :, None, :], dots)[:, :, 0, :]
     if relu == "post_sum":
         score = np.maximum(score, 0.0)
     s_pos = np.arange(S)[:, None] + q_off
@@ -166,6 +166,8 @@ def sparse_attention(q, k, v, idx, sm_scale=None, gate=None, gate_mode="off", q_
         sm_scale = 1.0 / np.sqrt(Dqk)
     out = np.zeros((B, S, H, v.shape[-1]), dtype=np.float64)
     for b in range(B):
+        kt = k[b].transpose(1, 0, 2)  # [H,T,Dqk]
+        vt = v[b].transpose(1, 0, 2)  # [H,T,Dv]
         for s in range(S):
             allowed = np.zeros(T, dtype=bool)
             sel = idx[b, s]
@@ -174,12 +176,12 @@ def sparse_attention(q, k, v, idx, sm_scale=None, gate=None, gate_mode="off", q_
             allowed[np.arange(T) > s + q_off] = False  # the causal mask
             if not allowed.any():
                 continue
-            logits = sm_scale * np.einsum("hd,thd->ht", q[b, s], k[b])
+            logits = sm_scale * np.matmul(kt, q[b, s][:, :, None])[:, :, 0]  # [H,T]
             logits[:, ~allowed] = -np.inf
             m = logits.max(axis=1, keepdims=True)
             p = np.exp(logits - m)
             p /= p.sum(axis=1, keepdims=True)
-            out[b, s] = np.einsum("ht,thd->hd", p, v[b])
+            out[b, s] = np.matmul(p[:, None, :], vt)[:, 0, :]
     if gate_mode != "off":
         out = apply_gate(out, gate, gate_mode)
     return out

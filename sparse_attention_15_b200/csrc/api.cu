@@ -1,0 +1,333 @@
+// libdsa C ABI: argument validation, workspace layout and kernel dispatch.
+// The contract of every entry point is documented in include/dsa.h.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+
+#include <string>
+
+#include "../../include/dsa.h"
+#include "common.cuh"
+#include "kernels.h"
+
+namespace dsa {
+__device__ unsigned int g_status = 0;
+}  // namespace dsa
+
+namespace {
+
+thread_local std::string g_last_error;
+
+dsa_status fail(dsa_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+dsa_status cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return DSA_OK;
+  if (e == cudaErrorNotSupported)
+    return fail(DSA_ERR_UNSUPPORTED, "%s: no kernel for this shape", what);
+  return fail(DSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t esize(dsa_dtype dt) { return dt == DSA_F32 ? 4 : 2; }
+
+bool dim_ok(dsa_dtype dt, int d) { return d > 0 && d % (dt == DSA_F32 ? 4 : 8) == 0; }
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+#define REQUIRE(cond, st, ...)                 \
+  do {                                         \
+    if (!(cond)) return fail(st, __VA_ARGS__); \
+  } while (0)
+
+dsa_status check_index_args(dsa_dtype dtype, const void* q_idx, const void* k_idx,
+                            const float* w, float scale, dsa_relu_mode relu, int B, int S,
+                            int T, int HI, int DI, const void* scores) {
+  REQUIRE(dtype == DSA_F32 || dtype == DSA_BF16, DSA_ERR_INVALID_ARG, "unknown dtype %d",
+          (int)dtype);
+  REQUIRE(q_idx && k_idx && w && scores, DSA_ERR_INVALID_ARG, "null pointer argument");
+  REQUIRE(B > 0 && S > 0 && T > 0 && HI > 0 && DI > 0, DSA_ERR_INVALID_ARG,
+          "sizes must be positive (B=%d S=%d T=%d HI=%d DI=%d)", B, S, T, HI, DI);
+  REQUIRE(T >= S, DSA_ERR_INVALID_ARG, "T (%d) must be >= S (%d): queries are the last S keys",
+          T, S);
+  REQUIRE(isfinite(scale) && scale > 0.f, DSA_ERR_INVALID_ARG,
+          "index scale must be finite and > 0");
+  REQUIRE(relu >= DSA_RELU_NONE && relu <= DSA_RELU_PER_HEAD, DSA_ERR_INVALID_ARG,
+          "unknown relu mode %d", (int)relu);
+  REQUIRE(HI <= 256, DSA_ERR_UNSUPPORTED, "HI=%d > 256", HI);
+  REQUIRE(DI <= 128 && dim_ok(dtype, DI), DSA_ERR_UNSUPPORTED,
+          "DI=%d must be <= 128 and a multiple of %d", DI, dtype == DSA_F32 ? 4 : 8);
+  REQUIRE(S <= 65535 * 8, DSA_ERR_UNSUPPORTED, "S=%d too large", S);
+  REQUIRE(B <= 65535, DSA_ERR_UNSUPPORTED, "B=%d too large", B);
+  REQUIRE(aligned16(q_idx) && aligned16(k_idx) && aligned16(w) && aligned16(scores),
+          DSA_ERR_UNSUPPORTED, "pointers must be 16-byte aligned");
+  return DSA_OK;
+}
+
+dsa_status run_index_scores(dsa_dtype dtype, const void* q_idx, const void* k_idx,
+                            const float* w, float scale, dsa_relu_mode relu, int B, int S,
+                            int T, int HI, int DI, int q_off, float* scores,
+                            cudaStream_t st) {
+  cudaError_t e;
+  if (dsa::index_scores_tc_supported((int)dtype, HI, DI))
+    e = dsa::launch_index_scores_tc(q_idx, k_idx, w, scale, (int)relu, B, S, T, HI, DI, q_off,
+                                    scores, 1, st);
+  else
+    e = dsa::launch_index_scores_simt((int)dtype, q_idx, k_idx, w, scale, (int)relu, B, S, T,
+                                      HI, DI, q_off, scores, st);
+  return cuda_status(e, "dsa_index_scores");
+}
+
+dsa_status check_attn_common(dsa_dtype dtype, const void* q, const void* k, const void* v,
+                             const void* gate, dsa_gate_mode gm, float sm_scale, int B, int S,
+                             int T, int H, int HKV, int DQK, int DV, const void* out) {
+  REQUIRE(dtype == DSA_F32 || dtype == DSA_BF16, DSA_ERR_INVALID_ARG, "unknown dtype %d",
+          (int)dtype);
+  REQUIRE(q && k && v && out, DSA_ERR_INVALID_ARG, "null pointer argument");
+  REQUIRE(B > 0 && S > 0 && T > 0 && H > 0 && HKV > 0 && DQK > 0 && DV > 0,
+          DSA_ERR_INVALID_ARG, "sizes must be positive");
+  REQUIRE(T >= S, DSA_ERR_INVALID_ARG, "T (%d) must be >= S (%d)", T, S);
+  REQUIRE(H % HKV == 0, DSA_ERR_INVALID_ARG, "H=%d not a multiple of HKV=%d", H, HKV);
+  REQUIRE(gm >= DSA_GATE_OFF && gm <= DSA_GATE_SILU, DSA_ERR_INVALID_ARG,
+          "unknown gate mode %d (only sigmoid and silu exist)", (int)gm);
+  REQUIRE((gm == DSA_GATE_OFF) == (gate == nullptr), DSA_ERR_INVALID_ARG,
+          "gate pointer must be given exactly when the gate is on");
+  REQUIRE(!isnan(sm_scale) && !isinf(sm_scale), DSA_ERR_INVALID_ARG, "sm_scale not finite");
+  REQUIRE(DQK <= 256 && DV <= 256 && dim_ok(dtype, DQK) && dim_ok(dtype, DV),
+          DSA_ERR_UNSUPPORTED, "DQK=%d / DV=%d must be <= 256 and multiples of %d", DQK, DV,
+          dtype == DSA_F32 ? 4 : 8);
+  REQUIRE(H <= 64, DSA_ERR_UNSUPPORTED, "H=%d > 64", H);
+  REQUIRE((HKV * DQK * esize(dtype)) % 16 == 0 && (HKV * DV * esize(dtype)) % 16 == 0,
+          DSA_ERR_UNSUPPORTED, "K/V rows must be multiples of 16 bytes");
+  REQUIRE(aligned16(q) && aligned16(k) && aligned16(v) && aligned16(out) &&
+              (gate == nullptr || aligned16(gate)),
+          DSA_ERR_UNSUPPORTED, "pointers must be 16-byte aligned");
+  return DSA_OK;
+}
+
+float default_scale(float sm_scale, int DQK) {
+  return sm_scale > 0.f ? sm_scale : 1.0f / sqrtf((float)DQK);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* dsa_status_string(dsa_status s) {
+  switch (s) {
+    case DSA_OK: return "ok";
+    case DSA_ERR_INVALID_ARG: return "invalid argument";
+    case DSA_ERR_UNSUPPORTED: return "unsupported shape or layout";
+    case DSA_ERR_CUDA: return "CUDA error";
+    case DSA_ERR_TIMEOUT: return "in-kernel wait timed out";
+    case DSA_ERR_INTERNAL: return "internal consistency check failed";
+  }
+  return "unknown status";
+}
+
+const char* dsa_last_error(void) { return g_last_error.c_str(); }
+
+const char* dsa_version(void) { return "dsa-b200 0.1.0 sm_100a"; }
+
+dsa_status dsa_device_status(int reset) {
+  unsigned v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, dsa::g_status, sizeof(v));
+  if (e != cudaSuccess) return fail(DSA_ERR_CUDA, "dsa_device_status: %s", cudaGetErrorString(e));
+  if (reset && v) {
+    unsigned z = 0;
+    e = cudaMemcpyToSymbol(dsa::g_status, &z, sizeof(z));
+    if (e != cudaSuccess)
+      return fail(DSA_ERR_CUDA, "dsa_device_status: %s", cudaGetErrorString(e));
+  }
+  if (v & dsa::kStatusTimeout) return fail(DSA_ERR_TIMEOUT, "an in-kernel wait timed out");
+  if (v & dsa::kStatusInternal) return fail(DSA_ERR_INTERNAL, "in-kernel check failed");
+  return DSA_OK;
+}
+
+dsa_status dsa_index_scores(dsa_dtype dtype, const void* q_idx, const void* k_idx,
+                            const float* w, float scale, dsa_relu_mode relu, int B, int S,
+                            int T, int HI, int DI, float* scores, dsa_stream_t stream) {
+  dsa_status st = check_index_args(dtype, q_idx, k_idx, w, scale, relu, B, S, T, HI, DI, scores);
+  if (st != DSA_OK) return st;
+  return run_index_scores(dtype, q_idx, k_idx, w, scale, relu, B, S, T, HI, DI, T - S, scores,
+                          (cudaStream_t)stream);
+}
+
+dsa_status dsa_topk(const float* scores, int B, int S, int T, int K, int32_t* idx,
+                    dsa_stream_t stream) {
+  REQUIRE(scores && idx, DSA_ERR_INVALID_ARG, "null pointer argument");
+  REQUIRE(B > 0 && S > 0 && T > 0 && K > 0, DSA_ERR_INVALID_ARG, "sizes must be positive");
+  REQUIRE(T >= S, DSA_ERR_INVALID_ARG, "T (%d) must be >= S (%d)", T, S);
+  REQUIRE((size_t)B * S <= 0x7fffffffu, DSA_ERR_UNSUPPORTED, "too many rows");
+  REQUIRE(aligned16(scores) && aligned16(idx), DSA_ERR_UNSUPPORTED,
+          "pointers must be 16-byte aligned");
+  return cuda_status(dsa::launch_topk(scores, B, S, T, K, T - S, idx, nullptr,
+                                      (cudaStream_t)stream),
+                     "dsa_topk");
+}
+
+size_t dsa_sparse_attn_workspace_bytes(int B, int S, int T, int H, int DV, int K) {
+  (void)T;
+  if (B <= 0 || S <= 0 || H <= 0 || DV <= 0 || K <= 0) return 0;
+  return dsa::gather_attn_workspace_bytes(B, S, H, DV, K);
+}
+
+dsa_status dsa_sparse_attn(dsa_dtype dtype, const void* q, const void* k, const void* v,
+                           const int32_t* idx, int K, const void* gate,
+                           dsa_gate_mode gate_mode, float sm_scale, int B, int S, int T,
+                           int H, int DQK, int DV, void* out, void* ws, size_t ws_bytes,
+                           dsa_stream_t stream) {
+  dsa_status st = check_attn_common(dtype, q, k, v, gate, gate_mode, sm_scale, B, S, T, H, H,
+                                    DQK, DV, out);
+  if (st != DSA_OK) return st;
+  REQUIRE(idx != nullptr && K > 0, DSA_ERR_INVALID_ARG, "idx must be given with K > 0");
+  REQUIRE(aligned16(idx), DSA_ERR_UNSUPPORTED, "idx must be 16-byte aligned");
+  const size_t need = dsa::gather_attn_workspace_bytes(B, S, H, DV, K);
+  REQUIRE(ws_bytes >= need && (need == 0 || ws != nullptr), DSA_ERR_INVALID_ARG,
+          "workspace too small: %zu bytes given, %zu needed", ws_bytes, need);
+  dsa::AttnProblem p{};
+  p.dtype = (int)dtype; p.q = q; p.k = k; p.v = v; p.idx = idx; p.K = K; p.window = 0;
+  p.gate = gate; p.gate_mode = (int)gate_mode; p.sm_scale = default_scale(sm_scale, DQK);
+  p.B = B; p.S = S; p.T = T; p.H = H; p.HKV = H; p.DQK = DQK; p.DV = DV; p.q_off = T - S;
+  p.out = out;
+  return cuda_status(dsa::launch_gather_attn(p, ws, ws_bytes, (cudaStream_t)stream),
+                     "dsa_sparse_attn");
+}
+
+dsa_status dsa_window_attn(dsa_dtype dtype, const void* q, const void* k, const void* v,
+                           const void* gate, dsa_gate_mode gate_mode, float sm_scale,
+                           int window, int B, int S, int T, int H, int HKV, int DQK, int DV,
+                           void* out, dsa_stream_t stream) {
+  dsa_status st = check_attn_common(dtype, q, k, v, gate, gate_mode, sm_scale, B, S, T, H, HKV,
+                                    DQK, DV, out);
+  if (st != DSA_OK) return st;
+  REQUIRE(window > 0, DSA_ERR_INVALID_ARG, "window must be positive");
+  const size_t need = dsa::gather_attn_workspace_bytes(B, S, H, DV, window);
+  REQUIRE(need == 0, DSA_ERR_UNSUPPORTED,
+          "window attention with so few query rows needs split keys; not supported");
+  dsa::AttnProblem p{};
+  p.dtype = (int)dtype; p.q = q; p.k = k; p.v = v; p.idx = nullptr; p.K = 0; p.window = window;
+  p.gate = gate; p.gate_mode = (int)gate_mode; p.sm_scale = default_scale(sm_scale, DQK);
+  p.B = B; p.S = S; p.T = T; p.H = H; p.HKV = HKV; p.DQK = DQK; p.DV = DV; p.q_off = T - S;
+  p.out = out;
+  return cuda_status(dsa::launch_gather_attn(p, nullptr, 0, (cudaStream_t)stream),
+                     "dsa_window_attn");
+}
+
+// ----------------------------------------------------------------------------- forward
+static dsa_status check_forward(const dsa_forward_args* a) {
+  REQUIRE(a != nullptr, DSA_ERR_INVALID_ARG, "null args");
+  dsa_status st = check_index_args(a->dtype, a->q_idx, a->k_idx, a->w, a->index_scale, a->relu,
+                                   a->B, a->S, a->T, a->HI, a->DI,
+                                   a->scores_out ? (const void*)a->scores_out : (const void*)a);
+  if (st != DSA_OK) return st;
+  st = check_attn_common(a->dtype, a->q, a->k, a->v, a->gate, a->gate_mode, a->sm_scale, a->B,
+                         a->S, a->T, a->H, a->H, a->DQK, a->DV, a->out);
+  if (st != DSA_OK) return st;
+  REQUIRE(a->K > 0, DSA_ERR_INVALID_ARG, "K must be positive");
+  REQUIRE(a->attn_algo >= DSA_ATTN_AUTO && a->attn_algo <= DSA_ATTN_MASKED_TILE,
+          DSA_ERR_INVALID_ARG, "unknown attention algorithm %d", (int)a->attn_algo);
+  REQUIRE(a->idx_out == nullptr || aligned16(a->idx_out), DSA_ERR_UNSUPPORTED,
+          "idx_out must be 16-byte aligned");
+  return DSA_OK;
+}
+
+struct FwdLayout {
+  size_t idx_off, attn_off, scores_off, total_full, total_min;
+  int k_eff;
+};
+
+static FwdLayout forward_layout(const dsa_forward_args* a) {
+  FwdLayout L{};
+  L.k_eff = a->K < a->T ? a->K : a->T;
+  size_t off = 0;
+  L.idx_off = off;
+  if (!a->idx_out) off += align256((size_t)a->B * a->S * L.k_eff * sizeof(int32_t));
+  L.attn_off = off;
+  off += align256(dsa::gather_attn_workspace_bytes(a->B, a->S, a->H, a->DV, L.k_eff));
+  L.scores_off = off;
+  if (a->scores_out) {
+    L.total_full = L.total_min = off;
+  } else {
+    L.total_full = off + align256((size_t)a->B * a->S * a->T * sizeof(float));
+    L.total_min = off + align256((size_t)a->T * sizeof(float));
+  }
+  return L;
+}
+
+size_t dsa_forward_workspace_bytes(const dsa_forward_args* a) {
+  if (!a || a->B <= 0 || a->S <= 0 || a->T <= 0 || a->K <= 0) return 0;
+  return forward_layout(a).total_full;
+}
+
+size_t dsa_forward_min_workspace_bytes(const dsa_forward_args* a) {
+  if (!a || a->B <= 0 || a->S <= 0 || a->T <= 0 || a->K <= 0) return 0;
+  return forward_layout(a).total_min;
+}
+
+dsa_status dsa_forward(const dsa_forward_args* a, void* ws, size_t ws_bytes,
+                       dsa_stream_t stream) {
+  dsa_status st = check_forward(a);
+  if (st != DSA_OK) return st;
+  const FwdLayout L = forward_layout(a);
+  REQUIRE(ws_bytes >= L.total_min && (L.total_min == 0 || ws != nullptr), DSA_ERR_INVALID_ARG,
+          "workspace too small: %zu bytes given, at least %zu needed", ws_bytes, L.total_min);
+  REQUIRE(ws == nullptr || aligned16(ws), DSA_ERR_UNSUPPORTED, "workspace must be 16-byte aligned");
+  cudaStream_t s = (cudaStream_t)stream;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  int32_t* idx = a->idx_out ? a->idx_out : reinterpret_cast<int32_t*>(base + L.idx_off);
+  void* attn_ws = base ? base + L.attn_off : nullptr;
+  const size_t attn_ws_bytes = L.scores_off - L.attn_off;
+  const int B = a->B, S = a->S, T = a->T, q_off = T - S;
+  const size_t es = esize(a->dtype);
+
+  if (a->scores_out || ws_bytes >= L.total_full) {
+    float* scores = a->scores_out ? a->scores_out : reinterpret_cast<float*>(base + L.scores_off);
+    st = run_index_scores(a->dtype, a->q_idx, a->k_idx, a->w, a->index_scale, a->relu, B, S, T,
+                          a->HI, a->DI, q_off, scores, s);
+    if (st != DSA_OK) return st;
+    st = cuda_status(dsa::launch_topk(scores, B, S, T, L.k_eff, q_off, idx, nullptr, s),
+                     "dsa_forward/topk");
+    if (st != DSA_OK) return st;
+  } else {
+    // row blocks that fit the score buffer, one batch row at a time
+    float* scores = reinterpret_cast<float*>(base + L.scores_off);
+    const size_t avail = ws_bytes - L.scores_off;
+    int rb = (int)(avail / ((size_t)T * sizeof(float)));
+    if (rb > S) rb = S;
+    for (int b = 0; b < B; ++b) {
+      for (int s0 = 0; s0 < S; s0 += rb) {
+        const int n = S - s0 < rb ? S - s0 : rb;
+        const uint8_t* qi = static_cast<const uint8_t*>(a->q_idx) +
+                            ((size_t)b * S + s0) * a->HI * a->DI * es;
+        const uint8_t* ki = static_cast<const uint8_t*>(a->k_idx) + (size_t)b * T * a->DI * es;
+        const float* wb = a->w + ((size_t)b * S + s0) * a->HI;
+        // this block's first query sits at key position q_off + s0
+        st = run_index_scores(a->dtype, qi, ki, wb, a->index_scale, a->relu, 1, n, T, a->HI,
+                              a->DI, q_off + s0, scores, s);
+        if (st != DSA_OK) return st;
+        st = cuda_status(dsa::launch_topk(scores, 1, n, T, L.k_eff, q_off + s0,
+                                          idx + ((size_t)b * S + s0) * L.k_eff, nullptr, s),
+                         "dsa_forward/topk");
+        if (st != DSA_OK) return st;
+      }
+    }
+  }
+  dsa::AttnProblem p{};
+  p.dtype = (int)a->dtype; p.q = a->q; p.k = a->k; p.v = a->v; p.idx = idx; p.K = L.k_eff;
+  p.window = 0; p.gate = a->gate; p.gate_mode = (int)a->gate_mode;
+  p.sm_scale = default_scale(a->sm_scale, a->DQK);
+  p.B = B; p.S = S; p.T = T; p.H = a->H; p.HKV = a->H; p.DQK = a->DQK; p.DV = a->DV;
+  p.q_off = q_off; p.out = a->out;
+  return cuda_status(dsa::launch_gather_attn(p, attn_ws, attn_ws_bytes, s), "dsa_forward/attn");
+}
+
+}  // extern "C"

@@ -1,0 +1,351 @@
+// Sparse attention by gathering the selected K/V rows, with the headwise gate fused.
+//
+// [AXK2] "注意力前向的骨架：MLA + 显式稀疏掩码": every query attends only to the keys the
+// indexer selected (all other positions are -inf), under the causal mask; the cache holds
+// the expanded per-head K/V (the expand_kv output).  [DSV2] items 4-6: q/k heads are
+// qk_nope + qk_rope wide, v heads v_head_dim wide.  [SPARK] "前向流程": the output of
+// head h is multiplied by act(gate[b,s,h]) in float32 before the cast.
+//
+// All heads of a query share its index set, so one selected key is one contiguous row of
+// the K cache (H*DQK elements) and one of the V cache (H*DV elements).  A producer warp
+// streams those rows into a ring of shared-memory slots with 1-D bulk copies (the TMA
+// engine, mbarrier transaction counts, no multicast); consumer warps own whole heads
+// (lane l holds dims 4l..4l+3 of every 128-wide slice) and run an online softmax in
+// float32, one key at a time, without any block-wide barrier.  Each consumer warp releases
+// a slot by arriving on its "empty" barrier.
+//
+// The same kernel computes the sliding-window layers: the index set is then the band
+// s+q_off-window < t <= s+q_off, and query head h reads KV head h / (H / HKV).
+//
+// Long index lists with few query rows (decode) are split over several CTAs; each writes
+// an unnormalised partial (o, m, l) and a second kernel merges them in a fixed order.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace dsa {
+
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct GatherArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const int32_t* idx;
+  const void* gate;
+  void* out;
+  float* part_o;   // [rows, nsplit, H, DV] (split mode)
+  float* part_ml;  // [rows, nsplit, H, 2]
+  int K, window, gate_mode;
+  float qk_scale;  // sm_scale * log2(e)
+  int S, T, H, HKV, DQK, DV, q_off;
+  int nsplit, keys_per_split;
+  int nslots;
+  uint32_t k_bytes, v_bytes, slot_bytes;
+};
+
+// Key j of this CTA's range, or -1 if it must be skipped.
+__device__ __forceinline__ int key_at(const GatherArgs& a, const int32_t* idx_row, int j,
+                                      int spos) {
+  int t;
+  if (idx_row) {
+    t = __ldg(idx_row + j);
+  } else {
+    t = spos - a.window + 1 + j;  // band: oldest key first
+  }
+  return (t >= 0 && t < a.T && t <= spos) ? t : -1;
+}
+
+template <typename T, int QKV, int VV, int HPW>
+__global__ void __launch_bounds__(544, HPW <= 2 ? 2 : 1) gather_attn_kernel(const GatherArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int nslots = a.nslots;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+  uint64_t* empty = full + nslots;
+  int* slot_key = reinterpret_cast<int*>(empty + nslots);
+  uint8_t* slots = smem + 1024;  // slot data starts 1 KB in (barriers and flags first)
+
+  const int nw = (blockDim.x >> 5) - 1;  // consumer warps; the last warp produces
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x / a.nsplit;
+  const int split = blockIdx.x % a.nsplit;
+  const int b = row / a.S, s = row % a.S;
+  const int spos = s + a.q_off;
+  const int nkeys_total = a.idx ? a.K : a.window;
+  const int j0 = split * a.keys_per_split;
+  const int nkeys = max(0, min(nkeys_total, j0 + a.keys_per_split) - j0);
+  const int32_t* idx_row = a.idx ? a.idx + (size_t)row * a.K + j0 : nullptr;
+  const int band0 = j0;  // band offset of this split
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < nslots; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], nw);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  const T* kbase = static_cast<const T*>(a.k) + (size_t)b * a.T * a.HKV * a.DQK;
+  const T* vbase = static_cast<const T*>(a.v) + (size_t)b * a.T * a.HKV * a.DV;
+
+  if (warp == nw) {
+    // ------------------------------------------------------------- producer
+    if (lane == 0) {
+      for (int j = 0; j < nkeys; ++j) {
+        const int slot = j % nslots;
+        const int round = j / nslots;
+        if (round > 0 && !mbar_wait(&empty[slot], (round - 1) & 1)) break;
+        int t = idx_row ? key_at(a, idx_row, j, spos) : key_at(a, nullptr, band0 + j, spos);
+        slot_key[slot] = t;
+        if (t >= 0) {
+          uint8_t* dst = slots + (size_t)slot * a.slot_bytes;
+          mbar_arrive_expect_tx(&full[slot], a.k_bytes + a.v_bytes);
+          bulk_g2s(dst, kbase + (size_t)t * a.HKV * a.DQK, a.k_bytes, &full[slot]);
+          bulk_g2s(dst + a.k_bytes, vbase + (size_t)t * a.HKV * a.DV, a.v_bytes, &full[slot]);
+        } else {
+          mbar_arrive(&full[slot]);
+        }
+      }
+    }
+    return;
+  }
+
+  // --------------------------------------------------------------- consumers
+  constexpr int hpw = HPW;  // heads per warp
+  constexpr int kMaxHpw = HPW;
+  const int group = a.H / a.HKV;
+  float qr[kMaxHpw][QKV][4];
+  float acc[kMaxHpw][VV][4];
+  float m[kMaxHpw], l[kMaxHpw];
+  const T* qrow = static_cast<const T*>(a.q) + (size_t)row * a.H * a.DQK;
+#pragma unroll
+  for (int hi = 0; hi < kMaxHpw; ++hi) {
+    m[hi] = -INFINITY;
+    l[hi] = 0.f;
+#pragma unroll
+    for (int c = 0; c < VV; ++c)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[hi][c][e] = 0.f;
+#pragma unroll
+    for (int c = 0; c < QKV; ++c) {
+      const int d = c * 128 + lane * 4;
+      float x[4] = {0.f, 0.f, 0.f, 0.f};
+      if (hi < hpw && d < a.DQK) load4(qrow + (size_t)(warp + nw * hi) * a.DQK + d, x);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) qr[hi][c][e] = x[e] * a.qk_scale;
+    }
+  }
+
+  bool ok = true;
+  for (int j = 0; j < nkeys && ok; ++j) {
+    const int slot = j % nslots;
+    ok = mbar_wait(&full[slot], (j / nslots) & 1);
+    if (ok && slot_key[slot] >= 0) {
+      const T* ks = reinterpret_cast<const T*>(slots + (size_t)slot * a.slot_bytes);
+      const T* vs = reinterpret_cast<const T*>(slots + (size_t)slot * a.slot_bytes + a.k_bytes);
+#pragma unroll
+      for (int hi = 0; hi < kMaxHpw; ++hi) {
+        if (hi >= hpw) break;
+        const int h = warp + nw * hi;
+        const int kvh = h / group;
+        float dot = 0.f;
+#pragma unroll
+        for (int c = 0; c < QKV; ++c) {
+          const int d = c * 128 + lane * 4;
+          if (d < a.DQK) {
+            float x[4];
+            load4(ks + (size_t)kvh * a.DQK + d, x);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dot = fmaf(qr[hi][c][e], x[e], dot);
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+        const float mn = fmaxf(m[hi], dot);
+        const float corr = exp2f(m[hi] - mn);
+        const float p = exp2f(dot - mn);
+        m[hi] = mn;
+        l[hi] = fmaf(l[hi], corr, p);
+#pragma unroll
+        for (int c = 0; c < VV; ++c) {
+          const int d = c * 128 + lane * 4;
+          if (d < a.DV) {
+            float x[4];
+            load4(vs + (size_t)kvh * a.DV + d, x);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[hi][c][e] = fmaf(p, x[e], acc[hi][c][e] * corr);
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[slot]);
+  }
+
+  // --------------------------------------------------------------- epilogue
+#pragma unroll
+  for (int hi = 0; hi < kMaxHpw; ++hi) {
+    if (hi >= hpw) break;
+    const int h = warp + nw * hi;
+    if (a.nsplit == 1) {
+      float f = l[hi] > 0.f ? 1.0f / l[hi] : 0.f;
+      if (a.gate)
+        f *= gate_act(to_f32(static_cast<const T*>(a.gate)[(size_t)row * a.H + h]), a.gate_mode);
+      T* o = static_cast<T*>(a.out) + ((size_t)row * a.H + h) * a.DV;
+#pragma unroll
+      for (int c = 0; c < VV; ++c) {
+        const int d = c * 128 + lane * 4;
+        if (d < a.DV)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) o[d + e] = from_f32<T>(acc[hi][c][e] * f);
+      }
+    } else {
+      const size_t base = ((size_t)row * a.nsplit + split) * a.H + h;
+      float* po = a.part_o + base * a.DV;
+#pragma unroll
+      for (int c = 0; c < VV; ++c) {
+        const int d = c * 128 + lane * 4;
+        if (d < a.DV)
+          *reinterpret_cast<float4*>(po + d) =
+              make_float4(acc[hi][c][0], acc[hi][c][1], acc[hi][c][2], acc[hi][c][3]);
+      }
+      if (lane == 0) {
+        a.part_ml[base * 2 + 0] = m[hi];
+        a.part_ml[base * 2 + 1] = l[hi];
+      }
+    }
+  }
+}
+
+// Merge the split partials of one row: out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p.
+template <typename T>
+__global__ void combine_kernel(const GatherArgs a) {
+  const int row = blockIdx.x;
+  for (int e = threadIdx.x; e < a.H * a.DV; e += blockDim.x) {
+    const int h = e / a.DV, d = e % a.DV;
+    float M = -INFINITY;
+    for (int p = 0; p < a.nsplit; ++p)
+      M = fmaxf(M, a.part_ml[(((size_t)row * a.nsplit + p) * a.H + h) * 2]);
+    float L = 0.f, O = 0.f;
+    if (M != -INFINITY) {
+      for (int p = 0; p < a.nsplit; ++p) {
+        const size_t base = ((size_t)row * a.nsplit + p) * a.H + h;
+        const float mp = a.part_ml[base * 2];
+        if (mp == -INFINITY) continue;
+        const float f = exp2f(mp - M);
+        L = fmaf(a.part_ml[base * 2 + 1], f, L);
+        O = fmaf(a.part_o[base * a.DV + d], f, O);
+      }
+    }
+    float r = L > 0.f ? O / L : 0.f;
+    if (a.gate)
+      r *= gate_act(to_f32(static_cast<const T*>(a.gate)[(size_t)row * a.H + h]), a.gate_mode);
+    static_cast<T*>(a.out)[((size_t)row * a.H + h) * a.DV + d] = from_f32<T>(r);
+  }
+}
+
+// Heads per consumer warp: the smallest of 1, 2, 4 that divides H and leaves at most
+// 16 consumer warps.
+int heads_per_warp(int H) {
+  for (int hpw = 1; hpw <= 4; hpw *= 2)
+    if (H % hpw == 0 && H / hpw <= 16) return hpw;
+  return 0;
+}
+
+// Split policy: few query rows and long key lists -> spread the keys over CTAs.
+void split_policy(int rows, int nkeys, int* nsplit, int* kps) {
+  const int target_ctas = 4 * 148;
+  if (rows >= target_ctas || nkeys <= 128) {
+    *nsplit = 1;
+    *kps = nkeys;
+    return;
+  }
+  int ns = (target_ctas + rows - 1) / rows;
+  int max_ns = (nkeys + 63) / 64;
+  if (ns > max_ns) ns = max_ns;
+  if (ns < 1) ns = 1;
+  *kps = (nkeys + ns - 1) / ns;
+  *nsplit = (nkeys + *kps - 1) / *kps;
+}
+
+template <typename T, int QKV, int VV, int HPW>
+cudaError_t launch_t(GatherArgs a, int nw, size_t smem, unsigned grid, int rows,
+                     cudaStream_t st) {
+  auto kern = gather_attn_kernel<T, QKV, VV, HPW>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, 32 * (nw + 1), smem, st>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || a.nsplit == 1) return e;
+  combine_kernel<T><<<rows, 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <typename T, int HPW>
+cudaError_t launch_dims(GatherArgs a, int nw, size_t smem, unsigned grid, int rows,
+                        cudaStream_t st) {
+  const int qkv = (a.DQK + 127) / 128, vv = (a.DV + 127) / 128;
+  if (qkv == 1 && vv == 1) return launch_t<T, 1, 1, HPW>(a, nw, smem, grid, rows, st);
+  if (qkv == 2 && vv == 1) return launch_t<T, 2, 1, HPW>(a, nw, smem, grid, rows, st);
+  if (qkv == 2 && vv == 2) return launch_t<T, 2, 2, HPW>(a, nw, smem, grid, rows, st);
+  if (qkv == 1 && vv == 2) return launch_t<T, 1, 2, HPW>(a, nw, smem, grid, rows, st);
+  return cudaErrorNotSupported;
+}
+
+template <typename T>
+cudaError_t launch_hpw(GatherArgs a, int hpw, size_t smem, unsigned grid, int rows,
+                       cudaStream_t st) {
+  const int nw = a.H / hpw;
+  if (hpw == 1) return launch_dims<T, 1>(a, nw, smem, grid, rows, st);
+  if (hpw == 2) return launch_dims<T, 2>(a, nw, smem, grid, rows, st);
+  if (hpw == 4) return launch_dims<T, 4>(a, nw, smem, grid, rows, st);
+  return cudaErrorNotSupported;
+}
+
+}  // namespace
+
+size_t gather_attn_workspace_bytes(int B, int S, int H, int DV, int K) {
+  const int rows = B * S;
+  int ns, kps;
+  split_policy(rows, K, &ns, &kps);
+  if (ns == 1) return 0;
+  return (size_t)rows * ns * H * (DV + 2) * sizeof(float);
+}
+
+cudaError_t launch_gather_attn(const AttnProblem& p, void* ws, size_t ws_bytes,
+                               cudaStream_t st) {
+  GatherArgs a{};
+  a.q = p.q; a.k = p.k; a.v = p.v; a.idx = p.idx; a.gate = p.gate; a.out = p.out;
+  a.K = p.K; a.window = p.window; a.gate_mode = p.gate_mode;
+  a.qk_scale = p.sm_scale * kLog2e;
+  a.S = p.S; a.T = p.T; a.H = p.H; a.HKV = p.HKV; a.DQK = p.DQK; a.DV = p.DV; a.q_off = p.q_off;
+  const int rows = p.B * p.S;
+  if (rows == 0) return cudaSuccess;
+  const int nkeys = p.idx ? p.K : p.window;
+  split_policy(rows, nkeys, &a.nsplit, &a.keys_per_split);
+  if (a.nsplit > 1) {
+    const size_t need = (size_t)rows * a.nsplit * p.H * (p.DV + 2) * sizeof(float);
+    if (ws == nullptr || ws_bytes < need) return cudaErrorInvalidValue;
+    a.part_o = static_cast<float*>(ws);
+    a.part_ml = a.part_o + (size_t)rows * a.nsplit * p.H * p.DV;
+  }
+  const size_t es = p.dtype == 0 ? 4 : 2;
+  a.k_bytes = (uint32_t)(p.HKV * p.DQK * es);
+  a.v_bytes = (uint32_t)(p.HKV * p.DV * es);
+  a.slot_bytes = (a.k_bytes + a.v_bytes + 127) & ~127u;
+  int ns = (int)((96 * 1024) / a.slot_bytes);
+  ns = ns < 2 ? 2 : (ns > 16 ? 16 : ns);
+  a.nslots = ns;
+  const size_t smem = 1024 + (size_t)ns * a.slot_bytes;
+  if (smem > 227 * 1024) return cudaErrorNotSupported;
+  const int hpw = heads_per_warp(p.H);
+  if (hpw == 0) return cudaErrorNotSupported;
+  const unsigned grid = (unsigned)(rows * a.nsplit);
+  if (p.dtype == 0) return launch_hpw<float>(a, hpw, smem, grid, rows, st);
+  return launch_hpw<__nv_bfloat16>(a, hpw, smem, grid, rows, st);
+}
+
+}  // namespace dsa

@@ -1,0 +1,49 @@
+// Host-side launchers of the libdsa kernels (internal; the public ABI is include/dsa.h).
+// Every launcher only enqueues work and returns the launch error, if any.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace dsa {
+
+// Indexer scores, SIMT (float32 FMA) kernel: any dtype, DI <= 128.
+cudaError_t launch_index_scores_simt(int dtype, const void* q_idx, const void* k_idx,
+                                     const float* w, float scale, int relu, int B, int S,
+                                     int T, int HI, int DI, int q_off, float* scores,
+                                     cudaStream_t st);
+
+// Indexer scores on the tensor cores (tcgen05 + TMEM + TMA): bf16, DI in {64,128,...}.
+// Returns cudaErrorNotSupported for shapes it does not take.
+bool index_scores_tc_supported(int dtype, int HI, int DI);
+cudaError_t launch_index_scores_tc(const void* q_idx, const void* k_idx, const float* w,
+                                   float scale, int relu, int B, int S, int T, int HI, int DI,
+                                   int q_off, float* scores, int write_masked,
+                                   cudaStream_t st);
+
+// Per-row top-k (radix select + ordered compaction).  `mask` (optional) receives the
+// selection bitmask [rows, ceil(T/32)] words.
+cudaError_t launch_topk(const float* scores, int B, int S, int T, int K, int q_off,
+                        int32_t* idx, uint32_t* mask, cudaStream_t st);
+
+// Gather attention (idx lists) and band attention (sliding window, GQA) share one kernel.
+struct AttnProblem {
+  int dtype;          // 0 f32, 1 bf16
+  const void* q;      // [B,S,H,DQK]
+  const void* k;      // [B,T,HKV,DQK]
+  const void* v;      // [B,T,HKV,DV]
+  const int32_t* idx; // [B,S,K] or NULL for the band
+  int K;              // idx columns
+  int window;         // band width when idx == NULL
+  const void* gate;   // [B,S,H] or NULL
+  int gate_mode;
+  float sm_scale;
+  int B, S, T, H, HKV, DQK, DV, q_off;
+  void* out;          // [B,S,H,DV]
+};
+size_t gather_attn_workspace_bytes(int B, int S, int H, int DV, int K);
+cudaError_t launch_gather_attn(const AttnProblem& p, void* ws, size_t ws_bytes,
+                               cudaStream_t st);
+
+}  // namespace dsa

@@ -1,0 +1,206 @@
+// Per-query top-k of the indexer scores.
+//
+// [AXK2] SGA: the indexer returns int32 indices [B, S, topk] of the keys each query keeps;
+// "AXK2Config" (index_topk): topk = min(index_topk, number of keys).  [PANGU] §3.3: the
+// number of selected keys is a fixed K.
+//
+// Order: higher score first, then lower key index (-0.0 == +0.0).  Output: the selected
+// keys in ascending index order, then -1 padding.  The selection is exact: a radix select
+// on order-preserving 32-bit keys (digits of 11, 11 and 10 bits, most significant first)
+// finds the threshold key tau and the number `need` of keys equal to tau that still fit;
+// an ordered compaction pass then keeps every key > tau and the first `need` keys == tau.
+//
+// One CTA per query row.  Pass 1 reads the row from HBM; the later passes re-read it from
+// L2 (a row is at most a few hundred KB and was just touched).  Histograms are built with
+// warp-aggregated shared-memory atomics (__match_any_sync groups equal digits, one atomic
+// per distinct digit per warp): integer-valued scores repeat heavily, so plain atomics
+// would serialise.  The compaction is a block-wide ballot/popc scan in index order, so the
+// output is deterministic and needs no sort.  The same ballots give the selection bitmask
+// (one bit per key) for the masked-tile attention path.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace dsa {
+
+namespace {
+
+constexpr int kBins = 2048;
+
+__device__ __forceinline__ uint32_t order_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  if ((u << 1) == 0u) u = 0u;  // -0.0 -> +0.0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Block-wide exclusive prefix sum of one int per thread (blockDim.x <= 1024).
+__device__ __forceinline__ int block_excl_scan(int v, int* warp_buf, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_buf[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int wv = lane < nwarps ? warp_buf[lane] : 0;
+    int ws = wv;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, ws, o);
+      if (lane >= o) ws += y;
+    }
+    if (lane < nwarps) warp_buf[lane] = ws - wv;  // exclusive warp offsets
+    if (lane == 31) *total = ws;
+  }
+  __syncthreads();
+  int r = warp_buf[warp] + x - v;
+  __syncthreads();  // warp_buf may be reused right after
+  return r;
+}
+
+template <int NT>
+__global__ void __launch_bounds__(NT) topk_rows_kernel(const float* __restrict__ scores, int S,
+                                                       int Tn, int K, int q_off,
+                                                       int32_t* __restrict__ idx,
+                                                       uint32_t* __restrict__ mask) {
+  __shared__ uint32_t hist[kBins];
+  __shared__ int warp_buf[32];
+  __shared__ int scan_total;
+  __shared__ uint32_t sel_bin;
+  __shared__ int sel_above;
+  __shared__ int wgt[NT / 32], weq[NT / 32];
+
+  const size_t row = blockIdx.x;
+  const int s = (int)(row % (size_t)S);
+  const int n = min(Tn, s + q_off + 1);
+  const float* sc = scores + row * (size_t)Tn;
+  int32_t* out = idx + row * (size_t)K;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int mwords = (Tn + 31) >> 5;
+  uint32_t* mrow = mask ? mask + row * (size_t)mwords : nullptr;
+
+  if (n <= K) {  // every valid key is kept
+    for (int i = tid; i < K; i += NT) out[i] = i < n ? i : -1;
+    if (mrow)
+      for (int wd = tid; wd < mwords; wd += NT) {
+        int lo = wd * 32;
+        uint32_t m = lo + 32 <= n ? 0xffffffffu : (lo >= n ? 0u : ((1u << (n - lo)) - 1u));
+        mrow[wd] = m;
+      }
+    return;
+  }
+
+  // ---------------- radix select: find the threshold prefix and `need`
+  uint32_t prefix = 0;
+  int pbits = 0;
+  int need = K;
+  const int widths[3] = {11, 11, 10};
+  for (int pass = 0; pass < 3; ++pass) {
+    const int dw = widths[pass];
+    const int shift = 32 - pbits - dw;
+    for (int i = tid; i < kBins; i += NT) hist[i] = 0;
+    __syncthreads();
+    for (int i0 = 0; i0 < n; i0 += NT) {
+      const int i = i0 + tid;
+      uint32_t digit = 0xffffffffu;
+      if (i < n) {
+        uint32_t key = order_key(sc[i]);
+        bool match = pbits == 0 || (key >> (32 - pbits)) == prefix;
+        if (match) digit = (key >> shift) & ((1u << dw) - 1u);
+      }
+      uint32_t peers = __match_any_sync(0xffffffffu, digit);
+      if (digit != 0xffffffffu && lane == __ffs(peers) - 1)
+        atomicAdd(&hist[digit], (uint32_t)__popc(peers));
+    }
+    __syncthreads();
+    // bins from the top: thread j owns a contiguous run of bins, highest first
+    constexpr int kPer = kBins / NT;
+    const int hi_bin = kBins - tid * kPer;  // exclusive upper end of my run
+    int local = 0;
+#pragma unroll
+    for (int q = 1; q <= kPer; ++q) local += (int)hist[hi_bin - q];
+    int above = block_excl_scan(local, warp_buf, &scan_total);
+#pragma unroll
+    for (int q = 1; q <= kPer; ++q) {
+      int c = (int)hist[hi_bin - q];
+      if (above < need && above + c >= need) {
+        sel_bin = (uint32_t)(hi_bin - q);
+        sel_above = above;
+      }
+      above += c;
+    }
+    __syncthreads();
+    const uint32_t bsel = sel_bin;
+    need -= sel_above;
+    prefix = (prefix << dw) | bsel;
+    pbits += dw;
+    const bool all_taken = (int)hist[bsel] == need;
+    __syncthreads();
+    if (all_taken) break;  // every key in the bucket is kept: no need to refine further
+  }
+
+  // ---------------- ordered compaction
+  const int fshift = 32 - pbits;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  int run_gt = 0, run_eq = 0;
+  for (int i0 = 0; i0 < n; i0 += NT) {
+    const int i = i0 + tid;
+    bool gt = false, eq = false;
+    if (i < n) {
+      uint32_t hi = order_key(sc[i]) >> fshift;
+      gt = hi > prefix;
+      eq = hi == prefix;
+    }
+    const uint32_t bgt = __ballot_sync(0xffffffffu, gt);
+    const uint32_t beq = __ballot_sync(0xffffffffu, eq);
+    if (lane == 0) {
+      wgt[warp] = __popc(bgt);
+      weq[warp] = __popc(beq);
+    }
+    __syncthreads();
+    int pg = run_gt, pe = run_eq, tg = 0, te = 0;
+#pragma unroll 4
+    for (int w2 = 0; w2 < NT / 32; ++w2) {
+      int a = wgt[w2], c = weq[w2];
+      if (w2 < warp) { pg += a; pe += c; }
+      tg += a; te += c;
+    }
+    const int my_gt = pg + __popc(bgt & lt_mask);
+    const int my_eq = pe + __popc(beq & lt_mask);
+    const bool sel = gt || (eq && my_eq < need);
+    const int pos = my_gt + min(my_eq, need);
+    if (sel && pos < K) out[pos] = i;
+    if (mrow) {
+      const uint32_t bsel = __ballot_sync(0xffffffffu, sel);
+      const int wd = (i0 >> 5) + warp;
+      if (lane == 0 && wd < mwords) mrow[wd] = bsel;
+    }
+    run_gt += tg;
+    run_eq += te;
+    __syncthreads();
+  }
+  if (mrow) {
+    const int written = min(mwords, ((n + NT - 1) / NT) * (NT / 32));
+    for (int wd = written + tid; wd < mwords; wd += NT) mrow[wd] = 0u;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_topk(const float* scores, int B, int S, int T, int K, int q_off,
+                        int32_t* idx, uint32_t* mask, cudaStream_t st) {
+  const size_t rows = (size_t)B * S;
+  if (rows == 0) return cudaSuccess;
+  if (T >= 8192)
+    topk_rows_kernel<1024><<<(unsigned)rows, 1024, 0, st>>>(scores, S, T, K, q_off, idx, mask);
+  else if (T >= 2048)
+    topk_rows_kernel<512><<<(unsigned)rows, 512, 0, st>>>(scores, S, T, K, q_off, idx, mask);
+  else
+    topk_rows_kernel<256><<<(unsigned)rows, 256, 0, st>>>(scores, S, T, K, q_off, idx, mask);
+  return cudaGetLastError();
+}
+
+}  // namespace dsa

@@ -1,0 +1,136 @@
+"""The C-ABI library: it loads without a GPU, exports every entry point include/dsa.h
+declares, and rejects invalid arguments on the host, before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(dsa_[a-z_]+)\s*\(",
+                                text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_path():
+    names = _declared_functions()
+    for required in ("dsa_index_scores", "dsa_topk", "dsa_sparse_attn", "dsa_forward"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    L = lib.lib()
+    for name in _declared_functions():
+        assert hasattr(L, name), f"libdsa.so does not export {name}"
+
+
+def test_version_and_status_strings(lib):
+    L = lib.lib()
+    assert b"sm_100a" in L.dsa_version()
+    assert L.dsa_status_string(0) == b"ok"
+    assert L.dsa_status_string(4) == b"in-kernel wait timed out"
+
+
+FAKE = ctypes.c_void_p(0x10000)  # never dereferenced: validation fails first
+FAKE_MIS = ctypes.c_void_p(0x10008)  # 8-byte aligned only
+
+
+def _index(L, **kw):
+    a = dict(dtype=1, q=FAKE, k=FAKE, w=FAKE, scale=0.5, relu=0, B=1, S=4, T=4, HI=2, DI=64,
+             scores=FAKE)
+    a.update(kw)
+    return L.dsa_index_scores(a["dtype"], a["q"], a["k"], a["w"], a["scale"], a["relu"], a["B"],
+                              a["S"], a["T"], a["HI"], a["DI"], a["scores"], None)
+
+
+def test_index_scores_rejects_bad_arguments(lib):
+    L = lib.lib()
+    assert _index(L, q=None) == 1
+    assert _index(L, B=0) == 1
+    assert _index(L, S=8, T=4) == 1          # queries must be the last S of T keys
+    assert _index(L, scale=0.0) == 1
+    assert _index(L, scale=float("nan")) == 1
+    assert _index(L, relu=7) == 1
+    assert _index(L, dtype=5) == 1
+    assert _index(L, DI=60) == 2             # not a multiple of 8 for bf16
+    assert _index(L, DI=256) == 2
+    assert _index(L, q=FAKE_MIS) == 2        # misaligned
+    assert b"16-byte" in L.dsa_last_error()
+
+
+def test_topk_rejects_bad_arguments(lib):
+    L = lib.lib()
+    assert L.dsa_topk(None, 1, 4, 4, 2, FAKE, None) == 1
+    assert L.dsa_topk(FAKE, 1, 4, 4, 0, FAKE, None) == 1
+    assert L.dsa_topk(FAKE, 1, 5, 4, 2, FAKE, None) == 1
+    assert L.dsa_topk(FAKE, 1, 4, 4, 2, FAKE_MIS, None) == 2
+
+
+def _attn(L, **kw):
+    a = dict(dtype=1, q=FAKE, k=FAKE, v=FAKE, idx=FAKE, K=4, gate=None, gm=0, sm=0.0, B=1, S=4,
+             T=8, H=4, DQK=64, DV=64, out=FAKE, ws=None, wsb=0)
+    a.update(kw)
+    return L.dsa_sparse_attn(a["dtype"], a["q"], a["k"], a["v"], a["idx"], a["K"], a["gate"],
+                             a["gm"], a["sm"], a["B"], a["S"], a["T"], a["H"], a["DQK"], a["DV"],
+                             a["out"], a["ws"], a["wsb"], None)
+
+
+def test_sparse_attn_rejects_bad_arguments(lib):
+    L = lib.lib()
+    assert _attn(L, gm=1) == 1                    # gate on but no gate pointer
+    assert _attn(L, gate=FAKE, gm=0) == 1         # gate pointer with the gate off
+    assert _attn(L, gate=FAKE, gm=3) == 1         # only sigmoid and silu exist
+    assert _attn(L, idx=None) == 1
+    assert _attn(L, K=0) == 1
+    assert _attn(L, DQK=300) == 2
+    assert _attn(L, v=FAKE_MIS) == 2
+    assert _attn(L, sm=float("inf")) == 1
+    # decode-shaped work needs a split-key workspace; too small a workspace is rejected
+    need = L.dsa_sparse_attn_workspace_bytes(2, 1, 131072, 32, 128, 2048)
+    assert need > 0
+    assert _attn(L, B=2, S=1, T=131072, H=32, DQK=192, DV=128, K=2048, ws=FAKE,
+                 wsb=need - 1) == 1
+
+
+def test_window_attn_rejects_bad_arguments(lib):
+    L = lib.lib()
+    f = L.dsa_window_attn
+    assert f(1, FAKE, FAKE, FAKE, None, 0, 0.0, 512, 1, 1024, 1024, 32, 6, 192, 128, FAKE,
+             None) == 1  # 32 heads over 6 KV heads
+    assert f(1, FAKE, FAKE, FAKE, None, 0, 0.0, 0, 1, 1024, 1024, 32, 8, 192, 128, FAKE,
+             None) == 1  # empty window
+
+
+def test_forward_workspace_and_validation(lib):
+    L = lib.lib()
+    a = lib.ForwardArgs(dtype=1, B=1, S=4096, T=4096, HI=16, DI=64, index_scale=2 ** -4,
+                        relu=0, K=512, H=20, DQK=128, DV=128, sm_scale=0.0, gate_mode=0,
+                        attn_algo=0, q_idx=0x10000, k_idx=0x10000, w=0x10000, q=0x10000,
+                        k=0x10000, v=0x10000, gate=None, out=0x10000, scores_out=None,
+                        idx_out=None)
+    full = lib.dsa_forward_workspace_bytes(a)
+    small = lib.dsa_forward_workspace_bytes(a, minimum=True)
+    assert full >= 4096 * 4096 * 4 + 4096 * 512 * 4
+    assert small < full
+    assert L.dsa_forward(ctypes.byref(a), FAKE, small - 1, None) == 1
+    a.gate_mode = 1  # gate on without a gate tensor
+    assert L.dsa_forward(ctypes.byref(a), FAKE, full, None) == 1
+    a.gate_mode = 0
+    a.attn_algo = 9
+    assert L.dsa_forward(ctypes.byref(a), FAKE, full, None) == 1
+
+
+def test_binding_fails_loudly_without_library(monkeypatch):
+    import sparse_attention_15_b200 as dsa
+    monkeypatch.setattr(dsa, "_LIB", None)
+    monkeypatch.setattr(dsa, "LIB_PATH", "/nonexistent/libdsa.so")
+    with pytest.raises(RuntimeError, match="no fallback"):
+        dsa.lib()

@@ -1,0 +1,266 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 CPU oracle.
+
+Small cases span several tiles with ragged tails and are compared element by element;
+the full-size workloads run in the launch configuration the benchmark times and are
+compared on sampled rows, plus size-independent properties on every row.
+Indices are compared bit-exactly; scores too (integer inputs, power-of-two scales make
+every float32 partial sum exact); attention outputs within the stated tolerance.
+"""
+import numpy as np
+import pytest
+import torch
+
+import sparse_attention_15_b200 as dsa
+from oracle import dsa_oracle as O
+import parity as P
+from workloads import dsa_inputs, get_config, swa_inputs
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+@pytest.fixture(autouse=True)
+def _gpu(lib, cuda_dev):
+    yield
+    torch.cuda.synchronize()
+    dsa.dsa_device_status(reset=True)  # raises if a kernel flagged a timeout
+    torch.cuda.empty_cache()
+
+
+def _inputs(name, S, T, B=1, seed=None, K=None):
+    cfg = get_config(name)
+    x = dsa_inputs(cfg, device="cpu", B=B, S=S, T=T, seed=seed)
+    return cfg, x, {k: (None if v is None else v.to(DEV)) for k, v in x.items()}
+
+
+# ------------------------------------------------------------------------------- indexer
+SMALL = [("c1", 256, 256), ("c2", 333, 333), ("c2", 100, 517), ("c3", 200, 455),
+         ("c5", 131, 300)]
+
+
+@pytest.mark.parametrize("name,S,T", SMALL)
+@pytest.mark.parametrize("relu", ["none", "post_sum", "per_head"])
+def test_index_scores_exact(name, S, T, relu):
+    cfg, x, g = _inputs(name, S, T)
+    got = dsa.dsa_index_scores(g["q_idx"], g["k_idx"], g["w"], cfg.scale, relu=relu)
+    ref = O.index_scores(x["q_idx"], x["k_idx"], x["w"], cfg.scale, relu=relu)
+    assert np.array_equal(P.to_np(got), ref.astype(np.float32))
+
+
+# ------------------------------------------------------------------------------- top-k
+@pytest.mark.parametrize("name,S,T", SMALL)
+@pytest.mark.parametrize("K", [1, 16, 100, 400])
+def test_topk_exact_on_indexer_scores(name, S, T, K):
+    cfg, x, g = _inputs(name, S, T)
+    sc = dsa.dsa_index_scores(g["q_idx"], g["k_idx"], g["w"], cfg.scale)
+    got = dsa.dsa_topk(sc, K)
+    ref = O.topk_indices(P.to_np(sc).astype(np.float64), K)
+    assert np.array_equal(P.to_np(got), ref)
+
+
+def _adversarial_scores(kind, S, T, seed):
+    g = torch.Generator().manual_seed(seed)
+    if kind == "all_equal":
+        x = torch.zeros(1, S, T)
+    elif kind == "signed_zeros":
+        x = torch.randint(-1, 2, (1, S, T), generator=g).float()
+        z = torch.rand(1, S, T, generator=g) < 0.5
+        x = torch.where((x == 0) & z, torch.tensor(-0.0), x)
+    elif kind == "few_values":
+        x = torch.randint(-3, 4, (1, S, T), generator=g).float() * 0.75
+    elif kind == "wide_range":
+        x = torch.randn(1, S, T, generator=g) * torch.exp(torch.randn(1, S, T, generator=g) * 8)
+    elif kind == "neg_inf_inside":
+        x = torch.randn(1, S, T, generator=g)
+        x[torch.rand(1, S, T, generator=g) < 0.3] = float("-inf")
+    elif kind == "dup_floats":
+        x = torch.randn(1, S, T // 4 + 1, generator=g).repeat(1, 1, 4)[..., :T].contiguous()
+    else:
+        raise ValueError(kind)
+    return x
+
+
+@pytest.mark.parametrize("kind", ["all_equal", "signed_zeros", "few_values", "wide_range",
+                                  "neg_inf_inside", "dup_floats"])
+@pytest.mark.parametrize("S,T,K", [(64, 64, 8), (40, 3000, 700), (6, 20000, 2048)])
+def test_topk_exact_adversarial(kind, S, T, K):
+    x = _adversarial_scores(kind, S, T, seed=S + T)
+    got = dsa.dsa_topk(x.to(DEV), K)
+    ref = O.topk_indices(x.double().numpy() + 0.0, K)
+    assert np.array_equal(P.to_np(got), ref)
+
+
+# ------------------------------------------------------------------------------- attention
+ATTN = [("c1", 256, 256, 16), ("c2", 333, 333, 64), ("c2", 100, 517, 512), ("c3", 150, 300, 40),
+        ("c5", 64, 200, 2048)]
+
+
+@pytest.mark.parametrize("name,S,T,K", ATTN)
+@pytest.mark.parametrize("gate_mode", ["off", "sigmoid", "silu"])
+def test_sparse_attn_parity(name, S, T, K, gate_mode):
+    cfg, x, g = _inputs(name, S, T)
+    sc = O.index_scores(x["q_idx"], x["k_idx"], x["w"], cfg.scale)
+    idx = O.topk_indices(sc, min(K, T))
+    gate = None
+    if gate_mode != "off":
+        gate = torch.randn(1, S, cfg.H, generator=torch.Generator().manual_seed(5)).to(
+            x["q"].dtype)
+    got = dsa.dsa_sparse_attn(g["q"], g["k"], g["v"], torch.from_numpy(idx).to(DEV),
+                              gate=None if gate is None else gate.to(DEV), gate_mode=gate_mode)
+    ref = O.sparse_attention(x["q"], x["k"], x["v"], idx, gate=gate, gate_mode=gate_mode)
+    P.assert_attn_close(got, ref, x["q"].dtype, f"{name} {gate_mode}")
+
+
+def test_sparse_attn_skips_invalid_and_future_indices():
+    cfg, x, g = _inputs("c2", 40, 90)
+    rng = np.random.default_rng(0)
+    idx = rng.integers(-3, 140, size=(1, 40, 24)).astype(np.int32)  # -1s, future, out of range
+    for s in range(40):  # entries must be distinct
+        row = idx[0, s]
+        _, first = np.unique(row, return_index=True)
+        dup = np.ones(row.size, bool)
+        dup[first] = False
+        row[dup] = -1
+    got = dsa.dsa_sparse_attn(g["q"], g["k"], g["v"], torch.from_numpy(idx).to(DEV))
+    ref = O.sparse_attention(x["q"], x["k"], x["v"], idx)
+    P.assert_attn_close(got, ref, torch.bfloat16, "invalid indices")
+
+
+# ------------------------------------------------------------------------------- forward
+@pytest.mark.parametrize("name,S,T", [("c1", 256, 256), ("c2", 600, 600), ("c3", 260, 330),
+                                      ("c2", 120, 700)])
+def test_forward_parity(name, S, T):
+    cfg, x, g = _inputs(name, S, T)
+    K = min(cfg.K, 96) if name != "c1" else cfg.K
+    scores = torch.empty((1, S, T), dtype=torch.float32, device=DEV)
+    out, idx = dsa.dsa_forward(g["q_idx"], g["k_idx"], g["w"], cfg.scale, K, g["q"], g["k"],
+                               g["v"], gate=g["gate"], scores_out=scores)
+    sc_ref, idx_ref, out_ref = O.dsa_forward(x["q_idx"], x["k_idx"], x["w"], cfg.scale, K,
+                                             x["q"], x["k"], x["v"], gate=x["gate"],
+                                             gate_mode=cfg.gate)
+    assert np.array_equal(P.to_np(scores), sc_ref.astype(np.float32))
+    assert np.array_equal(P.to_np(idx), idx_ref)
+    P.assert_attn_close(out, out_ref, x["q"].dtype, name)
+    # the row-blocked path (workspace smaller than the score matrix) gives the same bits
+    out2 = torch.empty_like(out)
+    idx2 = torch.empty_like(idx)
+    args = dsa._forward_args(g["q_idx"], g["k_idx"], g["w"], cfg.scale, K, g["q"], g["k"],
+                             g["v"], g["gate"], None, "none", 0.0, "auto", out2, None, idx2)
+    small = dsa.dsa_forward_workspace_bytes(args, minimum=True) + 37 * T * 4
+    dsa.dsa_forward(g["q_idx"], g["k_idx"], g["w"], cfg.scale, K, g["q"], g["k"], g["v"],
+                    gate=g["gate"], out=out2, idx_out=idx2, ws_bytes=small)
+    assert torch.equal(idx2, idx)
+    assert torch.equal(out2, out)
+
+
+# ------------------------------------------------------------------------------- window
+@pytest.mark.parametrize("S,T,W", [(300, 300, 128), (700, 700, 512), (100, 640, 512)])
+def test_window_attn_parity(S, T, W):
+    cfg = get_config("c5")
+    x = swa_inputs(cfg, 1, device="cpu", S=S, T=T)
+    g = {k: v.to(DEV) for k, v in x.items()}
+    got = dsa.dsa_window_attn(g["q"], g["k"], g["v"], W, gate=g["gate"])
+    ref = O.window_attention(x["q"], x["k"], x["v"], W, gate=x["gate"], gate_mode="sigmoid")
+    P.assert_attn_close(got, ref, torch.bfloat16, f"swa W={W}")
+
+
+# ------------------------------------------------------------------------------- invariants
+def test_gpu_invariants_gate_zero_halves_and_determinism():
+    cfg, x, g = _inputs("c3", 256, 256)
+    sc = dsa.dsa_index_scores(g["q_idx"], g["k_idx"], g["w"], cfg.scale)
+    idx = dsa.dsa_topk(sc, 64)
+    base = dsa.dsa_sparse_attn(g["q"], g["k"], g["v"], idx)
+    zero = torch.zeros(1, 256, cfg.H, dtype=torch.bfloat16, device=DEV)
+    gated = dsa.dsa_sparse_attn(g["q"], g["k"], g["v"], idx, gate=zero, gate_mode="sigmoid")
+    assert torch.equal(gated.float(), base.float() * 0.5)  # power-of-two scaling is exact
+    again = dsa.dsa_sparse_attn(g["q"], g["k"], g["v"], idx)
+    assert torch.equal(again, base)
+    # poisoning every unselected key leaves the outputs bitwise unchanged
+    sel = torch.zeros(256, dtype=torch.bool, device=DEV)
+    sel[idx[0].flatten()[idx[0].flatten() >= 0].long()] = True
+    k2, v2 = g["k"].clone(), g["v"].clone()
+    k2[0, ~sel] = 30.0
+    v2[0, ~sel] = 1e4
+    assert torch.equal(dsa.dsa_sparse_attn(g["q"], k2, v2, idx), base)
+
+
+# ------------------------------------------------------------------------------- full size
+def _full_inputs(name, B=None):
+    cfg = get_config(name)
+    return cfg, dsa_inputs(cfg, device=DEV, B=B)
+
+
+def _sample_rows(S, K, n=48, seed=0):
+    rng = np.random.default_rng(seed)
+    fixed = [0, 1, K - 2, K - 1, K, K + 1, S - 1]
+    rows = sorted(set([r for r in fixed if 0 <= r < S] + list(rng.integers(0, S, n))))
+    return rows
+
+
+@pytest.mark.parametrize("name", ["c2", "c3", "c5"])
+def test_full_size_prefill(name):
+    cfg, g = _full_inputs(name)
+    B, S, T, K = cfg.B, cfg.S, cfg.T, cfg.k_eff
+    scores = torch.empty((B, S, T), dtype=torch.float32, device=DEV)
+    out, idx = dsa.dsa_forward(g["q_idx"], g["k_idx"], g["w"], cfg.scale, cfg.K, g["q"], g["k"],
+                               g["v"], gate=g["gate"], scores_out=scores)
+    torch.cuda.synchronize()
+    # every score, exactly (integer arithmetic in torch float32)
+    ref_all = P.torch_exact_scores(g["q_idx"], g["k_idx"], g["w"], cfg.scale, cfg.q_off)
+    assert torch.equal(scores, ref_all)
+    del ref_all
+    # every row's indices: the unique top-k of those scores
+    P.check_topk_properties(scores, idx, K, cfg.q_off)
+    # sampled rows against the oracle: scores, indices, attention
+    rows = _sample_rows(S, K)
+    qi, ki, w = (g[n].cpu() for n in ("q_idx", "k_idx", "w"))
+    sc_ref = P.oracle_score_rows(qi, ki, w, cfg.scale, rows, cfg.q_off)
+    assert np.array_equal(P.to_np(scores[0, rows]), sc_ref.astype(np.float32))
+    idx_ref = np.stack([O.topk_indices(sc_ref[i][None, None], K, q_off=r + cfg.q_off)[0, 0]
+                        for i, r in enumerate(rows)])
+    assert np.array_equal(P.to_np(idx[0, rows]), idx_ref)
+    att_ref = P.oracle_attn_rows(g["q"], g["k"], g["v"], idx_ref, rows, cfg.q_off,
+                                 gate=g["gate"], gate_mode=cfg.gate)
+    P.assert_attn_close(out[0, rows], att_ref, torch.bfloat16, f"{name} full")
+
+
+def test_full_size_decode():
+    cfg = get_config("c4")
+    free, _ = torch.cuda.mem_get_info()
+    per_row = cfg.T * (cfg.DI + cfg.H * (cfg.dqk + cfg.dv)) * 2
+    B = cfg.B if free > per_row * cfg.B + (8 << 30) else max(1, int((free - (8 << 30)) // per_row))
+    if B < cfg.B:
+        print(f"decode parity at B={B} (free memory {free / 2**30:.1f} GiB)")
+    cfg, g = _full_inputs("c4", B=B)
+    K = cfg.k_eff
+    scores = torch.empty((B, 1, cfg.T), dtype=torch.float32, device=DEV)
+    out, idx = dsa.dsa_forward(g["q_idx"], g["k_idx"], g["w"], cfg.scale, cfg.K, g["q"], g["k"],
+                               g["v"], gate=g["gate"], scores_out=scores)
+    torch.cuda.synchronize()
+    assert torch.equal(scores, P.torch_exact_scores(g["q_idx"], g["k_idx"], g["w"], cfg.scale,
+                                                    cfg.q_off))
+    P.check_topk_properties(scores, idx, K, cfg.q_off)
+    qi, ki, w = (g[n].cpu() for n in ("q_idx", "k_idx", "w"))
+    for b in sorted(set([0, B - 1] + list(np.random.default_rng(1).integers(0, B, 6)))):
+        sc_ref = P.oracle_score_rows(qi, ki, w, cfg.scale, [0], cfg.q_off, b=b)
+        assert np.array_equal(P.to_np(scores[b, 0]), sc_ref[0].astype(np.float32))
+        idx_ref = O.topk_indices(sc_ref[None], K, q_off=cfg.q_off)[0]
+        assert np.array_equal(P.to_np(idx[b]), idx_ref)
+        att_ref = P.oracle_attn_rows(g["q"], g["k"], g["v"], idx_ref, [0], cfg.q_off, b=b)
+        P.assert_attn_close(out[b], att_ref, torch.bfloat16, f"decode b={b}")
+
+
+def test_full_size_window():
+    cfg = get_config("c5")
+    x = swa_inputs(cfg, 1, device=DEV)
+    out = dsa.dsa_window_attn(x["q"], x["k"], x["v"], cfg.window, gate=x["gate"])
+    torch.cuda.synchronize()
+    rows = _sample_rows(cfg.S, cfg.window, n=24)
+    for s in rows:
+        lo = max(0, s - cfg.window + 1)
+        sl = slice(lo, s + 1)
+        ref = O.window_attention(x["q"][:, s:s + 1].cpu(), x["k"][:, sl].cpu(), x["v"][:, sl].cpu(),
+                                 cfg.window, gate=x["gate"][:, s:s + 1].cpu(),
+                                 gate_mode="sigmoid")
+        P.assert_attn_close(out[:, s:s + 1], ref, torch.bfloat16, f"swa full s={s}")
