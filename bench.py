@@ -160,12 +160,17 @@ class Workload:
         x = dsa_inputs(cfg, device=device, B=B, seed=cfg.seed + seed_offset)
         self.x = x
         self.K = cfg.k_eff
-        self.scores = torch.empty((B, cfg.S, cfg.T), dtype=torch.float32, device=device)
         self.idx = torch.empty((B, cfg.S, self.K), dtype=torch.int32, device=device)
         self.out = torch.empty((B, cfg.S, cfg.H, cfg.dv), dtype=x["q"].dtype, device=device)
-        nb = dsa.dsa_sparse_attn_workspace_bytes(B, cfg.S, cfg.T, cfg.H, cfg.dv, self.K)
-        self.ws = torch.empty(max(nb, 16), dtype=torch.uint8, device=device)
-        self.ws_bytes = nb
+        self.args = dsa._forward_args(x["q_idx"], x["k_idx"], x["w"], cfg.scale, cfg.K, x["q"],
+                                      x["k"], x["v"], x["gate"], None, "none", 0.0, "auto",
+                                      self.out, None, self.idx)
+        self.ws_bytes = dsa.dsa_forward_workspace_bytes(self.args)
+        self.ws = torch.empty(max(self.ws_bytes, 16), dtype=torch.uint8, device=device)
+        dt = dsa.DTYPE[x["q"].dtype]
+        self.algo = dsa.dsa_sparse_attn_algo(dt, B, cfg.S, cfg.T, cfg.H, cfg.dqk, cfg.dv, self.K)
+        gather_ws = dsa.dsa_sparse_attn_workspace_bytes(dt, B, cfg.S, cfg.T, cfg.H, cfg.dqk,
+                                                        cfg.dv, self.K, "gather")
         self.swa = []
         for layer in range(1, cfg.swa_layers + 1):
             s = swa_inputs(cfg, layer, device=device, seed=cfg.seed + seed_offset)
@@ -173,19 +178,16 @@ class Workload:
             self.swa.append(s)
         self.stages = ["indexer", "topk", "attention"] + [f"swa{i + 1}" for i in
                                                           range(len(self.swa))]
-        self.launches_per_step = 3 + (1 if nb > 0 else 0) + len(self.swa)
+        # our kernels per step: indexer, top-k, attention (+ combine for split gathers), SWA
+        self.launches_per_step = 3 + (1 if self.algo == "gather" and gather_ws > 0 else 0) + \
+            len(self.swa)
 
     def step(self, ev):
-        """Run one step; ev is a list of len(stages)+1 CUDA events recorded between calls."""
+        """Run one step; ev is a list of len(stages)+1 CUDA events (stage boundaries)."""
         c, x, d = self.cfg, self.x, self.dsa
-        ev[0].record()
-        d.dsa_index_scores(x["q_idx"], x["k_idx"], x["w"], c.scale, scores=self.scores)
-        ev[1].record()
-        d.dsa_topk(self.scores, self.K, idx=self.idx)
-        ev[2].record()
-        d.dsa_sparse_attn(x["q"], x["k"], x["v"], self.idx, gate=x["gate"], out=self.out,
-                          ws=self.ws)
-        ev[3].record()
+        d.dsa_forward(x["q_idx"], x["k_idx"], x["w"], c.scale, c.K, x["q"], x["k"], x["v"],
+                      gate=x["gate"], out=self.out, idx_out=self.idx, ws=self.ws,
+                      ws_bytes=self.ws_bytes, events=ev[:4])
         for i, s in enumerate(self.swa):
             d.dsa_window_attn(s["q"], s["k"], s["v"], c.window, gate=s["gate"], out=s["out"])
             ev[4 + i].record()
@@ -201,29 +203,48 @@ class Workload:
             "indexer": ("tensor" if c.dtype == "bf16" else "alu", 2.0 * c.HI * c.DI * pairs,
                         "TFLOP/s"),
             "topk": ("hbm", 4.0 * pairs + 4.0 * rows * self.K, "GB/s"),
-            "attention": ("hbm", sel * c.H * (c.dqk + c.dv) * es +
-                          rows * c.H * (c.dqk + c.dv) * es, "GB/s"),
         }
+        if self.algo == "masked_tile":
+            # dense attention under the mask: QK^T and PV over every causal pair, all heads
+            w["attention"] = ("tensor", 2.0 * c.H * (c.dqk + c.dv) * pairs, "TFLOP/s")
+        else:
+            w["attention"] = ("hbm", sel * c.H * (c.dqk + c.dv) * es +
+                              rows * c.H * (c.dqk + c.dv) * es, "GB/s")
         for i in range(len(self.swa)):
             band = selected_pairs(c.S, c.T, B, c.q_off, c.window)
-            w[f"swa{i + 1}"] = ("hbm", band * c.swa_kv_heads * (c.dqk + c.dv) * es +
-                                rows * c.H * (c.dqk + c.dv) * es, "GB/s")
+            w[f"swa{i + 1}"] = ("tensor", 2.0 * c.H * (c.dqk + c.dv) * band, "TFLOP/s")
         return w
 
     def host_copy(self):
-        """Pinned host copies of every input of the DSA layer (for the end-to-end leg)."""
-        return {k: (None if v is None else v.cpu().pin_memory()) for k, v in self.x.items()}
+        """Pinned host copies of what one step takes from the host.  Prefill: every input of
+        the DSA layer.  Decode: the new queries and the new token's cache rows (the caches
+        themselves stay resident in HBM)."""
+        x = self.x
+        if self.cfg.S == 1:
+            sel = {"q_idx": x["q_idx"], "w": x["w"], "q": x["q"], "gate": x["gate"],
+                   "k_idx_row": x["k_idx"][:, -1:], "k_row": x["k"][:, -1:],
+                   "v_row": x["v"][:, -1:]}
+        else:
+            sel = dict(x)
+        return {k: (None if v is None else v.contiguous().cpu().pin_memory())
+                for k, v in sel.items()}
 
     def e2e_step(self, host, dev_bufs, out_host):
         """Host inputs -> device -> dsa_forward -> result back to the host."""
+        x = dict(self.x)
         for k, v in host.items():
-            if v is not None:
+            if v is None:
+                continue
+            if k.endswith("_row"):
+                name = k[:-4]
+                x[name][:, -1:].copy_(v, non_blocking=True)
+            else:
                 dev_bufs[k].copy_(v, non_blocking=True)
-        x = dev_bufs
+                x[k] = dev_bufs[k]
         c = self.cfg
         self.dsa.dsa_forward(x["q_idx"], x["k_idx"], x["w"], c.scale, c.K, x["q"], x["k"],
                              x["v"], gate=x["gate"], out=self.out, idx_out=self.idx,
-                             ws=self.fwd_ws, ws_bytes=self.fwd_ws_bytes)
+                             ws=self.ws, ws_bytes=self.ws_bytes)
         out_host.copy_(self.out, non_blocking=True)
 
 
@@ -422,16 +443,16 @@ def main():
                          "frac": round(ach / peak, 4),
                          "share": round(float(stage_ms[j]) / float(stage_ms.sum()), 4)}
     dom = max(kernels, key=lambda k: kernels[k]["ms"])
-    kname = {"indexer": "index_scores", "topk": "topk", "attention": "gather_attn"}.get(
-        dom, "gather_attn")
+    attn_k = "masked_attn" if wl.algo == "masked_tile" else "gather_attn"
+    kname = {"indexer": "index_scores", "topk": "topk", "attention": attn_k}.get(dom, "masked_attn")
     tr = NCU_TRAFFIC.get((kname, cfg.name))
-    srcfile = {"index_scores": "indexer_tc.cu", "topk": "topk.cu",
-               "gather_attn": "gather_attn.cu"}[kname]
+    srcfile = {"index_scores": "indexer_tc.cu", "topk": "topk.cu", "gather_attn": "gather_attn.cu",
+               "masked_attn": "attn_tc.cu"}[kname]
     traffic = tr[0] if tr and tr[1] == src_sha(srcfile) else None
     roof = dict(kernels[dom])
     roof.pop("ms")
     roof.pop("share")
-    roof.update({"kernel": dom, "traffic": traffic,
+    roof.update({"kernel": dom, "attention_algo": wl.algo, "traffic": traffic,
                  "peak_source": f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'profiling recipe fallback'})"})
 
     # end-to-end through the public call with host buffers
@@ -439,15 +460,8 @@ def main():
     if not args.no_e2e:
         host = wl.host_copy()
         dev_bufs = {k: (None if v is None else torch.empty_like(v, device=dev))
-                    for k, v in host.items()}
+                    for k, v in host.items() if not k.endswith("_row")}
         out_host = torch.empty(wl.out.shape, dtype=wl.out.dtype).pin_memory()
-        import sparse_attention_15_b200 as dsa
-
-        a = dsa._forward_args(dev_bufs["q_idx"], dev_bufs["k_idx"], dev_bufs["w"], cfg.scale,
-                              cfg.K, dev_bufs["q"], dev_bufs["k"], dev_bufs["v"],
-                              dev_bufs["gate"], None, "none", 0.0, "auto", wl.out, None, wl.idx)
-        wl.fwd_ws_bytes = dsa.dsa_forward_workspace_bytes(a)
-        wl.fwd_ws = torch.empty(max(wl.fwd_ws_bytes, 16), dtype=torch.uint8, device=dev)
         for _ in range(args.warmup):
             wl.e2e_step(host, dev_bufs, out_host)
         torch.cuda.synchronize(dev)

@@ -72,7 +72,7 @@ typedef enum { DSA_RELU_NONE = 0, DSA_RELU_POST_SUM = 1, DSA_RELU_PER_HEAD = 2 }
  * (token, head), evaluated in float32; any other mode is rejected (the page's ValueError). */
 typedef enum { DSA_GATE_OFF = 0, DSA_GATE_SIGMOID = 1, DSA_GATE_SILU = 2 } dsa_gate_mode;
 
-/* Attention algorithm for dsa_forward / dsa_sparse_attn_ex. */
+/* Attention algorithm for dsa_forward, dsa_sparse_attn and dsa_window_attn. */
 typedef enum {
   DSA_ATTN_AUTO = 0,      /* pick by the cost model (bytes gathered vs. dense tile work)  */
   DSA_ATTN_GATHER = 1,    /* gather the selected K/V rows per query (decode-shaped work) */
@@ -132,17 +132,32 @@ dsa_status dsa_topk(const float* scores, int B, int S, int T, int K, int32_t* id
  *   out   [B,S,H,DV]   dtype      out: softmax-weighted sum of the selected v rows (float32
  *                                 accumulation, one rounding to dtype, gate applied before
  *                                 that rounding); a row with no valid key gets zeros.
- *   ws / ws_bytes                 scratch for split-key partial results; the size comes
- *                                 from dsa_sparse_attn_workspace_bytes (may be 0 -> NULL ok).
+ *   algo                          DSA_ATTN_GATHER gathers each query's selected K/V rows
+ *                                 (all heads share the index set, so one key is one
+ *                                 contiguous K row and one V row); DSA_ATTN_MASKED_TILE runs
+ *                                 dense tensor-core tiles of 128 queries x 128 keys under the
+ *                                 selection bitmask, which is what the page describes (dense
+ *                                 attention with the additive sparse mask); DSA_ATTN_AUTO
+ *                                 picks by the cost model (gathered bytes vs. dense flops).
+ *                                 Both give the same result within rounding.  The masked
+ *                                 tile needs bf16, DQK in {128, 192}, DV == 128.
+ *   ws / ws_bytes                 scratch: split-key partial results (gather) or the
+ *                                 selection bitmask (masked tile); the size comes from
+ *                                 dsa_sparse_attn_workspace_bytes (0 -> NULL is fine).
  *   Requires DQK <= 256, DV <= 256, H <= 64 (H a multiple of 2 above 16, of 4 above 32),
  *   and H*DQK, H*DV rows that are multiples of 16 bytes.
  * --------------------------------------------------------------------------------- */
-size_t dsa_sparse_attn_workspace_bytes(int B, int S, int T, int H, int DV, int K);
+size_t dsa_sparse_attn_workspace_bytes(dsa_dtype dtype, int B, int S, int T, int H, int DQK,
+                                       int DV, int K, dsa_attn_algo algo);
+/* The algorithm DSA_ATTN_AUTO resolves to for this shape (DSA_ATTN_GATHER or
+ * DSA_ATTN_MASKED_TILE; a request the shape cannot take resolves to DSA_ATTN_AUTO). */
+dsa_attn_algo dsa_sparse_attn_algo(dsa_dtype dtype, int B, int S, int T, int H, int DQK, int DV,
+                                   int K, dsa_attn_algo algo);
 dsa_status dsa_sparse_attn(dsa_dtype dtype, const void* q, const void* k, const void* v,
                            const int32_t* idx, int K, const void* gate,
                            dsa_gate_mode gate_mode, float sm_scale, int B, int S, int T,
-                           int H, int DQK, int DV, void* out, void* ws, size_t ws_bytes,
-                           dsa_stream_t stream);
+                           int H, int DQK, int DV, dsa_attn_algo algo, void* out, void* ws,
+                           size_t ws_bytes, dsa_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
  * The whole DSA step: 1 -> 2 -> 3+4.  [AXK2] "注意力前向的骨架" steps 4-5.
@@ -171,6 +186,9 @@ typedef struct {
   void* out;               /* [B,S,H,DV] out                                             */
   float* scores_out;       /* optional [B,S,T] out                                       */
   int32_t* idx_out;        /* optional [B,S,K_eff] out                                   */
+  void* const* events;     /* optional: 4 caller-owned cudaEvent_t recorded on the stream
+                              before the indexer, after it, after the top-k and after the
+                              attention (per-stage timing); NULL for none                */
 } dsa_forward_args;
 
 /* Bytes of workspace dsa_forward needs to run without row blocking. */
@@ -187,12 +205,14 @@ dsa_status dsa_forward(const dsa_forward_args* a, void* ws, size_t ws_bytes,
  *
  *   q [B,S,H,DQK], k [B,T,HKV,DQK], v [B,T,HKV,DV], gate [B,S,H] or NULL, out [B,S,H,DV];
  *   query head h reads KV head h / (H/HKV); query s sees keys
- *   s+q_off-window < t <= s+q_off.  Same arithmetic contract as dsa_sparse_attn.
+ *   s+q_off-window < t <= s+q_off.  Same arithmetic contract as dsa_sparse_attn; algo
+ *   DSA_ATTN_MASKED_TILE (and AUTO for S >= 64 where supported) runs tensor-core tiles over
+ *   the band, DSA_ATTN_GATHER streams the band's K/V rows.  No workspace.
  * --------------------------------------------------------------------------------- */
 dsa_status dsa_window_attn(dsa_dtype dtype, const void* q, const void* k, const void* v,
                            const void* gate, dsa_gate_mode gate_mode, float sm_scale,
                            int window, int B, int S, int T, int H, int HKV, int DQK, int DV,
-                           void* out, dsa_stream_t stream);
+                           dsa_attn_algo algo, void* out, dsa_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
  * Status and introspection.

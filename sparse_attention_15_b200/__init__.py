@@ -15,7 +15,7 @@ import torch
 
 __all__ = [
     "DSAError", "lib", "dsa_index_scores", "dsa_topk", "dsa_sparse_attn",
-    "dsa_sparse_attn_workspace_bytes", "dsa_forward", "dsa_forward_workspace_bytes",
+    "dsa_sparse_attn_workspace_bytes", "dsa_sparse_attn_algo", "dsa_forward", "dsa_forward_workspace_bytes",
     "dsa_window_attn", "dsa_device_status", "dsa_version", "LIB_PATH",
 ]
 
@@ -46,7 +46,7 @@ class ForwardArgs(ctypes.Structure):
         ("q_idx", ctypes.c_void_p), ("k_idx", ctypes.c_void_p), ("w", ctypes.c_void_p),
         ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
         ("gate", ctypes.c_void_p), ("out", ctypes.c_void_p), ("scores_out", ctypes.c_void_p),
-        ("idx_out", ctypes.c_void_p),
+        ("idx_out", ctypes.c_void_p), ("events", ctypes.c_void_p),
     ]
 
 
@@ -59,14 +59,15 @@ _Z = ctypes.c_size_t
 _SIGNATURES = {
     "dsa_index_scores": (_I, [_I, _P, _P, _P, _F, _I, _I, _I, _I, _I, _I, _P, _P]),
     "dsa_topk": (_I, [_P, _I, _I, _I, _I, _P, _P]),
-    "dsa_sparse_attn_workspace_bytes": (_Z, [_I, _I, _I, _I, _I, _I]),
-    "dsa_sparse_attn": (_I, [_I, _P, _P, _P, _P, _I, _P, _I, _F, _I, _I, _I, _I, _I, _I, _P, _P,
-                             _Z, _P]),
+    "dsa_sparse_attn_workspace_bytes": (_Z, [_I, _I, _I, _I, _I, _I, _I, _I, _I]),
+    "dsa_sparse_attn_algo": (_I, [_I, _I, _I, _I, _I, _I, _I, _I, _I]),
+    "dsa_sparse_attn": (_I, [_I, _P, _P, _P, _P, _I, _P, _I, _F, _I, _I, _I, _I, _I, _I, _I, _P,
+                             _P, _Z, _P]),
     "dsa_forward_workspace_bytes": (_Z, [ctypes.POINTER(ForwardArgs)]),
     "dsa_forward_min_workspace_bytes": (_Z, [ctypes.POINTER(ForwardArgs)]),
     "dsa_forward": (_I, [ctypes.POINTER(ForwardArgs), _P, _Z, _P]),
-    "dsa_window_attn": (_I, [_I, _P, _P, _P, _P, _I, _F, _I, _I, _I, _I, _I, _I, _I, _I, _P,
-                             _P]),
+    "dsa_window_attn": (_I, [_I, _P, _P, _P, _P, _I, _F, _I, _I, _I, _I, _I, _I, _I, _I, _I,
+                             _P, _P]),
     "dsa_status_string": (ctypes.c_char_p, [_I]),
     "dsa_last_error": (ctypes.c_char_p, []),
     "dsa_device_status": (_I, [_I]),
@@ -153,8 +154,17 @@ def dsa_topk(scores, K, idx=None, stream=None):
     return idx
 
 
-def dsa_sparse_attn_workspace_bytes(B, S, T, H, DV, K) -> int:
-    return int(lib().dsa_sparse_attn_workspace_bytes(B, S, T, H, DV, K))
+def dsa_sparse_attn_workspace_bytes(dtype, B, S, T, H, DQK, DV, K, algo="auto") -> int:
+    code = dtype if isinstance(dtype, int) else DTYPE[dtype]
+    return int(lib().dsa_sparse_attn_workspace_bytes(code, B, S, T, H, DQK, DV, K,
+                                                     ATTN_ALGO[algo]))
+
+
+def dsa_sparse_attn_algo(dtype, B, S, T, H, DQK, DV, K, algo="auto") -> str:
+    """The algorithm ("gather" / "masked_tile") a request resolves to for this shape."""
+    code = dtype if isinstance(dtype, int) else DTYPE[dtype]
+    r = int(lib().dsa_sparse_attn_algo(code, B, S, T, H, DQK, DV, K, ATTN_ALGO[algo]))
+    return {v: k for k, v in ATTN_ALGO.items()}[r]
 
 
 def _workspace(nbytes, device, ws):
@@ -165,9 +175,10 @@ def _workspace(nbytes, device, ws):
     return ws
 
 
-def dsa_sparse_attn(q, k, v, idx, gate=None, gate_mode=None, sm_scale=0.0, out=None, ws=None,
-                    stream=None):
-    """Attention of each query over its selected keys (idx), with the optional gate."""
+def dsa_sparse_attn(q, k, v, idx, gate=None, gate_mode=None, sm_scale=0.0, algo="auto",
+                    out=None, ws=None, stream=None):
+    """Attention of each query over its selected keys (idx), with the optional gate.
+    algo: "auto", "gather" or "masked_tile"."""
     _dev(q, k, v, idx, gate, out, ws)
     B, S, H, DQK = q.shape
     T, DV = k.shape[1], v.shape[-1]
@@ -175,11 +186,11 @@ def dsa_sparse_attn(q, k, v, idx, gate=None, gate_mode=None, sm_scale=0.0, out=N
     gm = GATE[gate_mode or ("sigmoid" if gate is not None else "off")]
     if out is None:
         out = torch.empty((B, S, H, DV), dtype=q.dtype, device=q.device)
-    nbytes = dsa_sparse_attn_workspace_bytes(B, S, T, H, DV, K)
+    nbytes = dsa_sparse_attn_workspace_bytes(_dtype_code(q), B, S, T, H, DQK, DV, K, algo)
     ws = _workspace(nbytes, q.device, ws)
     _check(lib().dsa_sparse_attn(_dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), K,
-                                 _ptr(gate), gm, float(sm_scale), B, S, T, H, DQK, DV, _ptr(out),
-                                 _ptr(ws), nbytes, _stream(stream)))
+                                 _ptr(gate), gm, float(sm_scale), B, S, T, H, DQK, DV,
+                                 ATTN_ALGO[algo], _ptr(out), _ptr(ws), nbytes, _stream(stream)))
     return out
 
 
@@ -208,7 +219,7 @@ def dsa_forward_workspace_bytes(args: ForwardArgs, minimum: bool = False) -> int
 
 def dsa_forward(q_idx, k_idx, w, index_scale, K, q, k, v, gate=None, gate_mode=None,
                 relu="none", sm_scale=0.0, attn_algo="auto", out=None, scores_out=None,
-                idx_out=None, ws=None, ws_bytes=None, stream=None):
+                idx_out=None, ws=None, ws_bytes=None, stream=None, events=None):
     """The whole DSA step (indexer -> top-k -> sparse attention -> gate).
 
     Returns (out, idx); idx is idx_out if given, else a view of the workspace copy.
@@ -224,14 +235,21 @@ def dsa_forward(q_idx, k_idx, w, index_scale, K, q, k, v, gate=None, gate_mode=N
         idx_out = torch.empty((B, S, k_eff), dtype=torch.int32, device=q.device)
     a = _forward_args(q_idx, k_idx, w, index_scale, K, q, k, v, gate, gate_mode, relu, sm_scale,
                       attn_algo, out, scores_out, idx_out)
+    ev_arr = None
+    if events is not None:  # 4 torch.cuda.Event, recorded by the library at stage boundaries
+        for e in events:
+            if e.cuda_event == 0:
+                e.record()  # torch creates the CUDA event on first use
+        ev_arr = (ctypes.c_void_p * 4)(*[e.cuda_event for e in events])
+        a.events = ctypes.cast(ev_arr, ctypes.c_void_p).value
     nbytes = dsa_forward_workspace_bytes(a) if ws_bytes is None else int(ws_bytes)
     ws = _workspace(nbytes, q.device, ws)
     _check(lib().dsa_forward(ctypes.byref(a), _ptr(ws), nbytes, _stream(stream)))
     return out, idx_out
 
 
-def dsa_window_attn(q, k, v, window, gate=None, gate_mode=None, sm_scale=0.0, out=None,
-                    stream=None):
+def dsa_window_attn(q, k, v, window, gate=None, gate_mode=None, sm_scale=0.0, algo="auto",
+                    out=None, stream=None):
     """Sliding-window causal attention with grouped KV heads (window keys incl. self)."""
     _dev(q, k, v, gate, out)
     B, S, H, DQK = q.shape
@@ -241,5 +259,5 @@ def dsa_window_attn(q, k, v, window, gate=None, gate_mode=None, sm_scale=0.0, ou
         out = torch.empty((B, S, H, DV), dtype=q.dtype, device=q.device)
     _check(lib().dsa_window_attn(_dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(gate), gm,
                                  float(sm_scale), int(window), B, S, T, H, HKV, DQK, DV,
-                                 _ptr(out), _stream(stream)))
+                                 ATTN_ALGO[algo], _ptr(out), _stream(stream)))
     return out

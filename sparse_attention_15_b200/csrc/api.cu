@@ -74,12 +74,12 @@ dsa_status check_index_args(dsa_dtype dtype, const void* q_idx, const void* k_id
 
 dsa_status run_index_scores(dsa_dtype dtype, const void* q_idx, const void* k_idx,
                             const float* w, float scale, dsa_relu_mode relu, int B, int S,
-                            int T, int HI, int DI, int q_off, float* scores,
+                            int T, int HI, int DI, int q_off, float* scores, int write_masked,
                             cudaStream_t st) {
   cudaError_t e;
   if (dsa::index_scores_tc_supported((int)dtype, HI, DI))
     e = dsa::launch_index_scores_tc(q_idx, k_idx, w, scale, (int)relu, B, S, T, HI, DI, q_off,
-                                    scores, 1, st);
+                                    scores, write_masked, st);
   else
     e = dsa::launch_index_scores_simt((int)dtype, q_idx, k_idx, w, scale, (int)relu, B, S, T,
                                       HI, DI, q_off, scores, st);
@@ -115,6 +115,40 @@ dsa_status check_attn_common(dsa_dtype dtype, const void* q, const void* k, cons
 
 float default_scale(float sm_scale, int DQK) {
   return sm_scale > 0.f ? sm_scale : 1.0f / sqrtf((float)DQK);
+}
+
+constexpr int kNone = -1, kGather = 1, kMasked = 2;
+
+size_t mask_bytes(int B, int S, int T) {
+  return (size_t)B * S * dsa::mask_stride_words(T) * sizeof(uint32_t);
+}
+
+// Cost model of the two attention algorithms.  Gather: every selected (query, key) pair
+// moves one K row and one V row (H * (DQK + DV) elements).  Masked tile: every 128-query
+// block runs dense tiles over all its causal 128-key blocks, 4 * H * (DQK + DV) flops per
+// executed pair.  Rates: a sustained gather bandwidth of 4 TB/s and half the bf16 tensor
+// peak; only their ratio matters.
+int choose_algo(dsa_attn_algo req, dsa_dtype dt, int B, int S, int T, int H, int DQK, int DV,
+                int K) {
+  const bool tc = dsa::masked_attn_supported((int)dt, DQK, DV);
+  if (req == DSA_ATTN_GATHER) return kGather;
+  if (req == DSA_ATTN_MASKED_TILE) return tc ? kMasked : kNone;
+  if (!tc) return kGather;
+  const long long q_off = (long long)T - S;
+  double dense = 0.0, sel = 0.0;
+  for (long long s0 = 0; s0 < S; s0 += 128) {
+    const long long s_last = (S - 1 < s0 + 127) ? S - 1 : s0 + 127;
+    const long long t_hi = (T - 1 < s_last + q_off) ? T - 1 : s_last + q_off;
+    dense += 128.0 * (double)((t_hi / 128 + 1) * 128);
+  }
+  for (long long s = 0; s < S; ++s) {
+    const long long n = (s + q_off + 1 < T) ? s + q_off + 1 : T;
+    sel += (double)(n < K ? n : K);
+  }
+  const double per_pair = (double)H * (DQK + DV);
+  const double t_dense = B * dense * per_pair * 2.0 / 0.8e15;
+  const double t_gather = B * sel * per_pair * 2.0 / 4.0e12;
+  return t_dense < t_gather ? kMasked : kGather;
 }
 
 }  // namespace
@@ -158,7 +192,7 @@ dsa_status dsa_index_scores(dsa_dtype dtype, const void* q_idx, const void* k_id
   dsa_status st = check_index_args(dtype, q_idx, k_idx, w, scale, relu, B, S, T, HI, DI, scores);
   if (st != DSA_OK) return st;
   return run_index_scores(dtype, q_idx, k_idx, w, scale, relu, B, S, T, HI, DI, T - S, scores,
-                          (cudaStream_t)stream);
+                          1, (cudaStream_t)stream);
 }
 
 dsa_status dsa_topk(const float* scores, int B, int S, int T, int K, int32_t* idx,
@@ -169,57 +203,86 @@ dsa_status dsa_topk(const float* scores, int B, int S, int T, int K, int32_t* id
   REQUIRE((size_t)B * S <= 0x7fffffffu, DSA_ERR_UNSUPPORTED, "too many rows");
   REQUIRE(aligned16(scores) && aligned16(idx), DSA_ERR_UNSUPPORTED,
           "pointers must be 16-byte aligned");
-  return cuda_status(dsa::launch_topk(scores, B, S, T, K, T - S, idx, nullptr,
+  return cuda_status(dsa::launch_topk(scores, B, S, T, K, T - S, idx, nullptr, 0,
                                       (cudaStream_t)stream),
                      "dsa_topk");
 }
 
-size_t dsa_sparse_attn_workspace_bytes(int B, int S, int T, int H, int DV, int K) {
-  (void)T;
-  if (B <= 0 || S <= 0 || H <= 0 || DV <= 0 || K <= 0) return 0;
-  return dsa::gather_attn_workspace_bytes(B, S, H, DV, K);
+size_t dsa_sparse_attn_workspace_bytes(dsa_dtype dtype, int B, int S, int T, int H, int DQK,
+                                       int DV, int K, dsa_attn_algo algo) {
+  if (B <= 0 || S <= 0 || T <= 0 || H <= 0 || DQK <= 0 || DV <= 0 || K <= 0) return 0;
+  const int alg = choose_algo(algo, dtype, B, S, T, H, DQK, DV, K);
+  if (alg == kMasked) return mask_bytes(B, S, T);
+  if (alg == kGather) return dsa::gather_attn_workspace_bytes(B, S, H, DV, K);
+  return 0;
+}
+
+dsa_attn_algo dsa_sparse_attn_algo(dsa_dtype dtype, int B, int S, int T, int H, int DQK, int DV,
+                                   int K, dsa_attn_algo algo) {
+  if (B <= 0 || S <= 0 || T <= 0 || H <= 0 || DQK <= 0 || DV <= 0 || K <= 0) return DSA_ATTN_AUTO;
+  const int alg = choose_algo(algo, dtype, B, S, T, H, DQK, DV, K);
+  return alg == kMasked ? DSA_ATTN_MASKED_TILE : (alg == kGather ? DSA_ATTN_GATHER : DSA_ATTN_AUTO);
 }
 
 dsa_status dsa_sparse_attn(dsa_dtype dtype, const void* q, const void* k, const void* v,
                            const int32_t* idx, int K, const void* gate,
                            dsa_gate_mode gate_mode, float sm_scale, int B, int S, int T,
-                           int H, int DQK, int DV, void* out, void* ws, size_t ws_bytes,
-                           dsa_stream_t stream) {
+                           int H, int DQK, int DV, dsa_attn_algo algo, void* out, void* ws,
+                           size_t ws_bytes, dsa_stream_t stream) {
   dsa_status st = check_attn_common(dtype, q, k, v, gate, gate_mode, sm_scale, B, S, T, H, H,
                                     DQK, DV, out);
   if (st != DSA_OK) return st;
   REQUIRE(idx != nullptr && K > 0, DSA_ERR_INVALID_ARG, "idx must be given with K > 0");
   REQUIRE(aligned16(idx), DSA_ERR_UNSUPPORTED, "idx must be 16-byte aligned");
-  const size_t need = dsa::gather_attn_workspace_bytes(B, S, H, DV, K);
+  REQUIRE(algo >= DSA_ATTN_AUTO && algo <= DSA_ATTN_MASKED_TILE, DSA_ERR_INVALID_ARG,
+          "unknown attention algorithm %d", (int)algo);
+  const int alg = choose_algo(algo, dtype, B, S, T, H, DQK, DV, K);
+  REQUIRE(alg != kNone, DSA_ERR_UNSUPPORTED,
+          "the masked-tile algorithm needs bf16, DQK in {128,192} and DV == 128");
+  const size_t need = dsa_sparse_attn_workspace_bytes(dtype, B, S, T, H, DQK, DV, K, algo);
   REQUIRE(ws_bytes >= need && (need == 0 || ws != nullptr), DSA_ERR_INVALID_ARG,
           "workspace too small: %zu bytes given, %zu needed", ws_bytes, need);
+  REQUIRE(ws == nullptr || aligned16(ws), DSA_ERR_UNSUPPORTED, "workspace must be 16-byte aligned");
   dsa::AttnProblem p{};
   p.dtype = (int)dtype; p.q = q; p.k = k; p.v = v; p.idx = idx; p.K = K; p.window = 0;
   p.gate = gate; p.gate_mode = (int)gate_mode; p.sm_scale = default_scale(sm_scale, DQK);
   p.B = B; p.S = S; p.T = T; p.H = H; p.HKV = H; p.DQK = DQK; p.DV = DV; p.q_off = T - S;
   p.out = out;
-  return cuda_status(dsa::launch_gather_attn(p, ws, ws_bytes, (cudaStream_t)stream),
-                     "dsa_sparse_attn");
+  cudaStream_t s = (cudaStream_t)stream;
+  if (alg == kMasked) {
+    uint32_t* mask = static_cast<uint32_t*>(ws);
+    const int stride = dsa::mask_stride_words(T);
+    st = cuda_status(dsa::launch_idx_to_mask(idx, B, S, T, K, T - S, mask, stride, s),
+                     "dsa_sparse_attn/mask");
+    if (st != DSA_OK) return st;
+    return cuda_status(dsa::launch_masked_attn(p, mask, stride, s), "dsa_sparse_attn");
+  }
+  return cuda_status(dsa::launch_gather_attn(p, ws, ws_bytes, s), "dsa_sparse_attn");
 }
 
 dsa_status dsa_window_attn(dsa_dtype dtype, const void* q, const void* k, const void* v,
                            const void* gate, dsa_gate_mode gate_mode, float sm_scale,
                            int window, int B, int S, int T, int H, int HKV, int DQK, int DV,
-                           void* out, dsa_stream_t stream) {
+                           dsa_attn_algo algo, void* out, dsa_stream_t stream) {
   dsa_status st = check_attn_common(dtype, q, k, v, gate, gate_mode, sm_scale, B, S, T, H, HKV,
                                     DQK, DV, out);
   if (st != DSA_OK) return st;
   REQUIRE(window > 0, DSA_ERR_INVALID_ARG, "window must be positive");
-  const size_t need = dsa::gather_attn_workspace_bytes(B, S, H, DV, window);
-  REQUIRE(need == 0, DSA_ERR_UNSUPPORTED,
-          "window attention with so few query rows needs split keys; not supported");
+  REQUIRE(algo >= DSA_ATTN_AUTO && algo <= DSA_ATTN_MASKED_TILE, DSA_ERR_INVALID_ARG,
+          "unknown attention algorithm %d", (int)algo);
+  const bool tc = dsa::masked_attn_supported((int)dtype, DQK, DV);
+  REQUIRE(algo != DSA_ATTN_MASKED_TILE || tc, DSA_ERR_UNSUPPORTED,
+          "the masked-tile algorithm needs bf16, DQK in {128,192} and DV == 128");
   dsa::AttnProblem p{};
   p.dtype = (int)dtype; p.q = q; p.k = k; p.v = v; p.idx = nullptr; p.K = 0; p.window = window;
   p.gate = gate; p.gate_mode = (int)gate_mode; p.sm_scale = default_scale(sm_scale, DQK);
   p.B = B; p.S = S; p.T = T; p.H = H; p.HKV = HKV; p.DQK = DQK; p.DV = DV; p.q_off = T - S;
   p.out = out;
-  return cuda_status(dsa::launch_gather_attn(p, nullptr, 0, (cudaStream_t)stream),
-                     "dsa_window_attn");
+  cudaStream_t s = (cudaStream_t)stream;
+  // the band is dense work for every query block with at least a few rows: tensor cores
+  if (algo == DSA_ATTN_MASKED_TILE || (algo == DSA_ATTN_AUTO && tc && S >= 64))
+    return cuda_status(dsa::launch_masked_attn(p, nullptr, 0, s), "dsa_window_attn");
+  return cuda_status(dsa::launch_gather_attn(p, nullptr, 0, s), "dsa_window_attn");
 }
 
 // ----------------------------------------------------------------------------- forward
@@ -241,18 +304,23 @@ static dsa_status check_forward(const dsa_forward_args* a) {
 }
 
 struct FwdLayout {
-  size_t idx_off, attn_off, scores_off, total_full, total_min;
-  int k_eff;
+  size_t idx_off, attn_off, mask_off, scores_off, total_full, total_min;
+  int k_eff, alg, mask_stride;
 };
 
 static FwdLayout forward_layout(const dsa_forward_args* a) {
   FwdLayout L{};
   L.k_eff = a->K < a->T ? a->K : a->T;
+  L.alg = choose_algo(a->attn_algo, a->dtype, a->B, a->S, a->T, a->H, a->DQK, a->DV, L.k_eff);
+  L.mask_stride = dsa::mask_stride_words(a->T);
   size_t off = 0;
   L.idx_off = off;
   if (!a->idx_out) off += align256((size_t)a->B * a->S * L.k_eff * sizeof(int32_t));
   L.attn_off = off;
-  off += align256(dsa::gather_attn_workspace_bytes(a->B, a->S, a->H, a->DV, L.k_eff));
+  if (L.alg == kGather)
+    off += align256(dsa::gather_attn_workspace_bytes(a->B, a->S, a->H, a->DV, L.k_eff));
+  L.mask_off = off;
+  if (L.alg == kMasked) off += align256(mask_bytes(a->B, a->S, a->T));
   L.scores_off = off;
   if (a->scores_out) {
     L.total_full = L.total_min = off;
@@ -278,25 +346,35 @@ dsa_status dsa_forward(const dsa_forward_args* a, void* ws, size_t ws_bytes,
   dsa_status st = check_forward(a);
   if (st != DSA_OK) return st;
   const FwdLayout L = forward_layout(a);
+  REQUIRE(L.alg != kNone, DSA_ERR_UNSUPPORTED,
+          "the masked-tile algorithm needs bf16, DQK in {128,192} and DV == 128");
   REQUIRE(ws_bytes >= L.total_min && (L.total_min == 0 || ws != nullptr), DSA_ERR_INVALID_ARG,
           "workspace too small: %zu bytes given, at least %zu needed", ws_bytes, L.total_min);
   REQUIRE(ws == nullptr || aligned16(ws), DSA_ERR_UNSUPPORTED, "workspace must be 16-byte aligned");
   cudaStream_t s = (cudaStream_t)stream;
   uint8_t* base = static_cast<uint8_t*>(ws);
   int32_t* idx = a->idx_out ? a->idx_out : reinterpret_cast<int32_t*>(base + L.idx_off);
-  void* attn_ws = base ? base + L.attn_off : nullptr;
-  const size_t attn_ws_bytes = L.scores_off - L.attn_off;
+  void* attn_ws = (base && L.alg == kGather) ? base + L.attn_off : nullptr;
+  const size_t attn_ws_bytes = L.mask_off - L.attn_off;
+  uint32_t* mask = L.alg == kMasked ? reinterpret_cast<uint32_t*>(base + L.mask_off) : nullptr;
   const int B = a->B, S = a->S, T = a->T, q_off = T - S;
   const size_t es = esize(a->dtype);
+  const int write_masked = a->scores_out != nullptr;  // -inf only matters to the caller
+  cudaEvent_t const* ev = reinterpret_cast<cudaEvent_t const*>(a->events);
+  auto mark = [&](int i) -> dsa_status {
+    return ev ? cuda_status(cudaEventRecord(ev[i], s), "dsa_forward/event") : DSA_OK;
+  };
+  if ((st = mark(0)) != DSA_OK) return st;
 
   if (a->scores_out || ws_bytes >= L.total_full) {
     float* scores = a->scores_out ? a->scores_out : reinterpret_cast<float*>(base + L.scores_off);
     st = run_index_scores(a->dtype, a->q_idx, a->k_idx, a->w, a->index_scale, a->relu, B, S, T,
-                          a->HI, a->DI, q_off, scores, s);
-    if (st != DSA_OK) return st;
-    st = cuda_status(dsa::launch_topk(scores, B, S, T, L.k_eff, q_off, idx, nullptr, s),
+                          a->HI, a->DI, q_off, scores, write_masked, s);
+    if (st != DSA_OK || (st = mark(1)) != DSA_OK) return st;
+    st = cuda_status(dsa::launch_topk(scores, B, S, T, L.k_eff, q_off, idx, mask, L.mask_stride,
+                                      s),
                      "dsa_forward/topk");
-    if (st != DSA_OK) return st;
+    if (st != DSA_OK || (st = mark(2)) != DSA_OK) return st;
   } else {
     // row blocks that fit the score buffer, one batch row at a time
     float* scores = reinterpret_cast<float*>(base + L.scores_off);
@@ -312,14 +390,19 @@ dsa_status dsa_forward(const dsa_forward_args* a, void* ws, size_t ws_bytes,
         const float* wb = a->w + ((size_t)b * S + s0) * a->HI;
         // this block's first query sits at key position q_off + s0
         st = run_index_scores(a->dtype, qi, ki, wb, a->index_scale, a->relu, 1, n, T, a->HI,
-                              a->DI, q_off + s0, scores, s);
+                              a->DI, q_off + s0, scores, 0, s);
         if (st != DSA_OK) return st;
+        const size_t row0 = (size_t)b * S + s0;
         st = cuda_status(dsa::launch_topk(scores, 1, n, T, L.k_eff, q_off + s0,
-                                          idx + ((size_t)b * S + s0) * L.k_eff, nullptr, s),
+                                          idx + row0 * L.k_eff,
+                                          mask ? mask + row0 * L.mask_stride : nullptr,
+                                          L.mask_stride, s),
                          "dsa_forward/topk");
         if (st != DSA_OK) return st;
       }
     }
+    // row blocks interleave the two stages: both boundary events mark their end
+    if ((st = mark(1)) != DSA_OK || (st = mark(2)) != DSA_OK) return st;
   }
   dsa::AttnProblem p{};
   p.dtype = (int)a->dtype; p.q = a->q; p.k = a->k; p.v = a->v; p.idx = idx; p.K = L.k_eff;
@@ -327,7 +410,12 @@ dsa_status dsa_forward(const dsa_forward_args* a, void* ws, size_t ws_bytes,
   p.sm_scale = default_scale(a->sm_scale, a->DQK);
   p.B = B; p.S = S; p.T = T; p.H = a->H; p.HKV = a->H; p.DQK = a->DQK; p.DV = a->DV;
   p.q_off = q_off; p.out = a->out;
-  return cuda_status(dsa::launch_gather_attn(p, attn_ws, attn_ws_bytes, s), "dsa_forward/attn");
+  if (L.alg == kMasked)
+    st = cuda_status(dsa::launch_masked_attn(p, mask, L.mask_stride, s), "dsa_forward/attn");
+  else
+    st = cuda_status(dsa::launch_gather_attn(p, attn_ws, attn_ws_bytes, s), "dsa_forward/attn");
+  if (st != DSA_OK) return st;
+  return mark(3);
 }
 
 }  // extern "C"

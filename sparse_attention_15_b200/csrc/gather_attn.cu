@@ -43,6 +43,7 @@ struct GatherArgs {
   int nsplit, keys_per_split;
   int nslots;
   uint32_t k_bytes, v_bytes, slot_bytes;
+  uint32_t key_list_bytes;  // shared-memory bytes reserved for the key list
 };
 
 // Key j of this CTA's range, or -1 if it must be skipped.
@@ -64,7 +65,8 @@ __global__ void __launch_bounds__(544, HPW <= 2 ? 2 : 1) gather_attn_kernel(cons
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
   uint64_t* empty = full + nslots;
   int* slot_key = reinterpret_cast<int*>(empty + nslots);
-  uint8_t* slots = smem + 1024;  // slot data starts 1 KB in (barriers and flags first)
+  int* keys = reinterpret_cast<int*>(smem + 1024);    // this CTA's key list
+  uint8_t* slots = smem + 1024 + a.key_list_bytes;   // K/V row slots
 
   const int nw = (blockDim.x >> 5) - 1;  // consumer warps; the last warp produces
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -92,12 +94,16 @@ __global__ void __launch_bounds__(544, HPW <= 2 ? 2 : 1) gather_attn_kernel(cons
 
   if (warp == nw) {
     // ------------------------------------------------------------- producer
+    // stage the key list once (coalesced), then issue the row copies back to back
+    for (int j = lane; j < nkeys; j += 32)
+      keys[j] = idx_row ? key_at(a, idx_row, j, spos) : key_at(a, nullptr, band0 + j, spos);
+    __syncwarp();
     if (lane == 0) {
       for (int j = 0; j < nkeys; ++j) {
         const int slot = j % nslots;
         const int round = j / nslots;
         if (round > 0 && !mbar_wait(&empty[slot], (round - 1) & 1)) break;
-        int t = idx_row ? key_at(a, idx_row, j, spos) : key_at(a, nullptr, band0 + j, spos);
+        const int t = keys[j];
         slot_key[slot] = t;
         if (t >= 0) {
           uint8_t* dst = slots + (size_t)slot * a.slot_bytes;
@@ -255,9 +261,9 @@ int heads_per_warp(int H) {
 }
 
 // Split policy: few query rows and long key lists -> spread the keys over CTAs.
-void split_policy(int rows, int nkeys, int* nsplit, int* kps) {
+void split_policy(int rows, int nkeys, int* nsplit, int* kps, bool allow_split = true) {
   const int target_ctas = 4 * 148;
-  if (rows >= target_ctas || nkeys <= 128) {
+  if (!allow_split || rows >= target_ctas || nkeys <= 128) {
     *nsplit = 1;
     *kps = nkeys;
     return;
@@ -325,7 +331,8 @@ cudaError_t launch_gather_attn(const AttnProblem& p, void* ws, size_t ws_bytes,
   const int rows = p.B * p.S;
   if (rows == 0) return cudaSuccess;
   const int nkeys = p.idx ? p.K : p.window;
-  split_policy(rows, nkeys, &a.nsplit, &a.keys_per_split);
+  split_policy(rows, nkeys, &a.nsplit, &a.keys_per_split, p.idx != nullptr);
+  a.key_list_bytes = ((uint32_t)a.keys_per_split * 4u + 127u) & ~127u;
   if (a.nsplit > 1) {
     const size_t need = (size_t)rows * a.nsplit * p.H * (p.DV + 2) * sizeof(float);
     if (ws == nullptr || ws_bytes < need) return cudaErrorInvalidValue;
@@ -339,7 +346,7 @@ cudaError_t launch_gather_attn(const AttnProblem& p, void* ws, size_t ws_bytes,
   int ns = (int)((96 * 1024) / a.slot_bytes);
   ns = ns < 2 ? 2 : (ns > 16 ? 16 : ns);
   a.nslots = ns;
-  const size_t smem = 1024 + (size_t)ns * a.slot_bytes;
+  const size_t smem = 1024 + a.key_list_bytes + (size_t)ns * a.slot_bytes;
   if (smem > 227 * 1024) return cudaErrorNotSupported;
   const int hpw = heads_per_warp(p.H);
   if (hpw == 0) return cudaErrorNotSupported;

@@ -1,15 +1,434 @@
-// Lightning-indexer scores on the 5th-generation tensor cores (placeholder: the
-// tcgen05 kernel is not built yet, so every shape goes to the CUDA-core kernel).
+// Lightning-indexer scores on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+// [AXK2] "SK Telecom 三大改进 / 1. Sparse Gated Attention（SGA）":
+//   index_score[b,s,t] = sum_h weight[b,s,h] * softmax_scale * (q[b,s,h,:] . k[b,t,:]),
+// causal mask imposed while scoring.  [PANGU] §3.5 Table 1: the S^2 * N_head^I * D^I term
+// that dominates prefill.
+//
+// The per-head dot products are one dense contraction: keys x (query, head) pairs over the
+// indexer dimension.  One MMA tile is
+//   D[128 keys, N = NQ*HI columns] = k_idx[t0:t0+128, :] . q_idx[(s0..s0+NQ) x heads, :]^T
+// (A = the key tile, B = the query block, both K-major bf16 in shared memory with the
+// 128-byte swizzle, fetched by TMA; D = float32 in tensor memory).  Because a TMEM lane is
+// a key, each epilogue thread owns one key and reduces over the heads of its row in
+// registers -- sum_h w[s,h] * D[t, (s,h)] -- with no cross-lane traffic, then applies the
+// scale, the optional ReLU and the causal mask and writes one float per query, coalesced
+// along t.
+//
+// Roles (persistent CTAs, one per SM; all waits bounded):
+//   warp 0       TMA producer: the query block of each work unit (double-buffered) and a
+//                ring of key tiles
+//   warp 1       MMA issuer (one thread): DI/16 tcgen05.mma per tile into one of two TMEM
+//                accumulators; tcgen05.commit frees the key stage and hands the
+//                accumulator to the epilogue
+//   warps 4..    epilogue: tcgen05.ld of the accumulator, weighted head sum, store
+// A work unit is (batch row, query block, a chunk of key tiles up to the causal limit);
+// units are dealt to CTAs round-robin.  Key tiles after the last causal tile of a query
+// block are not computed: a separate fill kernel writes their -inf when asked to.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
 
 namespace dsa {
 
-bool index_scores_tc_supported(int, int, int) { return false; }
+namespace {
 
-cudaError_t launch_index_scores_tc(const void*, const void*, const float*, float, int, int, int,
-                                   int, int, int, int, float*, int, cudaStream_t) {
-  return cudaErrorNotSupported;
+constexpr int kTileM = 128;   // keys per tile = TMEM lanes
+constexpr int kEpiWarp0 = 4;  // first epilogue warp (warp % 4 = its TMEM lane quadrant)
+
+struct TcArgs {
+  const float* w;
+  float* scores;
+  float scale;
+  int B, S, T, q_off;
+  int nqb;    // query blocks per batch row
+  int chunk;  // key tiles per work unit
+};
+
+template <int HI_, int DI_, int NQ_, int NE_, int NA_>
+struct TcCfg {
+  static constexpr int HI = HI_, DI = DI_, NQ = NQ_, NE = NE_, NA = NA_;
+  static constexpr int N = NQ * HI;               // MMA N: (query, head) columns
+  static constexpr int KH = DI / 64;              // 64-element (128-byte) K slices
+  static constexpr int A_SLICE = kTileM * 128;    // bytes of one K slice of a key tile
+  static constexpr int A_BYTES = KH * A_SLICE;
+  static constexpr int B_SLICE = N * 128;
+  static constexpr int B_BYTES = KH * B_SLICE;
+  static constexpr int ACC_COLS = N;              // one accumulator
+  static constexpr int TMEM_COLS = 2 * N <= 32 ? 32 : 2 * N <= 64 ? 64 : 2 * N <= 128 ? 128
+                                   : 2 * N <= 256 ? 256 : 512;
+  static constexpr int EPI_GROUPS = NE / 4;       // epilogue warps per TMEM lane quadrant
+  static constexpr int COLS_PER_WARP = N / EPI_GROUPS;
+  static constexpr int THREADS = 32 * (kEpiWarp0 + NE);
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM = NA * A_BYTES + 2 * B_BYTES + BAR_BYTES + 1024;
+  static_assert(N % 16 == 0 && N >= 16 && N <= 256, "UMMA N");
+  static_assert(HI <= 32 && 32 % HI == 0, "heads per 32-column chunk");
+  static_assert(COLS_PER_WARP % 32 == 0, "epilogue chunking");
+  static_assert(DI % 64 == 0, "DI must be a multiple of 64");
+};
+
+// Iterates this CTA's work units in the global order (b, query block, key chunk).
+struct UnitIter {
+  int b = 0, qb = 0, c = -1, nch = 0;
+  long long u = -1;
+  int k0 = 0, k1 = 0;
+  __device__ __forceinline__ int ntiles(const TcArgs& a, int q, int NQ) const {
+    int s_last = min(a.S - 1, q * NQ + NQ - 1);
+    int t_last = min(a.T - 1, s_last + a.q_off);
+    return t_last / kTileM + 1;
+  }
+  // Advance to the next unit owned by CTA `cta` out of `ncta`; false when done.
+  __device__ __forceinline__ bool next(const TcArgs& a, int NQ, int cta, int ncta) {
+    for (;;) {
+      ++c;
+      if (c >= nch) {
+        if (u >= 0 || nch > 0) {
+          if (++qb >= a.nqb) { qb = 0; if (++b >= a.B) return false; }
+        }
+        c = 0;
+        nch = (ntiles(a, qb, NQ) + a.chunk - 1) / a.chunk;
+      }
+      ++u;
+      if (u % ncta == cta) {
+        const int nt = ntiles(a, qb, NQ);
+        k0 = c * a.chunk;
+        k1 = min(nt, k0 + a.chunk);
+        return true;
+      }
+    }
+  }
+};
+
+// A wait used on the way out: ignores a recorded timeout (copies and MMAs already in
+// flight must land before the CTA exits) but is bounded itself.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity))
+    if (clock64() - t0 > kWaitCycles) {
+      flag_status(kStatusTimeout);
+      return;
+    }
+}
+
+template <class C, int RELU>
+__global__ void __launch_bounds__(C::THREADS, 1)
+    index_scores_tc_kernel(const __grid_constant__ CUtensorMap kmap,
+                           const __grid_constant__ CUtensorMap qmap, const TcArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* As = smem;                               // NA key tiles
+  uint8_t* Bs = smem + C::NA * C::A_BYTES;          // 2 query blocks
+  uint64_t* bars = reinterpret_cast<uint64_t*>(Bs + 2 * C::B_BYTES);
+  uint64_t* a_full = bars;                          // [NA]
+  uint64_t* a_empty = a_full + C::NA;               // [NA]
+  uint64_t* b_full = a_empty + C::NA;               // [2]
+  uint64_t* b_empty = b_full + 2;                   // [2]
+  uint64_t* acc_full = b_empty + 2;                 // [2]
+  uint64_t* acc_empty = acc_full + 2;               // [2]
+  uint64_t* mma_done = acc_empty + 2;               // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int cta = blockIdx.x, ncta = gridDim.x;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::NA; ++i) { mbar_init(&a_full[i], 1); mbar_init(&a_empty[i], 1); }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&b_full[i], 1); mbar_init(&b_empty[i], 1);
+      mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], C::NE);
+    }
+    mbar_init(mma_done, 1);
+    fence_mbar_init();
+    prefetch_tmap(&kmap);
+    prefetch_tmap(&qmap);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      UnitIter it;
+      uint32_t ai = 0, bi = 0;
+      bool ok = true;
+      while (ok && it.next(a, C::NQ, cta, ncta)) {
+        const int bb = bi & 1;
+        if (bi >= 2 && !mbar_wait(&b_empty[bb], ((bi >> 1) - 1) & 1)) { ok = false; break; }
+        mbar_arrive_expect_tx(&b_full[bb], C::B_BYTES);
+        const int qrow = (it.b * a.S + it.qb * C::NQ) * C::HI;
+#pragma unroll
+        for (int kh = 0; kh < C::KH; ++kh)
+          tma_load_2d(Bs + bb * C::B_BYTES + kh * C::B_SLICE, &qmap, kh * 64, qrow, &b_full[bb]);
+        ++bi;
+        for (int kt = it.k0; kt < it.k1; ++kt) {
+          const int st = ai % C::NA;
+          if (ai >= (uint32_t)C::NA && !mbar_wait(&a_empty[st], ((ai / C::NA) - 1) & 1)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&a_full[st], C::A_BYTES);
+          const int krow = it.b * a.T + kt * kTileM;
+#pragma unroll
+          for (int kh = 0; kh < C::KH; ++kh)
+            tma_load_2d(As + st * C::A_BYTES + kh * C::A_SLICE, &kmap, kh * 64, krow,
+                        &a_full[st]);
+          ++ai;
+        }
+      }
+      // on the way out, let every copy this thread issued land
+      for (uint32_t j = (ai > (uint32_t)C::NA ? ai - C::NA : 0); j < ai; ++j)
+        drain_wait(&a_full[j % C::NA], (j / C::NA) & 1);
+      for (uint32_t j = (bi > 2 ? bi - 2 : 0); j < bi; ++j) drain_wait(&b_full[j & 1], (j >> 1) & 1);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kTileM, C::N);
+      UnitIter it;
+      uint32_t ai = 0, bi = 0, ci = 0;
+      bool ok = true;
+      while (ok && it.next(a, C::NQ, cta, ncta)) {
+        const int bb = bi & 1;
+        if (!mbar_wait(&b_full[bb], (bi >> 1) & 1)) { ok = false; break; }
+        const uint32_t b_base = smem_u32(Bs + bb * C::B_BYTES);
+        for (int kt = it.k0; kt < it.k1; ++kt) {
+          const int st = ai % C::NA;
+          if (!mbar_wait(&a_full[st], (ai / C::NA) & 1)) { ok = false; break; }
+          const int ab = ci & 1;
+          if (ci >= 2 && !mbar_wait(&acc_empty[ab], ((ci >> 1) - 1) & 1)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(As + st * C::A_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < C::DI / 16; ++kk) {
+            const uint32_t off = (kk & 3) * 32;  // 16 bf16 = 32 B along the swizzled row
+            const uint64_t adesc = sw128_kmajor_desc(a_base + (kk >> 2) * C::A_SLICE + off);
+            const uint64_t bdesc = sw128_kmajor_desc(b_base + (kk >> 2) * C::B_SLICE + off);
+            umma_f16_ss(tmem + ab * C::ACC_COLS, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&a_empty[st]);
+          umma_commit(&acc_full[ab]);
+          ++ai;
+          ++ci;
+        }
+        if (!ok) break;
+        umma_commit(&b_empty[bb]);
+        ++bi;
+      }
+      umma_commit(mma_done);
+      drain_wait(mma_done, 0);
+    }
+  } else if (warp >= kEpiWarp0) {
+    // ------------------------------------------------------------------ epilogue
+    const int ew = warp - kEpiWarp0;
+    const int quad = warp & 3;
+    const int group = ew >> 2;
+    const int col0 = group * C::COLS_PER_WARP;
+    const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
+    const float ninf = __int_as_float(0xff800000);
+    UnitIter it;
+    uint32_t ci = 0;
+    bool ok = true;
+    while (ok && it.next(a, C::NQ, cta, ncta)) {
+      const int s_base = it.qb * C::NQ;
+      for (int kt = it.k0; kt < it.k1; ++kt) {
+        const int ab = ci & 1;
+        if (!warp_wait(&acc_full[ab], (ci >> 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        const int t = kt * kTileM + quad * 32 + lane;
+        constexpr int NCH = C::COLS_PER_WARP / 32;
+        // double-buffered TMEM reads: chunk cc+1 is in flight while chunk cc is reduced
+        uint32_t rb[2][32];
+        tmem_ld32(t_lane + ab * C::ACC_COLS + col0, rb[0]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int cc = 0; cc < NCH; ++cc) {
+          if (cc + 1 < NCH) {
+            tmem_ld32(t_lane + ab * C::ACC_COLS + col0 + (cc + 1) * 32, rb[(cc + 1) & 1]);
+          } else {
+            // every column of this accumulator has been read: hand it back to the MMA
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[ab]);
+          }
+          const uint32_t* r = rb[cc & 1];
+#pragma unroll
+          for (int qi = 0; qi < 32 / C::HI; ++qi) {
+            const int j = (col0 + cc * 32) / C::HI + qi;  // query within the block
+            const int s = s_base + j;
+            if (s < a.S) {  // ragged tail of the last block (warp-uniform)
+              const float* wr = a.w + ((size_t)it.b * a.S + s) * C::HI;
+              float acc4[4] = {0.f, 0.f, 0.f, 0.f};  // four independent FMA chains
+#pragma unroll
+              for (int h = 0; h < C::HI; h += 4) {
+                const float4 w4 = __ldg(reinterpret_cast<const float4*>(wr + h));
+                float d0 = __uint_as_float(r[qi * C::HI + h + 0]);
+                float d1 = __uint_as_float(r[qi * C::HI + h + 1]);
+                float d2 = __uint_as_float(r[qi * C::HI + h + 2]);
+                float d3 = __uint_as_float(r[qi * C::HI + h + 3]);
+                if (RELU == 2) {
+                  d0 = fmaxf(d0, 0.f); d1 = fmaxf(d1, 0.f); d2 = fmaxf(d2, 0.f); d3 = fmaxf(d3, 0.f);
+                }
+                acc4[0] = fmaf(w4.x, d0, acc4[0]);
+                acc4[1] = fmaf(w4.y, d1, acc4[1]);
+                acc4[2] = fmaf(w4.z, d2, acc4[2]);
+                acc4[3] = fmaf(w4.w, d3, acc4[3]);
+              }
+              float v = ((acc4[0] + acc4[1]) + (acc4[2] + acc4[3])) * a.scale;
+              if (RELU == 1) v = fmaxf(v, 0.f);
+              if (t < a.T)
+                a.scores[((size_t)it.b * a.S + s) * a.T + t] = (t <= s + a.q_off) ? v : ninf;
+            }
+          }
+          if (cc + 1 < NCH) tmem_wait_ld();
+        }
+        ++ci;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// -inf for the keys after the last causal tile of each query block (row-wise fill).
+__global__ void fill_masked_kernel(float* __restrict__ scores, int S, int T, int q_off, int NQ) {
+  const size_t row = blockIdx.x;
+  const int s = (int)(row % (size_t)S);
+  const int qb = s / NQ;
+  const int s_last = min(S - 1, qb * NQ + NQ - 1);
+  const int t_last = min(T - 1, s_last + q_off);
+  const int start = (t_last / kTileM + 1) * kTileM;
+  float* r = scores + row * (size_t)T;
+  const float ninf = __int_as_float(0xff800000);
+  for (int t = start + threadIdx.x; t < T; t += blockDim.x) r[t] = ninf;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor map over a [rows, cols] row-major matrix, box [box_cols, box_rows],
+// 128-byte swizzle (box_cols * 2 must be 128).
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+template <class C>
+cudaError_t launch_cfg(const void* q_idx, const void* k_idx, const float* w, float scale,
+                       int relu, int B, int S, int T, int q_off, float* scores,
+                       int write_masked, cudaStream_t st) {
+  CUtensorMap kmap, qmap;
+  if (!make_map(&kmap, k_idx, (uint64_t)B * T, C::DI, kTileM)) return cudaErrorInvalidValue;
+  if (!make_map(&qmap, q_idx, (uint64_t)B * S * C::HI, C::DI, C::N)) return cudaErrorInvalidValue;
+  TcArgs a{};
+  a.w = w; a.scores = scores; a.scale = scale; a.B = B; a.S = S; a.T = T; a.q_off = q_off;
+  a.nqb = (S + C::NQ - 1) / C::NQ;
+  // total causal tiles -> chunk size giving each CTA several units
+  long long tiles = 0;
+  for (int qb = 0; qb < a.nqb; ++qb) {
+    int s_last = S - 1 < qb * C::NQ + C::NQ - 1 ? S - 1 : qb * C::NQ + C::NQ - 1;
+    int t_last = T - 1 < s_last + q_off ? T - 1 : s_last + q_off;
+    tiles += t_last / kTileM + 1;
+  }
+  tiles *= B;
+  const int nsm = sm_count();
+  long long ch = tiles / ((long long)nsm * 8);
+  a.chunk = (int)(ch < 2 ? 2 : (ch > 32 ? 32 : ch));
+  long long units = 0;
+  for (int qb = 0; qb < a.nqb; ++qb) {
+    int s_last = S - 1 < qb * C::NQ + C::NQ - 1 ? S - 1 : qb * C::NQ + C::NQ - 1;
+    int t_last = T - 1 < s_last + q_off ? T - 1 : s_last + q_off;
+    units += (t_last / kTileM + 1 + a.chunk - 1) / a.chunk;
+  }
+  units *= B;
+  const int grid = (int)(units < nsm ? units : nsm);
+  auto kern = relu == 1 ? index_scores_tc_kernel<C, 1>
+                        : (relu == 2 ? index_scores_tc_kernel<C, 2> : index_scores_tc_kernel<C, 0>);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, C::THREADS, C::SMEM, st>>>(kmap, qmap, a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || !write_masked) return e;
+  fill_masked_kernel<<<(unsigned)((size_t)B * S), 256, 0, st>>>(scores, S, T, q_off, C::NQ);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool index_scores_tc_supported(int dtype, int HI, int DI) {
+  return dtype == 1 && (HI == 16 || HI == 32) && (DI == 64 || DI == 128);
+}
+
+cudaError_t launch_index_scores_tc(const void* q_idx, const void* k_idx, const float* w,
+                                   float scale, int relu, int B, int S, int T, int HI, int DI,
+                                   int q_off, float* scores, int write_masked,
+                                   cudaStream_t st) {
+  if (!index_scores_tc_supported(1, HI, DI)) return cudaErrorNotSupported;
+  if (S == 1) {  // decode: one query per batch row, N = HI, deep key pipeline
+    if (HI == 32 && DI == 128)
+      return launch_cfg<TcCfg<32, 128, 1, 4, 6>>(q_idx, k_idx, w, scale, relu, B, S, T, q_off,
+                                                 scores, write_masked, st);
+    if (HI == 32 && DI == 64)
+      return launch_cfg<TcCfg<32, 64, 1, 4, 8>>(q_idx, k_idx, w, scale, relu, B, S, T, q_off,
+                                                scores, write_masked, st);
+    if (HI == 16 && DI == 128)
+      return launch_cfg<TcCfg<16, 128, 2, 4, 6>>(q_idx, k_idx, w, scale, relu, B, S, T, q_off,
+                                                 scores, write_masked, st);
+    return launch_cfg<TcCfg<16, 64, 2, 4, 8>>(q_idx, k_idx, w, scale, relu, B, S, T, q_off,
+                                              scores, write_masked, st);
+  }
+  if (HI == 32 && DI == 128)
+    return launch_cfg<TcCfg<32, 128, 8, 8, 3>>(q_idx, k_idx, w, scale, relu, B, S, T, q_off,
+                                               scores, write_masked, st);
+  if (HI == 32 && DI == 64)
+    return launch_cfg<TcCfg<32, 64, 8, 8, 4>>(q_idx, k_idx, w, scale, relu, B, S, T, q_off,
+                                              scores, write_masked, st);
+  if (HI == 16 && DI == 128)
+    return launch_cfg<TcCfg<16, 128, 16, 8, 3>>(q_idx, k_idx, w, scale, relu, B, S, T, q_off,
+                                                scores, write_masked, st);
+  return launch_cfg<TcCfg<16, 64, 16, 8, 4>>(q_idx, k_idx, w, scale, relu, B, S, T, q_off,
+                                             scores, write_masked, st);
 }
 
 }  // namespace dsa

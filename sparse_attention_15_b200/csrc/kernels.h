@@ -23,9 +23,15 @@ cudaError_t launch_index_scores_tc(const void* q_idx, const void* k_idx, const f
                                    cudaStream_t st);
 
 // Per-row top-k (radix select + ordered compaction).  `mask` (optional) receives the
-// selection bitmask [rows, ceil(T/32)] words.
+// selection bitmask, one bit per key, rows of `mask_stride` 32-bit words
+// (mask_stride >= ceil(T/32); words past the row's keys are zero).
 cudaError_t launch_topk(const float* scores, int B, int S, int T, int K, int q_off,
-                        int32_t* idx, uint32_t* mask, cudaStream_t st);
+                        int32_t* idx, uint32_t* mask, int mask_stride, cudaStream_t st);
+// Selection bitmask from index lists (valid, causal entries only).
+cudaError_t launch_idx_to_mask(const int32_t* idx, int B, int S, int T, int K, int q_off,
+                               uint32_t* mask, int mask_stride, cudaStream_t st);
+// Words per bitmask row used by the masked-tile attention (ceil(T/128) * 4).
+inline int mask_stride_words(int T) { return ((T + 127) / 128) * 4; }
 
 // Gather attention (idx lists) and band attention (sliding window, GQA) share one kernel.
 struct AttnProblem {
@@ -44,6 +50,12 @@ struct AttnProblem {
 };
 size_t gather_attn_workspace_bytes(int B, int S, int H, int DV, int K);
 cudaError_t launch_gather_attn(const AttnProblem& p, void* ws, size_t ws_bytes,
+                               cudaStream_t st);
+
+// Dense tensor-core attention tiles under the selection bitmask (or, with idx == NULL and
+// mask == NULL, under the sliding-window band).  bf16, DQK in {128, 192}, DV == 128.
+bool masked_attn_supported(int dtype, int DQK, int DV);
+cudaError_t launch_masked_attn(const AttnProblem& p, const uint32_t* mask, int mask_stride,
                                cudaStream_t st);
 
 }  // namespace dsa

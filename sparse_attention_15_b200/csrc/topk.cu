@@ -65,7 +65,8 @@ template <int NT>
 __global__ void __launch_bounds__(NT) topk_rows_kernel(const float* __restrict__ scores, int S,
                                                        int Tn, int K, int q_off,
                                                        int32_t* __restrict__ idx,
-                                                       uint32_t* __restrict__ mask) {
+                                                       uint32_t* __restrict__ mask,
+                                                       int mask_stride) {
   __shared__ uint32_t hist[kBins];
   __shared__ int warp_buf[32];
   __shared__ int scan_total;
@@ -79,7 +80,7 @@ __global__ void __launch_bounds__(NT) topk_rows_kernel(const float* __restrict__
   const float* sc = scores + row * (size_t)Tn;
   int32_t* out = idx + row * (size_t)K;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int mwords = (Tn + 31) >> 5;
+  const int mwords = mask_stride;  // words per mask row (>= ceil(Tn/32))
   uint32_t* mrow = mask ? mask + row * (size_t)mwords : nullptr;
 
   if (n <= K) {  // every valid key is kept
@@ -188,18 +189,46 @@ __global__ void __launch_bounds__(NT) topk_rows_kernel(const float* __restrict__
   }
 }
 
+// Selection bitmask from index lists: bit t of row (b,s) is set when t appears in the row,
+// 0 <= t < T and t <= s + q_off (the causal mask).  One CTA per row.
+__global__ void idx_to_mask_kernel(const int32_t* __restrict__ idx, int S, int Tn, int K,
+                                   int q_off, uint32_t* __restrict__ mask, int stride) {
+  const size_t row = blockIdx.x;
+  const int spos = (int)(row % (size_t)S) + q_off;
+  uint32_t* m = mask + row * (size_t)stride;
+  for (int w = threadIdx.x; w < stride; w += blockDim.x) m[w] = 0u;
+  __syncthreads();
+  const int32_t* ir = idx + row * (size_t)K;
+  for (int i = threadIdx.x; i < K; i += blockDim.x) {
+    const int t = ir[i];
+    if (t >= 0 && t < Tn && t <= spos) atomicOr(&m[t >> 5], 1u << (t & 31));
+  }
+}
+
 }  // namespace
 
-cudaError_t launch_topk(const float* scores, int B, int S, int T, int K, int q_off,
-                        int32_t* idx, uint32_t* mask, cudaStream_t st) {
+cudaError_t launch_idx_to_mask(const int32_t* idx, int B, int S, int T, int K, int q_off,
+                               uint32_t* mask, int mask_stride, cudaStream_t st) {
   const size_t rows = (size_t)B * S;
   if (rows == 0) return cudaSuccess;
+  idx_to_mask_kernel<<<(unsigned)rows, 256, 0, st>>>(idx, S, T, K, q_off, mask, mask_stride);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_topk(const float* scores, int B, int S, int T, int K, int q_off,
+                        int32_t* idx, uint32_t* mask, int mask_stride, cudaStream_t st) {
+  const size_t rows = (size_t)B * S;
+  if (rows == 0) return cudaSuccess;
+  if (mask && mask_stride < (T + 31) / 32) return cudaErrorInvalidValue;
   if (T >= 8192)
-    topk_rows_kernel<1024><<<(unsigned)rows, 1024, 0, st>>>(scores, S, T, K, q_off, idx, mask);
+    topk_rows_kernel<1024><<<(unsigned)rows, 1024, 0, st>>>(scores, S, T, K, q_off, idx, mask,
+                                                            mask_stride);
   else if (T >= 2048)
-    topk_rows_kernel<512><<<(unsigned)rows, 512, 0, st>>>(scores, S, T, K, q_off, idx, mask);
+    topk_rows_kernel<512><<<(unsigned)rows, 512, 0, st>>>(scores, S, T, K, q_off, idx, mask,
+                                                          mask_stride);
   else
-    topk_rows_kernel<256><<<(unsigned)rows, 256, 0, st>>>(scores, S, T, K, q_off, idx, mask);
+    topk_rows_kernel<256><<<(unsigned)rows, 256, 0, st>>>(scores, S, T, K, q_off, idx, mask,
+                                                          mask_stride);
   return cudaGetLastError();
 }
 

@@ -109,10 +109,10 @@ def check_topk_properties(scores, idx, K, q_off, chunk=1024):
             d = ix[:, 1:] - ix[:, :-1]
             assert bool(((d > 0) | ~live[:, 1:]).all()), "indices not strictly ascending"
             sel = torch.zeros((s1 - s0, T), dtype=torch.bool, device=dev)
-            sel.scatter_(1, ix.clamp(min=0), live)
+            r_of = torch.arange(s1 - s0, device=dev)[:, None].expand_as(ix)
+            sel[r_of[live], ix[live]] = True
             valid = t_all[None] < n[:, None]
             v = sc + 0.0  # -0.0 -> +0.0
-            big = torch.finfo(torch.float32).max
             tau = torch.where(sel, v, torch.full_like(v, float("inf"))).min(dim=1).values
             drop = valid & ~sel
             mx_drop = torch.where(drop, v, torch.full_like(v, -float("inf"))).max(dim=1).values
@@ -122,4 +122,3 @@ def check_topk_properties(scores, idx, K, q_off, chunk=1024):
             last_kept_tie = torch.where(sel & tie, t_all[None], -1).max(dim=1).values
             first_drop_tie = torch.where(drop & tie, t_all[None], T).min(dim=1).values
             assert bool((last_kept_tie < first_drop_tie).all()), "tie-break violated"
-            del big

@@ -80,7 +80,7 @@ def _attn(L, **kw):
     a.update(kw)
     return L.dsa_sparse_attn(a["dtype"], a["q"], a["k"], a["v"], a["idx"], a["K"], a["gate"],
                              a["gm"], a["sm"], a["B"], a["S"], a["T"], a["H"], a["DQK"], a["DV"],
-                             a["out"], a["ws"], a["wsb"], None)
+                             a.get("algo", 0), a["out"], a["ws"], a["wsb"], None)
 
 
 def test_sparse_attn_rejects_bad_arguments(lib):
@@ -93,20 +93,28 @@ def test_sparse_attn_rejects_bad_arguments(lib):
     assert _attn(L, DQK=300) == 2
     assert _attn(L, v=FAKE_MIS) == 2
     assert _attn(L, sm=float("inf")) == 1
+    assert _attn(L, algo=7) == 1
+    assert _attn(L, dtype=0, DQK=64, DV=64, algo=2) == 2  # masked tile is bf16 only
     # decode-shaped work needs a split-key workspace; too small a workspace is rejected
-    need = L.dsa_sparse_attn_workspace_bytes(2, 1, 131072, 32, 128, 2048)
+    need = L.dsa_sparse_attn_workspace_bytes(1, 2, 1, 131072, 32, 192, 128, 2048, 0)
     assert need > 0
     assert _attn(L, B=2, S=1, T=131072, H=32, DQK=192, DV=128, K=2048, ws=FAKE,
                  wsb=need - 1) == 1
+    # the cost model: long prefill -> masked tile (bitmask workspace), decode -> gather
+    pre = L.dsa_sparse_attn_workspace_bytes(1, 1, 4096, 4096, 20, 128, 128, 512, 0)
+    assert pre == 4096 * (4096 // 128) * 4 * 4
+    assert L.dsa_sparse_attn_workspace_bytes(1, 1, 4096, 4096, 20, 128, 128, 512, 1) == 0
 
 
 def test_window_attn_rejects_bad_arguments(lib):
     L = lib.lib()
     f = L.dsa_window_attn
-    assert f(1, FAKE, FAKE, FAKE, None, 0, 0.0, 512, 1, 1024, 1024, 32, 6, 192, 128, FAKE,
+    assert f(1, FAKE, FAKE, FAKE, None, 0, 0.0, 512, 1, 1024, 1024, 32, 6, 192, 128, 0, FAKE,
              None) == 1  # 32 heads over 6 KV heads
-    assert f(1, FAKE, FAKE, FAKE, None, 0, 0.0, 0, 1, 1024, 1024, 32, 8, 192, 128, FAKE,
+    assert f(1, FAKE, FAKE, FAKE, None, 0, 0.0, 0, 1, 1024, 1024, 32, 8, 192, 128, 0, FAKE,
              None) == 1  # empty window
+    assert f(1, FAKE, FAKE, FAKE, None, 0, 0.0, 512, 1, 1024, 1024, 32, 8, 96, 128, 2, FAKE,
+             None) == 2  # masked tile needs DQK 128 or 192
 
 
 def test_forward_workspace_and_validation(lib):
