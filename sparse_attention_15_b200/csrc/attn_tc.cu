@@ -15,8 +15,9 @@
 // 128-byte swizzle, via 3-D tensor maps over (dim, head, token)), V block [128 x Dv]
 // (MN-major operand of the second product).  Tensor memory: S0, S1 (128 columns each,
 // double-buffered so S_{j+1} = Q K_{j+1}^T overlaps the softmax of block j), O (Dv columns);
-// P (bf16, two per 32-bit column) overwrites the first 64 columns of its S buffer and feeds
-// O += P V as the tensor-memory A operand.  The running max is only raised (and O, l
+// P is split into bf16 P_hi + P_lo (two per 32-bit column, 64 columns each) that overwrite
+// their S buffer and feed O += P_hi V + P_lo V as tensor-memory A operands -- the low part
+// keeps the float32 probabilities' precision that a single bf16 P would lose.  The running max is only raised (and O, l
 // rescaled) when a row's block max exceeds it by more than 2^8, so exp2 arguments stay
 // <= 8 and rescales are rare.
 //
@@ -87,6 +88,13 @@ __device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t start, uint32_t 
   d |= (uint64_t)1 << 46;
   d |= (uint64_t)2 << 61;
   return d;
+}
+
+// 2^x on the special-function unit (flush-to-zero; exp2(-inf) = +0).
+__device__ __forceinline__ float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y,
@@ -259,9 +267,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
           for (int kk = 0; kk < kBlk / 16; ++kk) {
             // 16 keys: 8 packed P columns; 16 V rows = 2 swizzle atoms of 8 rows
-            umma_f16_ts(tmem + C::O_COL, p_tmem + kk * 8,
-                        sw128_mnmajor_desc(v_base + kk * 2048, C::SLICE, 1024), idesc_pv,
+            const uint64_t vdesc = sw128_mnmajor_desc(v_base + kk * 2048, C::SLICE, 1024);
+            umma_f16_ts(tmem + C::O_COL, p_tmem + kk * 8, vdesc, idesc_pv,
                         (j > 0 || kk > 0) ? 1u : 0u);
+            umma_f16_ts(tmem + C::O_COL, p_tmem + 64 + kk * 8, vdesc, idesc_pv, 1u);
           }
           umma_commit(&kv_empty[gg & 1]);
           umma_commit(&s_empty[gg & 1]);
@@ -312,19 +321,25 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                                                  : (((1u << (a1 - a0 + 1)) - 1u) << a0));
           }
         }
+        // raw S row: all four TMEM reads in flight, one wait
+        uint32_t r[kBlk];
+        tmem_ld32(t_lane + (gg & 1) * C::S_COLS + 0, *reinterpret_cast<uint32_t(*)[32]>(r + 0));
+        tmem_ld32(t_lane + (gg & 1) * C::S_COLS + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
+        tmem_ld32(t_lane + (gg & 1) * C::S_COLS + 64, *reinterpret_cast<uint32_t(*)[32]>(r + 64));
+        tmem_ld32(t_lane + (gg & 1) * C::S_COLS + 96, *reinterpret_cast<uint32_t(*)[32]>(r + 96));
+        tmem_wait_ld();
+        // masked raw scores (unselected -> -inf) and their max; the scale is positive, so
+        // max(scale * s) = scale * max(s) and the scale folds into the exp argument below
         float x[kBlk];
+        float mraw = ninf;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tmem_ld32(t_lane + (gg & 1) * C::S_COLS + c * 32, r);
-          tmem_wait_ld();
+        for (int c = 0; c < 4; ++c)
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            x[c * 32 + e] = ((bits[c] >> e) & 1u) ? __uint_as_float(r[e]) * a.qk_scale : ninf;
-        }
-        float mb = ninf;
-#pragma unroll
-        for (int e = 0; e < kBlk; ++e) mb = fmaxf(mb, x[e]);
+          for (int e = 0; e < 32; ++e) {
+            x[c * 32 + e] = (bits[c] & (1u << e)) ? __uint_as_float(r[c * 32 + e]) : ninf;
+            mraw = fmaxf(mraw, x[c * 32 + e]);
+          }
+        const float mb = mraw * a.qk_scale;
         const bool need = mb > m_used + kRescaleLog2;
         if (__any_sync(0xffffffffu, need)) {
           const float m_new = need ? mb : m_used;
@@ -351,24 +366,32 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             m_used = m_new;
           }
         }
+        // P = P_hi + P_lo, both bf16 (P_hi = bf16(p), P_lo = bf16(p - P_hi)): the second
+        // product recovers the bits bf16 drops, so O carries ~2^-17 relative error in P
+        // instead of 2^-9.  P_hi fills columns [0,64) of the S buffer, P_lo [64,128).
         float rs = 0.f;
-        uint32_t pk[kBlk / 2];
+        // exp2(scale * s - m); -inf (unselected) gives exactly 0.  With no selected key yet
+        // (m_used = -inf) every x is -inf as well; subtracting 0 keeps the result 0.
+        const float msub = m_used == ninf ? 0.f : m_used;
 #pragma unroll
-        for (int e = 0; e < kBlk; e += 2) {
-          const float p0 = x[e] == ninf ? 0.f : exp2f(x[e] - m_used);
-          const float p1 = x[e + 1] == ninf ? 0.f : exp2f(x[e + 1] - m_used);
-          rs += p0 + p1;
-          __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-          pk[e >> 1] = *reinterpret_cast<uint32_t*>(&h2);
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t ph[32], pl[32];
+#pragma unroll
+          for (int e2 = 0; e2 < 32; ++e2) {
+            const int e = hf * 64 + 2 * e2;
+            const float p0 = ex2_ftz(fmaf(x[e], a.qk_scale, -msub));
+            const float p1 = ex2_ftz(fmaf(x[e + 1], a.qk_scale, -msub));
+            rs += p0 + p1;
+            const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+            const float2 hf2 = __bfloat1622float2(h2);
+            const __nv_bfloat162 l2 = __floats2bfloat162_rn(p0 - hf2.x, p1 - hf2.y);
+            ph[e2] = *reinterpret_cast<const uint32_t*>(&h2);
+            pl[e2] = *reinterpret_cast<const uint32_t*>(&l2);
+          }
+          tmem_st32(t_lane + (gg & 1) * C::S_COLS + hf * 32, ph);
+          tmem_st32(t_lane + (gg & 1) * C::S_COLS + 64 + hf * 32, pl);
         }
         l += rs;
-        {
-          uint32_t r0[32], r1[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) { r0[e] = pk[e]; r1[e] = pk[32 + e]; }
-          tmem_st32(t_lane + (gg & 1) * C::S_COLS, r0);
-          tmem_st32(t_lane + (gg & 1) * C::S_COLS + 32, r1);
-        }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();

@@ -44,8 +44,9 @@ struct TcArgs {
   float* scores;
   float scale;
   int B, S, T, q_off;
-  int nqb;    // query blocks per batch row
-  int chunk;  // key tiles per work unit
+  int nqb;         // query blocks per batch row
+  int chunk;       // key tiles per work unit
+  int max_chunks;  // units per query block slot (chunks of the longest block)
 };
 
 template <int HI_, int DI_, int NQ_, int NE_, int NA_>
@@ -71,35 +72,34 @@ struct TcCfg {
   static_assert(DI % 64 == 0, "DI must be a multiple of 64");
 };
 
-// Iterates this CTA's work units in the global order (b, query block, key chunk).
+// This CTA's work units.  Unit u = (b * nqb + qb) * max_chunks + c covers key tiles
+// [c*chunk, min(ntiles(qb), (c+1)*chunk)); units with c >= chunks(qb) are empty and
+// skipped.  CTA i takes u = i, i + G, i + 2G, ... (decoded directly, no scan).
 struct UnitIter {
-  int b = 0, qb = 0, c = -1, nch = 0;
-  long long u = -1;
-  int k0 = 0, k1 = 0;
-  __device__ __forceinline__ int ntiles(const TcArgs& a, int q, int NQ) const {
-    int s_last = min(a.S - 1, q * NQ + NQ - 1);
-    int t_last = min(a.T - 1, s_last + a.q_off);
+  long long u;
+  int b = 0, qb = 0, k0 = 0, k1 = 0;
+  __device__ __forceinline__ explicit UnitIter(int cta) : u((long long)cta) {}
+  __device__ __forceinline__ static int ntiles(const TcArgs& a, int q, int NQ) {
+    const int s_last = min(a.S - 1, q * NQ + NQ - 1);
+    const int t_last = min(a.T - 1, s_last + a.q_off);
     return t_last / kTileM + 1;
   }
-  // Advance to the next unit owned by CTA `cta` out of `ncta`; false when done.
-  __device__ __forceinline__ bool next(const TcArgs& a, int NQ, int cta, int ncta) {
-    for (;;) {
-      ++c;
-      if (c >= nch) {
-        if (u >= 0 || nch > 0) {
-          if (++qb >= a.nqb) { qb = 0; if (++b >= a.B) return false; }
-        }
-        c = 0;
-        nch = (ntiles(a, qb, NQ) + a.chunk - 1) / a.chunk;
-      }
-      ++u;
-      if (u % ncta == cta) {
-        const int nt = ntiles(a, qb, NQ);
-        k0 = c * a.chunk;
-        k1 = min(nt, k0 + a.chunk);
-        return true;
-      }
+  // Next non-empty unit owned by this CTA; false when done.
+  __device__ __forceinline__ bool next(const TcArgs& a, int NQ, int ncta) {
+    const long long total = (long long)a.B * a.nqb * a.max_chunks;
+    for (; u < total; u += ncta) {
+      const int c = (int)(u % a.max_chunks);
+      const long long bq = u / a.max_chunks;
+      qb = (int)(bq % a.nqb);
+      b = (int)(bq / a.nqb);
+      const int nt = ntiles(a, qb, NQ);
+      k0 = c * a.chunk;
+      if (k0 >= nt) continue;
+      k1 = min(nt, k0 + a.chunk);
+      u += ncta;
+      return true;
     }
+    return false;
   }
 };
 
@@ -134,7 +134,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int cta = blockIdx.x, ncta = gridDim.x;
+  const int cta = blockIdx.x, ncta = gridDim.x;  // persistent CTAs
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NA; ++i) { mbar_init(&a_full[i], 1); mbar_init(&a_empty[i], 1); }
@@ -159,10 +159,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      UnitIter it;
+      UnitIter it(cta);
       uint32_t ai = 0, bi = 0;
       bool ok = true;
-      while (ok && it.next(a, C::NQ, cta, ncta)) {
+      while (ok && it.next(a, C::NQ, ncta)) {
         const int bb = bi & 1;
         if (bi >= 2 && !mbar_wait(&b_empty[bb], ((bi >> 1) - 1) & 1)) { ok = false; break; }
         mbar_arrive_expect_tx(&b_full[bb], C::B_BYTES);
@@ -195,10 +195,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(kTileM, C::N);
-      UnitIter it;
+      UnitIter it(cta);
       uint32_t ai = 0, bi = 0, ci = 0;
       bool ok = true;
-      while (ok && it.next(a, C::NQ, cta, ncta)) {
+      while (ok && it.next(a, C::NQ, ncta)) {
         const int bb = bi & 1;
         if (!mbar_wait(&b_full[bb], (bi >> 1) & 1)) { ok = false; break; }
         const uint32_t b_base = smem_u32(Bs + bb * C::B_BYTES);
@@ -236,10 +236,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const int col0 = group * C::COLS_PER_WARP;
     const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
     const float ninf = __int_as_float(0xff800000);
-    UnitIter it;
+    UnitIter it(cta);
     uint32_t ci = 0;
     bool ok = true;
-    while (ok && it.next(a, C::NQ, cta, ncta)) {
+    while (ok && it.next(a, C::NQ, ncta)) {
       const int s_base = it.qb * C::NQ;
       for (int kt = it.k0; kt < it.k1; ++kt) {
         const int ab = ci & 1;
@@ -366,19 +366,23 @@ cudaError_t launch_cfg(const void* q_idx, const void* k_idx, const float* w, flo
   a.nqb = (S + C::NQ - 1) / C::NQ;
   // total causal tiles -> chunk size giving each CTA several units
   long long tiles = 0;
+  int max_nt = 1;
   for (int qb = 0; qb < a.nqb; ++qb) {
-    int s_last = S - 1 < qb * C::NQ + C::NQ - 1 ? S - 1 : qb * C::NQ + C::NQ - 1;
-    int t_last = T - 1 < s_last + q_off ? T - 1 : s_last + q_off;
-    tiles += t_last / kTileM + 1;
+    const int s_last = S - 1 < qb * C::NQ + C::NQ - 1 ? S - 1 : qb * C::NQ + C::NQ - 1;
+    const int t_last = T - 1 < s_last + q_off ? T - 1 : s_last + q_off;
+    const int nt = t_last / kTileM + 1;
+    tiles += nt;
+    if (nt > max_nt) max_nt = nt;
   }
   tiles *= B;
   const int nsm = sm_count();
-  long long ch = tiles / ((long long)nsm * 8);
-  a.chunk = (int)(ch < 2 ? 2 : (ch > 32 ? 32 : ch));
+  long long ch = tiles / ((long long)nsm * 4);
+  a.chunk = (int)(ch < 4 ? 4 : (ch > 32 ? 32 : ch));
+  a.max_chunks = (max_nt + a.chunk - 1) / a.chunk;
   long long units = 0;
   for (int qb = 0; qb < a.nqb; ++qb) {
-    int s_last = S - 1 < qb * C::NQ + C::NQ - 1 ? S - 1 : qb * C::NQ + C::NQ - 1;
-    int t_last = T - 1 < s_last + q_off ? T - 1 : s_last + q_off;
+    const int s_last = S - 1 < qb * C::NQ + C::NQ - 1 ? S - 1 : qb * C::NQ + C::NQ - 1;
+    const int t_last = T - 1 < s_last + q_off ? T - 1 : s_last + q_off;
     units += (t_last / kTileM + 1 + a.chunk - 1) / a.chunk;
   }
   units *= B;

@@ -189,6 +189,260 @@ __global__ void __launch_bounds__(NT) topk_rows_kernel(const float* __restrict__
   }
 }
 
+// ------------------------------------------------------------------------------------
+// Two-read top-k with shared-memory bitmaps (rows up to kMaxBitmapKeys keys).
+//
+// Read 1 (HBM, float4 loads, 16 keys per thread in flight): histogram of the top 12 bits of
+// the order key -> bucket b1 holding the K-th key, `need` = keys of b1 still to take.
+// Read 2 (L2): keys in buckets above b1 go to the SELECTED bitmap, keys of b1 to the
+// CANDIDATE bitmap (bits assembled across lanes with shuffles, no atomics).  The low 20
+// bits are then resolved by two 10-bit histogram passes over the candidates only (a few
+// hundred scattered L2 reads), giving the exact threshold key tau.  Candidates above tau
+// join SELECTED; candidates equal to tau are ranked by index with a prefix scan of their
+// bitmap and the first `need` join SELECTED.  An ordered scan of SELECTED writes the indices
+// (ascending) and the bitmap itself is the selection mask row.
+// ------------------------------------------------------------------------------------
+constexpr int kMaxBitmapKeys = 1 << 20;
+constexpr int kBins1 = 4096;  // top 12 bits
+constexpr int kBins2 = 1024;  // 10-bit refinement digits
+
+template <int NT>
+__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t digit, bool valid) {
+  const uint32_t d = valid ? digit : 0xffffffffu;
+  const uint32_t peers = __match_any_sync(0xffffffffu, d);
+  if (valid && (threadIdx.x & 31) == (uint32_t)(__ffs(peers) - 1))
+    atomicAdd(&hist[d], (uint32_t)__popc(peers));
+}
+
+// Bucket holding the need-th largest key: writes (bin, count above it) to out[0..1].
+template <int NT>
+__device__ __forceinline__ void find_bucket(const uint32_t* hist, int nbins, int need,
+                                            int* warp_buf, int* scan_total, int* out) {
+  const int per = nbins / NT;
+  const int hi_bin = nbins - threadIdx.x * per;
+  int local = 0;
+  for (int q = 1; q <= per; ++q) local += (int)hist[hi_bin - q];
+  int above = block_excl_scan(local, warp_buf, scan_total);
+  for (int q = 1; q <= per; ++q) {
+    const int c = (int)hist[hi_bin - q];
+    if (above < need && above + c >= need) {
+      out[0] = hi_bin - q;
+      out[1] = above;
+    }
+    above += c;
+  }
+}
+
+template <int NT>
+__global__ void __launch_bounds__(NT) topk_bitmap_kernel(const float* __restrict__ scores, int S,
+                                                         int Tn, int K, int q_off,
+                                                         int32_t* __restrict__ idx,
+                                                         uint32_t* __restrict__ mask,
+                                                         int mask_stride) {
+  extern __shared__ uint32_t dsm[];
+  const int W = (Tn + 31) >> 5;              // bitmap words per row
+  uint32_t* hist = dsm;                      // [kBins1]
+  uint32_t* selb = hist + kBins1;            // [W]
+  uint32_t* candb = selb + W;                // [W]
+  __shared__ int warp_buf[32];
+  __shared__ int scan_total;
+  __shared__ int pick[2];
+
+  const size_t row = blockIdx.x;
+  const int s = (int)(row % (size_t)S);
+  const int n = min(Tn, s + q_off + 1);
+  const float* sc = scores + row * (size_t)Tn;
+  int32_t* out = idx + row * (size_t)K;
+  const int tid = threadIdx.x, lane = tid & 31;
+  uint32_t* mrow = mask ? mask + row * (size_t)mask_stride : nullptr;
+  const int nw = (n + 31) >> 5;
+
+  if (n <= K) {  // every valid key is kept
+    for (int i = tid; i < K; i += NT) out[i] = i < n ? i : -1;
+    if (mrow)
+      for (int wd = tid; wd < mask_stride; wd += NT) {
+        const int lo = wd * 32;
+        mrow[wd] = lo + 32 <= n ? 0xffffffffu : (lo >= n ? 0u : ((1u << (n - lo)) - 1u));
+      }
+    return;
+  }
+
+  for (int i = tid; i < kBins1; i += NT) hist[i] = 0u;
+  for (int i = tid; i < W; i += NT) { selb[i] = 0u; candb[i] = 0u; }
+  __syncthreads();
+
+  // ---------------- read 1: 12-bit histogram, 16 keys per thread in flight
+  const bool vec = ((Tn & 3) == 0);
+  constexpr int U = 4;
+  for (int base = 0; base < n; base += NT * 4 * U) {
+    float v[U][4];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = base + (u * NT + tid) * 4;
+      if (vec && i + 3 < n) {
+        const float4 f = __ldg(reinterpret_cast<const float4*>(sc + i));
+        v[u][0] = f.x; v[u][1] = f.y; v[u][2] = f.z; v[u][3] = f.w;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[u][e] = (i + e < n) ? __ldg(sc + i + e) : 0.f;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = base + (u * NT + tid) * 4;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) hist_add<NT>(hist, order_key(v[u][e]) >> 20, i + e < n);
+    }
+  }
+  __syncthreads();
+  find_bucket<NT>(hist, kBins1, K, warp_buf, &scan_total, pick);
+  __syncthreads();
+  const uint32_t b1 = (uint32_t)pick[0];
+  int need = K - pick[1];
+  const int cnt1 = (int)hist[b1];
+
+  // ---------------- read 2: SELECTED (above b1) and CANDIDATE (== b1) bitmaps
+  for (int base = 0; base < n; base += NT * 4) {
+    const int i = base + tid * 4;
+    float v[4];
+    if (vec && i + 3 < n) {
+      const float4 f = __ldg(reinterpret_cast<const float4*>(sc + i));
+      v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) v[e] = (i + e < n) ? __ldg(sc + i + e) : 0.f;
+    }
+    uint32_t gt = 0u, eq = 0u;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (i + e < n) {
+        const uint32_t d = order_key(v[e]) >> 20;
+        gt |= (d > b1 ? 1u : 0u) << e;
+        eq |= (d == b1 ? 1u : 0u) << e;
+      }
+    }
+    // lanes 8m..8m+7 cover one 32-key word: OR their nibbles together
+    const int sh = 4 * (lane & 7);
+    uint32_t wg = gt << sh, we = eq << sh;
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) {
+      wg |= __shfl_xor_sync(0xffffffffu, wg, o);
+      we |= __shfl_xor_sync(0xffffffffu, we, o);
+    }
+    const int wd = (i >> 5);
+    if ((lane & 7) == 0 && i < n) {
+      selb[wd] = wg;
+      candb[wd] = we;
+    }
+  }
+  __syncthreads();
+
+  // ---------------- refine the low 20 bits over the candidates only
+  uint32_t prefix = b1;
+  int pbits = 12;
+  if (cnt1 != need) {
+    for (int pass = 0; pass < 2; ++pass) {
+      const int shift = 20 - 10 * (pass + 1);
+      for (int i = tid; i < kBins2; i += NT) hist[i] = 0u;
+      __syncthreads();
+      for (int w0 = 0; w0 < nw; w0 += NT) {
+        const int wd = w0 + tid;
+        uint32_t bits = wd < nw ? candb[wd] : 0u;
+        // every lane walks its word; the histogram add is warp-aggregated per step
+        bool more = __any_sync(0xffffffffu, bits != 0u);
+        while (more) {
+          const bool has = bits != 0u;
+          uint32_t digit = 0u;
+          bool valid = false;
+          if (has) {
+            const int j = __ffs(bits) - 1;
+            bits &= bits - 1u;
+            const uint32_t key = order_key(__ldg(sc + wd * 32 + j));
+            if ((key >> (32 - pbits)) == prefix) {
+              digit = (key >> shift) & (kBins2 - 1);
+              valid = true;
+            }
+          }
+          hist_add<NT>(hist, digit, valid);
+          more = __any_sync(0xffffffffu, bits != 0u);
+        }
+      }
+      __syncthreads();
+      find_bucket<NT>(hist, kBins2, need, warp_buf, &scan_total, pick);
+      __syncthreads();
+      const uint32_t bsel = (uint32_t)pick[0];
+      need -= pick[1];
+      prefix = (prefix << 10) | bsel;
+      pbits += 10;
+      const bool done = (int)hist[bsel] == need;
+      __syncthreads();
+      if (done) break;
+    }
+  }
+
+  // ---------------- candidates: above the threshold -> SELECTED, at it -> ties (in candb)
+  const int fshift = 32 - pbits;
+  for (int wd = tid; wd < nw; wd += NT) {
+    uint32_t bits = candb[wd], sel = 0u, tie = 0u;
+    while (bits) {
+      const int j = __ffs(bits) - 1;
+      bits &= bits - 1u;
+      const uint32_t hi = order_key(__ldg(sc + wd * 32 + j)) >> fshift;
+      if (hi > prefix) sel |= 1u << j;
+      else if (hi == prefix) tie |= 1u << j;
+    }
+    selb[wd] |= sel;
+    candb[wd] = tie;
+  }
+  __syncthreads();
+  // ties ranked by index: the first `need` are kept.  Thread t owns words [t*per, t*per+per).
+  const int per = (nw + NT - 1) / NT;
+  {
+    int local = 0;
+    for (int q = 0; q < per; ++q) {
+      const int wd = tid * per + q;
+      if (wd < nw) local += __popc(candb[wd]);
+    }
+    int rank = block_excl_scan(local, warp_buf, &scan_total);
+    for (int q = 0; q < per && rank < need; ++q) {
+      const int wd = tid * per + q;
+      if (wd >= nw) break;
+      uint32_t bits = candb[wd];
+      while (bits && rank < need) {
+        const int j = __ffs(bits) - 1;
+        bits &= bits - 1u;
+        selb[wd] |= 1u << j;
+        ++rank;
+      }
+    }
+  }
+  __syncthreads();
+  // ---------------- ordered output: prefix popcounts of SELECTED
+  {
+    int local = 0;
+    for (int q = 0; q < per; ++q) {
+      const int wd = tid * per + q;
+      if (wd < nw) local += __popc(selb[wd]);
+    }
+    int pos = block_excl_scan(local, warp_buf, &scan_total);
+    for (int q = 0; q < per; ++q) {
+      const int wd = tid * per + q;
+      if (wd >= nw) break;
+      uint32_t bits = selb[wd];
+      while (bits) {
+        const int j = __ffs(bits) - 1;
+        bits &= bits - 1u;
+        if (pos < K) out[pos] = wd * 32 + j;
+        ++pos;
+      }
+    }
+    const int total = scan_total;
+    for (int i = total + tid; i < K; i += NT) out[i] = -1;  // only if something went wrong
+  }
+  if (mrow)
+    for (int wd = tid; wd < mask_stride; wd += NT) mrow[wd] = wd < nw ? selb[wd] : 0u;
+}
+
 // Selection bitmask from index lists: bit t of row (b,s) is set when t appears in the row,
 // 0 <= t < T and t <= s + q_off (the causal mask).  One CTA per row.
 __global__ void idx_to_mask_kernel(const int32_t* __restrict__ idx, int S, int Tn, int K,
@@ -220,6 +474,25 @@ cudaError_t launch_topk(const float* scores, int B, int S, int T, int K, int q_o
   const size_t rows = (size_t)B * S;
   if (rows == 0) return cudaSuccess;
   if (mask && mask_stride < (T + 31) / 32) return cudaErrorInvalidValue;
+  if (T <= kMaxBitmapKeys) {
+    const int W = (T + 31) / 32;
+    const size_t smem = (size_t)(kBins1 + 2 * W) * sizeof(uint32_t);
+    {  // dynamic + static shared memory may pass the 48 KB default
+      cudaError_t e = cudaFuncSetAttribute(topk_bitmap_kernel<1024>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      e = cudaFuncSetAttribute(topk_bitmap_kernel<512>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+    }
+    if (T >= 8192)
+      topk_bitmap_kernel<1024><<<(unsigned)rows, 1024, smem, st>>>(scores, S, T, K, q_off, idx,
+                                                                    mask, mask_stride);
+    else
+      topk_bitmap_kernel<512><<<(unsigned)rows, 512, smem, st>>>(scores, S, T, K, q_off, idx,
+                                                                  mask, mask_stride);
+    return cudaGetLastError();
+  }
   if (T >= 8192)
     topk_rows_kernel<1024><<<(unsigned)rows, 1024, 0, st>>>(scores, S, T, K, q_off, idx, mask,
                                                             mask_stride);
