@@ -215,6 +215,38 @@ dsa_status dsa_window_attn(dsa_dtype dtype, const void* q, const void* k, const 
                            dsa_attn_algo algo, void* out, dsa_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
+ * dsa_sparse_attn without any workspace: for callers that cannot allocate device memory.
+ * The pages have no counterpart of this call; it exists for embedding.
+ *
+ * Some callers get only their input and output buffers and may not create device memory
+ * themselves -- a plugin inside an inference runtime whose memory planner owns all device
+ * memory, or a decode loop with a fixed budget that must not pay for the implicit
+ * synchronisation and fragmentation of a new allocation.  This call computes exactly what
+ * dsa_sparse_attn computes with DSA_ATTN_GATHER (same kernels, same split of the keys), but
+ * keeps the split-key partial results in a fixed array of
+ * dsa_sparse_attn_noalloc_max_scratch_bytes() bytes (16 MiB) inside the library's own
+ * device memory, which every GPU that loads the library holds until the process exits.
+ *
+ *   - Nothing is allocated or freed by any call (no cudaMalloc, no allocating library call).
+ *   - The first call on a device, made with that device current, looks up the array's device
+ *     address (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - Shapes whose partial results need more than the fixed size are rejected with
+ *     DSA_ERR_UNSUPPORTED before anything is launched (the message states both sizes); use
+ *     dsa_sparse_attn with a workspace for those.  The decode shape of 64 rows x 32 heads x
+ *     128-wide values with 2048 selected keys fits.
+ *   - Every call on a device shares the one array, which keeps the previous call's
+ *     contents; nothing in it needs to start at zero (each call writes every partial it
+ *     reads).  Calls that can overlap on the GPU (different streams, or different host
+ *     threads) race on the array and must be serialised by the caller.
+ *   Arguments and results are those of dsa_sparse_attn (without algo and workspace).
+ * --------------------------------------------------------------------------------- */
+size_t dsa_sparse_attn_noalloc_max_scratch_bytes(void);
+dsa_status dsa_sparse_attn_noalloc(dsa_dtype dtype, const void* q, const void* k, const void* v,
+                                   const int32_t* idx, int K, const void* gate,
+                                   dsa_gate_mode gate_mode, float sm_scale, int B, int S, int T,
+                                   int H, int DQK, int DV, void* out, dsa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
  * Status and introspection.
  * --------------------------------------------------------------------------------- */
 const char* dsa_status_string(dsa_status s);

@@ -16,7 +16,8 @@ import torch
 __all__ = [
     "DSAError", "lib", "dsa_index_scores", "dsa_topk", "dsa_sparse_attn",
     "dsa_sparse_attn_workspace_bytes", "dsa_sparse_attn_algo", "dsa_forward", "dsa_forward_workspace_bytes",
-    "dsa_window_attn", "dsa_device_status", "dsa_version", "LIB_PATH",
+    "dsa_window_attn", "dsa_sparse_attn_noalloc", "dsa_device_status", "dsa_version",
+    "LIB_PATH",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdsa.so")
@@ -68,6 +69,9 @@ _SIGNATURES = {
     "dsa_forward": (_I, [ctypes.POINTER(ForwardArgs), _P, _Z, _P]),
     "dsa_window_attn": (_I, [_I, _P, _P, _P, _P, _I, _F, _I, _I, _I, _I, _I, _I, _I, _I, _I,
                              _P, _P]),
+    "dsa_sparse_attn_noalloc_max_scratch_bytes": (_Z, []),
+    "dsa_sparse_attn_noalloc": (_I, [_I, _P, _P, _P, _P, _I, _P, _I, _F, _I, _I, _I, _I, _I, _I,
+                                     _P, _P]),
     "dsa_status_string": (ctypes.c_char_p, [_I]),
     "dsa_last_error": (ctypes.c_char_p, []),
     "dsa_device_status": (_I, [_I]),
@@ -191,6 +195,24 @@ def dsa_sparse_attn(q, k, v, idx, gate=None, gate_mode=None, sm_scale=0.0, algo=
     _check(lib().dsa_sparse_attn(_dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), K,
                                  _ptr(gate), gm, float(sm_scale), B, S, T, H, DQK, DV,
                                  ATTN_ALGO[algo], _ptr(out), _ptr(ws), nbytes, _stream(stream)))
+    return out
+
+
+def dsa_sparse_attn_noalloc(q, k, v, idx, gate=None, gate_mode=None, sm_scale=0.0, out=None,
+                            stream=None):
+    """dsa_sparse_attn (gather form) with no workspace: the split-key partials live in the
+    library's fixed device array (see include/dsa.h).  Allocates nothing but ``out`` when
+    the caller gives none."""
+    _dev(q, k, v, idx, gate, out)
+    B, S, H, DQK = q.shape
+    T, DV = k.shape[1], v.shape[-1]
+    K = idx.shape[-1]
+    gm = GATE[gate_mode or ("sigmoid" if gate is not None else "off")]
+    if out is None:
+        out = torch.empty((B, S, H, DV), dtype=q.dtype, device=q.device)
+    _check(lib().dsa_sparse_attn_noalloc(_dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), K,
+                                         _ptr(gate), gm, float(sm_scale), B, S, T, H, DQK, DV,
+                                         _ptr(out), _stream(stream)))
     return out
 
 

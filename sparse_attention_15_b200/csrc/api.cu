@@ -153,6 +153,11 @@ int choose_algo(dsa_attn_algo req, dsa_dtype dt, int B, int S, int T, int H, int
 
 }  // namespace
 
+namespace dsa {
+// Records the thread-local text dsa_last_error() returns (for entry points in other files).
+void set_last_error(const char* msg) { g_last_error = msg ? msg : ""; }
+}  // namespace dsa
+
 extern "C" {
 
 const char* dsa_status_string(dsa_status s) {

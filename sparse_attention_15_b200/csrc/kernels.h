@@ -8,6 +8,9 @@
 
 namespace dsa {
 
+// Sets the thread-local text returned by dsa_last_error().
+void set_last_error(const char* msg);
+
 // Indexer scores, SIMT (float32 FMA) kernel: any dtype, DI <= 128.
 cudaError_t launch_index_scores_simt(int dtype, const void* q_idx, const void* k_idx,
                                      const float* w, float scale, int relu, int B, int S,
