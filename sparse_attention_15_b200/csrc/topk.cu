@@ -475,21 +475,29 @@ cudaError_t launch_topk(const float* scores, int B, int S, int T, int K, int q_o
   if (rows == 0) return cudaSuccess;
   if (mask && mask_stride < (T + 31) / 32) return cudaErrorInvalidValue;
   if (T <= kMaxBitmapKeys) {
+    // one CTA per row; small CTAs so that several rows are in flight per SM (each row is a
+    // chain of dependent reads and block-wide scans)
     const int W = (T + 31) / 32;
     const size_t smem = (size_t)(kBins1 + 2 * W) * sizeof(uint32_t);
     {  // dynamic + static shared memory may pass the 48 KB default
-      cudaError_t e = cudaFuncSetAttribute(topk_bitmap_kernel<1024>,
+      cudaError_t e = cudaFuncSetAttribute(topk_bitmap_kernel<512>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;
-      e = cudaFuncSetAttribute(topk_bitmap_kernel<512>,
+      e = cudaFuncSetAttribute(topk_bitmap_kernel<256>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      e = cudaFuncSetAttribute(topk_bitmap_kernel<1024>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;
     }
-    if (T >= 8192)
+    if (rows < 296 && T > 8192)  // few long rows (decode): the widest CTA per row
       topk_bitmap_kernel<1024><<<(unsigned)rows, 1024, smem, st>>>(scores, S, T, K, q_off, idx,
                                                                     mask, mask_stride);
-    else
+    else if (T > 8192)
       topk_bitmap_kernel<512><<<(unsigned)rows, 512, smem, st>>>(scores, S, T, K, q_off, idx,
+                                                                  mask, mask_stride);
+    else
+      topk_bitmap_kernel<256><<<(unsigned)rows, 256, smem, st>>>(scores, S, T, K, q_off, idx,
                                                                   mask, mask_stride);
     return cudaGetLastError();
   }
