@@ -139,15 +139,37 @@ class ClockSampler:
                 "power_w_max": max(num(f[3]) for f in win)}
 
 
+def reduce_max(value, dist=None, device="cpu"):
+    """Max of a float over all ranks (identity without a process group)."""
+    if dist is None:
+        return float(value)
+    t = torch.tensor([float(value)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(units_per_rank, world, step_ms_max):
+    """Whole-job throughput: every rank's units over the slowest rank's step time."""
+    return units_per_rank * world / (step_ms_max / 1e3)
+
+
 # ----------------------------------------------------------------------------- workloads
 class Workload:
     """Device buffers and the library calls of one step of config `name`."""
 
-    def __init__(self, name, device, seed_offset=0):
+    def __init__(self, name, device, seed_offset=0, S=None, T=None):
+        import dataclasses
+
         import sparse_attention_15_b200 as dsa
 
         self.dsa = dsa
-        self.cfg = cfg = get_config(name)
+        cfg = get_config(name)
+        if S is not None or T is not None:  # a reduced case of the same workload (profiling)
+            S = cfg.S if S is None else S
+            T = cfg.T if T is None else T
+            cfg = dataclasses.replace(cfg, S=S, T=T,
+                                      description=f"{cfg.description} [reduced: S={S}, T={T}]")
+        self.cfg = cfg
         self.device = device
         B = cfg.B
         if name == "c4":  # 174 GB of expanded K/V cache: shrink the batch only if it cannot fit
@@ -354,6 +376,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
+    ap.add_argument("--S", type=int, default=None, help="reduced query count (profiling cases)")
+    ap.add_argument("--T", type=int, default=None, help="reduced key count (profiling cases)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world, rank, local = dist_setup(args)
@@ -377,7 +401,7 @@ def main():
                                 device_id=dev)
         pg = dist
 
-    wl = Workload(args.config, dev, seed_offset=rank)
+    wl = Workload(args.config, dev, seed_offset=rank, S=args.S, T=args.T)
     cfg = wl.cfg
     nst = len(wl.stages)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
@@ -417,13 +441,9 @@ def main():
         for j in range(nst):
             stage_ms[j] += ev[i][j].elapsed_time(ev[i][j + 1])
     stage_ms /= args.steps
-    step_ms = float(stage_ms.sum())
-    if pg is not None:
-        t = torch.tensor([step_ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        step_ms = float(t.item())
+    step_ms = reduce_max(float(stage_ms.sum()), pg, dev)
     units = wl.B * cfg.S * world
-    value = units / (step_ms / 1e3)
+    value = job_value(wl.B * cfg.S, world, step_ms)
 
     # roofline of the dominant stage
     peaks, peak_src = load_peaks()
@@ -475,11 +495,8 @@ def main():
             wl.e2e_step(host, dev_bufs, out_host)
             e1[i].record()
         barrier()
-        e2e_ms = sum(e0[i].elapsed_time(e1[i]) for i in range(n_e2e)) / n_e2e
-        if pg is not None:
-            t = torch.tensor([e2e_ms], device=dev)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = reduce_max(sum(e0[i].elapsed_time(e1[i]) for i in range(n_e2e)) / n_e2e, pg,
+                            dev)
         h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
         e2e = {"value": units / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(out_host.numel() * out_host.element_size()),

@@ -21,9 +21,11 @@
 // rescaled) when a row's block max exceeds it by more than 2^8, so exp2 arguments stay
 // <= 8 and rescales are rare.
 //
-// Roles: warp 0 TMA producer, warp 1 MMA issuer (one thread), warps 4..7 softmax and
-// epilogue (thread = query row = TMEM lane).  Persistent CTAs take items round-robin,
-// longest first.  Every wait is bounded.
+// Roles: warp 0 TMA producer of Q and K, warp 2 of V, warp 1 MMA issuer (one thread), warps
+// 4..11 softmax and
+// epilogue in two groups that take alternate key blocks (thread = query row = TMEM lane),
+// each with its own O accumulator and running (max, sum); the groups merge at the end of
+// an item.  Persistent CTAs take items in snake order, longest first.  Every wait is bounded.
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -62,13 +64,15 @@ struct FaCfg {
   static constexpr int V_BYTES = VH * SLICE;
   static constexpr int KV_BYTES = K_BYTES + V_BYTES;
   static constexpr int STAGES = 2;
-  static constexpr int SMEM = Q_BYTES + STAGES * KV_BYTES + 256 + 1024;
-  static constexpr int THREADS = 32 * (kSoftWarp0 + 4);
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int ML_BYTES = 2 * 2 * kBlk * 2 * 4;  // [buffer][group][row][m,l] floats
+  static constexpr int SMEM = Q_BYTES + STAGES * KV_BYTES + BAR_BYTES + ML_BYTES + 1024;
+  static constexpr int THREADS = 32 * (kSoftWarp0 + 8);  // two softmax groups of 4 warps
   static constexpr int S_COLS = kBlk;              // fp32 columns of one S buffer
-  static constexpr int O_COL = 2 * S_COLS;         // O starts after S0, S1
+  static constexpr int O_COL = 2 * S_COLS;         // O0, O1 start after S0, S1
   static constexpr int TMEM_COLS = 512;
-  static_assert(DQK % 64 == 0 && DV % 64 == 0 && DV <= 256, "head dims");
-  static_assert(O_COL + DV <= TMEM_COLS, "TMEM budget");
+  static_assert(DQK % 64 == 0 && DV % 64 == 0 && DV <= 128, "head dims");
+  static_assert(O_COL + 2 * DV <= TMEM_COLS, "TMEM budget");
 };
 
 // Instruction descriptor, kind::f16, bf16 A/B, f32 D, with the B operand MN-major.
@@ -119,6 +123,11 @@ __device__ __forceinline__ void drain(uint64_t* bar, uint32_t parity) {
 struct Item {
   int qb, b, h;
 };
+// The k-th item of CTA c: items are dealt in snake order (0..G-1, then G-1..0, ...), so a CTA
+// that took one of the longest causal items in a round takes one of the shorter in the next.
+__device__ __forceinline__ int snake_item(int k, int c, int G) {
+  return k * G + ((k & 1) ? (G - 1 - c) : c);
+}
 __device__ __forceinline__ Item item_of(const AttnArgs& a, int i) {
   Item it;
   it.h = i % a.H;
@@ -154,15 +163,19 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(KVs + C::STAGES * C::KV_BYTES);
   uint64_t* q_full = bars;           // 1
   uint64_t* q_empty = bars + 1;      // 1
-  uint64_t* kv_full = bars + 2;      // [2]
-  uint64_t* kv_empty = bars + 4;     // [2]
+  uint64_t* k_full = bars + 2;       // [2] K block landed
+  uint64_t* k_empty = bars + 4;      // [2] K block consumed by S = Q K^T
   uint64_t* s_full = bars + 6;       // [2]
   uint64_t* s_empty = bars + 8;      // [2]
   uint64_t* p_full = bars + 10;      // [2]
-  uint64_t* pv_done = bars + 12;     // 1 (one phase per block)
-  uint64_t* o_empty = bars + 13;     // 1 (one phase per item)
-  uint64_t* mma_done = bars + 14;    // 1
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
+  uint64_t* pv_done = bars + 12;     // [2] (one phase per block of that parity)
+  uint64_t* o_empty = bars + 14;     // 1 (one phase per item)
+  uint64_t* ml_full = bars + 15;     // 1 (one phase per item)
+  uint64_t* mma_done = bars + 16;    // 1
+  uint64_t* v_full = bars + 17;      // [2] V block landed
+  uint64_t* v_empty = bars + 19;     // [2] V block consumed by O += P V
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 21);
+  float* ml = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + C::BAR_BYTES);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_items = a.B * a.H * a.nqb;
@@ -171,11 +184,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1); mbar_init(q_empty, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&kv_full[i], 1); mbar_init(&kv_empty[i], 1);
+      mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1);
+      mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1);
       mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], 1);
       mbar_init(&p_full[i], 4);
     }
-    mbar_init(pv_done, 1); mbar_init(o_empty, 4); mbar_init(mma_done, 1);
+    mbar_init(&pv_done[0], 1); mbar_init(&pv_done[1], 1);
+    mbar_init(o_empty, 8); mbar_init(ml_full, 8 * 32); mbar_init(mma_done, 1);
     fence_mbar_init();
     prefetch_tmap(&qmap); prefetch_tmap(&kmap); prefetch_tmap(&vmap);
   }
@@ -188,41 +203,53 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
+  if (warp == 0 || warp == 2) {
+    // ------------------------------------------------------------------ TMA producers
+    // warp 0: Q blocks and K blocks; warp 2: V blocks.  K and V have separate rings: a K
+    // stage is free as soon as S = Q K^T is done, long before the P V of the same block, so
+    // the next K blocks stream in while the softmax runs.
+    const bool kq = warp == 0;
     if (lane == 0) {
       uint32_t g = 0, ni = 0;
       bool ok = true;
-      for (int i = blockIdx.x; ok && i < n_items; i += gridDim.x, ++ni) {
+      uint64_t* full = kq ? k_full : v_full;
+      uint64_t* empty = kq ? k_empty : v_empty;
+      for (int kk_ = 0, i = snake_item(0, blockIdx.x, gridDim.x); ok && i < n_items;
+           i = snake_item(++kk_, blockIdx.x, gridDim.x), ++ni) {
         const Item it = item_of(a, i);
         int j0, j1;
         key_range<C::BAND>(a, it, &j0, &j1);
-        if (ni > 0 && !mbar_wait(q_empty, (ni - 1) & 1)) { ok = false; break; }
-        mbar_arrive_expect_tx(q_full, C::Q_BYTES);
-        const int qrow = it.b * a.S + it.qb * kBlk;
+        if (kq) {
+          if (ni > 0 && !mbar_wait(q_empty, (ni - 1) & 1)) { ok = false; break; }
+          mbar_arrive_expect_tx(q_full, C::Q_BYTES);
+          const int qrow = it.b * a.S + it.qb * kBlk;
 #pragma unroll
-        for (int x = 0; x < C::QKH; ++x)
-          tma_load_3d(Qs + x * C::SLICE, &qmap, x * 64, it.h, qrow, q_full);
+          for (int x = 0; x < C::QKH; ++x)
+            tma_load_3d(Qs + x * C::SLICE, &qmap, x * 64, it.h, qrow, q_full);
+        }
         const int kvh = it.h / group;
         for (int j = j0; j < j1; ++j, ++g) {
           const int st = g & 1;
-          if (g >= 2 && !mbar_wait(&kv_empty[st], ((g >> 1) - 1) & 1)) { ok = false; break; }
-          mbar_arrive_expect_tx(&kv_full[st], C::KV_BYTES);
-          uint8_t* kdst = KVs + st * C::KV_BYTES;
+          if (g >= 2 && !mbar_wait(&empty[st], ((g >> 1) - 1) & 1)) { ok = false; break; }
+          uint8_t* dst = KVs + st * C::KV_BYTES + (kq ? 0 : C::K_BYTES);
           const int krow = it.b * a.T + j * kBlk;
+          if (kq) {
+            mbar_arrive_expect_tx(&full[st], C::K_BYTES);
 #pragma unroll
-          for (int x = 0; x < C::QKH; ++x)
-            tma_load_3d(kdst + x * C::SLICE, &kmap, x * 64, kvh, krow, &kv_full[st]);
+            for (int x = 0; x < C::QKH; ++x)
+              tma_load_3d(dst + x * C::SLICE, &kmap, x * 64, kvh, krow, &full[st]);
+          } else {
+            mbar_arrive_expect_tx(&full[st], C::V_BYTES);
 #pragma unroll
-          for (int x = 0; x < C::VH; ++x)
-            tma_load_3d(kdst + C::K_BYTES + x * C::SLICE, &vmap, x * 64, kvh, krow,
-                        &kv_full[st]);
+            for (int x = 0; x < C::VH; ++x)
+              tma_load_3d(dst + x * C::SLICE, &vmap, x * 64, kvh, krow, &full[st]);
+          }
         }
       }
       // let the copies in flight land before exit
-      if (g >= 1) drain(&kv_full[(g - 1) & 1], ((g - 1) >> 1) & 1);
-      if (g >= 2) drain(&kv_full[(g - 2) & 1], ((g - 2) >> 1) & 1);
-      if (ni >= 1) drain(q_full, (ni - 1) & 1);
+      if (g >= 1) drain(&full[(g - 1) & 1], ((g - 1) >> 1) & 1);
+      if (g >= 2) drain(&full[(g - 2) & 1], ((g - 2) >> 1) & 1);
+      if (kq && ni >= 1) drain(q_full, (ni - 1) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
@@ -235,7 +262,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       // S_g = Q K_g^T into S[g & 1]
       auto issue_qk = [&](uint32_t gg) -> bool {
         const int st = gg & 1;
-        if (!mbar_wait(&kv_full[st], (gg >> 1) & 1)) return false;
+        if (!mbar_wait(&k_full[st], (gg >> 1) & 1)) return false;
         if (gg >= 2 && !mbar_wait(&s_empty[gg & 1], ((gg >> 1) - 1) & 1)) return false;
         tc_fence_after();
         const uint32_t k_base = smem_u32(KVs + st * C::KV_BYTES);
@@ -246,9 +273,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                       sw128_kmajor_desc(k_base + off), idesc_qk, kk > 0 ? 1u : 0u);
         }
         umma_commit(&s_full[gg & 1]);
+        umma_commit(&k_empty[st]);
         return true;
       };
-      for (int i = blockIdx.x; ok && i < n_items; i += gridDim.x, ++ni) {
+      for (int kk_ = 0, i = snake_item(0, blockIdx.x, gridDim.x); ok && i < n_items;
+           i = snake_item(++kk_, blockIdx.x, gridDim.x), ++ni) {
         const Item it = item_of(a, i);
         int j0, j1;
         key_range<C::BAND>(a, it, &j0, &j1);
@@ -261,20 +290,23 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           if (j + 1 == nb) umma_commit(q_empty);  // Q free once the last S is computed
           if (!mbar_wait(&p_full[gg & 1], (gg >> 1) & 1)) { ok = false; break; }
           if (j == 0 && ni > 0 && !mbar_wait(o_empty, (ni - 1) & 1)) { ok = false; break; }
+          if (!mbar_wait(&v_full[gg & 1], (gg >> 1) & 1)) { ok = false; break; }
           tc_fence_after();
           const uint32_t v_base = smem_u32(KVs + (gg & 1) * C::KV_BYTES + C::K_BYTES);
           const uint32_t p_tmem = tmem + (gg & 1) * C::S_COLS;
+          const uint32_t o_tmem = tmem + C::O_COL + (gg & 1) * C::DV;
 #pragma unroll
           for (int kk = 0; kk < kBlk / 16; ++kk) {
-            // 16 keys: 8 packed P columns; 16 V rows = 2 swizzle atoms of 8 rows
+            // keys 16kk..16kk+15: 8 packed columns of P_hi at 32*(kk/2) + 8*(kk%2), P_lo 16
+            // columns further; V rows 16kk..: 2 swizzle atoms of 8 rows
+            const uint32_t pc = 32 * (kk >> 1) + 8 * (kk & 1);
             const uint64_t vdesc = sw128_mnmajor_desc(v_base + kk * 2048, C::SLICE, 1024);
-            umma_f16_ts(tmem + C::O_COL, p_tmem + kk * 8, vdesc, idesc_pv,
-                        (j > 0 || kk > 0) ? 1u : 0u);
-            umma_f16_ts(tmem + C::O_COL, p_tmem + 64 + kk * 8, vdesc, idesc_pv, 1u);
+            umma_f16_ts(o_tmem, p_tmem + pc, vdesc, idesc_pv, (j >= 2 || kk > 0) ? 1u : 0u);
+            umma_f16_ts(o_tmem, p_tmem + pc + 16, vdesc, idesc_pv, 1u);
           }
-          umma_commit(&kv_empty[gg & 1]);
+          umma_commit(&v_empty[gg & 1]);
           umma_commit(&s_empty[gg & 1]);
-          umma_commit(pv_done);
+          umma_commit(&pv_done[gg & 1]);
         }
         g += nb;
       }
@@ -283,33 +315,41 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     }
   } else if (warp >= kSoftWarp0) {
     // ------------------------------------------------------------------ softmax + epilogue
+    // Group e (warps 4+4e..7+4e) owns the key blocks of parity e and accumulator O_e; thread =
+    // query row (TMEM lane).  At the end of an item the two groups exchange (m, l) through
+    // shared memory and each writes half of the output columns.
+    const int grp = (warp - kSoftWarp0) >> 2;
     const int quad = warp & 3;
+    const int row = quad * 32 + lane;
     const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
     const float ninf = __int_as_float(0xff800000);
     uint32_t g = 0, ni = 0;
     bool ok = true;
-    for (int i = blockIdx.x; ok && i < n_items; i += gridDim.x, ++ni) {
+    for (int kk_ = 0, i = snake_item(0, blockIdx.x, gridDim.x); ok && i < n_items;
+         i = snake_item(++kk_, blockIdx.x, gridDim.x), ++ni) {
       const Item it = item_of(a, i);
       int j0, j1;
       key_range<C::BAND>(a, it, &j0, &j1);
       const int nb = j1 - j0;
-      const int s = it.qb * kBlk + quad * 32 + lane;
+      const int s = it.qb * kBlk + row;
       const int spos = s + a.q_off;
       const bool row_ok = s < a.S;
       const uint32_t* mrow =
           (!C::BAND && row_ok) ? a.mask + ((size_t)it.b * a.S + s) * a.mask_stride : nullptr;
+      const int jfirst = (int)((grp - g) & 1u);  // first block of this group's parity
       float m_used = ninf, l = 0.f;
-      for (int j = 0; j < nb; ++j) {
+      uint4 nb4 = make_uint4(0u, 0u, 0u, 0u);
+      if (mrow && jfirst < nb)
+        nb4 = __ldg(reinterpret_cast<const uint4*>(mrow + (((j0 + jfirst) * kBlk) >> 5)));
+      const uint32_t o_col = C::O_COL + grp * C::DV;
+      for (int j = jfirst; j < nb; j += 2) {
         const uint32_t gg = g + j;
         const int t0 = (j0 + j) * kBlk;
-        if (!warp_wait(&s_full[gg & 1], (gg >> 1) & 1)) { ok = false; break; }
-        tc_fence_after();
         uint32_t bits[4] = {0u, 0u, 0u, 0u};
         if (!C::BAND) {
-          if (mrow) {
-            const uint4 w4 = __ldg(reinterpret_cast<const uint4*>(mrow + (t0 >> 5)));
-            bits[0] = w4.x; bits[1] = w4.y; bits[2] = w4.z; bits[3] = w4.w;
-          }
+          bits[0] = nb4.x; bits[1] = nb4.y; bits[2] = nb4.z; bits[3] = nb4.w;
+          if (mrow && j + 2 < nb)
+            nb4 = __ldg(reinterpret_cast<const uint4*>(mrow + ((t0 + 2 * kBlk) >> 5)));
         } else if (row_ok) {
           // band: spos - window < t <= spos, t < T
           const int lo = max(spos - a.window + 1, 0) - t0, hi = min(spos, a.T - 1) - t0;
@@ -321,43 +361,49 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                                                  : (((1u << (a1 - a0 + 1)) - 1u) << a0));
           }
         }
-        // raw S row: all four TMEM reads in flight, one wait
-        uint32_t r[kBlk];
-        tmem_ld32(t_lane + (gg & 1) * C::S_COLS + 0, *reinterpret_cast<uint32_t(*)[32]>(r + 0));
-        tmem_ld32(t_lane + (gg & 1) * C::S_COLS + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
-        tmem_ld32(t_lane + (gg & 1) * C::S_COLS + 64, *reinterpret_cast<uint32_t(*)[32]>(r + 64));
-        tmem_ld32(t_lane + (gg & 1) * C::S_COLS + 96, *reinterpret_cast<uint32_t(*)[32]>(r + 96));
-        tmem_wait_ld();
-        // masked raw scores (unselected -> -inf) and their max; the scale is positive, so
-        // max(scale * s) = scale * max(s) and the scale folds into the exp argument below
-        float x[kBlk];
+        if (!warp_wait(&s_full[gg & 1], (gg >> 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t s_col = t_lane + (gg & 1) * C::S_COLS;
+        // pass 1: max of the selected raw scores (the scale is positive: it commutes with max)
         float mraw = ninf;
+        {
+          uint32_t r[2][32];
+          tmem_ld32(s_col + 0, r[0]);
+          tmem_ld32(s_col + 32, r[1]);
+          tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+          for (int c = 0; c < 2; ++c)
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            x[c * 32 + e] = (bits[c] & (1u << e)) ? __uint_as_float(r[c * 32 + e]) : ninf;
-            mraw = fmaxf(mraw, x[c * 32 + e]);
-          }
+            for (int e = 0; e < 32; ++e)
+              if (bits[c] & (1u << e)) mraw = fmaxf(mraw, __uint_as_float(r[c][e]));
+          tmem_ld32(s_col + 64, r[0]);
+          tmem_ld32(s_col + 96, r[1]);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (bits[2 + c] & (1u << e)) mraw = fmaxf(mraw, __uint_as_float(r[c][e]));
+        }
         const float mb = mraw * a.qk_scale;
         const bool need = mb > m_used + kRescaleLog2;
         if (__any_sync(0xffffffffu, need)) {
           const float m_new = need ? mb : m_used;
           const float alpha = (l > 0.f) ? exp2f(m_used - m_new) : 0.f;
-          // O holds the previous blocks of this item: rescale it once the last P V landed
-          if (j > 0 && __any_sync(0xffffffffu, need && l > 0.f)) {
-            if (!warp_wait(pv_done, (gg - 1) & 1)) { ok = false; break; }
+          // O_grp holds this group's earlier blocks of the item: rescale it once their P V landed
+          if (j >= 2 && __any_sync(0xffffffffu, need && l > 0.f)) {
+            if (!warp_wait(&pv_done[gg & 1], ((gg >> 1) - 1) & 1)) { ok = false; break; }
             tc_fence_after();
 #pragma unroll 1
             for (int c = 0; c < C::DV / 16; ++c) {
               uint32_t r[16];
-              tmem_ld16(t_lane + C::O_COL + c * 16, r);
+              tmem_ld16(t_lane + o_col + c * 16, r);
               tmem_wait_ld();
               if (need) {
 #pragma unroll
                 for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
               }
-              tmem_st16(t_lane + C::O_COL + c * 16, r);
+              tmem_st16(t_lane + o_col + c * 16, r);
             }
             tmem_wait_st();
           }
@@ -366,21 +412,25 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             m_used = m_new;
           }
         }
-        // P = P_hi + P_lo, both bf16 (P_hi = bf16(p), P_lo = bf16(p - P_hi)): the second
-        // product recovers the bits bf16 drops, so O carries ~2^-17 relative error in P
-        // instead of 2^-9.  P_hi fills columns [0,64) of the S buffer, P_lo [64,128).
-        float rs = 0.f;
-        // exp2(scale * s - m); -inf (unselected) gives exactly 0.  With no selected key yet
-        // (m_used = -inf) every x is -inf as well; subtracting 0 keeps the result 0.
+        // pass 2, 32 keys at a time: P = exp2(scale*s - m) for selected keys, 0 otherwise,
+        // split into bf16 P_hi + P_lo (P_lo = bf16(p - P_hi) keeps ~2^-17 relative
+        // precision).  Chunk c's P_hi goes to its own columns [32c, 32c+16), P_lo to
+        // [32c+16, 32c+32): only columns already read are overwritten.
         const float msub = m_used == ninf ? 0.f : m_used;
+        float rs = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tmem_ld32(s_col + c * 32, r);
+          tmem_wait_ld();
+          uint32_t ph[16], pl[16];
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          uint32_t ph[32], pl[32];
-#pragma unroll
-          for (int e2 = 0; e2 < 32; ++e2) {
-            const int e = hf * 64 + 2 * e2;
-            const float p0 = ex2_ftz(fmaf(x[e], a.qk_scale, -msub));
-            const float p1 = ex2_ftz(fmaf(x[e + 1], a.qk_scale, -msub));
+          for (int e2 = 0; e2 < 16; ++e2) {
+            const int e = 2 * e2;
+            const float x0 = (bits[c] & (1u << e)) ? __uint_as_float(r[e]) : ninf;
+            const float x1 = (bits[c] & (1u << (e + 1))) ? __uint_as_float(r[e + 1]) : ninf;
+            const float p0 = ex2_ftz(fmaf(x0, a.qk_scale, -msub));
+            const float p1 = ex2_ftz(fmaf(x1, a.qk_scale, -msub));
             rs += p0 + p1;
             const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
             const float2 hf2 = __bfloat1622float2(h2);
@@ -388,8 +438,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             ph[e2] = *reinterpret_cast<const uint32_t*>(&h2);
             pl[e2] = *reinterpret_cast<const uint32_t*>(&l2);
           }
-          tmem_st32(t_lane + (gg & 1) * C::S_COLS + hf * 32, ph);
-          tmem_st32(t_lane + (gg & 1) * C::S_COLS + 64 + hf * 32, pl);
+          tmem_st16(s_col + c * 32, ph);
+          tmem_st16(s_col + c * 32 + 16, pl);
         }
         l += rs;
         tmem_wait_st();
@@ -398,41 +448,61 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         if (lane == 0) mbar_arrive(&p_full[gg & 1]);
       }
       if (!ok) break;
-      g += nb;
-      // epilogue: O / l, gate, bf16 store
-      if (!warp_wait(pv_done, (g - 1) & 1)) { ok = false; break; }
+      // ---------------- epilogue: merge the two groups, normalise, gate, bf16 store
+      const int jlast = ((nb - 1 - jfirst) >= 0) ? jfirst + ((nb - 1 - jfirst) & ~1) : -1;
+      if (jlast >= 0) {
+        const uint32_t gl = g + jlast;
+        if (!warp_wait(&pv_done[gl & 1], (gl >> 1) & 1)) { ok = false; break; }
+      }
+      float* mlb = ml + (ni & 1) * (2 * kBlk * 2);
+      mlb[(grp * kBlk + row) * 2 + 0] = m_used;
+      mlb[(grp * kBlk + row) * 2 + 1] = l;
+      mbar_arrive(ml_full);
+      if (!warp_wait(ml_full, ni & 1)) { ok = false; break; }
       tc_fence_after();
-      float f = l > 0.f ? 1.0f / l : 0.f;
+      const float m0 = mlb[(0 * kBlk + row) * 2], l0 = mlb[(0 * kBlk + row) * 2 + 1];
+      const float m1 = mlb[(1 * kBlk + row) * 2], l1 = mlb[(1 * kBlk + row) * 2 + 1];
+      const float M = fmaxf(m0, m1);
+      const float a0 = l0 > 0.f ? exp2f(m0 - M) : 0.f;
+      const float a1 = l1 > 0.f ? exp2f(m1 - M) : 0.f;
+      const float L = l0 * a0 + l1 * a1;
+      float f = L > 0.f ? 1.0f / L : 0.f;
       if (a.gate && row_ok)
-        f *= gate_act(__bfloat162float(
-                          static_cast<const __nv_bfloat16*>(a.gate)[((size_t)it.b * a.S + s) * a.H +
-                                                                   it.h]),
+        f *= gate_act(__bfloat162float(static_cast<const __nv_bfloat16*>(
+                          a.gate)[((size_t)it.b * a.S + s) * a.H + it.h]),
                       a.gate_mode);
+      const float w0 = a0 * f, w1 = a1 * f;
       __nv_bfloat16* orow = a.out + (((size_t)it.b * a.S + s) * a.H + it.h) * C::DV;
+      // this group writes output columns [grp*DV/2, (grp+1)*DV/2)
 #pragma unroll 1
-      for (int c = 0; c < C::DV / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(t_lane + C::O_COL + c * 32, r);
+      for (int c = 0; c < C::DV / 64; ++c) {
+        const int col = grp * (C::DV / 2) + c * 32;
+        uint32_t r0[32], r1[32];
+        tmem_ld32(t_lane + C::O_COL + col, r0);
+        tmem_ld32(t_lane + C::O_COL + C::DV + col, r1);
         tmem_wait_ld();
-        if (c == C::DV / 32 - 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(o_empty);
-        }
         if (row_ok) {
           uint4 v4[4];
           uint32_t* vw = reinterpret_cast<uint32_t*>(v4);
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(r[2 * e]) * f,
-                                                      __uint_as_float(r[2 * e + 1]) * f);
-            vw[e] = *reinterpret_cast<uint32_t*>(&h2);
+            // an O buffer with no weight (l = 0) may hold stale values: select, never multiply
+            const float y0 = (a0 > 0.f ? __uint_as_float(r0[2 * e]) * w0 : 0.f) +
+                             (a1 > 0.f ? __uint_as_float(r1[2 * e]) * w1 : 0.f);
+            const float y1 = (a0 > 0.f ? __uint_as_float(r0[2 * e + 1]) * w0 : 0.f) +
+                             (a1 > 0.f ? __uint_as_float(r1[2 * e + 1]) * w1 : 0.f);
+            const __nv_bfloat162 h2 = __floats2bfloat162_rn(y0, y1);
+            vw[e] = *reinterpret_cast<const uint32_t*>(&h2);
           }
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+          uint4* dst = reinterpret_cast<uint4*>(orow + col);
 #pragma unroll
           for (int e = 0; e < 4; ++e) dst[e] = v4[e];
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(o_empty);
+      g += nb;
     }
   }
 

@@ -260,19 +260,39 @@ int heads_per_warp(int H) {
   return 0;
 }
 
-// Split policy: few query rows and long key lists -> spread the keys over CTAs.
+// Split policy: few query rows and long key lists -> spread the keys over CTAs.  The split
+// count is chosen so that rows * nsplit fills whole waves of the resident CTAs (two per SM
+// on a 148-SM B200) as closely as possible, with at least 64 keys per split and at most 32
+// splits; the fewest splits within 5% of full waves win.  Depends on the shape only (no device query), so
+// workspace sizes are reproducible.
 void split_policy(int rows, int nkeys, int* nsplit, int* kps, bool allow_split = true) {
-  const int target_ctas = 4 * 148;
-  if (!allow_split || rows >= target_ctas || nkeys <= 128) {
+  const int resident = 2 * 148;
+  if (!allow_split || rows >= resident || nkeys <= 128) {
     *nsplit = 1;
     *kps = nkeys;
     return;
   }
-  int ns = (target_ctas + rows - 1) / rows;
   int max_ns = (nkeys + 63) / 64;
-  if (ns > max_ns) ns = max_ns;
-  if (ns < 1) ns = 1;
-  *kps = (nkeys + ns - 1) / ns;
+  if (max_ns > 32) max_ns = 32;
+  // the fewest splits whose waves are at least 95% full; else the fullest
+  int best = 1;
+  double best_eff = -1.0;
+  for (int ns = 1; ns <= max_ns; ++ns) {
+    const int k = (nkeys + ns - 1) / ns;
+    const int n = (nkeys + k - 1) / k;           // splits actually used
+    const long long items = (long long)rows * n;
+    const long long waves = (items + resident - 1) / resident;
+    const double eff = (double)items / (double)(waves * resident);
+    if (eff >= 0.95) {
+      best = ns;
+      break;
+    }
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best = ns;
+    }
+  }
+  *kps = (nkeys + best - 1) / best;
   *nsplit = (nkeys + *kps - 1) / *kps;
 }
 

@@ -59,8 +59,9 @@ def test_noalloc_rejects_shapes_beyond_its_scratch(lib):
     # rejected on the host before any device work (runs without a GPU)
     L = lib.lib()
     fake = ctypes.c_void_p(0x10000)
+    # 200 decode rows x 2048 keys: about 33 MB of split-key partials, over the 16 MiB
     st = L.dsa_sparse_attn_noalloc(1, fake, fake, fake, fake, 2048, None, 0, 0.0,
-                                   512, 1, 131072, 32, 192, 128, fake, None)
+                                   200, 1, 131072, 32, 192, 128, fake, None)
     assert st == 2
     assert b"more than the fixed" in L.dsa_last_error()
     assert L.dsa_sparse_attn_noalloc(1, None, fake, fake, fake, 8, None, 0, 0.0, 1, 1, 8, 4, 64,
