@@ -21,9 +21,9 @@
 // rescaled) when a row's block max exceeds it by more than 2^8, so exp2 arguments stay
 // <= 8 and rescales are rare.
 //
-// Roles: warp 0 TMA producer of Q and K, warp 2 of V, warp 1 MMA issuer (one thread), warps
-// 4..11 softmax and
+// Roles: warps 0..7 softmax and
 // epilogue in two groups that take alternate key blocks (thread = query row = TMEM lane),
+// warp 8 TMA producer of Q and K, warp 10 of V, warp 9 MMA issuer (one thread),
 // each with its own O accumulator and running (max, sum); the groups merge at the end of
 // an item.  Persistent CTAs take items in snake order, longest first.  Every wait is bounded.
 #include <cudaTypedefs.h>
@@ -38,7 +38,10 @@ namespace dsa {
 namespace {
 
 constexpr int kBlk = 128;     // queries per item = keys per block
-constexpr int kSoftWarp0 = 4; // softmax warps 4..7
+// Warp roles: 0..7 softmax (two groups of four: warp % 4 is the TMEM lane quadrant),
+// 8 TMA producer of Q and K, 9 MMA issuer (and TMEM owner), 10 TMA producer of V.
+constexpr int kSoftWarps = 8;
+constexpr int kWarpQK = 8, kWarpMma = 9, kWarpV = 10;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;
 
@@ -67,7 +70,7 @@ struct FaCfg {
   static constexpr int BAR_BYTES = 256;
   static constexpr int ML_BYTES = 2 * 2 * kBlk * 2 * 4;  // [buffer][group][row][m,l] floats
   static constexpr int SMEM = Q_BYTES + STAGES * KV_BYTES + BAR_BYTES + ML_BYTES + 1024;
-  static constexpr int THREADS = 32 * (kSoftWarp0 + 8);  // two softmax groups of 4 warps
+  static constexpr int THREADS = 32 * 11;
   static constexpr int S_COLS = kBlk;              // fp32 columns of one S buffer
   static constexpr int O_COL = 2 * S_COLS;         // O0, O1 start after S0, S1
   static constexpr int TMEM_COLS = 512;
@@ -194,7 +197,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     fence_mbar_init();
     prefetch_tmap(&qmap); prefetch_tmap(&kmap); prefetch_tmap(&vmap);
   }
-  if (warp == 1) {
+  if (warp == kWarpMma) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -203,12 +206,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0 || warp == 2) {
+  if (warp == kWarpQK || warp == kWarpV) {
     // ------------------------------------------------------------------ TMA producers
     // warp 0: Q blocks and K blocks; warp 2: V blocks.  K and V have separate rings: a K
     // stage is free as soon as S = Q K^T is done, long before the P V of the same block, so
     // the next K blocks stream in while the softmax runs.
-    const bool kq = warp == 0;
+    const bool kq = warp == kWarpQK;
     if (lane == 0) {
       uint32_t g = 0, ni = 0;
       bool ok = true;
@@ -251,7 +254,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       if (g >= 2) drain(&full[(g - 2) & 1], ((g - 2) >> 1) & 1);
       if (kq && ni >= 1) drain(q_full, (ni - 1) & 1);
     }
-  } else if (warp == 1) {
+  } else if (warp == kWarpMma) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kBlk, kBlk);
@@ -313,12 +316,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       umma_commit(mma_done);
       drain(mma_done, 0);
     }
-  } else if (warp >= kSoftWarp0) {
+  } else if (warp < kSoftWarps) {
     // ------------------------------------------------------------------ softmax + epilogue
-    // Group e (warps 4+4e..7+4e) owns the key blocks of parity e and accumulator O_e; thread =
+    // Group e (warps 4e..4e+3) owns the key blocks of parity e and accumulator O_e; thread =
     // query row (TMEM lane).  At the end of an item the two groups exchange (m, l) through
     // shared memory and each writes half of the output columns.
-    const int grp = (warp - kSoftWarp0) >> 2;
+    const int grp = warp >> 2;
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
     const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
@@ -364,26 +367,21 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         if (!warp_wait(&s_full[gg & 1], (gg >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
         const uint32_t s_col = t_lane + (gg & 1) * C::S_COLS;
-        // pass 1: max of the selected raw scores (the scale is positive: it commutes with max)
+        // pass 1: max of the selected raw scores (the scale is positive: it commutes with max);
+        // the whole row in one TMEM round trip
         float mraw = ninf;
         {
-          uint32_t r[2][32];
-          tmem_ld32(s_col + 0, r[0]);
-          tmem_ld32(s_col + 32, r[1]);
+          uint32_t r[kBlk];
+          tmem_ld32(s_col + 0, *reinterpret_cast<uint32_t(*)[32]>(r + 0));
+          tmem_ld32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
+          tmem_ld32(s_col + 64, *reinterpret_cast<uint32_t(*)[32]>(r + 64));
+          tmem_ld32(s_col + 96, *reinterpret_cast<uint32_t(*)[32]>(r + 96));
           tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 2; ++c)
+          for (int c = 0; c < 4; ++c)
 #pragma unroll
             for (int e = 0; e < 32; ++e)
-              if (bits[c] & (1u << e)) mraw = fmaxf(mraw, __uint_as_float(r[c][e]));
-          tmem_ld32(s_col + 64, r[0]);
-          tmem_ld32(s_col + 96, r[1]);
-          tmem_wait_ld();
-#pragma unroll
-          for (int c = 0; c < 2; ++c)
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (bits[2 + c] & (1u << e)) mraw = fmaxf(mraw, __uint_as_float(r[c][e]));
+              if (bits[c] & (1u << e)) mraw = fmaxf(mraw, __uint_as_float(r[c * 32 + e]));
         }
         const float mb = mraw * a.qk_scale;
         const bool need = mb > m_used + kRescaleLog2;
@@ -508,7 +506,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }

@@ -363,7 +363,10 @@ cudaError_t launch_gather_attn(const AttnProblem& p, void* ws, size_t ws_bytes,
   a.k_bytes = (uint32_t)(p.HKV * p.DQK * es);
   a.v_bytes = (uint32_t)(p.HKV * p.DV * es);
   a.slot_bytes = (a.k_bytes + a.v_bytes + 127) & ~127u;
-  int ns = (int)((96 * 1024) / a.slot_bytes);
+  // as many row slots as fit while two CTAs stay resident per SM (227 KB shared memory):
+  // the ring is what keeps HBM busy, a row pair being ~20 KB at the large shapes
+  const size_t per_cta = (227 * 1024) / 2 - 1024 - a.key_list_bytes - 512;
+  int ns = (int)(per_cta / a.slot_bytes);
   ns = ns < 2 ? 2 : (ns > 16 ? 16 : ns);
   a.nslots = ns;
   const size_t smem = 1024 + a.key_list_bytes + (size_t)ns * a.slot_bytes;

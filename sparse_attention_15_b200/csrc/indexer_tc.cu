@@ -49,9 +49,10 @@ struct TcArgs {
   int max_chunks;  // units per query block slot (chunks of the longest block)
 };
 
-template <int HI_, int DI_, int NQ_, int NE_, int NA_>
+template <int HI_, int DI_, int NQ_, int NE_, int NA_, int NB_ = 2>
 struct TcCfg {
   static constexpr int HI = HI_, DI = DI_, NQ = NQ_, NE = NE_, NA = NA_;
+  static constexpr int NB = NB_;                  // query-block buffers (1 or 2)
   static constexpr int N = NQ * HI;               // MMA N: (query, head) columns
   static constexpr int KH = DI / 64;              // 64-element (128-byte) K slices
   static constexpr int A_SLICE = kTileM * 128;    // bytes of one K slice of a key tile
@@ -65,7 +66,7 @@ struct TcCfg {
   static constexpr int COLS_PER_WARP = N / EPI_GROUPS;
   static constexpr int THREADS = 32 * (kEpiWarp0 + NE);
   static constexpr int BAR_BYTES = 256;
-  static constexpr int SMEM = NA * A_BYTES + 2 * B_BYTES + BAR_BYTES + 1024;
+  static constexpr int SMEM = NA * A_BYTES + NB * B_BYTES + BAR_BYTES + 1024;
   static_assert(N % 16 == 0 && N >= 16 && N <= 256, "UMMA N");
   static_assert(HI <= 32 && 32 % HI == 0, "heads per 32-column chunk");
   static_assert(COLS_PER_WARP % 32 == 0, "epilogue chunking");
@@ -122,8 +123,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* As = smem;                               // NA key tiles
-  uint8_t* Bs = smem + C::NA * C::A_BYTES;          // 2 query blocks
-  uint64_t* bars = reinterpret_cast<uint64_t*>(Bs + 2 * C::B_BYTES);
+  uint8_t* Bs = smem + C::NA * C::A_BYTES;          // NB query blocks
+  uint64_t* bars = reinterpret_cast<uint64_t*>(Bs + C::NB * C::B_BYTES);
   uint64_t* a_full = bars;                          // [NA]
   uint64_t* a_empty = a_full + C::NA;               // [NA]
   uint64_t* b_full = a_empty + C::NA;               // [2]
@@ -163,8 +164,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       uint32_t ai = 0, bi = 0;
       bool ok = true;
       while (ok && it.next(a, C::NQ, ncta)) {
-        const int bb = bi & 1;
-        if (bi >= 2 && !mbar_wait(&b_empty[bb], ((bi >> 1) - 1) & 1)) { ok = false; break; }
+        const int bb = bi % C::NB;
+        if (bi >= (uint32_t)C::NB && !mbar_wait(&b_empty[bb], ((bi / C::NB) - 1) & 1)) {
+          ok = false;
+          break;
+        }
         mbar_arrive_expect_tx(&b_full[bb], C::B_BYTES);
         const int qrow = (it.b * a.S + it.qb * C::NQ) * C::HI;
 #pragma unroll
@@ -189,7 +193,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       // on the way out, let every copy this thread issued land
       for (uint32_t j = (ai > (uint32_t)C::NA ? ai - C::NA : 0); j < ai; ++j)
         drain_wait(&a_full[j % C::NA], (j / C::NA) & 1);
-      for (uint32_t j = (bi > 2 ? bi - 2 : 0); j < bi; ++j) drain_wait(&b_full[j & 1], (j >> 1) & 1);
+      for (uint32_t j = (bi > (uint32_t)C::NB ? bi - C::NB : 0); j < bi; ++j)
+        drain_wait(&b_full[j % C::NB], (j / C::NB) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
@@ -199,8 +204,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       uint32_t ai = 0, bi = 0, ci = 0;
       bool ok = true;
       while (ok && it.next(a, C::NQ, ncta)) {
-        const int bb = bi & 1;
-        if (!mbar_wait(&b_full[bb], (bi >> 1) & 1)) { ok = false; break; }
+        const int bb = bi % C::NB;
+        if (!mbar_wait(&b_full[bb], (bi / C::NB) & 1)) { ok = false; break; }
         const uint32_t b_base = smem_u32(Bs + bb * C::B_BYTES);
         for (int kt = it.k0; kt < it.k1; ++kt) {
           const int st = ai % C::NA;
@@ -241,6 +246,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     bool ok = true;
     while (ok && it.next(a, C::NQ, ncta)) {
       const int s_base = it.qb * C::NQ;
+      // the head weights of this unit's queries are the same for every key tile: lane l
+      // keeps the weight of column col0 + 32cc + l of each chunk cc, and the reduction
+      // below broadcasts it with a shuffle (no memory access inside the tile loop)
+      float wv[C::COLS_PER_WARP / 32];
+#pragma unroll
+      for (int cc = 0; cc < C::COLS_PER_WARP / 32; ++cc) {
+        const int col = col0 + cc * 32 + lane;
+        const int s = s_base + col / C::HI;
+        wv[cc] = s < a.S ? __ldg(a.w + ((size_t)it.b * a.S + s) * C::HI + col % C::HI) : 0.f;
+      }
       for (int kt = it.k0; kt < it.k1; ++kt) {
         const int ab = ci & 1;
         if (!warp_wait(&acc_full[ab], (ci >> 1) & 1)) { ok = false; break; }
@@ -267,11 +282,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             const int j = (col0 + cc * 32) / C::HI + qi;  // query within the block
             const int s = s_base + j;
             if (s < a.S) {  // ragged tail of the last block (warp-uniform)
-              const float* wr = a.w + ((size_t)it.b * a.S + s) * C::HI;
               float acc4[4] = {0.f, 0.f, 0.f, 0.f};  // four independent FMA chains
 #pragma unroll
               for (int h = 0; h < C::HI; h += 4) {
-                const float4 w4 = __ldg(reinterpret_cast<const float4*>(wr + h));
+                const int src = qi * C::HI + h;
+                const float w0 = __shfl_sync(0xffffffffu, wv[cc], src + 0);
+                const float w1 = __shfl_sync(0xffffffffu, wv[cc], src + 1);
+                const float w2 = __shfl_sync(0xffffffffu, wv[cc], src + 2);
+                const float w3 = __shfl_sync(0xffffffffu, wv[cc], src + 3);
                 float d0 = __uint_as_float(r[qi * C::HI + h + 0]);
                 float d1 = __uint_as_float(r[qi * C::HI + h + 1]);
                 float d2 = __uint_as_float(r[qi * C::HI + h + 2]);
@@ -279,10 +297,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 if (RELU == 2) {
                   d0 = fmaxf(d0, 0.f); d1 = fmaxf(d1, 0.f); d2 = fmaxf(d2, 0.f); d3 = fmaxf(d3, 0.f);
                 }
-                acc4[0] = fmaf(w4.x, d0, acc4[0]);
-                acc4[1] = fmaf(w4.y, d1, acc4[1]);
-                acc4[2] = fmaf(w4.z, d2, acc4[2]);
-                acc4[3] = fmaf(w4.w, d3, acc4[3]);
+                acc4[0] = fmaf(w0, d0, acc4[0]);
+                acc4[1] = fmaf(w1, d1, acc4[1]);
+                acc4[2] = fmaf(w2, d2, acc4[2]);
+                acc4[3] = fmaf(w3, d3, acc4[3]);
               }
               float v = ((acc4[0] + acc4[1]) + (acc4[2] + acc4[3])) * a.scale;
               if (RELU == 1) v = fmaxf(v, 0.f);
