@@ -225,30 +225,42 @@ __global__ void __launch_bounds__(544, HPW <= 2 ? 2 : 1) gather_attn_kernel(cons
   }
 }
 
-// Merge the split partials of one row: out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p.
+// Merge the split partials of one (row, head): out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p,
+// summed in split order (deterministic).  One CTA per (row, head): the per-split weights are
+// computed once into shared memory, then each thread combines one output element.
 template <typename T>
 __global__ void combine_kernel(const GatherArgs a) {
-  const int row = blockIdx.x;
-  for (int e = threadIdx.x; e < a.H * a.DV; e += blockDim.x) {
-    const int h = e / a.DV, d = e % a.DV;
+  __shared__ float wsplit[64];
+  __shared__ float inv_l;
+  const int row = blockIdx.x / a.H, h = blockIdx.x % a.H;
+  const size_t base0 = (size_t)row * a.nsplit * a.H + h;  // partial (row, split 0, h)
+  if (threadIdx.x < 32) {
     float M = -INFINITY;
-    for (int p = 0; p < a.nsplit; ++p)
-      M = fmaxf(M, a.part_ml[(((size_t)row * a.nsplit + p) * a.H + h) * 2]);
-    float L = 0.f, O = 0.f;
-    if (M != -INFINITY) {
-      for (int p = 0; p < a.nsplit; ++p) {
-        const size_t base = ((size_t)row * a.nsplit + p) * a.H + h;
-        const float mp = a.part_ml[base * 2];
-        if (mp == -INFINITY) continue;
-        const float f = exp2f(mp - M);
-        L = fmaf(a.part_ml[base * 2 + 1], f, L);
-        O = fmaf(a.part_o[base * a.DV + d], f, O);
-      }
+    for (int p = threadIdx.x; p < a.nsplit; p += 32)
+      M = fmaxf(M, a.part_ml[(base0 + (size_t)p * a.H) * 2]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    for (int p = threadIdx.x; p < a.nsplit; p += 32) {
+      const float mp = a.part_ml[(base0 + (size_t)p * a.H) * 2];
+      wsplit[p] = (M == -INFINITY || mp == -INFINITY) ? 0.f : exp2f(mp - M);
     }
-    float r = L > 0.f ? O / L : 0.f;
-    if (a.gate)
-      r *= gate_act(to_f32(static_cast<const T*>(a.gate)[(size_t)row * a.H + h]), a.gate_mode);
-    static_cast<T*>(a.out)[((size_t)row * a.H + h) * a.DV + d] = from_f32<T>(r);
+    __syncwarp();
+    if (threadIdx.x == 0) {
+      float L = 0.f;
+      for (int p = 0; p < a.nsplit; ++p)
+        L = fmaf(a.part_ml[(base0 + (size_t)p * a.H) * 2 + 1], wsplit[p], L);
+      float f = L > 0.f ? 1.0f / L : 0.f;
+      if (a.gate)
+        f *= gate_act(to_f32(static_cast<const T*>(a.gate)[(size_t)row * a.H + h]), a.gate_mode);
+      inv_l = f;
+    }
+  }
+  __syncthreads();
+  for (int d = threadIdx.x; d < a.DV; d += blockDim.x) {
+    float O = 0.f;
+    for (int p = 0; p < a.nsplit; ++p)
+      O = fmaf(a.part_o[(base0 + (size_t)p * a.H) * a.DV + d], wsplit[p], O);
+    static_cast<T*>(a.out)[((size_t)row * a.H + h) * a.DV + d] = from_f32<T>(O * inv_l);
   }
 }
 
@@ -263,8 +275,8 @@ int heads_per_warp(int H) {
 // Split policy: few query rows and long key lists -> spread the keys over CTAs.  The split
 // count is chosen so that rows * nsplit fills whole waves of the resident CTAs (two per SM
 // on a 148-SM B200) as closely as possible, with at least 64 keys per split and at most 32
-// splits; the fewest splits within 5% of full waves win.  Depends on the shape only (no device query), so
-// workspace sizes are reproducible.
+// splits; the fewest splits within 5% of full waves win.  Depends on the shape only (no
+// device query), so workspace sizes are reproducible.
 void split_policy(int rows, int nkeys, int* nsplit, int* kps, bool allow_split = true) {
   const int resident = 2 * 148;
   if (!allow_split || rows >= resident || nkeys <= 128) {
@@ -306,7 +318,7 @@ cudaError_t launch_t(GatherArgs a, int nw, size_t smem, unsigned grid, int rows,
   kern<<<grid, 32 * (nw + 1), smem, st>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess || a.nsplit == 1) return e;
-  combine_kernel<T><<<rows, 256, 0, st>>>(a);
+  combine_kernel<T><<<(unsigned)rows * a.H, 128, 0, st>>>(a);
   return cudaGetLastError();
 }
 

@@ -441,15 +441,15 @@ cudaError_t launch_index_scores_tc(const void* q_idx, const void* k_idx, const f
                                               scores, write_masked, st);
   }
   if (HI == 32 && DI == 128)
-    return launch_cfg<TcCfg<32, 128, 8, 8, 3>>(q_idx, k_idx, w, scale, relu, B, S, T, q_off,
+    return launch_cfg<TcCfg<32, 128, 8, 16, 3>>(q_idx, k_idx, w, scale, relu, B, S, T, q_off,
                                                scores, write_masked, st);
   if (HI == 32 && DI == 64)
-    return launch_cfg<TcCfg<32, 64, 8, 8, 4>>(q_idx, k_idx, w, scale, relu, B, S, T, q_off,
+    return launch_cfg<TcCfg<32, 64, 8, 16, 4>>(q_idx, k_idx, w, scale, relu, B, S, T, q_off,
                                               scores, write_masked, st);
   if (HI == 16 && DI == 128)
-    return launch_cfg<TcCfg<16, 128, 16, 8, 3>>(q_idx, k_idx, w, scale, relu, B, S, T, q_off,
+    return launch_cfg<TcCfg<16, 128, 16, 16, 3>>(q_idx, k_idx, w, scale, relu, B, S, T, q_off,
                                                 scores, write_masked, st);
-  return launch_cfg<TcCfg<16, 64, 16, 8, 4>>(q_idx, k_idx, w, scale, relu, B, S, T, q_off,
+  return launch_cfg<TcCfg<16, 64, 16, 16, 4>>(q_idx, k_idx, w, scale, relu, B, S, T, q_off,
                                              scores, write_masked, st);
 }
 
