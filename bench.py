@@ -39,7 +39,10 @@ F32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 # DRAM traffic per launch from committed ncu captures: (kernel, config) -> (bytes,
 # sha256 of the kernel source when captured).  Reported as null when the source changed.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # masked_attn_tc_kernel, c2 full size: 64.31 MB read + 4.31 MB written
+    ("masked_attn", "c2"): (68619008, "ceb7f3c10dd75398"),
+}
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -157,18 +160,20 @@ def job_value(units_per_rank, world, step_ms_max):
 class Workload:
     """Device buffers and the library calls of one step of config `name`."""
 
-    def __init__(self, name, device, seed_offset=0, S=None, T=None):
+    def __init__(self, name, device, seed_offset=0, S=None, T=None, B=None):
         import dataclasses
 
         import sparse_attention_15_b200 as dsa
 
         self.dsa = dsa
         cfg = get_config(name)
-        if S is not None or T is not None:  # a reduced case of the same workload (profiling)
+        if S is not None or T is not None or B is not None:  # a reduced case (profiling)
             S = cfg.S if S is None else S
             T = cfg.T if T is None else T
-            cfg = dataclasses.replace(cfg, S=S, T=T,
-                                      description=f"{cfg.description} [reduced: S={S}, T={T}]")
+            B = cfg.B if B is None else B
+            cfg = dataclasses.replace(
+                cfg, S=S, T=T, B=B,
+                description=f"{cfg.description} [reduced: B={B}, S={S}, T={T}]")
         self.cfg = cfg
         self.device = device
         B = cfg.B
@@ -378,6 +383,7 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
     ap.add_argument("--S", type=int, default=None, help="reduced query count (profiling cases)")
     ap.add_argument("--T", type=int, default=None, help="reduced key count (profiling cases)")
+    ap.add_argument("--B", type=int, default=None, help="reduced batch (profiling cases)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world, rank, local = dist_setup(args)
@@ -401,7 +407,7 @@ def main():
                                 device_id=dev)
         pg = dist
 
-    wl = Workload(args.config, dev, seed_offset=rank, S=args.S, T=args.T)
+    wl = Workload(args.config, dev, seed_offset=rank, S=args.S, T=args.T, B=args.B)
     cfg = wl.cfg
     nst = len(wl.stages)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)

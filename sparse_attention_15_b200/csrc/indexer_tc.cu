@@ -21,7 +21,9 @@
 //   warp 1       MMA issuer (one thread): DI/16 tcgen05.mma per tile into one of two TMEM
 //                accumulators; tcgen05.commit frees the key stage and hands the
 //                accumulator to the epilogue
-//   warps 4..    epilogue: tcgen05.ld of the accumulator, weighted head sum, store
+//   warps 2..    epilogue (a multiple of 4 warps, so that each TMEM lane quadrant -- warp % 4 --
+//                has the same number of warps): tcgen05.ld of the accumulator, weighted
+//                head sum, store
 // A work unit is (batch row, query block, a chunk of key tiles up to the causal limit);
 // units are dealt to CTAs round-robin.  Key tiles after the last causal tile of a query
 // block are not computed: a separate fill kernel writes their -inf when asked to.
@@ -37,7 +39,7 @@ namespace dsa {
 namespace {
 
 constexpr int kTileM = 128;   // keys per tile = TMEM lanes
-constexpr int kEpiWarp0 = 4;  // first epilogue warp (warp % 4 = its TMEM lane quadrant)
+constexpr int kEpiWarp0 = 2;  // first epilogue warp (warp % 4 = its TMEM lane quadrant)
 
 struct TcArgs {
   const float* w;
@@ -69,7 +71,7 @@ struct TcCfg {
   static constexpr int SMEM = NA * A_BYTES + NB * B_BYTES + BAR_BYTES + 1024;
   static_assert(N % 16 == 0 && N >= 16 && N <= 256, "UMMA N");
   static_assert(HI <= 32 && 32 % HI == 0, "heads per 32-column chunk");
-  static_assert(COLS_PER_WARP % 32 == 0, "epilogue chunking");
+  static_assert(COLS_PER_WARP % 32 == 0 && COLS_PER_WARP % HI == 0, "epilogue chunking");
   static_assert(DI % 64 == 0, "DI must be a multiple of 64");
 };
 
@@ -246,30 +248,27 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     bool ok = true;
     while (ok && it.next(a, C::NQ, ncta)) {
       const int s_base = it.qb * C::NQ;
-      // the head weights of this unit's queries are the same for every key tile: lane l
-      // keeps the weight of column col0 + 32cc + l of each chunk cc, and the reduction
-      // below broadcasts it with a shuffle (no memory access inside the tile loop)
-      float wv[C::COLS_PER_WARP / 32];
-#pragma unroll
-      for (int cc = 0; cc < C::COLS_PER_WARP / 32; ++cc) {
-        const int col = col0 + cc * 32 + lane;
-        const int s = s_base + col / C::HI;
-        wv[cc] = s < a.S ? __ldg(a.w + ((size_t)it.b * a.S + s) * C::HI + col % C::HI) : 0.f;
-      }
+      // the head weights of this unit's queries (1-2 KB) are the same for every key tile and
+      // every lane: the reduction reads them as warp-wide broadcast float4 loads, which stay
+      // in L1 for the whole unit (one load per four heads, no shuffles)
+      const float4* wunit = reinterpret_cast<const float4*>(
+          a.w + ((size_t)it.b * a.S + s_base) * C::HI);
       for (int kt = it.k0; kt < it.k1; ++kt) {
         const int ab = ci & 1;
         if (!warp_wait(&acc_full[ab], (ci >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
         const int t = kt * kTileM + quad * 32 + lane;
-        constexpr int NCH = C::COLS_PER_WARP / 32;
-        // double-buffered TMEM reads: chunk cc+1 is in flight while chunk cc is reduced
-        uint32_t rb[2][32];
-        tmem_ld32(t_lane + ab * C::ACC_COLS + col0, rb[0]);
+        constexpr int NCH = C::COLS_PER_WARP / 16;
+        // double-buffered 16-column TMEM reads: chunk cc+1 is in flight while chunk cc is
+        // reduced.  A query's HI columns span HI/16 chunks; its four FMA chains carry over.
+        uint32_t rb[2][16];
+        tmem_ld16(t_lane + ab * C::ACC_COLS + col0, rb[0]);
         tmem_wait_ld();
+        float acc4[4] = {0.f, 0.f, 0.f, 0.f};  // four independent FMA chains
 #pragma unroll
         for (int cc = 0; cc < NCH; ++cc) {
           if (cc + 1 < NCH) {
-            tmem_ld32(t_lane + ab * C::ACC_COLS + col0 + (cc + 1) * 32, rb[(cc + 1) & 1]);
+            tmem_ld16(t_lane + ab * C::ACC_COLS + col0 + (cc + 1) * 16, rb[(cc + 1) & 1]);
           } else {
             // every column of this accumulator has been read: hand it back to the MMA
             tc_fence_before();
@@ -277,35 +276,31 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             if (lane == 0) mbar_arrive(&acc_empty[ab]);
           }
           const uint32_t* r = rb[cc & 1];
+          const int c0 = col0 + cc * 16;     // first column of the chunk
+          const int j = c0 / C::HI;          // query within the block
+          const int s = s_base + j;
+          if (s < a.S) {  // ragged tail of the last block (warp-uniform)
 #pragma unroll
-          for (int qi = 0; qi < 32 / C::HI; ++qi) {
-            const int j = (col0 + cc * 32) / C::HI + qi;  // query within the block
-            const int s = s_base + j;
-            if (s < a.S) {  // ragged tail of the last block (warp-uniform)
-              float acc4[4] = {0.f, 0.f, 0.f, 0.f};  // four independent FMA chains
-#pragma unroll
-              for (int h = 0; h < C::HI; h += 4) {
-                const int src = qi * C::HI + h;
-                const float w0 = __shfl_sync(0xffffffffu, wv[cc], src + 0);
-                const float w1 = __shfl_sync(0xffffffffu, wv[cc], src + 1);
-                const float w2 = __shfl_sync(0xffffffffu, wv[cc], src + 2);
-                const float w3 = __shfl_sync(0xffffffffu, wv[cc], src + 3);
-                float d0 = __uint_as_float(r[qi * C::HI + h + 0]);
-                float d1 = __uint_as_float(r[qi * C::HI + h + 1]);
-                float d2 = __uint_as_float(r[qi * C::HI + h + 2]);
-                float d3 = __uint_as_float(r[qi * C::HI + h + 3]);
-                if (RELU == 2) {
-                  d0 = fmaxf(d0, 0.f); d1 = fmaxf(d1, 0.f); d2 = fmaxf(d2, 0.f); d3 = fmaxf(d3, 0.f);
-                }
-                acc4[0] = fmaf(w0, d0, acc4[0]);
-                acc4[1] = fmaf(w1, d1, acc4[1]);
-                acc4[2] = fmaf(w2, d2, acc4[2]);
-                acc4[3] = fmaf(w3, d3, acc4[3]);
+            for (int h = 0; h < 16; h += 4) {
+              const float4 w4 = __ldg(wunit + (c0 + h) / 4);
+              float d0 = __uint_as_float(r[h + 0]);
+              float d1 = __uint_as_float(r[h + 1]);
+              float d2 = __uint_as_float(r[h + 2]);
+              float d3 = __uint_as_float(r[h + 3]);
+              if (RELU == 2) {
+                d0 = fmaxf(d0, 0.f); d1 = fmaxf(d1, 0.f); d2 = fmaxf(d2, 0.f); d3 = fmaxf(d3, 0.f);
               }
+              acc4[0] = fmaf(w4.x, d0, acc4[0]);
+              acc4[1] = fmaf(w4.y, d1, acc4[1]);
+              acc4[2] = fmaf(w4.z, d2, acc4[2]);
+              acc4[3] = fmaf(w4.w, d3, acc4[3]);
+            }
+            if ((c0 + 16) % C::HI == 0) {  // the query's last chunk: finish and store
               float v = ((acc4[0] + acc4[1]) + (acc4[2] + acc4[3])) * a.scale;
               if (RELU == 1) v = fmaxf(v, 0.f);
               if (t < a.T)
                 a.scores[((size_t)it.b * a.S + s) * a.T + t] = (t <= s + a.q_off) ? v : ninf;
+              acc4[0] = acc4[1] = acc4[2] = acc4[3] = 0.f;
             }
           }
           if (cc + 1 < NCH) tmem_wait_ld();

@@ -12,11 +12,9 @@
 //
 // One CTA per query row.  Pass 1 reads the row from HBM; the later passes re-read it from
 // L2 (a row is at most a few hundred KB and was just touched).  Histograms are built with
-// warp-aggregated shared-memory atomics (__match_any_sync groups equal digits, one atomic
-// per distinct digit per warp): integer-valued scores repeat heavily, so plain atomics
-// would serialise.  The compaction is a block-wide ballot/popc scan in index order, so the
-// output is deterministic and needs no sort.  The same ballots give the selection bitmask
-// (one bit per key) for the masked-tile attention path.
+// shared-memory atomics.  The compaction is a block-wide ballot/popc scan in index order, so
+// the output is deterministic and needs no sort.  The same ballots give the selection
+// bitmask (one bit per key) for the masked-tile attention path.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -56,9 +54,27 @@ __device__ __forceinline__ int block_excl_scan(int v, int* warp_buf, int* total)
     if (lane == 31) *total = ws;
   }
   __syncthreads();
-  int r = warp_buf[warp] + x - v;
-  __syncthreads();  // warp_buf may be reused right after
-  return r;
+  // callers pass a barrier before the next scan rewrites warp_buf
+  return warp_buf[warp] + x - v;
+}
+
+// Histogram bins are stored with one padding word per 32 bins, so that the contiguous runs
+// of 1..16 bins each thread scans in find_bucket start in distinct banks.
+constexpr int padded(int nbins) { return nbins + nbins / 32; }
+__device__ __forceinline__ uint32_t hpad(uint32_t b) { return b + (b >> 5); }
+
+template <int NT>
+__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t digit, bool valid) {
+  // Plain shared-memory atomics: equal digits within a warp serialise in the atomic unit,
+  // which costs less than grouping them first (__match_any_sync occupies the XU pipe for
+  // many cycles per call).  A warp whose 32 digits are all equal adds once.
+  const uint32_t d = valid ? digit : 0xffffffffu;
+  const uint32_t d0 = __shfl_sync(0xffffffffu, d, 0);
+  if (__all_sync(0xffffffffu, d == d0)) {
+    if ((threadIdx.x & 31) == 0 && valid) atomicAdd(&hist[hpad(d)], 32u);
+  } else if (valid) {
+    atomicAdd(&hist[hpad(d)], 1u);
+  }
 }
 
 template <int NT>
@@ -67,7 +83,7 @@ __global__ void __launch_bounds__(NT) topk_rows_kernel(const float* __restrict__
                                                        int32_t* __restrict__ idx,
                                                        uint32_t* __restrict__ mask,
                                                        int mask_stride) {
-  __shared__ uint32_t hist[kBins];
+  __shared__ uint32_t hist[padded(kBins)];
   __shared__ int warp_buf[32];
   __shared__ int scan_total;
   __shared__ uint32_t sel_bin;
@@ -102,7 +118,7 @@ __global__ void __launch_bounds__(NT) topk_rows_kernel(const float* __restrict__
   for (int pass = 0; pass < 3; ++pass) {
     const int dw = widths[pass];
     const int shift = 32 - pbits - dw;
-    for (int i = tid; i < kBins; i += NT) hist[i] = 0;
+    for (int i = tid; i < padded(kBins); i += NT) hist[i] = 0;
     __syncthreads();
     for (int i0 = 0; i0 < n; i0 += NT) {
       const int i = i0 + tid;
@@ -112,9 +128,7 @@ __global__ void __launch_bounds__(NT) topk_rows_kernel(const float* __restrict__
         bool match = pbits == 0 || (key >> (32 - pbits)) == prefix;
         if (match) digit = (key >> shift) & ((1u << dw) - 1u);
       }
-      uint32_t peers = __match_any_sync(0xffffffffu, digit);
-      if (digit != 0xffffffffu && lane == __ffs(peers) - 1)
-        atomicAdd(&hist[digit], (uint32_t)__popc(peers));
+      hist_add<NT>(hist, digit, digit != 0xffffffffu);
     }
     __syncthreads();
     // bins from the top: thread j owns a contiguous run of bins, highest first
@@ -122,11 +136,11 @@ __global__ void __launch_bounds__(NT) topk_rows_kernel(const float* __restrict__
     const int hi_bin = kBins - tid * kPer;  // exclusive upper end of my run
     int local = 0;
 #pragma unroll
-    for (int q = 1; q <= kPer; ++q) local += (int)hist[hi_bin - q];
+    for (int q = 1; q <= kPer; ++q) local += (int)hist[hpad(hi_bin - q)];
     int above = block_excl_scan(local, warp_buf, &scan_total);
 #pragma unroll
     for (int q = 1; q <= kPer; ++q) {
-      int c = (int)hist[hi_bin - q];
+      int c = (int)hist[hpad(hi_bin - q)];
       if (above < need && above + c >= need) {
         sel_bin = (uint32_t)(hi_bin - q);
         sel_above = above;
@@ -138,7 +152,7 @@ __global__ void __launch_bounds__(NT) topk_rows_kernel(const float* __restrict__
     need -= sel_above;
     prefix = (prefix << dw) | bsel;
     pbits += dw;
-    const bool all_taken = (int)hist[bsel] == need;
+    const bool all_taken = (int)hist[hpad(bsel)] == need;
     __syncthreads();
     if (all_taken) break;  // every key in the bucket is kept: no need to refine further
   }
@@ -192,61 +206,103 @@ __global__ void __launch_bounds__(NT) topk_rows_kernel(const float* __restrict__
 // ------------------------------------------------------------------------------------
 // Two-read top-k with shared-memory bitmaps (rows up to kMaxBitmapKeys keys).
 //
-// Read 1 (HBM, float4 loads, 16 keys per thread in flight): histogram of the top 12 bits of
-// the order key -> bucket b1 holding the K-th key, `need` = keys of b1 still to take.
-// Read 2 (L2): keys in buckets above b1 go to the SELECTED bitmap, keys of b1 to the
-// CANDIDATE bitmap (bits assembled across lanes with shuffles, no atomics).  The low 20
-// bits are then resolved by two 10-bit histogram passes over the candidates only (a few
-// hundred scattered L2 reads), giving the exact threshold key tau.  Candidates above tau
-// join SELECTED; candidates equal to tau are ranked by index with a prefix scan of their
-// bitmap and the first `need` join SELECTED.  An ordered scan of SELECTED writes the indices
-// (ascending) and the bitmap itself is the selection mask row.
+// Read 1 (HBM) finds a window of 12-bit buckets (top bits of the order key) that holds the
+// K-th key.  Long rows (8192 keys and more) histogram every 8th key and take the buckets
+// around the sample's K-th rank (a 3-sigma rank margin); short rows histogram every key and
+// the window is the exact bucket b1.  Read 2 (L2, or the registers when the whole row fit in
+// read 1's batch of loads): keys above the window go to the SELECTED bitmap, keys inside it
+// to the CANDIDATE bitmap (bits assembled across lanes with shuffles) and to a shared-memory
+// candidate list of (key, position).  On long rows an exact 12-bit histogram of the
+// candidates alone then gives b1; if the sampled window missed the K-th key, read 1 is
+// redone exactly.  Either way b1 and `need` (keys of b1 still to take) are exact.  The low
+// 20 bits are resolved by two 10-bit histogram passes over the candidate list (in shared
+// memory; only a list that overflowed is re-read from L2 through the bitmap), giving the
+// exact threshold key tau.  Candidates above tau join SELECTED; candidates equal to tau are
+// ranked by index with a prefix scan of their bitmap and the first `need` join SELECTED.
+// An ordered scan of SELECTED writes the indices (ascending) and the bitmap itself is the
+// selection mask row.
 // ------------------------------------------------------------------------------------
 constexpr int kMaxBitmapKeys = 1 << 20;
+constexpr size_t kMaxDynSmem = 220u * 1024u;  // leaves room for the static shared memory
 constexpr int kBins1 = 4096;  // top 12 bits
 constexpr int kBins2 = 1024;  // 10-bit refinement digits
 
-template <int NT>
-__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t digit, bool valid) {
-  const uint32_t d = valid ? digit : 0xffffffffu;
-  const uint32_t peers = __match_any_sync(0xffffffffu, d);
-  if (valid && (threadIdx.x & 31) == (uint32_t)(__ffs(peers) - 1))
-    atomicAdd(&hist[d], (uint32_t)__popc(peers));
-}
-
-// Bucket holding the need-th largest key: writes (bin, count above it) to out[0..1].
+// Bucket holding the need-th largest key: writes (bin, count above it, its count) to
+// out[0..2].
 template <int NT>
 __device__ __forceinline__ void find_bucket(const uint32_t* hist, int nbins, int need,
                                             int* warp_buf, int* scan_total, int* out) {
   const int per = nbins / NT;
   const int hi_bin = nbins - threadIdx.x * per;
   int local = 0;
-  for (int q = 1; q <= per; ++q) local += (int)hist[hi_bin - q];
+  for (int q = 1; q <= per; ++q) local += (int)hist[hpad(hi_bin - q)];
   int above = block_excl_scan(local, warp_buf, scan_total);
   for (int q = 1; q <= per; ++q) {
-    const int c = (int)hist[hi_bin - q];
+    const int c = (int)hist[hpad(hi_bin - q)];
     if (above < need && above + c >= need) {
       out[0] = hi_bin - q;
       out[1] = above;
+      out[2] = c;
     }
     above += c;
   }
 }
 
-template <int NT>
-__global__ void __launch_bounds__(NT) topk_bitmap_kernel(const float* __restrict__ scores, int S,
-                                                         int Tn, int K, int q_off,
-                                                         int32_t* __restrict__ idx,
-                                                         uint32_t* __restrict__ mask,
-                                                         int mask_stride) {
+// Reserves c consecutive slots per lane in a shared list; returns this lane's first slot.
+__device__ __forceinline__ int warp_reserve(int c, int* counter) {
+  const int lane = threadIdx.x & 31;
+  int x = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  int base = 0;
+  if (lane == 31 && x > 0) base = atomicAdd(counter, x);
+  base = __shfl_sync(0xffffffffu, base, 31);
+  return base + x - c;
+}
+
+// U chunks of 4 scores as order keys: chunk u of this thread covers keys
+// base + (u*NT + tid)*4 + 0..3.  Keys at or past n are loaded as 0.0 (callers mask them).
+template <int NT, int U>
+__device__ __forceinline__ void load_keys(const float* __restrict__ sc, int n, int base,
+                                          bool vec, uint32_t (&k)[U][4]) {
+  float v[U][4];
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int i = base + (u * NT + (int)threadIdx.x) * 4;
+    if (vec && i + 3 < n) {
+      const float4 f = __ldg(reinterpret_cast<const float4*>(sc + i));
+      v[u][0] = f.x; v[u][1] = f.y; v[u][2] = f.z; v[u][3] = f.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) v[u][e] = (i + e < n) ? __ldg(sc + i + e) : 0.f;
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < U; ++u)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) k[u][e] = order_key(v[u][e]);
+}
+
+// Register caps keep 5 (256-thread) or 3 (512-thread) rows in flight per SM.
+template <int NT, bool SAMPLE>
+__global__ void __launch_bounds__(NT, NT == 256 ? 5 : (NT == 512 ? 3 : 1))
+    topk_bitmap_kernel(const float* __restrict__ scores, int S, int Tn, int K, int q_off,
+                       int32_t* __restrict__ idx, uint32_t* __restrict__ mask, int mask_stride,
+                       int cl_cap) {
   extern __shared__ uint32_t dsm[];
   const int W = (Tn + 31) >> 5;              // bitmap words per row
-  uint32_t* hist = dsm;                      // [kBins1]
-  uint32_t* selb = hist + kBins1;            // [W]
+  uint32_t* hist = dsm;                      // [padded(kBins1)]
+  uint32_t* selb = hist + padded(kBins1);    // [W]
   uint32_t* candb = selb + W;                // [W]
+  uint32_t* cl_key = candb + W;              // [cl_cap] candidate keys
+  uint32_t* cl_idx = cl_key + cl_cap;        // [cl_cap] candidate positions
   __shared__ int warp_buf[32];
   __shared__ int scan_total;
-  __shared__ int pick[2];
+  __shared__ int pick[3];
+  __shared__ int cnt_sel, cl_n;
 
   const size_t row = blockIdx.x;
   const int s = (int)(row % (size_t)S);
@@ -267,75 +323,166 @@ __global__ void __launch_bounds__(NT) topk_bitmap_kernel(const float* __restrict
     return;
   }
 
-  for (int i = tid; i < kBins1; i += NT) hist[i] = 0u;
-  for (int i = tid; i < W; i += NT) { selb[i] = 0u; candb[i] = 0u; }
+  for (int i = tid; i < padded(kBins1); i += NT) hist[i] = 0u;
+  if (tid == 0) { cnt_sel = 0; cl_n = 0; }
   __syncthreads();
 
-  // ---------------- read 1: 12-bit histogram, 16 keys per thread in flight
+  constexpr int U = (SAMPLE && NT == 512) ? 2 : 4;  // float4 loads in flight per thread
+  constexpr int kChunk = NT * 4 * U;  // keys per batch of loads
   const bool vec = ((Tn & 3) == 0);
-  constexpr int U = 4;
-  for (int base = 0; base < n; base += NT * 4 * U) {
-    float v[U][4];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int i = base + (u * NT + tid) * 4;
-      if (vec && i + 3 < n) {
-        const float4 f = __ldg(reinterpret_cast<const float4*>(sc + i));
-        v[u][0] = f.x; v[u][1] = f.y; v[u][2] = f.z; v[u][3] = f.w;
-      } else {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) v[u][e] = (i + e < n) ? __ldg(sc + i + e) : 0.f;
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int i = base + (u * NT + tid) * 4;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) hist_add<NT>(hist, order_key(v[u][e]) >> 20, i + e < n);
-    }
-  }
-  __syncthreads();
-  find_bucket<NT>(hist, kBins1, K, warp_buf, &scan_total, pick);
-  __syncthreads();
-  const uint32_t b1 = (uint32_t)pick[0];
-  int need = K - pick[1];
-  const int cnt1 = (int)hist[b1];
+  uint32_t kh[U][4];  // the current batch of keys; the whole row when n <= kChunk
+  bool held = false;
+  uint32_t b1 = 0;
+  int need = K, cnt1 = 0;
 
-  // ---------------- read 2: SELECTED (above b1) and CANDIDATE (== b1) bitmaps
-  for (int base = 0; base < n; base += NT * 4) {
-    const int i = base + tid * 4;
-    float v[4];
-    if (vec && i + 3 < n) {
-      const float4 f = __ldg(reinterpret_cast<const float4*>(sc + i));
-      v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
-    } else {
+  // Exact read 1: 12-bit histogram of every key -> bucket b1 of the K-th key, `need`.
+  auto exact_read1 = [&]() {
+    for (int base = 0; base < n; base += kChunk) {
+      load_keys<NT, U>(sc, n, base, vec, kh);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) v[e] = (i + e < n) ? __ldg(sc + i + e) : 0.f;
-    }
-    uint32_t gt = 0u, eq = 0u;
+      for (int u = 0; u < U; ++u) {
+        const int i = base + (u * NT + tid) * 4;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      if (i + e < n) {
-        const uint32_t d = order_key(v[e]) >> 20;
-        gt |= (d > b1 ? 1u : 0u) << e;
-        eq |= (d == b1 ? 1u : 0u) << e;
+        for (int e = 0; e < 4; ++e) hist_add<NT>(hist, kh[u][e] >> 20, i + e < n);
       }
     }
-    // lanes 8m..8m+7 cover one 32-key word: OR their nibbles together
-    const int sh = 4 * (lane & 7);
-    uint32_t wg = gt << sh, we = eq << sh;
+    held = n <= kChunk;
+    __syncthreads();
+    find_bucket<NT>(hist, kBins1, K, warp_buf, &scan_total, pick);
+    __syncthreads();
+    b1 = (uint32_t)pick[0];
+    need = K - pick[1];
+    cnt1 = pick[2];
+  };
+
+  // Read 2: keys whose bucket is above [lo, hi] -> SELECTED bitmap; inside it -> CANDIDATE
+  // bitmap and the candidate list (key, position) while it has room.  Counts both.
+  auto read2 = [&](uint32_t lo, uint32_t hi) {
+    int my_sel = 0;
+    for (int base = 0; base < n; base += kChunk) {
+      if (!held) load_keys<NT, U>(sc, n, base, vec, kh);
+      uint32_t gt[U], in[U];
+      int c = 0;
 #pragma unroll
-    for (int o = 1; o < 8; o <<= 1) {
-      wg |= __shfl_xor_sync(0xffffffffu, wg, o);
-      we |= __shfl_xor_sync(0xffffffffu, we, o);
+      for (int u = 0; u < U; ++u) {
+        const int i = base + (u * NT + tid) * 4;
+        gt[u] = 0u;
+        in[u] = 0u;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if (i + e < n) {
+            const uint32_t d = kh[u][e] >> 20;
+            gt[u] |= (d > hi ? 1u : 0u) << e;
+            in[u] |= (d >= lo && d <= hi ? 1u : 0u) << e;
+          }
+        }
+        my_sel += __popc(gt[u]);
+        c += __popc(in[u]);
+        // lanes 8m..8m+7 cover one 32-key word: OR their nibbles together
+        const int sh = 4 * (lane & 7);
+        uint32_t wg = gt[u] << sh, we = in[u] << sh;
+#pragma unroll
+        for (int o = 1; o < 8; o <<= 1) {
+          wg |= __shfl_xor_sync(0xffffffffu, wg, o);
+          we |= __shfl_xor_sync(0xffffffffu, we, o);
+        }
+        if ((lane & 7) == 0 && i < n) {
+          selb[i >> 5] = wg;
+          candb[i >> 5] = we;
+        }
+      }
+      int pos = warp_reserve(c, &cl_n);
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if ((in[u] >> e) & 1u) {
+            if (pos < cl_cap) {
+              cl_key[pos] = kh[u][e];
+              cl_idx[pos] = (uint32_t)(base + (u * NT + tid) * 4 + e);
+            }
+            ++pos;
+          }
     }
-    const int wd = (i >> 5);
-    if ((lane & 7) == 0 && i < n) {
-      selb[wd] = wg;
-      candb[wd] = we;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) my_sel += __shfl_xor_sync(0xffffffffu, my_sel, o);
+    if (lane == 0 && my_sel) atomicAdd(&cnt_sel, my_sel);
+    __syncthreads();
+  };
+
+  if (SAMPLE && n >= 8192) {  // long rows only: on short rows the extra steps cost more
+    // ---------------- read 1 (sampled): 12-bit histogram of every 8th key -> a window of
+    // buckets that holds the K-th key with high probability (rank margin 3 sigma + 2)
+    const int ns = (n + 7) >> 3;
+    for (int m0 = 0; m0 < ns; m0 += NT * 4) {
+      float v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int m = m0 + u * NT + tid;
+        v[u] = m < ns ? __ldg(sc + 8 * m) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) hist_add<NT>(hist, order_key(v[u]) >> 20, m0 + u * NT + tid < ns);
     }
+    __syncthreads();
+    const float ks = (float)K * (float)ns / (float)n;
+    const int delta = (int)(3.0f * sqrtf(ks) + 2.0f);
+    const int r_hi = max(1, (int)ks - delta), r_lo = min(ns, (int)ks + delta + 1);
+    find_bucket<NT>(hist, kBins1, r_hi, warp_buf, &scan_total, pick);
+    __syncthreads();
+    const uint32_t b_hi = (uint32_t)pick[0];
+    find_bucket<NT>(hist, kBins1, r_lo, warp_buf, &scan_total, pick);
+    __syncthreads();
+    const uint32_t b_lo = (uint32_t)pick[0];
+    for (int i = tid; i < padded(kBins1); i += NT) hist[i] = 0u;
+    read2(b_lo, b_hi);  // ends with a barrier: the histogram is clear
+    const int nsel = cnt_sel, ncand = cl_n;
+    if (nsel < K && nsel + ncand >= K) {
+      // exact 12-bit histogram of the candidates only -> the bucket b1 of the K-th key
+      if (ncand <= cl_cap) {
+        for (int i0 = 0; i0 < ncand; i0 += NT) {
+          const int i = i0 + tid;
+          hist_add<NT>(hist, i < ncand ? cl_key[i] >> 20 : 0u, i < ncand);
+        }
+      } else {
+        for (int w0 = 0; w0 < nw; w0 += NT) {
+          const int wd = w0 + tid;
+          uint32_t bits = wd < nw ? candb[wd] : 0u;
+          bool more = __any_sync(0xffffffffu, bits != 0u);
+          while (more) {
+            uint32_t digit = 0u;
+            const bool has = bits != 0u;
+            if (has) {
+              const int j = __ffs(bits) - 1;
+              bits &= bits - 1u;
+              digit = order_key(__ldg(sc + wd * 32 + j)) >> 20;
+            }
+            hist_add<NT>(hist, digit, has);
+            more = __any_sync(0xffffffffu, bits != 0u);
+          }
+        }
+      }
+      __syncthreads();
+      find_bucket<NT>(hist, kBins1, K - nsel, warp_buf, &scan_total, pick);
+      __syncthreads();
+      b1 = (uint32_t)pick[0];
+      need = K - nsel - pick[1];
+      cnt1 = pick[2];
+    } else {
+      // the sample missed: exact read 1, then read 2 again with the window [b1, b1]
+      __syncthreads();  // every thread has read the counts before they are reset
+      for (int i = tid; i < padded(kBins1); i += NT) hist[i] = 0u;
+      if (tid == 0) { cnt_sel = 0; cl_n = 0; }
+      __syncthreads();
+      exact_read1();
+      read2(b1, b1);
+    }
+  } else {
+    exact_read1();
+    read2(b1, b1);
   }
-  __syncthreads();
+  const int ncl = cl_n;
+  const bool use_cl = ncl <= cl_cap;  // else the candidates are re-read through the bitmap
 
   // ---------------- refine the low 20 bits over the candidates only
   uint32_t prefix = b1;
@@ -343,28 +490,44 @@ __global__ void __launch_bounds__(NT) topk_bitmap_kernel(const float* __restrict
   if (cnt1 != need) {
     for (int pass = 0; pass < 2; ++pass) {
       const int shift = 20 - 10 * (pass + 1);
-      for (int i = tid; i < kBins2; i += NT) hist[i] = 0u;
+      for (int i = tid; i < padded(kBins2); i += NT) hist[i] = 0u;
       __syncthreads();
-      for (int w0 = 0; w0 < nw; w0 += NT) {
-        const int wd = w0 + tid;
-        uint32_t bits = wd < nw ? candb[wd] : 0u;
-        // every lane walks its word; the histogram add is warp-aggregated per step
-        bool more = __any_sync(0xffffffffu, bits != 0u);
-        while (more) {
-          const bool has = bits != 0u;
+      if (use_cl) {
+        for (int i0 = 0; i0 < ncl; i0 += NT) {
+          const int i = i0 + tid;
           uint32_t digit = 0u;
           bool valid = false;
-          if (has) {
-            const int j = __ffs(bits) - 1;
-            bits &= bits - 1u;
-            const uint32_t key = order_key(__ldg(sc + wd * 32 + j));
+          if (i < ncl) {
+            const uint32_t key = cl_key[i];
             if ((key >> (32 - pbits)) == prefix) {
               digit = (key >> shift) & (kBins2 - 1);
               valid = true;
             }
           }
           hist_add<NT>(hist, digit, valid);
-          more = __any_sync(0xffffffffu, bits != 0u);
+        }
+      } else {
+        for (int w0 = 0; w0 < nw; w0 += NT) {
+          const int wd = w0 + tid;
+          uint32_t bits = wd < nw ? candb[wd] : 0u;
+          // every lane walks its word; the histogram add is warp-aggregated per step
+          bool more = __any_sync(0xffffffffu, bits != 0u);
+          while (more) {
+            const bool has = bits != 0u;
+            uint32_t digit = 0u;
+            bool valid = false;
+            if (has) {
+              const int j = __ffs(bits) - 1;
+              bits &= bits - 1u;
+              const uint32_t key = order_key(__ldg(sc + wd * 32 + j));
+              if ((key >> (32 - pbits)) == prefix) {
+                digit = (key >> shift) & (kBins2 - 1);
+                valid = true;
+              }
+            }
+            hist_add<NT>(hist, digit, valid);
+            more = __any_sync(0xffffffffu, bits != 0u);
+          }
         }
       }
       __syncthreads();
@@ -374,25 +537,33 @@ __global__ void __launch_bounds__(NT) topk_bitmap_kernel(const float* __restrict
       need -= pick[1];
       prefix = (prefix << 10) | bsel;
       pbits += 10;
-      const bool done = (int)hist[bsel] == need;
-      __syncthreads();
-      if (done) break;
+      if (pick[2] == need) break;  // every key of the bucket is kept
     }
   }
 
   // ---------------- candidates: above the threshold -> SELECTED, at it -> ties (in candb)
   const int fshift = 32 - pbits;
-  for (int wd = tid; wd < nw; wd += NT) {
-    uint32_t bits = candb[wd], sel = 0u, tie = 0u;
-    while (bits) {
-      const int j = __ffs(bits) - 1;
-      bits &= bits - 1u;
-      const uint32_t hi = order_key(__ldg(sc + wd * 32 + j)) >> fshift;
-      if (hi > prefix) sel |= 1u << j;
-      else if (hi == prefix) tie |= 1u << j;
+  if (use_cl) {
+    for (int wd = tid; wd < nw; wd += NT) candb[wd] = 0u;
+    __syncthreads();
+    for (int i = tid; i < ncl; i += NT) {
+      const uint32_t hi = cl_key[i] >> fshift, t = cl_idx[i];
+      if (hi > prefix) atomicOr(&selb[t >> 5], 1u << (t & 31));
+      else if (hi == prefix) atomicOr(&candb[t >> 5], 1u << (t & 31));
     }
-    selb[wd] |= sel;
-    candb[wd] = tie;
+  } else {
+    for (int wd = tid; wd < nw; wd += NT) {
+      uint32_t bits = candb[wd], sel = 0u, tie = 0u;
+      while (bits) {
+        const int j = __ffs(bits) - 1;
+        bits &= bits - 1u;
+        const uint32_t hi = order_key(__ldg(sc + wd * 32 + j)) >> fshift;
+        if (hi > prefix) sel |= 1u << j;
+        else if (hi == prefix) tie |= 1u << j;
+      }
+      selb[wd] |= sel;
+      candb[wd] = tie;
+    }
   }
   __syncthreads();
   // ties ranked by index: the first `need` are kept.  Thread t owns words [t*per, t*per+per).
@@ -474,31 +645,35 @@ cudaError_t launch_topk(const float* scores, int B, int S, int T, int K, int q_o
   const size_t rows = (size_t)B * S;
   if (rows == 0) return cudaSuccess;
   if (mask && mask_stride < (T + 31) / 32) return cudaErrorInvalidValue;
-  if (T <= kMaxBitmapKeys) {
+  // Bitmap kernel while its shared memory fits: the 4096-bin histogram, two bitmaps of the
+  // row and a candidate list (1024 entries for short rows, 2048 for long ones, 512 when
+  // the bitmaps are large; the list overflowing only costs re-reads through the bitmap).
+  const int W = (T + 31) / 32;
+  int cap = T > 8192 ? 2048 : 1024;
+  auto smem_for = [&](int c) { return (size_t)(padded(kBins1) + 2 * W + 2 * c) * sizeof(uint32_t); };
+  if (smem_for(cap) > kMaxDynSmem) cap = 512;
+  if (T <= kMaxBitmapKeys && smem_for(cap) <= kMaxDynSmem) {
     // one CTA per row; small CTAs so that several rows are in flight per SM (each row is a
     // chain of dependent reads and block-wide scans)
-    const int W = (T + 31) / 32;
-    const size_t smem = (size_t)(kBins1 + 2 * W) * sizeof(uint32_t);
-    {  // dynamic + static shared memory may pass the 48 KB default
-      cudaError_t e = cudaFuncSetAttribute(topk_bitmap_kernel<512>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return e;
-      e = cudaFuncSetAttribute(topk_bitmap_kernel<256>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return e;
-      e = cudaFuncSetAttribute(topk_bitmap_kernel<1024>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return e;
+    const size_t smem = smem_for(cap);
+    // dynamic + static shared memory may pass the 48 KB default
+    auto setsmem = [&](const void* f) {
+      return cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    };
+    cudaError_t e;
+    if (rows < 296 && T > 8192) {  // few long rows (decode): the widest CTA per row
+      if ((e = setsmem((const void*)topk_bitmap_kernel<1024, true>)) != cudaSuccess) return e;
+      topk_bitmap_kernel<1024, true><<<(unsigned)rows, 1024, smem, st>>>(
+          scores, S, T, K, q_off, idx, mask, mask_stride, cap);
+    } else if (T > 8192) {
+      if ((e = setsmem((const void*)topk_bitmap_kernel<512, true>)) != cudaSuccess) return e;
+      topk_bitmap_kernel<512, true><<<(unsigned)rows, 512, smem, st>>>(
+          scores, S, T, K, q_off, idx, mask, mask_stride, cap);
+    } else {
+      if ((e = setsmem((const void*)topk_bitmap_kernel<256, false>)) != cudaSuccess) return e;
+      topk_bitmap_kernel<256, false><<<(unsigned)rows, 256, smem, st>>>(
+          scores, S, T, K, q_off, idx, mask, mask_stride, cap);
     }
-    if (rows < 296 && T > 8192)  // few long rows (decode): the widest CTA per row
-      topk_bitmap_kernel<1024><<<(unsigned)rows, 1024, smem, st>>>(scores, S, T, K, q_off, idx,
-                                                                    mask, mask_stride);
-    else if (T > 8192)
-      topk_bitmap_kernel<512><<<(unsigned)rows, 512, smem, st>>>(scores, S, T, K, q_off, idx,
-                                                                  mask, mask_stride);
-    else
-      topk_bitmap_kernel<256><<<(unsigned)rows, 256, smem, st>>>(scores, S, T, K, q_off, idx,
-                                                                  mask, mask_stride);
     return cudaGetLastError();
   }
   if (T >= 8192)

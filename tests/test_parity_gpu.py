@@ -83,7 +83,10 @@ def _adversarial_scores(kind, S, T, seed):
 
 @pytest.mark.parametrize("kind", ["all_equal", "signed_zeros", "few_values", "wide_range",
                                   "neg_inf_inside", "dup_floats"])
-@pytest.mark.parametrize("S,T,K", [(64, 64, 8), (40, 3000, 700), (6, 20000, 2048)])
+# (40, 3000): rows held in registers; (20, 6000): short rows read in two batches;
+# (300, 9000): many long rows (sampled first read, 512-thread CTAs); (6, 20000): few long rows
+@pytest.mark.parametrize("S,T,K", [(64, 64, 8), (40, 3000, 700), (20, 6000, 1000),
+                                   (300, 9000, 1000), (6, 20000, 2048)])
 def test_topk_exact_adversarial(kind, S, T, K):
     x = _adversarial_scores(kind, S, T, seed=S + T)
     got = dsa.dsa_topk(x.to(DEV), K)
