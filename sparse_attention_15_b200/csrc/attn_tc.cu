@@ -15,11 +15,12 @@
 // 128-byte swizzle, via 3-D tensor maps over (dim, head, token)), V block [128 x Dv]
 // (MN-major operand of the second product).  Tensor memory: S0, S1 (128 columns each,
 // double-buffered so S_{j+1} = Q K_{j+1}^T overlaps the softmax of block j), O (Dv columns);
-// P is split into bf16 P_hi + P_lo (two per 32-bit column, 64 columns each) that overwrite
-// their S buffer and feed O += P_hi V + P_lo V as tensor-memory A operands -- the low part
-// keeps the float32 probabilities' precision that a single bf16 P would lose.  The running max is only raised (and O, l
-// rescaled) when a row's block max exceeds it by more than 2^8, so exp2 arguments stay
-// <= 8 and rescales are rare.
+// P is split into bf16 P_hi + P_lo (two per 32-bit column): the 16 keys of each chunk write
+// P_hi into the first 8 of their own 16 S columns and P_lo into the next 8, which feed
+// O += P_hi V + P_lo V as tensor-memory A operands -- the low part keeps the float32
+// probabilities' precision that a single bf16 P would lose.  The running max is only raised
+// (and O, l rescaled) when a row's block max exceeds it by more than 2^8, so exp2 arguments
+// stay <= 8 and rescales are rare.
 //
 // Roles: warps 0..7 softmax and
 // epilogue in two groups that take alternate key blocks (thread = query row = TMEM lane),
@@ -102,6 +103,38 @@ __device__ __forceinline__ float ex2_ftz(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Packed float32 pair arithmetic (sm_100): one instruction for two lanes of work.
+__device__ __forceinline__ unsigned long long pack2(float x, float y) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(x), "f"(y));
+  return r;
+}
+__device__ __forceinline__ void unpack2(unsigned long long v, float& x, float& y) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(x), "=f"(y) : "l"(v));
+}
+__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b,
+                                                   unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ unsigned long long add2(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ unsigned long long sub2(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// max(a, b, c) in one instruction (sm_100)
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y,
@@ -300,12 +333,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           const uint32_t o_tmem = tmem + C::O_COL + (gg & 1) * C::DV;
 #pragma unroll
           for (int kk = 0; kk < kBlk / 16; ++kk) {
-            // keys 16kk..16kk+15: 8 packed columns of P_hi at 32*(kk/2) + 8*(kk%2), P_lo 16
-            // columns further; V rows 16kk..: 2 swizzle atoms of 8 rows
-            const uint32_t pc = 32 * (kk >> 1) + 8 * (kk & 1);
+            // keys 16kk..16kk+15: 8 packed columns of P_hi at 16kk, P_lo 8 columns further;
+            // V rows 16kk..: 2 swizzle atoms of 8 rows
+            const uint32_t pc = 16 * kk;
             const uint64_t vdesc = sw128_mnmajor_desc(v_base + kk * 2048, C::SLICE, 1024);
             umma_f16_ts(o_tmem, p_tmem + pc, vdesc, idesc_pv, (j >= 2 || kk > 0) ? 1u : 0u);
-            umma_f16_ts(o_tmem, p_tmem + pc + 16, vdesc, idesc_pv, 1u);
+            umma_f16_ts(o_tmem, p_tmem + pc + 8, vdesc, idesc_pv, 1u);
           }
           umma_commit(&v_empty[gg & 1]);
           umma_commit(&s_empty[gg & 1]);
@@ -377,11 +410,19 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           tmem_ld32(s_col + 64, *reinterpret_cast<uint32_t(*)[32]>(r + 64));
           tmem_ld32(s_col + 96, *reinterpret_cast<uint32_t(*)[32]>(r + 96));
           tmem_wait_ld();
+          float mx[4];  // four independent chains, two keys per three-input max
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
+          for (int c = 0; c < 4; ++c) {
+            mx[c] = ninf;
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (bits[c] & (1u << e)) mraw = fmaxf(mraw, __uint_as_float(r[c * 32 + e]));
+            for (int e = 0; e < 32; e += 2) {
+              const float x0 = (bits[c] & (1u << e)) ? __uint_as_float(r[c * 32 + e]) : ninf;
+              const float x1 =
+                  (bits[c] & (1u << (e + 1))) ? __uint_as_float(r[c * 32 + e + 1]) : ninf;
+              mx[c] = max3(mx[c], x0, x1);
+            }
+          }
+          mraw = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
         }
         const float mb = mraw * a.qk_scale;
         const bool need = mb > m_used + kRescaleLog2;
@@ -410,36 +451,58 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             m_used = m_new;
           }
         }
-        // pass 2, 32 keys at a time: P = exp2(scale*s - m) for selected keys, 0 otherwise,
-        // split into bf16 P_hi + P_lo (P_lo = bf16(p - P_hi) keeps ~2^-17 relative
-        // precision).  Chunk c's P_hi goes to its own columns [32c, 32c+16), P_lo to
-        // [32c+16, 32c+32): only columns already read are overwritten.
+        // pass 2: P = exp2(scale*s - m) for selected keys, 0 otherwise, split into bf16
+        // P_hi + P_lo (P_lo = bf16(p - P_hi) keeps ~2^-17 relative precision).
         const float msub = m_used == ninf ? 0.f : m_used;
-        float rs = 0.f;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tmem_ld32(s_col + c * 32, r);
-          tmem_wait_ld();
-          uint32_t ph[16], pl[16];
+        unsigned long long rs2 = pack2(0.f, 0.f);  // row sum, two partial sums
+        const unsigned long long scale2 = pack2(a.qk_scale, a.qk_scale);
+        const unsigned long long nm2 = pack2(-msub, -msub);
+        // 16 keys per chunk, double-buffered TMEM reads (chunk k+1 in flight while chunk k is
+        // exponentiated); chunk k's P_hi and P_lo overwrite its own 16 S columns
+        uint32_t ra[16], rc[16];
+        uint32_t b0 = bits[0], b1 = bits[1], b2 = bits[2], b3 = bits[3];
+        auto chunk = [&](const uint32_t (&r)[16], uint32_t bw, int kk) {
+          uint32_t ph[8], pl[8];
 #pragma unroll
-          for (int e2 = 0; e2 < 16; ++e2) {
+          for (int e2 = 0; e2 < 8; ++e2) {
             const int e = 2 * e2;
-            const float x0 = (bits[c] & (1u << e)) ? __uint_as_float(r[e]) : ninf;
-            const float x1 = (bits[c] & (1u << (e + 1))) ? __uint_as_float(r[e + 1]) : ninf;
-            const float p0 = ex2_ftz(fmaf(x0, a.qk_scale, -msub));
-            const float p1 = ex2_ftz(fmaf(x1, a.qk_scale, -msub));
-            rs += p0 + p1;
+            const float x0 = (bw & (1u << e)) ? __uint_as_float(r[e]) : ninf;
+            const float x1 = (bw & (1u << (e + 1))) ? __uint_as_float(r[e + 1]) : ninf;
+            float y0, y1;
+            unpack2(fma2(pack2(x0, x1), scale2, nm2), y0, y1);  // scale*s - m, two keys
+            const float p0 = ex2_ftz(y0), p1 = ex2_ftz(y1);
+            const unsigned long long p2 = pack2(p0, p1);
+            rs2 = add2(rs2, p2);
             const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-            const float2 hf2 = __bfloat1622float2(h2);
-            const __nv_bfloat162 l2 = __floats2bfloat162_rn(p0 - hf2.x, p1 - hf2.y);
-            ph[e2] = *reinterpret_cast<const uint32_t*>(&h2);
+            const uint32_t hb = *reinterpret_cast<const uint32_t*>(&h2);
+            // P_lo = bf16(p - float(P_hi)), the P_hi pair widened by bit moves
+            float d0, d1;
+            unpack2(sub2(p2, pack2(__uint_as_float(hb << 16), __uint_as_float(hb & 0xffff0000u))),
+                    d0, d1);
+            const __nv_bfloat162 l2 = __floats2bfloat162_rn(d0, d1);
+            ph[e2] = hb;
             pl[e2] = *reinterpret_cast<const uint32_t*>(&l2);
           }
-          tmem_st16(s_col + c * 32, ph);
-          tmem_st16(s_col + c * 32 + 16, pl);
+          tmem_st8(s_col + kk * 16, ph);
+          tmem_st8(s_col + kk * 16 + 8, pl);
+        };
+        tmem_ld16(s_col, ra);
+        tmem_wait_ld();
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          tmem_ld16(s_col + (2 * c + 1) * 16, rc);
+          chunk(ra, b0, 2 * c);
+          tmem_wait_ld();
+          if (c + 1 < 4) tmem_ld16(s_col + (2 * c + 2) * 16, ra);
+          chunk(rc, b0 >> 16, 2 * c + 1);
+          if (c + 1 < 4) tmem_wait_ld();
+          b0 = b1; b1 = b2; b2 = b3;
         }
-        l += rs;
+        {
+          float r0, r1;
+          unpack2(rs2, r0, r1);
+          l += r0 + r1;
+        }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
