@@ -40,8 +40,8 @@ F32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # DRAM traffic per launch from committed ncu captures: (kernel, config) -> (bytes,
 # sha256 of the kernel source when captured).  Reported as null when the source changed.
 NCU_TRAFFIC = {
-    # masked_attn_tc_kernel, c2 full size: 64.31 MB read + 4.31 MB written
-    ("masked_attn", "c2"): (68619008, "ceb7f3c10dd75398"),
+    # masked_attn_tc_kernel, c2 full size: 64.30 MB read + 5.21 MB written
+    ("masked_attn", "c2"): (69505024, "7b24d50f0fc68b67"),
 }
 
 
@@ -160,7 +160,7 @@ def job_value(units_per_rank, world, step_ms_max):
 class Workload:
     """Device buffers and the library calls of one step of config `name`."""
 
-    def __init__(self, name, device, seed_offset=0, S=None, T=None, B=None):
+    def __init__(self, name, device, seed_offset=0, S=None, T=None, B=None, indexer="per_head"):
         import dataclasses
 
         import sparse_attention_15_b200 as dsa
@@ -189,9 +189,11 @@ class Workload:
         self.K = cfg.k_eff
         self.idx = torch.empty((B, cfg.S, self.K), dtype=torch.int32, device=device)
         self.out = torch.empty((B, cfg.S, cfg.H, cfg.dv), dtype=x["q"].dtype, device=device)
+        self.indexer = indexer
         self.args = dsa._forward_args(x["q_idx"], x["k_idx"], x["w"], cfg.scale, cfg.K, x["q"],
                                       x["k"], x["v"], x["gate"], None, "none", 0.0, "auto",
-                                      self.out, None, self.idx)
+                                      self.out, None, self.idx,
+                                      indexer)
         self.ws_bytes = dsa.dsa_forward_workspace_bytes(self.args)
         self.ws = torch.empty(max(self.ws_bytes, 16), dtype=torch.uint8, device=device)
         dt = dsa.DTYPE[x["q"].dtype]
@@ -205,16 +207,17 @@ class Workload:
             self.swa.append(s)
         self.stages = ["indexer", "topk", "attention"] + [f"swa{i + 1}" for i in
                                                           range(len(self.swa))]
-        # our kernels per step: indexer, top-k, attention (+ combine for split gathers), SWA
+        # our kernels per step: indexer (+ the query collapse), top-k, attention (+ combine for
+        # split gathers), SWA
         self.launches_per_step = 3 + (1 if self.algo == "gather" and gather_ws > 0 else 0) + \
-            len(self.swa)
+            (1 if indexer == "collapsed" else 0) + len(self.swa)
 
     def step(self, ev):
         """Run one step; ev is a list of len(stages)+1 CUDA events (stage boundaries)."""
         c, x, d = self.cfg, self.x, self.dsa
         d.dsa_forward(x["q_idx"], x["k_idx"], x["w"], c.scale, c.K, x["q"], x["k"], x["v"],
                       gate=x["gate"], out=self.out, idx_out=self.idx, ws=self.ws,
-                      ws_bytes=self.ws_bytes, events=ev[:4])
+                      ws_bytes=self.ws_bytes, events=ev[:4], indexer=self.indexer)
         for i, s in enumerate(self.swa):
             d.dsa_window_attn(s["q"], s["k"], s["v"], c.window, gate=s["gate"], out=s["out"])
             ev[4 + i].record()
@@ -226,9 +229,21 @@ class Workload:
         pairs = causal_pairs(c.S, c.T, B, c.q_off)
         sel = selected_pairs(c.S, c.T, B, c.q_off, self.K)
         rows = B * c.S
+        if c.S == 1:
+            # decode: one query per batch row streams the whole k_I cache once; HBM-bound
+            # (k_I, the row's q_I and w, the score row written)
+            idx_work = ("hbm", B * c.T * c.DI * es + rows * c.HI * (c.DI * es + 4) +
+                        4.0 * pairs, "GB/s")
+        elif self.indexer == "collapsed":
+            # the head-collapsed form is not held to the per-head flop count: it is bound by
+            # the score writes (4 B per causal pair) plus its reads of q_I, w and k_I
+            idx_work = ("hbm", 4.0 * pairs + rows * c.HI * (c.DI * es + 4) +
+                        B * c.T * c.DI * es, "GB/s")
+        else:
+            idx_work = ("tensor" if c.dtype == "bf16" else "alu", 2.0 * c.HI * c.DI * pairs,
+                        "TFLOP/s")
         w = {
-            "indexer": ("tensor" if c.dtype == "bf16" else "alu", 2.0 * c.HI * c.DI * pairs,
-                        "TFLOP/s"),
+            "indexer": idx_work,
             "topk": ("hbm", 4.0 * pairs + 4.0 * rows * self.K, "GB/s"),
         }
         if self.algo == "masked_tile":
@@ -271,7 +286,7 @@ class Workload:
         c = self.cfg
         self.dsa.dsa_forward(x["q_idx"], x["k_idx"], x["w"], c.scale, c.K, x["q"], x["k"],
                              x["v"], gate=x["gate"], out=self.out, idx_out=self.idx,
-                             ws=self.ws, ws_bytes=self.ws_bytes)
+                             ws=self.ws, ws_bytes=self.ws_bytes, indexer=self.indexer)
         out_host.copy_(self.out, non_blocking=True)
 
 
@@ -384,6 +399,8 @@ def main():
     ap.add_argument("--S", type=int, default=None, help="reduced query count (profiling cases)")
     ap.add_argument("--T", type=int, default=None, help="reduced key count (profiling cases)")
     ap.add_argument("--B", type=int, default=None, help="reduced batch (profiling cases)")
+    ap.add_argument("--indexer", default="per_head", choices=["per_head", "collapsed"],
+                    help="indexer form (the pages' per-head work by default)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world, rank, local = dist_setup(args)
@@ -407,7 +424,8 @@ def main():
                                 device_id=dev)
         pg = dist
 
-    wl = Workload(args.config, dev, seed_offset=rank, S=args.S, T=args.T, B=args.B)
+    wl = Workload(args.config, dev, seed_offset=rank, S=args.S, T=args.T, B=args.B,
+                  indexer=args.indexer)
     cfg = wl.cfg
     nst = len(wl.stages)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
@@ -533,7 +551,7 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32" if cfg.dtype == "f32" else "bf16", "data": "synthetic",
-            "config": workload_config(cfg, wl.B),
+            "config": dict(workload_config(cfg, wl.B), indexer_form=wl.indexer),
             "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
             "clocks": clk, "gpu_launches": wl.launches_per_step * args.steps,
             "wall_ms_per_step_incl_flush": round(1e3 * t_wall / args.steps, 4),

@@ -72,6 +72,9 @@ typedef enum { DSA_RELU_NONE = 0, DSA_RELU_POST_SUM = 1, DSA_RELU_PER_HEAD = 2 }
  * (token, head), evaluated in float32; any other mode is rejected (the page's ValueError). */
 typedef enum { DSA_GATE_OFF = 0, DSA_GATE_SIGMOID = 1, DSA_GATE_SILU = 2 } dsa_gate_mode;
 
+/* How dsa_forward computes the indexer scores (section 1 or section 1b). */
+typedef enum { DSA_INDEXER_PER_HEAD = 0, DSA_INDEXER_COLLAPSED = 1 } dsa_indexer_mode;
+
 /* Attention algorithm for dsa_forward, dsa_sparse_attn and dsa_window_attn. */
 typedef enum {
   DSA_ATTN_AUTO = 0,      /* pick by the cost model (bytes gathered vs. dense tile work)  */
@@ -99,6 +102,27 @@ typedef enum {
 dsa_status dsa_index_scores(dsa_dtype dtype, const void* q_idx, const void* k_idx,
                             const float* w, float scale, dsa_relu_mode relu, int B, int S,
                             int T, int HI, int DI, float* scores, dsa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * 1b. Head-collapsed indexer scores.  Without a per-head ReLU the [AXK2] SGA score is
+ *    linear in the queries: sum_h w[s,h] * (q[s,h,:] . k[t,:]) = k[t,:] . qc[s,:] with
+ *    qc[s,:] = sum_h w[s,h] * q[s,h,:].  This entry point forms qc once per query (float32,
+ *    heads in order, kept as a bf16 hi + lo pair, about 2^-17 relative precision) and
+ *    scores every key against it: 1/HI of the tensor-core work of dsa_index_scores, for
+ *    the same scores (identical for the integer workloads, within float32 rounding of the
+ *    hi/lo split otherwise).  The per-head cost model of [PANGU] §3.5 Table 1 does not
+ *    apply to it; it is reported separately.
+ *
+ *   Arguments as dsa_index_scores, plus a workspace of
+ *   dsa_index_scores_collapsed_workspace_bytes(B, S, DI) bytes (16-byte aligned) for qc.
+ *   Requires dtype DSA_BF16, DI in {64, 128} and relu != DSA_RELU_PER_HEAD (the collapse
+ *   does not hold with a ReLU per head): DSA_ERR_UNSUPPORTED otherwise.
+ * --------------------------------------------------------------------------------- */
+size_t dsa_index_scores_collapsed_workspace_bytes(int B, int S, int DI);
+dsa_status dsa_index_scores_collapsed(dsa_dtype dtype, const void* q_idx, const void* k_idx,
+                                      const float* w, float scale, dsa_relu_mode relu, int B,
+                                      int S, int T, int HI, int DI, float* scores, void* ws,
+                                      size_t ws_bytes, dsa_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
  * 2. Per-query top-k.  [AXK2] SGA: the indexer returns int32 indices [B,S,topk];
@@ -189,6 +213,8 @@ typedef struct {
   void* const* events;     /* optional: 4 caller-owned cudaEvent_t recorded on the stream
                               before the indexer, after it, after the top-k and after the
                               attention (per-stage timing); NULL for none                */
+  dsa_indexer_mode indexer; /* DSA_INDEXER_PER_HEAD (0, the pages' per-head work) or
+                              DSA_INDEXER_COLLAPSED (the section 1b form)                */
 } dsa_forward_args;
 
 /* Bytes of workspace dsa_forward needs to run without row blocking. */

@@ -14,8 +14,9 @@ import os
 import torch
 
 __all__ = [
-    "DSAError", "lib", "dsa_index_scores", "dsa_topk", "dsa_sparse_attn",
-    "dsa_sparse_attn_workspace_bytes", "dsa_sparse_attn_algo", "dsa_forward", "dsa_forward_workspace_bytes",
+    "DSAError", "lib", "dsa_index_scores", "dsa_index_scores_collapsed", "dsa_topk",
+    "dsa_sparse_attn", "dsa_sparse_attn_workspace_bytes", "dsa_sparse_attn_algo", "dsa_forward",
+    "dsa_forward_workspace_bytes",
     "dsa_window_attn", "dsa_sparse_attn_noalloc", "dsa_device_status", "dsa_version",
     "LIB_PATH",
 ]
@@ -26,6 +27,7 @@ DTYPE = {torch.float32: 0, torch.bfloat16: 1}
 RELU = {"none": 0, "post_sum": 1, "per_head": 2}
 GATE = {"off": 0, "sigmoid": 1, "silu": 2}
 ATTN_ALGO = {"auto": 0, "gather": 1, "masked_tile": 2}
+INDEXER = {"per_head": 0, "collapsed": 1}
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "CUDA error", 4: "timeout",
           5: "internal"}
 
@@ -47,7 +49,7 @@ class ForwardArgs(ctypes.Structure):
         ("q_idx", ctypes.c_void_p), ("k_idx", ctypes.c_void_p), ("w", ctypes.c_void_p),
         ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
         ("gate", ctypes.c_void_p), ("out", ctypes.c_void_p), ("scores_out", ctypes.c_void_p),
-        ("idx_out", ctypes.c_void_p), ("events", ctypes.c_void_p),
+        ("idx_out", ctypes.c_void_p), ("events", ctypes.c_void_p), ("indexer", ctypes.c_int),
     ]
 
 
@@ -59,6 +61,9 @@ _Z = ctypes.c_size_t
 
 _SIGNATURES = {
     "dsa_index_scores": (_I, [_I, _P, _P, _P, _F, _I, _I, _I, _I, _I, _I, _P, _P]),
+    "dsa_index_scores_collapsed_workspace_bytes": (_Z, [_I, _I, _I]),
+    "dsa_index_scores_collapsed": (_I, [_I, _P, _P, _P, _F, _I, _I, _I, _I, _I, _I, _P, _P, _Z,
+                                        _P]),
     "dsa_topk": (_I, [_P, _I, _I, _I, _I, _P, _P]),
     "dsa_sparse_attn_workspace_bytes": (_Z, [_I, _I, _I, _I, _I, _I, _I, _I, _I]),
     "dsa_sparse_attn_algo": (_I, [_I, _I, _I, _I, _I, _I, _I, _I, _I]),
@@ -148,6 +153,23 @@ def dsa_index_scores(q_idx, k_idx, w, scale, relu="none", scores=None, stream=No
     return scores
 
 
+def dsa_index_scores_collapsed(q_idx, k_idx, w, scale, relu="none", scores=None, ws=None,
+                               stream=None):
+    """The same scores as dsa_index_scores from the head-collapsed query
+    sum_h w[b,s,h] q_idx[b,s,h,:] (bf16, no per-head ReLU; see include/dsa.h)."""
+    _dev(q_idx, k_idx, w, scores, ws)
+    B, S, HI, DI = q_idx.shape
+    T = k_idx.shape[1]
+    if scores is None:
+        scores = torch.empty((B, S, T), dtype=torch.float32, device=q_idx.device)
+    nbytes = int(lib().dsa_index_scores_collapsed_workspace_bytes(B, S, DI))
+    ws = _workspace(nbytes, q_idx.device, ws)
+    _check(lib().dsa_index_scores_collapsed(_dtype_code(q_idx), _ptr(q_idx), _ptr(k_idx), _ptr(w),
+                                            float(scale), RELU[relu], B, S, T, HI, DI,
+                                            _ptr(scores), _ptr(ws), nbytes, _stream(stream)))
+    return scores
+
+
 def dsa_topk(scores, K, idx=None, stream=None):
     """int32 [B,S,K]: the kept keys of each query in ascending order, -1 padded."""
     _dev(scores, idx)
@@ -217,7 +239,7 @@ def dsa_sparse_attn_noalloc(q, k, v, idx, gate=None, gate_mode=None, sm_scale=0.
 
 
 def _forward_args(q_idx, k_idx, w, index_scale, K, q, k, v, gate, gate_mode, relu, sm_scale,
-                  attn_algo, out, scores_out, idx_out):
+                  attn_algo, out, scores_out, idx_out, indexer="per_head"):
     B, S, HI, DI = q_idx.shape
     T = k_idx.shape[1]
     H, DQK = q.shape[2], q.shape[3]
@@ -230,7 +252,7 @@ def _forward_args(q_idx, k_idx, w, index_scale, K, q, k, v, gate, gate_mode, rel
         w=w.data_ptr(), q=q.data_ptr(), k=k.data_ptr(), v=v.data_ptr(),
         gate=None if gate is None else gate.data_ptr(), out=out.data_ptr(),
         scores_out=None if scores_out is None else scores_out.data_ptr(),
-        idx_out=None if idx_out is None else idx_out.data_ptr())
+        idx_out=None if idx_out is None else idx_out.data_ptr(), indexer=INDEXER[indexer])
     return a
 
 
@@ -241,8 +263,11 @@ def dsa_forward_workspace_bytes(args: ForwardArgs, minimum: bool = False) -> int
 
 def dsa_forward(q_idx, k_idx, w, index_scale, K, q, k, v, gate=None, gate_mode=None,
                 relu="none", sm_scale=0.0, attn_algo="auto", out=None, scores_out=None,
-                idx_out=None, ws=None, ws_bytes=None, stream=None, events=None):
+                idx_out=None, ws=None, ws_bytes=None, stream=None, events=None,
+                indexer="per_head"):
     """The whole DSA step (indexer -> top-k -> sparse attention -> gate).
+    indexer: "per_head" (the pages' per-head work) or "collapsed" (see
+    dsa_index_scores_collapsed).
 
     Returns (out, idx); idx is idx_out if given, else a view of the workspace copy.
     ``ws_bytes`` limits the workspace handed to the library (row blocking below the
@@ -256,7 +281,7 @@ def dsa_forward(q_idx, k_idx, w, index_scale, K, q, k, v, gate=None, gate_mode=N
     if idx_out is None:
         idx_out = torch.empty((B, S, k_eff), dtype=torch.int32, device=q.device)
     a = _forward_args(q_idx, k_idx, w, index_scale, K, q, k, v, gate, gate_mode, relu, sm_scale,
-                      attn_algo, out, scores_out, idx_out)
+                      attn_algo, out, scores_out, idx_out, indexer)
     ev_arr = None
     if events is not None:  # 4 torch.cuda.Event, recorded by the library at stage boundaries
         for e in events:

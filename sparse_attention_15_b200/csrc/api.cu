@@ -86,6 +86,31 @@ dsa_status run_index_scores(dsa_dtype dtype, const void* q_idx, const void* k_id
   return cuda_status(e, "dsa_index_scores");
 }
 
+size_t collapsed_q_bytes(int B, int S, int DI) {
+  return (size_t)B * S * 2 * DI * sizeof(uint16_t);
+}
+
+dsa_status check_collapsed(dsa_dtype dtype, dsa_relu_mode relu, int DI) {
+  REQUIRE(dsa::index_scores_collapsed_supported((int)dtype, DI, (int)relu), DSA_ERR_UNSUPPORTED,
+          "the collapsed indexer needs bf16, DI in {64,128} and no per-head ReLU");
+  return DSA_OK;
+}
+
+// qc for rows [0, B*S) (q_idx/w as given), then the collapsed scores of B x S queries.
+dsa_status run_collapse_q(const void* q_idx, const float* w, long long rows, int HI, int DI,
+                          void* qc, cudaStream_t st) {
+  return cuda_status(dsa::launch_collapse_q(q_idx, w, rows, HI, DI, qc, st),
+                     "collapse_q");
+}
+
+dsa_status run_index_scores_collapsed(const void* qc, const void* k_idx, float scale,
+                                      dsa_relu_mode relu, int B, int S, int T, int DI, int q_off,
+                                      float* scores, int write_masked, cudaStream_t st) {
+  return cuda_status(dsa::launch_index_scores_collapsed(qc, k_idx, scale, (int)relu, B, S, T, DI,
+                                                        q_off, scores, write_masked, st),
+                     "dsa_index_scores_collapsed");
+}
+
 dsa_status check_attn_common(dsa_dtype dtype, const void* q, const void* k, const void* v,
                              const void* gate, dsa_gate_mode gm, float sm_scale, int B, int S,
                              int T, int H, int HKV, int DQK, int DV, const void* out) {
@@ -200,6 +225,27 @@ dsa_status dsa_index_scores(dsa_dtype dtype, const void* q_idx, const void* k_id
                           1, (cudaStream_t)stream);
 }
 
+size_t dsa_index_scores_collapsed_workspace_bytes(int B, int S, int DI) {
+  if (B <= 0 || S <= 0 || DI <= 0) return 0;
+  return collapsed_q_bytes(B, S, DI);
+}
+
+dsa_status dsa_index_scores_collapsed(dsa_dtype dtype, const void* q_idx, const void* k_idx,
+                                      const float* w, float scale, dsa_relu_mode relu, int B,
+                                      int S, int T, int HI, int DI, float* scores, void* ws,
+                                      size_t ws_bytes, dsa_stream_t stream) {
+  dsa_status st = check_index_args(dtype, q_idx, k_idx, w, scale, relu, B, S, T, HI, DI, scores);
+  if (st != DSA_OK) return st;
+  if ((st = check_collapsed(dtype, relu, DI)) != DSA_OK) return st;
+  REQUIRE(ws != nullptr && ws_bytes >= collapsed_q_bytes(B, S, DI), DSA_ERR_INVALID_ARG,
+          "workspace too small: %zu bytes given, %zu needed", ws_bytes,
+          collapsed_q_bytes(B, S, DI));
+  REQUIRE(aligned16(ws), DSA_ERR_UNSUPPORTED, "workspace must be 16-byte aligned");
+  cudaStream_t s = (cudaStream_t)stream;
+  if ((st = run_collapse_q(q_idx, w, (long long)B * S, HI, DI, ws, s)) != DSA_OK) return st;
+  return run_index_scores_collapsed(ws, k_idx, scale, relu, B, S, T, DI, T - S, scores, 1, s);
+}
+
 dsa_status dsa_topk(const float* scores, int B, int S, int T, int K, int32_t* idx,
                     dsa_stream_t stream) {
   REQUIRE(scores && idx, DSA_ERR_INVALID_ARG, "null pointer argument");
@@ -305,11 +351,14 @@ static dsa_status check_forward(const dsa_forward_args* a) {
           DSA_ERR_INVALID_ARG, "unknown attention algorithm %d", (int)a->attn_algo);
   REQUIRE(a->idx_out == nullptr || aligned16(a->idx_out), DSA_ERR_UNSUPPORTED,
           "idx_out must be 16-byte aligned");
+  REQUIRE(a->indexer == DSA_INDEXER_PER_HEAD || a->indexer == DSA_INDEXER_COLLAPSED,
+          DSA_ERR_INVALID_ARG, "unknown indexer mode %d", (int)a->indexer);
+  if (a->indexer == DSA_INDEXER_COLLAPSED) return check_collapsed(a->dtype, a->relu, a->DI);
   return DSA_OK;
 }
 
 struct FwdLayout {
-  size_t idx_off, attn_off, mask_off, scores_off, total_full, total_min;
+  size_t idx_off, attn_off, mask_off, qc_off, scores_off, total_full, total_min;
   int k_eff, alg, mask_stride;
 };
 
@@ -326,6 +375,8 @@ static FwdLayout forward_layout(const dsa_forward_args* a) {
     off += align256(dsa::gather_attn_workspace_bytes(a->B, a->S, a->H, a->DV, L.k_eff));
   L.mask_off = off;
   if (L.alg == kMasked) off += align256(mask_bytes(a->B, a->S, a->T));
+  L.qc_off = off;
+  if (a->indexer == DSA_INDEXER_COLLAPSED) off += align256(collapsed_q_bytes(a->B, a->S, a->DI));
   L.scores_off = off;
   if (a->scores_out) {
     L.total_full = L.total_min = off;
@@ -360,6 +411,8 @@ dsa_status dsa_forward(const dsa_forward_args* a, void* ws, size_t ws_bytes,
   uint8_t* base = static_cast<uint8_t*>(ws);
   int32_t* idx = a->idx_out ? a->idx_out : reinterpret_cast<int32_t*>(base + L.idx_off);
   void* attn_ws = (base && L.alg == kGather) ? base + L.attn_off : nullptr;
+  const bool collapsed = a->indexer == DSA_INDEXER_COLLAPSED;
+  uint8_t* qc = collapsed ? base + L.qc_off : nullptr;
   const size_t attn_ws_bytes = L.mask_off - L.attn_off;
   uint32_t* mask = L.alg == kMasked ? reinterpret_cast<uint32_t*>(base + L.mask_off) : nullptr;
   const int B = a->B, S = a->S, T = a->T, q_off = T - S;
@@ -370,11 +423,17 @@ dsa_status dsa_forward(const dsa_forward_args* a, void* ws, size_t ws_bytes,
     return ev ? cuda_status(cudaEventRecord(ev[i], s), "dsa_forward/event") : DSA_OK;
   };
   if ((st = mark(0)) != DSA_OK) return st;
+  if (collapsed &&
+      (st = run_collapse_q(a->q_idx, a->w, (long long)B * S, a->HI, a->DI, qc, s)) != DSA_OK)
+    return st;
 
   if (a->scores_out || ws_bytes >= L.total_full) {
     float* scores = a->scores_out ? a->scores_out : reinterpret_cast<float*>(base + L.scores_off);
-    st = run_index_scores(a->dtype, a->q_idx, a->k_idx, a->w, a->index_scale, a->relu, B, S, T,
-                          a->HI, a->DI, q_off, scores, write_masked, s);
+    st = collapsed ? run_index_scores_collapsed(qc, a->k_idx, a->index_scale, a->relu, B, S, T,
+                                                a->DI, q_off, scores, write_masked, s)
+                   : run_index_scores(a->dtype, a->q_idx, a->k_idx, a->w, a->index_scale,
+                                      a->relu, B, S, T, a->HI, a->DI, q_off, scores,
+                                      write_masked, s);
     if (st != DSA_OK || (st = mark(1)) != DSA_OK) return st;
     st = cuda_status(dsa::launch_topk(scores, B, S, T, L.k_eff, q_off, idx, mask, L.mask_stride,
                                       s),
@@ -394,8 +453,11 @@ dsa_status dsa_forward(const dsa_forward_args* a, void* ws, size_t ws_bytes,
         const uint8_t* ki = static_cast<const uint8_t*>(a->k_idx) + (size_t)b * T * a->DI * es;
         const float* wb = a->w + ((size_t)b * S + s0) * a->HI;
         // this block's first query sits at key position q_off + s0
-        st = run_index_scores(a->dtype, qi, ki, wb, a->index_scale, a->relu, 1, n, T, a->HI,
-                              a->DI, q_off + s0, scores, 0, s);
+        const uint8_t* qcb = collapsed ? qc + ((size_t)b * S + s0) * 2 * a->DI * 2 : nullptr;
+        st = collapsed ? run_index_scores_collapsed(qcb, ki, a->index_scale, a->relu, 1, n, T,
+                                                    a->DI, q_off + s0, scores, 0, s)
+                       : run_index_scores(a->dtype, qi, ki, wb, a->index_scale, a->relu, 1, n,
+                                          T, a->HI, a->DI, q_off + s0, scores, 0, s);
         if (st != DSA_OK) return st;
         const size_t row0 = (size_t)b * S + s0;
         st = cuda_status(dsa::launch_topk(scores, 1, n, T, L.k_eff, q_off + s0,

@@ -51,9 +51,12 @@ struct TcArgs {
   int max_chunks;  // units per query block slot (chunks of the longest block)
 };
 
-template <int HI_, int DI_, int NQ_, int NE_, int NA_, int NB_ = 2>
+// CL_: the head-collapsed form -- the B operand holds two bf16 rows per query (the hi and
+// lo parts of sum_h w[s,h] q_I[s,h,:]) and a score is the sum of its two columns.
+template <int HI_, int DI_, int NQ_, int NE_, int NA_, int NB_ = 2, bool CL_ = false>
 struct TcCfg {
   static constexpr int HI = HI_, DI = DI_, NQ = NQ_, NE = NE_, NA = NA_;
+  static constexpr bool CL = CL_;
   static constexpr int NB = NB_;                  // query-block buffers (1 or 2)
   static constexpr int N = NQ * HI;               // MMA N: (query, head) columns
   static constexpr int KH = DI / 64;              // 64-element (128-byte) K slices
@@ -71,6 +74,8 @@ struct TcCfg {
   static constexpr int SMEM = NA * A_BYTES + NB * B_BYTES + BAR_BYTES + 1024;
   static_assert(N % 16 == 0 && N >= 16 && N <= 256, "UMMA N");
   static_assert(HI <= 32 && 32 % HI == 0, "heads per 32-column chunk");
+  static_assert(!CL || HI == 2, "the collapsed form has two columns (hi, lo) per query");
+  static_assert(CL || HI >= 16, "per-head epilogue: a query spans whole 16-column chunks");
   static_assert(COLS_PER_WARP % 32 == 0 && COLS_PER_WARP % HI == 0, "epilogue chunking");
   static_assert(DI % 64 == 0, "DI must be a multiple of 64");
 };
@@ -251,7 +256,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       // the head weights of this unit's queries (1-2 KB) are the same for every key tile and
       // every lane: the reduction reads them as warp-wide broadcast float4 loads, which stay
       // in L1 for the whole unit (one load per four heads, no shuffles)
-      const float4* wunit = reinterpret_cast<const float4*>(
+      const float4* wunit = C::CL ? nullptr : reinterpret_cast<const float4*>(
           a.w + ((size_t)it.b * a.S + s_base) * C::HI);
       for (int kt = it.k0; kt < it.k1; ++kt) {
         const int ab = ci & 1;
@@ -277,30 +282,45 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           }
           const uint32_t* r = rb[cc & 1];
           const int c0 = col0 + cc * 16;     // first column of the chunk
-          const int j = c0 / C::HI;          // query within the block
-          const int s = s_base + j;
-          if (s < a.S) {  // ragged tail of the last block (warp-uniform)
+          if constexpr (C::CL) {
+            // eight queries per chunk: score = scale * (D[t, hi] + D[t, lo])
+            const int sq = s_base + c0 / 2;
+            float* op = a.scores + ((size_t)it.b * a.S + sq) * a.T + t;
 #pragma unroll
-            for (int h = 0; h < 16; h += 4) {
-              const float4 w4 = __ldg(wunit + (c0 + h) / 4);
-              float d0 = __uint_as_float(r[h + 0]);
-              float d1 = __uint_as_float(r[h + 1]);
-              float d2 = __uint_as_float(r[h + 2]);
-              float d3 = __uint_as_float(r[h + 3]);
-              if (RELU == 2) {
-                d0 = fmaxf(d0, 0.f); d1 = fmaxf(d1, 0.f); d2 = fmaxf(d2, 0.f); d3 = fmaxf(d3, 0.f);
+            for (int q = 0; q < 8; ++q) {
+              if (sq + q < a.S && t < a.T) {
+                float v = (__uint_as_float(r[2 * q]) + __uint_as_float(r[2 * q + 1])) * a.scale;
+                if (RELU == 1) v = fmaxf(v, 0.f);
+                op[(size_t)q * a.T] = (t <= sq + q + a.q_off) ? v : ninf;
               }
-              acc4[0] = fmaf(w4.x, d0, acc4[0]);
-              acc4[1] = fmaf(w4.y, d1, acc4[1]);
-              acc4[2] = fmaf(w4.z, d2, acc4[2]);
-              acc4[3] = fmaf(w4.w, d3, acc4[3]);
             }
-            if ((c0 + 16) % C::HI == 0) {  // the query's last chunk: finish and store
-              float v = ((acc4[0] + acc4[1]) + (acc4[2] + acc4[3])) * a.scale;
-              if (RELU == 1) v = fmaxf(v, 0.f);
-              if (t < a.T)
-                a.scores[((size_t)it.b * a.S + s) * a.T + t] = (t <= s + a.q_off) ? v : ninf;
-              acc4[0] = acc4[1] = acc4[2] = acc4[3] = 0.f;
+          } else {
+            const int j = c0 / C::HI;          // query within the block
+            const int s = s_base + j;
+            if (s < a.S) {  // ragged tail of the last block (warp-uniform)
+#pragma unroll
+              for (int h = 0; h < 16; h += 4) {
+                const float4 w4 = __ldg(wunit + (c0 + h) / 4);
+                float d0 = __uint_as_float(r[h + 0]);
+                float d1 = __uint_as_float(r[h + 1]);
+                float d2 = __uint_as_float(r[h + 2]);
+                float d3 = __uint_as_float(r[h + 3]);
+                if (RELU == 2) {
+                  d0 = fmaxf(d0, 0.f); d1 = fmaxf(d1, 0.f); d2 = fmaxf(d2, 0.f);
+                  d3 = fmaxf(d3, 0.f);
+                }
+                acc4[0] = fmaf(w4.x, d0, acc4[0]);
+                acc4[1] = fmaf(w4.y, d1, acc4[1]);
+                acc4[2] = fmaf(w4.z, d2, acc4[2]);
+                acc4[3] = fmaf(w4.w, d3, acc4[3]);
+              }
+              if ((c0 + 16) % C::HI == 0) {  // the query's last chunk: finish and store
+                float v = ((acc4[0] + acc4[1]) + (acc4[2] + acc4[3])) * a.scale;
+                if (RELU == 1) v = fmaxf(v, 0.f);
+                if (t < a.T)
+                  a.scores[((size_t)it.b * a.S + s) * a.T + t] = (t <= s + a.q_off) ? v : ninf;
+                acc4[0] = acc4[1] = acc4[2] = acc4[3] = 0.f;
+              }
             }
           }
           if (cc + 1 < NCH) tmem_wait_ld();
@@ -329,6 +349,63 @@ __global__ void fill_masked_kernel(float* __restrict__ scores, int S, int T, int
   float* r = scores + row * (size_t)T;
   const float ninf = __int_as_float(0xff800000);
   for (int t = start + threadIdx.x; t < T; t += blockDim.x) r[t] = ninf;
+}
+
+// The head-collapsed query of each row: qc = sum_h w[s,h] * q_I[s,h,:] in float32 (heads in
+// order), stored as two bf16 rows, hi = bf16(qc) and lo = bf16(qc - hi), so that
+// k . hi + k . lo carries qc to about 2^-17 relative precision (exactly, for the integer
+// workloads, where lo = 0).  One warp per row; lane l owns dims l*E .. l*E+E-1.
+// E consecutive bf16 <-> float (E = 2 or 4; 4- or 8-byte aligned accesses).
+template <int E>
+__device__ __forceinline__ void load_bf16(const __nv_bfloat16* p, float (&x)[E]) {
+  if constexpr (E == 4) {
+    load4(p, x);
+  } else {
+    const uint32_t v = *reinterpret_cast<const uint32_t*>(p);
+    x[0] = __uint_as_float(v << 16);
+    x[1] = __uint_as_float(v & 0xffff0000u);
+  }
+}
+template <int E>
+__device__ __forceinline__ void store_bf16(__nv_bfloat16* p, const __nv_bfloat16 (&x)[E]) {
+  uint32_t u[E / 2];
+#pragma unroll
+  for (int i = 0; i < E / 2; ++i)
+    u[i] = (uint32_t)__bfloat16_as_ushort(x[2 * i]) |
+           ((uint32_t)__bfloat16_as_ushort(x[2 * i + 1]) << 16);
+  if constexpr (E == 4)
+    *reinterpret_cast<uint2*>(p) = make_uint2(u[0], u[1]);
+  else
+    *reinterpret_cast<uint32_t*>(p) = u[0];
+}
+
+template <int DI>
+__global__ void collapse_q_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ w,
+                                  __nv_bfloat16* __restrict__ qc, long long rows, int HI) {
+  constexpr int E = DI / 32;
+  const long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  float acc[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) acc[e] = 0.f;
+  const __nv_bfloat16* qr = q + row * HI * DI + lane * E;
+  const float* wr = w + row * HI;
+  for (int h = 0; h < HI; ++h) {
+    const float wh = __ldg(wr + h);
+    float x[E];
+    load_bf16<E>(qr + (size_t)h * DI, x);
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] = fmaf(wh, x[e], acc[e]);
+  }
+  __nv_bfloat16 hi[E], lo[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    hi[e] = __float2bfloat16_rn(acc[e]);
+    lo[e] = __float2bfloat16_rn(acc[e] - __bfloat162float(hi[e]));
+  }
+  store_bf16<E>(qc + (row * 2) * DI + lane * E, hi);
+  store_bf16<E>(qc + (row * 2 + 1) * DI + lane * E, lo);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
@@ -412,6 +489,37 @@ cudaError_t launch_cfg(const void* q_idx, const void* k_idx, const float* w, flo
 }
 
 }  // namespace
+
+bool index_scores_collapsed_supported(int dtype, int DI, int relu) {
+  return dtype == 1 && (DI == 64 || DI == 128) && relu != 2;
+}
+
+cudaError_t launch_collapse_q(const void* q_idx, const float* w, long long rows, int HI, int DI,
+                              void* qc, cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  const unsigned grid = (unsigned)((rows + 7) / 8);  // 8 rows (warps) per CTA
+  if (DI == 128)
+    collapse_q_kernel<128><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q_idx), w,
+                                                 static_cast<__nv_bfloat16*>(qc), rows, HI);
+  else if (DI == 64)
+    collapse_q_kernel<64><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q_idx), w,
+                                                static_cast<__nv_bfloat16*>(qc), rows, HI);
+  else
+    return cudaErrorNotSupported;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_index_scores_collapsed(const void* qc, const void* k_idx, float scale,
+                                          int relu, int B, int S, int T, int DI, int q_off,
+                                          float* scores, int write_masked, cudaStream_t st) {
+  if (!index_scores_collapsed_supported(1, DI, relu)) return cudaErrorNotSupported;
+  // 128 queries x (hi, lo) = 256 columns per tile
+  if (DI == 128)
+    return launch_cfg<TcCfg<2, 128, 128, 16, 3, 2, true>>(qc, k_idx, nullptr, scale, relu, B, S,
+                                                          T, q_off, scores, write_masked, st);
+  return launch_cfg<TcCfg<2, 64, 128, 16, 4, 2, true>>(qc, k_idx, nullptr, scale, relu, B, S, T,
+                                                       q_off, scores, write_masked, st);
+}
 
 bool index_scores_tc_supported(int dtype, int HI, int DI) {
   return dtype == 1 && (HI == 16 || HI == 32) && (DI == 64 || DI == 128);

@@ -25,6 +25,17 @@ cudaError_t launch_index_scores_tc(const void* q_idx, const void* k_idx, const f
                                    int q_off, float* scores, int write_masked,
                                    cudaStream_t st);
 
+// Head-collapsed indexer (valid when no ReLU is applied per head: the score is linear in
+// q_I): launch_collapse_q writes qc [rows, 2, DI] bf16 (hi and lo parts of
+// sum_h w[s,h] q_I[s,h,:]); launch_index_scores_collapsed scores k_I against them on the
+// tensor cores.  bf16, DI in {64, 128}, relu != per-head.
+bool index_scores_collapsed_supported(int dtype, int DI, int relu);
+cudaError_t launch_collapse_q(const void* q_idx, const float* w, long long rows, int HI, int DI,
+                              void* qc, cudaStream_t st);
+cudaError_t launch_index_scores_collapsed(const void* qc, const void* k_idx, float scale,
+                                          int relu, int B, int S, int T, int DI, int q_off,
+                                          float* scores, int write_masked, cudaStream_t st);
+
 // Per-row top-k (radix select + ordered compaction).  `mask` (optional) receives the
 // selection bitmask, one bit per key, rows of `mask_stride` 32-bit words
 // (mask_stride >= ceil(T/32); words past the row's keys are zero).

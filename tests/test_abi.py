@@ -66,6 +66,29 @@ def test_index_scores_rejects_bad_arguments(lib):
     assert b"16-byte" in L.dsa_last_error()
 
 
+def _collapsed(L, ws_bytes=1 << 20, **kw):
+    a = dict(dtype=1, q=FAKE, k=FAKE, w=FAKE, scale=0.5, relu=0, B=1, S=4, T=4, HI=16, DI=64,
+             scores=FAKE, ws=FAKE)
+    a.update(kw)
+    return L.dsa_index_scores_collapsed(a["dtype"], a["q"], a["k"], a["w"], a["scale"], a["relu"],
+                                        a["B"], a["S"], a["T"], a["HI"], a["DI"], a["scores"],
+                                        a["ws"], ws_bytes, None)
+
+
+def test_index_scores_collapsed_rejects_bad_arguments(lib):
+    L = lib.lib()
+    assert L.dsa_index_scores_collapsed_workspace_bytes(2, 5, 128) == 2 * 5 * 2 * 128 * 2
+    assert _collapsed(L, q=None) == 1
+    assert _collapsed(L, S=8, T=4) == 1
+    assert _collapsed(L, relu=2) == 2        # a per-head ReLU does not collapse
+    assert b"per-head" in L.dsa_last_error()
+    assert _collapsed(L, dtype=0, DI=32) == 2  # float32 / DI outside {64, 128}
+    assert _collapsed(L, DI=96) == 2
+    assert _collapsed(L, ws=None) == 1
+    assert _collapsed(L, ws_bytes=4 * 2 * 64 * 2 - 1) == 1  # one byte short
+    assert _collapsed(L, ws=FAKE_MIS) == 2
+
+
 def test_topk_rejects_bad_arguments(lib):
     L = lib.lib()
     assert L.dsa_topk(None, 1, 4, 4, 2, FAKE, None) == 1
@@ -134,6 +157,16 @@ def test_forward_workspace_and_validation(lib):
     a.gate_mode = 0
     a.attn_algo = 9
     assert L.dsa_forward(ctypes.byref(a), FAKE, full, None) == 1
+    a.attn_algo = 0
+    a.indexer = 7
+    assert L.dsa_forward(ctypes.byref(a), FAKE, full, None) == 1
+    # the collapsed indexer needs room for its query rows and no per-head ReLU
+    a.indexer = 1
+    full_c = lib.dsa_forward_workspace_bytes(a)
+    assert full_c == full + 4096 * 2 * 64 * 2
+    assert lib.dsa_forward_workspace_bytes(a, minimum=True) == small + 4096 * 2 * 64 * 2
+    a.relu = 2
+    assert L.dsa_forward(ctypes.byref(a), FAKE, full_c, None) == 2
 
 
 def test_binding_fails_loudly_without_library(monkeypatch):

@@ -48,6 +48,68 @@ def test_index_scores_exact(name, S, T, relu):
     assert np.array_equal(P.to_np(got), ref.astype(np.float32))
 
 
+# --------------------------------------------------------------- indexer, head-collapsed form
+COLLAPSED = [("c2", 333, 333), ("c2", 100, 517), ("c3", 200, 455), ("c5", 131, 300),
+             ("c3", 1, 700)]
+
+
+@pytest.mark.parametrize("name,S,T", COLLAPSED)
+@pytest.mark.parametrize("relu", ["none", "post_sum"])
+def test_index_scores_collapsed_exact(name, S, T, relu):
+    # integer inputs: the collapsed query is an integer vector (|qc| <= 4*HI*2), exact in bf16,
+    # so the scores equal the oracle's per-head sums bit for bit
+    cfg, x, g = _inputs(name, S, T)
+    got = dsa.dsa_index_scores_collapsed(g["q_idx"], g["k_idx"], g["w"], cfg.scale, relu=relu)
+    ref = O.index_scores(x["q_idx"], x["k_idx"], x["w"], cfg.scale, relu=relu)
+    assert np.array_equal(P.to_np(got), ref.astype(np.float32))
+
+
+def test_index_scores_collapsed_real_valued_inputs():
+    # N(0,1) bf16 inputs and non-integer weights: the collapsed scores differ from the exact
+    # sums only by float32 rounding -- qc in float32 (HI terms), its bf16 hi/lo split
+    # (<= 2^-16 |qc| per element) and the DI-term float32 dot product -- so
+    # |err| <= 2^-14 * scale * sum_d |k_d| * sum_h |w_h q_hd| is a safe bound.
+    g = torch.Generator().manual_seed(7)
+    B, S, T, HI, DI = 1, 300, 400, 32, 128
+    qi = torch.randn(B, S, HI, DI, generator=g).bfloat16()
+    ki = torch.randn(B, T, DI, generator=g).bfloat16()
+    w = torch.rand(B, S, HI, generator=g) * 2.0
+    scale = 0.0883
+    got = dsa.dsa_index_scores_collapsed(qi.to(DEV), ki.to(DEV), w.to(DEV), scale)
+    ref = O.index_scores(qi, ki, w, scale)
+    mag = scale * np.einsum("btd,bsd->bst", np.abs(ki.double().numpy()),
+                            np.einsum("bsh,bshd->bsd", np.abs(w.double().numpy()),
+                                      np.abs(qi.double().numpy())))
+    got_np = P.to_np(got).astype(np.float64)
+    causal = np.isfinite(ref)
+    assert np.array_equal(np.isfinite(got_np), causal)
+    err = np.abs(got_np[causal] - ref[causal])
+    assert np.all(err <= 2.0 ** -14 * mag[causal] + 1e-30), float((err / mag[causal]).max())
+
+
+@pytest.mark.parametrize("name,S,T", [("c2", 600, 600), ("c3", 260, 330)])
+def test_forward_collapsed_matches_per_head(name, S, T):
+    cfg, x, g = _inputs(name, S, T)
+    K = min(cfg.K, 96)
+    out1, idx1 = dsa.dsa_forward(g["q_idx"], g["k_idx"], g["w"], cfg.scale, K, g["q"], g["k"],
+                                 g["v"], gate=g["gate"])
+    out2, idx2 = dsa.dsa_forward(g["q_idx"], g["k_idx"], g["w"], cfg.scale, K, g["q"], g["k"],
+                                 g["v"], gate=g["gate"], indexer="collapsed")
+    assert torch.equal(idx1, idx2)
+    assert torch.equal(out1, out2)
+    # row-blocked collapsed path (score buffer smaller than the score matrix)
+    out3 = torch.empty_like(out1)
+    idx3 = torch.empty_like(idx1)
+    args = dsa._forward_args(g["q_idx"], g["k_idx"], g["w"], cfg.scale, K, g["q"], g["k"],
+                             g["v"], g["gate"], None, "none", 0.0, "auto", out3, None, idx3,
+                             "collapsed")
+    small = dsa.dsa_forward_workspace_bytes(args, minimum=True) + 41 * T * 4
+    dsa.dsa_forward(g["q_idx"], g["k_idx"], g["w"], cfg.scale, K, g["q"], g["k"], g["v"],
+                    gate=g["gate"], out=out3, idx_out=idx3, ws_bytes=small, indexer="collapsed")
+    assert torch.equal(idx3, idx1)
+    assert torch.equal(out3, out1)
+
+
 # ------------------------------------------------------------------------------- top-k
 @pytest.mark.parametrize("name,S,T", SMALL)
 @pytest.mark.parametrize("K", [1, 16, 100, 400])
