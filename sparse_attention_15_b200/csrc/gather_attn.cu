@@ -27,6 +27,52 @@ namespace dsa {
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLazyRescale = 8.0f;  // raise the running max only past 2^8 (log2 units)
+
+// 2^x on the special-function unit (flush-to-zero; exp2(-inf) = +0).
+__device__ __forceinline__ float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Warp sums of N per-lane partials (N = 1, 2, 4), every lane receiving all N sums.  The
+// first butterfly steps halve the values each lane carries (lanes split the heads between
+// them), so N sums cost N + 4 shuffles (plus N broadcasts) instead of 5N.
+template <int N>
+__device__ __forceinline__ void warp_sum_heads(const float (&x)[N], float (&out)[N]) {
+  const int lane = threadIdx.x & 31;
+  if constexpr (N == 1) {
+    float v = x[0];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    out[0] = v;
+  } else if constexpr (N == 2) {
+    const bool up = lane & 16;  // lanes 16..31 keep head 1
+    const float send = up ? x[0] : x[1];
+    const float keep = up ? x[1] : x[0];
+    float v = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    out[0] = __shfl_sync(0xffffffffu, v, 0);
+    out[1] = __shfl_sync(0xffffffffu, v, 16);
+  } else {
+    static_assert(N == 4, "1, 2 or 4 heads per warp");
+    const bool up16 = lane & 16, up8 = lane & 8;
+    // step 1: lanes 16..31 keep heads 2,3; lanes 0..15 keep heads 0,1
+    const float s0 = up16 ? x[0] : x[2], s1 = up16 ? x[1] : x[3];
+    const float k0 = up16 ? x[2] : x[0], k1 = up16 ? x[3] : x[1];
+    const float a0 = k0 + __shfl_xor_sync(0xffffffffu, s0, 16);
+    const float a1 = k1 + __shfl_xor_sync(0xffffffffu, s1, 16);
+    // step 2: within each half, lanes with bit 3 set keep the second head of the pair
+    float v = (up8 ? a1 : a0) + __shfl_xor_sync(0xffffffffu, up8 ? a0 : a1, 8);
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    // lane 0: head 0, lane 8: head 1, lane 16: head 2, lane 24: head 3
+#pragma unroll
+    for (int i = 0; i < 4; ++i) out[i] = __shfl_sync(0xffffffffu, v, 8 * i);
+  }
+}
 
 struct GatherArgs {
   const void* q;
@@ -119,15 +165,24 @@ __global__ void __launch_bounds__(544, HPW <= 2 ? 2 : 1) gather_attn_kernel(cons
   }
 
   // --------------------------------------------------------------- consumers
+  // Per key and head: dot = q.k (lanes hold 4 dims of each 128-wide slice), one butterfly
+  // reduction for every pair of heads, p = 2^(dot - m), acc += p v.  The running max m is
+  // only raised when a key exceeds it by more than 2^8 (p <= 256 otherwise), so the
+  // accumulator is rescaled rarely rather than on every key; the final (acc, m, l) is the
+  // same softmax as with a strict running max.
   constexpr int hpw = HPW;  // heads per warp
-  constexpr int kMaxHpw = HPW;
   const int group = a.H / a.HKV;
-  float qr[kMaxHpw][QKV][4];
-  float acc[kMaxHpw][VV][4];
-  float m[kMaxHpw], l[kMaxHpw];
+  float qr[hpw][QKV][4];
+  float acc[hpw][VV][4];
+  float m[hpw], l[hpw];
+  int koff[hpw], voff[hpw];  // element offsets of this warp's heads inside a slot
   const T* qrow = static_cast<const T*>(a.q) + (size_t)row * a.H * a.DQK;
 #pragma unroll
-  for (int hi = 0; hi < kMaxHpw; ++hi) {
+  for (int hi = 0; hi < hpw; ++hi) {
+    const int h = warp + nw * hi;
+    const int kvh = h / group;
+    koff[hi] = kvh * a.DQK;
+    voff[hi] = kvh * a.DV;
     m[hi] = -INFINITY;
     l[hi] = 0.f;
 #pragma unroll
@@ -138,62 +193,75 @@ __global__ void __launch_bounds__(544, HPW <= 2 ? 2 : 1) gather_attn_kernel(cons
     for (int c = 0; c < QKV; ++c) {
       const int d = c * 128 + lane * 4;
       float x[4] = {0.f, 0.f, 0.f, 0.f};
-      if (hi < hpw && d < a.DQK) load4(qrow + (size_t)(warp + nw * hi) * a.DQK + d, x);
+      if (d < a.DQK) load4(qrow + (size_t)h * a.DQK + d, x);
 #pragma unroll
       for (int e = 0; e < 4; ++e) qr[hi][c][e] = x[e] * a.qk_scale;
     }
   }
 
   bool ok = true;
+  int slot = 0;
+  uint32_t phase = 0;
   for (int j = 0; j < nkeys && ok; ++j) {
-    const int slot = j % nslots;
-    ok = mbar_wait(&full[slot], (j / nslots) & 1);
+    ok = mbar_wait(&full[slot], phase);
     if (ok && slot_key[slot] >= 0) {
       const T* ks = reinterpret_cast<const T*>(slots + (size_t)slot * a.slot_bytes);
       const T* vs = reinterpret_cast<const T*>(slots + (size_t)slot * a.slot_bytes + a.k_bytes);
+      float part[hpw];
 #pragma unroll
-      for (int hi = 0; hi < kMaxHpw; ++hi) {
-        if (hi >= hpw) break;
-        const int h = warp + nw * hi;
-        const int kvh = h / group;
+      for (int hi = 0; hi < hpw; ++hi) {
         float dot = 0.f;
 #pragma unroll
         for (int c = 0; c < QKV; ++c) {
           const int d = c * 128 + lane * 4;
           if (d < a.DQK) {
             float x[4];
-            load4(ks + (size_t)kvh * a.DQK + d, x);
+            load4(ks + koff[hi] + d, x);
 #pragma unroll
             for (int e = 0; e < 4; ++e) dot = fmaf(qr[hi][c][e], x[e], dot);
           }
         }
+        part[hi] = dot;
+      }
+      float dots[hpw];
+      warp_sum_heads<hpw>(part, dots);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-        const float mn = fmaxf(m[hi], dot);
-        const float corr = exp2f(m[hi] - mn);
-        const float p = exp2f(dot - mn);
-        m[hi] = mn;
-        l[hi] = fmaf(l[hi], corr, p);
+      for (int hi = 0; hi < hpw; ++hi) {
+        const float dot = dots[hi];
+        if (dot > m[hi] + kLazyRescale) {  // warp-uniform: every lane holds the same dot
+          const float alpha = ex2_ftz(m[hi] - dot);  // 0 for the first key (m = -inf)
+          l[hi] *= alpha;
+#pragma unroll
+          for (int c = 0; c < VV; ++c)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[hi][c][e] *= alpha;
+          m[hi] = dot;
+        }
+        const float p = ex2_ftz(dot - m[hi]);
+        l[hi] += p;
 #pragma unroll
         for (int c = 0; c < VV; ++c) {
           const int d = c * 128 + lane * 4;
           if (d < a.DV) {
             float x[4];
-            load4(vs + (size_t)kvh * a.DV + d, x);
+            load4(vs + voff[hi] + d, x);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) acc[hi][c][e] = fmaf(p, x[e], acc[hi][c][e] * corr);
+            for (int e = 0; e < 4; ++e) acc[hi][c][e] = fmaf(p, x[e], acc[hi][c][e]);
           }
         }
       }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[slot]);
+    if (++slot == nslots) {
+      slot = 0;
+      phase ^= 1u;
+    }
   }
 
   // --------------------------------------------------------------- epilogue
 #pragma unroll
-  for (int hi = 0; hi < kMaxHpw; ++hi) {
-    if (hi >= hpw) break;
+  for (int hi = 0; hi < hpw; ++hi) {
     const int h = warp + nw * hi;
     if (a.nsplit == 1) {
       float f = l[hi] > 0.f ? 1.0f / l[hi] : 0.f;
