@@ -42,6 +42,9 @@ F32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 NCU_TRAFFIC = {
     # masked_attn_tc_kernel, c2 full size: 64.30 MB read + 5.21 MB written
     ("masked_attn", "c2"): (69505024, "7b24d50f0fc68b67"),
+    # gather_attn_kernel, c4: captured at B = 32 (same per-row work: 9 splits x 228 keys),
+    # 1.3429 GB read + 6.27 MB written, scaled by the rows (x2) to the full B = 64 launch
+    ("gather_attn", "c4"): (2698253856, "e54ebdebc52f47b9"),
 }
 
 
@@ -160,7 +163,8 @@ def job_value(units_per_rank, world, step_ms_max):
 class Workload:
     """Device buffers and the library calls of one step of config `name`."""
 
-    def __init__(self, name, device, seed_offset=0, S=None, T=None, B=None, indexer="per_head"):
+    def __init__(self, name, device, seed_offset=0, S=None, T=None, B=None, indexer="per_head",
+                 index_dtype="as_dtype"):
         import dataclasses
 
         import sparse_attention_15_b200 as dsa
@@ -185,6 +189,10 @@ class Workload:
                 raise RuntimeError("not enough device memory for one decode batch row")
         self.B = B
         x = dsa_inputs(cfg, device=device, B=B, seed=cfg.seed + seed_offset)
+        self.index_dtype = index_dtype
+        if index_dtype == "e4m3":  # indexer inputs handed over as e4m3 (exact for the integers)
+            x["q_idx"] = x["q_idx"].to(torch.float8_e4m3fn)
+            x["k_idx"] = x["k_idx"].to(torch.float8_e4m3fn)
         self.x = x
         self.K = cfg.k_eff
         self.idx = torch.empty((B, cfg.S, self.K), dtype=torch.int32, device=device)
@@ -229,10 +237,11 @@ class Workload:
         pairs = causal_pairs(c.S, c.T, B, c.q_off)
         sel = selected_pairs(c.S, c.T, B, c.q_off, self.K)
         rows = B * c.S
+        ies = 1 if self.index_dtype == "e4m3" else es  # bytes per indexer input element
         if c.S == 1:
             # decode: one query per batch row streams the whole k_I cache once; HBM-bound
             # (k_I, the row's q_I and w, the score row written)
-            idx_work = ("hbm", B * c.T * c.DI * es + rows * c.HI * (c.DI * es + 4) +
+            idx_work = ("hbm", B * c.T * c.DI * ies + rows * c.HI * (c.DI * ies + 4) +
                         4.0 * pairs, "GB/s")
         elif self.indexer == "collapsed":
             # the head-collapsed form is not held to the per-head flop count: it is bound by
@@ -401,6 +410,8 @@ def main():
     ap.add_argument("--B", type=int, default=None, help="reduced batch (profiling cases)")
     ap.add_argument("--indexer", default="per_head", choices=["per_head", "collapsed"],
                     help="indexer form (the pages' per-head work by default)")
+    ap.add_argument("--index-dtype", default="as_dtype", choices=["as_dtype", "e4m3"],
+                    help="indexer input type (the workload's dtype by default)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world, rank, local = dist_setup(args)
@@ -425,7 +436,7 @@ def main():
         pg = dist
 
     wl = Workload(args.config, dev, seed_offset=rank, S=args.S, T=args.T, B=args.B,
-                  indexer=args.indexer)
+                  indexer=args.indexer, index_dtype=args.index_dtype)
     cfg = wl.cfg
     nst = len(wl.stages)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
@@ -482,7 +493,9 @@ def main():
         bound, amount, unit = work[name]
         sec = stage_ms[j] / 1e3
         if bound == "tensor":
-            ach, peak = amount / sec / 1e12, tensor_peak
+            # e4m3 indexer operands: the bf16 figure times the nominal fp8:bf16 ratio of 2
+            scale = 2.0 if (name == "indexer" and wl.index_dtype == "e4m3") else 1.0
+            ach, peak = amount / sec / 1e12, tensor_peak * scale
         elif bound == "alu":
             ach, peak = amount / sec / 1e12, F32_SIMT_TFLOPS
         else:
@@ -551,7 +564,8 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32" if cfg.dtype == "f32" else "bf16", "data": "synthetic",
-            "config": dict(workload_config(cfg, wl.B), indexer_form=wl.indexer),
+            "config": dict(workload_config(cfg, wl.B), indexer_form=wl.indexer,
+                           indexer_dtype=wl.index_dtype),
             "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
             "clocks": clk, "gpu_launches": wl.launches_per_step * args.steps,
             "wall_ms_per_step_incl_flush": round(1e3 * t_wall / args.steps, 4),

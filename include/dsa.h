@@ -60,7 +60,12 @@ typedef enum {
   DSA_ERR_INTERNAL = 5     /* an in-kernel consistency check failed                     */
 } dsa_status;
 
-typedef enum { DSA_F32 = 0, DSA_BF16 = 1 } dsa_dtype;
+/* Element types.  DSA_E4M3 (float8 e4m3, 1 byte) is an indexer input type only: q_idx and
+ * k_idx of dsa_index_scores (and of dsa_forward through index_dtype). */
+typedef enum { DSA_F32 = 0, DSA_BF16 = 1, DSA_E4M3 = 2 } dsa_dtype;
+
+/* Element type of dsa_forward's indexer inputs: the attention dtype, or e4m3. */
+typedef enum { DSA_INDEX_AS_DTYPE = 0, DSA_INDEX_E4M3 = 1 } dsa_index_dtype;
 
 /* Where the indexer applies ReLU.  [AXK2] SGA prints the score as a plain weighted sum
  * (DSA_RELU_NONE, the default reading); its prose adds "then ReLU" after the weighted sum
@@ -98,6 +103,11 @@ typedef enum {
  *   the score is scale * sum_h w[h] * dot_h (float32).  With integer-valued inputs and a
  *   power-of-two scale (the synthetic workloads) every intermediate is exact.
  *   Requires 1 <= HI <= 256, 1 <= DI <= 128, T >= S.
+ *   dtype DSA_E4M3: q_idx and k_idx are float8 e4m3 (the upstream indexer's FP8 operands,
+ *   [AXK2] SGA notes; integers in [-2, 2] are exact in e4m3), products accumulated in
+ *   float32 on the tensor cores at twice the bf16 rate; HI in {16, 32}, DI == 128, else
+ *   DSA_ERR_UNSUPPORTED.  The Hadamard rotation the upstream applies before quantising is
+ *   the caller's (it is part of producing the inputs).
  * --------------------------------------------------------------------------------- */
 dsa_status dsa_index_scores(dsa_dtype dtype, const void* q_idx, const void* k_idx,
                             const float* w, float scale, dsa_relu_mode relu, int B, int S,
@@ -215,6 +225,8 @@ typedef struct {
                               attention (per-stage timing); NULL for none                */
   dsa_indexer_mode indexer; /* DSA_INDEXER_PER_HEAD (0, the pages' per-head work) or
                               DSA_INDEXER_COLLAPSED (the section 1b form)                */
+  dsa_index_dtype index_dtype; /* DSA_INDEX_AS_DTYPE (0): q_idx / k_idx have `dtype`;
+                              DSA_INDEX_E4M3: they are e4m3 (per-head indexer only)      */
 } dsa_forward_args;
 
 /* Bytes of workspace dsa_forward needs to run without row blocking. */

@@ -23,7 +23,7 @@ __all__ = [
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdsa.so")
 
-DTYPE = {torch.float32: 0, torch.bfloat16: 1}
+DTYPE = {torch.float32: 0, torch.bfloat16: 1, torch.float8_e4m3fn: 2}  # e4m3: indexer inputs
 RELU = {"none": 0, "post_sum": 1, "per_head": 2}
 GATE = {"off": 0, "sigmoid": 1, "silu": 2}
 ATTN_ALGO = {"auto": 0, "gather": 1, "masked_tile": 2}
@@ -50,6 +50,7 @@ class ForwardArgs(ctypes.Structure):
         ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
         ("gate", ctypes.c_void_p), ("out", ctypes.c_void_p), ("scores_out", ctypes.c_void_p),
         ("idx_out", ctypes.c_void_p), ("events", ctypes.c_void_p), ("indexer", ctypes.c_int),
+        ("index_dtype", ctypes.c_int),
     ]
 
 
@@ -252,7 +253,8 @@ def _forward_args(q_idx, k_idx, w, index_scale, K, q, k, v, gate, gate_mode, rel
         w=w.data_ptr(), q=q.data_ptr(), k=k.data_ptr(), v=v.data_ptr(),
         gate=None if gate is None else gate.data_ptr(), out=out.data_ptr(),
         scores_out=None if scores_out is None else scores_out.data_ptr(),
-        idx_out=None if idx_out is None else idx_out.data_ptr(), indexer=INDEXER[indexer])
+        idx_out=None if idx_out is None else idx_out.data_ptr(), indexer=INDEXER[indexer],
+        index_dtype=1 if q_idx.dtype == torch.float8_e4m3fn else 0)
     return a
 
 

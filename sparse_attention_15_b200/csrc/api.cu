@@ -37,7 +37,7 @@ dsa_status cuda_status(cudaError_t e, const char* what) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-size_t esize(dsa_dtype dt) { return dt == DSA_F32 ? 4 : 2; }
+size_t esize(dsa_dtype dt) { return dt == DSA_F32 ? 4 : (dt == DSA_E4M3 ? 1 : 2); }
 
 bool dim_ok(dsa_dtype dt, int d) { return d > 0 && d % (dt == DSA_F32 ? 4 : 8) == 0; }
 
@@ -51,8 +51,8 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 dsa_status check_index_args(dsa_dtype dtype, const void* q_idx, const void* k_idx,
                             const float* w, float scale, dsa_relu_mode relu, int B, int S,
                             int T, int HI, int DI, const void* scores) {
-  REQUIRE(dtype == DSA_F32 || dtype == DSA_BF16, DSA_ERR_INVALID_ARG, "unknown dtype %d",
-          (int)dtype);
+  REQUIRE(dtype == DSA_F32 || dtype == DSA_BF16 || dtype == DSA_E4M3, DSA_ERR_INVALID_ARG,
+          "unknown dtype %d", (int)dtype);
   REQUIRE(q_idx && k_idx && w && scores, DSA_ERR_INVALID_ARG, "null pointer argument");
   REQUIRE(B > 0 && S > 0 && T > 0 && HI > 0 && DI > 0, DSA_ERR_INVALID_ARG,
           "sizes must be positive (B=%d S=%d T=%d HI=%d DI=%d)", B, S, T, HI, DI);
@@ -65,6 +65,8 @@ dsa_status check_index_args(dsa_dtype dtype, const void* q_idx, const void* k_id
   REQUIRE(HI <= 256, DSA_ERR_UNSUPPORTED, "HI=%d > 256", HI);
   REQUIRE(DI <= 128 && dim_ok(dtype, DI), DSA_ERR_UNSUPPORTED,
           "DI=%d must be <= 128 and a multiple of %d", DI, dtype == DSA_F32 ? 4 : 8);
+  REQUIRE(dtype != DSA_E4M3 || dsa::index_scores_e4m3_supported(HI, DI), DSA_ERR_UNSUPPORTED,
+          "e4m3 indexer inputs need HI in {16,32} and DI == 128 (HI=%d DI=%d)", HI, DI);
   REQUIRE(S <= 65535 * 8, DSA_ERR_UNSUPPORTED, "S=%d too large", S);
   REQUIRE(B <= 65535, DSA_ERR_UNSUPPORTED, "B=%d too large", B);
   REQUIRE(aligned16(q_idx) && aligned16(k_idx) && aligned16(w) && aligned16(scores),
@@ -77,7 +79,10 @@ dsa_status run_index_scores(dsa_dtype dtype, const void* q_idx, const void* k_id
                             int T, int HI, int DI, int q_off, float* scores, int write_masked,
                             cudaStream_t st) {
   cudaError_t e;
-  if (dsa::index_scores_tc_supported((int)dtype, HI, DI))
+  if (dtype == DSA_E4M3)
+    e = dsa::launch_index_scores_e4m3(q_idx, k_idx, w, scale, (int)relu, B, S, T, HI, DI, q_off,
+                                      scores, write_masked, st);
+  else if (dsa::index_scores_tc_supported((int)dtype, HI, DI))
     e = dsa::launch_index_scores_tc(q_idx, k_idx, w, scale, (int)relu, B, S, T, HI, DI, q_off,
                                     scores, write_masked, st);
   else
@@ -337,9 +342,21 @@ dsa_status dsa_window_attn(dsa_dtype dtype, const void* q, const void* k, const 
 }
 
 // ----------------------------------------------------------------------------- forward
+// The element type of q_idx / k_idx: the attention dtype, or e4m3 when asked for.
+static dsa_dtype index_dtype(const dsa_forward_args* a) {
+  return a->index_dtype == DSA_INDEX_E4M3 ? DSA_E4M3 : a->dtype;
+}
+
 static dsa_status check_forward(const dsa_forward_args* a) {
   REQUIRE(a != nullptr, DSA_ERR_INVALID_ARG, "null args");
-  dsa_status st = check_index_args(a->dtype, a->q_idx, a->k_idx, a->w, a->index_scale, a->relu,
+  REQUIRE(a->index_dtype == DSA_INDEX_AS_DTYPE || a->index_dtype == DSA_INDEX_E4M3,
+          DSA_ERR_INVALID_ARG, "unknown index dtype %d", (int)a->index_dtype);
+  REQUIRE(a->dtype != DSA_E4M3, DSA_ERR_INVALID_ARG,
+          "e4m3 is an indexer input type (index_dtype), not an attention dtype");
+  REQUIRE(a->index_dtype != DSA_INDEX_E4M3 || a->indexer == DSA_INDEXER_PER_HEAD,
+          DSA_ERR_UNSUPPORTED, "the collapsed indexer takes bf16 inputs");
+  dsa_status st = check_index_args(index_dtype(a), a->q_idx, a->k_idx, a->w, a->index_scale,
+                                   a->relu,
                                    a->B, a->S, a->T, a->HI, a->DI,
                                    a->scores_out ? (const void*)a->scores_out : (const void*)a);
   if (st != DSA_OK) return st;
@@ -416,7 +433,7 @@ dsa_status dsa_forward(const dsa_forward_args* a, void* ws, size_t ws_bytes,
   const size_t attn_ws_bytes = L.mask_off - L.attn_off;
   uint32_t* mask = L.alg == kMasked ? reinterpret_cast<uint32_t*>(base + L.mask_off) : nullptr;
   const int B = a->B, S = a->S, T = a->T, q_off = T - S;
-  const size_t es = esize(a->dtype);
+  const size_t es = esize(index_dtype(a));  // q_idx / k_idx elements
   const int write_masked = a->scores_out != nullptr;  // -inf only matters to the caller
   cudaEvent_t const* ev = reinterpret_cast<cudaEvent_t const*>(a->events);
   auto mark = [&](int i) -> dsa_status {
@@ -431,9 +448,9 @@ dsa_status dsa_forward(const dsa_forward_args* a, void* ws, size_t ws_bytes,
     float* scores = a->scores_out ? a->scores_out : reinterpret_cast<float*>(base + L.scores_off);
     st = collapsed ? run_index_scores_collapsed(qc, a->k_idx, a->index_scale, a->relu, B, S, T,
                                                 a->DI, q_off, scores, write_masked, s)
-                   : run_index_scores(a->dtype, a->q_idx, a->k_idx, a->w, a->index_scale,
-                                      a->relu, B, S, T, a->HI, a->DI, q_off, scores,
-                                      write_masked, s);
+                   : run_index_scores(index_dtype(a), a->q_idx, a->k_idx, a->w,
+                                      a->index_scale, a->relu, B, S, T, a->HI, a->DI, q_off,
+                                      scores, write_masked, s);
     if (st != DSA_OK || (st = mark(1)) != DSA_OK) return st;
     st = cuda_status(dsa::launch_topk(scores, B, S, T, L.k_eff, q_off, idx, mask, L.mask_stride,
                                       s),
@@ -456,8 +473,8 @@ dsa_status dsa_forward(const dsa_forward_args* a, void* ws, size_t ws_bytes,
         const uint8_t* qcb = collapsed ? qc + ((size_t)b * S + s0) * 2 * a->DI * 2 : nullptr;
         st = collapsed ? run_index_scores_collapsed(qcb, ki, a->index_scale, a->relu, 1, n, T,
                                                     a->DI, q_off + s0, scores, 0, s)
-                       : run_index_scores(a->dtype, qi, ki, wb, a->index_scale, a->relu, 1, n,
-                                          T, a->HI, a->DI, q_off + s0, scores, 0, s);
+                       : run_index_scores(index_dtype(a), qi, ki, wb, a->index_scale, a->relu,
+                                          1, n, T, a->HI, a->DI, q_off + s0, scores, 0, s);
         if (st != DSA_OK) return st;
         const size_t row0 = (size_t)b * S + s0;
         st = cuda_status(dsa::launch_topk(scores, 1, n, T, L.k_eff, q_off + s0,

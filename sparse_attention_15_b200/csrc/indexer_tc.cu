@@ -53,13 +53,20 @@ struct TcArgs {
 
 // CL_: the head-collapsed form -- the B operand holds two bf16 rows per query (the hi and
 // lo parts of sum_h w[s,h] q_I[s,h,:]) and a score is the sum of its two columns.
-template <int HI_, int DI_, int NQ_, int NE_, int NA_, int NB_ = 2, bool CL_ = false>
+// ES_: operand element bytes, 2 (bf16, kind::f16) or 1 (e4m3, kind::f8f6f4).  Every MMA
+// consumes 32 bytes of each 128-byte swizzled row either way, so the shared-memory layout
+// and the descriptor arithmetic are the same in bytes.
+template <int HI_, int DI_, int NQ_, int NE_, int NA_, int NB_ = 2, bool CL_ = false,
+          int ES_ = 2>
 struct TcCfg {
   static constexpr int HI = HI_, DI = DI_, NQ = NQ_, NE = NE_, NA = NA_;
   static constexpr bool CL = CL_;
+  static constexpr int ES = ES_;
+  static constexpr int ROW_BYTES = DI * ES;       // one operand row
+  static constexpr int SLICE_ELEMS = 128 / ES;    // elements per 128-byte swizzle row
   static constexpr int NB = NB_;                  // query-block buffers (1 or 2)
   static constexpr int N = NQ * HI;               // MMA N: (query, head) columns
-  static constexpr int KH = DI / 64;              // 64-element (128-byte) K slices
+  static constexpr int KH = ROW_BYTES / 128;      // 128-byte K slices
   static constexpr int A_SLICE = kTileM * 128;    // bytes of one K slice of a key tile
   static constexpr int A_BYTES = KH * A_SLICE;
   static constexpr int B_SLICE = N * 128;
@@ -77,7 +84,8 @@ struct TcCfg {
   static_assert(!CL || HI == 2, "the collapsed form has two columns (hi, lo) per query");
   static_assert(CL || HI >= 16, "per-head epilogue: a query spans whole 16-column chunks");
   static_assert(COLS_PER_WARP % 32 == 0 && COLS_PER_WARP % HI == 0, "epilogue chunking");
-  static_assert(DI % 64 == 0, "DI must be a multiple of 64");
+  static_assert(ROW_BYTES % 128 == 0, "operand rows must be whole 128-byte slices");
+  static_assert(ES == 2 || (ES == 1 && !CL), "e4m3 operands: per-head form only");
 };
 
 // This CTA's work units.  Unit u = (b * nqb + qb) * max_chunks + c covers key tiles
@@ -180,7 +188,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         const int qrow = (it.b * a.S + it.qb * C::NQ) * C::HI;
 #pragma unroll
         for (int kh = 0; kh < C::KH; ++kh)
-          tma_load_2d(Bs + bb * C::B_BYTES + kh * C::B_SLICE, &qmap, kh * 64, qrow, &b_full[bb]);
+          tma_load_2d(Bs + bb * C::B_BYTES + kh * C::B_SLICE, &qmap, kh * C::SLICE_ELEMS, qrow,
+                      &b_full[bb]);
         ++bi;
         for (int kt = it.k0; kt < it.k1; ++kt) {
           const int st = ai % C::NA;
@@ -192,7 +201,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           const int krow = it.b * a.T + kt * kTileM;
 #pragma unroll
           for (int kh = 0; kh < C::KH; ++kh)
-            tma_load_2d(As + st * C::A_BYTES + kh * C::A_SLICE, &kmap, kh * 64, krow,
+            tma_load_2d(As + st * C::A_BYTES + kh * C::A_SLICE, &kmap, kh * C::SLICE_ELEMS, krow,
                         &a_full[st]);
           ++ai;
         }
@@ -206,7 +215,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(kTileM, C::N);
+      constexpr uint32_t idesc =
+          C::ES == 2 ? idesc_bf16_f32(kTileM, C::N) : idesc_e4m3_f32(kTileM, C::N);
       UnitIter it(cta);
       uint32_t ai = 0, bi = 0, ci = 0;
       bool ok = true;
@@ -222,11 +232,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           tc_fence_after();
           const uint32_t a_base = smem_u32(As + st * C::A_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < C::DI / 16; ++kk) {
-            const uint32_t off = (kk & 3) * 32;  // 16 bf16 = 32 B along the swizzled row
+          for (int kk = 0; kk < C::ROW_BYTES / 32; ++kk) {
+            const uint32_t off = (kk & 3) * 32;  // 32 B (16 bf16 / 32 e4m3) along the row
             const uint64_t adesc = sw128_kmajor_desc(a_base + (kk >> 2) * C::A_SLICE + off);
             const uint64_t bdesc = sw128_kmajor_desc(b_base + (kk >> 2) * C::B_SLICE + off);
-            umma_f16_ss(tmem + ab * C::ACC_COLS, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+            if constexpr (C::ES == 2)
+              umma_f16_ss(tmem + ab * C::ACC_COLS, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+            else
+              umma_f8f6f4_ss(tmem + ab * C::ACC_COLS, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
           }
           umma_commit(&a_empty[st]);
           umma_commit(&acc_full[ab]);
@@ -422,16 +435,19 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
-// 2-D bf16 tensor map over a [rows, cols] row-major matrix, box [box_cols, box_rows],
-// 128-byte swizzle (box_cols * 2 must be 128).
-bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+// 2-D tensor map over a [rows, cols] row-major matrix of `es`-byte elements (bf16 or
+// e4m3 bytes), box [128 bytes of columns, box_rows], 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+              int es = 2) {
   auto enc = get_encode();
   if (!enc) return false;
   cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * 2};
-  cuuint32_t box[2] = {64, box_rows};
+  cuuint64_t strides[1] = {cols * (uint64_t)es};
+  cuuint32_t box[2] = {(cuuint32_t)(128 / es), box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+  const CUtensorMapDataType dt =
+      es == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  CUresult r = enc(m, dt, 2, const_cast<void*>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -449,8 +465,10 @@ cudaError_t launch_cfg(const void* q_idx, const void* k_idx, const float* w, flo
                        int relu, int B, int S, int T, int q_off, float* scores,
                        int write_masked, cudaStream_t st) {
   CUtensorMap kmap, qmap;
-  if (!make_map(&kmap, k_idx, (uint64_t)B * T, C::DI, kTileM)) return cudaErrorInvalidValue;
-  if (!make_map(&qmap, q_idx, (uint64_t)B * S * C::HI, C::DI, C::N)) return cudaErrorInvalidValue;
+  if (!make_map(&kmap, k_idx, (uint64_t)B * T, C::DI, kTileM, C::ES))
+    return cudaErrorInvalidValue;
+  if (!make_map(&qmap, q_idx, (uint64_t)B * S * C::HI, C::DI, C::N, C::ES))
+    return cudaErrorInvalidValue;
   TcArgs a{};
   a.w = w; a.scores = scores; a.scale = scale; a.B = B; a.S = S; a.T = T; a.q_off = q_off;
   a.nqb = (S + C::NQ - 1) / C::NQ;
@@ -489,6 +507,31 @@ cudaError_t launch_cfg(const void* q_idx, const void* k_idx, const float* w, flo
 }
 
 }  // namespace
+
+bool index_scores_e4m3_supported(int HI, int DI) {
+  return (HI == 16 || HI == 32) && DI == 128;
+}
+
+cudaError_t launch_index_scores_e4m3(const void* q_idx, const void* k_idx, const float* w,
+                                     float scale, int relu, int B, int S, int T, int HI, int DI,
+                                     int q_off, float* scores, int write_masked,
+                                     cudaStream_t st) {
+  if (!index_scores_e4m3_supported(HI, DI)) return cudaErrorNotSupported;
+  // one 128-byte slice per operand row: half the shared memory of the bf16 tiles, so the
+  // key ring is deeper
+  if (S == 1) {
+    if (HI == 32)
+      return launch_cfg<TcCfg<32, 128, 1, 4, 8, 2, false, 1>>(q_idx, k_idx, w, scale, relu, B, S,
+                                                              T, q_off, scores, write_masked, st);
+    return launch_cfg<TcCfg<16, 128, 2, 4, 8, 2, false, 1>>(q_idx, k_idx, w, scale, relu, B, S, T,
+                                                            q_off, scores, write_masked, st);
+  }
+  if (HI == 32)
+    return launch_cfg<TcCfg<32, 128, 8, 16, 6, 2, false, 1>>(q_idx, k_idx, w, scale, relu, B, S,
+                                                             T, q_off, scores, write_masked, st);
+  return launch_cfg<TcCfg<16, 128, 16, 16, 6, 2, false, 1>>(q_idx, k_idx, w, scale, relu, B, S, T,
+                                                            q_off, scores, write_masked, st);
+}
 
 bool index_scores_collapsed_supported(int dtype, int DI, int relu) {
   return dtype == 1 && (DI == 64 || DI == 128) && relu != 2;

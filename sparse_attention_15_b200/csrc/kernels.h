@@ -25,6 +25,13 @@ cudaError_t launch_index_scores_tc(const void* q_idx, const void* k_idx, const f
                                    int q_off, float* scores, int write_masked,
                                    cudaStream_t st);
 
+// Indexer scores with e4m3 operands (tcgen05 kind::f8f6f4): HI in {16, 32}, DI == 128.
+bool index_scores_e4m3_supported(int HI, int DI);
+cudaError_t launch_index_scores_e4m3(const void* q_idx, const void* k_idx, const float* w,
+                                     float scale, int relu, int B, int S, int T, int HI, int DI,
+                                     int q_off, float* scores, int write_masked,
+                                     cudaStream_t st);
+
 // Head-collapsed indexer (valid when no ReLU is applied per head: the score is linear in
 // q_I): launch_collapse_q writes qc [rows, 2, DI] bf16 (hi and lo parts of
 // sum_h w[s,h] q_I[s,h,:]); launch_index_scores_collapsed scores k_I against them on the

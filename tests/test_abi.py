@@ -64,6 +64,9 @@ def test_index_scores_rejects_bad_arguments(lib):
     assert _index(L, DI=256) == 2
     assert _index(L, q=FAKE_MIS) == 2        # misaligned
     assert b"16-byte" in L.dsa_last_error()
+    assert _index(L, dtype=2, HI=16, DI=64) == 2   # e4m3 needs DI == 128
+    assert b"e4m3" in L.dsa_last_error()
+    assert _index(L, dtype=2, HI=8, DI=128) == 2   # and HI in {16, 32}
 
 
 def _collapsed(L, ws_bytes=1 << 20, **kw):
@@ -167,6 +170,13 @@ def test_forward_workspace_and_validation(lib):
     assert lib.dsa_forward_workspace_bytes(a, minimum=True) == small + 4096 * 2 * 64 * 2
     a.relu = 2
     assert L.dsa_forward(ctypes.byref(a), FAKE, full_c, None) == 2
+    a.relu = 0
+    a.index_dtype = 1  # e4m3 indexer inputs: per-head indexer only, DI == 128
+    assert L.dsa_forward(ctypes.byref(a), FAKE, full_c, None) == 2
+    a.indexer = 0
+    assert L.dsa_forward(ctypes.byref(a), FAKE, full, None) == 2  # DI = 64
+    a.index_dtype = 5
+    assert L.dsa_forward(ctypes.byref(a), FAKE, full, None) == 1
 
 
 def test_binding_fails_loudly_without_library(monkeypatch):

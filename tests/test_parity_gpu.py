@@ -48,6 +48,59 @@ def test_index_scores_exact(name, S, T, relu):
     assert np.array_equal(P.to_np(got), ref.astype(np.float32))
 
 
+# --------------------------------------------------------------- indexer, e4m3 operands
+E4M3 = [("c3", 200, 455), ("c5", 131, 300), ("c3", 1, 700), ("c3", 3, 2000)]
+
+
+def _e4m3(t):
+    return t.to(torch.float8_e4m3fn)
+
+
+@pytest.mark.parametrize("name,S,T", E4M3)
+@pytest.mark.parametrize("relu", ["none", "post_sum", "per_head"])
+def test_index_scores_e4m3_exact(name, S, T, relu):
+    # integers in [-2, 2] are exact in e4m3: the scores equal the oracle's bit for bit
+    cfg, x, g = _inputs(name, S, T)
+    qi, ki = _e4m3(x["q_idx"]), _e4m3(x["k_idx"])
+    assert torch.equal(qi.float(), x["q_idx"].float())
+    got = dsa.dsa_index_scores(qi.to(DEV), ki.to(DEV), g["w"], cfg.scale, relu=relu)
+    ref = O.index_scores(x["q_idx"], x["k_idx"], x["w"], cfg.scale, relu=relu)
+    assert np.array_equal(P.to_np(got), ref.astype(np.float32))
+
+
+def test_index_scores_e4m3_real_valued_inputs():
+    # arbitrary e4m3 values: every product of two e4m3 numbers is exact in float32, so the
+    # only error is the float32 accumulation over DI terms and HI heads:
+    # |err| <= 2^-16 * scale * sum_h |w_h| sum_d |q_hd k_d| is a safe bound
+    g = torch.Generator().manual_seed(11)
+    B, S, T, HI, DI = 1, 257, 390, 16, 128
+    qi = _e4m3(torch.randn(B, S, HI, DI, generator=g) * 3.0)
+    ki = _e4m3(torch.randn(B, T, DI, generator=g) * 3.0)
+    w = torch.rand(B, S, HI, generator=g) * 2.0
+    scale = 0.0883
+    got = dsa.dsa_index_scores(qi.to(DEV), ki.to(DEV), w.to(DEV), scale)
+    ref = O.index_scores(qi, ki, w, scale)
+    aq, ak, aw = (np.abs(t.double().numpy()) for t in (qi, ki, w))
+    mag = scale * np.einsum("bsh,bshd,btd->bst", aw, aq, ak)
+    got_np = P.to_np(got).astype(np.float64)
+    causal = np.isfinite(ref)
+    assert np.array_equal(np.isfinite(got_np), causal)
+    err = np.abs(got_np[causal] - ref[causal])
+    assert np.all(err <= 2.0 ** -16 * mag[causal] + 1e-30), float((err / mag[causal]).max())
+
+
+@pytest.mark.parametrize("name,S,T", [("c3", 260, 330), ("c3", 1, 900)])
+def test_forward_e4m3_indexer_matches_bf16(name, S, T):
+    cfg, x, g = _inputs(name, S, T, B=2 if S == 1 else 1)
+    K = min(cfg.K, 96)
+    out1, idx1 = dsa.dsa_forward(g["q_idx"], g["k_idx"], g["w"], cfg.scale, K, g["q"], g["k"],
+                                 g["v"], gate=g["gate"])
+    out2, idx2 = dsa.dsa_forward(_e4m3(g["q_idx"]), _e4m3(g["k_idx"]), g["w"], cfg.scale, K,
+                                 g["q"], g["k"], g["v"], gate=g["gate"])
+    assert torch.equal(idx1, idx2)
+    assert torch.equal(out1, out2)
+
+
 # --------------------------------------------------------------- indexer, head-collapsed form
 COLLAPSED = [("c2", 333, 333), ("c2", 100, 517), ("c3", 200, 455), ("c5", 131, 300),
              ("c3", 1, 700)]
