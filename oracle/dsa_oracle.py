@@ -142,7 +142,8 @@ def apply_gate(o, g, gate_mode="sigmoid"):
     return o * _gate_factor(g, gate_mode)[..., None]
 
 
-def sparse_attention(q, k, v, idx, sm_scale=None, gate=None, gate_mode="off", q_off=None):
+def sparse_attention(q, k, v, idx, sm_scale=None, gate=None, gate_mode="off", q_off=None,
+                     sink_k=None, sink_v=None):
     """Attention over the indexer-selected keys, by dense masked softmax.
 
     [AXK2] "注意力前向的骨架": the selected positions become an additive sparse mask that
@@ -153,11 +154,20 @@ def sparse_attention(q, k, v, idx, sm_scale=None, gate=None, gate_mode="off", q_
 
     q [B,S,H,Dqk], k [B,T,H,Dqk], v [B,T,H,Dv], idx [B,S,K] (entries outside [0,T) or
     equal to -1 are ignored).  Returns float64 [B,S,H,Dv].
+
+    Optional attention sinks, [PANGU] §3.4 (PAS): a layer's learnable key-value pairs
+    act at inference as a fixed set of virtual KV entries that every query sees.  sink_k
+    [NS,H,Dqk] and sink_v [NS,H,Dv] (the per-head form, like the expanded cache) join the
+    softmax of every query, unmasked, beside its selected keys.
     """
     q = _f64(q)
     k = _f64(k)
     v = _f64(v)
     idx = np.asarray(idx)
+    sinks = sink_k is not None
+    if sinks:
+        sk = _f64(sink_k).transpose(1, 0, 2)  # [H,NS,Dqk]
+        sv = _f64(sink_v).transpose(1, 0, 2)  # [H,NS,Dv]
     B, S, H, Dqk = q.shape
     T = k.shape[1]
     if q_off is None:
@@ -174,14 +184,19 @@ def sparse_attention(q, k, v, idx, sm_scale=None, gate=None, gate_mode="off", q_
             sel = sel[(sel >= 0) & (sel < T)]
             allowed[sel] = True
             allowed[np.arange(T) > s + q_off] = False  # the causal mask
-            if not allowed.any():
+            if not allowed.any() and not sinks:
                 continue
             logits = sm_scale * np.matmul(kt, q[b, s][:, :, None])[:, :, 0]  # [H,T]
             logits[:, ~allowed] = -np.inf
+            vals = vt
+            if sinks:  # the sink entries, always visible
+                sl = sm_scale * np.matmul(sk, q[b, s][:, :, None])[:, :, 0]  # [H,NS]
+                logits = np.concatenate([logits, sl], axis=1)
+                vals = np.concatenate([vt, sv], axis=1)
             m = logits.max(axis=1, keepdims=True)
             p = np.exp(logits - m)
             p /= p.sum(axis=1, keepdims=True)
-            out[b, s] = np.matmul(p[:, None, :], vt)[:, 0, :]
+            out[b, s] = np.matmul(p[:, None, :], vals)[:, 0, :]
     if gate_mode != "off":
         out = apply_gate(out, gate, gate_mode)
     return out
@@ -230,15 +245,16 @@ def window_attention(q, k, v, window, sm_scale=None, gate=None, gate_mode="off",
 
 
 def dsa_forward(q_idx, k_idx, w, scale, K, q, k, v, sm_scale=None, gate=None,
-                gate_mode="off", relu="none", q_off=None):
+                gate_mode="off", relu="none", q_off=None, sink_k=None, sink_v=None):
     """The whole DSA step: indexer scores -> top-k -> sparse attention -> gate.
 
-    [AXK2] "注意力前向的骨架" steps 4-5 and the SGA section; [PANGU] §3.3.
+    [AXK2] "注意力前向的骨架" steps 4-5 and the SGA section; [PANGU] §3.3 (and §3.4 for
+    the optional sinks).
     Returns (scores float64 [B,S,T], idx int32 [B,S,min(K,T)], out float64 [B,S,H,Dv]).
     """
     T = _f64(k_idx).shape[1] if not hasattr(k_idx, "shape") else k_idx.shape[1]
     scores = index_scores(q_idx, k_idx, w, scale, relu=relu, q_off=q_off)
     idx = topk_indices(scores, min(K, T), q_off=q_off)
     out = sparse_attention(q, k, v, idx, sm_scale=sm_scale, gate=gate,
-                           gate_mode=gate_mode, q_off=q_off)
+                           gate_mode=gate_mode, q_off=q_off, sink_k=sink_k, sink_v=sink_v)
     return scores, idx, out

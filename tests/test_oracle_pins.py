@@ -184,6 +184,56 @@ def test_attention_two_keys_hand_worked():
     assert np.array_equal(outs, np.array(g["out_silu_gate_0"]))
 
 
+def test_attention_sinks_hand_worked():
+    g = _load("attention_sink.json")
+    q, k, v = (np.array(g[n]) for n in ("q", "k", "v"))
+    sk, sv = np.array(g["sink_k"]), np.array(g["sink_v"])
+    out = O.sparse_attention(q, k, v, np.array(g["idx"], dtype=np.int32), sm_scale=1.0,
+                             sink_k=sk, sink_v=sv)
+    assert np.allclose(out, np.array(g["out"]), rtol=0, atol=1e-12)
+    out0 = O.sparse_attention(q, k, v, np.array(g["idx_none"], dtype=np.int32), sm_scale=1.0,
+                              sink_k=sk, sink_v=sv)
+    assert np.allclose(out0, np.array(g["out_sinks_only"]), rtol=0, atol=1e-12)
+
+
+def test_attention_sinks_library_special_cases():
+    # (1) with no selected key the result is plain SDPA of the query over the sink entries;
+    # (2) a sink that copies a selected key equals SDPA with that key listed twice;
+    # (3) sinks far below every logit change nothing; (4) the order of the sinks does not matter
+    rng = np.random.default_rng(5)
+    B, S, T, H, D, DV, NS = 1, 5, 9, 3, 8, 6, 4
+    q, k = rng.standard_normal((B, S, H, D)), rng.standard_normal((B, T, H, D))
+    v = rng.standard_normal((B, T, H, DV))
+    sk, sv = rng.standard_normal((NS, H, D)), rng.standard_normal((NS, H, DV))
+    # (1)
+    none = -np.ones((B, S, 2), dtype=np.int32)
+    got = O.sparse_attention(q, k, v, none, sink_k=sk, sink_v=sv)
+    ref = _sdpa_f64(q, np.ascontiguousarray(np.broadcast_to(sk[None], (B, NS, H, D))),
+                    np.ascontiguousarray(np.broadcast_to(sv[None], (B, NS, H, DV))),
+                    causal=False)
+    assert np.allclose(got, ref, rtol=0, atol=1e-12)
+    # (2) every query selects keys 0 and 3 (3 only where causal: q_off = 4); the one sink
+    # is a copy of key 3, always visible
+    idx = np.stack([np.zeros((B, S), np.int32), np.full((B, S), 3, np.int32)], axis=-1)
+    got = O.sparse_attention(q, k, v, idx, sink_k=k[0, 3:4], sink_v=v[0, 3:4])
+    for s in range(S):
+        keys = [0, 3, 3] if s + (T - S) >= 3 else [0, 3]
+        ref = _sdpa_f64(q[:, s:s + 1], k[:, keys], v[:, keys], causal=False)
+        assert np.allclose(got[:, s:s + 1], ref, rtol=0, atol=1e-12)
+    # (3) positive queries and sink keys of -1e3: logits below the others by > 1e3 (keys
+    # 0..4 are visible to every query, q_off = 4, so no row is left to the sinks alone)
+    sel = rng.integers(0, T - S + 1, (B, S, 4)).astype(np.int32)
+    qq = np.abs(q) + 1.0
+    got = O.sparse_attention(qq, k, v, sel, sink_k=np.full((NS, H, D), -1e3),
+                             sink_v=np.full((NS, H, DV), 1e6))
+    assert np.array_equal(got, O.sparse_attention(qq, k, v, sel))
+    # (4)
+    perm = rng.permutation(NS)
+    a = O.sparse_attention(q, k, v, sel, sink_k=sk, sink_v=sv)
+    b = O.sparse_attention(q, k, v, sel, sink_k=sk[perm], sink_v=sv[perm])
+    assert np.allclose(a, b, rtol=0, atol=1e-13)
+
+
 def _sdpa_f64(q, k, v, causal=True, mask=None, scale=None):
     """torch's CPU float64 SDPA, [B,S,H,D] layout in and out."""
     tq, tk, tv = (torch.from_numpy(np.ascontiguousarray(x)).transpose(1, 2) for x in (q, k, v))
