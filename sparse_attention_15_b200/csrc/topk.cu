@@ -67,14 +67,8 @@ template <int NT>
 __device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t digit, bool valid) {
   // Plain shared-memory atomics: equal digits within a warp serialise in the atomic unit,
   // which costs less than grouping them first (__match_any_sync occupies the XU pipe for
-  // many cycles per call).  A warp whose 32 digits are all equal adds once.
-  const uint32_t d = valid ? digit : 0xffffffffu;
-  const uint32_t d0 = __shfl_sync(0xffffffffu, d, 0);
-  if (__all_sync(0xffffffffu, d == d0)) {
-    if ((threadIdx.x & 31) == 0 && valid) atomicAdd(&hist[hpad(d)], 32u);
-  } else if (valid) {
-    atomicAdd(&hist[hpad(d)], 1u);
-  }
+  // many cycles per call).
+  if (valid) atomicAdd(&hist[hpad(digit)], 1u);
 }
 
 template <int NT>
@@ -91,7 +85,7 @@ __global__ void __launch_bounds__(NT) topk_rows_kernel(const float* __restrict__
   __shared__ int wgt[NT / 32], weq[NT / 32];
 
   const size_t row = blockIdx.x;
-  const int s = (int)(row % (size_t)S);
+  const int s = (int)(blockIdx.x % (unsigned)S);  // 32-bit: rows < 2^31
   const int n = min(Tn, s + q_off + 1);
   const float* sc = scores + row * (size_t)Tn;
   int32_t* out = idx + row * (size_t)K;
@@ -228,23 +222,29 @@ constexpr int kBins1 = 4096;  // top 12 bits
 constexpr int kBins2 = 1024;  // 10-bit refinement digits
 
 // Bucket holding the need-th largest key: writes (bin, count above it, its count) to
-// out[0..2].
-template <int NT>
-__device__ __forceinline__ void find_bucket(const uint32_t* hist, int nbins, int need,
-                                            int* warp_buf, int* scan_total, int* out) {
-  const int per = nbins / NT;
-  const int hi_bin = nbins - threadIdx.x * per;
+// out[0..2].  Each thread owns a run of NBINS/NT bins, highest first; the counts stay in
+// registers across the block scan.
+template <int NT, int NBINS>
+__device__ __forceinline__ void find_bucket(const uint32_t* hist, int need, int* warp_buf,
+                                            int* scan_total, int* out) {
+  constexpr int per = NBINS / NT;
+  const int hi_bin = NBINS - threadIdx.x * per;
+  int c[per];
   int local = 0;
-  for (int q = 1; q <= per; ++q) local += (int)hist[hpad(hi_bin - q)];
+#pragma unroll
+  for (int q = 0; q < per; ++q) {
+    c[q] = (int)hist[hpad(hi_bin - 1 - q)];
+    local += c[q];
+  }
   int above = block_excl_scan(local, warp_buf, scan_total);
-  for (int q = 1; q <= per; ++q) {
-    const int c = (int)hist[hpad(hi_bin - q)];
-    if (above < need && above + c >= need) {
-      out[0] = hi_bin - q;
+#pragma unroll
+  for (int q = 0; q < per; ++q) {
+    if (above < need && above + c[q] >= need) {
+      out[0] = hi_bin - 1 - q;
       out[1] = above;
-      out[2] = c;
+      out[2] = c[q];
     }
-    above += c;
+    above += c[q];
   }
 }
 
@@ -305,7 +305,7 @@ __global__ void __launch_bounds__(NT, NT == 256 ? 5 : (NT == 512 ? 3 : 1))
   __shared__ int cnt_sel, cl_n;
 
   const size_t row = blockIdx.x;
-  const int s = (int)(row % (size_t)S);
+  const int s = (int)(blockIdx.x % (unsigned)S);  // 32-bit: rows < 2^31
   const int n = min(Tn, s + q_off + 1);
   const float* sc = scores + row * (size_t)Tn;
   int32_t* out = idx + row * (size_t)K;
@@ -348,7 +348,7 @@ __global__ void __launch_bounds__(NT, NT == 256 ? 5 : (NT == 512 ? 3 : 1))
     }
     held = n <= kChunk;
     __syncthreads();
-    find_bucket<NT>(hist, kBins1, K, warp_buf, &scan_total, pick);
+    find_bucket<NT, kBins1>(hist, K, warp_buf, &scan_total, pick);
     __syncthreads();
     b1 = (uint32_t)pick[0];
     need = K - pick[1];
@@ -428,10 +428,10 @@ __global__ void __launch_bounds__(NT, NT == 256 ? 5 : (NT == 512 ? 3 : 1))
     const float ks = (float)K * (float)ns / (float)n;
     const int delta = (int)(3.0f * sqrtf(ks) + 2.0f);
     const int r_hi = max(1, (int)ks - delta), r_lo = min(ns, (int)ks + delta + 1);
-    find_bucket<NT>(hist, kBins1, r_hi, warp_buf, &scan_total, pick);
+    find_bucket<NT, kBins1>(hist, r_hi, warp_buf, &scan_total, pick);
     __syncthreads();
     const uint32_t b_hi = (uint32_t)pick[0];
-    find_bucket<NT>(hist, kBins1, r_lo, warp_buf, &scan_total, pick);
+    find_bucket<NT, kBins1>(hist, r_lo, warp_buf, &scan_total, pick);
     __syncthreads();
     const uint32_t b_lo = (uint32_t)pick[0];
     for (int i = tid; i < padded(kBins1); i += NT) hist[i] = 0u;
@@ -463,7 +463,7 @@ __global__ void __launch_bounds__(NT, NT == 256 ? 5 : (NT == 512 ? 3 : 1))
         }
       }
       __syncthreads();
-      find_bucket<NT>(hist, kBins1, K - nsel, warp_buf, &scan_total, pick);
+      find_bucket<NT, kBins1>(hist, K - nsel, warp_buf, &scan_total, pick);
       __syncthreads();
       b1 = (uint32_t)pick[0];
       need = K - nsel - pick[1];
@@ -531,7 +531,7 @@ __global__ void __launch_bounds__(NT, NT == 256 ? 5 : (NT == 512 ? 3 : 1))
         }
       }
       __syncthreads();
-      find_bucket<NT>(hist, kBins2, need, warp_buf, &scan_total, pick);
+      find_bucket<NT, kBins2>(hist, need, warp_buf, &scan_total, pick);
       __syncthreads();
       const uint32_t bsel = (uint32_t)pick[0];
       need -= pick[1];
@@ -619,7 +619,7 @@ __global__ void __launch_bounds__(NT, NT == 256 ? 5 : (NT == 512 ? 3 : 1))
 __global__ void idx_to_mask_kernel(const int32_t* __restrict__ idx, int S, int Tn, int K,
                                    int q_off, uint32_t* __restrict__ mask, int stride) {
   const size_t row = blockIdx.x;
-  const int spos = (int)(row % (size_t)S) + q_off;
+  const int spos = (int)(blockIdx.x % (unsigned)S) + q_off;
   uint32_t* m = mask + row * (size_t)stride;
   for (int w = threadIdx.x; w < stride; w += blockDim.x) m[w] = 0u;
   __syncthreads();
@@ -650,7 +650,9 @@ cudaError_t launch_topk(const float* scores, int B, int S, int T, int K, int q_o
   // the bitmaps are large; the list overflowing only costs re-reads through the bitmap).
   const int W = (T + 31) / 32;
   int cap = T > 8192 ? 2048 : 1024;
-  auto smem_for = [&](int c) { return (size_t)(padded(kBins1) + 2 * W + 2 * c) * sizeof(uint32_t); };
+  auto smem_for = [&](int c) {
+    return (size_t)(padded(kBins1) + 2 * W + 2 * c) * sizeof(uint32_t);
+  };
   if (smem_for(cap) > kMaxDynSmem) cap = 512;
   if (T <= kMaxBitmapKeys && smem_for(cap) <= kMaxDynSmem) {
     // one CTA per row; small CTAs so that several rows are in flight per SM (each row is a
