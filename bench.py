@@ -164,7 +164,7 @@ class Workload:
     """Device buffers and the library calls of one step of config `name`."""
 
     def __init__(self, name, device, seed_offset=0, S=None, T=None, B=None, indexer="per_head",
-                 index_dtype="as_dtype"):
+                 index_dtype="as_dtype", nsink=0):
         import dataclasses
 
         import sparse_attention_15_b200 as dsa
@@ -194,6 +194,14 @@ class Workload:
             x["q_idx"] = x["q_idx"].to(torch.float8_e4m3fn)
             x["k_idx"] = x["k_idx"].to(torch.float8_e4m3fn)
         self.x = x
+        self.nsink = nsink
+        self.sink_k = self.sink_v = None
+        if nsink:  # attention sinks (PAS): synthetic per-head sink rows, N(0,1)
+            g = torch.Generator(device="cpu").manual_seed(cfg.seed + 7919)
+            self.sink_k = torch.randn(nsink, cfg.H, cfg.dqk, generator=g).to(
+                x["q"].dtype).to(device)
+            self.sink_v = torch.randn(nsink, cfg.H, cfg.dv, generator=g).to(
+                x["q"].dtype).to(device)
         self.K = cfg.k_eff
         self.idx = torch.empty((B, cfg.S, self.K), dtype=torch.int32, device=device)
         self.out = torch.empty((B, cfg.S, cfg.H, cfg.dv), dtype=x["q"].dtype, device=device)
@@ -201,7 +209,7 @@ class Workload:
         self.args = dsa._forward_args(x["q_idx"], x["k_idx"], x["w"], cfg.scale, cfg.K, x["q"],
                                       x["k"], x["v"], x["gate"], None, "none", 0.0, "auto",
                                       self.out, None, self.idx,
-                                      indexer)
+                                      indexer, self.sink_k, self.sink_v)
         self.ws_bytes = dsa.dsa_forward_workspace_bytes(self.args)
         self.ws = torch.empty(max(self.ws_bytes, 16), dtype=torch.uint8, device=device)
         dt = dsa.DTYPE[x["q"].dtype]
@@ -225,7 +233,8 @@ class Workload:
         c, x, d = self.cfg, self.x, self.dsa
         d.dsa_forward(x["q_idx"], x["k_idx"], x["w"], c.scale, c.K, x["q"], x["k"], x["v"],
                       gate=x["gate"], out=self.out, idx_out=self.idx, ws=self.ws,
-                      ws_bytes=self.ws_bytes, events=ev[:4], indexer=self.indexer)
+                      ws_bytes=self.ws_bytes, events=ev[:4], indexer=self.indexer,
+                      sink_k=self.sink_k, sink_v=self.sink_v)
         for i, s in enumerate(self.swa):
             d.dsa_window_attn(s["q"], s["k"], s["v"], c.window, gate=s["gate"], out=s["out"])
             ev[4 + i].record()
@@ -257,9 +266,11 @@ class Workload:
         }
         if self.algo == "masked_tile":
             # dense attention under the mask: QK^T and PV over every causal pair, all heads
-            w["attention"] = ("tensor", 2.0 * c.H * (c.dqk + c.dv) * pairs, "TFLOP/s")
+            # (+ every query against the sinks)
+            w["attention"] = ("tensor", 2.0 * c.H * (c.dqk + c.dv) * (pairs + rows * self.nsink),
+                              "TFLOP/s")
         else:
-            w["attention"] = ("hbm", sel * c.H * (c.dqk + c.dv) * es +
+            w["attention"] = ("hbm", (sel + rows * self.nsink) * c.H * (c.dqk + c.dv) * es +
                               rows * c.H * (c.dqk + c.dv) * es, "GB/s")
         for i in range(len(self.swa)):
             band = selected_pairs(c.S, c.T, B, c.q_off, c.window)
@@ -295,7 +306,8 @@ class Workload:
         c = self.cfg
         self.dsa.dsa_forward(x["q_idx"], x["k_idx"], x["w"], c.scale, c.K, x["q"], x["k"],
                              x["v"], gate=x["gate"], out=self.out, idx_out=self.idx,
-                             ws=self.ws, ws_bytes=self.ws_bytes, indexer=self.indexer)
+                             ws=self.ws, ws_bytes=self.ws_bytes, indexer=self.indexer,
+                             sink_k=self.sink_k, sink_v=self.sink_v)
         out_host.copy_(self.out, non_blocking=True)
 
 
@@ -412,6 +424,8 @@ def main():
                     help="indexer form (the pages' per-head work by default)")
     ap.add_argument("--index-dtype", default="as_dtype", choices=["as_dtype", "e4m3"],
                     help="indexer input type (the workload's dtype by default)")
+    ap.add_argument("--sinks", type=int, default=0,
+                    help="attention sinks (PAS virtual KV entries) per layer, 0..128")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world, rank, local = dist_setup(args)
@@ -436,7 +450,7 @@ def main():
         pg = dist
 
     wl = Workload(args.config, dev, seed_offset=rank, S=args.S, T=args.T, B=args.B,
-                  indexer=args.indexer, index_dtype=args.index_dtype)
+                  indexer=args.indexer, index_dtype=args.index_dtype, nsink=args.sinks)
     cfg = wl.cfg
     nst = len(wl.stages)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
@@ -565,7 +579,7 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32" if cfg.dtype == "f32" else "bf16", "data": "synthetic",
             "config": dict(workload_config(cfg, wl.B), indexer_form=wl.indexer,
-                           indexer_dtype=wl.index_dtype),
+                           indexer_dtype=wl.index_dtype, sinks=wl.nsink),
             "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
             "clocks": clk, "gpu_launches": wl.launches_per_step * args.steps,
             "wall_ms_per_step_incl_flush": round(1e3 * t_wall / args.steps, 4),

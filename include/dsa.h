@@ -194,6 +194,27 @@ dsa_status dsa_sparse_attn(dsa_dtype dtype, const void* q, const void* k, const 
                            size_t ws_bytes, dsa_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
+ * 3b. Sparse attention with attention sinks.  [PANGU] §3.4 (PAS): each layer's learnable
+ *    key-value pairs act at inference as a fixed set of virtual KV entries; here they are
+ *    `nsink` per-head rows (the expanded form, like the cache) that join every query's
+ *    softmax, unmasked, beside its selected keys.
+ *
+ *   sink_k [nsink,H,DQK] dtype, sink_v [nsink,H,DV] dtype, 1 <= nsink <= 128 (the pages'
+ *   128 entries fill one key block of the masked-tile kernel); other arguments and the
+ *   contract as dsa_sparse_attn, with the workspace from
+ *   dsa_sparse_attn_sinks_workspace_bytes.
+ * --------------------------------------------------------------------------------- */
+size_t dsa_sparse_attn_sinks_workspace_bytes(dsa_dtype dtype, int B, int S, int T, int H,
+                                             int DQK, int DV, int K, int nsink,
+                                             dsa_attn_algo algo);
+dsa_status dsa_sparse_attn_sinks(dsa_dtype dtype, const void* q, const void* k, const void* v,
+                                 const int32_t* idx, int K, const void* sink_k,
+                                 const void* sink_v, int nsink, const void* gate,
+                                 dsa_gate_mode gate_mode, float sm_scale, int B, int S, int T,
+                                 int H, int DQK, int DV, dsa_attn_algo algo, void* out, void* ws,
+                                 size_t ws_bytes, dsa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
  * The whole DSA step: 1 -> 2 -> 3+4.  [AXK2] "注意力前向的骨架" steps 4-5.
  * Scores and indices go to the caller's buffers when scores_out / idx_out are given,
  * else to the workspace.  Without scores_out the score buffer may be smaller than
@@ -227,6 +248,9 @@ typedef struct {
                               DSA_INDEXER_COLLAPSED (the section 1b form)                */
   dsa_index_dtype index_dtype; /* DSA_INDEX_AS_DTYPE (0): q_idx / k_idx have `dtype`;
                               DSA_INDEX_E4M3: they are e4m3 (per-head indexer only)      */
+  const void* sink_k;      /* optional [nsink,H,DQK] attention sinks (section 3b)        */
+  const void* sink_v;      /* [nsink,H,DV]                                               */
+  int nsink;               /* 0 (none) .. 128                                            */
 } dsa_forward_args;
 
 /* Bytes of workspace dsa_forward needs to run without row blocking. */

@@ -15,7 +15,8 @@ import torch
 
 __all__ = [
     "DSAError", "lib", "dsa_index_scores", "dsa_index_scores_collapsed", "dsa_topk",
-    "dsa_sparse_attn", "dsa_sparse_attn_workspace_bytes", "dsa_sparse_attn_algo", "dsa_forward",
+    "dsa_sparse_attn", "dsa_sparse_attn_sinks", "dsa_sparse_attn_workspace_bytes",
+    "dsa_sparse_attn_algo", "dsa_forward",
     "dsa_forward_workspace_bytes",
     "dsa_window_attn", "dsa_sparse_attn_noalloc", "dsa_device_status", "dsa_version",
     "LIB_PATH",
@@ -50,7 +51,8 @@ class ForwardArgs(ctypes.Structure):
         ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
         ("gate", ctypes.c_void_p), ("out", ctypes.c_void_p), ("scores_out", ctypes.c_void_p),
         ("idx_out", ctypes.c_void_p), ("events", ctypes.c_void_p), ("indexer", ctypes.c_int),
-        ("index_dtype", ctypes.c_int),
+        ("index_dtype", ctypes.c_int), ("sink_k", ctypes.c_void_p), ("sink_v", ctypes.c_void_p),
+        ("nsink", ctypes.c_int),
     ]
 
 
@@ -70,6 +72,9 @@ _SIGNATURES = {
     "dsa_sparse_attn_algo": (_I, [_I, _I, _I, _I, _I, _I, _I, _I, _I]),
     "dsa_sparse_attn": (_I, [_I, _P, _P, _P, _P, _I, _P, _I, _F, _I, _I, _I, _I, _I, _I, _I, _P,
                              _P, _Z, _P]),
+    "dsa_sparse_attn_sinks_workspace_bytes": (_Z, [_I, _I, _I, _I, _I, _I, _I, _I, _I, _I]),
+    "dsa_sparse_attn_sinks": (_I, [_I, _P, _P, _P, _P, _I, _P, _P, _I, _P, _I, _F, _I, _I, _I,
+                                   _I, _I, _I, _I, _P, _P, _Z, _P]),
     "dsa_forward_workspace_bytes": (_Z, [ctypes.POINTER(ForwardArgs)]),
     "dsa_forward_min_workspace_bytes": (_Z, [ctypes.POINTER(ForwardArgs)]),
     "dsa_forward": (_I, [ctypes.POINTER(ForwardArgs), _P, _Z, _P]),
@@ -221,6 +226,28 @@ def dsa_sparse_attn(q, k, v, idx, gate=None, gate_mode=None, sm_scale=0.0, algo=
     return out
 
 
+def dsa_sparse_attn_sinks(q, k, v, idx, sink_k, sink_v, gate=None, gate_mode=None,
+                          sm_scale=0.0, algo="auto", out=None, ws=None, stream=None):
+    """dsa_sparse_attn with attention sinks: sink_k [NS,H,DQK], sink_v [NS,H,DV] (NS <= 128)
+    join every query's softmax unmasked."""
+    _dev(q, k, v, idx, sink_k, sink_v, gate, out, ws)
+    B, S, H, DQK = q.shape
+    T, DV = k.shape[1], v.shape[-1]
+    K = idx.shape[-1]
+    NS = sink_k.shape[0]
+    gm = GATE[gate_mode or ("sigmoid" if gate is not None else "off")]
+    if out is None:
+        out = torch.empty((B, S, H, DV), dtype=q.dtype, device=q.device)
+    nbytes = int(lib().dsa_sparse_attn_sinks_workspace_bytes(_dtype_code(q), B, S, T, H, DQK, DV,
+                                                             K, NS, ATTN_ALGO[algo]))
+    ws = _workspace(nbytes, q.device, ws)
+    _check(lib().dsa_sparse_attn_sinks(_dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), K,
+                                       _ptr(sink_k), _ptr(sink_v), NS, _ptr(gate), gm,
+                                       float(sm_scale), B, S, T, H, DQK, DV, ATTN_ALGO[algo],
+                                       _ptr(out), _ptr(ws), nbytes, _stream(stream)))
+    return out
+
+
 def dsa_sparse_attn_noalloc(q, k, v, idx, gate=None, gate_mode=None, sm_scale=0.0, out=None,
                             stream=None):
     """dsa_sparse_attn (gather form) with no workspace: the split-key partials live in the
@@ -240,7 +267,8 @@ def dsa_sparse_attn_noalloc(q, k, v, idx, gate=None, gate_mode=None, sm_scale=0.
 
 
 def _forward_args(q_idx, k_idx, w, index_scale, K, q, k, v, gate, gate_mode, relu, sm_scale,
-                  attn_algo, out, scores_out, idx_out, indexer="per_head"):
+                  attn_algo, out, scores_out, idx_out, indexer="per_head", sink_k=None,
+                  sink_v=None):
     B, S, HI, DI = q_idx.shape
     T = k_idx.shape[1]
     H, DQK = q.shape[2], q.shape[3]
@@ -254,7 +282,10 @@ def _forward_args(q_idx, k_idx, w, index_scale, K, q, k, v, gate, gate_mode, rel
         gate=None if gate is None else gate.data_ptr(), out=out.data_ptr(),
         scores_out=None if scores_out is None else scores_out.data_ptr(),
         idx_out=None if idx_out is None else idx_out.data_ptr(), indexer=INDEXER[indexer],
-        index_dtype=1 if q_idx.dtype == torch.float8_e4m3fn else 0)
+        index_dtype=1 if q_idx.dtype == torch.float8_e4m3fn else 0,
+        sink_k=None if sink_k is None else sink_k.data_ptr(),
+        sink_v=None if sink_v is None else sink_v.data_ptr(),
+        nsink=0 if sink_k is None else int(sink_k.shape[0]))
     return a
 
 
@@ -266,7 +297,7 @@ def dsa_forward_workspace_bytes(args: ForwardArgs, minimum: bool = False) -> int
 def dsa_forward(q_idx, k_idx, w, index_scale, K, q, k, v, gate=None, gate_mode=None,
                 relu="none", sm_scale=0.0, attn_algo="auto", out=None, scores_out=None,
                 idx_out=None, ws=None, ws_bytes=None, stream=None, events=None,
-                indexer="per_head"):
+                indexer="per_head", sink_k=None, sink_v=None):
     """The whole DSA step (indexer -> top-k -> sparse attention -> gate).
     indexer: "per_head" (the pages' per-head work) or "collapsed" (see
     dsa_index_scores_collapsed).
@@ -274,7 +305,7 @@ def dsa_forward(q_idx, k_idx, w, index_scale, K, q, k, v, gate=None, gate_mode=N
     Returns (out, idx); idx is idx_out if given, else a view of the workspace copy.
     ``ws_bytes`` limits the workspace handed to the library (row blocking below the
     full size)."""
-    _dev(q_idx, k_idx, w, q, k, v, gate, out, scores_out, idx_out, ws)
+    _dev(q_idx, k_idx, w, q, k, v, gate, out, scores_out, idx_out, ws, sink_k, sink_v)
     B, S = q_idx.shape[:2]
     T = k_idx.shape[1]
     if out is None:
@@ -283,7 +314,7 @@ def dsa_forward(q_idx, k_idx, w, index_scale, K, q, k, v, gate=None, gate_mode=N
     if idx_out is None:
         idx_out = torch.empty((B, S, k_eff), dtype=torch.int32, device=q.device)
     a = _forward_args(q_idx, k_idx, w, index_scale, K, q, k, v, gate, gate_mode, relu, sm_scale,
-                      attn_algo, out, scores_out, idx_out, indexer)
+                      attn_algo, out, scores_out, idx_out, indexer, sink_k, sink_v)
     ev_arr = None
     if events is not None:  # 4 torch.cuda.Event, recorded by the library at stage boundaries
         for e in events:

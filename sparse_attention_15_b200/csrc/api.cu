@@ -116,6 +116,18 @@ dsa_status run_index_scores_collapsed(const void* qc, const void* k_idx, float s
                      "dsa_index_scores_collapsed");
 }
 
+// Attention sinks ([PANGU] §3.4 PAS): up to one 128-entry block, [nsink, H, D] rows.
+dsa_status check_sinks(const void* sink_k, const void* sink_v, int nsink) {
+  if (nsink == 0) return DSA_OK;
+  REQUIRE(nsink > 0 && nsink <= 128, DSA_ERR_UNSUPPORTED, "nsink=%d must be in [1, 128]",
+          nsink);
+  REQUIRE(sink_k != nullptr && sink_v != nullptr, DSA_ERR_INVALID_ARG,
+          "sink_k and sink_v must be given with nsink > 0");
+  REQUIRE(aligned16(sink_k) && aligned16(sink_v), DSA_ERR_UNSUPPORTED,
+          "sink pointers must be 16-byte aligned");
+  return DSA_OK;
+}
+
 dsa_status check_attn_common(dsa_dtype dtype, const void* q, const void* k, const void* v,
                              const void* gate, dsa_gate_mode gm, float sm_scale, int B, int S,
                              int T, int H, int HKV, int DQK, int DV, const void* out) {
@@ -266,10 +278,17 @@ dsa_status dsa_topk(const float* scores, int B, int S, int T, int K, int32_t* id
 
 size_t dsa_sparse_attn_workspace_bytes(dsa_dtype dtype, int B, int S, int T, int H, int DQK,
                                        int DV, int K, dsa_attn_algo algo) {
-  if (B <= 0 || S <= 0 || T <= 0 || H <= 0 || DQK <= 0 || DV <= 0 || K <= 0) return 0;
+  return dsa_sparse_attn_sinks_workspace_bytes(dtype, B, S, T, H, DQK, DV, K, 0, algo);
+}
+
+size_t dsa_sparse_attn_sinks_workspace_bytes(dsa_dtype dtype, int B, int S, int T, int H,
+                                             int DQK, int DV, int K, int nsink,
+                                             dsa_attn_algo algo) {
+  if (B <= 0 || S <= 0 || T <= 0 || H <= 0 || DQK <= 0 || DV <= 0 || K <= 0 || nsink < 0)
+    return 0;
   const int alg = choose_algo(algo, dtype, B, S, T, H, DQK, DV, K);
   if (alg == kMasked) return mask_bytes(B, S, T);
-  if (alg == kGather) return dsa::gather_attn_workspace_bytes(B, S, H, DV, K);
+  if (alg == kGather) return dsa::gather_attn_workspace_bytes(B, S, H, DV, K, nsink);
   return 0;
 }
 
@@ -280,11 +299,12 @@ dsa_attn_algo dsa_sparse_attn_algo(dsa_dtype dtype, int B, int S, int T, int H, 
   return alg == kMasked ? DSA_ATTN_MASKED_TILE : (alg == kGather ? DSA_ATTN_GATHER : DSA_ATTN_AUTO);
 }
 
-dsa_status dsa_sparse_attn(dsa_dtype dtype, const void* q, const void* k, const void* v,
-                           const int32_t* idx, int K, const void* gate,
-                           dsa_gate_mode gate_mode, float sm_scale, int B, int S, int T,
-                           int H, int DQK, int DV, dsa_attn_algo algo, void* out, void* ws,
-                           size_t ws_bytes, dsa_stream_t stream) {
+static dsa_status sparse_attn_impl(dsa_dtype dtype, const void* q, const void* k, const void* v,
+                                   const int32_t* idx, int K, const void* sink_k,
+                                   const void* sink_v, int nsink, const void* gate,
+                                   dsa_gate_mode gate_mode, float sm_scale, int B, int S, int T,
+                                   int H, int DQK, int DV, dsa_attn_algo algo, void* out,
+                                   void* ws, size_t ws_bytes, dsa_stream_t stream) {
   dsa_status st = check_attn_common(dtype, q, k, v, gate, gate_mode, sm_scale, B, S, T, H, H,
                                     DQK, DV, out);
   if (st != DSA_OK) return st;
@@ -292,10 +312,12 @@ dsa_status dsa_sparse_attn(dsa_dtype dtype, const void* q, const void* k, const 
   REQUIRE(aligned16(idx), DSA_ERR_UNSUPPORTED, "idx must be 16-byte aligned");
   REQUIRE(algo >= DSA_ATTN_AUTO && algo <= DSA_ATTN_MASKED_TILE, DSA_ERR_INVALID_ARG,
           "unknown attention algorithm %d", (int)algo);
+  if ((st = check_sinks(sink_k, sink_v, nsink)) != DSA_OK) return st;
   const int alg = choose_algo(algo, dtype, B, S, T, H, DQK, DV, K);
   REQUIRE(alg != kNone, DSA_ERR_UNSUPPORTED,
           "the masked-tile algorithm needs bf16, DQK in {128,192} and DV == 128");
-  const size_t need = dsa_sparse_attn_workspace_bytes(dtype, B, S, T, H, DQK, DV, K, algo);
+  const size_t need =
+      dsa_sparse_attn_sinks_workspace_bytes(dtype, B, S, T, H, DQK, DV, K, nsink, algo);
   REQUIRE(ws_bytes >= need && (need == 0 || ws != nullptr), DSA_ERR_INVALID_ARG,
           "workspace too small: %zu bytes given, %zu needed", ws_bytes, need);
   REQUIRE(ws == nullptr || aligned16(ws), DSA_ERR_UNSUPPORTED, "workspace must be 16-byte aligned");
@@ -304,6 +326,8 @@ dsa_status dsa_sparse_attn(dsa_dtype dtype, const void* q, const void* k, const 
   p.gate = gate; p.gate_mode = (int)gate_mode; p.sm_scale = default_scale(sm_scale, DQK);
   p.B = B; p.S = S; p.T = T; p.H = H; p.HKV = H; p.DQK = DQK; p.DV = DV; p.q_off = T - S;
   p.out = out;
+  p.sink_k = nsink > 0 ? sink_k : nullptr; p.sink_v = nsink > 0 ? sink_v : nullptr;
+  p.nsink = nsink;
   cudaStream_t s = (cudaStream_t)stream;
   if (alg == kMasked) {
     uint32_t* mask = static_cast<uint32_t*>(ws);
@@ -314,6 +338,26 @@ dsa_status dsa_sparse_attn(dsa_dtype dtype, const void* q, const void* k, const 
     return cuda_status(dsa::launch_masked_attn(p, mask, stride, s), "dsa_sparse_attn");
   }
   return cuda_status(dsa::launch_gather_attn(p, ws, ws_bytes, s), "dsa_sparse_attn");
+}
+
+dsa_status dsa_sparse_attn(dsa_dtype dtype, const void* q, const void* k, const void* v,
+                           const int32_t* idx, int K, const void* gate,
+                           dsa_gate_mode gate_mode, float sm_scale, int B, int S, int T,
+                           int H, int DQK, int DV, dsa_attn_algo algo, void* out, void* ws,
+                           size_t ws_bytes, dsa_stream_t stream) {
+  return sparse_attn_impl(dtype, q, k, v, idx, K, nullptr, nullptr, 0, gate, gate_mode, sm_scale,
+                          B, S, T, H, DQK, DV, algo, out, ws, ws_bytes, stream);
+}
+
+dsa_status dsa_sparse_attn_sinks(dsa_dtype dtype, const void* q, const void* k, const void* v,
+                                 const int32_t* idx, int K, const void* sink_k,
+                                 const void* sink_v, int nsink, const void* gate,
+                                 dsa_gate_mode gate_mode, float sm_scale, int B, int S, int T,
+                                 int H, int DQK, int DV, dsa_attn_algo algo, void* out, void* ws,
+                                 size_t ws_bytes, dsa_stream_t stream) {
+  REQUIRE(nsink > 0, DSA_ERR_INVALID_ARG, "nsink must be positive (use dsa_sparse_attn)");
+  return sparse_attn_impl(dtype, q, k, v, idx, K, sink_k, sink_v, nsink, gate, gate_mode,
+                          sm_scale, B, S, T, H, DQK, DV, algo, out, ws, ws_bytes, stream);
 }
 
 dsa_status dsa_window_attn(dsa_dtype dtype, const void* q, const void* k, const void* v,
@@ -370,6 +414,7 @@ static dsa_status check_forward(const dsa_forward_args* a) {
           "idx_out must be 16-byte aligned");
   REQUIRE(a->indexer == DSA_INDEXER_PER_HEAD || a->indexer == DSA_INDEXER_COLLAPSED,
           DSA_ERR_INVALID_ARG, "unknown indexer mode %d", (int)a->indexer);
+  if ((st = check_sinks(a->sink_k, a->sink_v, a->nsink)) != DSA_OK) return st;
   if (a->indexer == DSA_INDEXER_COLLAPSED) return check_collapsed(a->dtype, a->relu, a->DI);
   return DSA_OK;
 }
@@ -389,7 +434,8 @@ static FwdLayout forward_layout(const dsa_forward_args* a) {
   if (!a->idx_out) off += align256((size_t)a->B * a->S * L.k_eff * sizeof(int32_t));
   L.attn_off = off;
   if (L.alg == kGather)
-    off += align256(dsa::gather_attn_workspace_bytes(a->B, a->S, a->H, a->DV, L.k_eff));
+    off += align256(dsa::gather_attn_workspace_bytes(a->B, a->S, a->H, a->DV, L.k_eff,
+                                                     a->nsink > 0 ? a->nsink : 0));
   L.mask_off = off;
   if (L.alg == kMasked) off += align256(mask_bytes(a->B, a->S, a->T));
   L.qc_off = off;
@@ -494,6 +540,9 @@ dsa_status dsa_forward(const dsa_forward_args* a, void* ws, size_t ws_bytes,
   p.sm_scale = default_scale(a->sm_scale, a->DQK);
   p.B = B; p.S = S; p.T = T; p.H = a->H; p.HKV = a->H; p.DQK = a->DQK; p.DV = a->DV;
   p.q_off = q_off; p.out = a->out;
+  if (a->nsink > 0) {
+    p.sink_k = a->sink_k; p.sink_v = a->sink_v; p.nsink = a->nsink;
+  }
   if (L.alg == kMasked)
     st = cuda_status(dsa::launch_masked_attn(p, mask, L.mask_stride, s), "dsa_forward/attn");
   else

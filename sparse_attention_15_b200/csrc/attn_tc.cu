@@ -55,6 +55,7 @@ struct AttnArgs {
   int B, S, T, H, HKV, q_off, window;
   int mask_stride;       // words per mask row (multiple of 4)
   int nqb;
+  int nsink;             // attention sinks (PAS), 0..128: one extra block per item
 };
 
 template <int DQK_, int DV_, bool BAND_>
@@ -172,7 +173,9 @@ __device__ __forceinline__ Item item_of(const AttnArgs& a, int i) {
   it.qb = a.nqb - 1 - r / a.B;
   return it;
 }
-// Key blocks [j0, j1) item `it` must visit.
+// Key blocks [j0, j1) item `it` must visit.  With attention sinks an item first visits one
+// sink block (the nsink sink entries, always visible), then those key blocks: block r of
+// the item is the sink block for r < sink_blocks(a), else key block j0 + r - sink_blocks.
 template <bool BAND>
 __device__ __forceinline__ void key_range(const AttnArgs& a, const Item& it, int* j0, int* j1) {
   const int s0 = it.qb * kBlk;
@@ -186,11 +189,18 @@ __device__ __forceinline__ void key_range(const AttnArgs& a, const Item& it, int
   }
 }
 
+template <bool BAND>
+__device__ __forceinline__ int sink_blocks(const AttnArgs& a) {
+  return (!BAND && a.nsink > 0) ? 1 : 0;
+}
+
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1)
     masked_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
                           const __grid_constant__ CUtensorMap kmap,
-                          const __grid_constant__ CUtensorMap vmap, const AttnArgs a) {
+                          const __grid_constant__ CUtensorMap vmap,
+                          const __grid_constant__ CUtensorMap skmap,
+                          const __grid_constant__ CUtensorMap svmap, const AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -229,6 +239,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     mbar_init(o_empty, 8); mbar_init(ml_full, 8 * 32); mbar_init(mma_done, 1);
     fence_mbar_init();
     prefetch_tmap(&qmap); prefetch_tmap(&kmap); prefetch_tmap(&vmap);
+    if (sink_blocks<C::BAND>(a)) { prefetch_tmap(&skmap); prefetch_tmap(&svmap); }
   }
   if (warp == kWarpMma) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -264,21 +275,25 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             tma_load_3d(Qs + x * C::SLICE, &qmap, x * 64, it.h, qrow, q_full);
         }
         const int kvh = it.h / group;
-        for (int j = j0; j < j1; ++j, ++g) {
+        const int sb = sink_blocks<C::BAND>(a);
+        const int nb = j1 - j0 + sb;
+        for (int r = 0; r < nb; ++r, ++g) {
           const int st = g & 1;
           if (g >= 2 && !mbar_wait(&empty[st], ((g >> 1) - 1) & 1)) { ok = false; break; }
           uint8_t* dst = KVs + st * C::KV_BYTES + (kq ? 0 : C::K_BYTES);
-          const int krow = it.b * a.T + j * kBlk;
+          // the sink block reads rows 0..127 of the sink arrays (rows past nsink: zero fill)
+          const bool sink = r < sb;
+          const int krow = sink ? 0 : it.b * a.T + (j0 + r - sb) * kBlk;
           if (kq) {
             mbar_arrive_expect_tx(&full[st], C::K_BYTES);
 #pragma unroll
             for (int x = 0; x < C::QKH; ++x)
-              tma_load_3d(dst + x * C::SLICE, &kmap, x * 64, kvh, krow, &full[st]);
+              tma_load_3d(dst + x * C::SLICE, sink ? &skmap : &kmap, x * 64, kvh, krow, &full[st]);
           } else {
             mbar_arrive_expect_tx(&full[st], C::V_BYTES);
 #pragma unroll
             for (int x = 0; x < C::VH; ++x)
-              tma_load_3d(dst + x * C::SLICE, &vmap, x * 64, kvh, krow, &full[st]);
+              tma_load_3d(dst + x * C::SLICE, sink ? &svmap : &vmap, x * 64, kvh, krow, &full[st]);
           }
         }
       }
@@ -317,7 +332,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         const Item it = item_of(a, i);
         int j0, j1;
         key_range<C::BAND>(a, it, &j0, &j1);
-        const int nb = j1 - j0;
+        const int nb = j1 - j0 + sink_blocks<C::BAND>(a);
         if (!mbar_wait(q_full, ni & 1)) { ok = false; break; }
         if (!issue_qk(g)) { ok = false; break; }
         for (int j = 0; j < nb; ++j) {
@@ -366,7 +381,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       const Item it = item_of(a, i);
       int j0, j1;
       key_range<C::BAND>(a, it, &j0, &j1);
-      const int nb = j1 - j0;
+      const int sb = sink_blocks<C::BAND>(a);
+      const int nb = j1 - j0 + sb;
       const int s = it.qb * kBlk + row;
       const int spos = s + a.q_off;
       const bool row_ok = s < a.S;
@@ -374,18 +390,28 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           (!C::BAND && row_ok) ? a.mask + ((size_t)it.b * a.S + s) * a.mask_stride : nullptr;
       const int jfirst = (int)((grp - g) & 1u);  // first block of this group's parity
       float m_used = ninf, l = 0.f;
+      // the 4 selection words of item block r >= sb (key block j0 + r - sb)
+      auto mask_words = [&](int r) {
+        return __ldg(reinterpret_cast<const uint4*>(mrow + (((j0 + r - sb) * kBlk) >> 5)));
+      };
       uint4 nb4 = make_uint4(0u, 0u, 0u, 0u);
-      if (mrow && jfirst < nb)
-        nb4 = __ldg(reinterpret_cast<const uint4*>(mrow + (((j0 + jfirst) * kBlk) >> 5)));
+      if (mrow && jfirst < nb && jfirst >= sb) nb4 = mask_words(jfirst);
       const uint32_t o_col = C::O_COL + grp * C::DV;
       for (int j = jfirst; j < nb; j += 2) {
         const uint32_t gg = g + j;
-        const int t0 = (j0 + j) * kBlk;
+        const int t0 = (j0 + j - sb) * kBlk;
         uint32_t bits[4] = {0u, 0u, 0u, 0u};
         if (!C::BAND) {
-          bits[0] = nb4.x; bits[1] = nb4.y; bits[2] = nb4.z; bits[3] = nb4.w;
-          if (mrow && j + 2 < nb)
-            nb4 = __ldg(reinterpret_cast<const uint4*>(mrow + ((t0 + 2 * kBlk) >> 5)));
+          if (j < sb) {  // the sink block: its first nsink entries, visible to every query
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              const int n = a.nsink - 32 * w;
+              bits[w] = n >= 32 ? 0xffffffffu : (n > 0 ? (1u << n) - 1u : 0u);
+            }
+          } else {
+            bits[0] = nb4.x; bits[1] = nb4.y; bits[2] = nb4.z; bits[3] = nb4.w;
+          }
+          if (mrow && j + 2 < nb) nb4 = mask_words(j + 2);
         } else if (row_ok) {
           // band: spos - window < t <= spos, t < T
           const int lo = max(spos - a.window + 1, 0) - t0, hi = min(spos, a.T - 1) - t0;
@@ -614,16 +640,27 @@ int num_sms() {
 template <class C>
 cudaError_t launch_fa(const AttnProblem& p, const uint32_t* mask, int mask_stride,
                       cudaStream_t st) {
-  CUtensorMap qm, km, vm;
+  CUtensorMap qm, km, vm, skm, svm;
   if (!map3d(&qm, p.q, (uint64_t)p.B * p.S, p.H, C::DQK) ||
       !map3d(&km, p.k, (uint64_t)p.B * p.T, p.HKV, C::DQK) ||
       !map3d(&vm, p.v, (uint64_t)p.B * p.T, p.HKV, C::DV))
     return cudaErrorInvalidValue;
+  const bool sinks = !C::BAND && p.sink_k != nullptr && p.nsink > 0;
+  if (sinks) {
+    if (p.nsink > kBlk) return cudaErrorNotSupported;  // one sink block per item
+    if (!map3d(&skm, p.sink_k, (uint64_t)p.nsink, p.HKV, C::DQK) ||
+        !map3d(&svm, p.sink_v, (uint64_t)p.nsink, p.HKV, C::DV))
+      return cudaErrorInvalidValue;
+  } else {
+    skm = km;  // unused
+    svm = vm;
+  }
   AttnArgs a{};
   a.mask = mask; a.gate = p.gate; a.out = static_cast<__nv_bfloat16*>(p.out);
   a.gate_mode = p.gate_mode; a.qk_scale = p.sm_scale * kLog2e;
   a.B = p.B; a.S = p.S; a.T = p.T; a.H = p.H; a.HKV = p.HKV; a.q_off = p.q_off;
   a.window = p.window; a.mask_stride = mask_stride;
+  a.nsink = sinks ? p.nsink : 0;
   a.nqb = (p.S + kBlk - 1) / kBlk;
   const int items = p.B * p.H * a.nqb;
   const int nsm = num_sms();
@@ -631,7 +668,7 @@ cudaError_t launch_fa(const AttnProblem& p, const uint32_t* mask, int mask_strid
   auto kern = masked_attn_tc_kernel<C>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<grid, C::THREADS, C::SMEM, st>>>(qm, km, vm, a);
+  kern<<<grid, C::THREADS, C::SMEM, st>>>(qm, km, vm, skm, svm, a);
   return cudaGetLastError();
 }
 

@@ -90,17 +90,18 @@ struct GatherArgs {
   int nslots;
   uint32_t k_bytes, v_bytes, slot_bytes;
   uint32_t key_list_bytes;  // shared-memory bytes reserved for the key list
+  const void* sink_k;       // [nsink, HKV, DQK] attention sinks (PAS) or NULL
+  const void* sink_v;       // [nsink, HKV, DV]
+  int nsink;
 };
 
-// Key j of this CTA's range, or -1 if it must be skipped.
-__device__ __forceinline__ int key_at(const GatherArgs& a, const int32_t* idx_row, int j,
+// Entry jj of a query's key list: the nsink sinks come first (encoded as -2 - sink), then
+// the selected keys (or the band).  -1 marks an entry to skip.
+__device__ __forceinline__ int key_at(const GatherArgs& a, const int32_t* idx_row, int jj,
                                       int spos) {
-  int t;
-  if (idx_row) {
-    t = __ldg(idx_row + j);
-  } else {
-    t = spos - a.window + 1 + j;  // band: oldest key first
-  }
+  if (jj < a.nsink) return -2 - jj;
+  const int e = jj - a.nsink;
+  const int t = idx_row ? __ldg(idx_row + e) : spos - a.window + 1 + e;  // band: oldest first
   return (t >= 0 && t < a.T && t <= spos) ? t : -1;
 }
 
@@ -120,11 +121,10 @@ __global__ void __launch_bounds__(544, HPW <= 2 ? 2 : 1) gather_attn_kernel(cons
   const int split = blockIdx.x % a.nsplit;
   const int b = row / a.S, s = row % a.S;
   const int spos = s + a.q_off;
-  const int nkeys_total = a.idx ? a.K : a.window;
+  const int nkeys_total = a.nsink + (a.idx ? a.K : a.window);
   const int j0 = split * a.keys_per_split;
   const int nkeys = max(0, min(nkeys_total, j0 + a.keys_per_split) - j0);
-  const int32_t* idx_row = a.idx ? a.idx + (size_t)row * a.K + j0 : nullptr;
-  const int band0 = j0;  // band offset of this split
+  const int32_t* idx_row = a.idx ? a.idx + (size_t)row * a.K : nullptr;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < nslots; ++i) {
@@ -142,7 +142,7 @@ __global__ void __launch_bounds__(544, HPW <= 2 ? 2 : 1) gather_attn_kernel(cons
     // ------------------------------------------------------------- producer
     // stage the key list once (coalesced), then issue the row copies back to back
     for (int j = lane; j < nkeys; j += 32)
-      keys[j] = idx_row ? key_at(a, idx_row, j, spos) : key_at(a, nullptr, band0 + j, spos);
+      keys[j] = key_at(a, idx_row, j0 + j, spos);
     __syncwarp();
     if (lane == 0) {
       for (int j = 0; j < nkeys; ++j) {
@@ -151,11 +151,15 @@ __global__ void __launch_bounds__(544, HPW <= 2 ? 2 : 1) gather_attn_kernel(cons
         if (round > 0 && !mbar_wait(&empty[slot], (round - 1) & 1)) break;
         const int t = keys[j];
         slot_key[slot] = t;
-        if (t >= 0) {
+        if (t != -1) {
+          // a cache row, or (t <= -2) sink row -2 - t, which no batch row owns
+          const size_t r = t >= 0 ? (size_t)t : (size_t)(-2 - t);
+          const T* ksrc = (t >= 0 ? kbase : static_cast<const T*>(a.sink_k)) + r * a.HKV * a.DQK;
+          const T* vsrc = (t >= 0 ? vbase : static_cast<const T*>(a.sink_v)) + r * a.HKV * a.DV;
           uint8_t* dst = slots + (size_t)slot * a.slot_bytes;
           mbar_arrive_expect_tx(&full[slot], a.k_bytes + a.v_bytes);
-          bulk_g2s(dst, kbase + (size_t)t * a.HKV * a.DQK, a.k_bytes, &full[slot]);
-          bulk_g2s(dst + a.k_bytes, vbase + (size_t)t * a.HKV * a.DV, a.v_bytes, &full[slot]);
+          bulk_g2s(dst, ksrc, a.k_bytes, &full[slot]);
+          bulk_g2s(dst + a.k_bytes, vsrc, a.v_bytes, &full[slot]);
         } else {
           mbar_arrive(&full[slot]);
         }
@@ -204,7 +208,7 @@ __global__ void __launch_bounds__(544, HPW <= 2 ? 2 : 1) gather_attn_kernel(cons
   uint32_t phase = 0;
   for (int j = 0; j < nkeys && ok; ++j) {
     ok = mbar_wait(&full[slot], phase);
-    if (ok && slot_key[slot] >= 0) {
+    if (ok && slot_key[slot] != -1) {
       const T* ks = reinterpret_cast<const T*>(slots + (size_t)slot * a.slot_bytes);
       const T* vs = reinterpret_cast<const T*>(slots + (size_t)slot * a.slot_bytes + a.k_bytes);
       float part[hpw];
@@ -413,10 +417,10 @@ cudaError_t launch_hpw(GatherArgs a, int hpw, size_t smem, unsigned grid, int ro
 
 }  // namespace
 
-size_t gather_attn_workspace_bytes(int B, int S, int H, int DV, int K) {
+size_t gather_attn_workspace_bytes(int B, int S, int H, int DV, int K, int nsink) {
   const int rows = B * S;
   int ns, kps;
-  split_policy(rows, K, &ns, &kps);
+  split_policy(rows, K + nsink, &ns, &kps);
   if (ns == 1) return 0;
   return (size_t)rows * ns * H * (DV + 2) * sizeof(float);
 }
@@ -430,7 +434,8 @@ cudaError_t launch_gather_attn(const AttnProblem& p, void* ws, size_t ws_bytes,
   a.S = p.S; a.T = p.T; a.H = p.H; a.HKV = p.HKV; a.DQK = p.DQK; a.DV = p.DV; a.q_off = p.q_off;
   const int rows = p.B * p.S;
   if (rows == 0) return cudaSuccess;
-  const int nkeys = p.idx ? p.K : p.window;
+  a.sink_k = p.sink_k; a.sink_v = p.sink_v; a.nsink = p.sink_k ? p.nsink : 0;
+  const int nkeys = a.nsink + (p.idx ? p.K : p.window);
   split_policy(rows, nkeys, &a.nsplit, &a.keys_per_split, p.idx != nullptr);
   a.key_list_bytes = ((uint32_t)a.keys_per_split * 4u + 127u) & ~127u;
   if (a.nsplit > 1) {

@@ -68,8 +68,11 @@ struct AttnProblem {
   float sm_scale;
   int B, S, T, H, HKV, DQK, DV, q_off;
   void* out;          // [B,S,H,DV]
+  const void* sink_k = nullptr;  // [nsink,HKV,DQK] attention sinks (PAS), or NULL
+  const void* sink_v = nullptr;  // [nsink,HKV,DV]
+  int nsink = 0;
 };
-size_t gather_attn_workspace_bytes(int B, int S, int H, int DV, int K);
+size_t gather_attn_workspace_bytes(int B, int S, int H, int DV, int K, int nsink = 0);
 cudaError_t launch_gather_attn(const AttnProblem& p, void* ws, size_t ws_bytes,
                                cudaStream_t st);
 

@@ -132,6 +132,22 @@ def test_sparse_attn_rejects_bad_arguments(lib):
     assert L.dsa_sparse_attn_workspace_bytes(1, 1, 4096, 4096, 20, 128, 128, 512, 1) == 0
 
 
+def test_sparse_attn_sinks_rejects_bad_arguments(lib):
+    L = lib.lib()
+
+    def call(nsink=4, sk=FAKE, sv=FAKE, **kw):
+        a = dict(dtype=1, B=1, S=4, T=4, H=2, DQK=128, DV=128, K=2)
+        a.update(kw)
+        return L.dsa_sparse_attn_sinks(a["dtype"], FAKE, FAKE, FAKE, FAKE, a["K"], sk, sv, nsink,
+                                       None, 0, 0.0, a["B"], a["S"], a["T"], a["H"], a["DQK"],
+                                       a["DV"], 1, FAKE, FAKE, 1 << 20, None)
+    assert call(nsink=0) == 1          # use dsa_sparse_attn without sinks
+    assert call(nsink=129) == 2        # at most one 128-entry block
+    assert call(sk=None) == 1
+    assert call(sv=FAKE_MIS) == 2
+    assert L.dsa_sparse_attn_sinks_workspace_bytes(1, 1, 4, 4, 2, 128, 128, 2, 4, 1) >= 0
+
+
 def test_window_attn_rejects_bad_arguments(lib):
     L = lib.lib()
     f = L.dsa_window_attn

@@ -234,6 +234,62 @@ def test_sparse_attn_parity(name, S, T, K, gate_mode, algo):
     P.assert_attn_close(got, ref, x["q"].dtype, f"{name} {gate_mode} {algo}")
 
 
+def _sinks(cfg, NS, seed, dtype):
+    g = torch.Generator().manual_seed(seed)
+    sk = torch.randn(NS, cfg.H, cfg.dqk, generator=g).to(dtype)
+    sv = torch.randn(NS, cfg.H, cfg.dv, generator=g).to(dtype)
+    return sk, sv
+
+
+# attention sinks (PAS): both kernels, a full block of 128 and a ragged one, prefill and a
+# decode shape whose key lists are split over CTAs (the sinks land in the first split)
+SINKS = [("c3", 150, 300, 40, 128), ("c3", 150, 300, 40, 5), ("c2", 333, 333, 64, 128),
+         ("c2", 100, 517, 512, 77)]
+
+
+@pytest.mark.parametrize("name,S,T,K,NS", SINKS)
+@pytest.mark.parametrize("algo", ["gather", "masked_tile"])
+def test_sparse_attn_sinks_parity(name, S, T, K, NS, algo):
+    cfg, x, g = _inputs(name, S, T)
+    sc = O.index_scores(x["q_idx"], x["k_idx"], x["w"], cfg.scale)
+    idx = O.topk_indices(sc, min(K, T))
+    sk, sv = _sinks(cfg, NS, 21, x["q"].dtype)
+    gate = x["gate"]
+    got = dsa.dsa_sparse_attn_sinks(g["q"], g["k"], g["v"], torch.from_numpy(idx).to(DEV),
+                                    sk.to(DEV), sv.to(DEV), gate=g["gate"],
+                                    gate_mode=cfg.gate if gate is not None else None, algo=algo)
+    ref = O.sparse_attention(x["q"], x["k"], x["v"], idx, gate=gate, gate_mode=cfg.gate,
+                             sink_k=sk, sink_v=sv)
+    P.assert_attn_close(got, ref, x["q"].dtype, f"{name} sinks={NS} {algo}")
+
+
+def test_sparse_attn_sinks_decode_split():
+    cfg, x, g = _inputs("c3", 1, 3000, B=3)
+    sc = O.index_scores(x["q_idx"], x["k_idx"], x["w"], cfg.scale)
+    idx = O.topk_indices(sc, 2048)
+    sk, sv = _sinks(cfg, 128, 23, x["q"].dtype)
+    got = dsa.dsa_sparse_attn_sinks(g["q"], g["k"], g["v"], torch.from_numpy(idx).to(DEV),
+                                    sk.to(DEV), sv.to(DEV), gate=g["gate"], gate_mode="sigmoid",
+                                    algo="gather")
+    ref = O.sparse_attention(x["q"], x["k"], x["v"], idx, gate=x["gate"], gate_mode="sigmoid",
+                             sink_k=sk, sink_v=sv)
+    P.assert_attn_close(got, ref, x["q"].dtype, "decode sinks")
+
+
+@pytest.mark.parametrize("name,S,T", [("c2", 600, 600), ("c3", 260, 330)])
+def test_forward_sinks_parity(name, S, T):
+    cfg, x, g = _inputs(name, S, T)
+    K = min(cfg.K, 96)
+    sk, sv = _sinks(cfg, 128, 29, x["q"].dtype)
+    out, idx = dsa.dsa_forward(g["q_idx"], g["k_idx"], g["w"], cfg.scale, K, g["q"], g["k"],
+                               g["v"], gate=g["gate"], sink_k=sk.to(DEV), sink_v=sv.to(DEV))
+    _, idx_ref, out_ref = O.dsa_forward(x["q_idx"], x["k_idx"], x["w"], cfg.scale, K, x["q"],
+                                        x["k"], x["v"], gate=x["gate"], gate_mode=cfg.gate,
+                                        sink_k=sk, sink_v=sv)
+    assert np.array_equal(P.to_np(idx), idx_ref)
+    P.assert_attn_close(out, out_ref, x["q"].dtype, f"{name} forward sinks")
+
+
 @pytest.mark.parametrize("algo", ["gather", "masked_tile"])
 def test_sparse_attn_skips_invalid_and_future_indices(algo):
     cfg, x, g = _inputs("c2", 40, 90)
