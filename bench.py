@@ -40,8 +40,8 @@ F32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # DRAM traffic per launch from committed ncu captures: (kernel, config) -> (bytes,
 # sha256 of the kernel source when captured).  Reported as null when the source changed.
 NCU_TRAFFIC = {
-    # masked_attn_tc_kernel, c2 full size: 64.30 MB read + 5.21 MB written
-    ("masked_attn", "c2"): (69505024, "7b24d50f0fc68b67"),
+    # masked_attn_tc_kernel, c2 full size: 64.29 MB read + 3.94 MB written
+    ("masked_attn", "c2"): (68228096, "c5523d701892eb31"),
     # gather_attn_kernel, c4: captured at B = 32 (same per-row work: 9 splits x 228 keys),
     # 1.3429 GB read + 6.27 MB written, scaled by the rows (x2) to the full B = 64 launch
     ("gather_attn", "c4"): (2698253856, "e54ebdebc52f47b9"),
@@ -76,7 +76,9 @@ def selected_pairs(S, T, B, q_off, K):
 
 
 class ClockSampler:
-    """nvidia-smi sampling (200 ms) of the GPU this process uses, during the timed region."""
+    """nvidia-smi sampling (every 20 ms) of the GPU this process uses, during the timed
+    region (samples inside it; the nearest ones within 0.2 s when the region is shorter than
+    the sampling interval)."""
 
     FIELDS = ("pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -96,7 +98,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "20"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
             return
@@ -124,8 +126,10 @@ class ClockSampler:
                  f[0].lower().endswith(self.pci[-12:]))]
         if not rows:
             return None
-        win = [f for t, f in rows if self.t_start and self.t_stop and
-               self.t_start - 0.2 <= t <= self.t_stop + 0.2] or [f for _, f in rows]
+        inside = [f for t, f in rows if self.t_start and self.t_stop and
+                  self.t_start <= t <= self.t_stop]
+        win = inside or [f for t, f in rows if self.t_start and self.t_stop and
+                         self.t_start - 0.2 <= t <= self.t_stop + 0.2] or [f for _, f in rows]
 
         def num(x):
             try:
@@ -142,6 +146,7 @@ class ClockSampler:
                     reasons.add(n)
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": num(win[0][2]),
                 "reasons": sorted(reasons), "samples": len(win),
+                "samples_inside_timed_region": len(inside),
                 "power_w_max": max(num(f[3]) for f in win)}
 
 
