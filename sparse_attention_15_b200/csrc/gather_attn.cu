@@ -95,17 +95,20 @@ struct GatherArgs {
   int nsink;
 };
 
-// Entry jj of a query's key list: the nsink sinks come first (encoded as -2 - sink), then
-// the selected keys (or the band).  -1 marks an entry to skip.
+// Entry jj of a query's key list: with SINKS the nsink sinks come first (encoded as
+// -2 - sink), then the selected keys (or the band).  -1 marks an entry to skip.
+template <bool SINKS>
 __device__ __forceinline__ int key_at(const GatherArgs& a, const int32_t* idx_row, int jj,
                                       int spos) {
-  if (jj < a.nsink) return -2 - jj;
-  const int e = jj - a.nsink;
+  if (SINKS && jj < a.nsink) return -2 - jj;
+  const int e = SINKS ? jj - a.nsink : jj;
   const int t = idx_row ? __ldg(idx_row + e) : spos - a.window + 1 + e;  // band: oldest first
   return (t >= 0 && t < a.T && t <= spos) ? t : -1;
 }
 
-template <typename T, int QKV, int VV, int HPW>
+// SINKS: the key lists start with attention sinks (a separate instantiation, so the common
+// path carries none of their arithmetic).
+template <typename T, int QKV, int VV, int HPW, bool SINKS>
 __global__ void __launch_bounds__(544, HPW <= 2 ? 2 : 1) gather_attn_kernel(const GatherArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int nslots = a.nslots;
@@ -121,7 +124,7 @@ __global__ void __launch_bounds__(544, HPW <= 2 ? 2 : 1) gather_attn_kernel(cons
   const int split = blockIdx.x % a.nsplit;
   const int b = row / a.S, s = row % a.S;
   const int spos = s + a.q_off;
-  const int nkeys_total = a.nsink + (a.idx ? a.K : a.window);
+  const int nkeys_total = (SINKS ? a.nsink : 0) + (a.idx ? a.K : a.window);
   const int j0 = split * a.keys_per_split;
   const int nkeys = max(0, min(nkeys_total, j0 + a.keys_per_split) - j0);
   const int32_t* idx_row = a.idx ? a.idx + (size_t)row * a.K : nullptr;
@@ -142,7 +145,7 @@ __global__ void __launch_bounds__(544, HPW <= 2 ? 2 : 1) gather_attn_kernel(cons
     // ------------------------------------------------------------- producer
     // stage the key list once (coalesced), then issue the row copies back to back
     for (int j = lane; j < nkeys; j += 32)
-      keys[j] = key_at(a, idx_row, j0 + j, spos);
+      keys[j] = key_at<SINKS>(a, idx_row, j0 + j, spos);
     __syncwarp();
     if (lane == 0) {
       for (int j = 0; j < nkeys; ++j) {
@@ -151,11 +154,14 @@ __global__ void __launch_bounds__(544, HPW <= 2 ? 2 : 1) gather_attn_kernel(cons
         if (round > 0 && !mbar_wait(&empty[slot], (round - 1) & 1)) break;
         const int t = keys[j];
         slot_key[slot] = t;
-        if (t != -1) {
+        if (SINKS ? t != -1 : t >= 0) {
           // a cache row, or (t <= -2) sink row -2 - t, which no batch row owns
-          const size_t r = t >= 0 ? (size_t)t : (size_t)(-2 - t);
-          const T* ksrc = (t >= 0 ? kbase : static_cast<const T*>(a.sink_k)) + r * a.HKV * a.DQK;
-          const T* vsrc = (t >= 0 ? vbase : static_cast<const T*>(a.sink_v)) + r * a.HKV * a.DV;
+          const T* ksrc = kbase + (size_t)t * a.HKV * a.DQK;
+          const T* vsrc = vbase + (size_t)t * a.HKV * a.DV;
+          if (SINKS && t < 0) {
+            ksrc = static_cast<const T*>(a.sink_k) + (size_t)(-2 - t) * a.HKV * a.DQK;
+            vsrc = static_cast<const T*>(a.sink_v) + (size_t)(-2 - t) * a.HKV * a.DV;
+          }
           uint8_t* dst = slots + (size_t)slot * a.slot_bytes;
           mbar_arrive_expect_tx(&full[slot], a.k_bytes + a.v_bytes);
           bulk_g2s(dst, ksrc, a.k_bytes, &full[slot]);
@@ -208,7 +214,7 @@ __global__ void __launch_bounds__(544, HPW <= 2 ? 2 : 1) gather_attn_kernel(cons
   uint32_t phase = 0;
   for (int j = 0; j < nkeys && ok; ++j) {
     ok = mbar_wait(&full[slot], phase);
-    if (ok && slot_key[slot] != -1) {
+    if (ok && (SINKS ? slot_key[slot] != -1 : slot_key[slot] >= 0)) {
       const T* ks = reinterpret_cast<const T*>(slots + (size_t)slot * a.slot_bytes);
       const T* vs = reinterpret_cast<const T*>(slots + (size_t)slot * a.slot_bytes + a.k_bytes);
       float part[hpw];
@@ -383,7 +389,8 @@ void split_policy(int rows, int nkeys, int* nsplit, int* kps, bool allow_split =
 template <typename T, int QKV, int VV, int HPW>
 cudaError_t launch_t(GatherArgs a, int nw, size_t smem, unsigned grid, int rows,
                      cudaStream_t st) {
-  auto kern = gather_attn_kernel<T, QKV, VV, HPW>;
+  auto kern = a.nsink > 0 ? gather_attn_kernel<T, QKV, VV, HPW, true>
+                          : gather_attn_kernel<T, QKV, VV, HPW, false>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

@@ -56,8 +56,9 @@ struct TcArgs {
 // ES_: operand element bytes, 2 (bf16, kind::f16) or 1 (e4m3, kind::f8f6f4).  Every MMA
 // consumes 32 bytes of each 128-byte swizzled row either way, so the shared-memory layout
 // and the descriptor arithmetic are the same in bytes.
+// NACC_: TMEM accumulators (2 or 4): with more, the MMA runs further ahead of the epilogue.
 template <int HI_, int DI_, int NQ_, int NE_, int NA_, int NB_ = 2, bool CL_ = false,
-          int ES_ = 2>
+          int ES_ = 2, int NACC_ = 2>
 struct TcCfg {
   static constexpr int HI = HI_, DI = DI_, NQ = NQ_, NE = NE_, NA = NA_;
   static constexpr bool CL = CL_;
@@ -71,15 +72,17 @@ struct TcCfg {
   static constexpr int A_BYTES = KH * A_SLICE;
   static constexpr int B_SLICE = N * 128;
   static constexpr int B_BYTES = KH * B_SLICE;
+  static constexpr int NACC = NACC_;
   static constexpr int ACC_COLS = N;              // one accumulator
-  static constexpr int TMEM_COLS = 2 * N <= 32 ? 32 : 2 * N <= 64 ? 64 : 2 * N <= 128 ? 128
-                                   : 2 * N <= 256 ? 256 : 512;
+  static constexpr int TMEM_COLS = NACC * N <= 32 ? 32 : NACC * N <= 64 ? 64
+                                   : NACC * N <= 128 ? 128 : NACC * N <= 256 ? 256 : 512;
   static constexpr int EPI_GROUPS = NE / 4;       // epilogue warps per TMEM lane quadrant
   static constexpr int COLS_PER_WARP = N / EPI_GROUPS;
   static constexpr int THREADS = 32 * (kEpiWarp0 + NE);
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM = NA * A_BYTES + NB * B_BYTES + BAR_BYTES + 1024;
   static_assert(N % 16 == 0 && N >= 16 && N <= 256, "UMMA N");
+  static_assert((NACC == 2 || NACC == 4) && NACC * N <= 512, "accumulators must fit TMEM");
   static_assert(HI <= 32 && 32 % HI == 0, "heads per 32-column chunk");
   static_assert(!CL || HI == 2, "the collapsed form has two columns (hi, lo) per query");
   static_assert(CL || HI >= 16, "per-head epilogue: a query spans whole 16-column chunks");
@@ -144,9 +147,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   uint64_t* a_empty = a_full + C::NA;               // [NA]
   uint64_t* b_full = a_empty + C::NA;               // [2]
   uint64_t* b_empty = b_full + 2;                   // [2]
-  uint64_t* acc_full = b_empty + 2;                 // [2]
-  uint64_t* acc_empty = acc_full + 2;               // [2]
-  uint64_t* mma_done = acc_empty + 2;               // [1]
+  uint64_t* acc_full = b_empty + 2;                 // [NACC]
+  uint64_t* acc_empty = acc_full + C::NACC;         // [NACC]
+  uint64_t* mma_done = acc_empty + C::NACC;         // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -156,6 +159,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     for (int i = 0; i < C::NA; ++i) { mbar_init(&a_full[i], 1); mbar_init(&a_empty[i], 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&b_full[i], 1); mbar_init(&b_empty[i], 1);
+    }
+    for (int i = 0; i < C::NACC; ++i) {
       mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], C::NE);
     }
     mbar_init(mma_done, 1);
@@ -227,8 +232,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         for (int kt = it.k0; kt < it.k1; ++kt) {
           const int st = ai % C::NA;
           if (!mbar_wait(&a_full[st], (ai / C::NA) & 1)) { ok = false; break; }
-          const int ab = ci & 1;
-          if (ci >= 2 && !mbar_wait(&acc_empty[ab], ((ci >> 1) - 1) & 1)) { ok = false; break; }
+          const int ab = ci % C::NACC;
+          if (ci >= (uint32_t)C::NACC &&
+              !mbar_wait(&acc_empty[ab], ((ci / C::NACC) - 1) & 1)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_base = smem_u32(As + st * C::A_BYTES);
 #pragma unroll
@@ -272,8 +278,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       const float4* wunit = C::CL ? nullptr : reinterpret_cast<const float4*>(
           a.w + ((size_t)it.b * a.S + s_base) * C::HI);
       for (int kt = it.k0; kt < it.k1; ++kt) {
-        const int ab = ci & 1;
-        if (!warp_wait(&acc_full[ab], (ci >> 1) & 1)) { ok = false; break; }
+        const int ab = ci % C::NACC;
+        if (!warp_wait(&acc_full[ab], (ci / C::NACC) & 1)) { ok = false; break; }
         tc_fence_after();
         const int t = kt * kTileM + quad * 32 + lane;
         constexpr int NCH = C::COLS_PER_WARP / 16;
@@ -595,8 +601,9 @@ cudaError_t launch_index_scores_tc(const void* q_idx, const void* k_idx, const f
   if (HI == 16 && DI == 128)
     return launch_cfg<TcCfg<16, 128, 16, 16, 3>>(q_idx, k_idx, w, scale, relu, B, S, T, q_off,
                                                 scores, write_masked, st);
-  return launch_cfg<TcCfg<16, 64, 16, 16, 4>>(q_idx, k_idx, w, scale, relu, B, S, T, q_off,
-                                             scores, write_masked, st);
+  // N = 128 columns (8 queries): four accumulators in TMEM keep the epilogue's latency hidden
+  return launch_cfg<TcCfg<16, 64, 8, 16, 4, 2, false, 2, 4>>(q_idx, k_idx, w, scale, relu, B, S,
+                                                             T, q_off, scores, write_masked, st);
 }
 
 }  // namespace dsa
