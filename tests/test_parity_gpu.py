@@ -423,6 +423,14 @@ def test_full_size_prefill(name):
     att_ref = P.oracle_attn_rows(g["q"], g["k"], g["v"], idx_ref, rows, cfg.q_off,
                                  gate=g["gate"], gate_mode=cfg.gate)
     P.assert_attn_close(out[0, rows], att_ref, torch.bfloat16, f"{name} full")
+    # attention on many more rows -- every row of c2, 512 of c3/c5 -- against the oracle
+    # restated on the kernel's indices (checked above on every row against exact scores)
+    many = (list(range(S)) if S <= 4096 else
+            sorted(set(np.random.default_rng(2).integers(0, S, 512).tolist()) | set(rows)))
+    idx_np = P.to_np(idx[0])
+    att_many = P.oracle_attn_rows(g["q"], g["k"], g["v"], idx_np[many], many, cfg.q_off,
+                                  gate=g["gate"], gate_mode=cfg.gate)
+    P.assert_attn_close(out[0, many], att_many, torch.bfloat16, f"{name} full, {len(many)} rows")
 
 
 def test_full_size_decode():
