@@ -359,8 +359,23 @@ __global__ void __launch_bounds__(NT, NT == 256 ? 5 : (NT == 512 ? 3 : 1))
   // bitmap and the candidate list (key, position) while it has room.  Counts both.
   auto read2 = [&](uint32_t lo, uint32_t hi) {
     int my_sel = 0;
+    // long rows (SAMPLE): the next batch is in flight while this one is classified
+    uint32_t kn[SAMPLE ? U : 1][4];
+    if constexpr (SAMPLE) {
+      if (!held) load_keys<NT, U>(sc, n, 0, vec, kn);
+    }
     for (int base = 0; base < n; base += kChunk) {
-      if (!held) load_keys<NT, U>(sc, n, base, vec, kh);
+      if constexpr (SAMPLE) {
+        if (!held) {
+#pragma unroll
+          for (int u = 0; u < U; ++u)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) kh[u][e] = kn[u][e];
+          if (base + kChunk < n) load_keys<NT, U>(sc, n, base + kChunk, vec, kn);
+        }
+      } else {
+        if (!held) load_keys<NT, U>(sc, n, base, vec, kh);
+      }
       uint32_t gt[U], in[U];
       int c = 0;
 #pragma unroll
