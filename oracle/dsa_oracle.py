@@ -244,6 +244,21 @@ def window_attention(q, k, v, window, sm_scale=None, gate=None, gate_mode="off",
     return out
 
 
+def hadamard_rotate(x):
+    """The indexer's rotation of its inputs before FP8 quantisation.
+
+    [AXK2] SGA notes: the upstream indexer applies a Hadamard transform (rotate_activation)
+    before its FP8 scoring kernel, and since the transform is orthogonal (Hq . Hk = q . k)
+    the scores are unchanged.  Here: x [..., d] -> x @ H / sqrt(d) with H the d x d Sylvester
+    Hadamard matrix (natural order, H = H^T), d a power of two.  Returns float64.
+    """
+    from scipy.linalg import hadamard
+
+    x = _f64(x)
+    d = x.shape[-1]
+    return x @ hadamard(d).astype(np.float64) / np.sqrt(d)
+
+
 def dsa_forward(q_idx, k_idx, w, scale, K, q, k, v, sm_scale=None, gate=None,
                 gate_mode="off", relu="none", q_off=None, sink_k=None, sink_v=None):
     """The whole DSA step: indexer scores -> top-k -> sparse attention -> gate.

@@ -385,3 +385,33 @@ def test_decode_row_equals_last_prefill_row():
     assert np.array_equal(sc_d[:, 0], sc_p[:, -1])
     assert np.array_equal(idx_d[:, 0], idx_p[:, -1])
     assert np.allclose(out_d[:, 0], out_p[:, -1], rtol=1e-14, atol=1e-14)
+
+
+def test_hadamard_rotation_pins():
+    # H is symmetric and H H = d I: rotating twice is the identity; rotation preserves dot
+    # products (the scores do not change); the first basis vector maps to the all-equal
+    # vector 1/sqrt(d); a hand-written 4x4 case
+    rng = np.random.default_rng(9)
+    for d in (4, 64, 128):
+        x = rng.standard_normal((3, 5, d))
+        assert np.allclose(O.hadamard_rotate(O.hadamard_rotate(x)), x, rtol=0, atol=1e-12)
+        y = rng.standard_normal((7, d))
+        assert np.allclose(O.hadamard_rotate(x[0]) @ O.hadamard_rotate(y).T, x[0] @ y.T,
+                           rtol=0, atol=1e-10)
+        e0 = np.zeros(d)
+        e0[0] = 1.0
+        assert np.allclose(O.hadamard_rotate(e0), np.full(d, d ** -0.5), rtol=0, atol=1e-15)
+    x4 = np.array([1.0, 2.0, 3.0, 4.0])
+    # rows of H_4: (1,1,1,1), (1,-1,1,-1), (1,1,-1,-1), (1,-1,-1,1); x @ H / 2
+    assert np.allclose(O.hadamard_rotate(x4), np.array([10.0, -2.0, -4.0, 0.0]) / 2.0,
+                       rtol=0, atol=1e-15)
+    # the indexer scores are unchanged when both q_I and k_I are rotated
+    cfg_q = rng.integers(-2, 3, (1, 6, 4, 64)).astype(np.float64)
+    cfg_k = rng.integers(-2, 3, (1, 9, 64)).astype(np.float64)
+    w = rng.integers(1, 5, (1, 6, 4)).astype(np.float64)
+    a = O.index_scores(cfg_q, cfg_k, w, 0.25)
+    b = O.index_scores(O.hadamard_rotate(cfg_q), O.hadamard_rotate(cfg_k), w, 0.25)
+    fin = np.isfinite(a)
+    assert np.array_equal(np.isfinite(b), fin)
+    assert np.allclose(a[fin], b[fin], rtol=0, atol=1e-9)
+
