@@ -202,7 +202,8 @@ def sparse_attention(q, k, v, idx, sm_scale=None, gate=None, gate_mode="off", q_
     return out
 
 
-def window_attention(q, k, v, window, sm_scale=None, gate=None, gate_mode="off", q_off=None):
+def window_attention(q, k, v, window, sm_scale=None, gate=None, gate_mode="off", q_off=None,
+                     sink_k=None, sink_v=None):
     """Sliding-window causal attention with grouped KV heads (the SWA layers).
 
     [PANGU] §3.2: SWA layers interleave with DSA layers in a DSA-SWA-SWA pattern, with
@@ -211,6 +212,8 @@ def window_attention(q, k, v, window, sm_scale=None, gate=None, gate_mode="off",
 
     q [B,S,H,Dqk], k [B,T,HKV,Dqk], v [B,T,HKV,Dv]; query head h reads KV head
     h // (H // HKV).  Query s sees keys s+q_off-window < t <= s+q_off.
+    Optional attention sinks ([PANGU] §3.4, every layer): sink_k [NS,HKV,Dqk], sink_v
+    [NS,HKV,Dv], seen by every query (head h through KV head h // (H // HKV)).
     """
     q = _f64(q)
     k = _f64(k)
@@ -224,21 +227,28 @@ def window_attention(q, k, v, window, sm_scale=None, gate=None, gate_mode="off",
         q_off = T - S
     if sm_scale is None or sm_scale <= 0:
         sm_scale = 1.0 / np.sqrt(Dqk)
+    sinks = sink_k is not None
+    if sinks:
+        sk, sv = _f64(sink_k), _f64(sink_v)
     out = np.zeros((B, S, H, v.shape[-1]), dtype=np.float64)
     t_all = np.arange(T)
     for b in range(B):
         for s in range(S):
             pos = s + q_off
             allowed = (t_all <= pos) & (t_all > pos - window)
-            if not allowed.any():
+            if not allowed.any() and not sinks:
                 continue
             for h in range(H):
                 kh = h // G
                 logits = sm_scale * (k[b, :, kh, :] @ q[b, s, h, :])
                 logits[~allowed] = -np.inf
+                vals = v[b, :, kh, :]
+                if sinks:  # the sink entries, always visible
+                    logits = np.concatenate([logits, sm_scale * (sk[:, kh, :] @ q[b, s, h, :])])
+                    vals = np.concatenate([vals, sv[:, kh, :]])
                 p = np.exp(logits - logits.max())
                 p /= p.sum()
-                out[b, s, h] = p @ v[b, :, kh, :]
+                out[b, s, h] = p @ vals
     if gate_mode != "off":
         out = apply_gate(out, gate, gate_mode)
     return out

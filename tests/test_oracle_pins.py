@@ -366,6 +366,35 @@ def test_window_equals_sparse_with_band_indices():
         idx[0, s, : band.size] = band
     assert np.allclose(O.window_attention(q, k, v, W), O.sparse_attention(q, k, v, idx),
                        rtol=1e-13, atol=1e-13)
+    # the same with attention sinks in both (H == HKV, so the KV-head map is the identity)
+    sk, sv = rng.standard_normal((3, H, Dqk)), rng.standard_normal((3, H, Dv))
+    assert np.allclose(O.window_attention(q, k, v, W, sink_k=sk, sink_v=sv),
+                       O.sparse_attention(q, k, v, idx, sink_k=sk, sink_v=sv),
+                       rtol=1e-13, atol=1e-13)
+
+
+def test_window_sinks_with_grouped_heads():
+    # GQA: query head h sees the sinks of KV head h // G.  (1) Expanding K, V and the sinks
+    # to one head per query head gives the same result; (2) with window 1 (each query sees
+    # only its own key) the result is SDPA of the query over {its key, its head's sinks}.
+    rng = np.random.default_rng(13)
+    B, S, H, HKV, D, Dv, W, NS = 1, 7, 4, 2, 8, 5, 3, 2
+    G = H // HKV
+    q = rng.standard_normal((B, S, H, D))
+    k, v = rng.standard_normal((B, S, HKV, D)), rng.standard_normal((B, S, HKV, Dv))
+    sk, sv = rng.standard_normal((NS, HKV, D)), rng.standard_normal((NS, HKV, Dv))
+    got = O.window_attention(q, k, v, W, sink_k=sk, sink_v=sv)
+    rep = lambda x, ax: np.repeat(x, G, axis=ax)  # noqa: E731
+    ref = O.window_attention(q, rep(k, 2), rep(v, 2), W, sink_k=rep(sk, 1), sink_v=rep(sv, 1))
+    assert np.allclose(got, ref, rtol=0, atol=1e-13)
+    one = O.window_attention(q, k, v, 1, sink_k=sk, sink_v=sv)
+    for s in range(S):
+        for h in range(H):
+            kh = h // G
+            keys = np.concatenate([k[0, s:s + 1, kh], sk[:, kh]])[None, :, None]
+            vals = np.concatenate([v[0, s:s + 1, kh], sv[:, kh]])[None, :, None]
+            r = _sdpa_f64(q[:, s:s + 1, h:h + 1], keys, vals, causal=False)
+            assert np.allclose(one[0, s, h], r[0, 0, 0], rtol=0, atol=1e-12)
 
 
 # ----------------------------------------------------------------------------- decode
