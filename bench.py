@@ -169,7 +169,7 @@ class Workload:
     """Device buffers and the library calls of one step of config `name`."""
 
     def __init__(self, name, device, seed_offset=0, S=None, T=None, B=None, indexer="per_head",
-                 index_dtype="as_dtype", nsink=0):
+                 index_dtype="as_dtype", nsink=0, hadamard=False):
         import dataclasses
 
         import sparse_attention_15_b200 as dsa
@@ -225,24 +225,44 @@ class Workload:
         for layer in range(1, cfg.swa_layers + 1):
             s = swa_inputs(cfg, layer, device=device, seed=cfg.seed + seed_offset)
             s["out"] = torch.empty((B, cfg.S, cfg.H, cfg.dv), dtype=x["q"].dtype, device=device)
+            s["sink_k"] = s["sink_v"] = None
+            if nsink:  # every layer has its own sinks, one row per KV head
+                g = torch.Generator(device="cpu").manual_seed(cfg.seed + 7919 + layer)
+                hkv = s["k"].shape[2]
+                s["sink_k"] = torch.randn(nsink, hkv, cfg.dqk, generator=g).to(
+                    x["q"].dtype).to(device)
+                s["sink_v"] = torch.randn(nsink, hkv, cfg.dv, generator=g).to(
+                    x["q"].dtype).to(device)
             self.swa.append(s)
-        self.stages = ["indexer", "topk", "attention"] + [f"swa{i + 1}" for i in
-                                                          range(len(self.swa))]
+        # optional Hadamard rotation of the indexer inputs (prefill), a stage of its own
+        self.hadamard = hadamard and cfg.S > 1
+        if self.hadamard:
+            self.q_rot = torch.empty_like(x["q_idx"])
+            self.k_rot = torch.empty_like(x["k_idx"])
+        self.stages = (["hadamard"] if self.hadamard else []) + \
+            ["indexer", "topk", "attention"] + [f"swa{i + 1}" for i in range(len(self.swa))]
         # our kernels per step: indexer (+ the query collapse), top-k, attention (+ combine for
         # split gathers), SWA
         self.launches_per_step = 3 + (1 if self.algo == "gather" and gather_ws > 0 else 0) + \
-            (1 if indexer == "collapsed" else 0) + len(self.swa)
+            (1 if indexer == "collapsed" else 0) + (2 if self.hadamard else 0) + len(self.swa)
 
     def step(self, ev):
         """Run one step; ev is a list of len(stages)+1 CUDA events (stage boundaries)."""
         c, x, d = self.cfg, self.x, self.dsa
-        d.dsa_forward(x["q_idx"], x["k_idx"], x["w"], c.scale, c.K, x["q"], x["k"], x["v"],
+        qi, ki, e0 = x["q_idx"], x["k_idx"], 0
+        if self.hadamard:
+            ev[0].record()
+            qi = d.dsa_hadamard_rotate(x["q_idx"], out=self.q_rot)
+            ki = d.dsa_hadamard_rotate(x["k_idx"], out=self.k_rot)
+            e0 = 1
+        d.dsa_forward(qi, ki, x["w"], c.scale, c.K, x["q"], x["k"], x["v"],
                       gate=x["gate"], out=self.out, idx_out=self.idx, ws=self.ws,
-                      ws_bytes=self.ws_bytes, events=ev[:4], indexer=self.indexer,
+                      ws_bytes=self.ws_bytes, events=ev[e0:e0 + 4], indexer=self.indexer,
                       sink_k=self.sink_k, sink_v=self.sink_v)
         for i, s in enumerate(self.swa):
-            d.dsa_window_attn(s["q"], s["k"], s["v"], c.window, gate=s["gate"], out=s["out"])
-            ev[4 + i].record()
+            d.dsa_window_attn(s["q"], s["k"], s["v"], c.window, gate=s["gate"], out=s["out"],
+                              sink_k=s["sink_k"], sink_v=s["sink_v"])
+            ev[e0 + 4 + i].record()
 
     # algorithmic work per launch of each stage
     def work(self):
@@ -265,10 +285,13 @@ class Workload:
         else:
             idx_work = ("tensor" if c.dtype == "bf16" else "alu", 2.0 * c.HI * c.DI * pairs,
                         "TFLOP/s")
-        w = {
+        w = {}
+        if self.hadamard:  # read and write q_I and k_I once each
+            w["hadamard"] = ("hbm", 2.0 * (rows * c.HI * c.DI + B * c.T * c.DI) * es, "GB/s")
+        w.update({
             "indexer": idx_work,
             "topk": ("hbm", 4.0 * pairs + 4.0 * rows * self.K, "GB/s"),
-        }
+        })
         if self.algo == "masked_tile":
             # dense attention under the mask: QK^T and PV over every causal pair, all heads
             # (+ every query against the sinks)
@@ -279,7 +302,8 @@ class Workload:
                               rows * c.H * (c.dqk + c.dv) * es, "GB/s")
         for i in range(len(self.swa)):
             band = selected_pairs(c.S, c.T, B, c.q_off, c.window)
-            w[f"swa{i + 1}"] = ("tensor", 2.0 * c.H * (c.dqk + c.dv) * band, "TFLOP/s")
+            w[f"swa{i + 1}"] = ("tensor", 2.0 * c.H * (c.dqk + c.dv) * (band + rows * self.nsink),
+                                "TFLOP/s")
         return w
 
     def host_copy(self):
@@ -315,7 +339,8 @@ class Workload:
         for i, layer in enumerate(self.swa):
             g = {k: bufs.get(f"swa{i}_{k}", layer[k]) for k in ("q", "k", "v", "gate")}
             self.dsa.dsa_window_attn(g["q"], g["k"], g["v"], c.window, gate=g["gate"],
-                                     out=layer["out"])
+                                     out=layer["out"], sink_k=layer["sink_k"],
+                                     sink_v=layer["sink_v"])
 
     def e2e_pipelined(self, host, n, flush):
         """Prefill end to end over n steps: every step copies all its inputs from pinned host
@@ -494,6 +519,8 @@ def main():
                     help="indexer input type (the workload's dtype by default)")
     ap.add_argument("--sinks", type=int, default=0,
                     help="attention sinks (PAS virtual KV entries) per layer, 0..128")
+    ap.add_argument("--hadamard", action="store_true",
+                    help="rotate the indexer inputs (Hadamard) every prefill step")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world, rank, local = dist_setup(args)
@@ -518,7 +545,8 @@ def main():
         pg = dist
 
     wl = Workload(args.config, dev, seed_offset=rank, S=args.S, T=args.T, B=args.B,
-                  indexer=args.indexer, index_dtype=args.index_dtype, nsink=args.sinks)
+                  indexer=args.indexer, index_dtype=args.index_dtype, nsink=args.sinks,
+                  hadamard=args.hadamard)
     cfg = wl.cfg
     nst = len(wl.stages)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
@@ -661,7 +689,8 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32" if cfg.dtype == "f32" else "bf16", "data": "synthetic",
             "config": dict(workload_config(cfg, wl.B), indexer_form=wl.indexer,
-                           indexer_dtype=wl.index_dtype, sinks=wl.nsink),
+                           indexer_dtype=wl.index_dtype, sinks=wl.nsink,
+                           hadamard=wl.hadamard),
             "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
             "clocks": clk, "gpu_launches": wl.launches_per_step * args.steps,
             "wall_ms_per_step_incl_flush": round(1e3 * t_wall / args.steps, 4),

@@ -135,6 +135,19 @@ dsa_status dsa_index_scores_collapsed(dsa_dtype dtype, const void* q_idx, const 
                                       size_t ws_bytes, dsa_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
+ * 1c. Hadamard rotation of the indexer inputs.  [AXK2] SGA notes: the upstream indexer
+ *    rotates q_I and k_I with a Hadamard transform (rotate_activation) before quantising
+ *    them for FP8 scoring; the transform is orthogonal, so rotating both leaves every score
+ *    unchanged while spreading the values evenly over the dimensions.
+ *
+ *   x, out  [rows, d]  dtype (DSA_F32 or DSA_BF16), out = x @ H / sqrt(d), H the d x d
+ *           Sylvester Hadamard matrix; d in {64, 128}; out may be x (in place).
+ *   Float32 arithmetic, one rounding to dtype.  Pointers 16-byte aligned.
+ * --------------------------------------------------------------------------------- */
+dsa_status dsa_hadamard_rotate(dsa_dtype dtype, const void* x, long long rows, int d, void* out,
+                               dsa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
  * 2. Per-query top-k.  [AXK2] SGA: the indexer returns int32 indices [B,S,topk];
  *    "AXK2Config" (index_topk): topk = min(index_topk, number of keys).  [PANGU] §3.3:
  *    the number of selected keys is a fixed K.
@@ -275,6 +288,14 @@ dsa_status dsa_window_attn(dsa_dtype dtype, const void* q, const void* k, const 
                            const void* gate, dsa_gate_mode gate_mode, float sm_scale,
                            int window, int B, int S, int T, int H, int HKV, int DQK, int DV,
                            dsa_attn_algo algo, void* out, dsa_stream_t stream);
+/* The same with attention sinks ([PANGU] §3.4: every layer has its PAS entries): sink_k
+ * [nsink,HKV,DQK], sink_v [nsink,HKV,DV], 1 <= nsink <= 128, visible to every query (query
+ * head h through KV head h / (H/HKV)). */
+dsa_status dsa_window_attn_sinks(dsa_dtype dtype, const void* q, const void* k, const void* v,
+                                 const void* sink_k, const void* sink_v, int nsink,
+                                 const void* gate, dsa_gate_mode gate_mode, float sm_scale,
+                                 int window, int B, int S, int T, int H, int HKV, int DQK,
+                                 int DV, dsa_attn_algo algo, void* out, dsa_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
  * dsa_sparse_attn without any workspace: for callers that cannot allocate device memory.

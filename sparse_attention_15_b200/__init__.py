@@ -14,7 +14,8 @@ import os
 import torch
 
 __all__ = [
-    "DSAError", "lib", "dsa_index_scores", "dsa_index_scores_collapsed", "dsa_topk",
+    "DSAError", "lib", "dsa_index_scores", "dsa_index_scores_collapsed", "dsa_hadamard_rotate",
+    "dsa_topk",
     "dsa_sparse_attn", "dsa_sparse_attn_sinks", "dsa_sparse_attn_workspace_bytes",
     "dsa_sparse_attn_algo", "dsa_forward",
     "dsa_forward_workspace_bytes",
@@ -67,6 +68,7 @@ _SIGNATURES = {
     "dsa_index_scores_collapsed_workspace_bytes": (_Z, [_I, _I, _I]),
     "dsa_index_scores_collapsed": (_I, [_I, _P, _P, _P, _F, _I, _I, _I, _I, _I, _I, _P, _P, _Z,
                                         _P]),
+    "dsa_hadamard_rotate": (_I, [_I, _P, ctypes.c_longlong, _I, _P, _P]),
     "dsa_topk": (_I, [_P, _I, _I, _I, _I, _P, _P]),
     "dsa_sparse_attn_workspace_bytes": (_Z, [_I, _I, _I, _I, _I, _I, _I, _I, _I]),
     "dsa_sparse_attn_algo": (_I, [_I, _I, _I, _I, _I, _I, _I, _I, _I]),
@@ -80,6 +82,8 @@ _SIGNATURES = {
     "dsa_forward": (_I, [ctypes.POINTER(ForwardArgs), _P, _Z, _P]),
     "dsa_window_attn": (_I, [_I, _P, _P, _P, _P, _I, _F, _I, _I, _I, _I, _I, _I, _I, _I, _I,
                              _P, _P]),
+    "dsa_window_attn_sinks": (_I, [_I, _P, _P, _P, _P, _P, _I, _P, _I, _F, _I, _I, _I, _I, _I,
+                                   _I, _I, _I, _I, _P, _P]),
     "dsa_sparse_attn_noalloc_max_scratch_bytes": (_Z, []),
     "dsa_sparse_attn_noalloc": (_I, [_I, _P, _P, _P, _P, _I, _P, _I, _F, _I, _I, _I, _I, _I, _I,
                                      _P, _P]),
@@ -174,6 +178,17 @@ def dsa_index_scores_collapsed(q_idx, k_idx, w, scale, relu="none", scores=None,
                                             float(scale), RELU[relu], B, S, T, HI, DI,
                                             _ptr(scores), _ptr(ws), nbytes, _stream(stream)))
     return scores
+
+
+def dsa_hadamard_rotate(x, out=None, stream=None):
+    """x @ H / sqrt(d) over the last dimension (d in {64, 128}; float32 or bf16); out may be x."""
+    _dev(x, out)
+    d = x.shape[-1]
+    if out is None:
+        out = torch.empty_like(x)
+    _check(lib().dsa_hadamard_rotate(_dtype_code(x), _ptr(x), x.numel() // d, d, _ptr(out),
+                                     _stream(stream)))
+    return out
 
 
 def dsa_topk(scores, K, idx=None, stream=None):
@@ -329,15 +344,23 @@ def dsa_forward(q_idx, k_idx, w, index_scale, K, q, k, v, gate=None, gate_mode=N
 
 
 def dsa_window_attn(q, k, v, window, gate=None, gate_mode=None, sm_scale=0.0, algo="auto",
-                    out=None, stream=None):
-    """Sliding-window causal attention with grouped KV heads (window keys incl. self)."""
-    _dev(q, k, v, gate, out)
+                    out=None, stream=None, sink_k=None, sink_v=None):
+    """Sliding-window causal attention with grouped KV heads (window keys incl. self);
+    optional attention sinks sink_k [NS,HKV,DQK], sink_v [NS,HKV,DV] (NS <= 128)."""
+    _dev(q, k, v, gate, out, sink_k, sink_v)
     B, S, H, DQK = q.shape
     T, HKV, DV = k.shape[1], k.shape[2], v.shape[-1]
     gm = GATE[gate_mode or ("sigmoid" if gate is not None else "off")]
     if out is None:
         out = torch.empty((B, S, H, DV), dtype=q.dtype, device=q.device)
-    _check(lib().dsa_window_attn(_dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(gate), gm,
-                                 float(sm_scale), int(window), B, S, T, H, HKV, DQK, DV,
-                                 ATTN_ALGO[algo], _ptr(out), _stream(stream)))
+    if sink_k is None:
+        _check(lib().dsa_window_attn(_dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(gate), gm,
+                                     float(sm_scale), int(window), B, S, T, H, HKV, DQK, DV,
+                                     ATTN_ALGO[algo], _ptr(out), _stream(stream)))
+    else:
+        _check(lib().dsa_window_attn_sinks(_dtype_code(q), _ptr(q), _ptr(k), _ptr(v),
+                                           _ptr(sink_k), _ptr(sink_v), int(sink_k.shape[0]),
+                                           _ptr(gate), gm, float(sm_scale), int(window), B, S,
+                                           T, H, HKV, DQK, DV, ATTN_ALGO[algo], _ptr(out),
+                                           _stream(stream)))
     return out

@@ -263,6 +263,18 @@ dsa_status dsa_index_scores_collapsed(dsa_dtype dtype, const void* q_idx, const 
   return run_index_scores_collapsed(ws, k_idx, scale, relu, B, S, T, DI, T - S, scores, 1, s);
 }
 
+dsa_status dsa_hadamard_rotate(dsa_dtype dtype, const void* x, long long rows, int d, void* out,
+                               dsa_stream_t stream) {
+  REQUIRE(dtype == DSA_F32 || dtype == DSA_BF16, DSA_ERR_UNSUPPORTED,
+          "the rotation takes float32 or bf16 (dtype %d)", (int)dtype);
+  REQUIRE(x && out, DSA_ERR_INVALID_ARG, "null pointer argument");
+  REQUIRE(rows > 0, DSA_ERR_INVALID_ARG, "rows must be positive");
+  REQUIRE(d == 64 || d == 128, DSA_ERR_UNSUPPORTED, "d=%d must be 64 or 128", d);
+  REQUIRE(aligned16(x) && aligned16(out), DSA_ERR_UNSUPPORTED, "pointers must be 16-byte aligned");
+  return cuda_status(dsa::launch_hadamard((int)dtype, x, out, rows, d, (cudaStream_t)stream),
+                     "dsa_hadamard_rotate");
+}
+
 dsa_status dsa_topk(const float* scores, int B, int S, int T, int K, int32_t* idx,
                     dsa_stream_t stream) {
   REQUIRE(scores && idx, DSA_ERR_INVALID_ARG, "null pointer argument");
@@ -360,14 +372,16 @@ dsa_status dsa_sparse_attn_sinks(dsa_dtype dtype, const void* q, const void* k, 
                           sm_scale, B, S, T, H, DQK, DV, algo, out, ws, ws_bytes, stream);
 }
 
-dsa_status dsa_window_attn(dsa_dtype dtype, const void* q, const void* k, const void* v,
-                           const void* gate, dsa_gate_mode gate_mode, float sm_scale,
-                           int window, int B, int S, int T, int H, int HKV, int DQK, int DV,
-                           dsa_attn_algo algo, void* out, dsa_stream_t stream) {
+static dsa_status window_attn_impl(dsa_dtype dtype, const void* q, const void* k, const void* v,
+                                   const void* sink_k, const void* sink_v, int nsink,
+                                   const void* gate, dsa_gate_mode gate_mode, float sm_scale,
+                                   int window, int B, int S, int T, int H, int HKV, int DQK,
+                                   int DV, dsa_attn_algo algo, void* out, dsa_stream_t stream) {
   dsa_status st = check_attn_common(dtype, q, k, v, gate, gate_mode, sm_scale, B, S, T, H, HKV,
                                     DQK, DV, out);
   if (st != DSA_OK) return st;
   REQUIRE(window > 0, DSA_ERR_INVALID_ARG, "window must be positive");
+  if ((st = check_sinks(sink_k, sink_v, nsink)) != DSA_OK) return st;
   REQUIRE(algo >= DSA_ATTN_AUTO && algo <= DSA_ATTN_MASKED_TILE, DSA_ERR_INVALID_ARG,
           "unknown attention algorithm %d", (int)algo);
   const bool tc = dsa::masked_attn_supported((int)dtype, DQK, DV);
@@ -378,11 +392,31 @@ dsa_status dsa_window_attn(dsa_dtype dtype, const void* q, const void* k, const 
   p.gate = gate; p.gate_mode = (int)gate_mode; p.sm_scale = default_scale(sm_scale, DQK);
   p.B = B; p.S = S; p.T = T; p.H = H; p.HKV = HKV; p.DQK = DQK; p.DV = DV; p.q_off = T - S;
   p.out = out;
+  p.sink_k = nsink > 0 ? sink_k : nullptr; p.sink_v = nsink > 0 ? sink_v : nullptr;
+  p.nsink = nsink;
   cudaStream_t s = (cudaStream_t)stream;
   // the band is dense work for every query block with at least a few rows: tensor cores
   if (algo == DSA_ATTN_MASKED_TILE || (algo == DSA_ATTN_AUTO && tc && S >= 64))
     return cuda_status(dsa::launch_masked_attn(p, nullptr, 0, s), "dsa_window_attn");
   return cuda_status(dsa::launch_gather_attn(p, nullptr, 0, s), "dsa_window_attn");
+}
+
+dsa_status dsa_window_attn(dsa_dtype dtype, const void* q, const void* k, const void* v,
+                           const void* gate, dsa_gate_mode gate_mode, float sm_scale,
+                           int window, int B, int S, int T, int H, int HKV, int DQK, int DV,
+                           dsa_attn_algo algo, void* out, dsa_stream_t stream) {
+  return window_attn_impl(dtype, q, k, v, nullptr, nullptr, 0, gate, gate_mode, sm_scale, window,
+                          B, S, T, H, HKV, DQK, DV, algo, out, stream);
+}
+
+dsa_status dsa_window_attn_sinks(dsa_dtype dtype, const void* q, const void* k, const void* v,
+                                 const void* sink_k, const void* sink_v, int nsink,
+                                 const void* gate, dsa_gate_mode gate_mode, float sm_scale,
+                                 int window, int B, int S, int T, int H, int HKV, int DQK,
+                                 int DV, dsa_attn_algo algo, void* out, dsa_stream_t stream) {
+  REQUIRE(nsink > 0, DSA_ERR_INVALID_ARG, "nsink must be positive (use dsa_window_attn)");
+  return window_attn_impl(dtype, q, k, v, sink_k, sink_v, nsink, gate, gate_mode, sm_scale,
+                          window, B, S, T, H, HKV, DQK, DV, algo, out, stream);
 }
 
 // ----------------------------------------------------------------------------- forward

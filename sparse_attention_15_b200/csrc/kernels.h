@@ -43,6 +43,11 @@ cudaError_t launch_index_scores_collapsed(const void* qc, const void* k_idx, flo
                                           int relu, int B, int S, int T, int DI, int q_off,
                                           float* scores, int write_masked, cudaStream_t st);
 
+// Hadamard rotation of indexer inputs: out[r] = x[r] @ H / sqrt(d), d in {64, 128};
+// dtype 0 float32, 1 bf16; out may equal x.
+cudaError_t launch_hadamard(int dtype, const void* x, void* out, long long rows, int d,
+                            cudaStream_t st);
+
 // Per-row top-k (radix select + ordered compaction).  `mask` (optional) receives the
 // selection bitmask, one bit per key, rows of `mask_stride` 32-bit words
 // (mask_stride >= ceil(T/32); words past the row's keys are zero).

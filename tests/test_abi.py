@@ -92,6 +92,18 @@ def test_index_scores_collapsed_rejects_bad_arguments(lib):
     assert _collapsed(L, ws=FAKE_MIS) == 2
 
 
+def test_hadamard_rejects_bad_arguments(lib):
+    L = lib.lib()
+
+    def call(dtype=1, x=FAKE, rows=4, d=128, out=FAKE):
+        return L.dsa_hadamard_rotate(dtype, x, rows, d, out, None)
+    assert call(d=32) == 2
+    assert call(dtype=2) == 2            # e4m3 is quantised after the rotation
+    assert call(rows=0) == 1
+    assert call(x=None) == 1
+    assert call(out=FAKE_MIS) == 2
+
+
 def test_topk_rejects_bad_arguments(lib):
     L = lib.lib()
     assert L.dsa_topk(None, 1, 4, 4, 2, FAKE, None) == 1
@@ -146,6 +158,17 @@ def test_sparse_attn_sinks_rejects_bad_arguments(lib):
     assert call(sk=None) == 1
     assert call(sv=FAKE_MIS) == 2
     assert L.dsa_sparse_attn_sinks_workspace_bytes(1, 1, 4, 4, 2, 128, 128, 2, 4, 1) >= 0
+
+
+def test_window_attn_sinks_rejects_bad_arguments(lib):
+    L = lib.lib()
+
+    def call(nsink=4, sk=FAKE, sv=FAKE):
+        return L.dsa_window_attn_sinks(1, FAKE, FAKE, FAKE, sk, sv, nsink, None, 0, 0.0, 8, 1, 4,
+                                       4, 4, 2, 128, 128, 1, FAKE, None)
+    assert call(nsink=0) == 1
+    assert call(nsink=200) == 2
+    assert call(sv=None) == 1
 
 
 def test_window_attn_rejects_bad_arguments(lib):

@@ -101,6 +101,26 @@ def test_forward_e4m3_indexer_matches_bf16(name, S, T):
     assert torch.equal(out1, out2)
 
 
+# --------------------------------------------------------------- Hadamard rotation
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("rows,d", [(1, 64), (1001, 128), (77, 64), (4096, 128)])
+def test_hadamard_rotation_parity(dtype, rows, d):
+    # float32 butterflies over log2(d) stages: |err| <= 8 * 2^-24 * sum|x| / sqrt(d) per
+    # element, plus one rounding to the output type (2^-8 relative for bf16)
+    x = torch.randn(rows, d, generator=torch.Generator().manual_seed(rows + d)).to(dtype)
+    got = dsa.dsa_hadamard_rotate(x.to(DEV))
+    ref = O.hadamard_rotate(x)
+    bound = 8 * 2.0 ** -24 * np.abs(x.double().numpy()).sum(axis=1, keepdims=True) / np.sqrt(d)
+    if dtype == torch.bfloat16:
+        bound = bound + 2.0 ** -8 * np.abs(ref)
+    err = np.abs(P.to_np(got).astype(np.float64) - ref)
+    assert np.all(err <= bound + 1e-30), float((err - bound).max())
+    # in place gives the same bits
+    y = x.to(DEV)
+    dsa.dsa_hadamard_rotate(y, out=y)
+    assert torch.equal(y, got)
+
+
 # --------------------------------------------------------------- indexer, head-collapsed form
 COLLAPSED = [("c2", 333, 333), ("c2", 100, 517), ("c3", 200, 455), ("c5", 131, 300),
              ("c3", 1, 700)]
@@ -363,6 +383,24 @@ def test_window_attn_parity(S, T, W, algo):
     got = dsa.dsa_window_attn(g["q"], g["k"], g["v"], W, gate=g["gate"], algo=algo)
     ref = O.window_attention(x["q"], x["k"], x["v"], W, gate=x["gate"], gate_mode="sigmoid")
     P.assert_attn_close(got, ref, torch.bfloat16, f"swa W={W} {algo}")
+
+
+@pytest.mark.parametrize("S,T,W,NS", [(300, 300, 128, 128), (700, 700, 512, 77),
+                                      (100, 640, 512, 5)])
+@pytest.mark.parametrize("algo", ["gather", "masked_tile"])
+def test_window_attn_sinks_parity(S, T, W, NS, algo):
+    cfg = get_config("c5")
+    x = swa_inputs(cfg, 1, device="cpu", S=S, T=T)
+    g = {k: v.to(DEV) for k, v in x.items()}
+    gen = torch.Generator().manual_seed(NS + W)
+    HKV = x["k"].shape[2]
+    sk = torch.randn(NS, HKV, cfg.dqk, generator=gen).to(x["q"].dtype)
+    sv = torch.randn(NS, HKV, cfg.dv, generator=gen).to(x["q"].dtype)
+    got = dsa.dsa_window_attn(g["q"], g["k"], g["v"], W, gate=g["gate"], algo=algo,
+                              sink_k=sk.to(DEV), sink_v=sv.to(DEV))
+    ref = O.window_attention(x["q"], x["k"], x["v"], W, gate=x["gate"], gate_mode="sigmoid",
+                             sink_k=sk, sink_v=sv)
+    P.assert_attn_close(got, ref, torch.bfloat16, f"swa sinks W={W} NS={NS} {algo}")
 
 
 # ------------------------------------------------------------------------------- invariants
