@@ -191,7 +191,7 @@ __device__ __forceinline__ void key_range(const AttnArgs& a, const Item& it, int
 
 template <bool BAND>
 __device__ __forceinline__ int sink_blocks(const AttnArgs& a) {
-  return (!BAND && a.nsink > 0) ? 1 : 0;
+  return a.nsink > 0 ? 1 : 0;
 }
 
 template <class C>
@@ -401,16 +401,15 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         const uint32_t gg = g + j;
         const int t0 = (j0 + j - sb) * kBlk;
         uint32_t bits[4] = {0u, 0u, 0u, 0u};
-        if (!C::BAND) {
-          if (j < sb) {  // the sink block: its first nsink entries, visible to every query
+        if (j < sb) {  // the sink block: its first nsink entries, visible to every query
 #pragma unroll
-            for (int w = 0; w < 4; ++w) {
-              const int n = a.nsink - 32 * w;
-              bits[w] = n >= 32 ? 0xffffffffu : (n > 0 ? (1u << n) - 1u : 0u);
-            }
-          } else {
-            bits[0] = nb4.x; bits[1] = nb4.y; bits[2] = nb4.z; bits[3] = nb4.w;
+          for (int w = 0; w < 4; ++w) {
+            const int n = a.nsink - 32 * w;
+            bits[w] = n >= 32 ? 0xffffffffu : (n > 0 ? (1u << n) - 1u : 0u);
           }
+          if (!C::BAND && mrow && j + 2 < nb) nb4 = mask_words(j + 2);
+        } else if (!C::BAND) {
+          bits[0] = nb4.x; bits[1] = nb4.y; bits[2] = nb4.z; bits[3] = nb4.w;
           if (mrow && j + 2 < nb) nb4 = mask_words(j + 2);
         } else if (row_ok) {
           // band: spos - window < t <= spos, t < T
@@ -645,7 +644,7 @@ cudaError_t launch_fa(const AttnProblem& p, const uint32_t* mask, int mask_strid
       !map3d(&km, p.k, (uint64_t)p.B * p.T, p.HKV, C::DQK) ||
       !map3d(&vm, p.v, (uint64_t)p.B * p.T, p.HKV, C::DV))
     return cudaErrorInvalidValue;
-  const bool sinks = !C::BAND && p.sink_k != nullptr && p.nsink > 0;
+  const bool sinks = p.sink_k != nullptr && p.nsink > 0;
   if (sinks) {
     if (p.nsink > kBlk) return cudaErrorNotSupported;  // one sink block per item
     if (!map3d(&skm, p.sink_k, (uint64_t)p.nsink, p.HKV, C::DQK) ||
