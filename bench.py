@@ -626,7 +626,8 @@ def main():
     roof.pop("share")
     roof.update({"kernel": dom, "attention_algo": wl.algo, "traffic": traffic,
                  "tensor_peak_kind": "sustained" if long_step else "burst",
-                 "peak_source": f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'profiling recipe fallback'})"})
+                 "peak_source": "measured (MEASURED_PEAKS.json)" if peak_src == "measured" else
+                                "fallback (6.65 TB/s HBM, 1.59 / 1.40 PFLOP/s bf16 burst / sustained)"})
 
     # end-to-end through the public call with host buffers
     e2e = None

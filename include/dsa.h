@@ -54,7 +54,7 @@ typedef struct CUstream_st* dsa_stream_t;
 typedef enum {
   DSA_OK = 0,
   DSA_ERR_INVALID_ARG = 1, /* a null pointer, a non-positive size, an impossible shape   */
-  DSA_ERR_UNSUPPORTED = 2, /* a valid shape this build has no kernel for, misalignment  */
+  DSA_ERR_UNSUPPORTED = 2, /* a valid shape the library has no kernel for, misalignment */
   DSA_ERR_CUDA = 3,        /* a CUDA runtime / launch error                             */
   DSA_ERR_TIMEOUT = 4,     /* a bounded in-kernel wait gave up (see dsa_device_status)  */
   DSA_ERR_INTERNAL = 5     /* an in-kernel consistency check failed                     */
