@@ -32,6 +32,8 @@ Readings where the pages are silent (each also listed in the design notes):
 * gate rounding: multiply in float, round once (the A.X-K2 order).
 * an attention row with no selectable key outputs zeros.
 * SWA window W covers keys s+q_off-W < t <= s+q_off (W keys including the query itself).
+* latent (MQA-form) attention: every head attends over the same cached latent row, keys
+  = the whole row, values = its first dv dims (the absorbed MLA form flash-mla consumes).
 
 Parity pins: every function here is pinned by ``tests/test_oracle_pins.py`` against
 closed forms, hand-worked values (``tests/golden/``), brute force and library special
@@ -197,6 +199,58 @@ def sparse_attention(q, k, v, idx, sm_scale=None, gate=None, gate_mode="off", q_
             p = np.exp(logits - m)
             p /= p.sum(axis=1, keepdims=True)
             out[b, s] = np.matmul(p[:, None, :], vals)[:, 0, :]
+    if gate_mode != "off":
+        out = apply_gate(out, gate, gate_mode)
+    return out
+
+
+def sparse_attention_latent(q, kv, idx, dv, sm_scale=None, gate=None, gate_mode="off",
+                            q_off=None, sink_kv=None):
+    """Attention over the indexer-selected rows of a latent cache shared by all heads.
+
+    [AXK2] "注意力前向的骨架" step 2: kv_a_proj_with_mqa compresses K/V into a kv_lora_rank
+    latent plus a RoPE key slice shared by all heads; [AXK2] "注意力后端选择": the selected
+    positions are meant for flash-mla, which attends over that cache.  Reading taken: with
+    the up-projections absorbed into the queries and the output, head h's logit for key t is
+    sm_scale * q[h,:] . kv[t,:] and its output is the softmax-weighted sum of kv[t, :dv]
+    (the latent part of the row).  The mask is the one of sparse_attention: selected and
+    causal.  [PANGU] §3.4: for MLA the PAS pairs are latent KV rows, so the optional sinks
+    are sink_kv [NS,Dqk], visible to every query.
+
+    q [B,S,H,Dqk], kv [B,T,Dqk], idx [B,S,K].  Returns float64 [B,S,H,dv].
+    """
+    q = _f64(q)
+    kv = _f64(kv)
+    idx = np.asarray(idx)
+    B, S, H, Dqk = q.shape
+    T = kv.shape[1]
+    if q_off is None:
+        q_off = T - S
+    if sm_scale is None or sm_scale <= 0:
+        sm_scale = 1.0 / np.sqrt(Dqk)
+    sinks = sink_kv is not None
+    if sinks:
+        skv = _f64(sink_kv)  # [NS,Dqk]
+    out = np.zeros((B, S, H, dv), dtype=np.float64)
+    for b in range(B):
+        for s in range(S):
+            allowed = np.zeros(T, dtype=bool)
+            sel = idx[b, s]
+            sel = sel[(sel >= 0) & (sel < T)]
+            allowed[sel] = True
+            allowed[np.arange(T) > s + q_off] = False  # the causal mask
+            if not allowed.any() and not sinks:
+                continue
+            logits = sm_scale * (q[b, s] @ kv[b].T)  # [H,T]: every head reads the same rows
+            logits[:, ~allowed] = -np.inf
+            vals = kv[b, :, :dv]
+            if sinks:  # the latent sink rows, always visible
+                logits = np.concatenate([logits, sm_scale * (q[b, s] @ skv.T)], axis=1)
+                vals = np.concatenate([vals, skv[:, :dv]])
+            m = logits.max(axis=1, keepdims=True)
+            p = np.exp(logits - m)
+            p /= p.sum(axis=1, keepdims=True)
+            out[b, s] = p @ vals
     if gate_mode != "off":
         out = apply_gate(out, gate, gate_mode)
     return out

@@ -444,3 +444,74 @@ def test_hadamard_rotation_pins():
     assert np.array_equal(np.isfinite(b), fin)
     assert np.allclose(a[fin], b[fin], rtol=0, atol=1e-9)
 
+
+
+# ------------------------------------------------------------ latent (MQA-form) attention
+def test_latent_attention_hand_worked():
+    """Two selected rows of a 2-dim latent cache, dv = 1, sm_scale 1.  With q = (ln 3, 0) the
+    logits are 0 and ln 3, so the weights are 1/4 and 3/4; the values are the rows' first
+    dims, 0 and 1: output 3/4.  q = 0 weighs the two rows equally: 1/2.  Row 2 (a large
+    value) is not selected and must not count."""
+    kv = np.array([[[0.0, 0.0], [1.0, 5.0], [7.0, -3.0]]])  # [B=1, T=3, 2]
+    q = np.array([[[[math.log(3.0), 0.0], [0.0, 0.0]]]])  # [B=1, S=1, H=2, 2]
+    idx = np.array([[[0, 1]]])
+    out = O.sparse_attention_latent(q, kv, idx, dv=1, sm_scale=1.0)
+    assert out.shape == (1, 1, 2, 1)
+    np.testing.assert_allclose(out[0, 0, :, 0], [0.75, 0.5], rtol=0, atol=1e-15)
+
+
+def test_latent_attention_equals_the_per_head_form():
+    """Setting every head's key row to the shared latent row and its value row to the latent
+    row's first dv dims turns the per-head sparse attention (pinned against SDPA) into the
+    latent form: both give the same output, with and without sinks and the gate.  The index
+    lists hold -1, out-of-range and future entries."""
+    rng = np.random.default_rng(11)
+    B, S, T, H, D, dv, K = 2, 6, 9, 3, 8, 5, 4
+    q = rng.standard_normal((B, S, H, D))
+    kv = rng.standard_normal((B, T, D))
+    idx = rng.integers(-1, T + 2, size=(B, S, K))
+    g = rng.standard_normal((B, S, H))
+    k = np.repeat(kv[:, :, None, :], H, axis=2)
+    v = np.ascontiguousarray(k[..., :dv])
+    for sinks in (None, rng.standard_normal((3, D))):
+        for gm in ("off", "sigmoid"):
+            gate = g if gm != "off" else None
+            a = O.sparse_attention_latent(q, kv, idx, dv, gate=gate, gate_mode=gm, sink_kv=sinks)
+            sk = sv = None
+            if sinks is not None:
+                sk = np.repeat(sinks[:, None, :], H, axis=1)
+                sv = np.ascontiguousarray(sk[..., :dv])
+            b = O.sparse_attention(q, k, v, idx, gate=gate, gate_mode=gm, sink_k=sk, sink_v=sv)
+            np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-12)
+
+
+def test_latent_attention_closed_forms():
+    """One selected row gives every head that row's first dv dims; q = 0 gives every head
+    the mean of the selected rows' values; rows that are unselected or in the future never
+    count (poisoned with 1e4); permuting the heads of q permutes the output."""
+    rng = np.random.default_rng(12)
+    B, S, T, H, D, dv = 1, 4, 10, 5, 6, 4
+    kv = rng.standard_normal((B, T, D))
+    q = rng.standard_normal((B, S, H, D))
+    q_off = T - S
+    # a single selected key per query, plus a future key that the causal mask must drop
+    idx = np.array([[[3, T - 1], [5, -1], [0, 2 * T], [7, -1]]])
+    poisoned = kv.copy()
+    poisoned[0, 8] = 1e4  # selected only by the first query, at t = 9 > 0 + q_off: future
+    out = O.sparse_attention_latent(q, poisoned, idx, dv)
+    for s, t in enumerate([3, 5, 0, 7]):
+        np.testing.assert_allclose(out[0, s], np.broadcast_to(poisoned[0, t, :dv], (H, dv)),
+                                   rtol=0, atol=1e-12)
+    # q = 0: uniform weights over the selected causal rows
+    sel = np.array([[[1, 4, 6, -1]] * S])
+    out0 = O.sparse_attention_latent(np.zeros_like(q), kv, sel, dv)
+    mean = kv[0, [1, 4, 6], :dv].mean(axis=0)
+    for s in range(S):
+        np.testing.assert_allclose(out0[0, s], np.broadcast_to(mean, (H, dv)), rtol=0,
+                                   atol=1e-12)
+    # head permutation
+    perm = rng.permutation(H)
+    sel3 = rng.integers(0, q_off + 1, size=(B, S, 3))
+    a = O.sparse_attention_latent(q[:, :, perm], kv, sel3, dv)
+    b = O.sparse_attention_latent(q, kv, sel3, dv)[:, :, perm]
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)

@@ -13,6 +13,8 @@ from __future__ import annotations
 import torch
 
 _SLOTS = {"q_idx": 0, "k_idx": 1, "w": 2, "q": 3, "k": 4, "v": 5, "gate": 6}
+# the latent (MQA-form) attention inputs and the random selections use slots of their own
+_LATENT_SLOTS = {"q": 8, "kv": 9, "sink": 10, "sel": 11}
 
 
 def _gen(device, seed, slot):
@@ -92,3 +94,45 @@ def swa_inputs(cfg, layer, device="cpu", seed=None, B=None, S=None, T=None):
         "gate": (_normal((B, S, cfg.H), dt, device, _gen(device, seed, 6))
                  if cfg.gate != "off" else None),
     }
+
+
+def latent_inputs(cfg, H=128, dqk=576, device="cpu", seed=None, B=None, S=None, T=None,
+                  nsink=0):
+    """Inputs of the latent (MQA-form) attention of a DSA layer: absorbed queries
+    q [B,S,H,dqk], the latent cache kv [B,T,dqk] (one row per token, shared by all heads) and
+    optional latent sink rows sink_kv [nsink,dqk] (None when nsink == 0); N(0, 1) drawn in
+    float32 and rounded to the compute dtype, like the other attention inputs.  The gate,
+    when the config has one, is the config's own ``gate`` tensor (dsa_inputs) resized to H.
+    """
+    seed = cfg.seed if seed is None else seed
+    B = cfg.B if B is None else B
+    S = cfg.S if S is None else S
+    T = cfg.T if T is None else T
+    dt = _dtype(cfg.dtype)
+    sl = _LATENT_SLOTS
+    out = {
+        "q": _normal((B, S, H, dqk), dt, device, _gen(device, seed, sl["q"])),
+        "kv": _normal((B, T, dqk), dt, device, _gen(device, seed, sl["kv"])),
+        "sink_kv": (_normal((nsink, dqk), dt, device, _gen(device, seed, sl["sink"]))
+                    if nsink > 0 else None),
+        "gate": (_normal((B, S, H), dt, device, _gen(device, seed, 6))
+                 if cfg.gate != "off" else None),
+    }
+    return out
+
+
+def random_selection(B, S, T, K, seed, q_off=None):
+    """Random index lists shaped like the top-k output, on the CPU: row (b, s) holds
+    min(K, n) distinct keys drawn uniformly from the n = s + q_off + 1 causal keys, in
+    ascending order, then -1 padding.  int32 [B,S,K]."""
+    if q_off is None:
+        q_off = T - S
+    g = _gen("cpu", seed, _LATENT_SLOTS["sel"])
+    idx = torch.full((B, S, K), -1, dtype=torch.int32)
+    for b in range(B):
+        for s in range(S):
+            n = min(s + q_off + 1, T)
+            k = min(K, n)
+            pick = torch.randperm(n, generator=g)[:k]
+            idx[b, s, :k] = torch.sort(pick).values.to(torch.int32)
+    return idx
