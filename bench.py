@@ -30,6 +30,7 @@ import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 from workloads import dsa_inputs, get_config, swa_inputs  # noqa: E402
+from workloads.gen import latent_inputs  # noqa: E402
 
 METRIC = "query-tokens/s (indexer+top-k+sparse attn) and % of tensor/HBM roofline"
 UNIT = "query-tokens/s"
@@ -169,7 +170,8 @@ class Workload:
     """Device buffers and the library calls of one step of config `name`."""
 
     def __init__(self, name, device, seed_offset=0, S=None, T=None, B=None, indexer="per_head",
-                 index_dtype="as_dtype", nsink=0, hadamard=False):
+                 index_dtype="as_dtype", nsink=0, hadamard=False, attn_form="expanded",
+                 latent_heads=128):
         import dataclasses
 
         import sparse_attention_15_b200 as dsa
@@ -186,14 +188,27 @@ class Workload:
         self.cfg = cfg
         self.device = device
         B = cfg.B
+        self.attn_form = attn_form
+        latent = attn_form == "latent"
+        # latent (MQA-form) attention: one 512 + 64 latent row per token shared by the heads
+        self.H = latent_heads if latent else cfg.H
+        self.dqk, self.dv = (576, 512) if latent else (cfg.dqk, cfg.dv)
         if name == "c4":  # 174 GB of expanded K/V cache: shrink the batch only if it cannot fit
             free, _ = torch.cuda.mem_get_info(device)
-            per_row = cfg.T * (cfg.DI + cfg.H * (cfg.dqk + cfg.dv)) * 2
+            per_row = cfg.T * (cfg.DI + (self.dqk if latent else cfg.H * (cfg.dqk + cfg.dv))) * 2
             B = min(cfg.B, int((free - (6 << 30)) // per_row))
             if B < 1:
                 raise RuntimeError("not enough device memory for one decode batch row")
         self.B = B
-        x = dsa_inputs(cfg, device=device, B=B, seed=cfg.seed + seed_offset)
+        if latent:
+            x = dsa_inputs(cfg, device=device, B=B, seed=cfg.seed + seed_offset,
+                           need=("q_idx", "k_idx", "w"))
+            lt = latent_inputs(cfg, H=self.H, device=device, B=B, seed=cfg.seed + seed_offset,
+                               nsink=nsink)
+            # the attention tensors: q [B,S,H,576], k = the latent cache [B,T,576], no v
+            x.update({"q": lt["q"], "k": lt["kv"], "v": None, "gate": lt["gate"]})
+        else:
+            x = dsa_inputs(cfg, device=device, B=B, seed=cfg.seed + seed_offset)
         self.index_dtype = index_dtype
         if index_dtype == "e4m3":  # indexer inputs handed over as e4m3 (exact for the integers)
             x["q_idx"] = x["q_idx"].to(torch.float8_e4m3fn)
@@ -201,7 +216,9 @@ class Workload:
         self.x = x
         self.nsink = nsink
         self.sink_k = self.sink_v = None
-        if nsink:  # attention sinks (PAS): synthetic per-head sink rows, N(0,1)
+        if nsink and latent:  # latent sink rows [nsink, 576]
+            self.sink_k = lt["sink_kv"]
+        elif nsink:  # attention sinks (PAS): synthetic per-head sink rows, N(0,1)
             g = torch.Generator(device="cpu").manual_seed(cfg.seed + 7919)
             self.sink_k = torch.randn(nsink, cfg.H, cfg.dqk, generator=g).to(
                 x["q"].dtype).to(device)
@@ -209,18 +226,24 @@ class Workload:
                 x["q"].dtype).to(device)
         self.K = cfg.k_eff
         self.idx = torch.empty((B, cfg.S, self.K), dtype=torch.int32, device=device)
-        self.out = torch.empty((B, cfg.S, cfg.H, cfg.dv), dtype=x["q"].dtype, device=device)
+        self.out = torch.empty((B, cfg.S, self.H, self.dv), dtype=x["q"].dtype, device=device)
         self.indexer = indexer
         self.args = dsa._forward_args(x["q_idx"], x["k_idx"], x["w"], cfg.scale, cfg.K, x["q"],
                                       x["k"], x["v"], x["gate"], None, "none", 0.0, "auto",
                                       self.out, None, self.idx,
-                                      indexer, self.sink_k, self.sink_v)
+                                      indexer, self.sink_k, self.sink_v, attn_form, self.dv)
         self.ws_bytes = dsa.dsa_forward_workspace_bytes(self.args)
         self.ws = torch.empty(max(self.ws_bytes, 16), dtype=torch.uint8, device=device)
         dt = dsa.DTYPE[x["q"].dtype]
-        self.algo = dsa.dsa_sparse_attn_algo(dt, B, cfg.S, cfg.T, cfg.H, cfg.dqk, cfg.dv, self.K)
-        gather_ws = dsa.dsa_sparse_attn_workspace_bytes(dt, B, cfg.S, cfg.T, cfg.H, cfg.dqk,
-                                                        cfg.dv, self.K, "gather")
+        if latent:
+            self.algo = "latent"
+            split_ws = dsa.lib().dsa_sparse_attn_latent_workspace_bytes(B, cfg.S, self.H, self.K,
+                                                                        nsink)
+        else:
+            self.algo = dsa.dsa_sparse_attn_algo(dt, B, cfg.S, cfg.T, cfg.H, cfg.dqk, cfg.dv,
+                                                 self.K)
+            split_ws = dsa.dsa_sparse_attn_workspace_bytes(dt, B, cfg.S, cfg.T, cfg.H, cfg.dqk,
+                                                           cfg.dv, self.K, "gather")
         self.swa = []
         for layer in range(1, cfg.swa_layers + 1):
             s = swa_inputs(cfg, layer, device=device, seed=cfg.seed + seed_offset)
@@ -243,8 +266,18 @@ class Workload:
             ["indexer", "topk", "attention"] + [f"swa{i + 1}" for i in range(len(self.swa))]
         # our kernels per step: indexer (+ the query collapse), top-k, attention (+ combine for
         # split gathers), SWA
-        self.launches_per_step = 3 + (1 if self.algo == "gather" and gather_ws > 0 else 0) + \
+        self.launches_per_step = 3 + \
+            (1 if self.algo in ("gather", "latent") and split_ws > 0 else 0) + \
             (1 if indexer == "collapsed" else 0) + (2 if self.hadamard else 0) + len(self.swa)
+
+    def _forward(self, x, events=None):
+        """The DSA layer through the public whole-step call."""
+        c = self.cfg
+        self.dsa.dsa_forward(x["q_idx"], x["k_idx"], x["w"], c.scale, c.K, x["q"], x["k"],
+                             x["v"], gate=x["gate"], out=self.out, idx_out=self.idx,
+                             ws=self.ws, ws_bytes=self.ws_bytes, events=events,
+                             indexer=self.indexer, sink_k=self.sink_k, sink_v=self.sink_v,
+                             attn_form=self.attn_form, dv=self.dv)
 
     def step(self, ev):
         """Run one step; ev is a list of len(stages)+1 CUDA events (stage boundaries)."""
@@ -255,10 +288,7 @@ class Workload:
             qi = d.dsa_hadamard_rotate(x["q_idx"], out=self.q_rot)
             ki = d.dsa_hadamard_rotate(x["k_idx"], out=self.k_rot)
             e0 = 1
-        d.dsa_forward(qi, ki, x["w"], c.scale, c.K, x["q"], x["k"], x["v"],
-                      gate=x["gate"], out=self.out, idx_out=self.idx, ws=self.ws,
-                      ws_bytes=self.ws_bytes, events=ev[e0:e0 + 4], indexer=self.indexer,
-                      sink_k=self.sink_k, sink_v=self.sink_v)
+        self._forward(dict(x, q_idx=qi, k_idx=ki), events=ev[e0:e0 + 4])
         for i, s in enumerate(self.swa):
             d.dsa_window_attn(s["q"], s["k"], s["v"], c.window, gate=s["gate"], out=s["out"],
                               sink_k=s["sink_k"], sink_v=s["sink_v"])
@@ -292,7 +322,12 @@ class Workload:
             "indexer": idx_work,
             "topk": ("hbm", 4.0 * pairs + 4.0 * rows * self.K, "GB/s"),
         })
-        if self.algo == "masked_tile":
+        if self.algo == "latent":
+            # every selected (query, key) pair, all heads: S = q . kv (2*H*576 flops) and
+            # O += p kv[:512] (2*H*512); + every query against the sinks
+            w["attention"] = ("tensor", 2.0 * self.H * (self.dqk + self.dv) *
+                              (sel + rows * self.nsink), "TFLOP/s")
+        elif self.algo == "masked_tile":
             # dense attention under the mask: QK^T and PV over every causal pair, all heads
             # (+ every query against the sinks)
             w["attention"] = ("tensor", 2.0 * c.H * (c.dqk + c.dv) * (pairs + rows * self.nsink),
@@ -313,8 +348,9 @@ class Workload:
         x = self.x
         if self.cfg.S == 1:
             sel = {"q_idx": x["q_idx"], "w": x["w"], "q": x["q"], "gate": x["gate"],
-                   "k_idx_row": x["k_idx"][:, -1:], "k_row": x["k"][:, -1:],
-                   "v_row": x["v"][:, -1:]}
+                   "k_idx_row": x["k_idx"][:, -1:], "k_row": x["k"][:, -1:]}
+            if x["v"] is not None:
+                sel["v_row"] = x["v"][:, -1:]
         else:
             sel = dict(x)
             for i, layer in enumerate(self.swa):
@@ -332,10 +368,7 @@ class Workload:
         c = self.cfg
         x = dict(self.x)
         x.update({k: v for k, v in bufs.items() if not k.startswith("swa")})
-        self.dsa.dsa_forward(x["q_idx"], x["k_idx"], x["w"], c.scale, c.K, x["q"], x["k"],
-                             x["v"], gate=x["gate"], out=self.out, idx_out=self.idx,
-                             ws=self.ws, ws_bytes=self.ws_bytes, indexer=self.indexer,
-                             sink_k=self.sink_k, sink_v=self.sink_v)
+        self._forward(x)
         for i, layer in enumerate(self.swa):
             g = {k: bufs.get(f"swa{i}_{k}", layer[k]) for k in ("q", "k", "v", "gate")}
             self.dsa.dsa_window_attn(g["q"], g["k"], g["v"], c.window, gate=g["gate"],
@@ -396,18 +429,15 @@ class Workload:
             else:
                 dev_bufs[k].copy_(v, non_blocking=True)
                 x[k] = dev_bufs[k]
-        c = self.cfg
-        self.dsa.dsa_forward(x["q_idx"], x["k_idx"], x["w"], c.scale, c.K, x["q"], x["k"],
-                             x["v"], gate=x["gate"], out=self.out, idx_out=self.idx,
-                             ws=self.ws, ws_bytes=self.ws_bytes, indexer=self.indexer,
-                             sink_k=self.sink_k, sink_v=self.sink_v)
+        self._forward(x)
         out_host.copy_(self.out, non_blocking=True)
 
 
 # ----------------------------------------------------------------------------- oracle timing
-def oracle_rows_per_s(cfg, x_host, rows, budget_s):
+def oracle_rows_per_s(cfg, x_host, rows, budget_s, sink_kv=None):
     """The CPU oracle as it stands, on sampled query rows of batch row 0: returns
-    (rows done, seconds).  Each row runs scores -> top-k -> dense masked attention."""
+    (rows done, seconds).  Each row runs scores -> top-k -> dense masked attention (over
+    the shared latent rows when x_host has no v: the latent form)."""
     from oracle import dsa_oracle as O
 
     q_off = cfg.q_off
@@ -419,8 +449,12 @@ def oracle_rows_per_s(cfg, x_host, rows, budget_s):
                             cfg.scale, q_off=s + q_off)
         idx = O.topk_indices(sc, cfg.k_eff, q_off=s + q_off)
         g = None if x_host["gate"] is None else x_host["gate"][:1, sl]
-        O.sparse_attention(x_host["q"][:1, sl], x_host["k"][:1], x_host["v"][:1], idx,
-                           gate=g, gate_mode=cfg.gate, q_off=s + q_off)
+        if x_host["v"] is None:
+            O.sparse_attention_latent(x_host["q"][:1, sl], x_host["k"][:1], idx, 512, gate=g,
+                                      gate_mode=cfg.gate, q_off=s + q_off, sink_kv=sink_kv)
+        else:
+            O.sparse_attention(x_host["q"][:1, sl], x_host["k"][:1], x_host["v"][:1], idx,
+                               gate=g, gate_mode=cfg.gate, q_off=s + q_off)
         done += 1
         if time.perf_counter() - t0 > budget_s:
             break
@@ -521,6 +555,11 @@ def main():
                     help="attention sinks (PAS virtual KV entries) per layer, 0..128")
     ap.add_argument("--hadamard", action="store_true",
                     help="rotate the indexer inputs (Hadamard) every prefill step")
+    ap.add_argument("--attn", default="expanded", choices=["expanded", "latent"],
+                    help="attention over the expanded per-head K/V (the workloads' form) or "
+                         "over a shared 512+64 latent cache (MQA form)")
+    ap.add_argument("--latent-heads", type=int, default=128,
+                    help="query heads of the latent form (<= 128)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world, rank, local = dist_setup(args)
@@ -546,7 +585,7 @@ def main():
 
     wl = Workload(args.config, dev, seed_offset=rank, S=args.S, T=args.T, B=args.B,
                   indexer=args.indexer, index_dtype=args.index_dtype, nsink=args.sinks,
-                  hadamard=args.hadamard)
+                  hadamard=args.hadamard, attn_form=args.attn, latent_heads=args.latent_heads)
     cfg = wl.cfg
     nst = len(wl.stages)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
@@ -615,11 +654,11 @@ def main():
                          "frac": round(ach / peak, 4),
                          "share": round(float(stage_ms[j]) / float(stage_ms.sum()), 4)}
     dom = max(kernels, key=lambda k: kernels[k]["ms"])
-    attn_k = "masked_attn" if wl.algo == "masked_tile" else "gather_attn"
+    attn_k = {"masked_tile": "masked_attn", "latent": "latent_attn"}.get(wl.algo, "gather_attn")
     kname = {"indexer": "index_scores", "topk": "topk", "attention": attn_k}.get(dom, "masked_attn")
     tr = NCU_TRAFFIC.get((kname, cfg.name))
     srcfile = {"index_scores": "indexer_tc.cu", "topk": "topk.cu", "gather_attn": "gather_attn.cu",
-               "masked_attn": "attn_tc.cu"}[kname]
+               "masked_attn": "attn_tc.cu", "latent_attn": "latent_attn.cu"}[kname]
     traffic = tr[0] if tr and tr[1] == src_sha(srcfile) else None
     roof = dict(kernels[dom])
     roof.pop("ms")
@@ -677,7 +716,8 @@ def main():
         rows = sample_rows(cfg.S, 4096)
         rng = np.random.default_rng(0)
         rng.shuffle(rows)
-        n, sec = oracle_rows_per_s(cfg, xh, rows, args.cpu_budget)
+        skv = None if wl.sink_k is None or wl.attn_form != "latent" else wl.sink_k.cpu()
+        n, sec = oracle_rows_per_s(cfg, xh, rows, args.cpu_budget, sink_kv=skv)
         cpu = {"value": n / sec, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                "sample": f"{n} query rows of batch row 0 drawn evenly over the {cfg.S} "
                          f"queries, {sec:.1f} s of float64 numpy oracle work "
@@ -691,7 +731,9 @@ def main():
             "dtype": "f32" if cfg.dtype == "f32" else "bf16", "data": "synthetic",
             "config": dict(workload_config(cfg, wl.B), indexer_form=wl.indexer,
                            indexer_dtype=wl.index_dtype, sinks=wl.nsink,
-                           hadamard=wl.hadamard),
+                           hadamard=wl.hadamard, attention_form=wl.attn_form,
+                           **({"heads": wl.H, "qk_dim": "512+64 (latent, shared by all heads)",
+                               "v_dim": 512} if wl.attn_form == "latent" else {})),
             "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
             "clocks": clk, "gpu_launches": wl.launches_per_step * args.steps,
             "wall_ms_per_step_incl_flush": round(1e3 * t_wall / args.steps, 4),

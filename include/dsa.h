@@ -80,6 +80,10 @@ typedef enum { DSA_GATE_OFF = 0, DSA_GATE_SIGMOID = 1, DSA_GATE_SILU = 2 } dsa_g
 /* How dsa_forward computes the indexer scores (section 1 or section 1b). */
 typedef enum { DSA_INDEXER_PER_HEAD = 0, DSA_INDEXER_COLLAPSED = 1 } dsa_indexer_mode;
 
+/* Form of the attention cache dsa_forward attends over: per-head expanded K/V (section 3)
+ * or one latent row per token shared by all heads (section 3c). */
+typedef enum { DSA_ATTN_EXPANDED = 0, DSA_ATTN_LATENT = 1 } dsa_attn_form;
+
 /* Attention algorithm for dsa_forward, dsa_sparse_attn and dsa_window_attn. */
 typedef enum {
   DSA_ATTN_AUTO = 0,      /* pick by the cost model (bytes gathered vs. dense tile work)  */
@@ -228,6 +232,38 @@ dsa_status dsa_sparse_attn_sinks(dsa_dtype dtype, const void* q, const void* k, 
                                  size_t ws_bytes, dsa_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
+ * 3c. Sparse attention over a shared latent cache (the MQA form of MLA).
+ *    [AXK2] "注意力前向的骨架" step 2: kv_a_proj_with_mqa compresses K/V into a
+ *    kv_lora_rank latent plus a RoPE key slice shared by all heads; [AXK2] "注意力后端选择":
+ *    the indexer's positions are for flash-mla (flash_mla_with_kvcache), which attends over
+ *    that latent cache.  With the up-projections absorbed into q and the output, every head
+ *    attends over the same cached row: logit(h,t) = sm_scale * q[h,:] . kv[t,:] and
+ *    out[h,:] = sum_t p(h,t) kv[t, 0:DV].  [PANGU] §3.4: for MLA the PAS sinks are latent
+ *    rows as well.
+ *
+ *   q       [B,S,H,DQK]  bf16     absorbed queries ([latent | rope] per head)
+ *   kv      [B,T,DQK]    bf16     latent cache: keys are whole rows, values their first DV
+ *                                 dims
+ *   idx     [B,S,K]      int32    as dsa_sparse_attn (-1, out-of-range and future entries
+ *                                 are skipped; valid entries distinct)
+ *   sink_kv [nsink,DQK]  bf16     latent sink rows visible to every query, or NULL with
+ *                                 nsink == 0; 0 <= nsink <= 128
+ *   gate    [B,S,H]      bf16     or NULL with DSA_GATE_OFF
+ *   out     [B,S,H,DV]   bf16     float32 accumulation, one rounding, gate before it; a row
+ *                                 with no valid key gets zeros
+ *   Requires bf16, DQK == 576 and DV == 512 (kv_lora_rank 512 + a 64-dim RoPE slice),
+ *   1 <= H <= 128, 16-byte aligned pointers.  Tensor-core kernel: S = Q kv^T per block of 32
+ *   selected rows with M = 128 heads, then O += P V.  Workspace (split-key partials of
+ *   decode-shaped calls) from dsa_sparse_attn_latent_workspace_bytes; 0 -> NULL is fine.
+ * --------------------------------------------------------------------------------- */
+size_t dsa_sparse_attn_latent_workspace_bytes(int B, int S, int H, int K, int nsink);
+dsa_status dsa_sparse_attn_latent(dsa_dtype dtype, const void* q, const void* kv,
+                                  const int32_t* idx, int K, const void* sink_kv, int nsink,
+                                  const void* gate, dsa_gate_mode gate_mode, float sm_scale,
+                                  int B, int S, int T, int H, int DQK, int DV, void* out,
+                                  void* ws, size_t ws_bytes, dsa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
  * The whole DSA step: 1 -> 2 -> 3+4.  [AXK2] "注意力前向的骨架" steps 4-5.
  * Scores and indices go to the caller's buffers when scores_out / idx_out are given,
  * else to the workspace.  Without scores_out the score buffer may be smaller than
@@ -264,6 +300,10 @@ typedef struct {
   const void* sink_k;      /* optional [nsink,H,DQK] attention sinks (section 3b)        */
   const void* sink_v;      /* [nsink,H,DV]                                               */
   int nsink;               /* 0 (none) .. 128                                            */
+  dsa_attn_form attn_form; /* DSA_ATTN_EXPANDED (0): k, v and the sinks as above;
+                              DSA_ATTN_LATENT: k is the latent cache [B,T,DQK] of section
+                              3c, v is unused (NULL), sink_k holds [nsink,DQK] latent sink
+                              rows, sink_v is unused; attn_algo is ignored                */
 } dsa_forward_args;
 
 /* Bytes of workspace dsa_forward needs to run without row blocking. */

@@ -30,6 +30,7 @@ RELU = {"none": 0, "post_sum": 1, "per_head": 2}
 GATE = {"off": 0, "sigmoid": 1, "silu": 2}
 ATTN_ALGO = {"auto": 0, "gather": 1, "masked_tile": 2}
 INDEXER = {"per_head": 0, "collapsed": 1}
+ATTN_FORM = {"expanded": 0, "latent": 1}
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "CUDA error", 4: "timeout",
           5: "internal"}
 
@@ -53,7 +54,7 @@ class ForwardArgs(ctypes.Structure):
         ("gate", ctypes.c_void_p), ("out", ctypes.c_void_p), ("scores_out", ctypes.c_void_p),
         ("idx_out", ctypes.c_void_p), ("events", ctypes.c_void_p), ("indexer", ctypes.c_int),
         ("index_dtype", ctypes.c_int), ("sink_k", ctypes.c_void_p), ("sink_v", ctypes.c_void_p),
-        ("nsink", ctypes.c_int),
+        ("nsink", ctypes.c_int), ("attn_form", ctypes.c_int),
     ]
 
 
@@ -77,6 +78,9 @@ _SIGNATURES = {
     "dsa_sparse_attn_sinks_workspace_bytes": (_Z, [_I, _I, _I, _I, _I, _I, _I, _I, _I, _I]),
     "dsa_sparse_attn_sinks": (_I, [_I, _P, _P, _P, _P, _I, _P, _P, _I, _P, _I, _F, _I, _I, _I,
                                    _I, _I, _I, _I, _P, _P, _Z, _P]),
+    "dsa_sparse_attn_latent_workspace_bytes": (_Z, [_I, _I, _I, _I, _I]),
+    "dsa_sparse_attn_latent": (_I, [_I, _P, _P, _P, _I, _P, _I, _P, _I, _F, _I, _I, _I, _I, _I,
+                                    _I, _P, _P, _Z, _P]),
     "dsa_forward_workspace_bytes": (_Z, [ctypes.POINTER(ForwardArgs)]),
     "dsa_forward_min_workspace_bytes": (_Z, [ctypes.POINTER(ForwardArgs)]),
     "dsa_forward": (_I, [ctypes.POINTER(ForwardArgs), _P, _Z, _P]),
@@ -281,26 +285,48 @@ def dsa_sparse_attn_noalloc(q, k, v, idx, gate=None, gate_mode=None, sm_scale=0.
     return out
 
 
+def dsa_sparse_attn_latent(q, kv, idx, dv=512, sink_kv=None, gate=None, gate_mode=None,
+                           sm_scale=0.0, out=None, ws=None, stream=None):
+    """Sparse attention over a shared latent cache (MQA form): q [B,S,H,DQK], kv [B,T,DQK]
+    (keys = whole rows, values = their first ``dv`` dims), idx [B,S,K]; optional latent sink
+    rows sink_kv [NS,DQK] (NS <= 128).  bf16, DQK 576, dv 512, H <= 128."""
+    _dev(q, kv, idx, sink_kv, gate, out, ws)
+    B, S, H, DQK = q.shape
+    T = kv.shape[1]
+    K = idx.shape[-1]
+    NS = 0 if sink_kv is None else int(sink_kv.shape[0])
+    gm = GATE[gate_mode or ("sigmoid" if gate is not None else "off")]
+    if out is None:
+        out = torch.empty((B, S, H, dv), dtype=q.dtype, device=q.device)
+    nbytes = int(lib().dsa_sparse_attn_latent_workspace_bytes(B, S, H, K, NS))
+    ws = _workspace(nbytes, q.device, ws)
+    _check(lib().dsa_sparse_attn_latent(_dtype_code(q), _ptr(q), _ptr(kv), _ptr(idx), K,
+                                        _ptr(sink_kv), NS, _ptr(gate), gm, float(sm_scale), B, S,
+                                        T, H, DQK, int(dv), _ptr(out), _ptr(ws), nbytes,
+                                        _stream(stream)))
+    return out
+
+
 def _forward_args(q_idx, k_idx, w, index_scale, K, q, k, v, gate, gate_mode, relu, sm_scale,
                   attn_algo, out, scores_out, idx_out, indexer="per_head", sink_k=None,
-                  sink_v=None):
+                  sink_v=None, attn_form="expanded", dv=512):
     B, S, HI, DI = q_idx.shape
     T = k_idx.shape[1]
     H, DQK = q.shape[2], q.shape[3]
-    DV = v.shape[-1]
+    DV = int(dv) if attn_form == "latent" else v.shape[-1]
     gm = GATE[gate_mode or ("sigmoid" if gate is not None else "off")]
     a = ForwardArgs(
         dtype=_dtype_code(q), B=B, S=S, T=T, HI=HI, DI=DI, index_scale=float(index_scale),
         relu=RELU[relu], K=int(K), H=H, DQK=DQK, DV=DV, sm_scale=float(sm_scale), gate_mode=gm,
         attn_algo=ATTN_ALGO[attn_algo], q_idx=q_idx.data_ptr(), k_idx=k_idx.data_ptr(),
-        w=w.data_ptr(), q=q.data_ptr(), k=k.data_ptr(), v=v.data_ptr(),
+        w=w.data_ptr(), q=q.data_ptr(), k=k.data_ptr(), v=None if v is None else v.data_ptr(),
         gate=None if gate is None else gate.data_ptr(), out=out.data_ptr(),
         scores_out=None if scores_out is None else scores_out.data_ptr(),
         idx_out=None if idx_out is None else idx_out.data_ptr(), indexer=INDEXER[indexer],
         index_dtype=1 if q_idx.dtype == torch.float8_e4m3fn else 0,
         sink_k=None if sink_k is None else sink_k.data_ptr(),
         sink_v=None if sink_v is None else sink_v.data_ptr(),
-        nsink=0 if sink_k is None else int(sink_k.shape[0]))
+        nsink=0 if sink_k is None else int(sink_k.shape[0]), attn_form=ATTN_FORM[attn_form])
     return a
 
 
@@ -312,10 +338,11 @@ def dsa_forward_workspace_bytes(args: ForwardArgs, minimum: bool = False) -> int
 def dsa_forward(q_idx, k_idx, w, index_scale, K, q, k, v, gate=None, gate_mode=None,
                 relu="none", sm_scale=0.0, attn_algo="auto", out=None, scores_out=None,
                 idx_out=None, ws=None, ws_bytes=None, stream=None, events=None,
-                indexer="per_head", sink_k=None, sink_v=None):
+                indexer="per_head", sink_k=None, sink_v=None, attn_form="expanded", dv=512):
     """The whole DSA step (indexer -> top-k -> sparse attention -> gate).
     indexer: "per_head" (the pages' per-head work) or "collapsed" (see
-    dsa_index_scores_collapsed).
+    dsa_index_scores_collapsed).  attn_form "latent": k is the latent cache [B,T,DQK]
+    (values = its first ``dv`` dims), v is None, sink_k holds latent sink rows [NS,DQK].
 
     Returns (out, idx); idx is idx_out if given, else a view of the workspace copy.
     ``ws_bytes`` limits the workspace handed to the library (row blocking below the
@@ -324,12 +351,14 @@ def dsa_forward(q_idx, k_idx, w, index_scale, K, q, k, v, gate=None, gate_mode=N
     B, S = q_idx.shape[:2]
     T = k_idx.shape[1]
     if out is None:
-        out = torch.empty((B, S, q.shape[2], v.shape[-1]), dtype=q.dtype, device=q.device)
+        DV = int(dv) if attn_form == "latent" else v.shape[-1]
+        out = torch.empty((B, S, q.shape[2], DV), dtype=q.dtype, device=q.device)
     k_eff = min(int(K), T)
     if idx_out is None:
         idx_out = torch.empty((B, S, k_eff), dtype=torch.int32, device=q.device)
     a = _forward_args(q_idx, k_idx, w, index_scale, K, q, k, v, gate, gate_mode, relu, sm_scale,
-                      attn_algo, out, scores_out, idx_out, indexer, sink_k, sink_v)
+                      attn_algo, out, scores_out, idx_out, indexer, sink_k, sink_v, attn_form,
+                      dv)
     ev_arr = None
     if events is not None:  # 4 torch.cuda.Event, recorded by the library at stage boundaries
         for e in events:

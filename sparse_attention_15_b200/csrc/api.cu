@@ -159,7 +159,7 @@ float default_scale(float sm_scale, int DQK) {
   return sm_scale > 0.f ? sm_scale : 1.0f / sqrtf((float)DQK);
 }
 
-constexpr int kNone = -1, kGather = 1, kMasked = 2;
+constexpr int kNone = -1, kGather = 1, kMasked = 2, kLatent = 3;
 
 size_t mask_bytes(int B, int S, int T) {
   return (size_t)B * S * dsa::mask_stride_words(T) * sizeof(uint32_t);
@@ -311,6 +311,49 @@ dsa_attn_algo dsa_sparse_attn_algo(dsa_dtype dtype, int B, int S, int T, int H, 
   return alg == kMasked ? DSA_ATTN_MASKED_TILE : (alg == kGather ? DSA_ATTN_GATHER : DSA_ATTN_AUTO);
 }
 
+// Latent (MQA-form) attention: bf16, DQK 576 / DV 512, 1 <= H <= 128, latent sink rows.
+static dsa_status check_latent(dsa_dtype dtype, const void* q, const void* kv,
+                               const void* sink_kv, int nsink, const void* gate,
+                               dsa_gate_mode gm, float sm_scale, int B, int S, int T, int H,
+                               int DQK, int DV, const void* out) {
+  REQUIRE(dtype == DSA_F32 || dtype == DSA_BF16, DSA_ERR_INVALID_ARG, "unknown dtype %d",
+          (int)dtype);
+  REQUIRE(q && kv && out, DSA_ERR_INVALID_ARG, "null pointer argument");
+  REQUIRE(B > 0 && S > 0 && T > 0 && H > 0 && DQK > 0 && DV > 0, DSA_ERR_INVALID_ARG,
+          "sizes must be positive");
+  REQUIRE(T >= S, DSA_ERR_INVALID_ARG, "T (%d) must be >= S (%d)", T, S);
+  REQUIRE(DV <= DQK, DSA_ERR_INVALID_ARG, "DV=%d exceeds the latent row (DQK=%d)", DV, DQK);
+  REQUIRE(gm >= DSA_GATE_OFF && gm <= DSA_GATE_SILU, DSA_ERR_INVALID_ARG,
+          "unknown gate mode %d (only sigmoid and silu exist)", (int)gm);
+  REQUIRE((gm == DSA_GATE_OFF) == (gate == nullptr), DSA_ERR_INVALID_ARG,
+          "gate pointer must be given exactly when the gate is on");
+  REQUIRE(!isnan(sm_scale) && !isinf(sm_scale), DSA_ERR_INVALID_ARG, "sm_scale not finite");
+  REQUIRE(nsink >= 0 && nsink <= 128, DSA_ERR_UNSUPPORTED, "nsink=%d must be in [0, 128]",
+          nsink);
+  REQUIRE((nsink > 0) == (sink_kv != nullptr), DSA_ERR_INVALID_ARG,
+          "sink_kv must be given exactly when nsink > 0");
+  REQUIRE(dsa::latent_attn_supported((int)dtype, H, DQK, DV), DSA_ERR_UNSUPPORTED,
+          "latent attention needs bf16, DQK == 576, DV == 512 and 1 <= H <= 128");
+  REQUIRE((long long)B * S * 128 <= 0x7fffffffLL, DSA_ERR_UNSUPPORTED, "B*S=%lld too large",
+          (long long)B * S);
+  REQUIRE(aligned16(q) && aligned16(kv) && aligned16(out) &&
+              (gate == nullptr || aligned16(gate)) && (sink_kv == nullptr || aligned16(sink_kv)),
+          DSA_ERR_UNSUPPORTED, "pointers must be 16-byte aligned");
+  return DSA_OK;
+}
+
+static dsa::LatentProblem latent_problem(const void* q, const void* kv, const int32_t* idx, int K,
+                                         const void* sink_kv, int nsink, const void* gate,
+                                         dsa_gate_mode gm, float sm_scale, int B, int S, int T,
+                                         int H, int DQK, int DV, void* out) {
+  dsa::LatentProblem p{};
+  p.dtype = (int)DSA_BF16; p.q = q; p.kv = kv; p.idx = idx; p.K = K;
+  p.sink = nsink > 0 ? sink_kv : nullptr; p.nsink = nsink > 0 ? nsink : 0;
+  p.gate = gate; p.gate_mode = (int)gm; p.sm_scale = default_scale(sm_scale, DQK);
+  p.B = B; p.S = S; p.T = T; p.H = H; p.DQK = DQK; p.DV = DV; p.q_off = T - S; p.out = out;
+  return p;
+}
+
 static dsa_status sparse_attn_impl(dsa_dtype dtype, const void* q, const void* k, const void* v,
                                    const int32_t* idx, int K, const void* sink_k,
                                    const void* sink_v, int nsink, const void* gate,
@@ -370,6 +413,31 @@ dsa_status dsa_sparse_attn_sinks(dsa_dtype dtype, const void* q, const void* k, 
   REQUIRE(nsink > 0, DSA_ERR_INVALID_ARG, "nsink must be positive (use dsa_sparse_attn)");
   return sparse_attn_impl(dtype, q, k, v, idx, K, sink_k, sink_v, nsink, gate, gate_mode,
                           sm_scale, B, S, T, H, DQK, DV, algo, out, ws, ws_bytes, stream);
+}
+
+size_t dsa_sparse_attn_latent_workspace_bytes(int B, int S, int H, int K, int nsink) {
+  if (B <= 0 || S <= 0 || H <= 0 || K <= 0 || nsink < 0) return 0;
+  return dsa::latent_attn_workspace_bytes(B, S, H, K, nsink);
+}
+
+dsa_status dsa_sparse_attn_latent(dsa_dtype dtype, const void* q, const void* kv,
+                                  const int32_t* idx, int K, const void* sink_kv, int nsink,
+                                  const void* gate, dsa_gate_mode gate_mode, float sm_scale,
+                                  int B, int S, int T, int H, int DQK, int DV, void* out,
+                                  void* ws, size_t ws_bytes, dsa_stream_t stream) {
+  dsa_status st = check_latent(dtype, q, kv, sink_kv, nsink, gate, gate_mode, sm_scale, B, S, T,
+                               H, DQK, DV, out);
+  if (st != DSA_OK) return st;
+  REQUIRE(idx != nullptr && K > 0, DSA_ERR_INVALID_ARG, "idx must be given with K > 0");
+  REQUIRE(aligned16(idx), DSA_ERR_UNSUPPORTED, "idx must be 16-byte aligned");
+  const size_t need = dsa_sparse_attn_latent_workspace_bytes(B, S, H, K, nsink);
+  REQUIRE(ws_bytes >= need && (need == 0 || ws != nullptr), DSA_ERR_INVALID_ARG,
+          "workspace too small: %zu bytes given, %zu needed", ws_bytes, need);
+  REQUIRE(ws == nullptr || aligned16(ws), DSA_ERR_UNSUPPORTED, "workspace must be 16-byte aligned");
+  const dsa::LatentProblem p = latent_problem(q, kv, idx, K, sink_kv, nsink, gate, gate_mode,
+                                              sm_scale, B, S, T, H, DQK, DV, out);
+  return cuda_status(dsa::launch_latent_attn(p, ws, ws_bytes, (cudaStream_t)stream),
+                     "dsa_sparse_attn_latent");
 }
 
 static dsa_status window_attn_impl(dsa_dtype dtype, const void* q, const void* k, const void* v,
@@ -438,8 +506,14 @@ static dsa_status check_forward(const dsa_forward_args* a) {
                                    a->B, a->S, a->T, a->HI, a->DI,
                                    a->scores_out ? (const void*)a->scores_out : (const void*)a);
   if (st != DSA_OK) return st;
-  st = check_attn_common(a->dtype, a->q, a->k, a->v, a->gate, a->gate_mode, a->sm_scale, a->B,
-                         a->S, a->T, a->H, a->H, a->DQK, a->DV, a->out);
+  REQUIRE(a->attn_form == DSA_ATTN_EXPANDED || a->attn_form == DSA_ATTN_LATENT,
+          DSA_ERR_INVALID_ARG, "unknown attention form %d", (int)a->attn_form);
+  const bool latent = a->attn_form == DSA_ATTN_LATENT;
+  st = latent ? check_latent(a->dtype, a->q, a->k, a->sink_k, a->nsink, a->gate, a->gate_mode,
+                             a->sm_scale, a->B, a->S, a->T, a->H, a->DQK, a->DV, a->out)
+              : check_attn_common(a->dtype, a->q, a->k, a->v, a->gate, a->gate_mode,
+                                  a->sm_scale, a->B, a->S, a->T, a->H, a->H, a->DQK, a->DV,
+                                  a->out);
   if (st != DSA_OK) return st;
   REQUIRE(a->K > 0, DSA_ERR_INVALID_ARG, "K must be positive");
   REQUIRE(a->attn_algo >= DSA_ATTN_AUTO && a->attn_algo <= DSA_ATTN_MASKED_TILE,
@@ -448,7 +522,7 @@ static dsa_status check_forward(const dsa_forward_args* a) {
           "idx_out must be 16-byte aligned");
   REQUIRE(a->indexer == DSA_INDEXER_PER_HEAD || a->indexer == DSA_INDEXER_COLLAPSED,
           DSA_ERR_INVALID_ARG, "unknown indexer mode %d", (int)a->indexer);
-  if ((st = check_sinks(a->sink_k, a->sink_v, a->nsink)) != DSA_OK) return st;
+  if (!latent && (st = check_sinks(a->sink_k, a->sink_v, a->nsink)) != DSA_OK) return st;
   if (a->indexer == DSA_INDEXER_COLLAPSED) return check_collapsed(a->dtype, a->relu, a->DI);
   return DSA_OK;
 }
@@ -461,13 +535,19 @@ struct FwdLayout {
 static FwdLayout forward_layout(const dsa_forward_args* a) {
   FwdLayout L{};
   L.k_eff = a->K < a->T ? a->K : a->T;
-  L.alg = choose_algo(a->attn_algo, a->dtype, a->B, a->S, a->T, a->H, a->DQK, a->DV, L.k_eff);
+  const bool latent = a->attn_form == DSA_ATTN_LATENT;
+  L.alg = latent ? kLatent
+                 : choose_algo(a->attn_algo, a->dtype, a->B, a->S, a->T, a->H, a->DQK, a->DV,
+                               L.k_eff);
   L.mask_stride = dsa::mask_stride_words(a->T);
   size_t off = 0;
   L.idx_off = off;
   if (!a->idx_out) off += align256((size_t)a->B * a->S * L.k_eff * sizeof(int32_t));
   L.attn_off = off;
-  if (L.alg == kGather)
+  if (latent)
+    off += align256(dsa::latent_attn_workspace_bytes(a->B, a->S, a->H, L.k_eff,
+                                                     a->nsink > 0 ? a->nsink : 0));
+  else if (L.alg == kGather)
     off += align256(dsa::gather_attn_workspace_bytes(a->B, a->S, a->H, a->DV, L.k_eff,
                                                      a->nsink > 0 ? a->nsink : 0));
   L.mask_off = off;
@@ -507,7 +587,7 @@ dsa_status dsa_forward(const dsa_forward_args* a, void* ws, size_t ws_bytes,
   cudaStream_t s = (cudaStream_t)stream;
   uint8_t* base = static_cast<uint8_t*>(ws);
   int32_t* idx = a->idx_out ? a->idx_out : reinterpret_cast<int32_t*>(base + L.idx_off);
-  void* attn_ws = (base && L.alg == kGather) ? base + L.attn_off : nullptr;
+  void* attn_ws = (base && (L.alg == kGather || L.alg == kLatent)) ? base + L.attn_off : nullptr;
   const bool collapsed = a->indexer == DSA_INDEXER_COLLAPSED;
   uint8_t* qc = collapsed ? base + L.qc_off : nullptr;
   const size_t attn_ws_bytes = L.mask_off - L.attn_off;
@@ -567,6 +647,14 @@ dsa_status dsa_forward(const dsa_forward_args* a, void* ws, size_t ws_bytes,
     }
     // row blocks interleave the two stages: both boundary events mark their end
     if ((st = mark(1)) != DSA_OK || (st = mark(2)) != DSA_OK) return st;
+  }
+  if (L.alg == kLatent) {
+    const dsa::LatentProblem lp =
+        latent_problem(a->q, a->k, idx, L.k_eff, a->sink_k, a->nsink, a->gate, a->gate_mode,
+                       a->sm_scale, B, S, T, a->H, a->DQK, a->DV, a->out);
+    st = cuda_status(dsa::launch_latent_attn(lp, attn_ws, attn_ws_bytes, s), "dsa_forward/attn");
+    if (st != DSA_OK) return st;
+    return mark(3);
   }
   dsa::AttnProblem p{};
   p.dtype = (int)a->dtype; p.q = a->q; p.k = a->k; p.v = a->v; p.idx = idx; p.K = L.k_eff;

@@ -424,6 +424,24 @@ cudaError_t launch_hpw(GatherArgs a, int hpw, size_t smem, unsigned grid, int ro
 
 }  // namespace
 
+cudaError_t launch_split_combine(int dtype, const float* part_o, const float* part_ml, int rows,
+                                 int nsplit, int H, int DV, const void* gate, int gate_mode,
+                                 void* out, cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  if (nsplit < 1 || nsplit > 64) return cudaErrorInvalidValue;
+  GatherArgs a{};
+  a.part_o = const_cast<float*>(part_o);
+  a.part_ml = const_cast<float*>(part_ml);
+  a.nsplit = nsplit; a.H = H; a.DV = DV;
+  a.gate = gate; a.gate_mode = gate_mode; a.out = out;
+  const unsigned grid = (unsigned)rows * (unsigned)H;
+  if (dtype == 0)
+    combine_kernel<float><<<grid, 128, 0, st>>>(a);
+  else
+    combine_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
 size_t gather_attn_workspace_bytes(int B, int S, int H, int DV, int K, int nsink) {
   const int rows = B * S;
   int ns, kps;

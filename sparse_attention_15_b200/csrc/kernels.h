@@ -87,4 +87,31 @@ bool masked_attn_supported(int dtype, int DQK, int DV);
 cudaError_t launch_masked_attn(const AttnProblem& p, const uint32_t* mask, int mask_stride,
                                cudaStream_t st);
 
+// Merge of split-key partials (unnormalised o [rows, nsplit, H, DV] float32 and (m, l)
+// [rows, nsplit, H, 2], m in log2 units) into out [rows, H, DV], gate applied.  nsplit <= 64.
+cudaError_t launch_split_combine(int dtype, const float* part_o, const float* part_ml, int rows,
+                                 int nsplit, int H, int DV, const void* gate, int gate_mode,
+                                 void* out, cudaStream_t st);
+
+// Sparse attention over a shared latent cache (MQA form): q [B,S,H,576], kv [B,T,576] (keys =
+// whole rows, values = their first 512 dims), bf16, 1 <= H <= 128.
+struct LatentProblem {
+  int dtype;
+  const void* q;
+  const void* kv;
+  const int32_t* idx;  // [B,S,K]
+  int K;
+  const void* sink;    // [nsink, 576] latent sink rows (PAS) or NULL
+  int nsink;
+  const void* gate;    // [B,S,H] or NULL
+  int gate_mode;
+  float sm_scale;
+  int B, S, T, H, DQK, DV, q_off;
+  void* out;           // [B,S,H,DV]
+};
+bool latent_attn_supported(int dtype, int H, int DQK, int DV);
+size_t latent_attn_workspace_bytes(int B, int S, int H, int K, int nsink);
+cudaError_t launch_latent_attn(const LatentProblem& p, void* ws, size_t ws_bytes,
+                               cudaStream_t st);
+
 }  // namespace dsa

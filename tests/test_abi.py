@@ -160,6 +160,31 @@ def test_sparse_attn_sinks_rejects_bad_arguments(lib):
     assert L.dsa_sparse_attn_sinks_workspace_bytes(1, 1, 4, 4, 2, 128, 128, 2, 4, 1) >= 0
 
 
+def test_sparse_attn_latent_rejects_bad_arguments(lib):
+    L = lib.lib()
+
+    def call(dtype=1, H=128, DQK=576, DV=512, nsink=0, skv=None, q=FAKE, ws_bytes=1 << 30, **kw):
+        a = dict(B=2, S=1, T=5000, K=2048)
+        a.update(kw)
+        return L.dsa_sparse_attn_latent(dtype, q, FAKE, FAKE, a["K"], skv, nsink, None, 0, 0.0,
+                                        a["B"], a["S"], a["T"], H, DQK, DV, FAKE, FAKE, ws_bytes,
+                                        None)
+    assert call(dtype=0) == 2           # float32: no latent kernel
+    assert call(dtype=7) == 1
+    assert call(DQK=192, DV=128) == 2   # only the 512 + 64 latent row
+    assert call(DV=640) == 1            # values longer than the row
+    assert call(H=129) == 2
+    assert call(H=0) == 1
+    assert call(nsink=4) == 1           # sinks without rows
+    assert call(nsink=129, skv=FAKE) == 2
+    assert call(q=FAKE_MIS) == 2
+    assert call(S=2, T=1) == 1
+    need = L.dsa_sparse_attn_latent_workspace_bytes(2, 1, 128, 2048, 0)
+    assert need > 0                     # decode-shaped: split keys need partials
+    assert call(ws_bytes=need - 1) == 1
+    assert L.dsa_sparse_attn_latent_workspace_bytes(1, 4096, 128, 2048, 0) == 0
+
+
 def test_window_attn_sinks_rejects_bad_arguments(lib):
     L = lib.lib()
 
@@ -215,6 +240,15 @@ def test_forward_workspace_and_validation(lib):
     a.indexer = 0
     assert L.dsa_forward(ctypes.byref(a), FAKE, full, None) == 2  # DI = 64
     a.index_dtype = 5
+    assert L.dsa_forward(ctypes.byref(a), FAKE, full, None) == 1
+    a.index_dtype = 0
+    # the latent attention form: k is the latent cache, v unused; its own shape rules
+    a.attn_form = 1
+    assert L.dsa_forward(ctypes.byref(a), FAKE, full, None) == 2  # DQK 128 is not 576
+    a.H, a.DQK, a.DV, a.v = 128, 576, 512, None
+    # prefill: no split partials, and no selection bitmask (4096 rows x 4096 bits)
+    assert lib.dsa_forward_workspace_bytes(a) == full - 4096 * 4096 // 8
+    a.attn_form = 3
     assert L.dsa_forward(ctypes.byref(a), FAKE, full, None) == 1
 
 
