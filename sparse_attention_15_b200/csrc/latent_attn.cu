@@ -201,18 +201,26 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
       }
       cp_async_commit();
     }
+    // lane l resolves entry l of a block (every producer warp holds the block's 32 source
+    // rows); the next block's entries are read one block ahead, so no copy waits for them
+    const int lane_p = p & 31;
+    const __nv_bfloat16* nxt = NB > 0 ? key_row(a, idx_row, b, spos, p0 + lane_p, p1) : nullptr;
     for (int j = 0; j < NB; ++j) {
       const int st = j & (kStages - 1);
-      if (j >= kStages && !mbar_wait(&empty[st], ((j / kStages) - 1) & 1)) { ok = false; break; }
+      const unsigned long long cur = reinterpret_cast<unsigned long long>(nxt);
+      if (j + 1 < NB) nxt = key_row(a, idx_row, b, spos, p0 + (j + 1) * kNK + lane_p, p1);
+      // warp-uniform wait: the whole warp takes part in the shuffles below
+      if (j >= kStages && !warp_wait(&empty[st], ((j / kStages) - 1) & 1)) { ok = false; break; }
       uint8_t* stage = ring + st * kStageBytes;
       // 32 rows x 72 chunks of 16 bytes, 18 per thread; consecutive threads read one row
-#pragma unroll 6
+#pragma unroll
       for (int i = 0; i < kNK * (kDQK / 8) / kProdThreads; ++i) {
         const int e = p + kProdThreads * i;
         const int key = e / (kDQK / 8);
         const int k = e - key * (kDQK / 8);
         const int x = k >> 3, cc = k & 7;
-        const __nv_bfloat16* row = key_row(a, idx_row, b, spos, p0 + j * kNK + key, p1);
+        const __nv_bfloat16* row =
+            reinterpret_cast<const __nv_bfloat16*>(__shfl_sync(0xffffffffu, cur, key));
         cp_async16(stage + x * kKSlice + key * 128 + ((cc ^ (key & 7)) << 4),
                    row ? row + x * 64 + cc * 8 : a.kv, row ? 16u : 0u);
       }
@@ -288,16 +296,27 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
     bool ok = true;
     // Q dims 0..319 of head h -> TMEM columns kColQ.. (bf16 pairs; zeros for h >= H)
     {
+      // two batches of loads (slices 0..2, then 3..4), each all in flight before its stores
       const uint4* src = reinterpret_cast<const uint4*>(a.q + ((size_t)r * a.H + h) * kDQK);
-#pragma unroll 1
-      for (int x = 0; x < kQT; ++x) {
-        uint32_t v[32];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 u = head_ok ? __ldg(src + x * 8 + c) : make_uint4(0u, 0u, 0u, 0u);
-          v[4 * c] = u.x; v[4 * c + 1] = u.y; v[4 * c + 2] = u.z; v[4 * c + 3] = u.w;
+      for (int x0 = 0; x0 < kQT; x0 += 3) {
+        constexpr int kBatch = 3;
+        uint4 u[kBatch * 8];
+#pragma unroll
+        for (int c = 0; c < kBatch * 8; ++c)
+          u[c] = (head_ok && x0 * 8 + c < kQT * 8) ? __ldg(src + x0 * 8 + c)
+                                                   : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int x = 0; x < kBatch; ++x) {
+          if (x0 + x >= kQT) break;
+          uint32_t v[32];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            v[4 * c] = u[x * 8 + c].x; v[4 * c + 1] = u[x * 8 + c].y;
+            v[4 * c + 2] = u[x * 8 + c].z; v[4 * c + 3] = u[x * 8 + c].w;
+          }
+          tmem_st32(t_lane + kColQ + (x0 + x) * 32, v);
         }
-        tmem_st32(t_lane + kColQ + x * 32, v);
       }
       tmem_wait_st();
       tc_fence_before();
