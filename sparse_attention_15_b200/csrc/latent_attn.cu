@@ -202,38 +202,53 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
       cp_async_commit();
     }
     // lane l resolves entry l of a block (every producer warp holds the block's 32 source
-    // rows); the next block's entries are read one block ahead, so no copy waits for them
+    // rows); the next block's entries are read one block ahead, so no copy waits for them.
+    // Producer warp w copies keys 8w..8w+7; lane l copies chunks l, l+32, l+64 (< 72) of
+    // each row: chunk c is slice c/8, 16-byte column c%8 (swizzled by the row's index mod 8).
     const int lane_p = p & 31;
+    const int wp = p >> 5;
     const __nv_bfloat16* nxt = NB > 0 ? key_row(a, idx_row, b, spos, p0 + lane_p, p1) : nullptr;
+    uint32_t dst_off[3], src_off[3], cc_of[3];
+#pragma unroll
+    for (int m = 0; m < 3; ++m) {
+      const int c = lane_p + 32 * m;
+      cc_of[m] = c & 7;
+      dst_off[m] = (c >> 3) * kKSlice;
+      src_off[m] = (c >> 3) * 64 + (c & 7) * 8;
+    }
     for (int j = 0; j < NB; ++j) {
       const int st = j & (kStages - 1);
       const unsigned long long cur = reinterpret_cast<unsigned long long>(nxt);
       if (j + 1 < NB) nxt = key_row(a, idx_row, b, spos, p0 + (j + 1) * kNK + lane_p, p1);
       // warp-uniform wait: the whole warp takes part in the shuffles below
       if (j >= kStages && !warp_wait(&empty[st], ((j / kStages) - 1) & 1)) { ok = false; break; }
-      uint8_t* stage = ring + st * kStageBytes;
-      // 32 rows x 72 chunks of 16 bytes, 18 per thread; consecutive threads read one row
+      uint8_t* stage = ring + st * kStageBytes + wp * 8 * 128;
 #pragma unroll
-      for (int i = 0; i < kNK * (kDQK / 8) / kProdThreads; ++i) {
-        const int e = p + kProdThreads * i;
-        const int key = e / (kDQK / 8);
-        const int k = e - key * (kDQK / 8);
-        const int x = k >> 3, cc = k & 7;
+      for (int i = 0; i < 8; ++i) {
         const __nv_bfloat16* row =
-            reinterpret_cast<const __nv_bfloat16*>(__shfl_sync(0xffffffffu, cur, key));
-        cp_async16(stage + x * kKSlice + key * 128 + ((cc ^ (key & 7)) << 4),
-                   row ? row + x * 64 + cc * 8 : a.kv, row ? 16u : 0u);
+            reinterpret_cast<const __nv_bfloat16*>(__shfl_sync(0xffffffffu, cur, wp * 8 + i));
+        // key 8w+i: its row's 128-byte lines sit at (8w+i)*128 in each slice, swizzle i
+#pragma unroll
+        for (int m = 0; m < 3; ++m) {
+          if (m == 2 && lane_p >= kDQK / 8 - 64) break;
+          cp_async16(stage + dst_off[m] + i * 128 + ((cc_of[m] ^ i) << 4),
+                     row ? row + src_off[m] : a.kv, row ? 16u : 0u);
+        }
       }
       cp_async_commit();
-      // the group before this one (block j-1, or Q) has landed: publish it to the MMA
-      cp_async_wait<1>();
-      fence_proxy_async_smem();
-      mbar_arrive(j == 0 ? q_full : &full[(j - 1) & (kStages - 1)]);
+      // copy groups: Q, then one per block.  Three stay in flight; the oldest beyond them
+      // (Q after block 1 is issued, block j-2 after block j) has landed: publish it
+      if (j >= 1) {
+        cp_async_wait<2>();
+        fence_proxy_async_smem();
+        mbar_arrive(j == 1 ? q_full : &full[(j - 2) & (kStages - 1)]);
+      }
     }
     cp_async_wait<0>();
-    if (ok) {
+    if (ok) {  // publish what is left: Q (one block or none), the last two blocks
       fence_proxy_async_smem();
-      mbar_arrive(NB == 0 ? q_full : &full[(NB - 1) & (kStages - 1)]);
+      if (NB <= 1) mbar_arrive(q_full);
+      for (int jj = NB >= 2 ? NB - 2 : 0; jj < NB; ++jj) mbar_arrive(&full[jj & (kStages - 1)]);
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------------ MMA issuer
@@ -243,23 +258,27 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
       const uint32_t qs_base = smem_u32(Qs);
       bool ok = mbar_wait(q_full, 0) && mbar_wait(q_tm, 0);
       // S_j = Q C_j^T into S[j % 3]; the buffer last held P_{j-3}, consumed by PV_{j-3}
+      // descriptors: a base per operand plus constant offsets in the 16-byte address field
+      // (shared addresses stay below 256 KB, so the field never carries)
+      const uint64_t qdesc0 = sw128_kmajor_desc(qs_base);
+      const uint64_t kdesc0 = sw128_kmajor_desc(smem_u32(ring));
       auto issue_qk = [&](int j) -> bool {
         const int st = j & (kStages - 1), sb = j % kSB;
         if (!mbar_wait(&full[st], (j / kStages) & 1)) return false;
         if (j >= kSB && !mbar_wait(&pv_done[sb], ((j / kSB) - 1) & 1)) return false;
         tc_fence_after();
-        const uint32_t kb = smem_u32(ring + st * kStageBytes);
+        const uint64_t kd = kdesc0 + (uint64_t)(st * (kStageBytes >> 4));
         const uint32_t d = tmem + kColS + sb * kNK;
 #pragma unroll
         for (int x = 0; x < kSlices; ++x)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t bdesc = sw128_kmajor_desc(kb + x * kKSlice + kk * 32);
+            const uint64_t bdesc = kd + (uint64_t)((x * kKSlice + kk * 32) >> 4);
             const uint32_t acc = (x | kk) ? 1u : 0u;
             if (x < kQT)
               umma_f16_ts(d, tmem + kColQ + x * 32 + kk * 8, bdesc, idesc_qk, acc);
             else
-              umma_f16_ss(d, sw128_kmajor_desc(qs_base + (x - kQT) * kQSlice + kk * 32), bdesc,
+              umma_f16_ss(d, qdesc0 + (uint64_t)(((x - kQT) * kQSlice + kk * 32) >> 4), bdesc,
                           idesc_qk, acc);
           }
         umma_commit(&s_full[sb]);
@@ -272,12 +291,13 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
         if (!mbar_wait(&p_full[sb], (j / kSB) & 1)) { ok = false; break; }
         tc_fence_after();
         // V = the first DV columns of the key rows; this CTA's half starts at slice 4*hv
-        const uint32_t vb = smem_u32(ring + st * kStageBytes) + (uint32_t)(4 * hv * kKSlice);
+        const uint64_t vd = sw128_mn_desc(smem_u32(ring + st * kStageBytes) +
+                                              (uint32_t)(4 * hv * kKSlice), kKSlice, 1024);
         const uint32_t pt = tmem + kColS + sb * kNK;
 #pragma unroll
         for (int c = 0; c < kNK / 16; ++c) {
           // keys 16c..16c+15: P_hi in 8 columns at 16c, P_lo 8 further; 2 atoms of V rows
-          const uint64_t vdesc = sw128_mn_desc(vb + c * 2048, kKSlice, 1024);
+          const uint64_t vdesc = vd + (uint64_t)((c * 2048) >> 4);
           umma_f16_ts(tmem + kColO, pt + 16 * c, vdesc, idesc_pv, (j > 0 || c > 0) ? 1u : 0u);
           umma_f16_ts(tmem + kColO, pt + 16 * c + 8, vdesc, idesc_pv, 1u);
         }
