@@ -28,8 +28,8 @@
 //
 // Roles: warps 0..3 softmax and epilogue (thread = head = TMEM lane; they also write Q's
 // tensor-memory part), warp 4 MMA issuer and TMEM owner, warps 5..8 gather the selected rows
-// with 16-byte cp.async into the swizzled ring (zero fill for skipped entries).  Every wait
-// is bounded.
+// with 16-byte cp.async into the swizzled ring (zero fill for skipped entries), each warp
+// owning one ring stage.  Every wait is bounded.
 #include <climits>
 
 #include "common.cuh"
@@ -135,7 +135,7 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
   uint8_t* Qs = smem;                 // [kQS] slices of [128 rows x 64]
   uint8_t* ring = smem + kQBytes;     // [kStages] key blocks
   uint64_t* bars = reinterpret_cast<uint64_t*>(ring + kStages * kStageBytes);
-  uint64_t* full = bars;              // [4] key block landed (producer threads)
+  uint64_t* full = bars;              // [4] key block landed (its producer warp)
   uint64_t* empty = bars + 4;         // [4] key block consumed by its P V
   uint64_t* s_full = bars + 8;        // [3] S = Q C^T done
   uint64_t* p_full = bars + 11;       // [3] P written (softmax warps)
@@ -161,7 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&full[i], kProdThreads);
+      mbar_init(&full[i], 32);  // the producer warp that owns the stage
       mbar_init(&empty[i], 1);
     }
     for (int i = 0; i < kSB; ++i) {
@@ -201,13 +201,15 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
       }
       cp_async_commit();
     }
-    // lane l resolves entry l of a block (every producer warp holds the block's 32 source
-    // rows); the next block's entries are read one block ahead, so no copy waits for them.
-    // Producer warp w copies keys 8w..8w+7; lane l copies chunks l, l+32, l+64 (< 72) of
-    // each row: chunk c is slice c/8, 16-byte column c%8 (swizzled by the row's index mod 8).
+    // Producer warp w owns ring stage w and copies blocks w, w+4, w+8, ...: it issues a
+    // block's 32 rows, waits for its own copies, fences and publishes the stage at once, so
+    // a landed block is never held back by another stage.  Lane l resolves entry l of the
+    // block (read one round ahead) and copies chunks l, l+32, l+64 (< 72) of every row:
+    // chunk c is slice c/8, 16-byte column c%8, swizzled by the row's index mod 8.
     const int lane_p = p & 31;
     const int wp = p >> 5;
-    const __nv_bfloat16* nxt = NB > 0 ? key_row(a, idx_row, b, spos, p0 + lane_p, p1) : nullptr;
+    const __nv_bfloat16* nxt =
+        wp < NB ? key_row(a, idx_row, b, spos, p0 + wp * kNK + lane_p, p1) : nullptr;
     uint32_t dst_off[3], src_off[3], cc_of[3];
 #pragma unroll
     for (int m = 0; m < 3; ++m) {
@@ -216,39 +218,40 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
       dst_off[m] = (c >> 3) * kKSlice;
       src_off[m] = (c >> 3) * 64 + (c & 7) * 8;
     }
-    for (int j = 0; j < NB; ++j) {
-      const int st = j & (kStages - 1);
+    bool q_pending = true;  // this thread's Q copies not yet published
+    uint8_t* stage = ring + wp * kStageBytes;
+    for (int j = wp; j < NB; j += kStages) {
       const unsigned long long cur = reinterpret_cast<unsigned long long>(nxt);
-      if (j + 1 < NB) nxt = key_row(a, idx_row, b, spos, p0 + (j + 1) * kNK + lane_p, p1);
+      if (j + kStages < NB)
+        nxt = key_row(a, idx_row, b, spos, p0 + (j + kStages) * kNK + lane_p, p1);
       // warp-uniform wait: the whole warp takes part in the shuffles below
-      if (j >= kStages && !warp_wait(&empty[st], ((j / kStages) - 1) & 1)) { ok = false; break; }
-      uint8_t* stage = ring + st * kStageBytes + wp * 8 * 128;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
+      if (j >= kStages && !warp_wait(&empty[wp], ((j / kStages) - 1) & 1)) { ok = false; break; }
+#pragma unroll 4
+      for (int i = 0; i < kNK; ++i) {
         const __nv_bfloat16* row =
-            reinterpret_cast<const __nv_bfloat16*>(__shfl_sync(0xffffffffu, cur, wp * 8 + i));
-        // key 8w+i: its row's 128-byte lines sit at (8w+i)*128 in each slice, swizzle i
+            reinterpret_cast<const __nv_bfloat16*>(__shfl_sync(0xffffffffu, cur, i));
 #pragma unroll
         for (int m = 0; m < 3; ++m) {
           if (m == 2 && lane_p >= kDQK / 8 - 64) break;
-          cp_async16(stage + dst_off[m] + i * 128 + ((cc_of[m] ^ i) << 4),
+          cp_async16(stage + dst_off[m] + i * 128 + ((cc_of[m] ^ (i & 7)) << 4),
                      row ? row + src_off[m] : a.kv, row ? 16u : 0u);
         }
       }
       cp_async_commit();
-      // copy groups: Q, then one per block.  Three stay in flight; the oldest beyond them
-      // (Q after block 1 is issued, block j-2 after block j) has landed: publish it
-      if (j >= 1) {
-        cp_async_wait<2>();
+      if (q_pending) {  // the Q group (committed first) has landed
+        cp_async_wait<1>();
         fence_proxy_async_smem();
-        mbar_arrive(j == 1 ? q_full : &full[(j - 2) & (kStages - 1)]);
+        mbar_arrive(q_full);
+        q_pending = false;
       }
+      cp_async_wait<0>();
+      fence_proxy_async_smem();
+      mbar_arrive(&full[wp]);
     }
     cp_async_wait<0>();
-    if (ok) {  // publish what is left: Q (one block or none), the last two blocks
+    if (ok && q_pending) {  // a warp without blocks still publishes its Q copies
       fence_proxy_async_smem();
-      if (NB <= 1) mbar_arrive(q_full);
-      for (int jj = NB >= 2 ? NB - 2 : 0; jj < NB; ++jj) mbar_arrive(&full[jj & (kStages - 1)]);
+      mbar_arrive(q_full);
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------------ MMA issuer
