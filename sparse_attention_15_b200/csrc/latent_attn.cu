@@ -12,24 +12,25 @@
 //
 // Because the key row is shared by all heads, a block of selected keys is a real
 // [H x DQK] . [DQK x keys] tensor-core product: S = Q C^T with M = 128 heads (rows past H
-// are zero), N = 32 keys, K = 576; then O += P V with M = 128 heads, N = 256, K = 32 keys.
+// are zero), N = 64 keys, K = 576; then O += P V with M = 128 heads, N = 256, K = 64 keys.
 // O for all 512 latent columns would fill the whole tensor memory, so every (query row, key
 // split) is computed by two CTAs, one per half of DV; each computes the full S (the QK
 // product is repeated, nothing is exchanged between CTAs) and the two run side by side, so
-// the second reads the gathered rows from L2.
+// the second reads the gathered rows from L2.  64 keys per MMA keep the instruction count
+// per key low: a block is 36 QK and 8 PV instructions.
 //
-// Tensor memory (512 columns): Q dims 0..319 as the tensor-memory A operand of QK (5 x 32
-// columns of bf16 pairs, so those MMAs read only the key tile from shared memory), S0..S2
-// (32 columns each; P_hi / P_lo are written over them), O (256 columns).  Shared memory:
-// Q dims 320..575 (4 K-major slices with the 128-byte swizzle) and a ring of 4 key blocks
-// (32 rows x 576 dims, 9 slices).  The same bytes of a key block are the K-major B operand
+// Tensor memory (512 columns): Q dims 0..255 as the tensor-memory A operand of QK (4 x 32
+// columns of bf16 pairs, so those MMAs read only the key tile from shared memory), S0, S1
+// (64 columns each; P_hi / P_lo are written over them), O (256 columns).  Shared memory:
+// Q dims 256..575 (5 K-major slices with the 128-byte swizzle) and a ring of 2 key blocks
+// (64 rows x 576 dims, 9 slices).  The same bytes of a key block are the K-major B operand
 // of QK and, for the DV/2 columns of this CTA, the MN-major B operand of PV.  P is split into
 // bf16 P_hi + P_lo (as in the masked-tile kernel) to keep float32 probability precision.
 //
 // Roles: warps 0..3 softmax and epilogue (thread = head = TMEM lane; they also write Q's
 // tensor-memory part), warp 4 MMA issuer and TMEM owner, warps 5..8 gather the selected rows
-// with 16-byte cp.async into the swizzled ring (zero fill for skipped entries), each warp
-// owning one ring stage.  Every wait is bounded.
+// with 16-byte cp.async into the swizzled ring (zero fill for skipped entries), two warps
+// per ring stage.  Every wait is bounded.
 #include <climits>
 
 #include "common.cuh"
@@ -40,12 +41,12 @@ namespace dsa {
 namespace {
 
 constexpr int kDQK = 576, kDV = 512, kNV = kDV / 2;  // N of PV per CTA
-constexpr int kNK = 32;                              // keys per block
+constexpr int kNK = 64;                              // keys per block (N of QK)
 constexpr int kSlices = kDQK / 64;                   // 64-dim slices of a row
-constexpr int kQT = 5;                               // Q slices in tensor memory
+constexpr int kQT = 4;                               // Q slices in tensor memory
 constexpr int kQS = kSlices - kQT;                   // Q slices in shared memory
-constexpr int kStages = 4;                           // key blocks in the ring
-constexpr int kSB = 3;                               // S buffers
+constexpr int kStages = 2;                           // key blocks in the ring
+constexpr int kSB = 2;                               // S buffers
 constexpr int kKSlice = kNK * 128;                   // one slice of a key block (bytes)
 constexpr int kStageBytes = kSlices * kKSlice;
 constexpr int kQSlice = 128 * 128;                   // one slice of Q (128 rows)
@@ -54,12 +55,13 @@ constexpr int kBarBytes = 256;
 constexpr int kSmem = 1024 + kQBytes + kStages * kStageBytes + kBarBytes;
 constexpr uint32_t kColQ = 0, kColS = kQT * 32, kColO = kColS + kSB * kNK;
 constexpr int kWarpMma = 4, kWarpProd0 = 5, kProdThreads = 128;
+constexpr int kProdWarpsPerStage = 4 / kStages;      // each copies kNK / 2 keys of a block
 constexpr int kThreads = 32 * 9;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;
 static_assert(kColO + kNV == 512, "TMEM budget");
 static_assert(kSmem <= 227 * 1024, "shared memory budget");
-static_assert((kNK * (kDQK / 8)) % kProdThreads == 0, "gather split");
+static_assert(kNK == 32 * kProdWarpsPerStage, "one key per lane of each producer warp");
 
 struct LatentArgs {
   const __nv_bfloat16* q;     // [rows, H, 576]
@@ -135,15 +137,15 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
   uint8_t* Qs = smem;                 // [kQS] slices of [128 rows x 64]
   uint8_t* ring = smem + kQBytes;     // [kStages] key blocks
   uint64_t* bars = reinterpret_cast<uint64_t*>(ring + kStages * kStageBytes);
-  uint64_t* full = bars;              // [4] key block landed (its producer warp)
-  uint64_t* empty = bars + 4;         // [4] key block consumed by its P V
-  uint64_t* s_full = bars + 8;        // [3] S = Q C^T done
-  uint64_t* p_full = bars + 11;       // [3] P written (softmax warps)
-  uint64_t* pv_done = bars + 14;      // [3] O += P V of that block done
-  uint64_t* q_full = bars + 17;       // Q shared-memory part landed (producer threads)
-  uint64_t* q_tm = bars + 18;         // Q tensor-memory part written (softmax warps)
-  uint64_t* mma_done = bars + 19;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
+  uint64_t* full = bars;              // [2] key block landed (its producer warps)
+  uint64_t* empty = bars + 2;         // [2] key block consumed by its P V
+  uint64_t* s_full = bars + 4;        // [2] S = Q C^T done
+  uint64_t* p_full = bars + 6;        // [2] P written (softmax warps)
+  uint64_t* pv_done = bars + 8;       // [2] O += P V of that block done
+  uint64_t* q_full = bars + 10;       // Q shared-memory part landed (producer threads)
+  uint64_t* q_tm = bars + 11;         // Q tensor-memory part written (softmax warps)
+  uint64_t* mma_done = bars + 12;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // item = (query row, key split, DV half); the two halves of a split are neighbours
@@ -161,7 +163,7 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&full[i], 32);  // the producer warp that owns the stage
+      mbar_init(&full[i], 32 * kProdWarpsPerStage);  // the producer warps of the stage
       mbar_init(&empty[i], 1);
     }
     for (int i = 0; i < kSB; ++i) {
@@ -187,13 +189,13 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
     // ------------------------------------------------------------------ gather producers
     const int p = threadIdx.x - kWarpProd0 * 32;
     bool ok = true;
-    // Q dims 320..575 of every head: 128 rows x 32 chunks of 16 bytes
+    // Q dims 256..575 of every head: 128 rows x 40 chunks of 16 bytes
     {
       const __nv_bfloat16* q0 = a.q + (size_t)r * a.H * kDQK;
 #pragma unroll 4
-      for (int i = 0; i < 32; ++i) {
+      for (int i = 0; i < kQS * 8; ++i) {
         const int e = p + kProdThreads * i;
-        const int row = e >> 5, k = e & 31;
+        const int row = e / (kQS * 8), k = e - row * (kQS * 8);
         const int x = k >> 3, cc = k & 7;
         const bool in = row < a.H;
         const __nv_bfloat16* src = in ? q0 + (size_t)row * kDQK + (kQT + x) * 64 + cc * 8 : a.q;
@@ -201,15 +203,17 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
       }
       cp_async_commit();
     }
-    // Producer warp w owns ring stage w and copies blocks w, w+4, w+8, ...: it issues a
-    // block's 32 rows, waits for its own copies, fences and publishes the stage at once, so
-    // a landed block is never held back by another stage.  Lane l resolves entry l of the
-    // block (read one round ahead) and copies chunks l, l+32, l+64 (< 72) of every row:
-    // chunk c is slice c/8, 16-byte column c%8, swizzled by the row's index mod 8.
+    // Producer warps 2s and 2s+1 own ring stage s and copy blocks s, s+2, ...: warp h of the
+    // pair copies keys 32h..32h+31 of the block, waits for its own copies, fences and
+    // publishes at once.  Lane l resolves entry l of its 32 keys (read one round ahead) and
+    // copies chunks l, l+32, l+64 (< 72) of every row: chunk c is slice c/8, 16-byte column
+    // c%8, swizzled by the row's index mod 8.
     const int lane_p = p & 31;
     const int wp = p >> 5;
+    const int st = wp / kProdWarpsPerStage;
+    const int kh = (wp % kProdWarpsPerStage) * 32;  // first key of this warp in a block
     const __nv_bfloat16* nxt =
-        wp < NB ? key_row(a, idx_row, b, spos, p0 + wp * kNK + lane_p, p1) : nullptr;
+        st < NB ? key_row(a, idx_row, b, spos, p0 + st * kNK + kh + lane_p, p1) : nullptr;
     uint32_t dst_off[3], src_off[3], cc_of[3];
 #pragma unroll
     for (int m = 0; m < 3; ++m) {
@@ -219,15 +223,15 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
       src_off[m] = (c >> 3) * 64 + (c & 7) * 8;
     }
     bool q_pending = true;  // this thread's Q copies not yet published
-    uint8_t* stage = ring + wp * kStageBytes;
-    for (int j = wp; j < NB; j += kStages) {
+    uint8_t* stage = ring + st * kStageBytes + kh * 128;
+    for (int j = st; j < NB; j += kStages) {
       const unsigned long long cur = reinterpret_cast<unsigned long long>(nxt);
       if (j + kStages < NB)
-        nxt = key_row(a, idx_row, b, spos, p0 + (j + kStages) * kNK + lane_p, p1);
+        nxt = key_row(a, idx_row, b, spos, p0 + (j + kStages) * kNK + kh + lane_p, p1);
       // warp-uniform wait: the whole warp takes part in the shuffles below
-      if (j >= kStages && !warp_wait(&empty[wp], ((j / kStages) - 1) & 1)) { ok = false; break; }
+      if (j >= kStages && !warp_wait(&empty[st], ((j / kStages) - 1) & 1)) { ok = false; break; }
 #pragma unroll 4
-      for (int i = 0; i < kNK; ++i) {
+      for (int i = 0; i < 32; ++i) {
         const __nv_bfloat16* row =
             reinterpret_cast<const __nv_bfloat16*>(__shfl_sync(0xffffffffu, cur, i));
 #pragma unroll
@@ -246,7 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
       }
       cp_async_wait<0>();
       fence_proxy_async_smem();
-      mbar_arrive(&full[wp]);
+      mbar_arrive(&full[st]);
     }
     cp_async_wait<0>();
     if (ok && q_pending) {  // a warp without blocks still publishes its Q copies
@@ -258,15 +262,14 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kNK);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, kNV) | (1u << 16);  // B MN-major
-      const uint32_t qs_base = smem_u32(Qs);
       bool ok = mbar_wait(q_full, 0) && mbar_wait(q_tm, 0);
-      // S_j = Q C_j^T into S[j % 3]; the buffer last held P_{j-3}, consumed by PV_{j-3}
       // descriptors: a base per operand plus constant offsets in the 16-byte address field
       // (shared addresses stay below 256 KB, so the field never carries)
-      const uint64_t qdesc0 = sw128_kmajor_desc(qs_base);
+      const uint64_t qdesc0 = sw128_kmajor_desc(smem_u32(Qs));
       const uint64_t kdesc0 = sw128_kmajor_desc(smem_u32(ring));
+      // S_j = Q C_j^T into S[j % 2]; the buffer last held P_{j-2}, consumed by PV_{j-2}
       auto issue_qk = [&](int j) -> bool {
-        const int st = j & (kStages - 1), sb = j % kSB;
+        const int st = j % kStages, sb = j % kSB;
         if (!mbar_wait(&full[st], (j / kStages) & 1)) return false;
         if (j >= kSB && !mbar_wait(&pv_done[sb], ((j / kSB) - 1) & 1)) return false;
         tc_fence_after();
@@ -290,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
       if (ok && NB > 0) ok = issue_qk(0);
       for (int j = 0; ok && j < NB; ++j) {
         if (j + 1 < NB && !issue_qk(j + 1)) { ok = false; break; }
-        const int sb = j % kSB, st = j & (kStages - 1);
+        const int sb = j % kSB, st = j % kStages;
         if (!mbar_wait(&p_full[sb], (j / kSB) & 1)) { ok = false; break; }
         tc_fence_after();
         // V = the first DV columns of the key rows; this CTA's half starts at slice 4*hv
@@ -317,21 +320,18 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
     const uint32_t t_lane = tmem + ((uint32_t)(warp * 32) << 16);
     const float ninf = __int_as_float(0xff800000);
     bool ok = true;
-    // Q dims 0..319 of head h -> TMEM columns kColQ.. (bf16 pairs; zeros for h >= H)
+    // Q dims 0..255 of head h -> TMEM columns kColQ.. (bf16 pairs; zeros for h >= H), two
+    // batches of loads, each all in flight before its stores
     {
-      // two batches of loads (slices 0..2, then 3..4), each all in flight before its stores
       const uint4* src = reinterpret_cast<const uint4*>(a.q + ((size_t)r * a.H + h) * kDQK);
 #pragma unroll
-      for (int x0 = 0; x0 < kQT; x0 += 3) {
-        constexpr int kBatch = 3;
-        uint4 u[kBatch * 8];
+      for (int x0 = 0; x0 < kQT; x0 += 2) {
+        uint4 u[16];
 #pragma unroll
-        for (int c = 0; c < kBatch * 8; ++c)
-          u[c] = (head_ok && x0 * 8 + c < kQT * 8) ? __ldg(src + x0 * 8 + c)
-                                                   : make_uint4(0u, 0u, 0u, 0u);
+        for (int c = 0; c < 16; ++c)
+          u[c] = head_ok ? __ldg(src + x0 * 8 + c) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-        for (int x = 0; x < kBatch; ++x) {
-          if (x0 + x >= kQT) break;
+        for (int x = 0; x < 2; ++x) {
           uint32_t v[32];
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
@@ -349,20 +349,25 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
     float m_used = ninf, l = 0.f;
     for (int j = 0; j < NB; ++j) {
       const int sb = j % kSB;
-      // which of the block's 32 entries are attended (the same for every head)
-      const bool vk = key_row(a, idx_row, b, spos, p0 + j * kNK + lane, p1) != nullptr;
-      const uint32_t bits = __ballot_sync(0xffffffffu, vk);
+      // which of the block's 64 entries are attended (the same for every head)
+      const int e0 = p0 + j * kNK + lane;
+      const uint32_t bits0 = __ballot_sync(0xffffffffu, key_row(a, idx_row, b, spos, e0, p1) != nullptr);
+      const uint32_t bits1 =
+          __ballot_sync(0xffffffffu, key_row(a, idx_row, b, spos, e0 + 32, p1) != nullptr);
       if (!warp_wait(&s_full[sb], (j / kSB) & 1)) { ok = false; break; }
       tc_fence_after();
       const uint32_t s_col = t_lane + kColS + sb * kNK;
-      uint32_t rr[32];
-      tmem_ld32(s_col, rr);
+      uint32_t rr[64];
+      tmem_ld32(s_col, *reinterpret_cast<uint32_t(*)[32]>(rr));
+      tmem_ld32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(rr + 32));
       tmem_wait_ld();
       float mx0 = ninf, mx1 = ninf;
 #pragma unroll
       for (int e = 0; e < 32; e += 2) {
-        mx0 = fmaxf(mx0, (bits >> e) & 1u ? __uint_as_float(rr[e]) : ninf);
-        mx1 = fmaxf(mx1, (bits >> (e + 1)) & 1u ? __uint_as_float(rr[e + 1]) : ninf);
+        mx0 = fmaxf(mx0, (bits0 >> e) & 1u ? __uint_as_float(rr[e]) : ninf);
+        mx1 = fmaxf(mx1, (bits0 >> (e + 1)) & 1u ? __uint_as_float(rr[e + 1]) : ninf);
+        mx0 = fmaxf(mx0, (bits1 >> e) & 1u ? __uint_as_float(rr[32 + e]) : ninf);
+        mx1 = fmaxf(mx1, (bits1 >> (e + 1)) & 1u ? __uint_as_float(rr[33 + e]) : ninf);
       }
       const float mb = fmaxf(mx0, mx1) * a.qk_scale;
       // the running max is raised (and O, l rescaled) only when a block max exceeds it by
@@ -399,13 +404,14 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
       const float msub = m_used == ninf ? 0.f : m_used;
       float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < kNK / 16; ++c) {
+        const uint32_t bw = (c < 2 ? bits0 : bits1) >> (16 * (c & 1));
         uint32_t ph[8], pl[8];
 #pragma unroll
         for (int e2 = 0; e2 < 8; ++e2) {
-          const int e = 16 * c + 2 * e2;
-          const float x0 = (bits >> e) & 1u ? __uint_as_float(rr[e]) : ninf;
-          const float x1 = (bits >> (e + 1)) & 1u ? __uint_as_float(rr[e + 1]) : ninf;
+          const int e = 2 * e2;
+          const float x0 = (bw >> e) & 1u ? __uint_as_float(rr[16 * c + e]) : ninf;
+          const float x1 = (bw >> (e + 1)) & 1u ? __uint_as_float(rr[16 * c + e + 1]) : ninf;
           const float y0 = ex2_approx(fmaf(x0, a.qk_scale, -msub));
           const float y1 = ex2_approx(fmaf(x1, a.qk_scale, -msub));
           rs0 += y0;
@@ -491,7 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
 }
 
 // Key splits per query row: the count whose waves of CTA pairs (one CTA per SM, 148 SMs)
-// finish first, counting each item's set-up (the Q load) as about four key blocks.  A fixed
+// finish first, counting each item's set-up (the Q load) as about two key blocks.  A fixed
 // SM count keeps the workspace size a function of the shape alone.
 void latent_split(int rows, int nkeys, int* nsplit, int* kps) {
   const int blocks = (nkeys + kNK - 1) / kNK;
@@ -502,7 +508,7 @@ void latent_split(int rows, int nkeys, int* nsplit, int* kps) {
     const int n = (blocks + bps - 1) / bps;
     const long long items = 2LL * rows * n;
     const long long waves = (items + 147) / 148;
-    const long long cost = waves * (bps + 4);
+    const long long cost = waves * (bps + 2);
     if (cost < best_cost) {
       best_cost = cost;
       best_n = n;
