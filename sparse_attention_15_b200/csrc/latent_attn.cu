@@ -267,12 +267,10 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
       // (shared addresses stay below 256 KB, so the field never carries)
       const uint64_t qdesc0 = sw128_kmajor_desc(smem_u32(Qs));
       const uint64_t kdesc0 = sw128_kmajor_desc(smem_u32(ring));
-      // S_j = Q C_j^T into S[j % 2]; the buffer last held P_{j-2}, consumed by PV_{j-2}
-      auto issue_qk = [&](int j) -> bool {
+      // S_j = Q C_j^T into S[j % 2] (the buffer last held P_{j-2}); O += P_j V_j.  Issued in
+      // whatever order their inputs arrive: a P V never waits behind the next block's load.
+      auto issue_qk = [&](int j) {
         const int st = j % kStages, sb = j % kSB;
-        if (!mbar_wait(&full[st], (j / kStages) & 1)) return false;
-        if (j >= kSB && !mbar_wait(&pv_done[sb], ((j / kSB) - 1) & 1)) return false;
-        tc_fence_after();
         const uint64_t kd = kdesc0 + (uint64_t)(st * (kStageBytes >> 4));
         const uint32_t d = tmem + kColS + sb * kNK;
 #pragma unroll
@@ -288,14 +286,9 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
                           idesc_qk, acc);
           }
         umma_commit(&s_full[sb]);
-        return true;
       };
-      if (ok && NB > 0) ok = issue_qk(0);
-      for (int j = 0; ok && j < NB; ++j) {
-        if (j + 1 < NB && !issue_qk(j + 1)) { ok = false; break; }
+      auto issue_pv = [&](int j) {
         const int sb = j % kSB, st = j % kStages;
-        if (!mbar_wait(&p_full[sb], (j / kSB) & 1)) { ok = false; break; }
-        tc_fence_after();
         // V = the first DV columns of the key rows; this CTA's half starts at slice 4*hv
         const uint64_t vd = sw128_mn_desc(smem_u32(ring + st * kStageBytes) +
                                               (uint32_t)(4 * hv * kKSlice), kKSlice, 1024);
@@ -309,6 +302,33 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
         }
         umma_commit(&empty[st]);
         umma_commit(&pv_done[sb]);
+      };
+      // nq: next S to compute, np: next P V.  S_nq needs its key block and, for nq >= 2, the
+      // P V of block nq-2 (issued: np >= nq-1) to have finished with the buffer.  Every
+      // phase tested here is the one after the last phase consumed, so a parity test is
+      // unambiguous.  No progress for the wait limit -> timeout.
+      int nq = 0, np = 0;
+      long long t_prog = clock64();
+      while (ok && np < NB) {
+        bool prog = false;
+        if (nq < NB && (nq < kSB || np >= nq - 1) &&
+            mbar_try_wait(&full[nq % kStages], (nq / kStages) & 1) &&
+            (nq < kSB || mbar_try_wait(&pv_done[nq % kSB], ((nq / kSB) - 1) & 1))) {
+          tc_fence_after();
+          issue_qk(nq++);
+          prog = true;
+        }
+        if (np < nq && mbar_try_wait(&p_full[np % kSB], (np / kSB) & 1)) {
+          tc_fence_after();
+          issue_pv(np++);
+          prog = true;
+        }
+        if (prog) {
+          t_prog = clock64();
+        } else if (timeout_recorded() || clock64() - t_prog > kWaitCycles) {
+          flag_status(kStatusTimeout);
+          ok = false;
+        }
       }
       umma_commit(mma_done);
       drain_wait(mma_done, 0);
