@@ -29,8 +29,8 @@
 //
 // Roles: warps 0..3 softmax and epilogue (thread = head = TMEM lane; they also write Q's
 // tensor-memory part), warp 4 MMA issuer and TMEM owner, warps 5..8 gather the selected rows
-// with 16-byte cp.async into the swizzled ring (zero fill for skipped entries), two warps
-// per ring stage.  Every wait is bounded.
+// with 16-byte cp.async into the swizzled ring (zero fill for skipped entries), 16 rows of
+// every block each.  Every wait is bounded.
 #include <climits>
 
 #include "common.cuh"
@@ -55,13 +55,12 @@ constexpr int kBarBytes = 256;
 constexpr int kSmem = 1024 + kQBytes + kStages * kStageBytes + kBarBytes;
 constexpr uint32_t kColQ = 0, kColS = kQT * 32, kColO = kColS + kSB * kNK;
 constexpr int kWarpMma = 4, kWarpProd0 = 5, kProdThreads = 128;
-constexpr int kProdWarpsPerStage = 4 / kStages;      // each copies kNK / 2 keys of a block
 constexpr int kThreads = 32 * 9;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;
 static_assert(kColO + kNV == 512, "TMEM budget");
 static_assert(kSmem <= 227 * 1024, "shared memory budget");
-static_assert(kNK == 32 * kProdWarpsPerStage, "one key per lane of each producer warp");
+static_assert(kNK == 4 * 16, "16 keys per producer warp and block");
 
 struct LatentArgs {
   const __nv_bfloat16* q;     // [rows, H, 576]
@@ -137,7 +136,7 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
   uint8_t* Qs = smem;                 // [kQS] slices of [128 rows x 64]
   uint8_t* ring = smem + kQBytes;     // [kStages] key blocks
   uint64_t* bars = reinterpret_cast<uint64_t*>(ring + kStages * kStageBytes);
-  uint64_t* full = bars;              // [2] key block landed (its producer warps)
+  uint64_t* full = bars;              // [2] key block landed (producer threads)
   uint64_t* empty = bars + 2;         // [2] key block consumed by its P V
   uint64_t* s_full = bars + 4;        // [2] S = Q C^T done
   uint64_t* p_full = bars + 6;        // [2] P written (softmax warps)
@@ -163,7 +162,7 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&full[i], 32 * kProdWarpsPerStage);  // the producer warps of the stage
+      mbar_init(&full[i], kProdThreads);  // every producer thread copies part of a block
       mbar_init(&empty[i], 1);
     }
     for (int i = 0; i < kSB; ++i) {
@@ -203,35 +202,34 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
       }
       cp_async_commit();
     }
-    // Producer warps 2s and 2s+1 own ring stage s and copy blocks s, s+2, ...: warp h of the
-    // pair copies keys 32h..32h+31 of the block, waits for its own copies, fences and
-    // publishes at once.  Lane l resolves entry l of its 32 keys (read one round ahead) and
+    // All four producer warps copy every block, warp w the keys 16w..16w+15: each waits
+    // for its own copies, fences and arrives, so a block is published as soon as its last
+    // rows land.  Lane l resolves entry 16w + l%16 of the block (read one block ahead) and
     // copies chunks l, l+32, l+64 (< 72) of every row: chunk c is slice c/8, 16-byte column
     // c%8, swizzled by the row's index mod 8.
     const int lane_p = p & 31;
-    const int wp = p >> 5;
-    const int st = wp / kProdWarpsPerStage;
-    const int kh = (wp % kProdWarpsPerStage) * 32;  // first key of this warp in a block
+    const int kq = (p >> 5) * 16;  // first key of this warp in a block
     const __nv_bfloat16* nxt =
-        st < NB ? key_row(a, idx_row, b, spos, p0 + st * kNK + kh + lane_p, p1) : nullptr;
+        NB > 0 ? key_row(a, idx_row, b, spos, p0 + kq + (lane_p & 15), p1) : nullptr;
     uint32_t dst_off[3], src_off[3], cc_of[3];
 #pragma unroll
     for (int m = 0; m < 3; ++m) {
       const int c = lane_p + 32 * m;
       cc_of[m] = c & 7;
-      dst_off[m] = (c >> 3) * kKSlice;
+      dst_off[m] = (c >> 3) * kKSlice + kq * 128;
       src_off[m] = (c >> 3) * 64 + (c & 7) * 8;
     }
     bool q_pending = true;  // this thread's Q copies not yet published
-    uint8_t* stage = ring + st * kStageBytes + kh * 128;
-    for (int j = st; j < NB; j += kStages) {
+    for (int j = 0; j < NB; ++j) {
+      const int st = j % kStages;
       const unsigned long long cur = reinterpret_cast<unsigned long long>(nxt);
-      if (j + kStages < NB)
-        nxt = key_row(a, idx_row, b, spos, p0 + (j + kStages) * kNK + kh + lane_p, p1);
+      if (j + 1 < NB)
+        nxt = key_row(a, idx_row, b, spos, p0 + (j + 1) * kNK + kq + (lane_p & 15), p1);
       // warp-uniform wait: the whole warp takes part in the shuffles below
       if (j >= kStages && !warp_wait(&empty[st], ((j / kStages) - 1) & 1)) { ok = false; break; }
+      uint8_t* stage = ring + st * kStageBytes;
 #pragma unroll 4
-      for (int i = 0; i < 32; ++i) {
+      for (int i = 0; i < 16; ++i) {
         const __nv_bfloat16* row =
             reinterpret_cast<const __nv_bfloat16*>(__shfl_sync(0xffffffffu, cur, i));
 #pragma unroll
@@ -253,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
       mbar_arrive(&full[st]);
     }
     cp_async_wait<0>();
-    if (ok && q_pending) {  // a warp without blocks still publishes its Q copies
+    if (ok && q_pending) {  // no blocks: still publish the Q copies
       fence_proxy_async_smem();
       mbar_arrive(q_full);
     }
