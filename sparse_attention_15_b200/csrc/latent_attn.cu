@@ -12,24 +12,25 @@
 //
 // Because the key row is shared by all heads, a block of selected keys is a real
 // [H x DQK] . [DQK x keys] tensor-core product: S = Q C^T with M = 128 heads (rows past H
-// are zero), N = 64 keys, K = 576; then O += P V with M = 128 heads, N = 256, K = 64 keys.
+// are zero), N = 48 keys, K = 576; then O += P V with M = 128 heads, N = 256, K = 48 keys.
 // O for all 512 latent columns would fill the whole tensor memory, so every (query row, key
 // split) is computed by two CTAs, one per half of DV; each computes the full S (the QK
 // product is repeated, nothing is exchanged between CTAs) and the two run side by side, so
-// the second reads the gathered rows from L2.  64 keys per MMA keep the instruction count
-// per key low: a block is 36 QK and 8 PV instructions.
+// the second reads the gathered rows from L2.  A block is 36 QK and 6 PV instructions: the
+// MMA issue rate, not the tensor pipe, bounds this kernel, so the blocks are as wide as the
+// memory budgets allow while three of them stay in flight.
 //
-// Tensor memory (512 columns): Q dims 0..255 as the tensor-memory A operand of QK (4 x 32
+// Tensor memory (512 columns): Q dims 0..319 as the tensor-memory A operand of QK (5 x 32
 // columns of bf16 pairs, so those MMAs read only the key tile from shared memory), S0, S1
-// (64 columns each; P_hi / P_lo are written over them), O (256 columns).  Shared memory:
-// Q dims 256..575 (5 K-major slices with the 128-byte swizzle) and a ring of 2 key blocks
-// (64 rows x 576 dims, 9 slices).  The same bytes of a key block are the K-major B operand
+// (48 columns each; P_hi / P_lo are written over them), O (256 columns).  Shared memory:
+// Q dims 320..575 (4 K-major slices with the 128-byte swizzle) and a ring of 3 key blocks
+// (48 rows x 576 dims, 9 slices).  The same bytes of a key block are the K-major B operand
 // of QK and, for the DV/2 columns of this CTA, the MN-major B operand of PV.  P is split into
 // bf16 P_hi + P_lo (as in the masked-tile kernel) to keep float32 probability precision.
 //
 // Roles: warps 0..3 softmax and epilogue (thread = head = TMEM lane; they also write Q's
 // tensor-memory part), warp 4 MMA issuer and TMEM owner, warps 5..8 gather the selected rows
-// with 16-byte cp.async into the swizzled ring (zero fill for skipped entries), 16 rows of
+// with 16-byte cp.async into the swizzled ring (zero fill for skipped entries), 12 rows of
 // every block each.  Every wait is bounded.
 #include <climits>
 
@@ -41,18 +42,20 @@ namespace dsa {
 namespace {
 
 constexpr int kDQK = 576, kDV = 512, kNV = kDV / 2;  // N of PV per CTA
-constexpr int kNK = 64;                              // keys per block (N of QK)
+constexpr int kNK = 48;                              // keys per block (N of QK)
 constexpr int kSlices = kDQK / 64;                   // 64-dim slices of a row
-constexpr int kQT = 4;                               // Q slices in tensor memory
+constexpr int kQT = 5;                               // Q slices in tensor memory
 constexpr int kQS = kSlices - kQT;                   // Q slices in shared memory
-constexpr int kStages = 2;                           // key blocks in the ring
+constexpr int kStages = 3;                           // key blocks in the ring
 constexpr int kSB = 2;                               // S buffers
 constexpr int kKSlice = kNK * 128;                   // one slice of a key block (bytes)
 constexpr int kStageBytes = kSlices * kKSlice;
 constexpr int kQSlice = 128 * 128;                   // one slice of Q (128 rows)
 constexpr int kQBytes = kQS * kQSlice;
 constexpr int kBarBytes = 256;
-constexpr int kSmem = 1024 + kQBytes + kStages * kStageBytes + kBarBytes;
+// no alignment slack: the dynamic shared memory of a kernel without static shared memory
+// starts 1024-byte aligned (checked at run time)
+constexpr int kSmem = kQBytes + kStages * kStageBytes + kBarBytes;
 constexpr uint32_t kColQ = 0, kColS = kQT * 32, kColO = kColS + kSB * kNK;
 constexpr int kWarpMma = 4, kWarpProd0 = 5, kProdThreads = 128;
 constexpr int kThreads = 32 * 9;
@@ -60,7 +63,9 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;
 static_assert(kColO + kNV == 512, "TMEM budget");
 static_assert(kSmem <= 227 * 1024, "shared memory budget");
-static_assert(kNK == 4 * 16, "16 keys per producer warp and block");
+constexpr int kKeysPerWarp = kNK / 4;                // producer warp share of a block
+static_assert(kNK % 16 == 0 && kKeysPerWarp <= 32, "block split");
+static_assert(kKSlice % 1024 == 0, "swizzle atoms");
 
 struct LatentArgs {
   const __nv_bfloat16* q;     // [rows, H, 576]
@@ -130,21 +135,23 @@ __device__ __forceinline__ const __nv_bfloat16* key_row(const LatentArgs& a,
 }
 
 __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentArgs a) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if ((smem_u32(smem) & 1023u) != 0u) {  // the swizzled layout needs 1024-byte atoms
+    if (threadIdx.x == 0) flag_status(kStatusInternal);
+    return;
+  }
   uint8_t* Qs = smem;                 // [kQS] slices of [128 rows x 64]
   uint8_t* ring = smem + kQBytes;     // [kStages] key blocks
   uint64_t* bars = reinterpret_cast<uint64_t*>(ring + kStages * kStageBytes);
-  uint64_t* full = bars;              // [2] key block landed (producer threads)
-  uint64_t* empty = bars + 2;         // [2] key block consumed by its P V
-  uint64_t* s_full = bars + 4;        // [2] S = Q C^T done
-  uint64_t* p_full = bars + 6;        // [2] P written (softmax warps)
-  uint64_t* pv_done = bars + 8;       // [2] O += P V of that block done
-  uint64_t* q_full = bars + 10;       // Q shared-memory part landed (producer threads)
-  uint64_t* q_tm = bars + 11;         // Q tensor-memory part written (softmax warps)
-  uint64_t* mma_done = bars + 12;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  uint64_t* full = bars;              // [3] key block landed (producer threads)
+  uint64_t* empty = bars + 3;         // [3] key block consumed by its P V
+  uint64_t* s_full = bars + 6;        // [2] S = Q C^T done
+  uint64_t* p_full = bars + 8;        // [2] P written (softmax warps)
+  uint64_t* pv_done = bars + 10;      // [2] O += P V of that block done
+  uint64_t* q_full = bars + 12;       // Q shared-memory part landed (producer threads)
+  uint64_t* q_tm = bars + 13;         // Q tensor-memory part written (softmax warps)
+  uint64_t* mma_done = bars + 14;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // item = (query row, key split, DV half); the two halves of a split are neighbours
@@ -202,40 +209,40 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
       }
       cp_async_commit();
     }
-    // All four producer warps copy every block, warp w the keys 16w..16w+15: each waits
+    // All four producer warps copy every block, warp w its 12 keys 12w..12w+11: each waits
     // for its own copies, fences and arrives, so a block is published as soon as its last
-    // rows land.  Lane l resolves entry 16w + l%16 of the block (read one block ahead) and
+    // rows land.  Lane l < 12 resolves entry 12w + l of the block (read one block ahead) and
     // copies chunks l, l+32, l+64 (< 72) of every row: chunk c is slice c/8, 16-byte column
     // c%8, swizzled by the row's index mod 8.
     const int lane_p = p & 31;
-    const int kq = (p >> 5) * 16;  // first key of this warp in a block
-    const __nv_bfloat16* nxt =
-        NB > 0 ? key_row(a, idx_row, b, spos, p0 + kq + (lane_p & 15), p1) : nullptr;
+    const int kq = (p >> 5) * kKeysPerWarp;  // first key of this warp in a block
+    const int le = lane_p < kKeysPerWarp ? lane_p : 0;  // the entry this lane resolves
+    const __nv_bfloat16* nxt = NB > 0 ? key_row(a, idx_row, b, spos, p0 + kq + le, p1) : nullptr;
     uint32_t dst_off[3], src_off[3], cc_of[3];
 #pragma unroll
     for (int m = 0; m < 3; ++m) {
       const int c = lane_p + 32 * m;
       cc_of[m] = c & 7;
-      dst_off[m] = (c >> 3) * kKSlice + kq * 128;
+      dst_off[m] = (c >> 3) * kKSlice;
       src_off[m] = (c >> 3) * 64 + (c & 7) * 8;
     }
     bool q_pending = true;  // this thread's Q copies not yet published
     for (int j = 0; j < NB; ++j) {
       const int st = j % kStages;
       const unsigned long long cur = reinterpret_cast<unsigned long long>(nxt);
-      if (j + 1 < NB)
-        nxt = key_row(a, idx_row, b, spos, p0 + (j + 1) * kNK + kq + (lane_p & 15), p1);
+      if (j + 1 < NB) nxt = key_row(a, idx_row, b, spos, p0 + (j + 1) * kNK + kq + le, p1);
       // warp-uniform wait: the whole warp takes part in the shuffles below
       if (j >= kStages && !warp_wait(&empty[st], ((j / kStages) - 1) & 1)) { ok = false; break; }
       uint8_t* stage = ring + st * kStageBytes;
 #pragma unroll 4
-      for (int i = 0; i < 16; ++i) {
+      for (int i = 0; i < kKeysPerWarp; ++i) {
         const __nv_bfloat16* row =
             reinterpret_cast<const __nv_bfloat16*>(__shfl_sync(0xffffffffu, cur, i));
+        const int key = kq + i;  // row of the block; its 128-byte lines swizzle by key % 8
 #pragma unroll
         for (int m = 0; m < 3; ++m) {
           if (m == 2 && lane_p >= kDQK / 8 - 64) break;
-          cp_async16(stage + dst_off[m] + i * 128 + ((cc_of[m] ^ (i & 7)) << 4),
+          cp_async16(stage + dst_off[m] + key * 128 + ((cc_of[m] ^ (key & 7)) << 4),
                      row ? row + src_off[m] : a.kv, row ? 16u : 0u);
         }
       }
@@ -347,9 +354,11 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
         uint4 u[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c)
-          u[c] = head_ok ? __ldg(src + x0 * 8 + c) : make_uint4(0u, 0u, 0u, 0u);
+          u[c] = (head_ok && x0 * 8 + c < kQT * 8) ? __ldg(src + x0 * 8 + c)
+                                                   : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
         for (int x = 0; x < 2; ++x) {
+          if (x0 + x >= kQT) break;
           uint32_t v[32];
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
@@ -367,23 +376,27 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
     float m_used = ninf, l = 0.f;
     for (int j = 0; j < NB; ++j) {
       const int sb = j % kSB;
-      // which of the block's 64 entries are attended (the same for every head)
+      // which of the block's 48 entries are attended (the same for every head)
       const int e0 = p0 + j * kNK + lane;
-      const uint32_t bits0 = __ballot_sync(0xffffffffu, key_row(a, idx_row, b, spos, e0, p1) != nullptr);
-      const uint32_t bits1 =
-          __ballot_sync(0xffffffffu, key_row(a, idx_row, b, spos, e0 + 32, p1) != nullptr);
+      const uint32_t bits0 =
+          __ballot_sync(0xffffffffu, key_row(a, idx_row, b, spos, e0, p1) != nullptr);
+      const uint32_t bits1 = __ballot_sync(
+          0xffffffffu, lane < kNK - 32 && key_row(a, idx_row, b, spos, e0 + 32, p1) != nullptr);
       if (!warp_wait(&s_full[sb], (j / kSB) & 1)) { ok = false; break; }
       tc_fence_after();
       const uint32_t s_col = t_lane + kColS + sb * kNK;
-      uint32_t rr[64];
+      uint32_t rr[48];
       tmem_ld32(s_col, *reinterpret_cast<uint32_t(*)[32]>(rr));
-      tmem_ld32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(rr + 32));
+      tmem_ld16(s_col + 32, *reinterpret_cast<uint32_t(*)[16]>(rr + 32));
       tmem_wait_ld();
       float mx0 = ninf, mx1 = ninf;
 #pragma unroll
       for (int e = 0; e < 32; e += 2) {
         mx0 = fmaxf(mx0, (bits0 >> e) & 1u ? __uint_as_float(rr[e]) : ninf);
         mx1 = fmaxf(mx1, (bits0 >> (e + 1)) & 1u ? __uint_as_float(rr[e + 1]) : ninf);
+      }
+#pragma unroll
+      for (int e = 0; e < 16; e += 2) {
         mx0 = fmaxf(mx0, (bits1 >> e) & 1u ? __uint_as_float(rr[32 + e]) : ninf);
         mx1 = fmaxf(mx1, (bits1 >> (e + 1)) & 1u ? __uint_as_float(rr[33 + e]) : ninf);
       }
