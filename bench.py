@@ -46,6 +46,9 @@ NCU_TRAFFIC = {
     # gather_attn_kernel, c4: captured at B = 32 (same per-row work: 9 splits x 228 keys),
     # 1.3429 GB read + 5.86 MB written, scaled by the rows (x2) to the full B = 64 launch
     ("gather_attn", "c4"): (2697424000, "d0c02476b0c07381"),
+    # latent_attn_kernel, c4 with a 512+64 latent cache and 128 heads (--attn latent),
+    # captured at T = 8192 (same 64 x 2048 gathered rows): 161.01 MB read + 6.05 MB written
+    ("latent_attn", "c4"): (167062016, "3d872af04660a02e"),
 }
 
 
