@@ -307,7 +307,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kBlk, kBlk);
       constexpr uint32_t idesc_pv = idesc_bf16_f32_bmn(kBlk, C::DV);
-      const uint32_t q_base = smem_u32(Qs);
+      // descriptors: a base per operand plus constant offsets in the 16-byte address field
+      // (shared addresses stay below 256 KB, so the field never carries)
+      const uint64_t qdesc0 = sw128_kmajor_desc(smem_u32(Qs));
+      const uint64_t kdesc0 = sw128_kmajor_desc(smem_u32(KVs));
+      const uint64_t vdesc0 = sw128_mnmajor_desc(smem_u32(KVs + C::K_BYTES), C::SLICE, 1024);
       uint32_t g = 0, ni = 0;
       bool ok = true;
       // S_g = Q K_g^T into S[g & 1]
@@ -316,12 +320,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         if (!mbar_wait(&k_full[st], (gg >> 1) & 1)) return false;
         if (gg >= 2 && !mbar_wait(&s_empty[gg & 1], ((gg >> 1) - 1) & 1)) return false;
         tc_fence_after();
-        const uint32_t k_base = smem_u32(KVs + st * C::KV_BYTES);
+        const uint64_t kd = kdesc0 + (uint64_t)((st * C::KV_BYTES) >> 4);
 #pragma unroll
         for (int kk = 0; kk < C::DQK / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::SLICE + (kk & 3) * 32;
-          umma_f16_ss(tmem + (gg & 1) * C::S_COLS, sw128_kmajor_desc(q_base + off),
-                      sw128_kmajor_desc(k_base + off), idesc_qk, kk > 0 ? 1u : 0u);
+          umma_f16_ss(tmem + (gg & 1) * C::S_COLS, qdesc0 + (uint64_t)(off >> 4),
+                      kd + (uint64_t)(off >> 4), idesc_qk, kk > 0 ? 1u : 0u);
         }
         umma_commit(&s_full[gg & 1]);
         umma_commit(&k_empty[st]);
@@ -343,7 +347,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           if (j == 0 && ni > 0 && !mbar_wait(o_empty, (ni - 1) & 1)) { ok = false; break; }
           if (!mbar_wait(&v_full[gg & 1], (gg >> 1) & 1)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t v_base = smem_u32(KVs + (gg & 1) * C::KV_BYTES + C::K_BYTES);
+          const uint64_t vd = vdesc0 + (uint64_t)(((gg & 1) * C::KV_BYTES) >> 4);
           const uint32_t p_tmem = tmem + (gg & 1) * C::S_COLS;
           const uint32_t o_tmem = tmem + C::O_COL + (gg & 1) * C::DV;
 #pragma unroll
@@ -351,7 +355,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             // keys 16kk..16kk+15: 8 packed columns of P_hi at 16kk, P_lo 8 columns further;
             // V rows 16kk..: 2 swizzle atoms of 8 rows
             const uint32_t pc = 16 * kk;
-            const uint64_t vdesc = sw128_mnmajor_desc(v_base + kk * 2048, C::SLICE, 1024);
+            const uint64_t vdesc = vd + (uint64_t)((kk * 2048) >> 4);
             umma_f16_ts(o_tmem, p_tmem + pc, vdesc, idesc_pv, (j >= 2 || kk > 0) ? 1u : 0u);
             umma_f16_ts(o_tmem, p_tmem + pc + 8, vdesc, idesc_pv, 1u);
           }
@@ -426,10 +430,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         tc_fence_after();
         const uint32_t s_col = t_lane + (gg & 1) * C::S_COLS;
         // pass 1: max of the selected raw scores (the scale is positive: it commutes with max);
-        // the whole row in one TMEM round trip
+        // the whole row in one TMEM round trip, kept in registers for pass 2
         float mraw = ninf;
+        uint32_t r[kBlk];
         {
-          uint32_t r[kBlk];
           tmem_ld32(s_col + 0, *reinterpret_cast<uint32_t(*)[32]>(r + 0));
           tmem_ld32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
           tmem_ld32(s_col + 64, *reinterpret_cast<uint32_t(*)[32]>(r + 64));
@@ -451,26 +455,15 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
         const float mb = mraw * a.qk_scale;
         const bool need = mb > m_used + kRescaleLog2;
+        // a raised max rescales l now and O_grp (this group's earlier blocks of the item) after
+        // pass 2, once their P V landed -- before P_j is published, so P_j V never meets an
+        // unscaled O
+        float alpha = 1.f;
+        bool rescale_o = false;
         if (__any_sync(0xffffffffu, need)) {
           const float m_new = need ? mb : m_used;
-          const float alpha = (l > 0.f) ? exp2f(m_used - m_new) : 0.f;
-          // O_grp holds this group's earlier blocks of the item: rescale it once their P V landed
-          if (j >= 2 && __any_sync(0xffffffffu, need && l > 0.f)) {
-            if (!warp_wait(&pv_done[gg & 1], ((gg >> 1) - 1) & 1)) { ok = false; break; }
-            tc_fence_after();
-#pragma unroll 1
-            for (int c = 0; c < C::DV / 16; ++c) {
-              uint32_t r[16];
-              tmem_ld16(t_lane + o_col + c * 16, r);
-              tmem_wait_ld();
-              if (need) {
-#pragma unroll
-                for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-              }
-              tmem_st16(t_lane + o_col + c * 16, r);
-            }
-            tmem_wait_st();
-          }
+          alpha = (l > 0.f) ? exp2f(m_used - m_new) : 0.f;
+          rescale_o = j >= 2 && __any_sync(0xffffffffu, need && l > 0.f);
           if (need) {
             l *= alpha;
             m_used = m_new;
@@ -482,17 +475,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         unsigned long long rs2 = pack2(0.f, 0.f);  // row sum, two partial sums
         const unsigned long long scale2 = pack2(a.qk_scale, a.qk_scale);
         const unsigned long long nm2 = pack2(-msub, -msub);
-        // 16 keys per chunk, double-buffered TMEM reads (chunk k+1 in flight while chunk k is
-        // exponentiated); chunk k's P_hi and P_lo overwrite its own 16 S columns
-        uint32_t ra[16], rc[16];
-        uint32_t b0 = bits[0], b1 = bits[1], b2 = bits[2], b3 = bits[3];
-        auto chunk = [&](const uint32_t (&r)[16], uint32_t bw, int kk) {
+        // 16 keys per chunk, from the row held in registers since pass 1; chunk k's P_hi and
+        // P_lo overwrite its own 16 S columns
+        auto chunk = [&](uint32_t bw, int kk) {
           uint32_t ph[8], pl[8];
 #pragma unroll
           for (int e2 = 0; e2 < 8; ++e2) {
             const int e = 2 * e2;
-            const float x0 = (bw & (1u << e)) ? __uint_as_float(r[e]) : ninf;
-            const float x1 = (bw & (1u << (e + 1))) ? __uint_as_float(r[e + 1]) : ninf;
+            const float x0 = (bw & (1u << e)) ? __uint_as_float(r[16 * kk + e]) : ninf;
+            const float x1 =
+                (bw & (1u << (e + 1))) ? __uint_as_float(r[16 * kk + e + 1]) : ninf;
             float y0, y1;
             unpack2(fma2(pack2(x0, x1), scale2, nm2), y0, y1);  // scale*s - m, two keys
             const float p0 = ex2_ftz(y0), p1 = ex2_ftz(y1);
@@ -511,22 +503,30 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           tmem_st8(s_col + kk * 16, ph);
           tmem_st8(s_col + kk * 16 + 8, pl);
         };
-        tmem_ld16(s_col, ra);
-        tmem_wait_ld();
-#pragma unroll 1
+#pragma unroll
         for (int c = 0; c < 4; ++c) {
-          tmem_ld16(s_col + (2 * c + 1) * 16, rc);
-          chunk(ra, b0, 2 * c);
-          tmem_wait_ld();
-          if (c + 1 < 4) tmem_ld16(s_col + (2 * c + 2) * 16, ra);
-          chunk(rc, b0 >> 16, 2 * c + 1);
-          if (c + 1 < 4) tmem_wait_ld();
-          b0 = b1; b1 = b2; b2 = b3;
+          chunk(bits[c], 2 * c);
+          chunk(bits[c] >> 16, 2 * c + 1);
         }
         {
           float r0, r1;
           unpack2(rs2, r0, r1);
           l += r0 + r1;
+        }
+        if (rescale_o) {
+          if (!warp_wait(&pv_done[gg & 1], ((gg >> 1) - 1) & 1)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < C::DV / 16; ++c) {
+            uint32_t o[16];
+            tmem_ld16(t_lane + o_col + c * 16, o);
+            tmem_wait_ld();
+            if (need) {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            }
+            tmem_st16(t_lane + o_col + c * 16, o);
+          }
         }
         tmem_wait_st();
         tc_fence_before();
