@@ -80,32 +80,6 @@ struct FaCfg {
   static_assert(O_COL + 2 * DV <= TMEM_COLS, "TMEM budget");
 };
 
-// Instruction descriptor, kind::f16, bf16 A/B, f32 D, with the B operand MN-major.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32_bmn(int M, int N) {
-  return idesc_bf16_f32(M, N) | (1u << 16);
-}
-
-// Shared-memory descriptor of an MN-major tile with the 128-byte swizzle: 64 MN elements
-// (128 B) per swizzle row, K rows 128 B apart, 8-row atoms `sbo` apart, 64-element MN
-// groups `lbo` apart.
-__device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t start, uint32_t lbo,
-                                                       uint32_t sbo) {
-  uint64_t d = 0;
-  d |= (uint64_t)((start & 0x3FFFF) >> 4);
-  d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
-  d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
-  d |= (uint64_t)1 << 46;
-  d |= (uint64_t)2 << 61;
-  return d;
-}
-
-// 2^x on the special-function unit (flush-to-zero; exp2(-inf) = +0).
-__device__ __forceinline__ float ex2_ftz(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
 // Packed float32 pair arithmetic (sm_100): one instruction for two lanes of work.
 __device__ __forceinline__ unsigned long long pack2(float x, float y) {
   unsigned long long r;
@@ -145,15 +119,6 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, i
       " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
       "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
       : "memory");
-}
-
-__device__ __forceinline__ void drain(uint64_t* bar, uint32_t parity) {
-  const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity))
-    if (clock64() - t0 > kWaitCycles) {
-      flag_status(kStatusTimeout);
-      return;
-    }
 }
 
 // Item i -> (query block, batch row, head); longest query blocks first.
@@ -298,9 +263,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
       }
       // let the copies in flight land before exit
-      if (g >= 1) drain(&full[(g - 1) & 1], ((g - 1) >> 1) & 1);
-      if (g >= 2) drain(&full[(g - 2) & 1], ((g - 2) >> 1) & 1);
-      if (kq && ni >= 1) drain(q_full, (ni - 1) & 1);
+      if (g >= 1) drain_wait(&full[(g - 1) & 1], ((g - 1) >> 1) & 1);
+      if (g >= 2) drain_wait(&full[(g - 2) & 1], ((g - 2) >> 1) & 1);
+      if (kq && ni >= 1) drain_wait(q_full, (ni - 1) & 1);
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------------ MMA issuer
@@ -366,7 +331,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         g += nb;
       }
       umma_commit(mma_done);
-      drain(mma_done, 0);
+      drain_wait(mma_done, 0);
     }
   } else if (warp < kSoftWarps) {
     // ------------------------------------------------------------------ softmax + epilogue

@@ -56,6 +56,13 @@ __device__ __forceinline__ float gate_act(float g, int mode) {
   return mode == 2 ? g * sg : sg;
 }
 
+// 2^x on the special-function unit (flush-to-zero; exp2(-inf) = +0).
+__device__ __forceinline__ float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // ------------------------------------------------------------------------------------
 // Shared-memory addresses, mbarriers
 // ------------------------------------------------------------------------------------
@@ -112,6 +119,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
       }
     }
   }
+}
+
+// A wait used on the way out: ignores a recorded timeout (copies and MMAs already in
+// flight must land before the CTA exits) but is bounded itself.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity))
+    if (clock64() - t0 > kWaitCycles) {
+      flag_status(kStatusTimeout);
+      return;
+    }
 }
 
 // Warp-uniform bounded wait: every lane waits, and the warp proceeds only if all of them
@@ -293,6 +311,25 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          | (1u << 10)                   // B format: bf16
          | ((uint32_t)(N >> 3) << 17)   // N / 8
          | ((uint32_t)(M >> 4) << 24);  // M / 16
+}
+
+// Instruction descriptor, kind::f16, bf16 A/B, f32 D, with the B operand MN-major.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_bmn(int M, int N) {
+  return idesc_bf16_f32(M, N) | (1u << 16);
+}
+
+// Shared-memory descriptor of an MN-major tile with the 128-byte swizzle: 64 MN elements
+// (128 B) per swizzle row, K rows 128 B apart, 8-row atoms `sbo` apart, 64-element MN
+// groups `lbo` apart.
+__device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t start, uint32_t lbo,
+                                                       uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((start & 0x3FFFF) >> 4);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
 }
 
 // Instruction descriptor, kind::f8f6f4: A and B e4m3 (format code 0), f32 D, both K-major.

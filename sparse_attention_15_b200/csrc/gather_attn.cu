@@ -29,13 +29,6 @@ namespace {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLazyRescale = 8.0f;  // raise the running max only past 2^8 (log2 units)
 
-// 2^x on the special-function unit (flush-to-zero; exp2(-inf) = +0).
-__device__ __forceinline__ float ex2_ftz(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
 // Warp sums of N per-lane partials (N = 1, 2, 4), every lane receiving all N sums.  The
 // first butterfly steps halve the values each lane carries (lanes split the heads between
 // them), so N sums cost N + 4 shuffles (plus N broadcasts) instead of 5N.

@@ -122,17 +122,6 @@ struct UnitIter {
   }
 };
 
-// A wait used on the way out: ignores a recorded timeout (copies and MMAs already in
-// flight must land before the CTA exits) but is bounded itself.
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
-  const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity))
-    if (clock64() - t0 > kWaitCycles) {
-      flag_status(kStatusTimeout);
-      return;
-    }
-}
-
 template <class C, int RELU>
 __global__ void __launch_bounds__(C::THREADS, 1)
     index_scores_tc_kernel(const __grid_constant__ CUtensorMap kmap,

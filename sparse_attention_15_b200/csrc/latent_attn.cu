@@ -94,34 +94,6 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// Shared-memory descriptor of an MN-major tile with the 128-byte swizzle: 64 MN elements per
-// 128-byte row, K rows 128 B apart, 8-row atoms `sbo` apart, 64-element MN groups `lbo` apart.
-__device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t start, uint32_t lbo, uint32_t sbo) {
-  uint64_t d = 0;
-  d |= (uint64_t)((start & 0x3FFFF) >> 4);
-  d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
-  d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
-  d |= (uint64_t)1 << 46;
-  d |= (uint64_t)2 << 61;
-  return d;
-}
-
-__device__ __forceinline__ float ex2_approx(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-// Bounded wait used on the way out (copies or MMAs still in flight).
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
-  const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity))
-    if (clock64() - t0 > kWaitCycles) {
-      flag_status(kStatusTimeout);
-      return;
-    }
-}
-
 // Source row of entry p of a query's key list -- the nsink sinks first, then the selected
 // positions -- or NULL when the entry is skipped (past the split, -1, out of range, future).
 __device__ __forceinline__ const __nv_bfloat16* key_row(const LatentArgs& a,
@@ -266,7 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kNK);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, kNV) | (1u << 16);  // B MN-major
+      constexpr uint32_t idesc_pv = idesc_bf16_f32_bmn(128, kNV);
       bool ok = mbar_wait(q_full, 0) && mbar_wait(q_tm, 0);
       // descriptors: a base per operand plus constant offsets in the 16-byte address field
       // (shared addresses stay below 256 KB, so the field never carries)
@@ -295,7 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
       auto issue_pv = [&](int j) {
         const int sb = j % kSB, st = j % kStages;
         // V = the first DV columns of the key rows; this CTA's half starts at slice 4*hv
-        const uint64_t vd = sw128_mn_desc(smem_u32(ring + st * kStageBytes) +
+        const uint64_t vd = sw128_mnmajor_desc(smem_u32(ring + st * kStageBytes) +
                                               (uint32_t)(4 * hv * kKSlice), kKSlice, 1024);
         const uint32_t pt = tmem + kColS + sb * kNK;
 #pragma unroll
@@ -443,8 +415,8 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
           const int e = 2 * e2;
           const float x0 = (bw >> e) & 1u ? __uint_as_float(rr[16 * c + e]) : ninf;
           const float x1 = (bw >> (e + 1)) & 1u ? __uint_as_float(rr[16 * c + e + 1]) : ninf;
-          const float y0 = ex2_approx(fmaf(x0, a.qk_scale, -msub));
-          const float y1 = ex2_approx(fmaf(x1, a.qk_scale, -msub));
+          const float y0 = ex2_ftz(fmaf(x0, a.qk_scale, -msub));
+          const float y1 = ex2_ftz(fmaf(x1, a.qk_scale, -msub));
           rs0 += y0;
           rs1 += y1;
           const __nv_bfloat162 h2 = __floats2bfloat162_rn(y0, y1);
