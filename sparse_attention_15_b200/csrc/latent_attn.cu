@@ -11,30 +11,27 @@
 // visible to every query.
 //
 // Because the key row is shared by all heads, a block of selected keys is a real
-// [H x DQK] . [DQK x keys] tensor-core product.  Every (query row, key split) is computed by
-// a cluster of two CTAs on two SMs that split the row's dims: CTA 0 owns dims 0..255 (4
-// slices of 64), CTA 1 dims 256..575 (5 slices).  Each gathers only its slices of the
-// selected rows, computes the partial S_r = Q[:, dims_r] C[:, dims_r]^T (M = 128 heads, rows
-// past H zero; N = 48 keys), sends it to the other CTA through distributed shared memory and
-// adds the partial it receives: both CTAs then hold the same S (float addition commutes) and
-// run the same softmax, and each computes O += P V for the 256 value columns inside its own
-// dims (CTA 0: 0..255, CTA 1: 256..511).  Nothing is computed twice and every gathered byte
-// is read once.
+// [H x DQK] . [DQK x keys] tensor-core product: S = Q C^T with M = 128 heads (rows past H
+// are zero), N = 48 keys, K = 576; then O += P V with M = 128 heads, N = 256, K = 48 keys.
+// O for all 512 latent columns would fill the whole tensor memory, so every (query row, key
+// split) is computed by two CTAs, one per half of DV; each computes the full S (the QK
+// product is repeated, nothing is exchanged between CTAs) and the two run side by side, so
+// the second reads the gathered rows from L2.  A block is 36 QK and 6 PV instructions: the
+// MMA issue rate, not the tensor pipe, bounds this kernel, so the blocks are as wide as the
+// memory budgets allow while three of them stay in flight.
 //
-// Tensor memory (512 columns): Q's slices of this CTA as the tensor-memory A operand of QK
-// (32 columns of bf16 pairs per slice, all Q MMAs read only the key tile from shared
-// memory), S0, S1 (48 columns each; P_hi / P_lo are written over them), O (256 columns).
-// Shared memory: a ring of 5 key blocks (48 rows x this CTA's slices, 128-byte swizzle; the
-// same bytes are the K-major B operand of QK and, for the first 4 slices, the MN-major B
-// operand of PV) and two exchange slots for the other CTA's partial S.  P is split into bf16
-// P_hi + P_lo (as in the masked-tile kernel) to keep float32 probability precision.
+// Tensor memory (512 columns): Q dims 0..319 as the tensor-memory A operand of QK (5 x 32
+// columns of bf16 pairs, so those MMAs read only the key tile from shared memory), S0, S1
+// (48 columns each; P_hi / P_lo are written over them), O (256 columns).  Shared memory:
+// Q dims 320..575 (4 K-major slices with the 128-byte swizzle) and a ring of 3 key blocks
+// (48 rows x 576 dims, 9 slices).  The same bytes of a key block are the K-major B operand
+// of QK and, for the DV/2 columns of this CTA, the MN-major B operand of PV.  P is split into
+// bf16 P_hi + P_lo (as in the masked-tile kernel) to keep float32 probability precision.
 //
 // Roles: warps 0..3 softmax and epilogue (thread = head = TMEM lane; they also write Q's
-// slices to tensor memory and exchange the partial S), warp 4 MMA issuer and TMEM owner,
-// warps 5..8 gather the selected rows with 16-byte cp.async into the swizzled ring (zero
-// fill for skipped entries), 12 rows of every block each.  Every wait is bounded; the two
-// CTAs meet at a cluster barrier after initialisation and before exit, so neither touches
-// the other's shared memory after it has left.
+// tensor-memory part), warp 4 MMA issuer and TMEM owner, warps 5..8 gather the selected rows
+// with 16-byte cp.async into the swizzled ring (zero fill for skipped entries), 12 rows of
+// every block each.  Every wait is bounded.
 #include <climits>
 
 #include "common.cuh"
@@ -46,18 +43,20 @@ namespace {
 
 constexpr int kDQK = 576, kDV = 512, kNV = kDV / 2;  // N of PV per CTA
 constexpr int kNK = 48;                              // keys per block (N of QK)
-constexpr int kMaxSl = 5;                            // 64-dim slices per CTA (CTA 0: 4)
-constexpr int kStages = 5;                           // key blocks in the ring
+constexpr int kSlices = kDQK / 64;                   // 64-dim slices of a row
+constexpr int kQT = 5;                               // Q slices in tensor memory
+constexpr int kQS = kSlices - kQT;                   // Q slices in shared memory
+constexpr int kStages = 3;                           // key blocks in the ring
 constexpr int kSB = 2;                               // S buffers
 constexpr int kKSlice = kNK * 128;                   // one slice of a key block (bytes)
-constexpr int kStageBytes = kMaxSl * kKSlice;
-constexpr int kXRow = kNK + 4;                       // floats per exchanged row (padded)
-constexpr int kXSlot = 128 * kXRow * 4;              // one exchange slot (bytes)
+constexpr int kStageBytes = kSlices * kKSlice;
+constexpr int kQSlice = 128 * 128;                   // one slice of Q (128 rows)
+constexpr int kQBytes = kQS * kQSlice;
 constexpr int kBarBytes = 256;
 // no alignment slack: the dynamic shared memory of a kernel without static shared memory
 // starts 1024-byte aligned (checked at run time)
-constexpr int kSmem = kStages * kStageBytes + 2 * kXSlot + kBarBytes;
-constexpr uint32_t kColQ = 0, kColS = kMaxSl * 32, kColO = kColS + kSB * kNK;
+constexpr int kSmem = kQBytes + kStages * kStageBytes + kBarBytes;
+constexpr uint32_t kColQ = 0, kColS = kQT * 32, kColO = kColS + kSB * kNK;
 constexpr int kWarpMma = 4, kWarpProd0 = 5, kProdThreads = 128;
 constexpr int kThreads = 32 * 9;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -66,7 +65,7 @@ static_assert(kColO + kNV == 512, "TMEM budget");
 static_assert(kSmem <= 227 * 1024, "shared memory budget");
 constexpr int kKeysPerWarp = kNK / 4;                // producer warp share of a block
 static_assert(kNK % 16 == 0 && kKeysPerWarp <= 32, "block split");
-static_assert(kKSlice % 1024 == 0 && (kStages * kStageBytes) % 16 == 0, "alignment");
+static_assert(kKSlice % 1024 == 0, "swizzle atoms");
 
 struct LatentArgs {
   const __nv_bfloat16* q;     // [rows, H, 576]
@@ -95,67 +94,6 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// ---- the two CTAs of a cluster: rank, barrier, distributed shared memory
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-// Both CTAs arrive and wait (all threads of both CTAs, aligned).  Used twice: after the
-// mbarriers are initialised (no code path before it) and before exit (every wait of a CTA
-// is bounded, so each reaches it in bounded time).
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
-               "barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// Shared address of the same location in CTA `rank` of this cluster.
-__device__ __forceinline__ uint32_t map_peer(uint32_t local, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ void st_peer_v4(uint32_t addr, float a, float b, float c, float d) {
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b),
-               "f"(c), "f"(d)
-               : "memory");
-}
-// Arrive on an mbarrier of the other CTA, releasing this thread's earlier writes at cluster
-// scope.
-__device__ __forceinline__ void mbar_arrive_peer(uint32_t bar_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_addr)
-               : "memory");
-}
-// Bounded wait with cluster-scope acquire: the other CTA's writes released by its arrives
-// are visible afterwards.
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ bool warp_wait_cluster(uint64_t* bar, uint32_t parity) {
-  bool ok = mbar_try_wait_cluster(bar, parity);
-  if (!ok) {
-    const long long t0 = clock64();
-    for (uint32_t i = 1;; ++i) {
-      if (mbar_try_wait_cluster(bar, parity)) { ok = true; break; }
-      if ((i & 255u) == 0u) {
-        if (timeout_recorded()) break;
-        if (clock64() - t0 > kWaitCycles) {
-          flag_status(kStatusTimeout);
-          break;
-        }
-      }
-    }
-  }
-  return __all_sync(0xffffffffu, ok);
-}
-
 // Source row of entry p of a query's key list -- the nsink sinks first, then the selected
 // positions -- or NULL when the entry is skipped (past the split, -1, out of range, future).
 __device__ __forceinline__ const __nv_bfloat16* key_row(const LatentArgs& a,
@@ -170,26 +108,26 @@ __device__ __forceinline__ const __nv_bfloat16* key_row(const LatentArgs& a,
 
 __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  uint8_t* ring = smem;                                          // [kStages] key blocks
-  float* xb = reinterpret_cast<float*>(smem + kStages * kStageBytes);  // [2][128][kXRow]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes + 2 * kXSlot);
-  uint64_t* full = bars;              // [5] key block landed (producer threads)
-  uint64_t* empty = bars + 5;         // [5] key block consumed by its P V
-  uint64_t* s_full = bars + 10;       // [2] partial S = Q_r C_r^T done
-  uint64_t* p_full = bars + 12;       // [2] P written (softmax warps)
-  uint64_t* pv_done = bars + 14;      // [2] O += P V of that block done
-  uint64_t* q_tm = bars + 16;         // Q written to tensor memory (softmax warps)
-  uint64_t* mma_done = bars + 17;
-  uint64_t* x_full = bars + 18;       // [2] the other CTA's partial S is in xb[slot]
-  uint64_t* x_free = bars + 20;       // [2] the other CTA has read the partial sent to it
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 22);
+  if ((smem_u32(smem) & 1023u) != 0u) {  // the swizzled layout needs 1024-byte atoms
+    if (threadIdx.x == 0) flag_status(kStatusInternal);
+    return;
+  }
+  uint8_t* Qs = smem;                 // [kQS] slices of [128 rows x 64]
+  uint8_t* ring = smem + kQBytes;     // [kStages] key blocks
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + kStages * kStageBytes);
+  uint64_t* full = bars;              // [3] key block landed (producer threads)
+  uint64_t* empty = bars + 3;         // [3] key block consumed by its P V
+  uint64_t* s_full = bars + 6;        // [2] S = Q C^T done
+  uint64_t* p_full = bars + 8;        // [2] P written (softmax warps)
+  uint64_t* pv_done = bars + 10;      // [2] O += P V of that block done
+  uint64_t* q_full = bars + 12;       // Q shared-memory part landed (producer threads)
+  uint64_t* q_tm = bars + 13;         // Q tensor-memory part written (softmax warps)
+  uint64_t* mma_done = bars + 14;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_rank();   // = the value half this CTA computes
-  const uint32_t peer = rank ^ 1u;
-  const int fs = rank ? 4 : 0;            // first 64-dim slice this CTA owns
-  const int ns = rank ? 5 : 4;            // slices it owns
-  // item = (query row, key split); the cluster's two CTAs take the two halves
+  // item = (query row, key split, DV half); the two halves of a split are neighbours
+  const int hv = blockIdx.x & 1;
   const int rs = blockIdx.x >> 1;
   const int sp = rs % a.nsplit;
   const int r = rs / a.nsplit;
@@ -198,12 +136,10 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
   const int nkeys = a.nsink + a.K;
   const int p0 = sp * a.kps;
   const int p1 = min(nkeys, p0 + a.kps);
-  const bool aligned = (smem_u32(smem) & 1023u) == 0u;  // the swizzled layout needs it
-  const int NB = aligned ? (p1 - p0 + kNK - 1) / kNK : 0;
+  const int NB = (p1 - p0 + kNK - 1) / kNK;
   const int32_t* idx_row = a.idx + (size_t)r * a.K;
 
   if (threadIdx.x == 0) {
-    if (!aligned) flag_status(kStatusInternal);
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&full[i], kProdThreads);  // every producer thread copies part of a block
       mbar_init(&empty[i], 1);
@@ -212,9 +148,8 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 4);
       mbar_init(&pv_done[i], 1);
-      mbar_init(&x_full[i], 128);  // every softmax thread of the other CTA
-      mbar_init(&x_free[i], 128);
     }
+    mbar_init(q_full, kProdThreads);
     mbar_init(q_tm, 4);
     mbar_init(mma_done, 1);
     fence_mbar_init();
@@ -226,85 +161,114 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  cluster_sync();  // the other CTA's barriers are initialised before anyone arrives on them
   const uint32_t tmem = *tmem_slot;
 
   if (warp >= kWarpProd0) {
     // ------------------------------------------------------------------ gather producers
+    const int p = threadIdx.x - kWarpProd0 * 32;
+    bool ok = true;
+    // Q dims 256..575 of every head: 128 rows x 40 chunks of 16 bytes
+    {
+      const __nv_bfloat16* q0 = a.q + (size_t)r * a.H * kDQK;
+#pragma unroll 4
+      for (int i = 0; i < kQS * 8; ++i) {
+        const int e = p + kProdThreads * i;
+        const int row = e / (kQS * 8), k = e - row * (kQS * 8);
+        const int x = k >> 3, cc = k & 7;
+        const bool in = row < a.H;
+        const __nv_bfloat16* src = in ? q0 + (size_t)row * kDQK + (kQT + x) * 64 + cc * 8 : a.q;
+        cp_async16(Qs + x * kQSlice + row * 128 + ((cc ^ (row & 7)) << 4), src, in ? 16u : 0u);
+      }
+      cp_async_commit();
+    }
     // All four producer warps copy every block, warp w its 12 keys 12w..12w+11: each waits
     // for its own copies, fences and arrives, so a block is published as soon as its last
     // rows land.  Lane l < 12 resolves entry 12w + l of the block (read one block ahead) and
-    // copies chunks l, l+32 (< 8 * ns) of this CTA's part of every row: chunk c is slice
-    // fs + c/8, 16-byte column c%8, swizzled by the row's index mod 8.
-    const int p = threadIdx.x - kWarpProd0 * 32;
+    // copies chunks l, l+32, l+64 (< 72) of every row: chunk c is slice c/8, 16-byte column
+    // c%8, swizzled by the row's index mod 8.
     const int lane_p = p & 31;
     const int kq = (p >> 5) * kKeysPerWarp;  // first key of this warp in a block
     const int le = lane_p < kKeysPerWarp ? lane_p : 0;  // the entry this lane resolves
     const __nv_bfloat16* nxt = NB > 0 ? key_row(a, idx_row, b, spos, p0 + kq + le, p1) : nullptr;
-    uint32_t dst_off[2], src_off[2], cc_of[2];
+    uint32_t dst_off[3], src_off[3], cc_of[3];
 #pragma unroll
-    for (int m = 0; m < 2; ++m) {
+    for (int m = 0; m < 3; ++m) {
       const int c = lane_p + 32 * m;
       cc_of[m] = c & 7;
       dst_off[m] = (c >> 3) * kKSlice;
-      src_off[m] = (fs + (c >> 3)) * 64 + (c & 7) * 8;
+      src_off[m] = (c >> 3) * 64 + (c & 7) * 8;
     }
-    const bool two = lane_p + 32 < ns * 8;  // this lane copies a second chunk of each row
+    bool q_pending = true;  // this thread's Q copies not yet published
     for (int j = 0; j < NB; ++j) {
       const int st = j % kStages;
       const unsigned long long cur = reinterpret_cast<unsigned long long>(nxt);
       if (j + 1 < NB) nxt = key_row(a, idx_row, b, spos, p0 + (j + 1) * kNK + kq + le, p1);
       // warp-uniform wait: the whole warp takes part in the shuffles below
-      if (j >= kStages && !warp_wait(&empty[st], ((j / kStages) - 1) & 1)) break;
+      if (j >= kStages && !warp_wait(&empty[st], ((j / kStages) - 1) & 1)) { ok = false; break; }
       uint8_t* stage = ring + st * kStageBytes;
 #pragma unroll 4
       for (int i = 0; i < kKeysPerWarp; ++i) {
         const __nv_bfloat16* row =
             reinterpret_cast<const __nv_bfloat16*>(__shfl_sync(0xffffffffu, cur, i));
         const int key = kq + i;  // row of the block; its 128-byte lines swizzle by key % 8
-        cp_async16(stage + dst_off[0] + key * 128 + ((cc_of[0] ^ (key & 7)) << 4),
-                   row ? row + src_off[0] : a.kv, row ? 16u : 0u);
-        if (two)
-          cp_async16(stage + dst_off[1] + key * 128 + ((cc_of[1] ^ (key & 7)) << 4),
-                     row ? row + src_off[1] : a.kv, row ? 16u : 0u);
+#pragma unroll
+        for (int m = 0; m < 3; ++m) {
+          if (m == 2 && lane_p >= kDQK / 8 - 64) break;
+          cp_async16(stage + dst_off[m] + key * 128 + ((cc_of[m] ^ (key & 7)) << 4),
+                     row ? row + src_off[m] : a.kv, row ? 16u : 0u);
+        }
       }
       cp_async_commit();
+      if (q_pending) {  // the Q group (committed first) has landed
+        cp_async_wait<1>();
+        fence_proxy_async_smem();
+        mbar_arrive(q_full);
+        q_pending = false;
+      }
       cp_async_wait<0>();
       fence_proxy_async_smem();
       mbar_arrive(&full[st]);
     }
     cp_async_wait<0>();
+    if (ok && q_pending) {  // no blocks: still publish the Q copies
+      fence_proxy_async_smem();
+      mbar_arrive(q_full);
+    }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kNK);
       constexpr uint32_t idesc_pv = idesc_bf16_f32_bmn(128, kNV);
-      bool ok = NB == 0 || mbar_wait(q_tm, 0);
-      // descriptors: a base plus constant offsets in the 16-byte address field (shared
-      // addresses stay below 256 KB, so the field never carries)
+      bool ok = mbar_wait(q_full, 0) && mbar_wait(q_tm, 0);
+      // descriptors: a base per operand plus constant offsets in the 16-byte address field
+      // (shared addresses stay below 256 KB, so the field never carries)
+      const uint64_t qdesc0 = sw128_kmajor_desc(smem_u32(Qs));
       const uint64_t kdesc0 = sw128_kmajor_desc(smem_u32(ring));
-      // partial S_j = Q_r C_j^T into S[j % 2] (the buffer last held P_{j-2}); O += P_j V_j.
-      // Issued in whatever order their inputs arrive.
+      // S_j = Q C_j^T into S[j % 2] (the buffer last held P_{j-2}); O += P_j V_j.  Issued in
+      // whatever order their inputs arrive: a P V never waits behind the next block's load.
       auto issue_qk = [&](int j) {
         const int st = j % kStages, sb = j % kSB;
-        const uint64_t kd = kdesc0 + (uint64_t)((st * kStageBytes) >> 4);
+        const uint64_t kd = kdesc0 + (uint64_t)(st * (kStageBytes >> 4));
         const uint32_t d = tmem + kColS + sb * kNK;
 #pragma unroll
-        for (int x = 0; x < kMaxSl; ++x) {
-          if (x >= ns) break;
+        for (int x = 0; x < kSlices; ++x)
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            umma_f16_ts(d, tmem + kColQ + x * 32 + kk * 8,
-                        kd + (uint64_t)((x * kKSlice + kk * 32) >> 4), idesc_qk,
-                        (x | kk) ? 1u : 0u);
-        }
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t bdesc = kd + (uint64_t)((x * kKSlice + kk * 32) >> 4);
+            const uint32_t acc = (x | kk) ? 1u : 0u;
+            if (x < kQT)
+              umma_f16_ts(d, tmem + kColQ + x * 32 + kk * 8, bdesc, idesc_qk, acc);
+            else
+              umma_f16_ss(d, qdesc0 + (uint64_t)(((x - kQT) * kQSlice + kk * 32) >> 4), bdesc,
+                          idesc_qk, acc);
+          }
         umma_commit(&s_full[sb]);
       };
       auto issue_pv = [&](int j) {
         const int sb = j % kSB, st = j % kStages;
-        // V = this CTA's value half: the first 4 slices of its part of the rows
-        const uint64_t vd =
-            sw128_mnmajor_desc(smem_u32(ring + st * kStageBytes), kKSlice, 1024);
+        // V = the first DV columns of the key rows; this CTA's half starts at slice 4*hv
+        const uint64_t vd = sw128_mnmajor_desc(smem_u32(ring + st * kStageBytes) +
+                                              (uint32_t)(4 * hv * kKSlice), kKSlice, 1024);
         const uint32_t pt = tmem + kColS + sb * kNK;
 #pragma unroll
         for (int c = 0; c < kNK / 16; ++c) {
@@ -353,32 +317,34 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
     const uint32_t t_lane = tmem + ((uint32_t)(warp * 32) << 16);
     const float ninf = __int_as_float(0xff800000);
     bool ok = true;
-    // Q's slices of this CTA for head h -> TMEM columns kColQ.. (bf16 pairs; zeros for
-    // h >= H), each slice's 8 loads in flight before its store
+    // Q dims 0..255 of head h -> TMEM columns kColQ.. (bf16 pairs; zeros for h >= H), two
+    // batches of loads, each all in flight before its stores
     {
-      const uint4* src =
-          reinterpret_cast<const uint4*>(a.q + ((size_t)r * a.H + h) * kDQK + fs * 64);
+      const uint4* src = reinterpret_cast<const uint4*>(a.q + ((size_t)r * a.H + h) * kDQK);
 #pragma unroll
-      for (int x = 0; x < kMaxSl; ++x) {
-        if (x >= ns) break;
-        uint32_t v[32];
+      for (int x0 = 0; x0 < kQT; x0 += 2) {
+        uint4 u[16];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 u = head_ok ? __ldg(src + x * 8 + c) : make_uint4(0u, 0u, 0u, 0u);
-          v[4 * c] = u.x; v[4 * c + 1] = u.y; v[4 * c + 2] = u.z; v[4 * c + 3] = u.w;
+        for (int c = 0; c < 16; ++c)
+          u[c] = (head_ok && x0 * 8 + c < kQT * 8) ? __ldg(src + x0 * 8 + c)
+                                                   : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          if (x0 + x >= kQT) break;
+          uint32_t v[32];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            v[4 * c] = u[x * 8 + c].x; v[4 * c + 1] = u[x * 8 + c].y;
+            v[4 * c + 2] = u[x * 8 + c].z; v[4 * c + 3] = u[x * 8 + c].w;
+          }
+          tmem_st32(t_lane + kColQ + (x0 + x) * 32, v);
         }
-        tmem_st32(t_lane + kColQ + x * 32, v);
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(q_tm);
     }
-    // this thread's row of the exchange slots, here and in the other CTA
-    const uint32_t xrow = smem_u32(xb) + (uint32_t)(h * kXRow * 4);
-    const uint32_t xrow_peer = map_peer(xrow, peer);
-    const uint32_t x_free_peer = map_peer(smem_u32(x_free), peer);
-    const uint32_t x_full_peer = map_peer(smem_u32(x_full), peer);
     float m_used = ninf, l = 0.f;
     for (int j = 0; j < NB; ++j) {
       const int sb = j % kSB;
@@ -395,30 +361,6 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
       tmem_ld32(s_col, *reinterpret_cast<uint32_t(*)[32]>(rr));
       tmem_ld16(s_col + 32, *reinterpret_cast<uint32_t(*)[16]>(rr + 32));
       tmem_wait_ld();
-      // send this partial to the other CTA (its slot sb, once it has read block j-2 from it)
-      if (j >= kSB && !warp_wait_cluster(&x_free[sb], ((j / kSB) - 1) & 1)) { ok = false; break; }
-      const uint32_t slot_off = (uint32_t)(sb * kXSlot);
-#pragma unroll
-      for (int c = 0; c < kNK / 4; ++c)
-        st_peer_v4(xrow_peer + slot_off + c * 16, __uint_as_float(rr[4 * c]),
-                   __uint_as_float(rr[4 * c + 1]), __uint_as_float(rr[4 * c + 2]),
-                   __uint_as_float(rr[4 * c + 3]));
-      mbar_arrive_peer(x_full_peer + sb * 8);
-      // receive the other CTA's partial and add it: S = S_0 + S_1 in both CTAs
-      if (!warp_wait_cluster(&x_full[sb], (j / kSB) & 1)) { ok = false; break; }
-      {
-        const float4* xr = reinterpret_cast<const float4*>(
-            reinterpret_cast<const uint8_t*>(xb) + slot_off + h * kXRow * 4);
-#pragma unroll
-        for (int c = 0; c < kNK / 4; ++c) {
-          const float4 o = xr[c];
-          rr[4 * c] = __float_as_uint(__uint_as_float(rr[4 * c]) + o.x);
-          rr[4 * c + 1] = __float_as_uint(__uint_as_float(rr[4 * c + 1]) + o.y);
-          rr[4 * c + 2] = __float_as_uint(__uint_as_float(rr[4 * c + 2]) + o.z);
-          rr[4 * c + 3] = __float_as_uint(__uint_as_float(rr[4 * c + 3]) + o.w);
-        }
-      }
-      mbar_arrive_peer(x_free_peer + sb * 8);  // the slot may be refilled
       float mx0 = ninf, mx1 = ninf;
 #pragma unroll
       for (int e = 0; e < 32; e += 2) {
@@ -504,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
         float f = l > 0.f ? 1.0f / l : 0.f;
         if (a.gate && head_ok)
           f *= gate_act(__bfloat162float(a.gate[(size_t)r * a.H + h]), a.gate_mode);
-        __nv_bfloat16* orow = a.out + ((size_t)r * a.H + h) * kDV + rank * kNV;
+        __nv_bfloat16* orow = a.out + ((size_t)r * a.H + h) * kDV + hv * kNV;
 #pragma unroll 1
         for (int c = 0; c < kNV / 32; ++c) {
           uint32_t o[32];
@@ -526,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
         }
       } else {
         const size_t pi = ((size_t)r * a.nsplit + sp) * a.H + h;
-        float* po = a.part_o + pi * kDV + rank * kNV;
+        float* po = a.part_o + pi * kDV + hv * kNV;
 #pragma unroll 1
         for (int c = 0; c < kNV / 32; ++c) {
           uint32_t o[32];
@@ -540,8 +482,8 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
                                    __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3]));
           }
         }
-        // both CTAs hold the same (m, l): the first writes them
-        if (rank == 0 && head_ok) {
+        // both halves hold the same (m, l): the first writes them
+        if (hv == 0 && head_ok) {
           a.part_ml[pi * 2] = l > 0.f ? m_used : ninf;
           a.part_ml[pi * 2 + 1] = l;
         }
@@ -555,7 +497,6 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
-  cluster_sync();  // the other CTA is done with this CTA's shared memory
 }
 
 // Key splits per query row: the count whose waves of CTA pairs (one CTA per SM, 148 SMs)
@@ -624,21 +565,8 @@ cudaError_t launch_latent_attn(const LatentProblem& p, void* ws, size_t ws_bytes
   cudaError_t e = cudaFuncSetAttribute(latent_attn_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
-  // clusters of the two CTAs of a (row, split): co-scheduled on two SMs
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)grid);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kSmem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, latent_attn_kernel, a);
-  if (e == cudaSuccess) e = cudaGetLastError();
+  latent_attn_kernel<<<(unsigned)grid, kThreads, kSmem, st>>>(a);
+  e = cudaGetLastError();
   if (e != cudaSuccess || a.nsplit == 1) return e;
   return launch_split_combine(1, a.part_o, a.part_ml, (int)rows, a.nsplit, p.H, kDV, p.gate,
                               p.gate_mode, p.out, st);
