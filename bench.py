@@ -41,14 +41,14 @@ F32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # DRAM traffic per launch from committed ncu captures: (kernel, config) -> (bytes,
 # sha256 of the kernel source when captured).  Reported as null when the source changed.
 NCU_TRAFFIC = {
-    # masked_attn_tc_kernel, c2 full size: 64.29 MB read + 3.71 MB written
-    ("masked_attn", "c2"): (68003584, "821b60f19b62a88f"),
+    # masked_attn_tc_kernel, c2 full size: 64.60 MB read + 5.00 MB written
+    ("masked_attn", "c2"): (69596928, "d6d3e430c765aa96"),
     # gather_attn_kernel, c4: captured at B = 32 (same per-row work: 9 splits x 228 keys),
-    # 1.3429 GB read + 5.63 MB written, scaled by the rows (x2) to the full B = 64 launch
-    ("gather_attn", "c4"): (2697052672, "c2327dbecd157b64"),
+    # 1.3430 GB read + 5.71 MB written, scaled by the rows (x2) to the full B = 64 launch
+    ("gather_attn", "c4"): (2697416704, "1cec4a66ced24331"),
     # latent_attn_kernel, c4 with a 512+64 latent cache and 128 heads (--attn latent),
-    # captured at T = 8192 (same 64 x 2048 gathered rows): 161.01 MB read + 6.05 MB written
-    ("latent_attn", "c4"): (167062016, "3d872af04660a02e"),
+    # captured at T = 8192 (same 64 x 2048 gathered rows): 161.02 MB read + 6.96 MB written
+    ("latent_attn", "c4"): (167974656, "95e4f381d8160992"),
 }
 
 
