@@ -277,7 +277,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         uint32_t rb[2][16];
         tmem_ld16(t_lane + ab * C::ACC_COLS + col0, rb[0]);
         tmem_wait_ld();
-        float acc4[4] = {0.f, 0.f, 0.f, 0.f};  // four independent FMA chains
+        // four independent FMA chains (heads h % 4) as two packed float32 pairs
+        unsigned long long acc01 = pack2(0.f, 0.f), acc23 = pack2(0.f, 0.f);
 #pragma unroll
         for (int cc = 0; cc < NCH; ++cc) {
           if (cc + 1 < NCH) {
@@ -317,17 +318,18 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                   d0 = fmaxf(d0, 0.f); d1 = fmaxf(d1, 0.f); d2 = fmaxf(d2, 0.f);
                   d3 = fmaxf(d3, 0.f);
                 }
-                acc4[0] = fmaf(w4.x, d0, acc4[0]);
-                acc4[1] = fmaf(w4.y, d1, acc4[1]);
-                acc4[2] = fmaf(w4.z, d2, acc4[2]);
-                acc4[3] = fmaf(w4.w, d3, acc4[3]);
+                acc01 = fma2(pack2(w4.x, w4.y), pack2(d0, d1), acc01);
+                acc23 = fma2(pack2(w4.z, w4.w), pack2(d2, d3), acc23);
               }
               if ((c0 + 16) % C::HI == 0) {  // the query's last chunk: finish and store
-                float v = ((acc4[0] + acc4[1]) + (acc4[2] + acc4[3])) * a.scale;
+                float a0, a1, a2, a3;
+                unpack2(acc01, a0, a1);
+                unpack2(acc23, a2, a3);
+                float v = ((a0 + a1) + (a2 + a3)) * a.scale;
                 if (RELU == 1) v = fmaxf(v, 0.f);
                 if (t < a.T)
                   a.scores[((size_t)it.b * a.S + s) * a.T + t] = (t <= s + a.q_off) ? v : ninf;
-                acc4[0] = acc4[1] = acc4[2] = acc4[3] = 0.f;
+                acc01 = acc23 = pack2(0.f, 0.f);
               }
             }
           }
