@@ -41,8 +41,8 @@ F32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # DRAM traffic per launch from committed ncu captures: (kernel, config) -> (bytes,
 # sha256 of the kernel source when captured).  Reported as null when the source changed.
 NCU_TRAFFIC = {
-    # masked_attn_tc_kernel, c2 full size: 64.60 MB read + 5.00 MB written
-    ("masked_attn", "c2"): (69596928, "d6d3e430c765aa96"),
+    # masked_attn_tc_kernel, c2 full size: 64.77 MB read + 5.32 MB written
+    ("masked_attn", "c2"): (70092544, "c156aeec6972c935"),
     # gather_attn_kernel, c4: captured at B = 32 (same per-row work: 9 splits x 228 keys),
     # 1.3430 GB read + 5.71 MB written, scaled by the rows (x2) to the full B = 64 launch
     ("gather_attn", "c4"): (2697416704, "1cec4a66ced24331"),
