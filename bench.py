@@ -500,7 +500,13 @@ def run_reference(args, world, rank):
     if rank != 0:
         return
     cfg = get_config(args.config)
-    x = dsa_inputs(cfg, device="cpu", B=1)
+    latent = getattr(args, "attn", "expanded") == "latent"
+    if latent:  # the latent form: shared 512+64 rows, the oracle's latent attention
+        x = dsa_inputs(cfg, device="cpu", B=1, need=("q_idx", "k_idx", "w"))
+        lt = latent_inputs(cfg, H=args.latent_heads, device="cpu", B=1)
+        x.update({"q": lt["q"], "k": lt["kv"], "v": None, "gate": lt["gate"]})
+    else:
+        x = dsa_inputs(cfg, device="cpu", B=1)
     per_step = {"c1": 16, "c2": 4, "c3": 1, "c4": 1, "c5": 1}[cfg.name]
     rows_all = sample_rows(cfg.S, max(per_step * (args.steps + args.warmup), 1))
     rng = np.random.default_rng(0)
@@ -520,7 +526,8 @@ def run_reference(args, world, rank):
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total_s / max(args.steps, 1), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(cfg, cfg.B if cfg.name != "c4" else cfg.B),
+        "config": dict(workload_config(cfg, cfg.B), attention_form="latent" if latent else
+                       "expanded"),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": f"{per_step} query row(s) per step of batch row 0, spread "
                                    f"over the {cfg.S} queries; float64 numpy oracle"},
