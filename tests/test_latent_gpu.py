@@ -152,3 +152,34 @@ def test_full_size_latent(name, rows):
         ref = _oracle_rows(x, idx.numpy(), rows, "off")
         P.assert_attn_close(got[0, rows], ref, torch.bfloat16, f"{name} latent rows")
     assert torch.isfinite(got.float()).all()
+
+
+@pytest.mark.parametrize("NS", [0, 3])
+def test_latent_attn_rows_without_valid_keys(NS):
+    # rows whose lists hold only -1 or future entries: zeros without sinks, the sinks'
+    # softmax alone with them
+    B, S, T, H, K = 1, 8, 100, 128, 48
+    x = _latent(B, S, T, H, NS, seed=9)
+    idx = random_selection(B, S, T, K, seed=19).numpy()
+    q_off = T - S
+    idx[0, 0, :] = -1
+    idx[0, 3, :] = -1
+    idx[0, 5, :] = np.arange(K) % 3 + 5 + q_off + 1  # all in the future of query 5
+    idx[0, 5, 1::2] = -1
+    got = dsa.dsa_sparse_attn_latent(_dev(x["q"]), _dev(x["kv"]), torch.from_numpy(idx).to(DEV),
+                                     sink_kv=_dev(x["sink_kv"]))
+    ref = O.sparse_attention_latent(x["q"], x["kv"], idx, DV, sink_kv=x["sink_kv"])
+    if NS == 0:
+        assert float(np.abs(ref[0, [0, 3, 5]]).max()) == 0.0
+        assert torch.count_nonzero(got[0, [0, 3, 5]].float()).item() == 0
+    P.assert_attn_close(got, ref, torch.bfloat16, f"latent empty rows NS={NS}")
+
+
+@pytest.mark.parametrize("H", [1, 128])
+def test_latent_attn_smallest_shapes(H):
+    # one query against one key, one head (127 padded tile rows) or all 128
+    x = _latent(1, 1, 1, H, seed=29)
+    idx = torch.zeros((1, 1, 1), dtype=torch.int32)
+    got = dsa.dsa_sparse_attn_latent(_dev(x["q"]), _dev(x["kv"]), idx.to(DEV))
+    ref = O.sparse_attention_latent(x["q"], x["kv"], idx.numpy(), DV)
+    P.assert_attn_close(got, ref, torch.bfloat16, f"latent 1x1 H={H}")
