@@ -252,7 +252,7 @@ dsa_status dsa_sparse_attn_sinks(dsa_dtype dtype, const void* q, const void* k, 
  *   out     [B,S,H,DV]   bf16     float32 accumulation, one rounding, gate before it; a row
  *                                 with no valid key gets zeros
  *   Requires bf16, DQK == 576 and DV == 512 (kv_lora_rank 512 + a 64-dim RoPE slice),
- *   1 <= H <= 128, 16-byte aligned pointers.  Tensor-core kernel: S = Q kv^T per block of 32
+ *   1 <= H <= 128, 16-byte aligned pointers.  Tensor-core kernel: S = Q kv^T per block of 48
  *   selected rows with M = 128 heads, then O += P V.  Workspace (split-key partials of
  *   decode-shaped calls) from dsa_sparse_attn_latent_workspace_bytes; 0 -> NULL is fine.
  * --------------------------------------------------------------------------------- */
