@@ -48,7 +48,8 @@ NCU_TRAFFIC = {
     ("gather_attn", "c4"): (2697416704, "1cec4a66ced24331"),
     # latent_attn_kernel, c4 with a 512+64 latent cache and 128 heads (--attn latent),
     # captured at T = 8192 (same 64 x 2048 gathered rows): 161.02 MB read + 6.96 MB written
-    ("latent_attn", "c4"): (167974656, "95e4f381d8160992"),
+    # (source hash after two comment-only corrections to the captured file)
+    ("latent_attn", "c4"): (167974656, "213cb481e4ce1559"),
 }
 
 

@@ -167,7 +167,7 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
     // ------------------------------------------------------------------ gather producers
     const int p = threadIdx.x - kWarpProd0 * 32;
     bool ok = true;
-    // Q dims 256..575 of every head: 128 rows x 40 chunks of 16 bytes
+    // Q dims 320..575 of every head: 128 rows x 32 chunks of 16 bytes
     {
       const __nv_bfloat16* q0 = a.q + (size_t)r * a.H * kDQK;
 #pragma unroll 4
@@ -317,8 +317,8 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_kernel(const LatentAr
     const uint32_t t_lane = tmem + ((uint32_t)(warp * 32) << 16);
     const float ninf = __int_as_float(0xff800000);
     bool ok = true;
-    // Q dims 0..255 of head h -> TMEM columns kColQ.. (bf16 pairs; zeros for h >= H), two
-    // batches of loads, each all in flight before its stores
+    // Q dims 0..319 of head h -> TMEM columns kColQ.. (bf16 pairs; zeros for h >= H), in
+    // batches of two slices, each batch's loads all in flight before its stores
     {
       const uint4* src = reinterpret_cast<const uint4*>(a.q + ((size_t)r * a.H + h) * kDQK);
 #pragma unroll
