@@ -515,3 +515,21 @@ def test_latent_attention_closed_forms():
     a = O.sparse_attention_latent(q[:, :, perm], kv, sel3, dv)
     b = O.sparse_attention_latent(q, kv, sel3, dv)[:, :, perm]
     np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+
+
+def test_latent_decode_row_equals_last_prefill_row():
+    """A decode call (one query at position T-1) equals the last query row of the prefill call
+    over the same cache and the same index list, sinks and gate included."""
+    rng = np.random.default_rng(13)
+    B, S, T, H, D, dv, K = 2, 7, 7, 4, 8, 6, 5
+    q = rng.standard_normal((B, S, H, D))
+    kv = rng.standard_normal((B, T, D))
+    idx = np.stack([np.stack([np.sort(rng.choice(s + 1, size=min(K, s + 1), replace=False))
+                              .tolist() + [-1] * (K - min(K, s + 1)) for s in range(S)])
+                    for _ in range(B)])
+    g = rng.standard_normal((B, S, H))
+    sink = rng.standard_normal((2, D))
+    full = O.sparse_attention_latent(q, kv, idx, dv, gate=g, gate_mode="sigmoid", sink_kv=sink)
+    last = O.sparse_attention_latent(q[:, -1:], kv, idx[:, -1:], dv, gate=g[:, -1:],
+                                     gate_mode="sigmoid", sink_kv=sink)
+    np.testing.assert_allclose(last[:, 0], full[:, -1], rtol=0, atol=1e-13)
