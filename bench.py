@@ -175,7 +175,7 @@ class Workload:
 
     def __init__(self, name, device, seed_offset=0, S=None, T=None, B=None, indexer="per_head",
                  index_dtype="as_dtype", nsink=0, hadamard=False, attn_form="expanded",
-                 latent_heads=128):
+                 latent_heads=128, score_rows=0):
         import dataclasses
 
         import sparse_attention_15_b200 as dsa
@@ -237,6 +237,13 @@ class Workload:
                                       self.out, None, self.idx,
                                       indexer, self.sink_k, self.sink_v, attn_form, self.dv)
         self.ws_bytes = dsa.dsa_forward_workspace_bytes(self.args)
+        self.score_rows = 0
+        if score_rows and cfg.S > score_rows:
+            # a score buffer of `score_rows` rows: dsa_forward then runs the indexer and the
+            # top-k block by block, and a block's scores stay in L2 between the two
+            small = dsa.dsa_forward_workspace_bytes(self.args, minimum=True)
+            self.ws_bytes = small + (score_rows - 1) * cfg.T * 4
+            self.score_rows = score_rows
         self.ws = torch.empty(max(self.ws_bytes, 16), dtype=torch.uint8, device=device)
         dt = dsa.DTYPE[x["q"].dtype]
         if latent:
@@ -571,6 +578,9 @@ def main():
                          "over a shared 512+64 latent cache (MQA form)")
     ap.add_argument("--latent-heads", type=int, default=128,
                     help="query heads of the latent form (<= 128)")
+    ap.add_argument("--score-rows", type=int, default=0,
+                    help="score buffer of this many query rows (indexer and top-k run block "
+                         "by block, the scores staying in L2); 0 = the whole matrix")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world, rank, local = dist_setup(args)
@@ -596,7 +606,8 @@ def main():
 
     wl = Workload(args.config, dev, seed_offset=rank, S=args.S, T=args.T, B=args.B,
                   indexer=args.indexer, index_dtype=args.index_dtype, nsink=args.sinks,
-                  hadamard=args.hadamard, attn_form=args.attn, latent_heads=args.latent_heads)
+                  hadamard=args.hadamard, attn_form=args.attn, latent_heads=args.latent_heads,
+                  score_rows=args.score_rows)
     cfg = wl.cfg
     nst = len(wl.stages)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
@@ -664,6 +675,11 @@ def main():
                          "achieved": round(ach, 2), "peak": peak, "unit": unit,
                          "frac": round(ach / peak, 4),
                          "share": round(float(stage_ms[j]) / float(stage_ms.sum()), 4)}
+    if wl.score_rows:
+        # row blocks interleave the indexer and the top-k: the first event pair spans both
+        kernels["indexer_and_topk"] = dict(kernels.pop("indexer"), bound="mixed",
+                                           achieved=None, frac=None)
+        kernels.pop("topk")
     dom = max(kernels, key=lambda k: kernels[k]["ms"])
     attn_k = {"masked_tile": "masked_attn", "latent": "latent_attn"}.get(wl.algo, "gather_attn")
     kname = {"indexer": "index_scores", "topk": "topk", "attention": attn_k}.get(dom, "masked_attn")
@@ -743,6 +759,7 @@ def main():
             "config": dict(workload_config(cfg, wl.B), indexer_form=wl.indexer,
                            indexer_dtype=wl.index_dtype, sinks=wl.nsink,
                            hadamard=wl.hadamard, attention_form=wl.attn_form,
+                           score_block_rows=wl.score_rows or None,
                            **({"heads": wl.H, "qk_dim": "512+64 (latent, shared by all heads)",
                                "v_dim": 512} if wl.attn_form == "latent" else {})),
             "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
