@@ -1,7 +1,9 @@
 """Build libdsa.so (all CUDA sources, sm_100a) in-tree with nvcc.
 
-The library links the CUDA runtime statically and reaches the driver API (tensor-map
-encoding) through cudaGetDriverEntryPoint, so it loads on a machine without a GPU driver.
+Every source is compiled to relocatable device code in parallel (objects under `_build/`
+next to this file), then one nvcc call device-links them into the shared library.  The
+library links the CUDA runtime statically and reaches the driver API (tensor-map encoding)
+through cudaGetDriverEntryPoint, so it loads on a machine without a GPU driver.
 """
 from __future__ import annotations
 
@@ -9,29 +11,33 @@ import glob
 import os
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libdsa.so")
+OBJDIR = os.path.join(HERE, "_build")
 
-NVCC_FLAGS = [
-    "-gencode", "arch=compute_100a,code=sm_100a",
-    "-O3", "-lineinfo", "-std=c++17",
-    "-Xcompiler", "-fPIC", "-shared", "-cudart", "static",
-    "--expt-relaxed-constexpr", "-rdc=true",
-]
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+COMPILE_FLAGS = [*ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
+                 "--expt-relaxed-constexpr", "-rdc=true"]
+LINK_FLAGS = [*ARCH, "-Xcompiler", "-fPIC", "-shared", "-cudart", "static", "-rdc=true"]
 
 
 def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _inputs():
-    return sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + \
+def _headers():
+    return sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + \
         sorted(glob.glob(os.path.join(CSRC, "*.h"))) + \
         sorted(glob.glob(os.path.join(INCLUDE, "*.h"))) + [os.path.abspath(__file__)]
+
+
+def _inputs():
+    return sources() + _headers()
 
 
 def is_stale() -> bool:
@@ -48,17 +54,38 @@ def nvcc() -> str:
     return "nvcc"
 
 
-def build(verbose: bool = False, extra_flags=None) -> str:
-    """Compile every CUDA source into libdsa.so next to this file; returns its path."""
-    tmp = LIB + ".tmp"
-    cmd = [nvcc(), *NVCC_FLAGS, *(extra_flags or []), "-I", INCLUDE, "-o", tmp, *sources()]
-    if verbose:
-        print(" ".join(cmd), file=sys.stderr)
+def _run(cmd):
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
-        raise RuntimeError(f"nvcc failed ({r.returncode}):\n{r.stdout}\n{r.stderr}")
-    if verbose and r.stderr:
-        print(r.stderr, file=sys.stderr)
+        raise RuntimeError(f"nvcc failed ({r.returncode}): {' '.join(cmd)}\n{r.stdout}\n{r.stderr}")
+    return r.stderr
+
+
+def build(verbose: bool = False, extra_flags=None) -> str:
+    """Compile every CUDA source into libdsa.so next to this file; returns its path."""
+    os.makedirs(OBJDIR, exist_ok=True)
+    hdr_time = max(os.path.getmtime(p) for p in _headers())
+    jobs = []
+    for src in sources():
+        obj = os.path.join(OBJDIR, os.path.basename(src)[:-3] + ".o")
+        fresh = (not extra_flags and os.path.exists(obj) and
+                 os.path.getmtime(obj) > max(os.path.getmtime(src), hdr_time))
+        if not fresh:
+            jobs.append([nvcc(), *COMPILE_FLAGS, *(extra_flags or []), "-I", INCLUDE, "-dc",
+                         "-o", obj, src])
+    objs = [os.path.join(OBJDIR, os.path.basename(s)[:-3] + ".o") for s in sources()]
+    if verbose:
+        for j in jobs:
+            print(" ".join(j), file=sys.stderr)
+    with ThreadPoolExecutor(max_workers=max(1, min(len(jobs), os.cpu_count() or 4))) as ex:
+        for err in ex.map(_run, jobs):
+            if verbose and err:
+                print(err, file=sys.stderr)
+    tmp = LIB + ".tmp"
+    link = [nvcc(), *LINK_FLAGS, "-o", tmp, *objs]
+    if verbose:
+        print(" ".join(link), file=sys.stderr)
+    _run(link)
     os.replace(tmp, LIB)
     return LIB
 
