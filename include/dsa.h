@@ -351,8 +351,11 @@ dsa_status dsa_window_attn_sinks(dsa_dtype dtype, const void* q, const void* k, 
  * device memory, which every GPU that loads the library holds until the process exits.
  *
  *   - Nothing is allocated or freed by any call (no cudaMalloc, no allocating library call).
- *   - The first call on a device, made with that device current, looks up the array's device
- *     address (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - The first call in a CUDA context (normally the current device's primary context)
+ *     looks up the array's device address there (cudaGetSymbolAddress) and keeps it for that
+ *     context; make that first call before any stream capture.  A later context on the same
+ *     device (after cudaDeviceReset, or a driver-API context made current by the caller) is
+ *     a new context: its first call looks the address up again, so no stale address is used.
  *   - Shapes whose partial results need more than the fixed size are rejected with
  *     DSA_ERR_UNSUPPORTED before anything is launched (the message states both sizes); use
  *     dsa_sparse_attn with a workspace for those.  The decode shape of 64 rows x 32 heads x
@@ -381,6 +384,18 @@ const char* dsa_last_error(void);
 dsa_status dsa_device_status(int reset);
 /* Library version, e.g. "dsa-b200 0.1.0 sm_100a". */
 const char* dsa_version(void);
+
+/* Testing aid for the failure detection (the pages have no counterpart: they describe no
+ * failure handling).  Arms a one-shot fault: the next gather-attention launch in this process
+ * (dsa_sparse_attn / dsa_sparse_attn_sinks with the gather algorithm, dsa_sparse_attn_noalloc,
+ * or a dsa_forward / dsa_window_attn call that takes the gather kernel) makes its first CTA
+ * fill none of its shared-memory key slots.  That CTA's consumer warps then wait on a slot
+ * that never fills until their bounded wait (about 2 s) runs out; the wait records
+ * DSA_ERR_TIMEOUT in the device status word, every later wait of that launch gives up at
+ * once, and the launch ends with undefined output.  Nothing faults or hangs: no copy is left
+ * in flight, and dsa_device_status(1) reports DSA_ERR_TIMEOUT and clears the word, after which
+ * the device is usable as before.  Returns DSA_OK. */
+dsa_status dsa_test_arm_wait_timeout(void);
 
 #ifdef __cplusplus
 } /* extern "C" */

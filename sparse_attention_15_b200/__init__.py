@@ -20,7 +20,7 @@ __all__ = [
     "dsa_sparse_attn_algo", "dsa_forward",
     "dsa_forward_workspace_bytes",
     "dsa_window_attn", "dsa_sparse_attn_noalloc", "dsa_device_status", "dsa_version",
-    "LIB_PATH",
+    "dsa_test_arm_wait_timeout", "LIB_PATH",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdsa.so")
@@ -95,6 +95,7 @@ _SIGNATURES = {
     "dsa_last_error": (ctypes.c_char_p, []),
     "dsa_device_status": (_I, [_I]),
     "dsa_version": (ctypes.c_char_p, []),
+    "dsa_test_arm_wait_timeout": (_I, []),
 }
 
 
@@ -152,6 +153,12 @@ def dsa_device_status(reset: bool = True) -> int:
     st = lib().dsa_device_status(1 if reset else 0)
     _check(st)
     return st
+
+
+def dsa_test_arm_wait_timeout() -> None:
+    """Testing aid: the next gather-attention launch runs one bounded wait out on purpose
+    (it records DSA_ERR_TIMEOUT; its output is undefined).  One-shot."""
+    _check(lib().dsa_test_arm_wait_timeout())
 
 
 def dsa_index_scores(q_idx, k_idx, w, scale, relu="none", scores=None, stream=None):

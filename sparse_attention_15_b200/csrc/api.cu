@@ -7,6 +7,7 @@
 #include <string>
 
 #include "../../include/dsa.h"
+#include "checks.h"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -128,32 +129,6 @@ dsa_status check_sinks(const void* sink_k, const void* sink_v, int nsink) {
   return DSA_OK;
 }
 
-dsa_status check_attn_common(dsa_dtype dtype, const void* q, const void* k, const void* v,
-                             const void* gate, dsa_gate_mode gm, float sm_scale, int B, int S,
-                             int T, int H, int HKV, int DQK, int DV, const void* out) {
-  REQUIRE(dtype == DSA_F32 || dtype == DSA_BF16, DSA_ERR_INVALID_ARG, "unknown dtype %d",
-          (int)dtype);
-  REQUIRE(q && k && v && out, DSA_ERR_INVALID_ARG, "null pointer argument");
-  REQUIRE(B > 0 && S > 0 && T > 0 && H > 0 && HKV > 0 && DQK > 0 && DV > 0,
-          DSA_ERR_INVALID_ARG, "sizes must be positive");
-  REQUIRE(T >= S, DSA_ERR_INVALID_ARG, "T (%d) must be >= S (%d)", T, S);
-  REQUIRE(H % HKV == 0, DSA_ERR_INVALID_ARG, "H=%d not a multiple of HKV=%d", H, HKV);
-  REQUIRE(gm >= DSA_GATE_OFF && gm <= DSA_GATE_SILU, DSA_ERR_INVALID_ARG,
-          "unknown gate mode %d (only sigmoid and silu exist)", (int)gm);
-  REQUIRE((gm == DSA_GATE_OFF) == (gate == nullptr), DSA_ERR_INVALID_ARG,
-          "gate pointer must be given exactly when the gate is on");
-  REQUIRE(!isnan(sm_scale) && !isinf(sm_scale), DSA_ERR_INVALID_ARG, "sm_scale not finite");
-  REQUIRE(DQK <= 256 && DV <= 256 && dim_ok(dtype, DQK) && dim_ok(dtype, DV),
-          DSA_ERR_UNSUPPORTED, "DQK=%d / DV=%d must be <= 256 and multiples of %d", DQK, DV,
-          dtype == DSA_F32 ? 4 : 8);
-  REQUIRE(H <= 64, DSA_ERR_UNSUPPORTED, "H=%d > 64", H);
-  REQUIRE((HKV * DQK * esize(dtype)) % 16 == 0 && (HKV * DV * esize(dtype)) % 16 == 0,
-          DSA_ERR_UNSUPPORTED, "K/V rows must be multiples of 16 bytes");
-  REQUIRE(aligned16(q) && aligned16(k) && aligned16(v) && aligned16(out) &&
-              (gate == nullptr || aligned16(gate)),
-          DSA_ERR_UNSUPPORTED, "pointers must be 16-byte aligned");
-  return DSA_OK;
-}
 
 float default_scale(float sm_scale, int DQK) {
   return sm_scale > 0.f ? sm_scale : 1.0f / sqrtf((float)DQK);
@@ -198,6 +173,40 @@ int choose_algo(dsa_attn_algo req, dsa_dtype dt, int B, int S, int T, int H, int
 namespace dsa {
 // Records the thread-local text dsa_last_error() returns (for entry points in other files).
 void set_last_error(const char* msg) { g_last_error = msg ? msg : ""; }
+
+// Argument checks shared by the attention entry points (declared in checks.h).
+dsa_status check_attn_common(dsa_dtype dtype, const void* q, const void* k, const void* v,
+                             const void* gate, dsa_gate_mode gm, float sm_scale, int B, int S,
+                             int T, int H, int HKV, int DQK, int DV, const void* out) {
+  REQUIRE(dtype == DSA_F32 || dtype == DSA_BF16, DSA_ERR_INVALID_ARG, "unknown dtype %d",
+          (int)dtype);
+  REQUIRE(q && k && v && out, DSA_ERR_INVALID_ARG, "null pointer argument");
+  REQUIRE(B > 0 && S > 0 && T > 0 && H > 0 && HKV > 0 && DQK > 0 && DV > 0,
+          DSA_ERR_INVALID_ARG, "sizes must be positive");
+  REQUIRE(T >= S, DSA_ERR_INVALID_ARG, "T (%d) must be >= S (%d)", T, S);
+  REQUIRE(H % HKV == 0, DSA_ERR_INVALID_ARG, "H=%d not a multiple of HKV=%d", H, HKV);
+  REQUIRE(gm >= DSA_GATE_OFF && gm <= DSA_GATE_SILU, DSA_ERR_INVALID_ARG,
+          "unknown gate mode %d (only sigmoid and silu exist)", (int)gm);
+  REQUIRE((gm == DSA_GATE_OFF) == (gate == nullptr), DSA_ERR_INVALID_ARG,
+          "gate pointer must be given exactly when the gate is on");
+  REQUIRE(!isnan(sm_scale) && !isinf(sm_scale), DSA_ERR_INVALID_ARG, "sm_scale not finite");
+  REQUIRE(DQK <= 256 && DV <= 256 && dim_ok(dtype, DQK) && dim_ok(dtype, DV),
+          DSA_ERR_UNSUPPORTED, "DQK=%d / DV=%d must be <= 256 and multiples of %d", DQK, DV,
+          dtype == DSA_F32 ? 4 : 8);
+  REQUIRE(H <= 64, DSA_ERR_UNSUPPORTED, "H=%d > 64", H);
+  REQUIRE((HKV * DQK * esize(dtype)) % 16 == 0 && (HKV * DV * esize(dtype)) % 16 == 0,
+          DSA_ERR_UNSUPPORTED, "K/V rows must be multiples of 16 bytes");
+  REQUIRE(aligned16(q) && aligned16(k) && aligned16(v) && aligned16(out) &&
+              (gate == nullptr || aligned16(gate)),
+          DSA_ERR_UNSUPPORTED, "pointers must be 16-byte aligned");
+  return DSA_OK;
+}
+
+dsa_status check_idx_args(const int32_t* idx, int K) {
+  REQUIRE(idx != nullptr && K > 0, DSA_ERR_INVALID_ARG, "idx must be given with K > 0");
+  REQUIRE(aligned16(idx), DSA_ERR_UNSUPPORTED, "idx must be 16-byte aligned");
+  return DSA_OK;
+}
 }  // namespace dsa
 
 extern "C" {
@@ -216,7 +225,12 @@ const char* dsa_status_string(dsa_status s) {
 
 const char* dsa_last_error(void) { return g_last_error.c_str(); }
 
-const char* dsa_version(void) { return "dsa-b200 0.1.0 sm_100a"; }
+const char* dsa_version(void) { return "dsa-b200 0.2.0 sm_100a"; }
+
+dsa_status dsa_test_arm_wait_timeout(void) {
+  dsa::arm_gather_skip_copy();
+  return DSA_OK;
+}
 
 dsa_status dsa_device_status(int reset) {
   unsigned v = 0;
@@ -360,11 +374,10 @@ static dsa_status sparse_attn_impl(dsa_dtype dtype, const void* q, const void* k
                                    dsa_gate_mode gate_mode, float sm_scale, int B, int S, int T,
                                    int H, int DQK, int DV, dsa_attn_algo algo, void* out,
                                    void* ws, size_t ws_bytes, dsa_stream_t stream) {
-  dsa_status st = check_attn_common(dtype, q, k, v, gate, gate_mode, sm_scale, B, S, T, H, H,
-                                    DQK, DV, out);
+  dsa_status st = dsa::check_attn_common(dtype, q, k, v, gate, gate_mode, sm_scale, B, S, T, H,
+                                         H, DQK, DV, out);
   if (st != DSA_OK) return st;
-  REQUIRE(idx != nullptr && K > 0, DSA_ERR_INVALID_ARG, "idx must be given with K > 0");
-  REQUIRE(aligned16(idx), DSA_ERR_UNSUPPORTED, "idx must be 16-byte aligned");
+  if ((st = dsa::check_idx_args(idx, K)) != DSA_OK) return st;
   REQUIRE(algo >= DSA_ATTN_AUTO && algo <= DSA_ATTN_MASKED_TILE, DSA_ERR_INVALID_ARG,
           "unknown attention algorithm %d", (int)algo);
   if ((st = check_sinks(sink_k, sink_v, nsink)) != DSA_OK) return st;
@@ -445,7 +458,7 @@ static dsa_status window_attn_impl(dsa_dtype dtype, const void* q, const void* k
                                    const void* gate, dsa_gate_mode gate_mode, float sm_scale,
                                    int window, int B, int S, int T, int H, int HKV, int DQK,
                                    int DV, dsa_attn_algo algo, void* out, dsa_stream_t stream) {
-  dsa_status st = check_attn_common(dtype, q, k, v, gate, gate_mode, sm_scale, B, S, T, H, HKV,
+  dsa_status st = dsa::check_attn_common(dtype, q, k, v, gate, gate_mode, sm_scale, B, S, T, H, HKV,
                                     DQK, DV, out);
   if (st != DSA_OK) return st;
   REQUIRE(window > 0, DSA_ERR_INVALID_ARG, "window must be positive");
@@ -511,7 +524,7 @@ static dsa_status check_forward(const dsa_forward_args* a) {
   const bool latent = a->attn_form == DSA_ATTN_LATENT;
   st = latent ? check_latent(a->dtype, a->q, a->k, a->sink_k, a->nsink, a->gate, a->gate_mode,
                              a->sm_scale, a->B, a->S, a->T, a->H, a->DQK, a->DV, a->out)
-              : check_attn_common(a->dtype, a->q, a->k, a->v, a->gate, a->gate_mode,
+              : dsa::check_attn_common(a->dtype, a->q, a->k, a->v, a->gate, a->gate_mode,
                                   a->sm_scale, a->B, a->S, a->T, a->H, a->H, a->DQK, a->DV,
                                   a->out);
   if (st != DSA_OK) return st;

@@ -19,12 +19,19 @@
 //
 // Long index lists with few query rows (decode) are split over several CTAs; each writes
 // an unnormalised partial (o, m, l) and a second kernel merges them in a fixed order.
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 
 namespace dsa {
 
 namespace {
+
+// Testing aid (dsa_test_arm_wait_timeout): when armed, the next gather launch's first CTA
+// fills none of its slots, so that CTA's consumers wait on a slot that never fills until
+// their bounded wait runs out and records the timeout.  One-shot.
+std::atomic<int> g_arm_skip_copy{0};
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLazyRescale = 8.0f;  // raise the running max only past 2^8 (log2 units)
@@ -86,6 +93,7 @@ struct GatherArgs {
   const void* sink_k;       // [nsink, HKV, DQK] attention sinks (PAS) or NULL
   const void* sink_v;       // [nsink, HKV, DV]
   int nsink;
+  int skip_first_copy;      // testing aid: CTA 0 fills no slot
 };
 
 // Entry jj of a query's key list: with SINKS the nsink sinks come first (encoded as
@@ -141,10 +149,16 @@ __global__ void __launch_bounds__(544, HPW <= 2 ? 2 : 1) gather_attn_kernel(cons
       keys[j] = key_at<SINKS>(a, idx_row, j0 + j, spos);
     __syncwarp();
     if (lane == 0) {
+      const bool skip_first = a.skip_first_copy != 0 && blockIdx.x == 0;
+      int issued = 0;  // keys whose slot fill was issued
       for (int j = 0; j < nkeys; ++j) {
         const int slot = j % nslots;
         const int round = j / nslots;
         if (round > 0 && !mbar_wait(&empty[slot], (round - 1) & 1)) break;
+        // testing aid: the first slot never fills and nothing more is issued, so this CTA
+        // has no copy in flight while its consumers wait for that slot until they give up
+        if (skip_first) break;
+        issued = j + 1;
         const int t = keys[j];
         slot_key[slot] = t;
         if (SINKS ? t != -1 : t >= 0) {
@@ -162,6 +176,13 @@ __global__ void __launch_bounds__(544, HPW <= 2 ? 2 : 1) gather_attn_kernel(cons
         } else {
           mbar_arrive(&full[slot]);
         }
+      }
+      // Copies still in flight must land before the CTA exits, also when the consumers gave
+      // up early (a recorded timeout): wait, bounded, for the last fill of every slot that
+      // had a copy issued.
+      for (int j = issued - 1; j >= 0 && j >= issued - nslots; --j) {
+        const int t = keys[j];
+        if (SINKS ? t != -1 : t >= 0) drain_wait(&full[j % nslots], (j / nslots) & 1);
       }
     }
     return;
@@ -206,7 +227,7 @@ __global__ void __launch_bounds__(544, HPW <= 2 ? 2 : 1) gather_attn_kernel(cons
   int slot = 0;
   uint32_t phase = 0;
   for (int j = 0; j < nkeys && ok; ++j) {
-    ok = mbar_wait(&full[slot], phase);
+    ok = warp_wait(&full[slot], phase);  // warp-uniform: the shuffles below need all lanes
     if (ok && (SINKS ? slot_key[slot] != -1 : slot_key[slot] >= 0)) {
       const T* ks = reinterpret_cast<const T*>(slots + (size_t)slot * a.slot_bytes);
       const T* vs = reinterpret_cast<const T*>(slots + (size_t)slot * a.slot_bytes + a.k_bytes);
@@ -417,6 +438,8 @@ cudaError_t launch_hpw(GatherArgs a, int hpw, size_t smem, unsigned grid, int ro
 
 }  // namespace
 
+void arm_gather_skip_copy() { g_arm_skip_copy.store(1); }
+
 cudaError_t launch_split_combine(int dtype, const float* part_o, const float* part_ml, int rows,
                                  int nsplit, int H, int DV, const void* gate, int gate_mode,
                                  void* out, cudaStream_t st) {
@@ -453,6 +476,7 @@ cudaError_t launch_gather_attn(const AttnProblem& p, void* ws, size_t ws_bytes,
   const int rows = p.B * p.S;
   if (rows == 0) return cudaSuccess;
   a.sink_k = p.sink_k; a.sink_v = p.sink_v; a.nsink = p.sink_k ? p.nsink : 0;
+  a.skip_first_copy = g_arm_skip_copy.exchange(0);
   const int nkeys = a.nsink + (p.idx ? p.K : p.window);
   split_policy(rows, nkeys, &a.nsplit, &a.keys_per_split, p.idx != nullptr);
   a.key_list_bytes = ((uint32_t)a.keys_per_split * 4u + 127u) & ~127u;

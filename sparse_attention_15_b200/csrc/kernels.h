@@ -78,6 +78,9 @@ struct AttnProblem {
   int nsink = 0;
 };
 size_t gather_attn_workspace_bytes(int B, int S, int H, int DV, int K, int nsink = 0);
+// Testing aid: the next launch_gather_attn makes its first CTA fill none of its key slots,
+// so that CTA's bounded waits run out and record the timeout (one-shot).
+void arm_gather_skip_copy();
 cudaError_t launch_gather_attn(const AttnProblem& p, void* ws, size_t ws_bytes,
                                cudaStream_t st);
 

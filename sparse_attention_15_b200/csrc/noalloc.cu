@@ -10,14 +10,19 @@
 // inputs and outputs only and nothing is allocated on any call.
 //
 // The array is a file-scope __device__ variable of kNoAllocScratchBytes.  In host code its
-// name is only a host-side stand-in, so its device address is looked up once per device with
-// cudaGetSymbolAddress (on the first call made with that device current) and passed to the
-// kernels.  Every GPU that loads the library holds the array until the process exits.
+// name is only a host-side stand-in, so its device address is looked up with
+// cudaGetSymbolAddress once per CUDA context (on the first call made in that context, the
+// current device's) and passed to the kernels.  The cache is keyed by the context's
+// process-unique ID, so a context created later on the same device -- after
+// cudaDeviceReset, or a driver-API context made current by the caller -- gets a fresh
+// lookup instead of a stale address.  Every GPU that loads the library holds the array
+// until the process exits.
 #include <stdio.h>
 
 #include <mutex>
 
 #include "../../include/dsa.h"
+#include "checks.h"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -26,28 +31,70 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = 16u << 20;  // 16 MiB per device
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-constexpr int kMaxDevices = 64;
-void* g_scratch_addr[kMaxDevices] = {};
+// (context ID, device address of g_noalloc_scratch in that context), most recent first.
+struct ScratchEntry {
+  unsigned long long ctx_id;
+  void* addr;
+};
+constexpr int kMaxContexts = 16;
+ScratchEntry g_scratch_cache[kMaxContexts] = {};
+int g_scratch_entries = 0;
 std::mutex g_scratch_mu;
 
-// Device address of g_noalloc_scratch on the current device (looked up once per device).
-cudaError_t scratch_address(void** out) {
-  int dev = -1;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// The current context's process-unique ID; false if the driver does not provide it.
+bool current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
-  return cudaSuccess;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
 }
 
-bool is_aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+// Device address of g_noalloc_scratch in the current context.  When no context is current
+// yet, cudaGetSymbolAddress makes the current device's primary context current, and the
+// entry is keyed by that context.
+cudaError_t scratch_address(void** out) {
+  cudaError_t e;
+  unsigned long long id = 0;
+  const bool have_id = current_context_id(&id);
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (have_id) {
+    for (int i = 0; i < g_scratch_entries; ++i)
+      if (g_scratch_cache[i].ctx_id == id) {
+        *out = g_scratch_cache[i].addr;
+        return cudaSuccess;
+      }
+  }
+  void* p = nullptr;
+  e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess) return e;
+  // the lookup may have made the primary context current: key the entry by that context
+  if (!have_id && !current_context_id(&id)) {
+    *out = p;  // no context IDs from this driver: look the address up on every call
+    return cudaSuccess;
+  }
+  const int n = g_scratch_entries < kMaxContexts ? g_scratch_entries + 1 : kMaxContexts;
+  for (int i = n - 1; i > 0; --i) g_scratch_cache[i] = g_scratch_cache[i - 1];
+  g_scratch_cache[0] = ScratchEntry{id, p};
+  g_scratch_entries = n;
+  *out = p;
+  return cudaSuccess;
+}
 
 dsa_status reject(dsa_status st, const char* msg) {
   dsa::set_last_error(msg);
@@ -64,25 +111,11 @@ dsa_status dsa_sparse_attn_noalloc(dsa_dtype dtype, const void* q, const void* k
                                    const int32_t* idx, int K, const void* gate,
                                    dsa_gate_mode gate_mode, float sm_scale, int B, int S, int T,
                                    int H, int DQK, int DV, void* out, dsa_stream_t stream) {
-  if (dtype != DSA_F32 && dtype != DSA_BF16)
-    return reject(DSA_ERR_INVALID_ARG, "dsa_sparse_attn_noalloc: unknown dtype");
-  if (!q || !k || !v || !idx || !out)
-    return reject(DSA_ERR_INVALID_ARG, "dsa_sparse_attn_noalloc: null pointer argument");
-  if (B <= 0 || S <= 0 || T <= 0 || H <= 0 || DQK <= 0 || DV <= 0 || K <= 0 || T < S)
-    return reject(DSA_ERR_INVALID_ARG, "dsa_sparse_attn_noalloc: invalid sizes");
-  if (gate_mode < DSA_GATE_OFF || gate_mode > DSA_GATE_SILU ||
-      (gate_mode == DSA_GATE_OFF) != (gate == nullptr))
-    return reject(DSA_ERR_INVALID_ARG, "dsa_sparse_attn_noalloc: invalid gate arguments");
-  if (sm_scale != sm_scale || sm_scale > 3.0e38f || sm_scale < -3.0e38f)
-    return reject(DSA_ERR_INVALID_ARG, "dsa_sparse_attn_noalloc: sm_scale not finite");
-  const int vec = dtype == DSA_F32 ? 4 : 8;
-  const size_t es = dtype == DSA_F32 ? 4 : 2;
-  if (DQK > 256 || DV > 256 || DQK % vec || DV % vec || H > 64 || (H * DQK * es) % 16 ||
-      (H * DV * es) % 16)
-    return reject(DSA_ERR_UNSUPPORTED, "dsa_sparse_attn_noalloc: unsupported head shape");
-  if (!is_aligned16(q) || !is_aligned16(k) || !is_aligned16(v) || !is_aligned16(idx) ||
-      !is_aligned16(out) || (gate && !is_aligned16(gate)))
-    return reject(DSA_ERR_UNSUPPORTED, "dsa_sparse_attn_noalloc: pointers must be 16-byte aligned");
+  // the same argument checks as dsa_sparse_attn (same statuses and messages)
+  dsa_status st = dsa::check_attn_common(dtype, q, k, v, gate, gate_mode, sm_scale, B, S, T, H,
+                                         H, DQK, DV, out);
+  if (st != DSA_OK) return st;
+  if ((st = dsa::check_idx_args(idx, K)) != DSA_OK) return st;
   const size_t need = dsa::gather_attn_workspace_bytes(B, S, H, DV, K);
   if (need > kNoAllocScratchBytes) {
     char msg[256];
