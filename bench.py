@@ -275,10 +275,13 @@ class Workload:
         self.stages = (["hadamard"] if self.hadamard else []) + \
             ["indexer", "topk", "attention"] + [f"swa{i + 1}" for i in range(len(self.swa))]
         # our kernels per step: indexer (+ the query collapse), top-k, attention (+ combine for
-        # split gathers), SWA
+        # split gathers), SWA.  The fused indexer launches six: the sampled indexer, the
+        # thresholds, the filtering indexer, the candidate select and the two fallback
+        # kernels (which return at once when the filter held)
         self.launches_per_step = 3 + \
             (1 if self.algo in ("gather", "latent") and split_ws > 0 else 0) + \
-            (1 if indexer == "collapsed" else 0) + (2 if self.hadamard else 0) + len(self.swa)
+            (1 if indexer == "collapsed" else 0) + (4 if indexer == "fused" else 0) + \
+            (2 if self.hadamard else 0) + len(self.swa)
 
     def _forward(self, x, events=None):
         """The DSA layer through the public whole-step call."""
@@ -590,8 +593,9 @@ def main():
     ap.add_argument("--S", type=int, default=None, help="reduced query count (profiling cases)")
     ap.add_argument("--T", type=int, default=None, help="reduced key count (profiling cases)")
     ap.add_argument("--B", type=int, default=None, help="reduced batch (profiling cases)")
-    ap.add_argument("--indexer", default="per_head", choices=["per_head", "collapsed"],
-                    help="indexer form (the pages' per-head work by default)")
+    ap.add_argument("--indexer", default="per_head", choices=["per_head", "collapsed", "fused"],
+                    help="indexer form: the pages' per-head work (default), head-collapsed, or "
+                         "per-head with the top-k candidates filtered inside the indexer")
     ap.add_argument("--index-dtype", default="as_dtype", choices=["as_dtype", "e4m3"],
                     help="indexer input type (the workload's dtype by default)")
     ap.add_argument("--sinks", type=int, default=0,
@@ -711,9 +715,23 @@ def main():
         kernels["indexer_and_topk"] = dict(kernels.pop("indexer"), bound="mixed",
                                            achieved=None, frac=None)
         kernels.pop("topk")
+    elif wl.indexer == "fused":
+        # one fused stage: the sampled pass, the filtering indexer and the candidate select
+        # (+ the fallback check), held to the per-head indexer's flops over both event spans
+        ki, kt = kernels.pop("indexer"), kernels.pop("topk")
+        ms = ki["ms"] + kt["ms"]
+        ach = ki["achieved"] * ki["ms"] / ms
+        kernels["indexer_and_topk"] = dict(
+            ki, ms=round(ms, 5), achieved=round(ach, 2), frac=round(ach / ki["peak"], 4),
+            share=round(ki["share"] + kt["share"], 4),
+            split_ms={"sample_and_filter": ki["ms"], "select": kt["ms"]})
+        if "frac_of_sustained" in ki:
+            kernels["indexer_and_topk"]["frac_of_sustained"] = round(
+                ki["frac_of_sustained"] * ki["ms"] / ms, 4)
     dom = max(kernels, key=lambda k: kernels[k]["ms"])
     attn_k = {"masked_tile": "masked_attn", "latent": "latent_attn"}.get(wl.algo, "gather_attn")
-    kname = {"indexer": "index_scores", "topk": "topk", "attention": attn_k}.get(dom, "masked_attn")
+    kname = {"indexer": "index_scores", "topk": "topk", "attention": attn_k,
+             "indexer_and_topk": "index_scores"}.get(dom, "masked_attn")
     tr = NCU_TRAFFIC.get((kname, cfg.name))
     srcfile = {"index_scores": "indexer_tc.cu", "topk": "topk.cu", "gather_attn": "gather_attn.cu",
                "masked_attn": "attn_tc.cu", "latent_attn": "latent_attn.cu"}[kname]

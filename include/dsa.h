@@ -77,8 +77,14 @@ typedef enum { DSA_RELU_NONE = 0, DSA_RELU_POST_SUM = 1, DSA_RELU_PER_HEAD = 2 }
  * (token, head), evaluated in float32; any other mode is rejected (the page's ValueError). */
 typedef enum { DSA_GATE_OFF = 0, DSA_GATE_SIGMOID = 1, DSA_GATE_SILU = 2 } dsa_gate_mode;
 
-/* How dsa_forward computes the indexer scores (section 1 or section 1b). */
-typedef enum { DSA_INDEXER_PER_HEAD = 0, DSA_INDEXER_COLLAPSED = 1 } dsa_indexer_mode;
+/* How dsa_forward computes the indexer scores and the top-k: per-head scores written out and
+ * selected (sections 1 and 2), the head-collapsed scores (section 1b), or the per-head
+ * scores filtered inside the indexer and selected from the candidates (section 2b). */
+typedef enum {
+  DSA_INDEXER_PER_HEAD = 0,
+  DSA_INDEXER_COLLAPSED = 1,
+  DSA_INDEXER_FUSED = 2
+} dsa_indexer_mode;
 
 /* Form of the attention cache dsa_forward attends over: per-head expanded K/V (section 3)
  * or one latent row per token shared by all heads (section 3c). */
@@ -166,6 +172,36 @@ dsa_status dsa_hadamard_rotate(dsa_dtype dtype, const void* x, long long rows, i
  * --------------------------------------------------------------------------------- */
 dsa_status dsa_topk(const float* scores, int B, int S, int T, int K, int32_t* idx,
                     dsa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * 2b. Fused indexer -> top-k.  The same selection as dsa_index_scores followed by dsa_topk
+ *    ([AXK2] SGA scores, [PANGU] §3.3 a fixed K per query), without writing the S x T
+ *    score matrix: the indexer keeps, per query row, only the keys whose score reaches a
+ *    threshold tau, and the top-k is selected exactly from those candidates.
+ *
+ *    tau comes from a sampled pass (every kstride-th key tile of the row, kstride =
+ *    max(4, key tiles / 32)): the r-th largest sampled score, r being the sample rank the
+ *    K-th key is expected at plus a six-sigma margin.  Rows with at most 2K + 1024 causal
+ *    keys keep every key.  The result does not depend on the sample: when every row has
+ *    at least K and at most 2K + 1024 candidates, the candidates hold every key of the row's
+ *    top-k (and every key tied with its K-th), so the exact select over them is the top-k;
+ *    otherwise the call runs the full-score indexer and top-k itself (on the device, no
+ *    host synchronisation) and reports that in *fallback_out.  Either way idx is what
+ *    dsa_index_scores + dsa_topk give, bit for bit.
+ *
+ *   dtype bf16; HI in {16, 32}, DI in {64, 128} (the tensor-core indexer), else
+ *   DSA_ERR_UNSUPPORTED.  Other arguments as dsa_index_scores; K as dsa_topk.
+ *   idx          [B,S,K_eff] int32 out, ascending, -1 padded (as dsa_topk)
+ *   ws           device workspace of dsa_index_topk_workspace_bytes(B,S,T,K) bytes, 16-byte
+ *                aligned (the sample, thresholds, candidate lists and the score matrix the
+ *                fallback would need), owned by the caller
+ *   fallback_out optional device int32: 1 if the fallback ran, else 0
+ * --------------------------------------------------------------------------------- */
+size_t dsa_index_topk_workspace_bytes(int B, int S, int T, int K);
+dsa_status dsa_index_topk(dsa_dtype dtype, const void* q_idx, const void* k_idx,
+                          const float* w, float scale, dsa_relu_mode relu, int B, int S, int T,
+                          int HI, int DI, int K, int32_t* idx, void* ws, size_t ws_bytes,
+                          int32_t* fallback_out, dsa_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
  * 3+4. Sparse attention over the selected keys, with the optional headwise gate.
@@ -293,8 +329,12 @@ typedef struct {
   void* const* events;     /* optional: 4 caller-owned cudaEvent_t recorded on the stream
                               before the indexer, after it, after the top-k and after the
                               attention (per-stage timing); NULL for none                */
-  dsa_indexer_mode indexer; /* DSA_INDEXER_PER_HEAD (0, the pages' per-head work) or
-                              DSA_INDEXER_COLLAPSED (the section 1b form)                */
+  dsa_indexer_mode indexer; /* DSA_INDEXER_PER_HEAD (0, the pages' per-head work),
+                              DSA_INDEXER_COLLAPSED (the section 1b form) or
+                              DSA_INDEXER_FUSED (section 2b: per-head scores filtered in
+                              the indexer; bf16 tensor-core indexer shapes; with scores_out
+                              or a workspace below dsa_forward_workspace_bytes it runs as
+                              DSA_INDEXER_PER_HEAD -- the results are the same)          */
   dsa_index_dtype index_dtype; /* DSA_INDEX_AS_DTYPE (0): q_idx / k_idx have `dtype`;
                               DSA_INDEX_E4M3: they are e4m3 (per-head indexer only)      */
   const void* sink_k;      /* optional [nsink,H,DQK] attention sinks (section 3b)        */
@@ -304,6 +344,9 @@ typedef struct {
                               DSA_ATTN_LATENT: k is the latent cache [B,T,DQK] of section
                               3c, v is unused (NULL), sink_k holds [nsink,DQK] latent sink
                               rows, sink_v is unused; attn_algo is ignored                */
+  int32_t* topk_fallback_out; /* optional device int32, DSA_INDEXER_FUSED only: written 1
+                              when the candidate filter did not hold for some row and the
+                              full-score indexer and top-k ran instead, else 0            */
 } dsa_forward_args;
 
 /* Bytes of workspace dsa_forward needs to run without row blocking. */

@@ -15,7 +15,7 @@ import torch
 
 __all__ = [
     "DSAError", "lib", "dsa_index_scores", "dsa_index_scores_collapsed", "dsa_hadamard_rotate",
-    "dsa_topk",
+    "dsa_topk", "dsa_index_topk", "dsa_index_topk_workspace_bytes",
     "dsa_sparse_attn", "dsa_sparse_attn_sinks", "dsa_sparse_attn_workspace_bytes",
     "dsa_sparse_attn_algo", "dsa_forward",
     "dsa_forward_workspace_bytes",
@@ -29,7 +29,7 @@ DTYPE = {torch.float32: 0, torch.bfloat16: 1, torch.float8_e4m3fn: 2}  # e4m3: i
 RELU = {"none": 0, "post_sum": 1, "per_head": 2}
 GATE = {"off": 0, "sigmoid": 1, "silu": 2}
 ATTN_ALGO = {"auto": 0, "gather": 1, "masked_tile": 2}
-INDEXER = {"per_head": 0, "collapsed": 1}
+INDEXER = {"per_head": 0, "collapsed": 1, "fused": 2}
 ATTN_FORM = {"expanded": 0, "latent": 1}
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "CUDA error", 4: "timeout",
           5: "internal"}
@@ -55,6 +55,7 @@ class ForwardArgs(ctypes.Structure):
         ("idx_out", ctypes.c_void_p), ("events", ctypes.c_void_p), ("indexer", ctypes.c_int),
         ("index_dtype", ctypes.c_int), ("sink_k", ctypes.c_void_p), ("sink_v", ctypes.c_void_p),
         ("nsink", ctypes.c_int), ("attn_form", ctypes.c_int),
+        ("topk_fallback_out", ctypes.c_void_p),
     ]
 
 
@@ -71,6 +72,9 @@ _SIGNATURES = {
                                         _P]),
     "dsa_hadamard_rotate": (_I, [_I, _P, ctypes.c_longlong, _I, _P, _P]),
     "dsa_topk": (_I, [_P, _I, _I, _I, _I, _P, _P]),
+    "dsa_index_topk_workspace_bytes": (_Z, [_I, _I, _I, _I]),
+    "dsa_index_topk": (_I, [_I, _P, _P, _P, _F, _I, _I, _I, _I, _I, _I, _I, _P, _P, _Z, _P,
+                            _P]),
     "dsa_sparse_attn_workspace_bytes": (_Z, [_I, _I, _I, _I, _I, _I, _I, _I, _I]),
     "dsa_sparse_attn_algo": (_I, [_I, _I, _I, _I, _I, _I, _I, _I, _I]),
     "dsa_sparse_attn": (_I, [_I, _P, _P, _P, _P, _I, _P, _I, _F, _I, _I, _I, _I, _I, _I, _I, _P,
@@ -212,6 +216,29 @@ def dsa_topk(scores, K, idx=None, stream=None):
     return idx
 
 
+
+def dsa_index_topk_workspace_bytes(B, S, T, K) -> int:
+    return int(lib().dsa_index_topk_workspace_bytes(B, S, T, K))
+
+
+def dsa_index_topk(q_idx, k_idx, w, scale, K, relu="none", idx=None, ws=None,
+                   fallback_out=None, stream=None):
+    """Fused indexer -> top-k: the indices dsa_index_scores + dsa_topk give, without the
+    score matrix (candidates filtered inside the indexer).  fallback_out: optional int32
+    device tensor of one element, set to 1 when the full-score fallback ran."""
+    _dev(q_idx, k_idx, w, idx, ws, fallback_out)
+    B, S, HI, DI = q_idx.shape
+    T = k_idx.shape[1]
+    k_eff = min(int(K), T)
+    if idx is None:
+        idx = torch.empty((B, S, k_eff), dtype=torch.int32, device=q_idx.device)
+    nbytes = dsa_index_topk_workspace_bytes(B, S, T, int(K))
+    ws = _workspace(nbytes, q_idx.device, ws)
+    _check(lib().dsa_index_topk(_dtype_code(q_idx), _ptr(q_idx), _ptr(k_idx), _ptr(w),
+                                float(scale), RELU[relu], B, S, T, HI, DI, int(K), _ptr(idx),
+                                _ptr(ws), nbytes, _ptr(fallback_out), _stream(stream)))
+    return idx
+
 def dsa_sparse_attn_workspace_bytes(dtype, B, S, T, H, DQK, DV, K, algo="auto") -> int:
     code = dtype if isinstance(dtype, int) else DTYPE[dtype]
     return int(lib().dsa_sparse_attn_workspace_bytes(code, B, S, T, H, DQK, DV, K,
@@ -316,7 +343,7 @@ def dsa_sparse_attn_latent(q, kv, idx, dv=512, sink_kv=None, gate=None, gate_mod
 
 def _forward_args(q_idx, k_idx, w, index_scale, K, q, k, v, gate, gate_mode, relu, sm_scale,
                   attn_algo, out, scores_out, idx_out, indexer="per_head", sink_k=None,
-                  sink_v=None, attn_form="expanded", dv=512):
+                  sink_v=None, attn_form="expanded", dv=512, topk_fallback_out=None):
     B, S, HI, DI = q_idx.shape
     T = k_idx.shape[1]
     H, DQK = q.shape[2], q.shape[3]
@@ -333,7 +360,8 @@ def _forward_args(q_idx, k_idx, w, index_scale, K, q, k, v, gate, gate_mode, rel
         index_dtype=1 if q_idx.dtype == torch.float8_e4m3fn else 0,
         sink_k=None if sink_k is None else sink_k.data_ptr(),
         sink_v=None if sink_v is None else sink_v.data_ptr(),
-        nsink=0 if sink_k is None else int(sink_k.shape[0]), attn_form=ATTN_FORM[attn_form])
+        nsink=0 if sink_k is None else int(sink_k.shape[0]), attn_form=ATTN_FORM[attn_form],
+        topk_fallback_out=None if topk_fallback_out is None else topk_fallback_out.data_ptr())
     return a
 
 
@@ -345,16 +373,19 @@ def dsa_forward_workspace_bytes(args: ForwardArgs, minimum: bool = False) -> int
 def dsa_forward(q_idx, k_idx, w, index_scale, K, q, k, v, gate=None, gate_mode=None,
                 relu="none", sm_scale=0.0, attn_algo="auto", out=None, scores_out=None,
                 idx_out=None, ws=None, ws_bytes=None, stream=None, events=None,
-                indexer="per_head", sink_k=None, sink_v=None, attn_form="expanded", dv=512):
+                indexer="per_head", sink_k=None, sink_v=None, attn_form="expanded", dv=512,
+                topk_fallback_out=None):
     """The whole DSA step (indexer -> top-k -> sparse attention -> gate).
-    indexer: "per_head" (the pages' per-head work) or "collapsed" (see
-    dsa_index_scores_collapsed).  attn_form "latent": k is the latent cache [B,T,DQK]
+    indexer: "per_head" (the pages' per-head work), "collapsed" (see
+    dsa_index_scores_collapsed) or "fused" (see dsa_index_topk; topk_fallback_out, an
+    optional int32 device tensor of one element, receives whether its fallback ran).  attn_form "latent": k is the latent cache [B,T,DQK]
     (values = its first ``dv`` dims), v is None, sink_k holds latent sink rows [NS,DQK].
 
     Returns (out, idx); idx is idx_out if given, else a view of the workspace copy.
     ``ws_bytes`` limits the workspace handed to the library (row blocking below the
     full size)."""
-    _dev(q_idx, k_idx, w, q, k, v, gate, out, scores_out, idx_out, ws, sink_k, sink_v)
+    _dev(q_idx, k_idx, w, q, k, v, gate, out, scores_out, idx_out, ws, sink_k, sink_v,
+         topk_fallback_out)
     B, S = q_idx.shape[:2]
     T = k_idx.shape[1]
     if out is None:
@@ -365,7 +396,7 @@ def dsa_forward(q_idx, k_idx, w, index_scale, K, q, k, v, gate=None, gate_mode=N
         idx_out = torch.empty((B, S, k_eff), dtype=torch.int32, device=q.device)
     a = _forward_args(q_idx, k_idx, w, index_scale, K, q, k, v, gate, gate_mode, relu, sm_scale,
                       attn_algo, out, scores_out, idx_out, indexer, sink_k, sink_v, attn_form,
-                      dv)
+                      dv, topk_fallback_out)
     ev_arr = None
     if events is not None:  # 4 torch.cuda.Event, recorded by the library at stage boundaries
         for e in events:

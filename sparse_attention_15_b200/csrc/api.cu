@@ -117,6 +117,108 @@ dsa_status run_index_scores_collapsed(const void* qc, const void* k_idx, float s
                      "dsa_index_scores_collapsed");
 }
 
+// ----------------------------------------------------------------------------- fused
+// Workspace of the fused indexer -> top-k (section 2b of dsa.h): the sampled scores, the
+// thresholds, the candidate counters (+ the fallback flag), the candidate lists and the
+// full score matrix the fallback uses.
+struct FusedLayout {
+  int kstride, cap;
+  long long ld;  // sampled columns per row
+  size_t qc_off, sample_off, tau_off, cnt_off, ck_off, ct_off, scores_off, total;
+};
+
+FusedLayout fused_layout(int B, int S, int T, int K_eff) {
+  FusedLayout L{};
+  const int ntiles = (T + 127) / 128;
+  L.kstride = ntiles / 32 > 4 ? ntiles / 32 : 4;
+  L.cap = 2 * K_eff + 1024;
+  L.ld = (long long)(((ntiles - 1) / L.kstride) + 1) * 128;
+  const size_t rows = (size_t)B * S;
+  size_t off = 0;
+  L.qc_off = off;     off += align256(rows * 2 * 128 * sizeof(uint16_t));  // collapsed q_I
+  L.sample_off = off; off += align256(rows * (size_t)L.ld * sizeof(float));
+  L.tau_off = off;    off += align256(rows * sizeof(uint32_t));
+  L.cnt_off = off;    off += align256((rows + 1) * sizeof(int));  // + the fallback flag
+  L.ck_off = off;     off += align256(rows * (size_t)L.cap * sizeof(uint32_t));
+  L.ct_off = off;     off += align256(rows * (size_t)L.cap * sizeof(int32_t));
+  L.scores_off = off; off += align256(rows * (size_t)T * sizeof(float));
+  L.total = off;
+  return L;
+}
+
+bool fused_supported(dsa_dtype dtype, int HI, int DI, int T, int K_eff) {
+  return dsa::index_scores_tc_supported((int)dtype, HI, DI) &&
+         dsa::topk_candidates_smem(T, 2 * K_eff + 1024) <= 220u * 1024u;
+}
+
+// Enqueues the fused indexer -> top-k into ws (laid out by fused_layout): idx (and the
+// selection mask, if given) for every row; *fallback_out (optional) = whether the
+// full-score path ran.
+dsa_status run_fused_index_topk(const void* q_idx, const void* k_idx, const float* w,
+                                float scale, dsa_relu_mode relu, int B, int S, int T, int HI,
+                                int DI, int K_eff, int32_t* idx, uint32_t* mask,
+                                int mask_stride, uint8_t* ws, int32_t* fallback_out,
+                                cudaStream_t st, cudaEvent_t after_indexer) {
+  const FusedLayout L = fused_layout(B, S, T, K_eff);
+  const int q_off = T - S;
+  const size_t rows = (size_t)B * S;
+  float* sample = reinterpret_cast<float*>(ws + L.sample_off);
+  uint32_t* tau = reinterpret_cast<uint32_t*>(ws + L.tau_off);
+  int* cnt = reinterpret_cast<int*>(ws + L.cnt_off);
+  int* fail = cnt + rows;
+  uint32_t* ck = reinterpret_cast<uint32_t*>(ws + L.ck_off);
+  int32_t* ct = reinterpret_cast<int32_t*>(ws + L.ct_off);
+  float* scores = reinterpret_cast<float*>(ws + L.scores_off);
+  cudaError_t e = cudaMemsetAsync(cnt, 0, (rows + 1) * sizeof(int), st);
+  if (e != cudaSuccess) return cuda_status(e, "fused/clear");
+  // 1. the sample: every kstride-th key tile of each row.  Without a per-head ReLU the score
+  // is linear in q_I and the head-collapsed indexer gives the same scores (exactly for
+  // integer inputs, to float32 rounding of its hi/lo split otherwise) for 1/HI of the work;
+  // the threshold only steers how many candidates pass, the count check keeps it exact
+  dsa::IndexerExtra xs{};
+  xs.kstride = L.kstride;
+  xs.ldT = L.ld;
+  if (dsa::index_scores_collapsed_supported(1, DI, (int)relu)) {
+    void* qc = ws + L.qc_off;
+    e = dsa::launch_collapse_q(q_idx, w, (long long)rows, HI, DI, qc, st);
+    if (e == cudaSuccess)
+      e = dsa::launch_index_scores_collapsed(qc, k_idx, scale, (int)relu, B, S, T, DI, q_off,
+                                             sample, 0, st, &xs);
+  } else {
+    e = dsa::launch_index_scores_tc(q_idx, k_idx, w, scale, (int)relu, B, S, T, HI, DI, q_off,
+                                    sample, 0, st, &xs);
+  }
+  if (e != cudaSuccess) return cuda_status(e, "fused/sample");
+  // 2. the thresholds
+  e = dsa::launch_topk_tau(sample, L.ld, B, S, T, K_eff, q_off, L.kstride, L.cap, tau, st);
+  if (e != cudaSuccess) return cuda_status(e, "fused/tau");
+  // 3. every score, kept only as a candidate when it reaches its row's threshold
+  dsa::IndexerExtra xf{};
+  xf.tau = tau; xf.cand_key = ck; xf.cand_t = ct; xf.cand_cnt = cnt; xf.cand_cap = L.cap;
+  e = dsa::launch_index_scores_tc(q_idx, k_idx, w, scale, (int)relu, B, S, T, HI, DI, q_off,
+                                  nullptr, 0, st, &xf);
+  if (e != cudaSuccess) return cuda_status(e, "fused/filter");
+  if (after_indexer && (e = cudaEventRecord(after_indexer, st)) != cudaSuccess)
+    return cuda_status(e, "fused/event");
+  // 4. the exact top-k of every row from its candidates (or the fallback flag)
+  e = dsa::launch_topk_candidates(ck, ct, cnt, L.cap, B, S, T, K_eff, q_off, idx, mask,
+                                  mask_stride, fail, st);
+  if (e != cudaSuccess) return cuda_status(e, "fused/select");
+  // 5. the fallback, a no-op unless some row raised the flag: full scores, full top-k
+  dsa::IndexerExtra xr{};
+  xr.run_if = fail;
+  e = dsa::launch_index_scores_tc(q_idx, k_idx, w, scale, (int)relu, B, S, T, HI, DI, q_off,
+                                  scores, 0, st, &xr);
+  if (e != cudaSuccess) return cuda_status(e, "fused/fallback scores");
+  e = dsa::launch_topk(scores, B, S, T, K_eff, q_off, idx, mask, mask_stride, st, fail);
+  if (e != cudaSuccess) return cuda_status(e, "fused/fallback top-k");
+  if (fallback_out &&
+      (e = cudaMemcpyAsync(fallback_out, fail, sizeof(int), cudaMemcpyDeviceToDevice, st)) !=
+          cudaSuccess)
+    return cuda_status(e, "fused/fallback flag");
+  return DSA_OK;
+}
+
 // Attention sinks ([PANGU] §3.4 PAS): up to one 128-entry block, [nsink, H, D] rows.
 dsa_status check_sinks(const void* sink_k, const void* sink_v, int nsink) {
   if (nsink == 0) return DSA_OK;
@@ -136,9 +238,7 @@ float default_scale(float sm_scale, int DQK) {
 
 constexpr int kNone = -1, kGather = 1, kMasked = 2, kLatent = 3;
 
-size_t mask_bytes(int B, int S, int T) {
-  return (size_t)B * S * dsa::mask_stride_words(T) * sizeof(uint32_t);
-}
+size_t mask_bytes(int B, int S, int T) { return dsa::masked_attn_mask_bytes(B, S, T); }
 
 // Cost model of the two attention algorithms.  Gather: every selected (query, key) pair
 // moves one K row and one V row (H * (DQK + DV) elements).  Masked tile: every 128-query
@@ -302,6 +402,33 @@ dsa_status dsa_topk(const float* scores, int B, int S, int T, int K, int32_t* id
                      "dsa_topk");
 }
 
+size_t dsa_index_topk_workspace_bytes(int B, int S, int T, int K) {
+  if (B <= 0 || S <= 0 || T <= 0 || K <= 0) return 0;
+  return fused_layout(B, S, T, K < T ? K : T).total;
+}
+
+dsa_status dsa_index_topk(dsa_dtype dtype, const void* q_idx, const void* k_idx,
+                          const float* w, float scale, dsa_relu_mode relu, int B, int S, int T,
+                          int HI, int DI, int K, int32_t* idx, void* ws, size_t ws_bytes,
+                          int32_t* fallback_out, dsa_stream_t stream) {
+  dsa_status st = check_index_args(dtype, q_idx, k_idx, w, scale, relu, B, S, T, HI, DI, idx);
+  if (st != DSA_OK) return st;
+  REQUIRE(K > 0, DSA_ERR_INVALID_ARG, "K must be positive");
+  REQUIRE((size_t)B * S <= 0x7fffffffu, DSA_ERR_UNSUPPORTED, "too many rows");
+  const int k_eff = K < T ? K : T;
+  REQUIRE(fused_supported(dtype, HI, DI, T, k_eff), DSA_ERR_UNSUPPORTED,
+          "the fused indexer -> top-k needs bf16 inputs, HI in {16,32}, DI in {64,128} and "
+          "T, K small enough for the candidate select (T=%d, K=%d)", T, k_eff);
+  const size_t need = fused_layout(B, S, T, k_eff).total;
+  REQUIRE(ws != nullptr && ws_bytes >= need, DSA_ERR_INVALID_ARG,
+          "workspace too small: %zu bytes given, %zu needed", ws_bytes, need);
+  REQUIRE(aligned16(ws) && (fallback_out == nullptr || aligned16(fallback_out)),
+          DSA_ERR_UNSUPPORTED, "workspace and fallback_out must be 16-byte aligned");
+  return run_fused_index_topk(q_idx, k_idx, w, scale, relu, B, S, T, HI, DI, k_eff, idx,
+                              nullptr, 0, static_cast<uint8_t*>(ws), fallback_out,
+                              (cudaStream_t)stream, nullptr);
+}
+
 size_t dsa_sparse_attn_workspace_bytes(dsa_dtype dtype, int B, int S, int T, int H, int DQK,
                                        int DV, int K, dsa_attn_algo algo) {
   return dsa_sparse_attn_sinks_workspace_bytes(dtype, B, S, T, H, DQK, DV, K, 0, algo);
@@ -403,7 +530,9 @@ static dsa_status sparse_attn_impl(dsa_dtype dtype, const void* q, const void* k
     st = cuda_status(dsa::launch_idx_to_mask(idx, B, S, T, K, T - S, mask, stride, s),
                      "dsa_sparse_attn/mask");
     if (st != DSA_OK) return st;
-    return cuda_status(dsa::launch_masked_attn(p, mask, stride, s), "dsa_sparse_attn");
+    return cuda_status(dsa::launch_masked_attn(p, mask, stride,
+                                               dsa::masked_attn_occ(mask, B, S, T), s),
+                       "dsa_sparse_attn");
   }
   return cuda_status(dsa::launch_gather_attn(p, ws, ws_bytes, s), "dsa_sparse_attn");
 }
@@ -478,7 +607,7 @@ static dsa_status window_attn_impl(dsa_dtype dtype, const void* q, const void* k
   cudaStream_t s = (cudaStream_t)stream;
   // the band is dense work for every query block with at least a few rows: tensor cores
   if (algo == DSA_ATTN_MASKED_TILE || (algo == DSA_ATTN_AUTO && tc && S >= 64))
-    return cuda_status(dsa::launch_masked_attn(p, nullptr, 0, s), "dsa_window_attn");
+    return cuda_status(dsa::launch_masked_attn(p, nullptr, 0, nullptr, s), "dsa_window_attn");
   return cuda_status(dsa::launch_gather_attn(p, nullptr, 0, s), "dsa_window_attn");
 }
 
@@ -533,8 +662,19 @@ static dsa_status check_forward(const dsa_forward_args* a) {
           DSA_ERR_INVALID_ARG, "unknown attention algorithm %d", (int)a->attn_algo);
   REQUIRE(a->idx_out == nullptr || aligned16(a->idx_out), DSA_ERR_UNSUPPORTED,
           "idx_out must be 16-byte aligned");
-  REQUIRE(a->indexer == DSA_INDEXER_PER_HEAD || a->indexer == DSA_INDEXER_COLLAPSED,
+  REQUIRE(a->indexer == DSA_INDEXER_PER_HEAD || a->indexer == DSA_INDEXER_COLLAPSED ||
+              a->indexer == DSA_INDEXER_FUSED,
           DSA_ERR_INVALID_ARG, "unknown indexer mode %d", (int)a->indexer);
+  if (a->indexer == DSA_INDEXER_FUSED) {
+    const int k_eff = a->K < a->T ? a->K : a->T;
+    REQUIRE(a->index_dtype == DSA_INDEX_AS_DTYPE &&
+                fused_supported(a->dtype, a->HI, a->DI, a->T, k_eff),
+            DSA_ERR_UNSUPPORTED,
+            "the fused indexer needs bf16 inputs, HI in {16,32}, DI in {64,128} and T, K small "
+            "enough for the candidate select");
+    REQUIRE(a->topk_fallback_out == nullptr || aligned16(a->topk_fallback_out),
+            DSA_ERR_UNSUPPORTED, "topk_fallback_out must be 16-byte aligned");
+  }
   if (!latent && (st = check_sinks(a->sink_k, a->sink_v, a->nsink)) != DSA_OK) return st;
   if (a->indexer == DSA_INDEXER_COLLAPSED) return check_collapsed(a->dtype, a->relu, a->DI);
   return DSA_OK;
@@ -542,6 +682,7 @@ static dsa_status check_forward(const dsa_forward_args* a) {
 
 struct FwdLayout {
   size_t idx_off, attn_off, mask_off, qc_off, scores_off, total_full, total_min;
+  size_t fused_off;  // DSA_INDEXER_FUSED: its workspace (fused_layout) starts here
   int k_eff, alg, mask_stride;
 };
 
@@ -568,11 +709,14 @@ static FwdLayout forward_layout(const dsa_forward_args* a) {
   L.qc_off = off;
   if (a->indexer == DSA_INDEXER_COLLAPSED) off += align256(collapsed_q_bytes(a->B, a->S, a->DI));
   L.scores_off = off;
+  L.fused_off = off;
   if (a->scores_out) {
     L.total_full = L.total_min = off;
   } else {
     L.total_full = off + align256((size_t)a->B * a->S * a->T * sizeof(float));
     L.total_min = off + align256((size_t)a->T * sizeof(float));
+    if (a->indexer == DSA_INDEXER_FUSED)  // its layout ends with the full score matrix
+      L.total_full = off + fused_layout(a->B, a->S, a->T, L.k_eff).total;
   }
   return L;
 }
@@ -613,11 +757,28 @@ dsa_status dsa_forward(const dsa_forward_args* a, void* ws, size_t ws_bytes,
     return ev ? cuda_status(cudaEventRecord(ev[i], s), "dsa_forward/event") : DSA_OK;
   };
   if ((st = mark(0)) != DSA_OK) return st;
-  if (collapsed &&
+  // the fused indexer -> top-k needs its whole workspace and no score matrix output; else
+  // the per-head path below computes the same indices
+  const bool fused =
+      a->indexer == DSA_INDEXER_FUSED && !a->scores_out && ws_bytes >= L.total_full;
+  if (fused) {
+    st = run_fused_index_topk(a->q_idx, a->k_idx, a->w, a->index_scale, a->relu, B, S, T,
+                              a->HI, a->DI, L.k_eff, idx, mask, L.mask_stride,
+                              base + L.fused_off, a->topk_fallback_out, s,
+                              ev ? ev[1] : nullptr);
+    if (st != DSA_OK || (st = mark(2)) != DSA_OK) return st;
+  } else if (a->indexer == DSA_INDEXER_FUSED && a->topk_fallback_out &&
+             (st = cuda_status(cudaMemsetAsync(a->topk_fallback_out, 0, sizeof(int32_t), s),
+                               "dsa_forward/fallback flag")) != DSA_OK) {
+    return st;
+  }
+  if (!fused && collapsed &&
       (st = run_collapse_q(a->q_idx, a->w, (long long)B * S, a->HI, a->DI, qc, s)) != DSA_OK)
     return st;
 
-  if (a->scores_out || ws_bytes >= L.total_full) {
+  if (fused) {
+    // indices and the selection mask are done
+  } else if (a->scores_out || ws_bytes >= L.total_full) {
     float* scores = a->scores_out ? a->scores_out : reinterpret_cast<float*>(base + L.scores_off);
     st = collapsed ? run_index_scores_collapsed(qc, a->k_idx, a->index_scale, a->relu, B, S, T,
                                                 a->DI, q_off, scores, write_masked, s)
@@ -679,7 +840,9 @@ dsa_status dsa_forward(const dsa_forward_args* a, void* ws, size_t ws_bytes,
     p.sink_k = a->sink_k; p.sink_v = a->sink_v; p.nsink = a->nsink;
   }
   if (L.alg == kMasked)
-    st = cuda_status(dsa::launch_masked_attn(p, mask, L.mask_stride, s), "dsa_forward/attn");
+    st = cuda_status(dsa::launch_masked_attn(p, mask, L.mask_stride,
+                                             dsa::masked_attn_occ(mask, B, S, T), s),
+                     "dsa_forward/attn");
   else
     st = cuda_status(dsa::launch_gather_attn(p, attn_ws, attn_ws_bytes, s), "dsa_forward/attn");
   if (st != DSA_OK) return st;

@@ -56,6 +56,8 @@ struct AttnArgs {
   int mask_stride;       // words per mask row (multiple of 4)
   int nqb;
   int nsink;             // attention sinks (PAS), 0..128: one extra block per item
+  const uint32_t* occ;   // tile occupancy [B, nqb, occ_words] (mask mode) or NULL
+  int occ_words;
 };
 
 template <int DQK_, int DV_, bool BAND_>
@@ -89,7 +91,10 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
-// Item i -> (query block, batch row, head); longest query blocks first.
+// Item i -> (query block, batch row, head): head-major, longest query blocks first within a
+// head.  The CTAs working at the same time then walk the key blocks of one head (42 MB of
+// K/V at the 65536-token shapes), which stays in L2 while they share it, instead of every
+// head's K/V at once.
 struct Item {
   int qb, b, h;
 };
@@ -100,8 +105,9 @@ __device__ __forceinline__ int snake_item(int k, int c, int G) {
 }
 __device__ __forceinline__ Item item_of(const AttnArgs& a, int i) {
   Item it;
-  it.h = i % a.H;
-  const int r = i / a.H;
+  const int per_head = a.B * a.nqb;
+  it.h = i / per_head;
+  const int r = i - it.h * per_head;
   it.b = r % a.B;
   it.qb = a.nqb - 1 - r / a.B;
   return it;
@@ -127,6 +133,53 @@ __device__ __forceinline__ int sink_blocks(const AttnArgs& a) {
   return a.nsink > 0 ? 1 : 0;
 }
 
+// Empty tiles are skipped ([AXK2] "注意力前向的骨架": under the additive sparse mask a key block
+// no query of the item selected contributes exp(-inf) = 0 to every row): with an occupancy
+// summary an item visits only the occupied key blocks of [j0, j1), in ascending order -- or,
+// when none is occupied, key block j0 alone, so that every item has a block and its outputs
+// (zeros) are written by the same path.
+struct KeyBlocks {
+  const uint32_t* w;  // the item's occupancy words, or NULL: every block of [j0, j1)
+  int j0, j1;
+  __device__ __forceinline__ int next_occupied(int j) const {  // first occupied >= j, or j1
+    while (j < j1) {
+      const uint32_t m = __ldg(w + (j >> 5)) >> (j & 31);
+      if (m) return min(j + __ffs(m) - 1, j1);
+      j = (j | 31) + 1;
+    }
+    return j1;
+  }
+  __device__ __forceinline__ int count() const {  // popcounts of the range's words
+    if (!w) return j1 - j0;
+    int n = 0;
+    const int w0 = j0 >> 5, w1 = (j1 - 1) >> 5;
+    for (int wi = w0; wi <= w1; ++wi) {  // independent loads
+      uint32_t m = __ldg(w + wi);
+      if (wi == w0) m &= 0xffffffffu << (j0 & 31);
+      if (wi == w1 && (j1 & 31)) m &= (1u << (j1 & 31)) - 1u;
+      n += __popc(m);
+    }
+    return n > 0 ? n : 1;
+  }
+  __device__ __forceinline__ int first() const {
+    if (!w) return j0;
+    const int j = next_occupied(j0);
+    return j < j1 ? j : j0;
+  }
+  __device__ __forceinline__ int next(int j) const {
+    return w ? next_occupied(j + 1) : j + 1;
+  }
+};
+
+__device__ __forceinline__ KeyBlocks key_blocks(const AttnArgs& a, const Item& it, int j0,
+                                                int j1) {
+  KeyBlocks kb;
+  kb.w = a.occ ? a.occ + ((size_t)it.b * a.nqb + it.qb) * a.occ_words : nullptr;
+  kb.j0 = j0;
+  kb.j1 = j1;
+  return kb;
+}
+
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1)
     masked_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
@@ -145,7 +198,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   uint64_t* k_full = bars + 2;       // [2] K block landed
   uint64_t* k_empty = bars + 4;      // [2] K block consumed by S = Q K^T
   uint64_t* s_full = bars + 6;       // [2]
-  uint64_t* s_empty = bars + 8;      // [2]
   uint64_t* p_full = bars + 10;      // [2]
   uint64_t* pv_done = bars + 12;     // [2] (one phase per block of that parity)
   uint64_t* o_empty = bars + 14;     // 1 (one phase per item)
@@ -165,7 +217,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1);
       mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1);
-      mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], 1);
+      mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 4);
     }
     mbar_init(&pv_done[0], 1); mbar_init(&pv_done[1], 1);
@@ -209,14 +261,17 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
         const int kvh = it.h / group;
         const int sb = sink_blocks<C::BAND>(a);
-        const int nb = j1 - j0 + sb;
+        const KeyBlocks kb = key_blocks(a, it, j0, j1);
+        const int nb = kb.count() + sb;
+        int jc = kb.first();  // key block of the next non-sink item block
         for (int r = 0; r < nb; ++r, ++g) {
           const int st = g & 1;
           if (g >= 2 && !mbar_wait(&empty[st], ((g >> 1) - 1) & 1)) { ok = false; break; }
           uint8_t* dst = KVs + st * C::KV_BYTES + (kq ? 0 : C::K_BYTES);
           // the sink block reads rows 0..127 of the sink arrays (rows past nsink: zero fill)
           const bool sink = r < sb;
-          const int krow = sink ? 0 : it.b * a.T + (j0 + r - sb) * kBlk;
+          const int krow = sink ? 0 : it.b * a.T + jc * kBlk;
+          if (!sink) jc = kb.next(jc);
           if (kq) {
             mbar_arrive_expect_tx(&full[st], C::K_BYTES);
 #pragma unroll
@@ -247,11 +302,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       const uint64_t vdesc0 = sw128_mnmajor_desc(smem_u32(KVs + C::K_BYTES), C::SLICE, 1024);
       uint32_t g = 0, ni = 0;
       bool ok = true;
-      // S_g = Q K_g^T into S[g & 1]
+      // S_g = Q K_g^T into S[g & 1].  S[g & 1] last held P_{g-2}, read by P V_{g-2}, which
+      // this thread issued before: one thread's tcgen05.mma instructions execute in issue
+      // order, so those reads are done before this product writes the columns -- no wait
+      // for P V_{g-2} to complete, and the tensor pipe never drains between blocks.
       auto issue_qk = [&](uint32_t gg) -> bool {
         const int st = gg & 1;
         if (!mbar_wait(&k_full[st], (gg >> 1) & 1)) return false;
-        if (gg >= 2 && !mbar_wait(&s_empty[gg & 1], ((gg >> 1) - 1) & 1)) return false;
         tc_fence_after();
         const uint64_t kd = kdesc0 + (uint64_t)((st * C::KV_BYTES) >> 4);
 #pragma unroll
@@ -269,7 +326,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         const Item it = item_of(a, i);
         int j0, j1;
         key_range<C::BAND>(a, it, &j0, &j1);
-        const int nb = j1 - j0 + sink_blocks<C::BAND>(a);
+        const int nb = key_blocks(a, it, j0, j1).count() + sink_blocks<C::BAND>(a);
         if (!mbar_wait(q_full, ni & 1)) { ok = false; break; }
         if (!issue_qk(g)) { ok = false; break; }
         for (int j = 0; j < nb; ++j) {
@@ -293,7 +350,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             umma_f16_ts(o_tmem, p_tmem + pc + 8, vdesc, idesc_pv, 1u);
           }
           umma_commit(&v_empty[gg & 1]);
-          umma_commit(&s_empty[gg & 1]);
           umma_commit(&pv_done[gg & 1]);
         }
         g += nb;
@@ -319,7 +375,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       int j0, j1;
       key_range<C::BAND>(a, it, &j0, &j1);
       const int sb = sink_blocks<C::BAND>(a);
-      const int nb = j1 - j0 + sb;
+      const KeyBlocks kb = key_blocks(a, it, j0, j1);
+      const int nb = kb.count() + sb;
       const int s = it.qb * kBlk + row;
       const int spos = s + a.q_off;
       const bool row_ok = s < a.S;
@@ -327,9 +384,18 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           (!C::BAND && row_ok) ? a.mask + ((size_t)it.b * a.S + s) * a.mask_stride : nullptr;
       const int jfirst = (int)((grp - g) & 1u);  // first block of this group's parity
       float m_used = ninf, l = 0.f;
-      // the 4 selection words of item block r >= sb (key block j0 + r - sb)
+      // key block of item block r >= sb, for non-decreasing r (a cursor over the visited
+      // blocks), and its 4 selection words
+      int cur_r = sb, cur_j = kb.first();
+      auto key_block = [&](int r) {
+        while (cur_r < r) {
+          cur_j = kb.next(cur_j);
+          ++cur_r;
+        }
+        return cur_j;
+      };
       auto mask_words = [&](int r) {
-        return __ldg(reinterpret_cast<const uint4*>(mrow + (((j0 + r - sb) * kBlk) >> 5)));
+        return __ldg(reinterpret_cast<const uint4*>(mrow + ((key_block(r) * kBlk) >> 5)));
       };
       uint4 nb4 = make_uint4(0u, 0u, 0u, 0u);
       if (mrow && jfirst < nb && jfirst >= sb) nb4 = mask_words(jfirst);
@@ -378,9 +444,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             mx[c] = ninf;
 #pragma unroll
             for (int e = 0; e < 32; e += 2) {
+              // unselected keys become -inf here, once: pass 2 reads the masked row
               const float x0 = (bits[c] & (1u << e)) ? __uint_as_float(r[c * 32 + e]) : ninf;
               const float x1 =
                   (bits[c] & (1u << (e + 1))) ? __uint_as_float(r[c * 32 + e + 1]) : ninf;
+              r[c * 32 + e] = __float_as_uint(x0);
+              r[c * 32 + e + 1] = __float_as_uint(x1);
               mx[c] = max3(mx[c], x0, x1);
             }
           }
@@ -410,14 +479,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         const unsigned long long nm2 = pack2(-msub, -msub);
         // 16 keys per chunk, from the row held in registers since pass 1; chunk k's P_hi and
         // P_lo overwrite its own 16 S columns
-        auto chunk = [&](uint32_t bw, int kk) {
+        auto chunk = [&](int kk) {
           uint32_t ph[8], pl[8];
 #pragma unroll
           for (int e2 = 0; e2 < 8; ++e2) {
             const int e = 2 * e2;
-            const float x0 = (bw & (1u << e)) ? __uint_as_float(r[16 * kk + e]) : ninf;
-            const float x1 =
-                (bw & (1u << (e + 1))) ? __uint_as_float(r[16 * kk + e + 1]) : ninf;
+            const float x0 = __uint_as_float(r[16 * kk + e]);
+            const float x1 = __uint_as_float(r[16 * kk + e + 1]);
             float y0, y1;
             unpack2(fma2(pack2(x0, x1), scale2, nm2), y0, y1);  // scale*s - m, two keys
             const float p0 = ex2_ftz(y0), p1 = ex2_ftz(y1);
@@ -437,10 +505,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           tmem_st8(s_col + kk * 16 + 8, pl);
         };
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          chunk(bits[c], 2 * c);
-          chunk(bits[c] >> 16, 2 * c + 1);
-        }
+        for (int kk = 0; kk < 8; ++kk) chunk(kk);
         {
           float r0, r1;
           unpack2(rs2, r0, r1);
@@ -533,6 +598,29 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   }
 }
 
+// The tile-occupancy summary of a selection mask: one CTA per (batch row, 128-query block);
+// thread j covers key block j (its 4 mask words in every row of the block, coalesced across
+// the threads), and each warp's 32 key blocks become one word by a ballot.
+__global__ void tile_occupancy_kernel(const uint32_t* __restrict__ mask, int mask_stride, int S,
+                                      int nqb, int nkb, uint32_t* __restrict__ occ,
+                                      int occ_words) {
+  const int b = blockIdx.x / nqb, qb = blockIdx.x % nqb;
+  const int s0 = qb * kBlk, s1 = min(S, s0 + kBlk);
+  const uint32_t* m0 = mask + ((size_t)b * S + s0) * mask_stride;
+  uint32_t* o = occ + (size_t)blockIdx.x * occ_words;
+  for (int jb = 0; jb < occ_words * 32; jb += blockDim.x) {
+    const int j = jb + (int)threadIdx.x;
+    uint32_t any = 0u;
+    if (j < nkb)
+      for (int s = 0; s < s1 - s0 && !any; ++s) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(m0 + (size_t)s * mask_stride) + j);
+        any = v.x | v.y | v.z | v.w;
+      }
+    const uint32_t word = __ballot_sync(0xffffffffu, any != 0u);
+    if ((threadIdx.x & 31) == 0 && (j >> 5) < occ_words) o[j >> 5] = word;
+  }
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -571,7 +659,7 @@ int num_sms() {
 
 template <class C>
 cudaError_t launch_fa(const AttnProblem& p, const uint32_t* mask, int mask_stride,
-                      cudaStream_t st) {
+                      const uint32_t* occ, cudaStream_t st) {
   CUtensorMap qm, km, vm, skm, svm;
   if (!map3d(&qm, p.q, (uint64_t)p.B * p.S, p.H, C::DQK) ||
       !map3d(&km, p.k, (uint64_t)p.B * p.T, p.HKV, C::DQK) ||
@@ -594,6 +682,8 @@ cudaError_t launch_fa(const AttnProblem& p, const uint32_t* mask, int mask_strid
   a.window = p.window; a.mask_stride = mask_stride;
   a.nsink = sinks ? p.nsink : 0;
   a.nqb = (p.S + kBlk - 1) / kBlk;
+  a.occ = occ;
+  a.occ_words = occ_words(p.T);
   const int items = p.B * p.H * a.nqb;
   const int nsm = num_sms();
   const int grid = items < nsm ? items : nsm;
@@ -611,15 +701,24 @@ bool masked_attn_supported(int dtype, int DQK, int DV) {
 }
 
 cudaError_t launch_masked_attn(const AttnProblem& p, const uint32_t* mask, int mask_stride,
-                               cudaStream_t st) {
+                               uint32_t* occ, cudaStream_t st) {
   if (!masked_attn_supported(p.dtype, p.DQK, p.DV)) return cudaErrorNotSupported;
   const bool band = p.idx == nullptr && mask == nullptr;
   if (!band && mask == nullptr) return cudaErrorInvalidValue;
+  if (band) occ = nullptr;
+  if (occ != nullptr) {  // which key blocks each 128-query block selected anything from
+    const int nqb = (p.S + kBlk - 1) / kBlk;
+    const int nkb = (p.T + kBlk - 1) / kBlk;
+    tile_occupancy_kernel<<<(unsigned)(p.B * nqb), 256, 0, st>>>(mask, mask_stride, p.S, nqb,
+                                                                nkb, occ, occ_words(p.T));
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   if (p.DQK == 128)
-    return band ? launch_fa<FaCfg<128, 128, true>>(p, mask, mask_stride, st)
-                : launch_fa<FaCfg<128, 128, false>>(p, mask, mask_stride, st);
-  return band ? launch_fa<FaCfg<192, 128, true>>(p, mask, mask_stride, st)
-              : launch_fa<FaCfg<192, 128, false>>(p, mask, mask_stride, st);
+    return band ? launch_fa<FaCfg<128, 128, true>>(p, mask, mask_stride, occ, st)
+                : launch_fa<FaCfg<128, 128, false>>(p, mask, mask_stride, occ, st);
+  return band ? launch_fa<FaCfg<192, 128, true>>(p, mask, mask_stride, occ, st)
+              : launch_fa<FaCfg<192, 128, false>>(p, mask, mask_stride, occ, st);
 }
 
 }  // namespace dsa

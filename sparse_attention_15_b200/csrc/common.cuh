@@ -56,6 +56,14 @@ __device__ __forceinline__ float gate_act(float g, int mode) {
   return mode == 2 ? g * sg : sg;
 }
 
+// Order-preserving 32-bit image of a float score: unsigned comparison of the images is the
+// float order, with -0.0 mapped to +0.0 (so the two compare equal) and -inf the smallest.
+__device__ __forceinline__ uint32_t order_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  if ((u << 1) == 0u) u = 0u;  // -0.0 -> +0.0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
 // 2^x on the special-function unit (flush-to-zero; exp2(-inf) = +0).
 __device__ __forceinline__ float ex2_ftz(float x) {
   float y;

@@ -49,6 +49,21 @@ struct TcArgs {
   int nqb;         // query blocks per batch row
   int chunk;       // key tiles per work unit
   int max_chunks;  // units per query block slot (chunks of the longest block)
+  // Key tile kt of a unit is key tile kt * kstride of the row (1: every tile; > 1: a strided
+  // sample of the tiles).  Scores land in column kt * 128 + r of rows ldT floats long.
+  int kstride;
+  long long ldT;
+  // Filter mode (tau != NULL): instead of storing scores, append every causal key whose
+  // order key is >= tau[row] to the row's candidate list (order key, key index) -- the first
+  // cand_cap of them; cand_cnt[row] counts all of them.
+  const uint32_t* tau;
+  uint32_t* cand_key;
+  int32_t* cand_t;
+  int* cand_cnt;
+  int cand_cap;
+  // If non-NULL, the launch does nothing unless *run_if != 0 (set on the device by an
+  // earlier kernel of the stream).
+  const int* run_if;
 };
 
 // CL_: the head-collapsed form -- the B operand holds two bf16 rows per query (the hi and
@@ -101,7 +116,7 @@ struct UnitIter {
   __device__ __forceinline__ static int ntiles(const TcArgs& a, int q, int NQ) {
     const int s_last = min(a.S - 1, q * NQ + NQ - 1);
     const int t_last = min(a.T - 1, s_last + a.q_off);
-    return t_last / kTileM + 1;
+    return (t_last / kTileM) / a.kstride + 1;
   }
   // Next non-empty unit owned by this CTA; false when done.
   __device__ __forceinline__ bool next(const TcArgs& a, int NQ, int ncta) {
@@ -122,10 +137,12 @@ struct UnitIter {
   }
 };
 
-template <class C, int RELU>
+template <class C, int RELU, bool FILTER>
 __global__ void __launch_bounds__(C::THREADS, 1)
     index_scores_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                            const __grid_constant__ CUtensorMap qmap, const TcArgs a) {
+  // a launch kept for a fallback that was not needed: every thread leaves at once
+  if (a.run_if != nullptr && *reinterpret_cast<const volatile int*>(a.run_if) == 0) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -192,7 +209,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             break;
           }
           mbar_arrive_expect_tx(&a_full[st], C::A_BYTES);
-          const int krow = it.b * a.T + kt * kTileM;
+          const int krow = it.b * a.T + kt * a.kstride * kTileM;
 #pragma unroll
           for (int kh = 0; kh < C::KH; ++kh)
             tma_load_2d(As + st * C::A_BYTES + kh * C::A_SLICE, &kmap, kh * C::SLICE_ELEMS, krow,
@@ -259,8 +276,42 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     UnitIter it(cta);
     uint32_t ci = 0;
     bool ok = true;
+    // Filter mode: the candidates of each of this warp's queries found in one key tile are
+    // written when that query comes round again in the next tile (or at the end of the
+    // unit): the list position comes from a global atomicAdd issued when the scores are
+    // ready, and its round trip overlaps the next tile's work instead of stalling this one.
+    constexpr int QW = C::CL ? 1 : (C::COLS_PER_WARP / C::HI);  // queries per warp and tile
+    struct Pending {
+      uint32_t bal, key;
+      int t, base;
+      size_t off;
+    };
+    Pending pend[QW];
+    uint32_t tau_q[QW];
+#pragma unroll
+    for (int q = 0; q < QW; ++q) pend[q].bal = 0u;
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    auto flush = [&](Pending& p) {  // p.bal is warp-uniform
+      if (p.bal) {
+        const int base = __shfl_sync(0xffffffffu, p.base, 0);
+        const int pos = base + __popc(p.bal & lt_mask);
+        if (((p.bal >> lane) & 1u) && pos < a.cand_cap) {
+          a.cand_key[p.off + pos] = p.key;
+          a.cand_t[p.off + pos] = p.t;
+        }
+        p.bal = 0u;
+      }
+    };
     while (ok && it.next(a, C::NQ, ncta)) {
       const int s_base = it.qb * C::NQ;
+      if constexpr (FILTER) {
+#pragma unroll
+        for (int q = 0; q < QW; ++q) {
+          flush(pend[q]);
+          const int sq = s_base + col0 / C::HI + q;
+          tau_q[q] = sq < a.S ? __ldg(a.tau + (size_t)it.b * a.S + sq) : 0xffffffffu;
+        }
+      }
       // the head weights of this unit's queries (1-2 KB) are the same for every key tile and
       // every lane: the reduction reads them as warp-wide broadcast float4 loads, which stay
       // in L1 for the whole unit (one load per four heads, no shuffles)
@@ -270,7 +321,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         const int ab = ci % C::NACC;
         if (!warp_wait(&acc_full[ab], (ci / C::NACC) & 1)) { ok = false; break; }
         tc_fence_after();
-        const int t = kt * kTileM + quad * 32 + lane;
+        const int tcol = kt * kTileM + quad * 32 + lane;  // output column
+        const int t = kt * a.kstride * kTileM + quad * 32 + lane;  // key position
         constexpr int NCH = C::COLS_PER_WARP / 16;
         // double-buffered 16-column TMEM reads: chunk cc+1 is in flight while chunk cc is
         // reduced.  A query's HI columns span HI/16 chunks; its four FMA chains carry over.
@@ -294,13 +346,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           if constexpr (C::CL) {
             // eight queries per chunk: score = scale * (D[t, hi] + D[t, lo])
             const int sq = s_base + c0 / 2;
-            float* op = a.scores + ((size_t)it.b * a.S + sq) * a.T + t;
+            float* op = a.scores + ((size_t)it.b * a.S + sq) * a.ldT + tcol;
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
               if (sq + q < a.S && t < a.T) {
                 float v = (__uint_as_float(r[2 * q]) + __uint_as_float(r[2 * q + 1])) * a.scale;
                 if (RELU == 1) v = fmaxf(v, 0.f);
-                op[(size_t)q * a.T] = (t <= sq + q + a.q_off) ? v : ninf;
+                op[(size_t)q * a.ldT] = (t <= sq + q + a.q_off) ? v : ninf;
               }
             }
           } else {
@@ -327,8 +379,24 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 unpack2(acc23, a2, a3);
                 float v = ((a0 + a1) + (a2 + a3)) * a.scale;
                 if (RELU == 1) v = fmaxf(v, 0.f);
-                if (t < a.T)
-                  a.scores[((size_t)it.b * a.S + s) * a.T + t] = (t <= s + a.q_off) ? v : ninf;
+                const size_t row = (size_t)it.b * a.S + s;
+                if constexpr (FILTER) {
+                  // candidates of this query among the warp's 32 keys: one atomic per warp,
+                  // the writes deferred to this query's next tile
+                  Pending& p = pend[(cc * 16) / C::HI];  // compile-time slot
+                  flush(p);
+                  const uint32_t key = order_key(v);
+                  const bool keep =
+                      t < a.T && t <= s + a.q_off && key >= tau_q[(cc * 16) / C::HI];
+                  p.bal = __ballot_sync(0xffffffffu, keep);
+                  p.key = key;
+                  p.t = t;
+                  p.off = row * (size_t)a.cand_cap;
+                  p.base = 0;
+                  if (p.bal && lane == 0) p.base = atomicAdd(a.cand_cnt + row, __popc(p.bal));
+                } else if (t < a.T) {
+                  a.scores[row * a.ldT + tcol] = (t <= s + a.q_off) ? v : ninf;
+                }
                 acc01 = acc23 = pack2(0.f, 0.f);
               }
             }
@@ -337,6 +405,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
         ++ci;
       }
+    }
+    if constexpr (FILTER) {
+#pragma unroll
+      for (int q = 0; q < QW; ++q) flush(pend[q]);
     }
   }
 
@@ -460,7 +532,10 @@ int sm_count() {
 template <class C>
 cudaError_t launch_cfg(const void* q_idx, const void* k_idx, const float* w, float scale,
                        int relu, int B, int S, int T, int q_off, float* scores,
-                       int write_masked, cudaStream_t st) {
+                       int write_masked, cudaStream_t st, const IndexerExtra* ex = nullptr) {
+  const IndexerExtra none{};
+  const IndexerExtra& x = ex ? *ex : none;
+  const int ks = x.kstride > 0 ? x.kstride : 1;
   CUtensorMap kmap, qmap;
   if (!make_map(&kmap, k_idx, (uint64_t)B * T, C::DI, kTileM, C::ES))
     return cudaErrorInvalidValue;
@@ -469,13 +544,18 @@ cudaError_t launch_cfg(const void* q_idx, const void* k_idx, const float* w, flo
   TcArgs a{};
   a.w = w; a.scores = scores; a.scale = scale; a.B = B; a.S = S; a.T = T; a.q_off = q_off;
   a.nqb = (S + C::NQ - 1) / C::NQ;
+  a.kstride = ks;
+  a.ldT = x.ldT > 0 ? x.ldT : T;
+  a.tau = x.tau; a.cand_key = x.cand_key; a.cand_t = x.cand_t; a.cand_cnt = x.cand_cnt;
+  a.cand_cap = x.cand_cap; a.run_if = x.run_if;
+  const bool filter = x.tau != nullptr;
   // total causal tiles -> chunk size giving each CTA several units
   long long tiles = 0;
   int max_nt = 1;
   for (int qb = 0; qb < a.nqb; ++qb) {
     const int s_last = S - 1 < qb * C::NQ + C::NQ - 1 ? S - 1 : qb * C::NQ + C::NQ - 1;
     const int t_last = T - 1 < s_last + q_off ? T - 1 : s_last + q_off;
-    const int nt = t_last / kTileM + 1;
+    const int nt = (t_last / kTileM) / ks + 1;
     tiles += nt;
     if (nt > max_nt) max_nt = nt;
   }
@@ -488,17 +568,21 @@ cudaError_t launch_cfg(const void* q_idx, const void* k_idx, const float* w, flo
   for (int qb = 0; qb < a.nqb; ++qb) {
     const int s_last = S - 1 < qb * C::NQ + C::NQ - 1 ? S - 1 : qb * C::NQ + C::NQ - 1;
     const int t_last = T - 1 < s_last + q_off ? T - 1 : s_last + q_off;
-    units += (t_last / kTileM + 1 + a.chunk - 1) / a.chunk;
+    units += ((t_last / kTileM) / ks + 1 + a.chunk - 1) / a.chunk;
   }
   units *= B;
   const int grid = (int)(units < nsm ? units : nsm);
-  auto kern = relu == 1 ? index_scores_tc_kernel<C, 1>
-                        : (relu == 2 ? index_scores_tc_kernel<C, 2> : index_scores_tc_kernel<C, 0>);
+  auto kern = filter ? (relu == 1 ? index_scores_tc_kernel<C, 1, true>
+                                   : (relu == 2 ? index_scores_tc_kernel<C, 2, true>
+                                                : index_scores_tc_kernel<C, 0, true>))
+                     : (relu == 1 ? index_scores_tc_kernel<C, 1, false>
+                                  : (relu == 2 ? index_scores_tc_kernel<C, 2, false>
+                                               : index_scores_tc_kernel<C, 0, false>));
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   kern<<<grid, C::THREADS, C::SMEM, st>>>(kmap, qmap, a);
   e = cudaGetLastError();
-  if (e != cudaSuccess || !write_masked) return e;
+  if (e != cudaSuccess || !write_masked || filter || ks != 1) return e;
   fill_masked_kernel<<<(unsigned)((size_t)B * S), 256, 0, st>>>(scores, S, T, q_off, C::NQ);
   return cudaGetLastError();
 }
@@ -551,14 +635,16 @@ cudaError_t launch_collapse_q(const void* q_idx, const float* w, long long rows,
 
 cudaError_t launch_index_scores_collapsed(const void* qc, const void* k_idx, float scale,
                                           int relu, int B, int S, int T, int DI, int q_off,
-                                          float* scores, int write_masked, cudaStream_t st) {
+                                          float* scores, int write_masked, cudaStream_t st,
+                                          const IndexerExtra* ex) {
   if (!index_scores_collapsed_supported(1, DI, relu)) return cudaErrorNotSupported;
+  if (ex && ex->tau) return cudaErrorNotSupported;  // the filter is a per-head epilogue
   // 128 queries x (hi, lo) = 256 columns per tile
   if (DI == 128)
     return launch_cfg<TcCfg<2, 128, 128, 16, 3, 2, true>>(qc, k_idx, nullptr, scale, relu, B, S,
-                                                          T, q_off, scores, write_masked, st);
+                                                          T, q_off, scores, write_masked, st, ex);
   return launch_cfg<TcCfg<2, 64, 128, 16, 4, 2, true>>(qc, k_idx, nullptr, scale, relu, B, S, T,
-                                                       q_off, scores, write_masked, st);
+                                                       q_off, scores, write_masked, st, ex);
 }
 
 bool index_scores_tc_supported(int dtype, int HI, int DI) {
@@ -568,33 +654,33 @@ bool index_scores_tc_supported(int dtype, int HI, int DI) {
 cudaError_t launch_index_scores_tc(const void* q_idx, const void* k_idx, const float* w,
                                    float scale, int relu, int B, int S, int T, int HI, int DI,
                                    int q_off, float* scores, int write_masked,
-                                   cudaStream_t st) {
+                                   cudaStream_t st, const IndexerExtra* ex) {
   if (!index_scores_tc_supported(1, HI, DI)) return cudaErrorNotSupported;
   if (S == 1) {  // decode: one query per batch row, N = HI, deep key pipeline
     if (HI == 32 && DI == 128)
       return launch_cfg<TcCfg<32, 128, 1, 4, 6>>(q_idx, k_idx, w, scale, relu, B, S, T, q_off,
-                                                 scores, write_masked, st);
+                                                 scores, write_masked, st, ex);
     if (HI == 32 && DI == 64)
       return launch_cfg<TcCfg<32, 64, 1, 4, 8>>(q_idx, k_idx, w, scale, relu, B, S, T, q_off,
-                                                scores, write_masked, st);
+                                                scores, write_masked, st, ex);
     if (HI == 16 && DI == 128)
       return launch_cfg<TcCfg<16, 128, 2, 4, 6>>(q_idx, k_idx, w, scale, relu, B, S, T, q_off,
-                                                 scores, write_masked, st);
+                                                 scores, write_masked, st, ex);
     return launch_cfg<TcCfg<16, 64, 2, 4, 8>>(q_idx, k_idx, w, scale, relu, B, S, T, q_off,
-                                              scores, write_masked, st);
+                                              scores, write_masked, st, ex);
   }
   if (HI == 32 && DI == 128)
     return launch_cfg<TcCfg<32, 128, 8, 16, 3>>(q_idx, k_idx, w, scale, relu, B, S, T, q_off,
-                                               scores, write_masked, st);
+                                               scores, write_masked, st, ex);
   if (HI == 32 && DI == 64)
     return launch_cfg<TcCfg<32, 64, 8, 16, 4>>(q_idx, k_idx, w, scale, relu, B, S, T, q_off,
-                                              scores, write_masked, st);
+                                              scores, write_masked, st, ex);
   if (HI == 16 && DI == 128)
     return launch_cfg<TcCfg<16, 128, 16, 16, 3>>(q_idx, k_idx, w, scale, relu, B, S, T, q_off,
-                                                scores, write_masked, st);
+                                                scores, write_masked, st, ex);
   // N = 128 columns (8 queries): four accumulators in TMEM keep the epilogue's latency hidden
   return launch_cfg<TcCfg<16, 64, 8, 16, 4, 2, false, 2, 4>>(q_idx, k_idx, w, scale, relu, B, S,
-                                                             T, q_off, scores, write_masked, st);
+                                                             T, q_off, scores, write_masked, st, ex);
 }
 
 }  // namespace dsa

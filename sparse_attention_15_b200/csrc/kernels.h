@@ -11,11 +11,24 @@ namespace dsa {
 // Sets the thread-local text returned by dsa_last_error().
 void set_last_error(const char* msg);
 
+// Options of the tensor-core indexer used by the fused indexer -> top-k.
+struct IndexerExtra {
+  int kstride = 1;        // score key tiles 0, kstride, 2*kstride, ... only (a sample)
+  long long ldT = 0;      // output row length in floats (0: T); tile kt -> columns kt*128..
+  const uint32_t* tau = nullptr;  // filter mode: per-row order-key thresholds [B*S]
+  uint32_t* cand_key = nullptr;   // [B*S, cand_cap] order keys of the candidates
+  int32_t* cand_t = nullptr;      // [B*S, cand_cap] their key positions
+  int* cand_cnt = nullptr;        // [B*S] candidates found (may exceed cand_cap), zeroed
+  int cand_cap = 0;
+  const int* run_if = nullptr;    // device flag: the launch does nothing while it is 0
+};
+
 // Indexer scores, SIMT (float32 FMA) kernel: any dtype, DI <= 128.
 cudaError_t launch_index_scores_simt(int dtype, const void* q_idx, const void* k_idx,
                                      const float* w, float scale, int relu, int B, int S,
                                      int T, int HI, int DI, int q_off, float* scores,
                                      cudaStream_t st);
+
 
 // Indexer scores on the tensor cores (tcgen05 + TMEM + TMA): bf16, DI in {64,128,...}.
 // Returns cudaErrorNotSupported for shapes it does not take.
@@ -23,7 +36,7 @@ bool index_scores_tc_supported(int dtype, int HI, int DI);
 cudaError_t launch_index_scores_tc(const void* q_idx, const void* k_idx, const float* w,
                                    float scale, int relu, int B, int S, int T, int HI, int DI,
                                    int q_off, float* scores, int write_masked,
-                                   cudaStream_t st);
+                                   cudaStream_t st, const IndexerExtra* ex = nullptr);
 
 // Indexer scores with e4m3 operands (tcgen05 kind::f8f6f4): HI in {16, 32}, DI == 128.
 bool index_scores_e4m3_supported(int HI, int DI);
@@ -41,7 +54,8 @@ cudaError_t launch_collapse_q(const void* q_idx, const float* w, long long rows,
                               void* qc, cudaStream_t st);
 cudaError_t launch_index_scores_collapsed(const void* qc, const void* k_idx, float scale,
                                           int relu, int B, int S, int T, int DI, int q_off,
-                                          float* scores, int write_masked, cudaStream_t st);
+                                          float* scores, int write_masked, cudaStream_t st,
+                                          const IndexerExtra* ex = nullptr);
 
 // Hadamard rotation of indexer inputs: out[r] = x[r] @ H / sqrt(d), d in {64, 128};
 // dtype 0 float32, 1 bf16; out may equal x.
@@ -52,12 +66,38 @@ cudaError_t launch_hadamard(int dtype, const void* x, void* out, long long rows,
 // selection bitmask, one bit per key, rows of `mask_stride` 32-bit words
 // (mask_stride >= ceil(T/32); words past the row's keys are zero).
 cudaError_t launch_topk(const float* scores, int B, int S, int T, int K, int q_off,
-                        int32_t* idx, uint32_t* mask, int mask_stride, cudaStream_t st);
+                        int32_t* idx, uint32_t* mask, int mask_stride, cudaStream_t st,
+                        const int* run_if = nullptr);
+// Fused indexer -> top-k, after the sampled indexer pass: tau[row] = the order key of the
+// r-th largest sampled score (0, i.e. keep everything, for rows of at most `cap` keys).
+cudaError_t launch_topk_tau(const float* sample, long long ld, int B, int S, int T, int K,
+                            int q_off, int kstride, int cap, uint32_t* tau, cudaStream_t st);
+// ... and after the filtered indexer pass: the exact top-k of every row from its candidate
+// list, or *fail = 1 when some row's list cannot hold it (< K or > cap candidates).
+size_t topk_candidates_smem(int T, int cap);
+cudaError_t launch_topk_candidates(const uint32_t* cand_key, const int32_t* cand_t,
+                                   const int* cand_cnt, int cap, int B, int S, int T, int K,
+                                   int q_off, int32_t* idx, uint32_t* mask, int mask_stride,
+                                   int* fail, cudaStream_t st);
 // Selection bitmask from index lists (valid, causal entries only).
 cudaError_t launch_idx_to_mask(const int32_t* idx, int B, int S, int T, int K, int q_off,
                                uint32_t* mask, int mask_stride, cudaStream_t st);
 // Words per bitmask row used by the masked-tile attention (ceil(T/128) * 4).
 inline int mask_stride_words(int T) { return ((T + 127) / 128) * 4; }
+// Tile-occupancy words per (batch row, block of 128 queries): bit j is set when some query
+// of the block selected some key of key block j (128 keys).
+inline int occ_words(int T) { return ((T + 127) / 128 + 31) / 32; }
+// Bytes of the selection mask rows plus, 256-byte aligned after them, the tile-occupancy
+// summary: the masked-tile attention's workspace.
+inline size_t masked_attn_mask_bytes(int B, int S, int T) {
+  const size_t m = ((size_t)B * S * mask_stride_words(T) * 4 + 255) & ~(size_t)255;
+  return m + (size_t)B * ((S + 127) / 128) * occ_words(T) * 4;
+}
+inline uint32_t* masked_attn_occ(uint32_t* mask, int B, int S, int T) {
+  return reinterpret_cast<uint32_t*>(
+      reinterpret_cast<uint8_t*>(mask) +
+      (((size_t)B * S * mask_stride_words(T) * 4 + 255) & ~(size_t)255));
+}
 
 // Gather attention (idx lists) and band attention (sliding window, GQA) share one kernel.
 struct AttnProblem {
@@ -87,8 +127,10 @@ cudaError_t launch_gather_attn(const AttnProblem& p, void* ws, size_t ws_bytes,
 // Dense tensor-core attention tiles under the selection bitmask (or, with idx == NULL and
 // mask == NULL, under the sliding-window band).  bf16, DQK in {128, 192}, DV == 128.
 bool masked_attn_supported(int dtype, int DQK, int DV);
+// With a mask, `occ` (masked_attn_occ of the mask buffer) receives the tile-occupancy
+// summary first, and key blocks no query of a 128-query block selected are skipped.
 cudaError_t launch_masked_attn(const AttnProblem& p, const uint32_t* mask, int mask_stride,
-                               cudaStream_t st);
+                               uint32_t* occ, cudaStream_t st);
 
 // Merge of split-key partials (unnormalised o [rows, nsplit, H, DV] float32 and (m, l)
 // [rows, nsplit, H, 2], m in log2 units) into out [rows, H, DV], gate applied.  nsplit <= 64.

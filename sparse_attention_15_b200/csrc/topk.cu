@@ -24,12 +24,6 @@ namespace {
 
 constexpr int kBins = 2048;
 
-__device__ __forceinline__ uint32_t order_key(float f) {
-  uint32_t u = __float_as_uint(f);
-  if ((u << 1) == 0u) u = 0u;  // -0.0 -> +0.0
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
 // Block-wide exclusive prefix sum of one int per thread (blockDim.x <= 1024).
 __device__ __forceinline__ int block_excl_scan(int v, int* warp_buf, int* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -76,7 +70,8 @@ __global__ void __launch_bounds__(NT) topk_rows_kernel(const float* __restrict__
                                                        int Tn, int K, int q_off,
                                                        int32_t* __restrict__ idx,
                                                        uint32_t* __restrict__ mask,
-                                                       int mask_stride) {
+                                                       int mask_stride, const int* run_if) {
+  if (run_if != nullptr && *reinterpret_cast<const volatile int*>(run_if) == 0) return;
   __shared__ uint32_t hist[padded(kBins)];
   __shared__ int warp_buf[32];
   __shared__ int scan_total;
@@ -291,7 +286,8 @@ template <int NT, bool SAMPLE>
 __global__ void __launch_bounds__(NT, NT == 256 ? 5 : (NT == 512 ? 3 : 1))
     topk_bitmap_kernel(const float* __restrict__ scores, int S, int Tn, int K, int q_off,
                        int32_t* __restrict__ idx, uint32_t* __restrict__ mask, int mask_stride,
-                       int cl_cap) {
+                       int cl_cap, const int* run_if) {
+  if (run_if != nullptr && *reinterpret_cast<const volatile int*>(run_if) == 0) return;
   extern __shared__ uint32_t dsm[];
   const int W = (Tn + 31) >> 5;              // bitmap words per row
   uint32_t* hist = dsm;                      // [padded(kBins1)]
@@ -629,6 +625,248 @@ __global__ void __launch_bounds__(NT, NT == 256 ? 5 : (NT == 512 ? 3 : 1))
     for (int wd = tid; wd < mask_stride; wd += NT) mrow[wd] = wd < nw ? selb[wd] : 0u;
 }
 
+
+// ------------------------------------------------------------------------------------
+// Fused indexer -> top-k: the threshold and the exact select over candidates.
+//
+// The top-k of a row only depends on its keys whose score is at least the row's K-th
+// largest score tau*.  If a threshold tau <= tau* is known before the row's scores exist,
+// the indexer can keep only the keys with score >= tau (its candidates) instead of writing
+// every score: when at least K keys pass, tau* >= tau, so every key of the top-k -- and
+// every key tied with the K-th -- is a candidate, and the exact select over the candidates
+// (same order: higher score, then lower index) is the top-k of the row.
+//
+// tau comes from a sample: the indexer first scores every kstride-th key tile of each row;
+// tau is the r-th largest sampled score, with r the expected sample rank of the K-th key
+// (K * n_s / n) plus a six-sigma binomial margin.  Rows with at most `cap` causal keys keep
+// every key (tau = the smallest order key).  Whether the sample was right is checked, not
+// assumed: a row with fewer than K candidates (tau too high) or more than `cap` (the list
+// overflowed) raises a flag, and the stream then runs the full-score indexer and top-k over
+// the whole launch, so the result is the same in every case.
+// ------------------------------------------------------------------------------------
+
+// Sample keys of a row with last causal key t_last: tiles j = 0..jmax at positions
+// j*kstride*128 (all full but the last).
+__device__ __forceinline__ int sample_keys(int t_last, int kstride, int* jmax) {
+  const int jm = (t_last / 128) / kstride;
+  *jmax = jm;
+  return jm * 128 + min(128, t_last + 1 - jm * kstride * 128);
+}
+
+// tau[row]: the order key of the r-th largest sampled score of the row (radix select on
+// the order keys, digits of 11, 11 and 10 bits; an early stop keeps the bucket's smallest
+// key, which is <= the r-th largest, so the threshold stays conservative).
+template <int NT>
+__global__ void __launch_bounds__(NT) topk_tau_kernel(const float* __restrict__ sample,
+                                                      long long ld, int S, int Tn, int K,
+                                                      int q_off, int kstride, int cap,
+                                                      uint32_t* __restrict__ tau) {
+  __shared__ uint32_t hist[padded(kBins)];
+  __shared__ int warp_buf[32];
+  __shared__ int scan_total;
+  __shared__ uint32_t sel_bin;
+  __shared__ int sel_above;
+  const size_t row = blockIdx.x;
+  const int s = (int)(blockIdx.x % (unsigned)S);
+  const int t_last = min(Tn - 1, s + q_off);
+  const int n = t_last + 1;
+  const int tid = threadIdx.x;
+  if (n <= cap) {  // the whole row fits the candidate list: keep every key
+    if (tid == 0) tau[row] = 0u;
+    return;
+  }
+  int jmax;
+  const int ns = sample_keys(t_last, kstride, &jmax);
+  const int m = (jmax + 1) * 128;  // sampled columns of this row
+  const float mu = (float)K * (float)ns / (float)n;
+  const int r = min(ns, (int)ceilf(mu + 6.0f * sqrtf(mu) + 8.0f));
+  const float* sc = sample + row * (size_t)ld;
+  uint32_t prefix = 0;
+  int pbits = 0, need = r;
+  const int widths[3] = {11, 11, 10};
+  for (int pass = 0; pass < 3; ++pass) {
+    const int dw = widths[pass];
+    const int shift = 32 - pbits - dw;
+    for (int i = tid; i < padded(kBins); i += NT) hist[i] = 0;
+    __syncthreads();
+    for (int i = tid; i < m; i += NT) {
+      // column i holds key (i / 128) * kstride * 128 + i % 128; columns past the row's last
+      // causal key are skipped (-inf, or never written when they lie past T)
+      if ((i >> 7) * kstride * 128 + (i & 127) > t_last) continue;
+      const uint32_t key = order_key(__ldg(sc + i));
+      const bool match = pbits == 0 || (key >> (32 - pbits)) == prefix;
+      hist_add<NT>(hist, (key >> shift) & ((1u << dw) - 1u), match);
+    }
+    __syncthreads();
+    constexpr int kPer = kBins / NT;
+    const int hi_bin = kBins - tid * kPer;
+    int local = 0;
+#pragma unroll
+    for (int q = 1; q <= kPer; ++q) local += (int)hist[hpad(hi_bin - q)];
+    int above = block_excl_scan(local, warp_buf, &scan_total);
+#pragma unroll
+    for (int q = 1; q <= kPer; ++q) {
+      const int c = (int)hist[hpad(hi_bin - q)];
+      if (above < need && above + c >= need) {
+        sel_bin = (uint32_t)(hi_bin - q);
+        sel_above = above;
+      }
+      above += c;
+    }
+    __syncthreads();
+    const uint32_t bsel = sel_bin;
+    need -= sel_above;
+    prefix = (prefix << dw) | bsel;
+    pbits += dw;
+    const bool all_taken = (int)hist[hpad(bsel)] == need;
+    __syncthreads();
+    if (all_taken) break;
+  }
+  if (tid == 0) tau[row] = pbits == 32 ? prefix : prefix << (32 - pbits);
+}
+
+// The exact top-k of a row from its candidate list (order key, key index; unordered), or
+// the fallback flag when the list cannot hold it.  Output as topk_bitmap_kernel: ascending
+// indices, -1 padding, and the selection bitmask.
+template <int NT>
+__global__ void __launch_bounds__(NT) topk_candidates_kernel(
+    const uint32_t* __restrict__ cand_key, const int32_t* __restrict__ cand_t,
+    const int* __restrict__ cand_cnt, int cap, int S, int Tn, int K, int q_off,
+    int32_t* __restrict__ idx, uint32_t* __restrict__ mask, int mask_stride,
+    int* __restrict__ fail) {
+  extern __shared__ uint32_t dsm[];
+  __shared__ int warp_buf[32];
+  __shared__ int scan_total;
+  __shared__ uint32_t sel_bin;
+  __shared__ int sel_above;
+  const size_t row = blockIdx.x;
+  const int s = (int)(blockIdx.x % (unsigned)S);
+  const int n = min(Tn, s + q_off + 1);
+  const int tid = threadIdx.x;
+  int32_t* out = idx + row * (size_t)K;
+  uint32_t* mrow = mask ? mask + row * (size_t)mask_stride : nullptr;
+  if (n <= K) {  // every valid key is kept
+    for (int i = tid; i < K; i += NT) out[i] = i < n ? i : -1;
+    if (mrow)
+      for (int wd = tid; wd < mask_stride; wd += NT) {
+        const int lo = wd * 32;
+        mrow[wd] = lo + 32 <= n ? 0xffffffffu : (lo >= n ? 0u : ((1u << (n - lo)) - 1u));
+      }
+    return;
+  }
+  const int m = __ldg(cand_cnt + row);
+  if (m < K || m > cap) {  // the threshold missed (too high) or the list overflowed
+    if (tid == 0) atomicExch(fail, 1);
+    return;
+  }
+  const int nw = (n + 31) >> 5;
+  uint32_t* hist = dsm;                     // [padded(kBins)]
+  uint32_t* ck = hist + padded(kBins);      // [cap]
+  uint32_t* ct = ck + cap;                  // [cap]
+  uint32_t* selb = ct + cap;                // [nw]
+  uint32_t* tieb = selb + nw;               // [nw]
+  const uint32_t* gk = cand_key + row * (size_t)cap;
+  const int32_t* gt = cand_t + row * (size_t)cap;
+  for (int i = tid; i < m; i += NT) {
+    ck[i] = __ldg(gk + i);
+    ct[i] = (uint32_t)__ldg(gt + i);
+  }
+  for (int wd = tid; wd < nw; wd += NT) { selb[wd] = 0u; tieb[wd] = 0u; }
+  // ---------------- radix select of the K-th largest candidate key
+  uint32_t prefix = 0;
+  int pbits = 0, need = K;
+  const int widths[3] = {11, 11, 10};
+  for (int pass = 0; pass < 3; ++pass) {
+    const int dw = widths[pass];
+    const int shift = 32 - pbits - dw;
+    for (int i = tid; i < padded(kBins); i += NT) hist[i] = 0;
+    __syncthreads();
+    for (int i = tid; i < m; i += NT) {
+      const uint32_t key = ck[i];
+      const bool match = pbits == 0 || (key >> (32 - pbits)) == prefix;
+      hist_add<NT>(hist, (key >> shift) & ((1u << dw) - 1u), match);
+    }
+    __syncthreads();
+    constexpr int kPer = kBins / NT;
+    const int hi_bin = kBins - tid * kPer;
+    int local = 0;
+#pragma unroll
+    for (int q = 1; q <= kPer; ++q) local += (int)hist[hpad(hi_bin - q)];
+    int above = block_excl_scan(local, warp_buf, &scan_total);
+#pragma unroll
+    for (int q = 1; q <= kPer; ++q) {
+      const int c = (int)hist[hpad(hi_bin - q)];
+      if (above < need && above + c >= need) {
+        sel_bin = (uint32_t)(hi_bin - q);
+        sel_above = above;
+      }
+      above += c;
+    }
+    __syncthreads();
+    const uint32_t bsel = sel_bin;
+    need -= sel_above;
+    prefix = (prefix << dw) | bsel;
+    pbits += dw;
+    const bool all_taken = (int)hist[hpad(bsel)] == need;
+    __syncthreads();
+    if (all_taken) break;
+  }
+  // ---------------- above the threshold -> SELECTED, at it -> ties
+  const int fshift = 32 - pbits;
+  for (int i = tid; i < m; i += NT) {
+    const uint32_t hi = ck[i] >> fshift, t = ct[i];
+    if (hi > prefix) atomicOr(&selb[t >> 5], 1u << (t & 31));
+    else if (hi == prefix) atomicOr(&tieb[t >> 5], 1u << (t & 31));
+  }
+  __syncthreads();
+  // ties ranked by index: the first `need` are kept.  Thread t owns words [t*per, t*per+per).
+  const int per = (nw + NT - 1) / NT;
+  {
+    int local = 0;
+    for (int q = 0; q < per; ++q) {
+      const int wd = tid * per + q;
+      if (wd < nw) local += __popc(tieb[wd]);
+    }
+    int rank = block_excl_scan(local, warp_buf, &scan_total);
+    for (int q = 0; q < per && rank < need; ++q) {
+      const int wd = tid * per + q;
+      if (wd >= nw) break;
+      uint32_t bits = tieb[wd];
+      while (bits && rank < need) {
+        const int j = __ffs(bits) - 1;
+        bits &= bits - 1u;
+        selb[wd] |= 1u << j;
+        ++rank;
+      }
+    }
+  }
+  __syncthreads();
+  // ---------------- ordered output: prefix popcounts of SELECTED
+  {
+    int local = 0;
+    for (int q = 0; q < per; ++q) {
+      const int wd = tid * per + q;
+      if (wd < nw) local += __popc(selb[wd]);
+    }
+    int pos = block_excl_scan(local, warp_buf, &scan_total);
+    for (int q = 0; q < per; ++q) {
+      const int wd = tid * per + q;
+      if (wd >= nw) break;
+      uint32_t bits = selb[wd];
+      while (bits) {
+        const int j = __ffs(bits) - 1;
+        bits &= bits - 1u;
+        if (pos < K) out[pos] = wd * 32 + j;
+        ++pos;
+      }
+    }
+    const int total = scan_total;
+    for (int i = total + tid; i < K; i += NT) out[i] = -1;
+  }
+  if (mrow)
+    for (int wd = tid; wd < mask_stride; wd += NT) mrow[wd] = wd < nw ? selb[wd] : 0u;
+}
+
 // Selection bitmask from index lists: bit t of row (b,s) is set when t appears in the row,
 // 0 <= t < T and t <= s + q_off (the causal mask).  One CTA per row.
 __global__ void idx_to_mask_kernel(const int32_t* __restrict__ idx, int S, int Tn, int K,
@@ -655,8 +893,40 @@ cudaError_t launch_idx_to_mask(const int32_t* idx, int B, int S, int T, int K, i
   return cudaGetLastError();
 }
 
+cudaError_t launch_topk_tau(const float* sample, long long ld, int B, int S, int T, int K,
+                            int q_off, int kstride, int cap, uint32_t* tau, cudaStream_t st) {
+  const size_t rows = (size_t)B * S;
+  if (rows == 0) return cudaSuccess;
+  topk_tau_kernel<256><<<(unsigned)rows, 256, 0, st>>>(sample, ld, S, T, K, q_off, kstride, cap,
+                                                       tau);
+  return cudaGetLastError();
+}
+
+size_t topk_candidates_smem(int T, int cap) {
+  const int W = (T + 31) / 32;
+  return (size_t)(padded(kBins) + 2 * cap + 2 * W) * sizeof(uint32_t);
+}
+
+cudaError_t launch_topk_candidates(const uint32_t* cand_key, const int32_t* cand_t,
+                                   const int* cand_cnt, int cap, int B, int S, int T, int K,
+                                   int q_off, int32_t* idx, uint32_t* mask, int mask_stride,
+                                   int* fail, cudaStream_t st) {
+  const size_t rows = (size_t)B * S;
+  if (rows == 0) return cudaSuccess;
+  if (mask && mask_stride < (T + 31) / 32) return cudaErrorInvalidValue;
+  const size_t smem = topk_candidates_smem(T, cap);
+  if (smem > kMaxDynSmem) return cudaErrorNotSupported;
+  cudaError_t e = cudaFuncSetAttribute((const void*)topk_candidates_kernel<256>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  topk_candidates_kernel<256><<<(unsigned)rows, 256, smem, st>>>(
+      cand_key, cand_t, cand_cnt, cap, S, T, K, q_off, idx, mask, mask_stride, fail);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_topk(const float* scores, int B, int S, int T, int K, int q_off,
-                        int32_t* idx, uint32_t* mask, int mask_stride, cudaStream_t st) {
+                        int32_t* idx, uint32_t* mask, int mask_stride, cudaStream_t st,
+                        const int* run_if) {
   const size_t rows = (size_t)B * S;
   if (rows == 0) return cudaSuccess;
   if (mask && mask_stride < (T + 31) / 32) return cudaErrorInvalidValue;
@@ -681,27 +951,27 @@ cudaError_t launch_topk(const float* scores, int B, int S, int T, int K, int q_o
     if (rows < 296 && T > 8192) {  // few long rows (decode): the widest CTA per row
       if ((e = setsmem((const void*)topk_bitmap_kernel<1024, true>)) != cudaSuccess) return e;
       topk_bitmap_kernel<1024, true><<<(unsigned)rows, 1024, smem, st>>>(
-          scores, S, T, K, q_off, idx, mask, mask_stride, cap);
+          scores, S, T, K, q_off, idx, mask, mask_stride, cap, run_if);
     } else if (T > 8192) {
       if ((e = setsmem((const void*)topk_bitmap_kernel<512, true>)) != cudaSuccess) return e;
       topk_bitmap_kernel<512, true><<<(unsigned)rows, 512, smem, st>>>(
-          scores, S, T, K, q_off, idx, mask, mask_stride, cap);
+          scores, S, T, K, q_off, idx, mask, mask_stride, cap, run_if);
     } else {
       if ((e = setsmem((const void*)topk_bitmap_kernel<256, false>)) != cudaSuccess) return e;
       topk_bitmap_kernel<256, false><<<(unsigned)rows, 256, smem, st>>>(
-          scores, S, T, K, q_off, idx, mask, mask_stride, cap);
+          scores, S, T, K, q_off, idx, mask, mask_stride, cap, run_if);
     }
     return cudaGetLastError();
   }
   if (T >= 8192)
     topk_rows_kernel<1024><<<(unsigned)rows, 1024, 0, st>>>(scores, S, T, K, q_off, idx, mask,
-                                                            mask_stride);
+                                                            mask_stride, run_if);
   else if (T >= 2048)
     topk_rows_kernel<512><<<(unsigned)rows, 512, 0, st>>>(scores, S, T, K, q_off, idx, mask,
-                                                          mask_stride);
+                                                          mask_stride, run_if);
   else
     topk_rows_kernel<256><<<(unsigned)rows, 256, 0, st>>>(scores, S, T, K, q_off, idx, mask,
-                                                          mask_stride);
+                                                          mask_stride, run_if);
   return cudaGetLastError();
 }
 

@@ -112,6 +112,32 @@ def test_topk_rejects_bad_arguments(lib):
     assert L.dsa_topk(FAKE, 1, 4, 4, 2, FAKE_MIS, None) == 2
 
 
+def test_index_topk_rejects_bad_arguments(lib):
+    L = lib.lib()
+
+    def call(**kw):
+        a = dict(dtype=1, q=FAKE, k=FAKE, w=FAKE, scale=0.0625, relu=0, B=1, S=4096, T=4096,
+                 HI=16, DI=64, K=512, idx=FAKE, ws=FAKE, wsb=1 << 40, fb=None)
+        a.update(kw)
+        return L.dsa_index_topk(a["dtype"], a["q"], a["k"], a["w"], a["scale"], a["relu"],
+                                a["B"], a["S"], a["T"], a["HI"], a["DI"], a["K"], a["idx"],
+                                a["ws"], a["wsb"], a["fb"], None)
+
+    need = L.dsa_index_topk_workspace_bytes(1, 4096, 4096, 512)
+    # sampled scores + thresholds + counters + 2 candidate lists + the fallback's scores
+    assert need >= 4096 * 4096 * 4 + 2 * 4096 * (2 * 512 + 1024) * 4
+    assert L.dsa_index_topk_workspace_bytes(0, 4096, 4096, 512) == 0
+    assert call(dtype=0) == 2                 # float32: no tensor-core indexer
+    assert call(HI=8) == 2
+    assert call(q=None) == 1
+    assert call(K=0) == 1
+    assert call(S=8192) == 1                  # T < S
+    assert call(wsb=need - 1) == 1            # workspace too small
+    assert call(ws=None) == 1
+    assert call(ws=FAKE_MIS) == 2
+    assert call(fb=FAKE_MIS) == 2
+
+
 def _attn(L, **kw):
     a = dict(dtype=1, q=FAKE, k=FAKE, v=FAKE, idx=FAKE, K=4, gate=None, gm=0, sm=0.0, B=1, S=4,
              T=8, H=4, DQK=64, DV=64, out=FAKE, ws=None, wsb=0)
@@ -140,7 +166,9 @@ def test_sparse_attn_rejects_bad_arguments(lib):
                  wsb=need - 1) == 1
     # the cost model: long prefill -> masked tile (bitmask workspace), decode -> gather
     pre = L.dsa_sparse_attn_workspace_bytes(1, 1, 4096, 4096, 20, 128, 128, 512, 0)
-    assert pre == 4096 * (4096 // 128) * 4 * 4
+    # the selection mask (one bit per key, rows padded to 128 keys) and, after it, the tile
+    # occupancy summary (one bit per 128 x 128 tile)
+    assert pre == 4096 * (4096 // 128) * 4 * 4 + (4096 // 128) * 1 * 4
     assert L.dsa_sparse_attn_workspace_bytes(1, 1, 4096, 4096, 20, 128, 128, 512, 1) == 0
 
 
@@ -246,8 +274,9 @@ def test_forward_workspace_and_validation(lib):
     a.attn_form = 1
     assert L.dsa_forward(ctypes.byref(a), FAKE, full, None) == 2  # DQK 128 is not 576
     a.H, a.DQK, a.DV, a.v = 128, 576, 512, None
-    # prefill: no split partials, and no selection bitmask (4096 rows x 4096 bits)
-    assert lib.dsa_forward_workspace_bytes(a) == full - 4096 * 4096 // 8
+    # prefill: no split partials, and no selection bitmask (4096 rows x 4096 bits) nor its
+    # tile-occupancy summary (32 query blocks x one 32-bit word, 256-byte aligned)
+    assert lib.dsa_forward_workspace_bytes(a) == full - 4096 * 4096 // 8 - 256
     a.attn_form = 3
     assert L.dsa_forward(ctypes.byref(a), FAKE, full, None) == 1
 

@@ -256,6 +256,49 @@ def test_sparse_attn_parity(name, S, T, K, gate_mode, algo):
     P.assert_attn_close(got, ref, x["q"].dtype, f"{name} {gate_mode} {algo}")
 
 
+def _clustered_selection(S, T, K, seed, empty_rows=()):
+    """Index lists clustered near the diagonal: query s selects min(K, s+1) distinct keys
+    from its most recent 2K keys, so every 128-query block selects from a few key blocks
+    and the masked-tile kernel skips the rest.  Rows in empty_rows select nothing (-1)."""
+    g = torch.Generator().manual_seed(seed)
+    q_off = T - S
+    idx = torch.full((1, S, K), -1, dtype=torch.int32)
+    for s in range(S):
+        if s in empty_rows:
+            continue
+        hi = s + q_off + 1
+        lo = max(0, hi - 2 * K)
+        k = min(K, hi - lo)
+        pick = lo + torch.randperm(hi - lo, generator=g)[:k]
+        idx[0, s, :k] = torch.sort(pick).values.to(torch.int32)
+    return idx.numpy()
+
+
+# (config, S, T, K, rows with no selection): one 128-query block with no selection at all
+# (rows 128..255) is visited through one empty block and must come out as zeros
+CLUSTERED = [("c2", 700, 700, 48, ()), ("c3", 512, 1000, 64, tuple(range(128, 256))),
+             ("c3", 300, 300, 16, (0, 5, 299))]
+
+
+@pytest.mark.parametrize("name,S,T,K,empty", CLUSTERED)
+def test_masked_tile_skips_empty_tiles(name, S, T, K, empty):
+    # clustered selections leave most (query block, key block) tiles empty: the kernel
+    # visits only the occupied ones, with the same results as the oracle's dense masked
+    # softmax over every key
+    cfg, x, g = _inputs(name, S, T)
+    idx = _clustered_selection(S, T, K, 9, empty)
+    got = dsa.dsa_sparse_attn(g["q"], g["k"], g["v"], torch.from_numpy(idx).to(DEV),
+                              gate=g["gate"], gate_mode=cfg.gate if g["gate"] is not None
+                              else None, algo="masked_tile")
+    torch.cuda.synchronize()
+    dsa.dsa_device_status(reset=True)
+    ref = O.sparse_attention(x["q"], x["k"], x["v"], idx, gate=x["gate"],
+                             gate_mode=cfg.gate if x["gate"] is not None else "off")
+    P.assert_attn_close(got, ref, x["q"].dtype, f"{name} clustered")
+    for s in empty:
+        assert not bool(got[0, s].float().abs().any()), f"row {s} has no keys: zeros"
+
+
 def _sinks(cfg, NS, seed, dtype):
     g = torch.Generator().manual_seed(seed)
     sk = torch.randn(NS, cfg.H, cfg.dqk, generator=g).to(dtype)
