@@ -124,7 +124,7 @@ dsa_status run_index_scores_collapsed(const void* qc, const void* k_idx, float s
 struct FusedLayout {
   int kstride, cap;
   long long ld;  // sampled columns per row
-  size_t qc_off, sample_off, tau_off, cnt_off, ck_off, ct_off, scores_off, total;
+  size_t qc_off, sample_off, tau_off, cnt_off, cand_off, scores_off, total;
 };
 
 FusedLayout fused_layout(int B, int S, int T, int K_eff) {
@@ -139,8 +139,7 @@ FusedLayout fused_layout(int B, int S, int T, int K_eff) {
   L.sample_off = off; off += align256(rows * (size_t)L.ld * sizeof(float));
   L.tau_off = off;    off += align256(rows * sizeof(uint32_t));
   L.cnt_off = off;    off += align256((rows + 1) * sizeof(int));  // + the fallback flag
-  L.ck_off = off;     off += align256(rows * (size_t)L.cap * sizeof(uint32_t));
-  L.ct_off = off;     off += align256(rows * (size_t)L.cap * sizeof(int32_t));
+  L.cand_off = off;   off += align256(rows * (size_t)L.cap * sizeof(uint2));
   L.scores_off = off; off += align256(rows * (size_t)T * sizeof(float));
   L.total = off;
   return L;
@@ -166,8 +165,7 @@ dsa_status run_fused_index_topk(const void* q_idx, const void* k_idx, const floa
   uint32_t* tau = reinterpret_cast<uint32_t*>(ws + L.tau_off);
   int* cnt = reinterpret_cast<int*>(ws + L.cnt_off);
   int* fail = cnt + rows;
-  uint32_t* ck = reinterpret_cast<uint32_t*>(ws + L.ck_off);
-  int32_t* ct = reinterpret_cast<int32_t*>(ws + L.ct_off);
+  uint2* cand = reinterpret_cast<uint2*>(ws + L.cand_off);
   float* scores = reinterpret_cast<float*>(ws + L.scores_off);
   cudaError_t e = cudaMemsetAsync(cnt, 0, (rows + 1) * sizeof(int), st);
   if (e != cudaSuccess) return cuda_status(e, "fused/clear");
@@ -194,14 +192,14 @@ dsa_status run_fused_index_topk(const void* q_idx, const void* k_idx, const floa
   if (e != cudaSuccess) return cuda_status(e, "fused/tau");
   // 3. every score, kept only as a candidate when it reaches its row's threshold
   dsa::IndexerExtra xf{};
-  xf.tau = tau; xf.cand_key = ck; xf.cand_t = ct; xf.cand_cnt = cnt; xf.cand_cap = L.cap;
+  xf.tau = tau; xf.cand = cand; xf.cand_cnt = cnt; xf.cand_cap = L.cap;
   e = dsa::launch_index_scores_tc(q_idx, k_idx, w, scale, (int)relu, B, S, T, HI, DI, q_off,
                                   nullptr, 0, st, &xf);
   if (e != cudaSuccess) return cuda_status(e, "fused/filter");
   if (after_indexer && (e = cudaEventRecord(after_indexer, st)) != cudaSuccess)
     return cuda_status(e, "fused/event");
   // 4. the exact top-k of every row from its candidates (or the fallback flag)
-  e = dsa::launch_topk_candidates(ck, ct, cnt, L.cap, B, S, T, K_eff, q_off, idx, mask,
+  e = dsa::launch_topk_candidates(cand, cnt, L.cap, B, S, T, K_eff, q_off, idx, mask,
                                   mask_stride, fail, st);
   if (e != cudaSuccess) return cuda_status(e, "fused/select");
   // 5. the fallback, a no-op unless some row raised the flag: full scores, full top-k
@@ -531,7 +529,7 @@ static dsa_status sparse_attn_impl(dsa_dtype dtype, const void* q, const void* k
                      "dsa_sparse_attn/mask");
     if (st != DSA_OK) return st;
     return cuda_status(dsa::launch_masked_attn(p, mask, stride,
-                                               dsa::masked_attn_occ(mask, B, S, T), s),
+                                               dsa::masked_attn_blocks(mask, B, S, T), s),
                        "dsa_sparse_attn");
   }
   return cuda_status(dsa::launch_gather_attn(p, ws, ws_bytes, s), "dsa_sparse_attn");
@@ -841,7 +839,7 @@ dsa_status dsa_forward(const dsa_forward_args* a, void* ws, size_t ws_bytes,
   }
   if (L.alg == kMasked)
     st = cuda_status(dsa::launch_masked_attn(p, mask, L.mask_stride,
-                                             dsa::masked_attn_occ(mask, B, S, T), s),
+                                             dsa::masked_attn_blocks(mask, B, S, T), s),
                      "dsa_forward/attn");
   else
     st = cuda_status(dsa::launch_gather_attn(p, attn_ws, attn_ws_bytes, s), "dsa_forward/attn");

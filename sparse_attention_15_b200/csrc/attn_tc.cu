@@ -56,8 +56,12 @@ struct AttnArgs {
   int mask_stride;       // words per mask row (multiple of 4)
   int nqb;
   int nsink;             // attention sinks (PAS), 0..128: one extra block per item
-  const uint32_t* occ;   // tile occupancy [B, nqb, occ_words] (mask mode) or NULL
-  int occ_words;
+  // the key blocks each 128-query block visits (mask mode; NULL: every causal block):
+  // bcount[b*nqb+qb] of them, in ascending order in blist[(b*nqb+qb)*nkb ...]
+  const int* bcount;
+  const uint16_t* blist;
+  int nkb;
+  int band;              // item order: 0 = heads fastest, > 0 = bands of query blocks
 };
 
 template <int DQK_, int DV_, bool BAND_>
@@ -91,10 +95,12 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
-// Item i -> (query block, batch row, head): head-major, longest query blocks first within a
-// head.  The CTAs working at the same time then walk the key blocks of one head (42 MB of
-// K/V at the 65536-token shapes), which stays in L2 while they share it, instead of every
-// head's K/V at once.
+// Item i -> (query block, batch row, head), longest query blocks first.  When every head's
+// K/V fits in L2 the heads vary fastest (a plain longest-first order, which balances the
+// CTAs best).  Otherwise (band > 0) the query blocks go in bands of `band` blocks, longest
+// band first, and within a band head by head: the CTAs working at the same time then walk
+// the key blocks of a few heads, whose K/V stays in L2 while they share it, instead of
+// every head's K/V at once; the lengths inside a band differ by at most `band` blocks.
 struct Item {
   int qb, b, h;
 };
@@ -103,14 +109,30 @@ struct Item {
 __device__ __forceinline__ int snake_item(int k, int c, int G) {
   return k * G + ((k & 1) ? (G - 1 - c) : c);
 }
-__device__ __forceinline__ Item item_of(const AttnArgs& a, int i) {
+// Items over `nq` query blocks per (batch row, head), in the order above.
+__device__ __forceinline__ Item order_item(int i, int H, int B, int nq, int band) {
   Item it;
-  const int per_head = a.B * a.nqb;
-  it.h = i / per_head;
-  const int r = i - it.h * per_head;
-  it.b = r % a.B;
-  it.qb = a.nqb - 1 - r / a.B;
+  if (band <= 0) {
+    it.h = i % H;
+    const int r = i / H;
+    it.b = r % B;
+    it.qb = nq - 1 - r / B;
+    return it;
+  }
+  const int per_band = band * B * H;  // items of one full band
+  const int bi = i / per_band;        // band index (longest first)
+  const int r0 = i - bi * per_band;
+  const int q0 = bi * band;           // first (reversed) query block of the band
+  const int nb = min(band, nq - q0);  // blocks in this band (the last may be short)
+  const int per_head = nb * B;
+  it.h = r0 / per_head;
+  const int r = r0 - it.h * per_head;
+  it.b = r % B;
+  it.qb = nq - 1 - (q0 + r / B);
   return it;
+}
+__device__ __forceinline__ Item item_of(const AttnArgs& a, int i) {
+  return order_item(i, a.H, a.B, a.nqb, a.band);
 }
 // Key blocks [j0, j1) item `it` must visit.  With attention sinks an item first visits one
 // sink block (the nsink sink entries, always visible), then those key blocks: block r of
@@ -134,49 +156,28 @@ __device__ __forceinline__ int sink_blocks(const AttnArgs& a) {
 }
 
 // Empty tiles are skipped ([AXK2] "注意力前向的骨架": under the additive sparse mask a key block
-// no query of the item selected contributes exp(-inf) = 0 to every row): with an occupancy
-// summary an item visits only the occupied key blocks of [j0, j1), in ascending order -- or,
-// when none is occupied, key block j0 alone, so that every item has a block and its outputs
-// (zeros) are written by the same path.
+// no query of the item selected contributes exp(-inf) = 0 to every row): with a block list
+// an item visits only the key blocks some query of its 128-query block selected from, in
+// ascending order (a block with no selection at all still gets one block, key block 0, so
+// that every item has one and its outputs -- zeros -- are written by the same path).
 struct KeyBlocks {
-  const uint32_t* w;  // the item's occupancy words, or NULL: every block of [j0, j1)
-  int j0, j1;
-  __device__ __forceinline__ int next_occupied(int j) const {  // first occupied >= j, or j1
-    while (j < j1) {
-      const uint32_t m = __ldg(w + (j >> 5)) >> (j & 31);
-      if (m) return min(j + __ffs(m) - 1, j1);
-      j = (j | 31) + 1;
-    }
-    return j1;
-  }
-  __device__ __forceinline__ int count() const {  // popcounts of the range's words
-    if (!w) return j1 - j0;
-    int n = 0;
-    const int w0 = j0 >> 5, w1 = (j1 - 1) >> 5;
-    for (int wi = w0; wi <= w1; ++wi) {  // independent loads
-      uint32_t m = __ldg(w + wi);
-      if (wi == w0) m &= 0xffffffffu << (j0 & 31);
-      if (wi == w1 && (j1 & 31)) m &= (1u << (j1 & 31)) - 1u;
-      n += __popc(m);
-    }
-    return n > 0 ? n : 1;
-  }
-  __device__ __forceinline__ int first() const {
-    if (!w) return j0;
-    const int j = next_occupied(j0);
-    return j < j1 ? j : j0;
-  }
-  __device__ __forceinline__ int next(int j) const {
-    return w ? next_occupied(j + 1) : j + 1;
-  }
+  const uint16_t* list;  // the item's key blocks, or NULL: every block of [j0, j1)
+  int n, j0;
+  __device__ __forceinline__ int at(int r) const { return list ? (int)__ldg(list + r) : j0 + r; }
 };
 
 __device__ __forceinline__ KeyBlocks key_blocks(const AttnArgs& a, const Item& it, int j0,
                                                 int j1) {
   KeyBlocks kb;
-  kb.w = a.occ ? a.occ + ((size_t)it.b * a.nqb + it.qb) * a.occ_words : nullptr;
   kb.j0 = j0;
-  kb.j1 = j1;
+  if (a.blist) {
+    const size_t q = (size_t)it.b * a.nqb + it.qb;
+    kb.list = a.blist + q * a.nkb;
+    kb.n = __ldg(a.bcount + q);
+  } else {
+    kb.list = nullptr;
+    kb.n = j1 - j0;
+  }
   return kb;
 }
 
@@ -262,16 +263,21 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         const int kvh = it.h / group;
         const int sb = sink_blocks<C::BAND>(a);
         const KeyBlocks kb = key_blocks(a, it, j0, j1);
-        const int nb = kb.count() + sb;
-        int jc = kb.first();  // key block of the next non-sink item block
+        const int nb = kb.n + sb;
+        // key block of position r, read from the block list one position ahead
+        int blk_next = nb > sb ? kb.at(0) : 0;
         for (int r = 0; r < nb; ++r, ++g) {
           const int st = g & 1;
-          if (g >= 2 && !mbar_wait(&empty[st], ((g >> 1) - 1) & 1)) { ok = false; break; }
-          uint8_t* dst = KVs + st * C::KV_BYTES + (kq ? 0 : C::K_BYTES);
           // the sink block reads rows 0..127 of the sink arrays (rows past nsink: zero fill)
           const bool sink = r < sb;
-          const int krow = sink ? 0 : it.b * a.T + jc * kBlk;
-          if (!sink) jc = kb.next(jc);
+          int blk = 0;
+          if (!sink) {
+            blk = blk_next;
+            if (r + 1 < nb) blk_next = kb.at(r + 1 - sb);
+          }
+          if (g >= 2 && !mbar_wait(&empty[st], ((g >> 1) - 1) & 1)) { ok = false; break; }
+          uint8_t* dst = KVs + st * C::KV_BYTES + (kq ? 0 : C::K_BYTES);
+          const int krow = sink ? 0 : it.b * a.T + blk * kBlk;
           if (kq) {
             mbar_arrive_expect_tx(&full[st], C::K_BYTES);
 #pragma unroll
@@ -326,7 +332,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         const Item it = item_of(a, i);
         int j0, j1;
         key_range<C::BAND>(a, it, &j0, &j1);
-        const int nb = key_blocks(a, it, j0, j1).count() + sink_blocks<C::BAND>(a);
+        const int nb = key_blocks(a, it, j0, j1).n + sink_blocks<C::BAND>(a);
         if (!mbar_wait(q_full, ni & 1)) { ok = false; break; }
         if (!issue_qk(g)) { ok = false; break; }
         for (int j = 0; j < nb; ++j) {
@@ -376,7 +382,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       key_range<C::BAND>(a, it, &j0, &j1);
       const int sb = sink_blocks<C::BAND>(a);
       const KeyBlocks kb = key_blocks(a, it, j0, j1);
-      const int nb = kb.count() + sb;
+      const int nb = kb.n + sb;
       const int s = it.qb * kBlk + row;
       const int spos = s + a.q_off;
       const bool row_ok = s < a.S;
@@ -384,21 +390,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           (!C::BAND && row_ok) ? a.mask + ((size_t)it.b * a.S + s) * a.mask_stride : nullptr;
       const int jfirst = (int)((grp - g) & 1u);  // first block of this group's parity
       float m_used = ninf, l = 0.f;
-      // key block of item block r >= sb, for non-decreasing r (a cursor over the visited
-      // blocks), and its 4 selection words
-      int cur_r = sb, cur_j = kb.first();
-      auto key_block = [&](int r) {
-        while (cur_r < r) {
-          cur_j = kb.next(cur_j);
-          ++cur_r;
-        }
-        return cur_j;
+      // the 4 selection words of key block `blk`
+      auto mask_words = [&](int blk) {
+        return __ldg(reinterpret_cast<const uint4*>(mrow + ((blk * kBlk) >> 5)));
       };
-      auto mask_words = [&](int r) {
-        return __ldg(reinterpret_cast<const uint4*>(mrow + ((key_block(r) * kBlk) >> 5)));
-      };
+      // The words of this group's next block are fetched one step ahead, and the index of
+      // the key block after it (from the block list) one step before that, so neither load
+      // stalls the chain from S to P.
       uint4 nb4 = make_uint4(0u, 0u, 0u, 0u);
-      if (mrow && jfirst < nb && jfirst >= sb) nb4 = mask_words(jfirst);
+      if (mrow && jfirst < nb && jfirst >= sb) nb4 = mask_words(kb.at(jfirst - sb));
+      int blk2 = (mrow && jfirst + 2 < nb) ? kb.at(jfirst + 2 - sb) : 0;
       const uint32_t o_col = C::O_COL + grp * C::DV;
       for (int j = jfirst; j < nb; j += 2) {
         const uint32_t gg = g + j;
@@ -410,10 +411,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             const int n = a.nsink - 32 * w;
             bits[w] = n >= 32 ? 0xffffffffu : (n > 0 ? (1u << n) - 1u : 0u);
           }
-          if (!C::BAND && mrow && j + 2 < nb) nb4 = mask_words(j + 2);
         } else if (!C::BAND) {
           bits[0] = nb4.x; bits[1] = nb4.y; bits[2] = nb4.z; bits[3] = nb4.w;
-          if (mrow && j + 2 < nb) nb4 = mask_words(j + 2);
+        }
+        if (!C::BAND && mrow && j + 2 < nb) {
+          nb4 = mask_words(blk2);
+          if (j + 4 < nb) blk2 = kb.at(j + 4 - sb);
         } else if (row_ok) {
           // band: spos - window < t <= spos, t < T
           const int lo = max(spos - a.window + 1, 0) - t0, hi = min(spos, a.T - 1) - t0;
@@ -598,26 +601,80 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   }
 }
 
-// The tile-occupancy summary of a selection mask: one CTA per (batch row, 128-query block);
-// thread j covers key block j (its 4 mask words in every row of the block, coalesced across
-// the threads), and each warp's 32 key blocks become one word by a ballot.
-__global__ void tile_occupancy_kernel(const uint32_t* __restrict__ mask, int mask_stride, int S,
-                                      int nqb, int nkb, uint32_t* __restrict__ occ,
-                                      int occ_words) {
+// The block list of a selection mask: one CTA per (batch row, 128-query block).  Thread j
+// looks at key block j (its 4 mask words in every row of the block, coalesced across the
+// threads, stopping at the first row that selected anything there); the occupied blocks are
+// then compacted in ascending order (a ballot per warp, a scan over the warps) into
+// list[0 .. count).  A query block that selected nothing gets the one block 0.
+__global__ void __launch_bounds__(256) block_list_kernel(const uint32_t* __restrict__ mask,
+                                                         int mask_stride, int S, int T, int q_off,
+                                                         int nqb, int nkb,
+                                                         int* __restrict__ count,
+                                                         uint16_t* __restrict__ list) {
+  // one CTA per (b, 128-query block): which causal key blocks hold a selected key of any of
+  // its rows.  G threads share a key block, each over every G-th row, eight independent row
+  // loads at a time; a thread stops at the first selected key, or once another thread has
+  // marked the block.  Blocks past the block's last causal key hold no selection and are
+  // not read.
+  extern __shared__ uint32_t occ[];
   const int b = blockIdx.x / nqb, qb = blockIdx.x % nqb;
-  const int s0 = qb * kBlk, s1 = min(S, s0 + kBlk);
+  const int s0 = qb * kBlk, rows = min(S, s0 + kBlk) - s0;
+  const int t_hi = min(T - 1, s0 + rows - 1 + q_off);
+  const int jn = t_hi < 0 ? 0 : min(nkb, t_hi / kBlk + 1);
+  const int nw = (jn + 31) >> 5;
   const uint32_t* m0 = mask + ((size_t)b * S + s0) * mask_stride;
-  uint32_t* o = occ + (size_t)blockIdx.x * occ_words;
-  for (int jb = 0; jb < occ_words * 32; jb += blockDim.x) {
-    const int j = jb + (int)threadIdx.x;
-    uint32_t any = 0u;
-    if (j < nkb)
-      for (int s = 0; s < s1 - s0 && !any; ++s) {
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(m0 + (size_t)s * mask_stride) + j);
-        any = v.x | v.y | v.z | v.w;
+  uint16_t* out = list + (size_t)blockIdx.x * nkb;
+  for (int i = threadIdx.x; i < nw; i += blockDim.x) occ[i] = 0u;
+  __syncthreads();
+  int G = 1;
+  while (G < 16 && 2 * G * jn <= (int)blockDim.x) G *= 2;
+  for (int i = threadIdx.x; i < jn * G; i += blockDim.x) {
+    const int j = i % jn, g = i / jn;
+    const uint4* col = reinterpret_cast<const uint4*>(m0) + j;
+    bool any = false;
+    for (int r0 = g; r0 < rows && !any; r0 += 8 * G) {
+      uint32_t o = 0u;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int s = r0 + k * G;
+        if (s < rows) {
+          const uint4 v = __ldg(col + (size_t)s * (mask_stride >> 2));
+          o |= v.x | v.y | v.z | v.w;
+        }
       }
-    const uint32_t word = __ballot_sync(0xffffffffu, any != 0u);
-    if ((threadIdx.x & 31) == 0 && (j >> 5) < occ_words) o[j >> 5] = word;
+      any = o != 0u;
+      if (!any && ((*(volatile uint32_t*)&occ[j >> 5] >> (j & 31)) & 1u)) break;
+    }
+    if (any) atomicOr(&occ[j >> 5], 1u << (j & 31));
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {  // warp 0 compacts the marked blocks in ascending order
+    const int lane = threadIdx.x;
+    int base = 0;
+    for (int w0 = 0; w0 < nw; w0 += 32) {
+      const int w = w0 + lane;
+      uint32_t bits = w < nw ? occ[w] : 0u;
+      const int c = __popc(bits);
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int pos = base + incl - c;
+      while (bits) {
+        out[pos++] = (uint16_t)(w * 32 + __ffs(bits) - 1);
+        bits &= bits - 1u;
+      }
+      base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) {
+      if (base == 0) {  // nothing selected: one block, every key of it masked
+        out[0] = 0;
+        base = 1;
+      }
+      count[blockIdx.x] = base;
+    }
   }
 }
 
@@ -659,7 +716,7 @@ int num_sms() {
 
 template <class C>
 cudaError_t launch_fa(const AttnProblem& p, const uint32_t* mask, int mask_stride,
-                      const uint32_t* occ, cudaStream_t st) {
+                      const int* bcount, const uint16_t* blist, cudaStream_t st) {
   CUtensorMap qm, km, vm, skm, svm;
   if (!map3d(&qm, p.q, (uint64_t)p.B * p.S, p.H, C::DQK) ||
       !map3d(&km, p.k, (uint64_t)p.B * p.T, p.HKV, C::DQK) ||
@@ -682,10 +739,15 @@ cudaError_t launch_fa(const AttnProblem& p, const uint32_t* mask, int mask_strid
   a.window = p.window; a.mask_stride = mask_stride;
   a.nsink = sinks ? p.nsink : 0;
   a.nqb = (p.S + kBlk - 1) / kBlk;
-  a.occ = occ;
-  a.occ_words = occ_words(p.T);
+  a.bcount = bcount;
+  a.blist = blist;
+  a.nkb = (p.T + kBlk - 1) / kBlk;
   const int items = p.B * p.H * a.nqb;
   const int nsm = num_sms();
+  // the K/V all items read; above the L2 size (126 MB on B200) the bands keep about four
+  // heads' K/V in use at a time
+  const double kv_bytes = (double)p.B * p.T * p.HKV * (C::DQK + C::DV) * 2.0;
+  a.band = kv_bytes > 96.0 * (1 << 20) ? (nsm / 4 > 1 ? nsm / 4 : 1) : 0;
   const int grid = items < nsm ? items : nsm;
   auto kern = masked_attn_tc_kernel<C>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -701,24 +763,30 @@ bool masked_attn_supported(int dtype, int DQK, int DV) {
 }
 
 cudaError_t launch_masked_attn(const AttnProblem& p, const uint32_t* mask, int mask_stride,
-                               uint32_t* occ, cudaStream_t st) {
+                               void* blocks, cudaStream_t st) {
   if (!masked_attn_supported(p.dtype, p.DQK, p.DV)) return cudaErrorNotSupported;
   const bool band = p.idx == nullptr && mask == nullptr;
   if (!band && mask == nullptr) return cudaErrorInvalidValue;
-  if (band) occ = nullptr;
-  if (occ != nullptr) {  // which key blocks each 128-query block selected anything from
+  const int* bcount = nullptr;
+  const uint16_t* blist = nullptr;
+  if (!band && blocks != nullptr) {  // the key blocks each 128-query block selected from
     const int nqb = (p.S + kBlk - 1) / kBlk;
     const int nkb = (p.T + kBlk - 1) / kBlk;
-    tile_occupancy_kernel<<<(unsigned)(p.B * nqb), 256, 0, st>>>(mask, mask_stride, p.S, nqb,
-                                                                nkb, occ, occ_words(p.T));
+    int* cnt = static_cast<int*>(blocks);
+    uint16_t* lst = reinterpret_cast<uint16_t*>(cnt + (size_t)p.B * nqb);
+    const size_t occ_bytes = (size_t)((nkb + 31) / 32) * sizeof(uint32_t);
+    block_list_kernel<<<(unsigned)(p.B * nqb), 256, occ_bytes, st>>>(
+        mask, mask_stride, p.S, p.T, p.q_off, nqb, nkb, cnt, lst);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+    bcount = cnt;
+    blist = lst;
   }
   if (p.DQK == 128)
-    return band ? launch_fa<FaCfg<128, 128, true>>(p, mask, mask_stride, occ, st)
-                : launch_fa<FaCfg<128, 128, false>>(p, mask, mask_stride, occ, st);
-  return band ? launch_fa<FaCfg<192, 128, true>>(p, mask, mask_stride, occ, st)
-              : launch_fa<FaCfg<192, 128, false>>(p, mask, mask_stride, occ, st);
+    return band ? launch_fa<FaCfg<128, 128, true>>(p, mask, mask_stride, bcount, blist, st)
+                : launch_fa<FaCfg<128, 128, false>>(p, mask, mask_stride, bcount, blist, st);
+  return band ? launch_fa<FaCfg<192, 128, true>>(p, mask, mask_stride, bcount, blist, st)
+              : launch_fa<FaCfg<192, 128, false>>(p, mask, mask_stride, bcount, blist, st);
 }
 
 }  // namespace dsa

@@ -57,8 +57,7 @@ struct TcArgs {
   // order key is >= tau[row] to the row's candidate list (order key, key index) -- the first
   // cand_cap of them; cand_cnt[row] counts all of them.
   const uint32_t* tau;
-  uint32_t* cand_key;
-  int32_t* cand_t;
+  uint2* cand;
   int* cand_cnt;
   int cand_cap;
   // If non-NULL, the launch does nothing unless *run_if != 0 (set on the device by an
@@ -295,10 +294,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       if (p.bal) {
         const int base = __shfl_sync(0xffffffffu, p.base, 0);
         const int pos = base + __popc(p.bal & lt_mask);
-        if (((p.bal >> lane) & 1u) && pos < a.cand_cap) {
-          a.cand_key[p.off + pos] = p.key;
-          a.cand_t[p.off + pos] = p.t;
-        }
+        if (((p.bal >> lane) & 1u) && pos < a.cand_cap)
+          a.cand[p.off + pos] = make_uint2(p.key, (uint32_t)p.t);
         p.bal = 0u;
       }
     };
@@ -546,7 +543,7 @@ cudaError_t launch_cfg(const void* q_idx, const void* k_idx, const float* w, flo
   a.nqb = (S + C::NQ - 1) / C::NQ;
   a.kstride = ks;
   a.ldT = x.ldT > 0 ? x.ldT : T;
-  a.tau = x.tau; a.cand_key = x.cand_key; a.cand_t = x.cand_t; a.cand_cnt = x.cand_cnt;
+  a.tau = x.tau; a.cand = x.cand; a.cand_cnt = x.cand_cnt;
   a.cand_cap = x.cand_cap; a.run_if = x.run_if;
   const bool filter = x.tau != nullptr;
   // total causal tiles -> chunk size giving each CTA several units

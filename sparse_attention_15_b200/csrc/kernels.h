@@ -16,8 +16,7 @@ struct IndexerExtra {
   int kstride = 1;        // score key tiles 0, kstride, 2*kstride, ... only (a sample)
   long long ldT = 0;      // output row length in floats (0: T); tile kt -> columns kt*128..
   const uint32_t* tau = nullptr;  // filter mode: per-row order-key thresholds [B*S]
-  uint32_t* cand_key = nullptr;   // [B*S, cand_cap] order keys of the candidates
-  int32_t* cand_t = nullptr;      // [B*S, cand_cap] their key positions
+  uint2* cand = nullptr;          // [B*S, cand_cap] candidates: (order key, key position)
   int* cand_cnt = nullptr;        // [B*S] candidates found (may exceed cand_cap), zeroed
   int cand_cap = 0;
   const int* run_if = nullptr;    // device flag: the launch does nothing while it is 0
@@ -75,8 +74,8 @@ cudaError_t launch_topk_tau(const float* sample, long long ld, int B, int S, int
 // ... and after the filtered indexer pass: the exact top-k of every row from its candidate
 // list, or *fail = 1 when some row's list cannot hold it (< K or > cap candidates).
 size_t topk_candidates_smem(int T, int cap);
-cudaError_t launch_topk_candidates(const uint32_t* cand_key, const int32_t* cand_t,
-                                   const int* cand_cnt, int cap, int B, int S, int T, int K,
+cudaError_t launch_topk_candidates(const uint2* cand, const int* cand_cnt, int cap, int B,
+                                   int S, int T, int K,
                                    int q_off, int32_t* idx, uint32_t* mask, int mask_stride,
                                    int* fail, cudaStream_t st);
 // Selection bitmask from index lists (valid, causal entries only).
@@ -84,19 +83,18 @@ cudaError_t launch_idx_to_mask(const int32_t* idx, int B, int S, int T, int K, i
                                uint32_t* mask, int mask_stride, cudaStream_t st);
 // Words per bitmask row used by the masked-tile attention (ceil(T/128) * 4).
 inline int mask_stride_words(int T) { return ((T + 127) / 128) * 4; }
-// Tile-occupancy words per (batch row, block of 128 queries): bit j is set when some query
-// of the block selected some key of key block j (128 keys).
-inline int occ_words(int T) { return ((T + 127) / 128 + 31) / 32; }
-// Bytes of the selection mask rows plus, 256-byte aligned after them, the tile-occupancy
-// summary: the masked-tile attention's workspace.
+// The masked-tile attention's workspace: the selection mask rows, then (256-byte aligned) its
+// block list -- per (batch row, block of 128 queries) the number of key blocks (of 128 keys)
+// any of its queries selected from, [B * nqb] int32, and those blocks in ascending order,
+// [B * nqb, nkb] uint16.
 inline size_t masked_attn_mask_bytes(int B, int S, int T) {
   const size_t m = ((size_t)B * S * mask_stride_words(T) * 4 + 255) & ~(size_t)255;
-  return m + (size_t)B * ((S + 127) / 128) * occ_words(T) * 4;
+  const size_t nqb = (size_t)((S + 127) / 128), nkb = (size_t)((T + 127) / 128);
+  return m + (size_t)B * nqb * 4 + (size_t)B * nqb * nkb * 2;
 }
-inline uint32_t* masked_attn_occ(uint32_t* mask, int B, int S, int T) {
-  return reinterpret_cast<uint32_t*>(
-      reinterpret_cast<uint8_t*>(mask) +
-      (((size_t)B * S * mask_stride_words(T) * 4 + 255) & ~(size_t)255));
+inline void* masked_attn_blocks(uint32_t* mask, int B, int S, int T) {
+  return reinterpret_cast<uint8_t*>(mask) +
+         (((size_t)B * S * mask_stride_words(T) * 4 + 255) & ~(size_t)255);
 }
 
 // Gather attention (idx lists) and band attention (sliding window, GQA) share one kernel.
@@ -127,10 +125,10 @@ cudaError_t launch_gather_attn(const AttnProblem& p, void* ws, size_t ws_bytes,
 // Dense tensor-core attention tiles under the selection bitmask (or, with idx == NULL and
 // mask == NULL, under the sliding-window band).  bf16, DQK in {128, 192}, DV == 128.
 bool masked_attn_supported(int dtype, int DQK, int DV);
-// With a mask, `occ` (masked_attn_occ of the mask buffer) receives the tile-occupancy
-// summary first, and key blocks no query of a 128-query block selected are skipped.
+// With a mask, `blocks` (masked_attn_blocks of the mask buffer) receives the block list first,
+// and key blocks no query of a 128-query block selected are skipped.
 cudaError_t launch_masked_attn(const AttnProblem& p, const uint32_t* mask, int mask_stride,
-                               uint32_t* occ, cudaStream_t st);
+                               void* blocks, cudaStream_t st);
 
 // Merge of split-key partials (unnormalised o [rows, nsplit, H, DV] float32 and (m, l)
 // [rows, nsplit, H, 2], m in log2 units) into out [rows, H, DV], gate applied.  nsplit <= 64.

@@ -66,12 +66,10 @@ __device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t digit, bool va
 }
 
 template <int NT>
-__global__ void __launch_bounds__(NT) topk_rows_kernel(const float* __restrict__ scores, int S,
-                                                       int Tn, int K, int q_off,
-                                                       int32_t* __restrict__ idx,
-                                                       uint32_t* __restrict__ mask,
-                                                       int mask_stride, const int* run_if) {
-  if (run_if != nullptr && *reinterpret_cast<const volatile int*>(run_if) == 0) return;
+__device__ __forceinline__ void topk_rows_row(const size_t row, const float* __restrict__ scores,
+                                              int S, int Tn, int K, int q_off,
+                                              int32_t* __restrict__ idx,
+                                              uint32_t* __restrict__ mask, int mask_stride) {
   __shared__ uint32_t hist[padded(kBins)];
   __shared__ int warp_buf[32];
   __shared__ int scan_total;
@@ -79,8 +77,7 @@ __global__ void __launch_bounds__(NT) topk_rows_kernel(const float* __restrict__
   __shared__ int sel_above;
   __shared__ int wgt[NT / 32], weq[NT / 32];
 
-  const size_t row = blockIdx.x;
-  const int s = (int)(blockIdx.x % (unsigned)S);  // 32-bit: rows < 2^31
+  const int s = (int)(row % (unsigned)S);  // 32-bit: rows < 2^31
   const int n = min(Tn, s + q_off + 1);
   const float* sc = scores + row * (size_t)Tn;
   int32_t* out = idx + row * (size_t)K;
@@ -192,6 +189,26 @@ __global__ void __launch_bounds__(NT) topk_rows_kernel(const float* __restrict__
   }
 }
 
+// One row per CTA iteration over rows blockIdx.x, blockIdx.x + gridDim.x, ...; with run_if,
+// nothing happens unless *run_if != 0 (the fused path's fallback).
+template <int NT, bool STRIDED>
+__global__ void __launch_bounds__(NT) topk_rows_kernel(const float* __restrict__ scores, int S,
+                                                       int Tn, int K, int q_off,
+                                                       int32_t* __restrict__ idx,
+                                                       uint32_t* __restrict__ mask,
+                                                       int mask_stride, const int* run_if,
+                                                       size_t rows) {
+  if (!STRIDED) {
+    topk_rows_row<NT>(blockIdx.x, scores, S, Tn, K, q_off, idx, mask, mask_stride);
+    return;
+  }
+  if (*reinterpret_cast<const volatile int*>(run_if) == 0) return;
+  for (size_t row = blockIdx.x; row < rows; row += gridDim.x) {
+    topk_rows_row<NT>(row, scores, S, Tn, K, q_off, idx, mask, mask_stride);
+    __syncthreads();  // shared memory is reused by the next row
+  }
+}
+
 // ------------------------------------------------------------------------------------
 // Two-read top-k with shared-memory bitmaps (rows up to kMaxBitmapKeys keys).
 //
@@ -281,13 +298,12 @@ __device__ __forceinline__ void load_keys(const float* __restrict__ sc, int n, i
     for (int e = 0; e < 4; ++e) k[u][e] = order_key(v[u][e]);
 }
 
-// Register caps keep 5 (256-thread) or 3 (512-thread) rows in flight per SM.
 template <int NT, bool SAMPLE>
-__global__ void __launch_bounds__(NT, NT == 256 ? 5 : (NT == 512 ? 3 : 1))
-    topk_bitmap_kernel(const float* __restrict__ scores, int S, int Tn, int K, int q_off,
-                       int32_t* __restrict__ idx, uint32_t* __restrict__ mask, int mask_stride,
-                       int cl_cap, const int* run_if) {
-  if (run_if != nullptr && *reinterpret_cast<const volatile int*>(run_if) == 0) return;
+__device__ __forceinline__ void topk_bitmap_row(const size_t row, const float* __restrict__ scores,
+                                                int S, int Tn, int K, int q_off,
+                                                int32_t* __restrict__ idx,
+                                                uint32_t* __restrict__ mask, int mask_stride,
+                                                int cl_cap) {
   extern __shared__ uint32_t dsm[];
   const int W = (Tn + 31) >> 5;              // bitmap words per row
   uint32_t* hist = dsm;                      // [padded(kBins1)]
@@ -300,8 +316,7 @@ __global__ void __launch_bounds__(NT, NT == 256 ? 5 : (NT == 512 ? 3 : 1))
   __shared__ int pick[3];
   __shared__ int cnt_sel, cl_n;
 
-  const size_t row = blockIdx.x;
-  const int s = (int)(blockIdx.x % (unsigned)S);  // 32-bit: rows < 2^31
+  const int s = (int)(row % (unsigned)S);  // 32-bit: rows < 2^31
   const int n = min(Tn, s + q_off + 1);
   const float* sc = scores + row * (size_t)Tn;
   int32_t* out = idx + row * (size_t)K;
@@ -626,6 +641,26 @@ __global__ void __launch_bounds__(NT, NT == 256 ? 5 : (NT == 512 ? 3 : 1))
 }
 
 
+// Register caps keep 5 (256-thread) or 3 (512-thread) rows in flight per SM.  One row per
+// CTA; the STRIDED form (the fused path's fallback) takes rows blockIdx.x, blockIdx.x +
+// gridDim.x, ... and does nothing unless *run_if != 0.
+template <int NT, bool SAMPLE, bool STRIDED>
+__global__ void __launch_bounds__(NT, NT == 256 ? 5 : (NT == 512 ? 3 : 1))
+    topk_bitmap_kernel(const float* __restrict__ scores, int S, int Tn, int K, int q_off,
+                       int32_t* __restrict__ idx, uint32_t* __restrict__ mask, int mask_stride,
+                       int cl_cap, const int* run_if, size_t rows) {
+  if (!STRIDED) {
+    topk_bitmap_row<NT, SAMPLE>(blockIdx.x, scores, S, Tn, K, q_off, idx, mask, mask_stride,
+                                cl_cap);
+    return;
+  }
+  if (*reinterpret_cast<const volatile int*>(run_if) == 0) return;
+  for (size_t row = blockIdx.x; row < rows; row += gridDim.x) {
+    topk_bitmap_row<NT, SAMPLE>(row, scores, S, Tn, K, q_off, idx, mask, mask_stride, cl_cap);
+    __syncthreads();  // shared memory is reused by the next row
+  }
+}
+
 // ------------------------------------------------------------------------------------
 // Fused indexer -> top-k: the threshold and the exact select over candidates.
 //
@@ -661,6 +696,7 @@ __global__ void __launch_bounds__(NT) topk_tau_kernel(const float* __restrict__ 
                                                       long long ld, int S, int Tn, int K,
                                                       int q_off, int kstride, int cap,
                                                       uint32_t* __restrict__ tau) {
+  extern __shared__ uint32_t row_keys[];  // [ld] order keys of the sampled row
   __shared__ uint32_t hist[padded(kBins)];
   __shared__ int warp_buf[32];
   __shared__ int scan_total;
@@ -681,6 +717,11 @@ __global__ void __launch_bounds__(NT) topk_tau_kernel(const float* __restrict__ 
   const float mu = (float)K * (float)ns / (float)n;
   const int r = min(ns, (int)ceilf(mu + 6.0f * sqrtf(mu) + 8.0f));
   const float* sc = sample + row * (size_t)ld;
+  // the row's sampled keys, read once: column i holds key (i / 128) * kstride * 128 + i % 128;
+  // columns past the row's last causal key (-inf, or never written when they lie past T)
+  // become key 0, below every real score's key, and are not counted
+  for (int i = tid; i < m; i += NT)
+    row_keys[i] = (i >> 7) * kstride * 128 + (i & 127) > t_last ? 0u : order_key(__ldg(sc + i));
   uint32_t prefix = 0;
   int pbits = 0, need = r;
   const int widths[3] = {11, 11, 10};
@@ -690,10 +731,8 @@ __global__ void __launch_bounds__(NT) topk_tau_kernel(const float* __restrict__ 
     for (int i = tid; i < padded(kBins); i += NT) hist[i] = 0;
     __syncthreads();
     for (int i = tid; i < m; i += NT) {
-      // column i holds key (i / 128) * kstride * 128 + i % 128; columns past the row's last
-      // causal key are skipped (-inf, or never written when they lie past T)
-      if ((i >> 7) * kstride * 128 + (i & 127) > t_last) continue;
-      const uint32_t key = order_key(__ldg(sc + i));
+      const uint32_t key = row_keys[i];
+      if (key == 0u) continue;  // not a sampled causal key
       const bool match = pbits == 0 || (key >> (32 - pbits)) == prefix;
       hist_add<NT>(hist, (key >> shift) & ((1u << dw) - 1u), match);
     }
@@ -730,8 +769,8 @@ __global__ void __launch_bounds__(NT) topk_tau_kernel(const float* __restrict__ 
 // indices, -1 padding, and the selection bitmask.
 template <int NT>
 __global__ void __launch_bounds__(NT) topk_candidates_kernel(
-    const uint32_t* __restrict__ cand_key, const int32_t* __restrict__ cand_t,
-    const int* __restrict__ cand_cnt, int cap, int S, int Tn, int K, int q_off,
+    const uint2* __restrict__ cand, const int* __restrict__ cand_cnt, int cap, int S, int Tn,
+    int K, int q_off,
     int32_t* __restrict__ idx, uint32_t* __restrict__ mask, int mask_stride,
     int* __restrict__ fail) {
   extern __shared__ uint32_t dsm[];
@@ -765,11 +804,11 @@ __global__ void __launch_bounds__(NT) topk_candidates_kernel(
   uint32_t* ct = ck + cap;                  // [cap]
   uint32_t* selb = ct + cap;                // [nw]
   uint32_t* tieb = selb + nw;               // [nw]
-  const uint32_t* gk = cand_key + row * (size_t)cap;
-  const int32_t* gt = cand_t + row * (size_t)cap;
+  const uint2* gc = cand + row * (size_t)cap;
   for (int i = tid; i < m; i += NT) {
-    ck[i] = __ldg(gk + i);
-    ct[i] = (uint32_t)__ldg(gt + i);
+    const uint2 c = __ldg(gc + i);
+    ck[i] = c.x;
+    ct[i] = c.y;
   }
   for (int wd = tid; wd < nw; wd += NT) { selb[wd] = 0u; tieb[wd] = 0u; }
   // ---------------- radix select of the K-th largest candidate key
@@ -893,12 +932,35 @@ cudaError_t launch_idx_to_mask(const int32_t* idx, int B, int S, int T, int K, i
   return cudaGetLastError();
 }
 
+// The bitmap top-k with its dynamic shared memory: one CTA per row, or (strided) the fused
+// path's fallback form.
+template <int NT, bool SAMPLE>
+cudaError_t launch_bitmap(bool strided, unsigned grid, size_t smem, cudaStream_t st,
+                          const float* scores, int S, int T, int K, int q_off, int32_t* idx,
+                          uint32_t* mask, int mask_stride, int cap, const int* run_if,
+                          size_t rows) {
+  auto kern = strided ? topk_bitmap_kernel<NT, SAMPLE, true>
+                      : topk_bitmap_kernel<NT, SAMPLE, false>;
+  // dynamic + static shared memory may pass the 48 KB default
+  cudaError_t e =
+      cudaFuncSetAttribute((const void*)kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, NT, smem, st>>>(scores, S, T, K, q_off, idx, mask, mask_stride, cap, run_if, rows);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_topk_tau(const float* sample, long long ld, int B, int S, int T, int K,
                             int q_off, int kstride, int cap, uint32_t* tau, cudaStream_t st) {
   const size_t rows = (size_t)B * S;
   if (rows == 0) return cudaSuccess;
-  topk_tau_kernel<256><<<(unsigned)rows, 256, 0, st>>>(sample, ld, S, T, K, q_off, kstride, cap,
-                                                       tau);
+  const size_t smem = (size_t)ld * sizeof(uint32_t);
+  if (smem > kMaxDynSmem) return cudaErrorNotSupported;
+  cudaError_t e = cudaFuncSetAttribute((const void*)topk_tau_kernel<256>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  topk_tau_kernel<256><<<(unsigned)rows, 256, smem, st>>>(sample, ld, S, T, K, q_off, kstride,
+                                                          cap, tau);
   return cudaGetLastError();
 }
 
@@ -907,8 +969,8 @@ size_t topk_candidates_smem(int T, int cap) {
   return (size_t)(padded(kBins) + 2 * cap + 2 * W) * sizeof(uint32_t);
 }
 
-cudaError_t launch_topk_candidates(const uint32_t* cand_key, const int32_t* cand_t,
-                                   const int* cand_cnt, int cap, int B, int S, int T, int K,
+cudaError_t launch_topk_candidates(const uint2* cand, const int* cand_cnt, int cap, int B,
+                                   int S, int T, int K,
                                    int q_off, int32_t* idx, uint32_t* mask, int mask_stride,
                                    int* fail, cudaStream_t st) {
   const size_t rows = (size_t)B * S;
@@ -920,7 +982,7 @@ cudaError_t launch_topk_candidates(const uint32_t* cand_key, const int32_t* cand
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   topk_candidates_kernel<256><<<(unsigned)rows, 256, smem, st>>>(
-      cand_key, cand_t, cand_cnt, cap, S, T, K, q_off, idx, mask, mask_stride, fail);
+      cand, cand_cnt, cap, S, T, K, q_off, idx, mask, mask_stride, fail);
   return cudaGetLastError();
 }
 
@@ -929,6 +991,9 @@ cudaError_t launch_topk(const float* scores, int B, int S, int T, int K, int q_o
                         const int* run_if) {
   const size_t rows = (size_t)B * S;
   if (rows == 0) return cudaSuccess;
+  // one CTA per row; a fallback launch (run_if) takes a grid of a few CTAs per SM that loop
+  // over the rows, so that it costs almost nothing when it has nothing to do
+  const unsigned grid = (unsigned)(run_if ? (rows < 148u * 4u ? rows : 148u * 4u) : rows);
   if (mask && mask_stride < (T + 31) / 32) return cudaErrorInvalidValue;
   // Bitmap kernel while its shared memory fits: the 4096-bin histogram, two bitmaps of the
   // row and a candidate list (1024 entries for short rows, 2048 for long ones, 512 when
@@ -943,35 +1008,21 @@ cudaError_t launch_topk(const float* scores, int B, int S, int T, int K, int q_o
     // one CTA per row; small CTAs so that several rows are in flight per SM (each row is a
     // chain of dependent reads and block-wide scans)
     const size_t smem = smem_for(cap);
-    // dynamic + static shared memory may pass the 48 KB default
-    auto setsmem = [&](const void* f) {
-      return cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    };
-    cudaError_t e;
-    if (rows < 296 && T > 8192) {  // few long rows (decode): the widest CTA per row
-      if ((e = setsmem((const void*)topk_bitmap_kernel<1024, true>)) != cudaSuccess) return e;
-      topk_bitmap_kernel<1024, true><<<(unsigned)rows, 1024, smem, st>>>(
-          scores, S, T, K, q_off, idx, mask, mask_stride, cap, run_if);
-    } else if (T > 8192) {
-      if ((e = setsmem((const void*)topk_bitmap_kernel<512, true>)) != cudaSuccess) return e;
-      topk_bitmap_kernel<512, true><<<(unsigned)rows, 512, smem, st>>>(
-          scores, S, T, K, q_off, idx, mask, mask_stride, cap, run_if);
-    } else {
-      if ((e = setsmem((const void*)topk_bitmap_kernel<256, false>)) != cudaSuccess) return e;
-      topk_bitmap_kernel<256, false><<<(unsigned)rows, 256, smem, st>>>(
-          scores, S, T, K, q_off, idx, mask, mask_stride, cap, run_if);
-    }
-    return cudaGetLastError();
+    const bool strided = run_if != nullptr;
+    if (rows < 296 && T > 8192)  // few long rows (decode): the widest CTA per row
+      return launch_bitmap<1024, true>(strided, grid, smem, st, scores, S, T, K, q_off, idx, mask,
+                                       mask_stride, cap, run_if, rows);
+    if (T > 8192)
+      return launch_bitmap<512, true>(strided, grid, smem, st, scores, S, T, K, q_off, idx, mask,
+                                      mask_stride, cap, run_if, rows);
+    return launch_bitmap<256, false>(strided, grid, smem, st, scores, S, T, K, q_off, idx, mask,
+                                     mask_stride, cap, run_if, rows);
   }
-  if (T >= 8192)
-    topk_rows_kernel<1024><<<(unsigned)rows, 1024, 0, st>>>(scores, S, T, K, q_off, idx, mask,
-                                                            mask_stride, run_if);
-  else if (T >= 2048)
-    topk_rows_kernel<512><<<(unsigned)rows, 512, 0, st>>>(scores, S, T, K, q_off, idx, mask,
-                                                          mask_stride, run_if);
-  else
-    topk_rows_kernel<256><<<(unsigned)rows, 256, 0, st>>>(scores, S, T, K, q_off, idx, mask,
-                                                          mask_stride, run_if);
+  const int nt = T >= 8192 ? 1024 : (T >= 2048 ? 512 : 256);
+  auto kern = nt == 1024 ? (run_if ? topk_rows_kernel<1024, true> : topk_rows_kernel<1024, false>)
+            : nt == 512  ? (run_if ? topk_rows_kernel<512, true> : topk_rows_kernel<512, false>)
+                         : (run_if ? topk_rows_kernel<256, true> : topk_rows_kernel<256, false>);
+  kern<<<grid, nt, 0, st>>>(scores, S, T, K, q_off, idx, mask, mask_stride, run_if, rows);
   return cudaGetLastError();
 }
 

@@ -166,9 +166,10 @@ def test_sparse_attn_rejects_bad_arguments(lib):
                  wsb=need - 1) == 1
     # the cost model: long prefill -> masked tile (bitmask workspace), decode -> gather
     pre = L.dsa_sparse_attn_workspace_bytes(1, 1, 4096, 4096, 20, 128, 128, 512, 0)
-    # the selection mask (one bit per key, rows padded to 128 keys) and, after it, the tile
-    # occupancy summary (one bit per 128 x 128 tile)
-    assert pre == 4096 * (4096 // 128) * 4 * 4 + (4096 // 128) * 1 * 4
+    # the selection mask (one bit per key, rows padded to 128 keys) and, after it, the block
+    # list: per 128-query block a count (int32) and up to 32 key-block numbers (uint16)
+    nqb = nkb = 4096 // 128
+    assert pre == 4096 * nkb * 4 * 4 + nqb * 4 + nqb * nkb * 2
     assert L.dsa_sparse_attn_workspace_bytes(1, 1, 4096, 4096, 20, 128, 128, 512, 1) == 0
 
 
@@ -275,8 +276,9 @@ def test_forward_workspace_and_validation(lib):
     assert L.dsa_forward(ctypes.byref(a), FAKE, full, None) == 2  # DQK 128 is not 576
     a.H, a.DQK, a.DV, a.v = 128, 576, 512, None
     # prefill: no split partials, and no selection bitmask (4096 rows x 4096 bits) nor its
-    # tile-occupancy summary (32 query blocks x one 32-bit word, 256-byte aligned)
-    assert lib.dsa_forward_workspace_bytes(a) == full - 4096 * 4096 // 8 - 256
+    # block list (32 counts and 32 x 32 block numbers, the region 256-byte aligned)
+    blocks = 32 * 4 + 32 * 32 * 2
+    assert lib.dsa_forward_workspace_bytes(a) == full - 4096 * 4096 // 8 - ((blocks + 255) // 256) * 256
     a.attn_form = 3
     assert L.dsa_forward(ctypes.byref(a), FAKE, full, None) == 1
 
