@@ -1,7 +1,8 @@
 """Build libdsa.so (all CUDA sources, sm_100a) in-tree with nvcc.
 
-Every source is compiled to relocatable device code in parallel (objects under `_build/`
-next to this file), then one nvcc call device-links them into the shared library.  The
+Every source is compiled as a whole program in parallel (objects under `_build/` next to
+this file; no relocatable device code, so ptxas applies setmaxnreg register splits), then
+one nvcc call links them into the shared library.  The
 library links the CUDA runtime statically and reaches the driver API (tensor-map encoding)
 through cudaGetDriverEntryPoint, so it loads on a machine without a GPU driver.
 """
@@ -22,8 +23,8 @@ OBJDIR = os.path.join(HERE, "_build")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMPILE_FLAGS = [*ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
-                 "--expt-relaxed-constexpr", "-rdc=true"]
-LINK_FLAGS = [*ARCH, "-Xcompiler", "-fPIC", "-shared", "-cudart", "static", "-rdc=true"]
+                 "--expt-relaxed-constexpr"]
+LINK_FLAGS = [*ARCH, "-Xcompiler", "-fPIC", "-shared", "-cudart", "static"]
 
 
 def sources():
@@ -71,7 +72,7 @@ def build(verbose: bool = False, extra_flags=None) -> str:
         fresh = (not extra_flags and os.path.exists(obj) and
                  os.path.getmtime(obj) > max(os.path.getmtime(src), hdr_time))
         if not fresh:
-            jobs.append([nvcc(), *COMPILE_FLAGS, *(extra_flags or []), "-I", INCLUDE, "-dc",
+            jobs.append([nvcc(), *COMPILE_FLAGS, *(extra_flags or []), "-I", INCLUDE, "-c",
                          "-o", obj, src])
     objs = [os.path.join(OBJDIR, os.path.basename(s)[:-3] + ".o") for s in sources()]
     if verbose:

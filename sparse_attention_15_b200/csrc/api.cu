@@ -4,7 +4,9 @@
 #include <stdarg.h>
 #include <stdio.h>
 
+#include <mutex>
 #include <string>
+#include <vector>
 
 #include "../../include/dsa.h"
 #include "checks.h"
@@ -12,7 +14,17 @@
 #include "kernels.h"
 
 namespace dsa {
-__device__ unsigned int g_status = 0;
+namespace {
+std::mutex g_status_mu;
+std::vector<const void*>& status_words() {
+  static std::vector<const void*> words;
+  return words;
+}
+}  // namespace
+void register_status_word(const void* symbol) {
+  std::lock_guard<std::mutex> lk(g_status_mu);
+  status_words().push_back(symbol);
+}
 }  // namespace dsa
 
 namespace {
@@ -331,14 +343,24 @@ dsa_status dsa_test_arm_wait_timeout(void) {
 }
 
 dsa_status dsa_device_status(int reset) {
+  std::vector<const void*> words;
+  {
+    std::lock_guard<std::mutex> lk(dsa::g_status_mu);
+    words = dsa::status_words();
+  }
   unsigned v = 0;
-  cudaError_t e = cudaMemcpyFromSymbol(&v, dsa::g_status, sizeof(v));
-  if (e != cudaSuccess) return fail(DSA_ERR_CUDA, "dsa_device_status: %s", cudaGetErrorString(e));
-  if (reset && v) {
-    unsigned z = 0;
-    e = cudaMemcpyToSymbol(dsa::g_status, &z, sizeof(z));
+  for (const void* sym : words) {  // every source file's word
+    unsigned w = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&w, sym, sizeof(w));
     if (e != cudaSuccess)
       return fail(DSA_ERR_CUDA, "dsa_device_status: %s", cudaGetErrorString(e));
+    if (reset && w) {
+      const unsigned z = 0;
+      e = cudaMemcpyToSymbol(sym, &z, sizeof(z));
+      if (e != cudaSuccess)
+        return fail(DSA_ERR_CUDA, "dsa_device_status: %s", cudaGetErrorString(e));
+    }
+    v |= w;
   }
   if (v & dsa::kStatusTimeout) return fail(DSA_ERR_TIMEOUT, "an in-kernel wait timed out");
   if (v & dsa::kStatusInternal) return fail(DSA_ERR_INTERNAL, "in-kernel check failed");

@@ -40,9 +40,15 @@ namespace {
 
 constexpr int kBlk = 128;     // queries per item = keys per block
 // Warp roles: 0..7 softmax (two groups of four: warp % 4 is the TMEM lane quadrant),
-// 8 TMA producer of Q and K, 9 MMA issuer (and TMEM owner), 10 TMA producer of V.
+// 8 TMA producer of Q and K, 9 MMA issuer (and TMEM owner), 10 TMA producer of V; warp 11
+// only completes the third warpgroup, so that the register split below applies to it.
 constexpr int kSoftWarps = 8;
 constexpr int kWarpQK = 8, kWarpMma = 9, kWarpV = 10;
+// Register split (setmaxnreg, per warpgroup): the CTA is launched with 384 threads x 168
+// registers = 64512; the two softmax warpgroups raise theirs to 216 and the control
+// warpgroup (producers, MMA issuer) lowers its to 64: 2 x 128 x 216 + 128 x 64 = 63488.
+constexpr int kRegsSoft = 216, kRegsCtl = 64;
+static_assert(2 * 128 * kRegsSoft + 128 * kRegsCtl <= 384 * 168, "register split");
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;
 
@@ -78,7 +84,7 @@ struct FaCfg {
   static constexpr int BAR_BYTES = 256;
   static constexpr int ML_BYTES = 2 * 2 * kBlk * 2 * 4;  // [buffer][group][row][m,l] floats
   static constexpr int SMEM = Q_BYTES + STAGES * KV_BYTES + BAR_BYTES + ML_BYTES + 1024;
-  static constexpr int THREADS = 32 * 11;
+  static constexpr int THREADS = 32 * 12;
   static constexpr int S_COLS = kBlk;              // fp32 columns of one S buffer
   static constexpr int O_COL = 2 * S_COLS;         // O0, O1 start after S0, S1
   static constexpr int TMEM_COLS = 512;
@@ -236,6 +242,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  if (warp >= kSoftWarps) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl));
   if (warp == kWarpQK || warp == kWarpV) {
     // ------------------------------------------------------------------ TMA producers
     // warp 0: Q blocks and K blocks; warp 2: V blocks.  K and V have separate rings: a K
@@ -363,7 +371,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       umma_commit(mma_done);
       drain_wait(mma_done, 0);
     }
-  } else if (warp < kSoftWarps) {
+  }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoft));
     // ------------------------------------------------------------------ softmax + epilogue
     // Group e (warps 4e..4e+3) owns the key blocks of parity e and accumulator O_e; thread =
     // query row (TMEM lane).  At the end of an item the two groups exchange (m, l) through
@@ -413,10 +423,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           }
         } else if (!C::BAND) {
           bits[0] = nb4.x; bits[1] = nb4.y; bits[2] = nb4.z; bits[3] = nb4.w;
-        }
-        if (!C::BAND && mrow && j + 2 < nb) {
-          nb4 = mask_words(blk2);
-          if (j + 4 < nb) blk2 = kb.at(j + 4 - sb);
         } else if (row_ok) {
           // band: spos - window < t <= spos, t < T
           const int lo = max(spos - a.window + 1, 0) - t0, hi = min(spos, a.T - 1) - t0;
@@ -428,67 +434,39 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                                                  : (((1u << (a1 - a0 + 1)) - 1u) << a0));
           }
         }
+        if (!C::BAND && mrow && j + 2 < nb) {
+          nb4 = mask_words(blk2);
+          if (j + 4 < nb) blk2 = kb.at(j + 4 - sb);
+        }
         if (!warp_wait(&s_full[gg & 1], (gg >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
         const uint32_t s_col = t_lane + (gg & 1) * C::S_COLS;
-        // pass 1: max of the selected raw scores (the scale is positive: it commutes with max);
-        // the whole row in one TMEM round trip, kept in registers for pass 2
-        float mraw = ninf;
+        // The whole row in one TMEM round trip, kept in registers; unselected keys become
+        // -inf there, once.
         uint32_t r[kBlk];
-        {
-          tmem_ld32(s_col + 0, *reinterpret_cast<uint32_t(*)[32]>(r + 0));
-          tmem_ld32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
-          tmem_ld32(s_col + 64, *reinterpret_cast<uint32_t(*)[32]>(r + 64));
-          tmem_ld32(s_col + 96, *reinterpret_cast<uint32_t(*)[32]>(r + 96));
-          tmem_wait_ld();
-          float mx[4];  // four independent chains, two keys per three-input max
+        tmem_ld32(s_col + 0, *reinterpret_cast<uint32_t(*)[32]>(r + 0));
+        tmem_ld32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
+        tmem_ld32(s_col + 64, *reinterpret_cast<uint32_t(*)[32]>(r + 64));
+        tmem_ld32(s_col + 96, *reinterpret_cast<uint32_t(*)[32]>(r + 96));
+        tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            mx[c] = ninf;
+        for (int c = 0; c < 4; ++c)
 #pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              // unselected keys become -inf here, once: pass 2 reads the masked row
-              const float x0 = (bits[c] & (1u << e)) ? __uint_as_float(r[c * 32 + e]) : ninf;
-              const float x1 =
-                  (bits[c] & (1u << (e + 1))) ? __uint_as_float(r[c * 32 + e + 1]) : ninf;
-              r[c * 32 + e] = __float_as_uint(x0);
-              r[c * 32 + e + 1] = __float_as_uint(x1);
-              mx[c] = max3(mx[c], x0, x1);
-            }
-          }
-          mraw = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-        }
-        const float mb = mraw * a.qk_scale;
-        const bool need = mb > m_used + kRescaleLog2;
-        // a raised max rescales l now and O_grp (this group's earlier blocks of the item) after
-        // pass 2, once their P V landed -- before P_j is published, so P_j V never meets an
-        // unscaled O
-        float alpha = 1.f;
-        bool rescale_o = false;
-        if (__any_sync(0xffffffffu, need)) {
-          const float m_new = need ? mb : m_used;
-          alpha = (l > 0.f) ? exp2f(m_used - m_new) : 0.f;
-          rescale_o = j >= 2 && __any_sync(0xffffffffu, need && l > 0.f);
-          if (need) {
-            l *= alpha;
-            m_used = m_new;
-          }
-        }
-        // pass 2: P = exp2(scale*s - m) for selected keys, 0 otherwise, split into bf16
-        // P_hi + P_lo (P_lo = bf16(p - P_hi) keeps ~2^-17 relative precision).
-        const float msub = m_used == ninf ? 0.f : m_used;
-        unsigned long long rs2 = pack2(0.f, 0.f);  // row sum, two partial sums
+          for (int e = 0; e < 32; ++e)
+            if (!(bits[c] & (1u << e))) r[c * 32 + e] = __float_as_uint(ninf);
         const unsigned long long scale2 = pack2(a.qk_scale, a.qk_scale);
-        const unsigned long long nm2 = pack2(-msub, -msub);
-        // 16 keys per chunk, from the row held in registers since pass 1; chunk k's P_hi and
-        // P_lo overwrite its own 16 S columns
-        auto chunk = [&](int kk) {
+        unsigned long long rs2 = pack2(0.f, 0.f);  // row sum, two partial sums
+        // 16 keys per chunk: P = exp2(scale*s - m) (0 for unselected keys), split into bf16
+        // P_hi + P_lo (P_lo = bf16(p - P_hi) keeps ~2^-17 relative precision), written over
+        // the chunk's own 16 S columns; mx collects the raw maximum on the way.
+        auto chunk = [&](int kk, unsigned long long nm2, float& mx) {
           uint32_t ph[8], pl[8];
 #pragma unroll
           for (int e2 = 0; e2 < 8; ++e2) {
             const int e = 2 * e2;
             const float x0 = __uint_as_float(r[16 * kk + e]);
             const float x1 = __uint_as_float(r[16 * kk + e + 1]);
+            mx = max3(mx, x0, x1);
             float y0, y1;
             unpack2(fma2(pack2(x0, x1), scale2, nm2), y0, y1);  // scale*s - m, two keys
             const float p0 = ex2_ftz(y0), p1 = ex2_ftz(y1);
@@ -507,8 +485,56 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           tmem_st8(s_col + kk * 16, ph);
           tmem_st8(s_col + kk * 16 + 8, pl);
         };
+        // One pass when every row of the warp already has a running max: P against it at once,
+        // the block max taken on the way.  Only a block max above the running one by more than
+        // 2^8 (rare after an item's first block) makes the block run again with the raised max,
+        // as does a first block, whose max is taken first.  Both give the same P for a row
+        // whose max stays.
+        float mraw = ninf;
+        bool again = true;
+        if (__all_sync(0xffffffffu, m_used != ninf)) {
+          const unsigned long long nm2 = pack2(-m_used, -m_used);
+          float mx[2] = {ninf, ninf};  // two chains
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) chunk(kk);
+          for (int kk = 0; kk < 8; ++kk) chunk(kk, nm2, mx[kk & 1]);
+          mraw = fmaxf(mx[0], mx[1]);
+          again = __any_sync(0xffffffffu, mraw * a.qk_scale > m_used + kRescaleLog2);
+          if (again) {
+            tmem_wait_st();  // the second pass writes the same columns
+            rs2 = pack2(0.f, 0.f);
+          }
+        } else {
+          float mx[4] = {ninf, ninf, ninf, ninf};
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int e = 0; e < 32; e += 2)
+              mx[c] = max3(mx[c], __uint_as_float(r[c * 32 + e]), __uint_as_float(r[c * 32 + e + 1]));
+          mraw = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        }
+        // a raised max rescales l now and O_grp (this group's earlier blocks of the item) after
+        // P is written, once their P V landed -- before P_j is published, so P_j V never meets
+        // an unscaled O
+        float alpha = 1.f;
+        bool rescale_o = false, need = false;
+        if (again) {
+          const float mb = mraw * a.qk_scale;
+          need = mb > m_used + kRescaleLog2;
+          if (__any_sync(0xffffffffu, need)) {
+            const float m_new = need ? mb : m_used;
+            alpha = (l > 0.f) ? exp2f(m_used - m_new) : 0.f;
+            rescale_o = j >= 2 && __any_sync(0xffffffffu, need && l > 0.f);
+            if (need) {
+              l *= alpha;
+              m_used = m_new;
+            }
+          }
+          const float msub = m_used == ninf ? 0.f : m_used;
+          const unsigned long long nm2 = pack2(-msub, -msub);
+          float mx = ninf;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) chunk(kk, nm2, mx);
+        }
         {
           float r0, r1;
           unpack2(rs2, r0, r1);
@@ -601,21 +627,18 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   }
 }
 
-// The block list of a selection mask: one CTA per (batch row, 128-query block).  Thread j
-// looks at key block j (its 4 mask words in every row of the block, coalesced across the
-// threads, stopping at the first row that selected anything there); the occupied blocks are
-// then compacted in ascending order (a ballot per warp, a scan over the warps) into
-// list[0 .. count).  A query block that selected nothing gets the one block 0.
+// The block list of a selection mask, per (batch row, 128-query block): the key blocks of 128
+// that hold a selected key of any of its queries, in ascending order, in list[0 .. count).  A
+// query block that selected nothing gets the one block 0 (every key of it masked).
 __global__ void __launch_bounds__(256) block_list_kernel(const uint32_t* __restrict__ mask,
                                                          int mask_stride, int S, int T, int q_off,
                                                          int nqb, int nkb,
                                                          int* __restrict__ count,
                                                          uint16_t* __restrict__ list) {
-  // one CTA per (b, 128-query block): which causal key blocks hold a selected key of any of
-  // its rows.  G threads share a key block, each over every G-th row, eight independent row
-  // loads at a time; a thread stops at the first selected key, or once another thread has
-  // marked the block.  Blocks past the block's last causal key hold no selection and are
-  // not read.
+  // One CTA per (b, query block).  G threads share a key block, each over every G-th row,
+  // eight independent row loads at a time; a thread stops at the first selected key, or once
+  // another thread has marked the block.  Key blocks past the query block's last causal key
+  // hold no selection and are not read.
   extern __shared__ uint32_t occ[];
   const int b = blockIdx.x / nqb, qb = blockIdx.x % nqb;
   const int s0 = qb * kBlk, rows = min(S, s0 + kBlk) - s0;
@@ -752,6 +775,12 @@ cudaError_t launch_fa(const AttnProblem& p, const uint32_t* mask, int mask_strid
   auto kern = masked_attn_tc_kernel<C>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
+  // the register split only completes if the launch holds the registers it hands out
+  static const int launch_regs = [&] {
+    cudaFuncAttributes fa{};
+    return cudaFuncGetAttributes(&fa, kern) == cudaSuccess ? fa.numRegs : 0;
+  }();
+  if (launch_regs * C::THREADS < 2 * 128 * kRegsSoft + 128 * kRegsCtl) return cudaErrorInvalidConfiguration;
   kern<<<grid, C::THREADS, C::SMEM, st>>>(qm, km, vm, skm, svm, a);
   return cudaGetLastError();
 }

@@ -11,11 +11,21 @@
 namespace dsa {
 
 // ------------------------------------------------------------------------------------
-// Per-device status word.  Kernels OR a bit in and carry on; the host reads it with
-// dsa_device_status() after synchronising.
+// Status words.  Kernels OR a bit in and carry on; the host reads them with
+// dsa_device_status() after synchronising.  Every source file is compiled as a whole
+// program (no relocatable device code, which would stop ptxas from giving the warpgroups
+// of a setmaxnreg split their own register budgets), so each one has its own word; each
+// registers it at load time and the host ORs them all.
 // ------------------------------------------------------------------------------------
 enum : unsigned { kStatusTimeout = 1u, kStatusInternal = 2u };
-extern __device__ unsigned int g_status;
+void register_status_word(const void* symbol);  // host side, defined in api.cu
+namespace {
+__device__ unsigned int g_status = 0;
+struct StatusWordRegistration {
+  StatusWordRegistration() { register_status_word(&g_status); }
+};
+const StatusWordRegistration g_status_registration;
+}  // namespace
 
 __device__ __forceinline__ void flag_status(unsigned bits) { atomicOr(&g_status, bits); }
 
