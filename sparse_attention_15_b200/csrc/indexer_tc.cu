@@ -21,9 +21,14 @@
 //   warp 1       MMA issuer (one thread): DI/16 tcgen05.mma per tile into one of two TMEM
 //                accumulators; tcgen05.commit frees the key stage and hands the
 //                accumulator to the epilogue
-//   warps 2..    epilogue (a multiple of 4 warps, so that each TMEM lane quadrant -- warp % 4 --
+//   warps 2, 3   idle (they complete the first warpgroup)
+//   warps 4..    epilogue (a multiple of 4 warps, so that each TMEM lane quadrant -- warp % 4 --
 //                has the same number of warps): tcgen05.ld of the accumulator, weighted
-//                head sum, store
+//                head sum, store.  In the per-head form each epilogue warp keeps the head
+//                weights of its columns in registers for a whole work unit: read per tile,
+//                those broadcast loads filled the load/store unit's data path (one wavefront
+//                per weight, warp and tile) and held the tensor pipe back.  setmaxnreg moves
+//                registers from the first warpgroup to the epilogue to make room.
 // A work unit is (batch row, query block, a chunk of key tiles up to the causal limit);
 // units are dealt to CTAs round-robin.  Key tiles after the last causal tile of a query
 // block are not computed: a separate fill kernel writes their -inf when asked to.
@@ -39,7 +44,11 @@ namespace dsa {
 namespace {
 
 constexpr int kTileM = 128;   // keys per tile = TMEM lanes
-constexpr int kEpiWarp0 = 2;  // first epilogue warp (warp % 4 = its TMEM lane quadrant)
+// First epilogue warp (warp % 4 = its TMEM lane quadrant): 4 when the kernel splits its
+// registers (the producer and the MMA issuer then fill a warpgroup of their own), else 2.
+template <bool SPLIT>
+constexpr int epi_warp0() { return SPLIT ? 4 : 2; }
+constexpr int kRegsCtl = 40;  // registers of the first warpgroup after the split
 
 struct TcArgs {
   const float* w;
@@ -92,7 +101,19 @@ struct TcCfg {
                                    : NACC * N <= 128 ? 128 : NACC * N <= 256 ? 256 : 512;
   static constexpr int EPI_GROUPS = NE / 4;       // epilogue warps per TMEM lane quadrant
   static constexpr int COLS_PER_WARP = N / EPI_GROUPS;
-  static constexpr int THREADS = 32 * (kEpiWarp0 + NE);
+  // the register split and the per-unit weights apply to the wide per-head prefill form
+  static constexpr bool SPLIT = !CL_ && NE_ == 16;
+  // threads of the plain kernel (split registers) and of the filter kernel (no split)
+  static constexpr int THREADS = 32 * (epi_warp0<SPLIT>() + NE);
+  static constexpr int THREADS_FILTER = 32 * (epi_warp0<false>() + NE);
+  // Registers: at launch the per-thread count the SM sub-partition with the most warps
+  // allows (ptxas launches a kernel that uses setmaxnreg with this maximum); the epilogue
+  // warpgroups then take what the first warpgroup gives up.
+  static constexpr int WARPS_PER_SMSP = (epi_warp0<SPLIT>() + NE + 3) / 4;
+  static constexpr int REGS_LAUNCH_RAW = 16384 / (32 * WARPS_PER_SMSP);
+  static constexpr int REGS_LAUNCH = (REGS_LAUNCH_RAW > 255 ? 255 : REGS_LAUNCH_RAW) & ~7;
+  static constexpr int REGS_EPI_RAW = (REGS_LAUNCH * THREADS - 128 * kRegsCtl) / (32 * NE);
+  static constexpr int REGS_EPI = (REGS_EPI_RAW > 248 ? 248 : REGS_EPI_RAW) & ~7;
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM = NA * A_BYTES + NB * B_BYTES + BAR_BYTES + 1024;
   static_assert(N % 16 == 0 && N >= 16 && N <= 256, "UMMA N");
@@ -137,7 +158,7 @@ struct UnitIter {
 };
 
 template <class C, int RELU, bool FILTER>
-__global__ void __launch_bounds__(C::THREADS, 1)
+__global__ void __launch_bounds__(FILTER ? C::THREADS_FILTER : C::THREADS, 1)
     index_scores_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                            const __grid_constant__ CUtensorMap qmap, const TcArgs a) {
   // a launch kept for a fallback that was not needed: every thread leaves at once
@@ -182,230 +203,31 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      UnitIter it(cta);
-      uint32_t ai = 0, bi = 0;
-      bool ok = true;
-      while (ok && it.next(a, C::NQ, ncta)) {
-        const int bb = bi % C::NB;
-        if (bi >= (uint32_t)C::NB && !mbar_wait(&b_empty[bb], ((bi / C::NB) - 1) & 1)) {
-          ok = false;
-          break;
-        }
-        mbar_arrive_expect_tx(&b_full[bb], C::B_BYTES);
-        const int qrow = (it.b * a.S + it.qb * C::NQ) * C::HI;
-#pragma unroll
-        for (int kh = 0; kh < C::KH; ++kh)
-          tma_load_2d(Bs + bb * C::B_BYTES + kh * C::B_SLICE, &qmap, kh * C::SLICE_ELEMS, qrow,
-                      &b_full[bb]);
-        ++bi;
-        for (int kt = it.k0; kt < it.k1; ++kt) {
-          const int st = ai % C::NA;
-          if (ai >= (uint32_t)C::NA && !mbar_wait(&a_empty[st], ((ai / C::NA) - 1) & 1)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&a_full[st], C::A_BYTES);
-          const int krow = it.b * a.T + kt * a.kstride * kTileM;
-#pragma unroll
-          for (int kh = 0; kh < C::KH; ++kh)
-            tma_load_2d(As + st * C::A_BYTES + kh * C::A_SLICE, &kmap, kh * C::SLICE_ELEMS, krow,
-                        &a_full[st]);
-          ++ai;
-        }
+  constexpr bool kSplit = C::SPLIT && !FILTER;
+  constexpr int kEpiWarp0 = epi_warp0<kSplit>();
+  // The roles.  With the register split the producer and the MMA issuer run inside the
+  // first warpgroup's branch, after its setmaxnreg (ptxas gives a warpgroup its own budget
+  // only for code under that instruction); without it the flat dispatch lets ptxas
+  // allocate the filter form without spills.
+  if constexpr (kSplit) {
+    if (warp < kEpiWarp0) {
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl));
+      if (warp == 0) {
+#include "indexer_tc_producer.cuh"
+      } else if (warp == 1) {
+#include "indexer_tc_mma.cuh"
       }
-      // on the way out, let every copy this thread issued land
-      for (uint32_t j = (ai > (uint32_t)C::NA ? ai - C::NA : 0); j < ai; ++j)
-        drain_wait(&a_full[j % C::NA], (j / C::NA) & 1);
-      for (uint32_t j = (bi > (uint32_t)C::NB ? bi - C::NB : 0); j < bi; ++j)
-        drain_wait(&b_full[j % C::NB], (j / C::NB) & 1);
+    } else {
+      asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::REGS_EPI));
+#include "indexer_tc_epilogue.cuh"
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc =
-          C::ES == 2 ? idesc_bf16_f32(kTileM, C::N) : idesc_e4m3_f32(kTileM, C::N);
-      UnitIter it(cta);
-      uint32_t ai = 0, bi = 0, ci = 0;
-      bool ok = true;
-      while (ok && it.next(a, C::NQ, ncta)) {
-        const int bb = bi % C::NB;
-        if (!mbar_wait(&b_full[bb], (bi / C::NB) & 1)) { ok = false; break; }
-        const uint32_t b_base = smem_u32(Bs + bb * C::B_BYTES);
-        for (int kt = it.k0; kt < it.k1; ++kt) {
-          const int st = ai % C::NA;
-          if (!mbar_wait(&a_full[st], (ai / C::NA) & 1)) { ok = false; break; }
-          const int ab = ci % C::NACC;
-          if (ci >= (uint32_t)C::NACC &&
-              !mbar_wait(&acc_empty[ab], ((ci / C::NACC) - 1) & 1)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t a_base = smem_u32(As + st * C::A_BYTES);
-#pragma unroll
-          for (int kk = 0; kk < C::ROW_BYTES / 32; ++kk) {
-            const uint32_t off = (kk & 3) * 32;  // 32 B (16 bf16 / 32 e4m3) along the row
-            const uint64_t adesc = sw128_kmajor_desc(a_base + (kk >> 2) * C::A_SLICE + off);
-            const uint64_t bdesc = sw128_kmajor_desc(b_base + (kk >> 2) * C::B_SLICE + off);
-            if constexpr (C::ES == 2)
-              umma_f16_ss(tmem + ab * C::ACC_COLS, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
-            else
-              umma_f8f6f4_ss(tmem + ab * C::ACC_COLS, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
-          }
-          umma_commit(&a_empty[st]);
-          umma_commit(&acc_full[ab]);
-          ++ai;
-          ++ci;
-        }
-        if (!ok) break;
-        umma_commit(&b_empty[bb]);
-        ++bi;
-      }
-      umma_commit(mma_done);
-      drain_wait(mma_done, 0);
-    }
-  } else if (warp >= kEpiWarp0) {
-    // ------------------------------------------------------------------ epilogue
-    const int ew = warp - kEpiWarp0;
-    const int quad = warp & 3;
-    const int group = ew >> 2;
-    const int col0 = group * C::COLS_PER_WARP;
-    const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
-    const float ninf = __int_as_float(0xff800000);
-    UnitIter it(cta);
-    uint32_t ci = 0;
-    bool ok = true;
-    // Filter mode: the candidates of each of this warp's queries found in one key tile are
-    // written when that query comes round again in the next tile (or at the end of the
-    // unit): the list position comes from a global atomicAdd issued when the scores are
-    // ready, and its round trip overlaps the next tile's work instead of stalling this one.
-    constexpr int QW = C::CL ? 1 : (C::COLS_PER_WARP / C::HI);  // queries per warp and tile
-    struct Pending {
-      uint32_t bal, key;
-      int t, base;
-      size_t off;
-    };
-    Pending pend[QW];
-    uint32_t tau_q[QW];
-#pragma unroll
-    for (int q = 0; q < QW; ++q) pend[q].bal = 0u;
-    const uint32_t lt_mask = (1u << lane) - 1u;
-    auto flush = [&](Pending& p) {  // p.bal is warp-uniform
-      if (p.bal) {
-        const int base = __shfl_sync(0xffffffffu, p.base, 0);
-        const int pos = base + __popc(p.bal & lt_mask);
-        if (((p.bal >> lane) & 1u) && pos < a.cand_cap)
-          a.cand[p.off + pos] = make_uint2(p.key, (uint32_t)p.t);
-        p.bal = 0u;
-      }
-    };
-    while (ok && it.next(a, C::NQ, ncta)) {
-      const int s_base = it.qb * C::NQ;
-      if constexpr (FILTER) {
-#pragma unroll
-        for (int q = 0; q < QW; ++q) {
-          flush(pend[q]);
-          const int sq = s_base + col0 / C::HI + q;
-          tau_q[q] = sq < a.S ? __ldg(a.tau + (size_t)it.b * a.S + sq) : 0xffffffffu;
-        }
-      }
-      // the head weights of this unit's queries (1-2 KB) are the same for every key tile and
-      // every lane: the reduction reads them as warp-wide broadcast float4 loads, which stay
-      // in L1 for the whole unit (one load per four heads, no shuffles)
-      const float4* wunit = C::CL ? nullptr : reinterpret_cast<const float4*>(
-          a.w + ((size_t)it.b * a.S + s_base) * C::HI);
-      for (int kt = it.k0; kt < it.k1; ++kt) {
-        const int ab = ci % C::NACC;
-        if (!warp_wait(&acc_full[ab], (ci / C::NACC) & 1)) { ok = false; break; }
-        tc_fence_after();
-        const int tcol = kt * kTileM + quad * 32 + lane;  // output column
-        const int t = kt * a.kstride * kTileM + quad * 32 + lane;  // key position
-        constexpr int NCH = C::COLS_PER_WARP / 16;
-        // double-buffered 16-column TMEM reads: chunk cc+1 is in flight while chunk cc is
-        // reduced.  A query's HI columns span HI/16 chunks; its four FMA chains carry over.
-        uint32_t rb[2][16];
-        tmem_ld16(t_lane + ab * C::ACC_COLS + col0, rb[0]);
-        tmem_wait_ld();
-        // four independent FMA chains (heads h % 4) as two packed float32 pairs
-        unsigned long long acc01 = pack2(0.f, 0.f), acc23 = pack2(0.f, 0.f);
-#pragma unroll
-        for (int cc = 0; cc < NCH; ++cc) {
-          if (cc + 1 < NCH) {
-            tmem_ld16(t_lane + ab * C::ACC_COLS + col0 + (cc + 1) * 16, rb[(cc + 1) & 1]);
-          } else {
-            // every column of this accumulator has been read: hand it back to the MMA
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[ab]);
-          }
-          const uint32_t* r = rb[cc & 1];
-          const int c0 = col0 + cc * 16;     // first column of the chunk
-          if constexpr (C::CL) {
-            // eight queries per chunk: score = scale * (D[t, hi] + D[t, lo])
-            const int sq = s_base + c0 / 2;
-            float* op = a.scores + ((size_t)it.b * a.S + sq) * a.ldT + tcol;
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              if (sq + q < a.S && t < a.T) {
-                float v = (__uint_as_float(r[2 * q]) + __uint_as_float(r[2 * q + 1])) * a.scale;
-                if (RELU == 1) v = fmaxf(v, 0.f);
-                op[(size_t)q * a.ldT] = (t <= sq + q + a.q_off) ? v : ninf;
-              }
-            }
-          } else {
-            const int j = c0 / C::HI;          // query within the block
-            const int s = s_base + j;
-            if (s < a.S) {  // ragged tail of the last block (warp-uniform)
-#pragma unroll
-              for (int h = 0; h < 16; h += 4) {
-                const float4 w4 = __ldg(wunit + (c0 + h) / 4);
-                float d0 = __uint_as_float(r[h + 0]);
-                float d1 = __uint_as_float(r[h + 1]);
-                float d2 = __uint_as_float(r[h + 2]);
-                float d3 = __uint_as_float(r[h + 3]);
-                if (RELU == 2) {
-                  d0 = fmaxf(d0, 0.f); d1 = fmaxf(d1, 0.f); d2 = fmaxf(d2, 0.f);
-                  d3 = fmaxf(d3, 0.f);
-                }
-                acc01 = fma2(pack2(w4.x, w4.y), pack2(d0, d1), acc01);
-                acc23 = fma2(pack2(w4.z, w4.w), pack2(d2, d3), acc23);
-              }
-              if ((c0 + 16) % C::HI == 0) {  // the query's last chunk: finish and store
-                float a0, a1, a2, a3;
-                unpack2(acc01, a0, a1);
-                unpack2(acc23, a2, a3);
-                float v = ((a0 + a1) + (a2 + a3)) * a.scale;
-                if (RELU == 1) v = fmaxf(v, 0.f);
-                const size_t row = (size_t)it.b * a.S + s;
-                if constexpr (FILTER) {
-                  // candidates of this query among the warp's 32 keys: one atomic per warp,
-                  // the writes deferred to this query's next tile
-                  Pending& p = pend[(cc * 16) / C::HI];  // compile-time slot
-                  flush(p);
-                  const uint32_t key = order_key(v);
-                  const bool keep =
-                      t < a.T && t <= s + a.q_off && key >= tau_q[(cc * 16) / C::HI];
-                  p.bal = __ballot_sync(0xffffffffu, keep);
-                  p.key = key;
-                  p.t = t;
-                  p.off = row * (size_t)a.cand_cap;
-                  p.base = 0;
-                  if (p.bal && lane == 0) p.base = atomicAdd(a.cand_cnt + row, __popc(p.bal));
-                } else if (t < a.T) {
-                  a.scores[row * a.ldT + tcol] = (t <= s + a.q_off) ? v : ninf;
-                }
-                acc01 = acc23 = pack2(0.f, 0.f);
-              }
-            }
-          }
-          if (cc + 1 < NCH) tmem_wait_ld();
-        }
-        ++ci;
-      }
-    }
-    if constexpr (FILTER) {
-#pragma unroll
-      for (int q = 0; q < QW; ++q) flush(pend[q]);
+  } else {
+    if (warp == 0) {
+#include "indexer_tc_producer.cuh"
+    } else if (warp == 1) {
+#include "indexer_tc_mma.cuh"
+    } else if (warp >= kEpiWarp0) {
+#include "indexer_tc_epilogue.cuh"
     }
   }
 
@@ -577,7 +399,15 @@ cudaError_t launch_cfg(const void* q_idx, const void* k_idx, const float* w, flo
                                                : index_scores_tc_kernel<C, 0, false>));
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<grid, C::THREADS, C::SMEM, st>>>(kmap, qmap, a);
+  if (C::SPLIT && !filter) {
+    // the register split only completes if the launch holds the registers it hands out
+    cudaFuncAttributes fa{};
+    e = cudaFuncGetAttributes(&fa, kern);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs * C::THREADS < 128 * kRegsCtl + 32 * C::NE * C::REGS_EPI)
+      return cudaErrorInvalidConfiguration;
+  }
+  kern<<<grid, filter ? C::THREADS_FILTER : C::THREADS, C::SMEM, st>>>(kmap, qmap, a);
   e = cudaGetLastError();
   if (e != cudaSuccess || !write_masked || filter || ks != 1) return e;
   fill_masked_kernel<<<(unsigned)((size_t)B * S), 256, 0, st>>>(scores, S, T, q_off, C::NQ);
