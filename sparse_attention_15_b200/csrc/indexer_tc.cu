@@ -126,9 +126,14 @@ struct TcCfg {
   static_assert(ES == 2 || (ES == 1 && !CL), "e4m3 operands: per-head form only");
 };
 
-// This CTA's work units.  Unit u = (b * nqb + qb) * max_chunks + c covers key tiles
+// This CTA's work units.  Unit u = c * (B * nqb) + (b * nqb + qb) covers key tiles
 // [c*chunk, min(ntiles(qb), (c+1)*chunk)); units with c >= chunks(qb) are empty and
-// skipped.  CTA i takes u = i, i + G, i + 2G, ... (decoded directly, no scan).
+// skipped.  CTA i takes u = i, i + G, i + 2G, ... (decoded directly, no scan).  The order is
+// chunk-major: the non-empty units of a layer c are a contiguous run of query blocks, which
+// the stride G spreads evenly over the CTAs, and the CTAs working together read the same
+// key tiles.  (With the chunk index fastest, G = 148 -- a multiple of 4, as max_chunks
+// often is -- gave CTA i only the chunks c = i mod 4, ..., and the CTAs holding the late
+// chunks, which only the long query blocks have, ran out of work early.)
 struct UnitIter {
   long long u;
   int b = 0, qb = 0, k0 = 0, k1 = 0;
@@ -140,10 +145,11 @@ struct UnitIter {
   }
   // Next non-empty unit owned by this CTA; false when done.
   __device__ __forceinline__ bool next(const TcArgs& a, int NQ, int ncta) {
-    const long long total = (long long)a.B * a.nqb * a.max_chunks;
+    const long long nbq = (long long)a.B * a.nqb;
+    const long long total = nbq * a.max_chunks;
     for (; u < total; u += ncta) {
-      const int c = (int)(u % a.max_chunks);
-      const long long bq = u / a.max_chunks;
+      const int c = (int)(u / nbq);
+      const long long bq = u - (long long)c * nbq;
       qb = (int)(bq % a.nqb);
       b = (int)(bq / a.nqb);
       const int nt = ntiles(a, qb, NQ);
