@@ -40,15 +40,21 @@ namespace {
 
 constexpr int kBlk = 128;     // queries per item = keys per block
 // Warp roles: 0..7 softmax (two groups of four: warp % 4 is the TMEM lane quadrant),
-// 8 TMA producer of Q and K, 9 MMA issuer (and TMEM owner), 10 TMA producer of V; warp 11
-// only completes the third warpgroup, so that the register split below applies to it.
+// 8 TMA producer of Q and K, 9 MMA issuer (and TMEM owner), 10 TMA producer of V (warp 11
+// only completes that warpgroup), 12..15 the output epilogue of each item (one thread per
+// query row): the softmax groups hand over their (m, l) and go on to the next item while
+// the epilogue reads O out.  In band mode (items of a few key blocks, whose epilogue is on
+// the path to the next item's first P V) the two softmax groups write the output themselves,
+// each half of the columns, and warps 12..15 idle.
 constexpr int kSoftWarps = 8;
 constexpr int kWarpQK = 8, kWarpMma = 9, kWarpV = 10;
-// Register split (setmaxnreg, per warpgroup): the CTA is launched with 384 threads x 168
-// registers = 64512; the two softmax warpgroups raise theirs to 216 and the control
-// warpgroup (producers, MMA issuer) lowers its to 64: 2 x 128 x 216 + 128 x 64 = 63488.
-constexpr int kRegsSoft = 216, kRegsCtl = 64;
-static_assert(2 * 128 * kRegsSoft + 128 * kRegsCtl <= 384 * 168, "register split");
+constexpr int kEpiWarp0 = 12;
+// Register split (setmaxnreg, per warpgroup): the CTA is launched with 512 threads x 128
+// registers = 65536; the two softmax warpgroups raise theirs and the control and epilogue
+// warpgroups lower theirs.
+constexpr int kRegsSoft = 192, kRegsCtl = 64, kRegsEpi = 64;
+static_assert(2 * 128 * kRegsSoft + 128 * kRegsCtl + 128 * kRegsEpi <= 512 * 128,
+              "register split");
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;
 
@@ -84,7 +90,7 @@ struct FaCfg {
   static constexpr int BAR_BYTES = 256;
   static constexpr int ML_BYTES = 2 * 2 * kBlk * 2 * 4;  // [buffer][group][row][m,l] floats
   static constexpr int SMEM = Q_BYTES + STAGES * KV_BYTES + BAR_BYTES + ML_BYTES + 1024;
-  static constexpr int THREADS = 32 * 12;
+  static constexpr int THREADS = 32 * 16;
   static constexpr int S_COLS = kBlk;              // fp32 columns of one S buffer
   static constexpr int O_COL = 2 * S_COLS;         // O0, O1 start after S0, S1
   static constexpr int TMEM_COLS = 512;
@@ -208,11 +214,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   uint64_t* p_full = bars + 10;      // [2]
   uint64_t* pv_done = bars + 12;     // [2] (one phase per block of that parity)
   uint64_t* o_empty = bars + 14;     // 1 (one phase per item)
-  uint64_t* ml_full = bars + 15;     // 1 (one phase per item)
   uint64_t* mma_done = bars + 16;    // 1
   uint64_t* v_full = bars + 17;      // [2] V block landed
   uint64_t* v_empty = bars + 19;     // [2] V block consumed by O += P V
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 21);
+  uint64_t* ml_full = bars + 22;     // [2] (m, l) of item ni in buffer ni & 1 written
+  uint64_t* ml_empty = bars + 24;    // [2] ... and read by the epilogue
   float* ml = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + C::BAR_BYTES);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -228,7 +235,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       mbar_init(&p_full[i], 4);
     }
     mbar_init(&pv_done[0], 1); mbar_init(&pv_done[1], 1);
-    mbar_init(o_empty, 8); mbar_init(ml_full, 8 * 32); mbar_init(mma_done, 1);
+    // o_empty: the four epilogue warps, or in band mode the eight softmax warps
+    mbar_init(o_empty, C::BAND ? 8 : 4); mbar_init(mma_done, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&ml_full[i], 8 * 32);
+      mbar_init(&ml_empty[i], 4 * 32);
+    }
     fence_mbar_init();
     prefetch_tmap(&qmap); prefetch_tmap(&kmap); prefetch_tmap(&vmap);
     if (sink_blocks<C::BAND>(a)) { prefetch_tmap(&skmap); prefetch_tmap(&svmap); }
@@ -242,7 +254,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp >= kSoftWarps) {
+  if (warp >= kSoftWarps && warp < kEpiWarp0) {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl));
   if (warp == kWarpQK || warp == kWarpV) {
     // ------------------------------------------------------------------ TMA producers
@@ -372,12 +384,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       drain_wait(mma_done, 0);
     }
   }
-  } else {
+  } else if (warp < kSoftWarps) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoft));
-    // ------------------------------------------------------------------ softmax + epilogue
+    // ------------------------------------------------------------------ softmax
     // Group e (warps 4e..4e+3) owns the key blocks of parity e and accumulator O_e; thread =
-    // query row (TMEM lane).  At the end of an item the two groups exchange (m, l) through
-    // shared memory and each writes half of the output columns.
+    // query row (TMEM lane).  At the end of an item each group leaves its (m, l) in shared
+    // memory for the epilogue warps and goes on with the next item.
     const int grp = warp >> 2;
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
@@ -561,20 +573,118 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         if (lane == 0) mbar_arrive(&p_full[gg & 1]);
       }
       if (!ok) break;
-      // ---------------- epilogue: merge the two groups, normalise, gate, bf16 store
-      const int jlast = ((nb - 1 - jfirst) >= 0) ? jfirst + ((nb - 1 - jfirst) & ~1) : -1;
-      if (jlast >= 0) {
-        const uint32_t gl = g + jlast;
-        if (!warp_wait(&pv_done[gl & 1], (gl >> 1) & 1)) { ok = false; break; }
+      if constexpr (!C::BAND) {
+        // hand this group's (m, l) to the epilogue warps; buffer ni & 1 was last read for
+        // item ni - 2 (a group without blocks in an item must not run further ahead)
+        const int mbuf = (int)(ni & 1);
+        if (ni >= 2 && !warp_wait(&ml_empty[mbuf], ((ni >> 1) - 1) & 1)) { ok = false; break; }
+        float* mlb = ml + mbuf * (2 * kBlk * 2);
+        mlb[(grp * kBlk + row) * 2 + 0] = m_used;
+        mlb[(grp * kBlk + row) * 2 + 1] = l;
+        mbar_arrive(&ml_full[mbuf]);
+      } else {
+        // Band items are a few key blocks long and their output epilogue is on the path to
+        // the next item's first P V: the two groups merge and store it themselves, each
+        // half of the columns (the epilogue warps stay idle).
+        const int jlast = ((nb - 1 - jfirst) >= 0) ? jfirst + ((nb - 1 - jfirst) & ~1) : -1;
+        if (jlast >= 0) {
+          const uint32_t gl = g + jlast;
+          if (!warp_wait(&pv_done[gl & 1], (gl >> 1) & 1)) { ok = false; break; }
+        }
+        float* mlb = ml + (ni & 1) * (2 * kBlk * 2);
+        mlb[(grp * kBlk + row) * 2 + 0] = m_used;
+        mlb[(grp * kBlk + row) * 2 + 1] = l;
+        mbar_arrive(&ml_full[0]);
+        if (!warp_wait(&ml_full[0], ni & 1)) { ok = false; break; }
+        tc_fence_after();
+        const float m0 = mlb[(0 * kBlk + row) * 2], l0 = mlb[(0 * kBlk + row) * 2 + 1];
+        const float m1 = mlb[(1 * kBlk + row) * 2], l1 = mlb[(1 * kBlk + row) * 2 + 1];
+        const float M = fmaxf(m0, m1);
+        const float a0 = l0 > 0.f ? exp2f(m0 - M) : 0.f;
+        const float a1 = l1 > 0.f ? exp2f(m1 - M) : 0.f;
+        const float L = l0 * a0 + l1 * a1;
+        float f = L > 0.f ? 1.0f / L : 0.f;
+        if (a.gate && row_ok)
+          f *= gate_act(__bfloat162float(static_cast<const __nv_bfloat16*>(
+                            a.gate)[((size_t)it.b * a.S + s) * a.H + it.h]),
+                        a.gate_mode);
+        const float w0 = a0 * f, w1 = a1 * f;
+        __nv_bfloat16* orow = a.out + (((size_t)it.b * a.S + s) * a.H + it.h) * C::DV;
+        // this group writes output columns [grp*DV/2, (grp+1)*DV/2)
+#pragma unroll 1
+        for (int c = 0; c < C::DV / 64; ++c) {
+          const int col = grp * (C::DV / 2) + c * 32;
+          uint32_t r0[32], r1[32];
+          tmem_ld32(t_lane + C::O_COL + col, r0);
+          tmem_ld32(t_lane + C::O_COL + C::DV + col, r1);
+          tmem_wait_ld();
+          if (row_ok) {
+            uint4 v4[4];
+            uint32_t* vw = reinterpret_cast<uint32_t*>(v4);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              // an O buffer with no weight (l = 0) may hold stale values: select, never multiply
+              const float y0 = (a0 > 0.f ? __uint_as_float(r0[2 * e]) * w0 : 0.f) +
+                               (a1 > 0.f ? __uint_as_float(r1[2 * e]) * w1 : 0.f);
+              const float y1 = (a0 > 0.f ? __uint_as_float(r0[2 * e + 1]) * w0 : 0.f) +
+                               (a1 > 0.f ? __uint_as_float(r1[2 * e + 1]) * w1 : 0.f);
+              const __nv_bfloat162 h2 = __floats2bfloat162_rn(y0, y1);
+              vw[e] = *reinterpret_cast<const uint32_t*>(&h2);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(orow + col);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dst[e] = v4[e];
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(o_empty);
       }
-      float* mlb = ml + (ni & 1) * (2 * kBlk * 2);
-      mlb[(grp * kBlk + row) * 2 + 0] = m_used;
-      mlb[(grp * kBlk + row) * 2 + 1] = l;
-      mbar_arrive(ml_full);
-      if (!warp_wait(ml_full, ni & 1)) { ok = false; break; }
+      g += nb;
+    }
+  } else {
+    // every warpgroup takes part in the register split (the softmax's setmaxnreg.inc waits
+    // for the registers the others give back), in band mode too, where these warps idle
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsEpi));
+    if constexpr (!C::BAND) {
+    // ------------------------------------------------------------------ output epilogue
+    // Thread = query row (TMEM lane).  Per item: wait for the last P V of each group and for
+    // the groups' (m, l); merge, normalise, gate, store bf16; free O for the next item.
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
+    uint32_t g = 0, ni = 0;
+    bool ok = true;
+    for (int kk_ = 0, i = snake_item(0, blockIdx.x, gridDim.x); ok && i < n_items;
+         i = snake_item(++kk_, blockIdx.x, gridDim.x), ++ni) {
+      const Item it = item_of(a, i);
+      int j0, j1;
+      key_range<C::BAND>(a, it, &j0, &j1);
+      const int nb = key_blocks(a, it, j0, j1).n + sink_blocks<C::BAND>(a);
+      const int s = it.qb * kBlk + row;
+      const bool row_ok = s < a.S;
+      // First the groups' (m, l): a group hands them over after publishing its last P, by
+      // which time the P V of its block before that has completed (its S needed the Q K^T
+      // issued after that P V), so each pv_done barrier below is at most at the phase
+      // waited for -- waited for earlier, a barrier one phase behind would pass on the
+      // parity of the phase before.
+      const int mbuf = (int)(ni & 1);
+      if (!warp_wait(&ml_full[mbuf], (ni >> 1) & 1)) { ok = false; break; }
+      // the last block of each parity (group): its P V completes that group's O
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int jf = (int)((e - g) & 1u);
+        if (jf < nb) {
+          const uint32_t gl = g + jf + ((nb - 1 - jf) & ~1);
+          if (!warp_wait(&pv_done[gl & 1], (gl >> 1) & 1)) { ok = false; break; }
+        }
+      }
+      if (!ok) break;
       tc_fence_after();
+      const float* mlb = ml + mbuf * (2 * kBlk * 2);
       const float m0 = mlb[(0 * kBlk + row) * 2], l0 = mlb[(0 * kBlk + row) * 2 + 1];
       const float m1 = mlb[(1 * kBlk + row) * 2], l1 = mlb[(1 * kBlk + row) * 2 + 1];
+      mbar_arrive(&ml_empty[mbuf]);
       const float M = fmaxf(m0, m1);
       const float a0 = l0 > 0.f ? exp2f(m0 - M) : 0.f;
       const float a1 = l1 > 0.f ? exp2f(m1 - M) : 0.f;
@@ -586,19 +696,18 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                       a.gate_mode);
       const float w0 = a0 * f, w1 = a1 * f;
       __nv_bfloat16* orow = a.out + (((size_t)it.b * a.S + s) * a.H + it.h) * C::DV;
-      // this group writes output columns [grp*DV/2, (grp+1)*DV/2)
 #pragma unroll 1
-      for (int c = 0; c < C::DV / 64; ++c) {
-        const int col = grp * (C::DV / 2) + c * 32;
-        uint32_t r0[32], r1[32];
-        tmem_ld32(t_lane + C::O_COL + col, r0);
-        tmem_ld32(t_lane + C::O_COL + C::DV + col, r1);
+      for (int c = 0; c < C::DV / 16; ++c) {
+        const int col = c * 16;
+        uint32_t r0[16], r1[16];
+        tmem_ld16(t_lane + C::O_COL + col, r0);
+        tmem_ld16(t_lane + C::O_COL + C::DV + col, r1);
         tmem_wait_ld();
         if (row_ok) {
-          uint4 v4[4];
+          uint4 v4[2];
           uint32_t* vw = reinterpret_cast<uint32_t*>(v4);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
+          for (int e = 0; e < 8; ++e) {
             // an O buffer with no weight (l = 0) may hold stale values: select, never multiply
             const float y0 = (a0 > 0.f ? __uint_as_float(r0[2 * e]) * w0 : 0.f) +
                              (a1 > 0.f ? __uint_as_float(r1[2 * e]) * w1 : 0.f);
@@ -608,14 +717,15 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             vw[e] = *reinterpret_cast<const uint32_t*>(&h2);
           }
           uint4* dst = reinterpret_cast<uint4*>(orow + col);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) dst[e] = v4[e];
+          dst[0] = v4[0];
+          dst[1] = v4[1];
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(o_empty);
       g += nb;
+    }
     }
   }
 
@@ -780,7 +890,8 @@ cudaError_t launch_fa(const AttnProblem& p, const uint32_t* mask, int mask_strid
     cudaFuncAttributes fa{};
     return cudaFuncGetAttributes(&fa, kern) == cudaSuccess ? fa.numRegs : 0;
   }();
-  if (launch_regs * C::THREADS < 2 * 128 * kRegsSoft + 128 * kRegsCtl) return cudaErrorInvalidConfiguration;
+  if (launch_regs * C::THREADS < 2 * 128 * kRegsSoft + 128 * kRegsCtl + 128 * kRegsEpi)
+    return cudaErrorInvalidConfiguration;
   kern<<<grid, C::THREADS, C::SMEM, st>>>(qm, km, vm, skm, svm, a);
   return cudaGetLastError();
 }

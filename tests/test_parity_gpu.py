@@ -468,6 +468,31 @@ def test_gpu_invariants_gate_zero_halves_and_determinism():
     assert torch.equal(dsa.dsa_sparse_attn(g["q"], k2, v2, idx), base)
 
 
+def test_masked_tile_deterministic_over_many_short_items():
+    # Many items per CTA, most of them short: every item boundary hands O and (m, l) from the
+    # softmax groups to the epilogue warps while the next item starts.  Three runs must agree
+    # bit for bit, both in the selection form (c2 shapes, 640 items of 1..32 key blocks) and
+    # in the band form (window 512: five key blocks per item, 2048 items).
+    cfg, x, g = _inputs("c2", 4096, 4096)
+    sc = dsa.dsa_index_scores(g["q_idx"], g["k_idx"], g["w"], cfg.scale)
+    idx = dsa.dsa_topk(sc, cfg.K)
+    runs = [dsa.dsa_sparse_attn(g["q"], g["k"], g["v"], idx, algo="masked_tile")
+            for _ in range(3)]
+    assert torch.equal(runs[0], runs[1]) and torch.equal(runs[0], runs[2])
+    c5 = get_config("c5")
+    w = swa_inputs(c5, 1, device=DEV, S=8192, T=8192)
+    outs = [dsa.dsa_window_attn(w["q"], w["k"], w["v"], c5.window, gate=w["gate"],
+                                algo="masked_tile") for _ in range(3)]
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
+    torch.cuda.synchronize()
+    for s in (0, 511, 512, 4097, 8191):
+        lo = max(0, s - c5.window + 1)
+        ref = O.window_attention(w["q"][:, s:s + 1].cpu(), w["k"][:, lo:s + 1].cpu(),
+                                 w["v"][:, lo:s + 1].cpu(), c5.window,
+                                 gate=w["gate"][:, s:s + 1].cpu(), gate_mode="sigmoid")
+        P.assert_attn_close(outs[0][:, s:s + 1], ref, torch.bfloat16, f"swa s={s}")
+
+
 # ------------------------------------------------------------------------------- full size
 def _full_inputs(name, B=None):
     cfg = get_config(name)
