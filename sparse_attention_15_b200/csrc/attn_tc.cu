@@ -209,13 +209,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   uint64_t* q_full = bars;           // 1
   uint64_t* q_empty = bars + 1;      // 1
   uint64_t* k_full = bars + 2;       // [2] K block landed
-  uint64_t* s_full = bars + 6;       // [2] S = Q K^T of the block done (its K stage free)
+  uint64_t* k_empty = bars + 4;      // [2] K block consumed by S = Q K^T
+  uint64_t* s_full = bars + 6;       // [2]
   uint64_t* p_full = bars + 10;      // [2]
-  uint64_t* pv_done = bars + 12;     // [2] P V of the block done (its V stage free);
-                                     // one phase per block of that parity
+  uint64_t* pv_done = bars + 12;     // [2] (one phase per block of that parity)
   uint64_t* o_empty = bars + 14;     // 1 (one phase per item)
   uint64_t* mma_done = bars + 16;    // 1
   uint64_t* v_full = bars + 17;      // [2] V block landed
+  uint64_t* v_empty = bars + 19;     // [2] V block consumed by O += P V
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 21);
   uint64_t* ml_full = bars + 22;     // [2] (m, l) of item ni in buffer ni & 1 written
   uint64_t* ml_empty = bars + 24;    // [2] ... and read by the epilogue
@@ -228,8 +229,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1); mbar_init(q_empty, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&k_full[i], 1);
-      mbar_init(&v_full[i], 1);
+      mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1);
+      mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1);
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 4);
     }
@@ -264,9 +265,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     if (lane == 0) {
       uint32_t g = 0, ni = 0;
       bool ok = true;
-      // a K stage is free once the S of its block is done, a V stage once its P V is
       uint64_t* full = kq ? k_full : v_full;
-      uint64_t* empty = kq ? s_full : pv_done;
+      uint64_t* empty = kq ? k_empty : v_empty;
       for (int kk_ = 0, i = snake_item(0, blockIdx.x, gridDim.x); ok && i < n_items;
            i = snake_item(++kk_, blockIdx.x, gridDim.x), ++ni) {
         const Item it = item_of(a, i);
@@ -344,6 +344,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                       kd + (uint64_t)(off >> 4), idesc_qk, kk > 0 ? 1u : 0u);
         }
         umma_commit(&s_full[gg & 1]);
+        umma_commit(&k_empty[st]);
         return true;
       };
       for (int kk_ = 0, i = snake_item(0, blockIdx.x, gridDim.x); ok && i < n_items;
@@ -360,9 +361,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           if (j + 1 == nb) umma_commit(q_empty);  // Q free once the last S is computed
           if (!mbar_wait(&p_full[gg & 1], (gg >> 1) & 1)) { ok = false; break; }
           if (j == 0 && ni > 0 && !mbar_wait(o_empty, (ni - 1) & 1)) { ok = false; break; }
-          // V_gg: in the selection form the softmax group waited for it before publishing
-          // P_gg; the band form's items are short and their softmax chain is the critical one
-          if (C::BAND && !mbar_wait(&v_full[gg & 1], (gg >> 1) & 1)) { ok = false; break; }
+          if (!mbar_wait(&v_full[gg & 1], (gg >> 1) & 1)) { ok = false; break; }
           tc_fence_after();
           const uint64_t vd = vdesc0 + (uint64_t)(((gg & 1) * C::KV_BYTES) >> 4);
           const uint32_t p_tmem = tmem + (gg & 1) * C::S_COLS;
@@ -376,6 +375,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             umma_f16_ts(o_tmem, p_tmem + pc, vdesc, idesc_pv, (j >= 2 || kk > 0) ? 1u : 0u);
             umma_f16_ts(o_tmem, p_tmem + pc + 8, vdesc, idesc_pv, 1u);
           }
+          umma_commit(&v_empty[gg & 1]);
           umma_commit(&pv_done[gg & 1]);
         }
         g += nb;
@@ -569,12 +569,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
         tmem_wait_st();
         tc_fence_before();
-        // Selection form: P_gg is published only once V_gg has landed, so the MMA thread --
-        // the critical resource on long items -- waits on one barrier per P V instead of two.
-        // V_gg was requested when P V_{gg-2} finished, well before P_gg is ready, so this
-        // costs the softmax nothing.  (Folding the wait for the group's next K block in the
-        // same way delayed P: that K stage frees only when this block's S is done.)
-        if (!C::BAND && !warp_wait(&v_full[gg & 1], (gg >> 1) & 1)) { ok = false; break; }
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[gg & 1]);
       }
@@ -883,10 +877,10 @@ cudaError_t launch_fa(const AttnProblem& p, const uint32_t* mask, int mask_strid
   a.nkb = (p.T + kBlk - 1) / kBlk;
   const int items = p.B * p.H * a.nqb;
   const int nsm = num_sms();
-  // the K/V all items read; above the L2 size (126 MB on B200) the bands keep about four
-  // heads' K/V in use at a time
+  // the K/V all items read; above the L2 size (126 MB on B200) the bands (half as many
+  // query blocks as SMs) keep about two heads' K/V in use at a time
   const double kv_bytes = (double)p.B * p.T * p.HKV * (C::DQK + C::DV) * 2.0;
-  a.band = kv_bytes > 96.0 * (1 << 20) ? (nsm / 4 > 1 ? nsm / 4 : 1) : 0;
+  a.band = kv_bytes > 96.0 * (1 << 20) ? (nsm / 2 > 1 ? nsm / 2 : 1) : 0;
   const int grid = items < nsm ? items : nsm;
   auto kern = masked_attn_tc_kernel<C>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
