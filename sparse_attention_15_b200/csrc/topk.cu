@@ -52,6 +52,48 @@ __device__ __forceinline__ int block_excl_scan(int v, int* warp_buf, int* total)
   return warp_buf[warp] + x - v;
 }
 
+// The same scan over two ints per thread at once (one pair of barriers for both).  The block
+// totals go through shared memory (*total_s): every thread reads them after the last barrier.
+__device__ __forceinline__ void block_excl_scan2(int v0, int v1, int2* warp_buf2, int2* total_s,
+                                                 int* ex0, int* ex1, int* total0, int* total1) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+  int x0 = v0, x1 = v1;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y0 = __shfl_up_sync(0xffffffffu, x0, o);
+    const int y1 = __shfl_up_sync(0xffffffffu, x1, o);
+    if (lane >= o) {
+      x0 += y0;
+      x1 += y1;
+    }
+  }
+  if (lane == 31) warp_buf2[warp] = make_int2(x0, x1);
+  __syncthreads();
+  if (warp == 0) {
+    const int2 wv = lane < nwarps ? warp_buf2[lane] : make_int2(0, 0);
+    int s0 = wv.x, s1 = wv.y;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y0 = __shfl_up_sync(0xffffffffu, s0, o);
+      const int y1 = __shfl_up_sync(0xffffffffu, s1, o);
+      if (lane >= o) {
+        s0 += y0;
+        s1 += y1;
+      }
+    }
+    if (lane < nwarps) warp_buf2[lane] = make_int2(s0 - wv.x, s1 - wv.y);
+    if (lane == 31) *total_s = make_int2(s0, s1);
+  }
+  __syncthreads();
+  const int2 off = warp_buf2[warp];
+  const int2 tot = *total_s;
+  *ex0 = off.x + x0 - v0;
+  *ex1 = off.y + x1 - v1;
+  *total0 = tot.x;
+  *total1 = tot.y;
+}
+
 // Histogram bins are stored with one padding word per 32 bins, so that the contiguous runs
 // of 1..16 bins each thread scans in find_bucket start in distinct banks.
 constexpr int padded(int nbins) { return nbins + nbins / 32; }
@@ -260,6 +302,31 @@ __device__ __forceinline__ void find_bucket(const uint32_t* hist, int need, int*
   }
 }
 
+// find_bucket for two ranks need_a <= need_b over one scan: writes the bins holding the
+// need_a-th and the need_b-th largest keys to *bin_a, *bin_b (shared; callers pass a barrier
+// before reading them).
+template <int NT, int NBINS>
+__device__ __forceinline__ void find_bucket2(const uint32_t* hist, int need_a, int need_b,
+                                             int* warp_buf, int* scan_total, int* bin_a,
+                                             int* bin_b) {
+  constexpr int per = NBINS / NT;
+  const int hi_bin = NBINS - threadIdx.x * per;
+  int c[per];
+  int local = 0;
+#pragma unroll
+  for (int q = 0; q < per; ++q) {
+    c[q] = (int)hist[hpad(hi_bin - 1 - q)];
+    local += c[q];
+  }
+  int above = block_excl_scan(local, warp_buf, scan_total);
+#pragma unroll
+  for (int q = 0; q < per; ++q) {
+    if (above < need_a && above + c[q] >= need_a) *bin_a = hi_bin - 1 - q;
+    if (above < need_b && above + c[q] >= need_b) *bin_b = hi_bin - 1 - q;
+    above += c[q];
+  }
+}
+
 // Reserves c consecutive slots per lane in a shared list; returns this lane's first slot.
 __device__ __forceinline__ int warp_reserve(int c, int* counter) {
   const int lane = threadIdx.x & 31;
@@ -312,6 +379,8 @@ __device__ __forceinline__ void topk_bitmap_row(const size_t row, const float* _
   uint32_t* cl_key = candb + W;              // [cl_cap] candidate keys
   uint32_t* cl_idx = cl_key + cl_cap;        // [cl_cap] candidate positions
   __shared__ int warp_buf[32];
+  __shared__ int2 warp_buf2[32];
+  __shared__ int2 scan_total2;
   __shared__ int scan_total;
   __shared__ int pick[3];
   __shared__ int cnt_sel, cl_n;
@@ -454,12 +523,9 @@ __device__ __forceinline__ void topk_bitmap_row(const size_t row, const float* _
     const float ks = (float)K * (float)ns / (float)n;
     const int delta = (int)(3.0f * sqrtf(ks) + 2.0f);
     const int r_hi = max(1, (int)ks - delta), r_lo = min(ns, (int)ks + delta + 1);
-    find_bucket<NT, kBins1>(hist, r_hi, warp_buf, &scan_total, pick);
+    find_bucket2<NT, kBins1>(hist, r_hi, r_lo, warp_buf, &scan_total, &pick[0], &pick[1]);
     __syncthreads();
-    const uint32_t b_hi = (uint32_t)pick[0];
-    find_bucket<NT, kBins1>(hist, r_lo, warp_buf, &scan_total, pick);
-    __syncthreads();
-    const uint32_t b_lo = (uint32_t)pick[0];
+    const uint32_t b_hi = (uint32_t)pick[0], b_lo = (uint32_t)pick[1];
     for (int i = tid; i < padded(kBins1); i += NT) hist[i] = 0u;
     read2(b_lo, b_hi);  // ends with a barrier: the histogram is clear
     const int nsel = cnt_sel, ncand = cl_n;
@@ -592,40 +658,39 @@ __device__ __forceinline__ void topk_bitmap_row(const size_t row, const float* _
     }
   }
   __syncthreads();
-  // ties ranked by index: the first `need` are kept.  Thread t owns words [t*per, t*per+per).
+  // Ordered output.  Thread t owns words [t*per, t*per+per); one scan gives, per thread, the
+  // selected keys and the ties before its words.  Ties are ranked by index: the first `need`
+  // are kept, so a thread keeps its first max(0, min(ties, need - ties before)) ties, and
+  // its first output slot is (selected before) + min(ties before, need).  The mask row gets
+  // the same words.
   const int per = (nw + NT - 1) / NT;
   {
-    int local = 0;
+    int lsel = 0, ltie = 0;
     for (int q = 0; q < per; ++q) {
       const int wd = tid * per + q;
-      if (wd < nw) local += __popc(candb[wd]);
-    }
-    int rank = block_excl_scan(local, warp_buf, &scan_total);
-    for (int q = 0; q < per && rank < need; ++q) {
-      const int wd = tid * per + q;
-      if (wd >= nw) break;
-      uint32_t bits = candb[wd];
-      while (bits && rank < need) {
-        const int j = __ffs(bits) - 1;
-        bits &= bits - 1u;
-        selb[wd] |= 1u << j;
-        ++rank;
+      if (wd < nw) {
+        lsel += __popc(selb[wd]);
+        ltie += __popc(candb[wd]);
       }
     }
-  }
-  __syncthreads();
-  // ---------------- ordered output: prefix popcounts of SELECTED
-  {
-    int local = 0;
-    for (int q = 0; q < per; ++q) {
-      const int wd = tid * per + q;
-      if (wd < nw) local += __popc(selb[wd]);
-    }
-    int pos = block_excl_scan(local, warp_buf, &scan_total);
+    int sel_before, tie_before, sel_total, tie_total;
+    block_excl_scan2(lsel, ltie, warp_buf2, &scan_total2, &sel_before, &tie_before, &sel_total,
+                     &tie_total);
+    const int kneed = max(need, 0);
+    int keep = max(0, min(ltie, kneed - tie_before));
+    int pos = sel_before + min(tie_before, kneed);
     for (int q = 0; q < per; ++q) {
       const int wd = tid * per + q;
       if (wd >= nw) break;
-      uint32_t bits = selb[wd];
+      uint32_t tb = candb[wd], kept = 0u;
+      while (tb && keep > 0) {
+        const uint32_t low = tb & (0u - tb);
+        kept |= low;
+        tb ^= low;
+        --keep;
+      }
+      uint32_t bits = selb[wd] | kept;
+      if (mrow) mrow[wd] = bits;
       while (bits) {
         const int j = __ffs(bits) - 1;
         bits &= bits - 1u;
@@ -633,11 +698,11 @@ __device__ __forceinline__ void topk_bitmap_row(const size_t row, const float* _
         ++pos;
       }
     }
-    const int total = scan_total;
+    const int total = sel_total + min(tie_total, kneed);
     for (int i = total + tid; i < K; i += NT) out[i] = -1;  // only if something went wrong
   }
   if (mrow)
-    for (int wd = tid; wd < mask_stride; wd += NT) mrow[wd] = wd < nw ? selb[wd] : 0u;
+    for (int wd = nw + tid; wd < mask_stride; wd += NT) mrow[wd] = 0u;
 }
 
 
