@@ -14,7 +14,8 @@
 // Layout of one work item: Q block [128 x Dqk], K block [128 x Dqk] (both K-major bf16,
 // 128-byte swizzle, via 3-D tensor maps over (dim, head, token)), V block [128 x Dv]
 // (MN-major operand of the second product).  Tensor memory: S0, S1 (128 columns each,
-// double-buffered so S_{j+1} = Q K_{j+1}^T overlaps the softmax of block j), O (Dv columns);
+// double-buffered so S_{j+1} = Q K_{j+1}^T overlaps the softmax of block j), O0, O1 (Dv
+// columns each, one per softmax group);
 // P is split into bf16 P_hi + P_lo (two per 32-bit column): the 16 keys of each chunk write
 // P_hi into the first 8 of their own 16 S columns and P_lo into the next 8, which feed
 // O += P_hi V + P_lo V as tensor-memory A operands -- the low part keeps the float32
@@ -22,11 +23,14 @@
 // (and O, l rescaled) when a row's block max exceeds it by more than 2^8, so exp2 arguments
 // stay <= 8 and rescales are rare.
 //
-// Roles: warps 0..7 softmax and
-// epilogue in two groups that take alternate key blocks (thread = query row = TMEM lane),
-// warp 8 TMA producer of Q and K, warp 10 of V, warp 9 MMA issuer (one thread),
-// each with its own O accumulator and running (max, sum); the groups merge at the end of
-// an item.  Persistent CTAs take items in snake order, longest first.  Every wait is bounded.
+// Roles (16 warps, a setmaxnreg split per warpgroup): warps 0..7 softmax in two groups that
+// take alternate key blocks (thread = query row = TMEM lane), each with its own O accumulator
+// and running (max, sum); warp 8 TMA producer of Q and K, warp 10 of V, warp 9 the MMA issuer
+// (one thread); warps 12..15 merge the two groups' O at the end of an item, normalise, gate
+// and store it while the softmax groups start the next item (band items keep that in the
+// softmax groups).  Key blocks come from a per-query-block list of the blocks that hold a
+// selected key.  Persistent CTAs take items in snake order, longest first (in bands of query
+// blocks when K/V exceeds the L2).  Every wait is bounded.
 #include <cudaTypedefs.h>
 
 #include <mutex>
