@@ -259,10 +259,11 @@ __global__ void __launch_bounds__(NT) topk_rows_kernel(const float* __restrict__
 // around the sample's K-th rank (a 3-sigma rank margin); short rows histogram every key and
 // the window is the exact bucket b1.  Read 2 (L2, or the registers when the whole row fit in
 // read 1's batch of loads): keys above the window go to the SELECTED bitmap, keys inside it
-// to the CANDIDATE bitmap (bits assembled across lanes with shuffles) and to a shared-memory
-// candidate list of (key, position).  On long rows an exact 12-bit histogram of the
-// candidates alone then gives b1; if the sampled window missed the K-th key, read 1 is
-// redone exactly.  Either way b1 and `need` (keys of b1 still to take) are exact.  The low
+// to the CANDIDATE bitmap -- two float comparisons per key against the window's bucket
+// bounds and one warp vote per 32-key word.  The candidates (a few percent of the keys) are
+// then listed in shared memory as (key, position) from the bitmap, their scores re-read
+// from L2.  On long rows an exact 12-bit histogram of the candidates alone then gives b1;
+// if the sampled window missed the K-th key, read 1 is redone exactly.  Either way b1 and `need` (keys of b1 still to take) are exact.  The low
 // 20 bits are resolved by two 10-bit histogram passes over the candidate list (in shared
 // memory; only a list that overflowed is re-read from L2 through the bitmap), giving the
 // exact threshold key tau.  Candidates above tau join SELECTED; candidates equal to tau are
@@ -342,27 +343,31 @@ __device__ __forceinline__ int warp_reserve(int c, int* counter) {
   return base + x - c;
 }
 
-// U chunks of 4 scores as order keys: chunk u of this thread covers keys
-// base + (u*NT + tid)*4 + 0..3.  Keys at or past n are loaded as 0.0 (callers mask them).
+// U scores per thread, lane-contiguous: slot j of this thread is key base + j*NT + tid, so
+// the 32 lanes of a warp hold one 32-key bitmap word per slot.  Keys at or past n load as
+// 0.0 (callers mask them).
 template <int NT, int U>
-__device__ __forceinline__ void load_keys(const float* __restrict__ sc, int n, int base,
-                                          bool vec, uint32_t (&k)[U][4]) {
-  float v[U][4];
+__device__ __forceinline__ void load_vals(const float* __restrict__ sc, int n, int base,
+                                          float (&v)[U]) {
 #pragma unroll
-  for (int u = 0; u < U; ++u) {
-    const int i = base + (u * NT + (int)threadIdx.x) * 4;
-    if (vec && i + 3 < n) {
-      const float4 f = __ldg(reinterpret_cast<const float4*>(sc + i));
-      v[u][0] = f.x; v[u][1] = f.y; v[u][2] = f.z; v[u][3] = f.w;
-    } else {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) v[u][e] = (i + e < n) ? __ldg(sc + i + e) : 0.f;
-    }
+  for (int j = 0; j < U; ++j) {
+    const int i = base + j * NT + (int)threadIdx.x;
+    v[j] = i < n ? __ldg(sc + i) : 0.f;
   }
-#pragma unroll
-  for (int u = 0; u < U; ++u)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) k[u][e] = order_key(v[u][e]);
+}
+
+// The smallest float whose order key lies in bucket b or above (b = 0..4096 over the top 12
+// key bits): for every score v that is not NaN, (order_key(v) >> 20) >= b  <=>  v >= this.
+// Buckets 0..7 hold only NaN images and, at the top of bucket 7, -inf; bucket 8 starts at
+// -FLT_MAX; a bucket past the one of +inf has no float (NaN: no comparison passes).  -0.0 and
+// +0.0 share a key and compare equal as floats, so the two tests agree on them as well.
+__device__ __forceinline__ float bucket_floor(uint32_t b) {
+  if (b >= 4096u) return __uint_as_float(0x7fffffffu);
+  const uint32_t k = b << 20;
+  if (k < 0x00800000u) return __uint_as_float(0xff800000u);       // -inf
+  if (k < 0x80000000u) return __uint_as_float(~k);                // a negative float
+  const uint32_t u = k ^ 0x80000000u;                             // +0.0 and up
+  return u <= 0x7f800000u ? __uint_as_float(u) : __uint_as_float(0x7fffffffu);
 }
 
 template <int NT, bool SAMPLE>
@@ -389,7 +394,7 @@ __device__ __forceinline__ void topk_bitmap_row(const size_t row, const float* _
   const int n = min(Tn, s + q_off + 1);
   const float* sc = scores + row * (size_t)Tn;
   int32_t* out = idx + row * (size_t)K;
-  const int tid = threadIdx.x, lane = tid & 31;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint32_t* mrow = mask ? mask + row * (size_t)mask_stride : nullptr;
   const int nw = (n + 31) >> 5;
 
@@ -407,10 +412,9 @@ __device__ __forceinline__ void topk_bitmap_row(const size_t row, const float* _
   if (tid == 0) { cnt_sel = 0; cl_n = 0; }
   __syncthreads();
 
-  constexpr int U = (SAMPLE && NT == 512) ? 2 : 4;  // float4 loads in flight per thread
-  constexpr int kChunk = NT * 4 * U;  // keys per batch of loads
-  const bool vec = ((Tn & 3) == 0);
-  uint32_t kh[U][4];  // the current batch of keys; the whole row when n <= kChunk
+  constexpr int U = (NT == 256 && !SAMPLE) ? 16 : 8;  // scores per thread per batch of loads
+  constexpr int kChunk = NT * U;                        // keys per batch
+  float kv[U];  // the current batch of scores; the whole row when n <= kChunk
   bool held = false;
   uint32_t b1 = 0;
   int need = K, cnt1 = 0;
@@ -418,13 +422,10 @@ __device__ __forceinline__ void topk_bitmap_row(const size_t row, const float* _
   // Exact read 1: 12-bit histogram of every key -> bucket b1 of the K-th key, `need`.
   auto exact_read1 = [&]() {
     for (int base = 0; base < n; base += kChunk) {
-      load_keys<NT, U>(sc, n, base, vec, kh);
+      load_vals<NT, U>(sc, n, base, kv);
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int i = base + (u * NT + tid) * 4;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) hist_add<NT>(hist, kh[u][e] >> 20, i + e < n);
-      }
+      for (int j = 0; j < U; ++j)
+        hist_add<NT>(hist, order_key(kv[j]) >> 20, base + j * NT + tid < n);
     }
     held = n <= kChunk;
     __syncthreads();
@@ -435,73 +436,81 @@ __device__ __forceinline__ void topk_bitmap_row(const size_t row, const float* _
     cnt1 = pick[2];
   };
 
-  // Read 2: keys whose bucket is above [lo, hi] -> SELECTED bitmap; inside it -> CANDIDATE
-  // bitmap and the candidate list (key, position) while it has room.  Counts both.
+  // Read 2: keys whose bucket is above [lo, hi] -> SELECTED bitmap, inside it -> CANDIDATE
+  // bitmap.  The buckets are compared as floats (bucket_floor) and each warp's 32 lanes
+  // vote one bitmap word per slot.
   auto read2 = [&](uint32_t lo, uint32_t hi) {
-    int my_sel = 0;
+    const float f_lo = bucket_floor(lo), f_hi = bucket_floor(hi + 1u);
     // long rows (SAMPLE): the next batch is in flight while this one is classified
-    uint32_t kn[SAMPLE ? U : 1][4];
+    float vn[SAMPLE ? U : 1];
     if constexpr (SAMPLE) {
-      if (!held) load_keys<NT, U>(sc, n, 0, vec, kn);
+      if (!held) load_vals<NT, U>(sc, n, 0, vn);
     }
     for (int base = 0; base < n; base += kChunk) {
       if constexpr (SAMPLE) {
         if (!held) {
 #pragma unroll
-          for (int u = 0; u < U; ++u)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) kh[u][e] = kn[u][e];
-          if (base + kChunk < n) load_keys<NT, U>(sc, n, base + kChunk, vec, kn);
+          for (int j = 0; j < U; ++j) kv[j] = vn[j];
+          if (base + kChunk < n) load_vals<NT, U>(sc, n, base + kChunk, vn);
         }
       } else {
-        if (!held) load_keys<NT, U>(sc, n, base, vec, kh);
+        if (!held) load_vals<NT, U>(sc, n, base, kv);
       }
-      uint32_t gt[U], in[U];
-      int c = 0;
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int i = base + (u * NT + tid) * 4;
-        gt[u] = 0u;
-        in[u] = 0u;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          if (i + e < n) {
-            const uint32_t d = kh[u][e] >> 20;
-            gt[u] |= (d > hi ? 1u : 0u) << e;
-            in[u] |= (d >= lo && d <= hi ? 1u : 0u) << e;
-          }
-        }
-        my_sel += __popc(gt[u]);
-        c += __popc(in[u]);
-        // lanes 8m..8m+7 cover one 32-key word: OR their nibbles together
-        const int sh = 4 * (lane & 7);
-        uint32_t wg = gt[u] << sh, we = in[u] << sh;
-#pragma unroll
-        for (int o = 1; o < 8; o <<= 1) {
-          wg |= __shfl_xor_sync(0xffffffffu, wg, o);
-          we |= __shfl_xor_sync(0xffffffffu, we, o);
-        }
-        if ((lane & 7) == 0 && i < n) {
-          selb[i >> 5] = wg;
-          candb[i >> 5] = we;
+      for (int j = 0; j < U; ++j) {
+        const int w0 = base + j * NT + warp * 32;  // first key of this warp's word
+        const bool ok = w0 + lane < n;
+        const uint32_t gt = __ballot_sync(0xffffffffu, ok && kv[j] >= f_hi);
+        const uint32_t ge = __ballot_sync(0xffffffffu, ok && kv[j] >= f_lo);
+        if (lane == 0 && w0 < n) {
+          selb[w0 >> 5] = gt;
+          candb[w0 >> 5] = ge & ~gt;
         }
       }
-      int pos = warp_reserve(c, &cl_n);
-#pragma unroll
-      for (int u = 0; u < U; ++u)
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          if ((in[u] >> e) & 1u) {
-            if (pos < cl_cap) {
-              cl_key[pos] = kh[u][e];
-              cl_idx[pos] = (uint32_t)(base + (u * NT + tid) * 4 + e);
-            }
-            ++pos;
-          }
+    }
+    __syncthreads();
+  };
+
+  // After read 2: the candidate list (order key, position), built from the CANDIDATE
+  // bitmap with the scores re-read from L2, and its length cl_n.  A list longer than cl_cap
+  // keeps its first cl_cap entries (cl_n still counts them all); the later steps then walk
+  // the bitmap instead.  The sampled window also needs the SELECTED count (cnt_sel) and the
+  // 12-bit histogram of the candidates (into `hist`, which is clear).
+  auto collect = [&](bool sampled) {
+    int lsel = 0;
+    for (int w0 = 0; w0 < nw; w0 += NT) {
+      const int wd = w0 + tid;
+      uint32_t cb = 0u;
+      if (wd < nw) {
+        if (sampled) lsel += __popc(selb[wd]);
+        cb = candb[wd];
+      }
+      int pos = warp_reserve(__popc(cb), &cl_n);
+      while (__any_sync(0xffffffffu, cb != 0u)) {
+        // two candidates per step, so that two loads are in flight
+        int t0 = -1, t1 = -1;
+        if (cb) { t0 = wd * 32 + __ffs(cb) - 1; cb &= cb - 1u; }
+        if (cb) { t1 = wd * 32 + __ffs(cb) - 1; cb &= cb - 1u; }
+        const float v0 = t0 >= 0 ? __ldg(sc + t0) : 0.f;
+        const float v1 = t1 >= 0 ? __ldg(sc + t1) : 0.f;
+        const uint32_t k0 = order_key(v0), k1 = order_key(v1);
+        if (t0 >= 0) {
+          if (pos < cl_cap) { cl_key[pos] = k0; cl_idx[pos] = (uint32_t)t0; }
+          ++pos;
+        }
+        if (t1 >= 0) {
+          if (pos < cl_cap) { cl_key[pos] = k1; cl_idx[pos] = (uint32_t)t1; }
+          ++pos;
+        }
+        if (sampled) {
+          hist_add<NT>(hist, k0 >> 20, t0 >= 0);
+          hist_add<NT>(hist, k1 >> 20, t1 >= 0);
+        }
+      }
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) my_sel += __shfl_xor_sync(0xffffffffu, my_sel, o);
-    if (lane == 0 && my_sel) atomicAdd(&cnt_sel, my_sel);
+    for (int o = 16; o > 0; o >>= 1) lsel += __shfl_xor_sync(0xffffffffu, lsel, o);
+    if (lane == 0 && lsel) atomicAdd(&cnt_sel, lsel);
     __syncthreads();
   };
 
@@ -509,15 +518,15 @@ __device__ __forceinline__ void topk_bitmap_row(const size_t row, const float* _
     // ---------------- read 1 (sampled): 12-bit histogram of every 8th key -> a window of
     // buckets that holds the K-th key with high probability (rank margin 3 sigma + 2)
     const int ns = (n + 7) >> 3;
-    for (int m0 = 0; m0 < ns; m0 += NT * 4) {
-      float v[4];
+    for (int m0 = 0; m0 < ns; m0 += NT * 8) {
+      float v[8];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < 8; ++u) {
         const int m = m0 + u * NT + tid;
         v[u] = m < ns ? __ldg(sc + 8 * m) : 0.f;
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) hist_add<NT>(hist, order_key(v[u]) >> 20, m0 + u * NT + tid < ns);
+      for (int u = 0; u < 8; ++u) hist_add<NT>(hist, order_key(v[u]) >> 20, m0 + u * NT + tid < ns);
     }
     __syncthreads();
     const float ks = (float)K * (float)ns / (float)n;
@@ -528,33 +537,9 @@ __device__ __forceinline__ void topk_bitmap_row(const size_t row, const float* _
     const uint32_t b_hi = (uint32_t)pick[0], b_lo = (uint32_t)pick[1];
     for (int i = tid; i < padded(kBins1); i += NT) hist[i] = 0u;
     read2(b_lo, b_hi);  // ends with a barrier: the histogram is clear
+    collect(true);      // + the SELECTED count and the candidates' 12-bit histogram
     const int nsel = cnt_sel, ncand = cl_n;
     if (nsel < K && nsel + ncand >= K) {
-      // exact 12-bit histogram of the candidates only -> the bucket b1 of the K-th key
-      if (ncand <= cl_cap) {
-        for (int i0 = 0; i0 < ncand; i0 += NT) {
-          const int i = i0 + tid;
-          hist_add<NT>(hist, i < ncand ? cl_key[i] >> 20 : 0u, i < ncand);
-        }
-      } else {
-        for (int w0 = 0; w0 < nw; w0 += NT) {
-          const int wd = w0 + tid;
-          uint32_t bits = wd < nw ? candb[wd] : 0u;
-          bool more = __any_sync(0xffffffffu, bits != 0u);
-          while (more) {
-            uint32_t digit = 0u;
-            const bool has = bits != 0u;
-            if (has) {
-              const int j = __ffs(bits) - 1;
-              bits &= bits - 1u;
-              digit = order_key(__ldg(sc + wd * 32 + j)) >> 20;
-            }
-            hist_add<NT>(hist, digit, has);
-            more = __any_sync(0xffffffffu, bits != 0u);
-          }
-        }
-      }
-      __syncthreads();
       find_bucket<NT, kBins1>(hist, K - nsel, warp_buf, &scan_total, pick);
       __syncthreads();
       b1 = (uint32_t)pick[0];
@@ -568,10 +553,12 @@ __device__ __forceinline__ void topk_bitmap_row(const size_t row, const float* _
       __syncthreads();
       exact_read1();
       read2(b1, b1);
+      collect(false);
     }
   } else {
     exact_read1();
     read2(b1, b1);
+    collect(false);
   }
   const int ncl = cl_n;
   const bool use_cl = ncl <= cl_cap;  // else the candidates are re-read through the bitmap

@@ -213,13 +213,22 @@ def _adversarial_scores(kind, S, T, seed):
         x[torch.rand(1, S, T, generator=g) < 0.3] = float("-inf")
     elif kind == "dup_floats":
         x = torch.randn(1, S, T // 4 + 1, generator=g).repeat(1, 1, 4)[..., :T].contiguous()
+    elif kind == "extremes":
+        # the K-th key in the first and last buckets of the 12-bit key prefix and next to the
+        # sign change: infinities, +-FLT_MAX, the smallest normals and subnormals, signed zeros
+        fmax, tiny, sub = 3.4028234663852886e38, 1.1754943508222875e-38, 1.401298464324817e-45
+        vals = torch.tensor([float("inf"), float("-inf"), fmax, -fmax, tiny, -tiny, sub, -sub,
+                             0.0, -0.0, 1.0, -1.0])
+        pick = torch.randint(0, len(vals), (1, S, T), generator=g)
+        x = torch.where(torch.rand(1, S, T, generator=g) < 0.8, vals[pick],
+                        torch.randn(1, S, T, generator=g))
     else:
         raise ValueError(kind)
     return x
 
 
 @pytest.mark.parametrize("kind", ["all_equal", "signed_zeros", "few_values", "wide_range",
-                                  "neg_inf_inside", "dup_floats"])
+                                  "neg_inf_inside", "dup_floats", "extremes"])
 # (40, 3000): rows held in registers; (20, 6000): short rows read in two batches;
 # (300, 9000): many long rows (sampled first read, 512-thread CTAs); (6, 20000): few long rows
 @pytest.mark.parametrize("S,T,K", [(64, 64, 8), (40, 3000, 700), (20, 6000, 1000),
