@@ -275,6 +275,7 @@ constexpr int kMaxBitmapKeys = 1 << 20;
 constexpr size_t kMaxDynSmem = 220u * 1024u;  // leaves room for the static shared memory
 constexpr int kBins1 = 4096;  // top 12 bits
 constexpr int kBins2 = 1024;  // 10-bit refinement digits
+static_assert(padded(kBins1) % 4 == 0 && padded(kBins2) % 4 == 0, "clear_words wants x4");
 
 // Bucket holding the need-th largest key: writes (bin, count above it, its count) to
 // out[0..2].  Each thread owns a run of NBINS/NT bins, highest first; the counts stay in
@@ -292,14 +293,16 @@ __device__ __forceinline__ void find_bucket(const uint32_t* hist, int need, int*
     local += c[q];
   }
   int above = block_excl_scan(local, warp_buf, scan_total);
+  if (above < need && above + local >= need) {  // the one thread whose run holds the bin
 #pragma unroll
-  for (int q = 0; q < per; ++q) {
-    if (above < need && above + c[q] >= need) {
-      out[0] = hi_bin - 1 - q;
-      out[1] = above;
-      out[2] = c[q];
+    for (int q = 0; q < per; ++q) {
+      if (above < need && above + c[q] >= need) {
+        out[0] = hi_bin - 1 - q;
+        out[1] = above;
+        out[2] = c[q];
+      }
+      above += c[q];
     }
-    above += c[q];
   }
 }
 
@@ -320,12 +323,50 @@ __device__ __forceinline__ void find_bucket2(const uint32_t* hist, int need_a, i
     local += c[q];
   }
   int above = block_excl_scan(local, warp_buf, scan_total);
+  const bool has_a = above < need_a && above + local >= need_a;
+  const bool has_b = above < need_b && above + local >= need_b;
+  if (has_a || has_b) {  // only the threads whose runs hold one of the bins
 #pragma unroll
-  for (int q = 0; q < per; ++q) {
-    if (above < need_a && above + c[q] >= need_a) *bin_a = hi_bin - 1 - q;
-    if (above < need_b && above + c[q] >= need_b) *bin_b = hi_bin - 1 - q;
-    above += c[q];
+    for (int q = 0; q < per; ++q) {
+      if (above < need_a && above + c[q] >= need_a) *bin_a = hi_bin - 1 - q;
+      if (above < need_b && above + c[q] >= need_b) *bin_b = hi_bin - 1 - q;
+      above += c[q];
+    }
   }
+}
+
+// find_bucket restricted to the bins [lo, hi] (the histogram holds nothing else): the bins
+// of a narrow window are scanned by warp 0 alone, highest first; `need` is at most their
+// total.  Writes (bin, count above it, its count) to out[0..2]; callers pass a barrier
+// before reading them.
+template <int NT, int NBINS>
+__device__ __forceinline__ void find_bucket_window(const uint32_t* hist, int lo, int hi, int need,
+                                                   int* warp_buf, int* scan_total, int* out) {
+  if (hi - lo >= 32) {
+    find_bucket<NT, NBINS>(hist, need, warp_buf, scan_total, out);
+    return;
+  }
+  if (threadIdx.x >= 32) return;
+  const int lane = threadIdx.x, b = hi - lane;
+  const int c = b >= lo ? (int)hist[hpad(b)] : 0;
+  int x = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  const int above = x - c;
+  if (b >= lo && above < need && x >= need) {
+    out[0] = b;
+    out[1] = above;
+    out[2] = c;
+  }
+}
+
+// Zeroes nwords (a multiple of 4) 32-bit words at a 16-byte aligned address, block-wide.
+__device__ __forceinline__ void clear_words(uint32_t* p, int nwords) {
+  uint4* q = reinterpret_cast<uint4*>(p);
+  for (int i = threadIdx.x; i < nwords / 4; i += blockDim.x) q[i] = make_uint4(0u, 0u, 0u, 0u);
 }
 
 // Reserves c consecutive slots per lane in a shared list; returns this lane's first slot.
@@ -408,7 +449,7 @@ __device__ __forceinline__ void topk_bitmap_row(const size_t row, const float* _
     return;
   }
 
-  for (int i = tid; i < padded(kBins1); i += NT) hist[i] = 0u;
+  clear_words(hist, padded(kBins1));
   if (tid == 0) { cnt_sel = 0; cl_n = 0; }
   __syncthreads();
 
@@ -535,12 +576,18 @@ __device__ __forceinline__ void topk_bitmap_row(const size_t row, const float* _
     find_bucket2<NT, kBins1>(hist, r_hi, r_lo, warp_buf, &scan_total, &pick[0], &pick[1]);
     __syncthreads();
     const uint32_t b_hi = (uint32_t)pick[0], b_lo = (uint32_t)pick[1];
-    for (int i = tid; i < padded(kBins1); i += NT) hist[i] = 0u;
+    // the candidates fall in the window's bins only: a narrow window clears just those
+    if (b_hi - b_lo < 32u) {
+      for (int b = (int)b_lo + tid; b <= (int)b_hi; b += NT) hist[hpad(b)] = 0u;
+    } else {
+      clear_words(hist, padded(kBins1));
+    }
     read2(b_lo, b_hi);  // ends with a barrier: the histogram is clear
     collect(true);      // + the SELECTED count and the candidates' 12-bit histogram
     const int nsel = cnt_sel, ncand = cl_n;
     if (nsel < K && nsel + ncand >= K) {
-      find_bucket<NT, kBins1>(hist, K - nsel, warp_buf, &scan_total, pick);
+      find_bucket_window<NT, kBins1>(hist, (int)b_lo, (int)b_hi, K - nsel, warp_buf,
+                                     &scan_total, pick);
       __syncthreads();
       b1 = (uint32_t)pick[0];
       need = K - nsel - pick[1];
@@ -548,7 +595,7 @@ __device__ __forceinline__ void topk_bitmap_row(const size_t row, const float* _
     } else {
       // the sample missed: exact read 1, then read 2 again with the window [b1, b1]
       __syncthreads();  // every thread has read the counts before they are reset
-      for (int i = tid; i < padded(kBins1); i += NT) hist[i] = 0u;
+      clear_words(hist, padded(kBins1));
       if (tid == 0) { cnt_sel = 0; cl_n = 0; }
       __syncthreads();
       exact_read1();
@@ -569,7 +616,7 @@ __device__ __forceinline__ void topk_bitmap_row(const size_t row, const float* _
   if (cnt1 != need) {
     for (int pass = 0; pass < 2; ++pass) {
       const int shift = 20 - 10 * (pass + 1);
-      for (int i = tid; i < padded(kBins2); i += NT) hist[i] = 0u;
+      clear_words(hist, padded(kBins2));
       __syncthreads();
       if (use_cl) {
         for (int i0 = 0; i0 < ncl; i0 += NT) {
