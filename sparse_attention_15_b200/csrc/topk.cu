@@ -411,6 +411,28 @@ __device__ __forceinline__ float bucket_floor(uint32_t b) {
   return u <= 0x7f800000u ? __uint_as_float(u) : __uint_as_float(0x7fffffffu);
 }
 
+// Read 2's vote over one batch of U scores per thread (load_vals layout): slot j of the warp
+// is bitmap word (base >> 5) + j * NT/32 + warp; lane 0 stores (keys >= f_hi, keys >= f_lo)
+// as one 64-bit pair.  Only a batch that runs past n (FULL false) tests the bounds.
+template <int NT, int U, bool FULL>
+__device__ __forceinline__ void vote_words(const float (&v)[U], int base, int n, float f_lo,
+                                           float f_hi, uint2* bm) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint2* dst = bm + (base >> 5) + warp;
+#pragma unroll
+  for (int j = 0; j < U; ++j) {
+    const int w0 = base + j * NT + warp * 32;  // first key of this warp's word
+    bool a = v[j] >= f_hi, b = v[j] >= f_lo;
+    if (!FULL) {
+      a = a && w0 + lane < n;
+      b = b && w0 + lane < n;
+    }
+    const uint32_t gt = __ballot_sync(0xffffffffu, a);
+    const uint32_t ge = __ballot_sync(0xffffffffu, b);
+    if (lane == 0 && (FULL || w0 < n)) dst[j * (NT / 32)] = make_uint2(gt, ge);
+  }
+}
+
 template <int NT, bool SAMPLE>
 __device__ __forceinline__ void topk_bitmap_row(const size_t row, const float* __restrict__ scores,
                                                 int S, int Tn, int K, int q_off,
@@ -420,10 +442,11 @@ __device__ __forceinline__ void topk_bitmap_row(const size_t row, const float* _
   extern __shared__ uint32_t dsm[];
   const int W = (Tn + 31) >> 5;              // bitmap words per row
   uint32_t* hist = dsm;                      // [padded(kBins1)]
-  uint32_t* selb = hist + padded(kBins1);    // [W]
-  uint32_t* candb = selb + W;                // [W]
-  uint32_t* cl_key = candb + W;              // [cl_cap] candidate keys
-  uint32_t* cl_idx = cl_key + cl_cap;        // [cl_cap] candidate positions
+  // [W] bitmap words: .x SELECTED, .y CANDIDATE (read 2 leaves there the keys at or above
+  // the window, collect() removes the SELECTED ones; later the ties at the threshold)
+  uint2* bm = reinterpret_cast<uint2*>(hist + padded(kBins1));
+  uint32_t* cl_key = reinterpret_cast<uint32_t*>(bm + W);  // [cl_cap] candidate keys
+  uint32_t* cl_idx = cl_key + cl_cap;                      // [cl_cap] candidate positions
   __shared__ int warp_buf[32];
   __shared__ int2 warp_buf2[32];
   __shared__ int2 scan_total2;
@@ -435,7 +458,7 @@ __device__ __forceinline__ void topk_bitmap_row(const size_t row, const float* _
   const int n = min(Tn, s + q_off + 1);
   const float* sc = scores + row * (size_t)Tn;
   int32_t* out = idx + row * (size_t)K;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x, lane = tid & 31;
   uint32_t* mrow = mask ? mask + row * (size_t)mask_stride : nullptr;
   const int nw = (n + 31) >> 5;
 
@@ -477,36 +500,31 @@ __device__ __forceinline__ void topk_bitmap_row(const size_t row, const float* _
     cnt1 = pick[2];
   };
 
-  // Read 2: keys whose bucket is above [lo, hi] -> SELECTED bitmap, inside it -> CANDIDATE
-  // bitmap.  The buckets are compared as floats (bucket_floor) and each warp's 32 lanes
-  // vote one bitmap word per slot.
+  // Read 2: keys whose bucket is above [lo, hi] -> SELECTED bitmap, at or above lo -> the
+  // CANDIDATE word (collect() removes the SELECTED keys from it).  The buckets are compared
+  // as floats (bucket_floor) and each warp's 32 lanes vote one bitmap word per slot.
   auto read2 = [&](uint32_t lo, uint32_t hi) {
     const float f_lo = bucket_floor(lo), f_hi = bucket_floor(hi + 1u);
-    // long rows (SAMPLE): the next batch is in flight while this one is classified
-    float vn[SAMPLE ? U : 1];
-    if constexpr (SAMPLE) {
-      if (!held) load_vals<NT, U>(sc, n, 0, vn);
-    }
-    for (int base = 0; base < n; base += kChunk) {
-      if constexpr (SAMPLE) {
-        if (!held) {
-#pragma unroll
-          for (int j = 0; j < U; ++j) kv[j] = vn[j];
-          if (base + kChunk < n) load_vals<NT, U>(sc, n, base + kChunk, vn);
-        }
-      } else {
-        if (!held) load_vals<NT, U>(sc, n, base, kv);
+    if (held) {
+      vote_words<NT, U, false>(kv, 0, n, f_lo, f_hi, bm);
+    } else if (SAMPLE) {
+      // long rows: two register buffers, the next batch in flight while one is voted
+      float vb[U];
+      load_vals<NT, U>(sc, n, 0, kv);
+      for (int base = 0; base < n; base += 2 * kChunk) {
+        if (base + kChunk < n) load_vals<NT, U>(sc, n, base + kChunk, vb);
+        if (base + kChunk <= n) vote_words<NT, U, true>(kv, base, n, f_lo, f_hi, bm);
+        else vote_words<NT, U, false>(kv, base, n, f_lo, f_hi, bm);
+        if (base + kChunk >= n) break;
+        if (base + 2 * kChunk < n) load_vals<NT, U>(sc, n, base + 2 * kChunk, kv);
+        if (base + 2 * kChunk <= n) vote_words<NT, U, true>(vb, base + kChunk, n, f_lo, f_hi, bm);
+        else vote_words<NT, U, false>(vb, base + kChunk, n, f_lo, f_hi, bm);
       }
-#pragma unroll
-      for (int j = 0; j < U; ++j) {
-        const int w0 = base + j * NT + warp * 32;  // first key of this warp's word
-        const bool ok = w0 + lane < n;
-        const uint32_t gt = __ballot_sync(0xffffffffu, ok && kv[j] >= f_hi);
-        const uint32_t ge = __ballot_sync(0xffffffffu, ok && kv[j] >= f_lo);
-        if (lane == 0 && w0 < n) {
-          selb[w0 >> 5] = gt;
-          candb[w0 >> 5] = ge & ~gt;
-        }
+    } else {
+      for (int base = 0; base < n; base += kChunk) {
+        load_vals<NT, U>(sc, n, base, kv);
+        if (base + kChunk <= n) vote_words<NT, U, true>(kv, base, n, f_lo, f_hi, bm);
+        else vote_words<NT, U, false>(kv, base, n, f_lo, f_hi, bm);
       }
     }
     __syncthreads();
@@ -523,8 +541,10 @@ __device__ __forceinline__ void topk_bitmap_row(const size_t row, const float* _
       const int wd = w0 + tid;
       uint32_t cb = 0u;
       if (wd < nw) {
-        if (sampled) lsel += __popc(selb[wd]);
-        cb = candb[wd];
+        const uint2 w = bm[wd];
+        if (sampled) lsel += __popc(w.x);
+        cb = w.y & ~w.x;
+        bm[wd].y = cb;
       }
       int pos = warp_reserve(__popc(cb), &cl_n);
       while (__any_sync(0xffffffffu, cb != 0u)) {
@@ -635,7 +655,7 @@ __device__ __forceinline__ void topk_bitmap_row(const size_t row, const float* _
       } else {
         for (int w0 = 0; w0 < nw; w0 += NT) {
           const int wd = w0 + tid;
-          uint32_t bits = wd < nw ? candb[wd] : 0u;
+          uint32_t bits = wd < nw ? bm[wd].y : 0u;
           // every lane walks its word; the histogram add is warp-aggregated per step
           bool more = __any_sync(0xffffffffu, bits != 0u);
           while (more) {
@@ -667,19 +687,19 @@ __device__ __forceinline__ void topk_bitmap_row(const size_t row, const float* _
     }
   }
 
-  // ---------------- candidates: above the threshold -> SELECTED, at it -> ties (in candb)
+  // ---------------- candidates: above the threshold -> SELECTED, at it -> ties (CANDIDATE)
   const int fshift = 32 - pbits;
   if (use_cl) {
-    for (int wd = tid; wd < nw; wd += NT) candb[wd] = 0u;
+    for (int wd = tid; wd < nw; wd += NT) bm[wd].y = 0u;
     __syncthreads();
     for (int i = tid; i < ncl; i += NT) {
       const uint32_t hi = cl_key[i] >> fshift, t = cl_idx[i];
-      if (hi > prefix) atomicOr(&selb[t >> 5], 1u << (t & 31));
-      else if (hi == prefix) atomicOr(&candb[t >> 5], 1u << (t & 31));
+      if (hi > prefix) atomicOr(&bm[t >> 5].x, 1u << (t & 31));
+      else if (hi == prefix) atomicOr(&bm[t >> 5].y, 1u << (t & 31));
     }
   } else {
     for (int wd = tid; wd < nw; wd += NT) {
-      uint32_t bits = candb[wd], sel = 0u, tie = 0u;
+      uint32_t bits = bm[wd].y, sel = 0u, tie = 0u;
       while (bits) {
         const int j = __ffs(bits) - 1;
         bits &= bits - 1u;
@@ -687,8 +707,8 @@ __device__ __forceinline__ void topk_bitmap_row(const size_t row, const float* _
         if (hi > prefix) sel |= 1u << j;
         else if (hi == prefix) tie |= 1u << j;
       }
-      selb[wd] |= sel;
-      candb[wd] = tie;
+      bm[wd].x |= sel;
+      bm[wd].y = tie;
     }
   }
   __syncthreads();
@@ -703,8 +723,9 @@ __device__ __forceinline__ void topk_bitmap_row(const size_t row, const float* _
     for (int q = 0; q < per; ++q) {
       const int wd = tid * per + q;
       if (wd < nw) {
-        lsel += __popc(selb[wd]);
-        ltie += __popc(candb[wd]);
+        const uint2 w = bm[wd];
+        lsel += __popc(w.x);
+        ltie += __popc(w.y);
       }
     }
     int sel_before, tie_before, sel_total, tie_total;
@@ -716,14 +737,14 @@ __device__ __forceinline__ void topk_bitmap_row(const size_t row, const float* _
     for (int q = 0; q < per; ++q) {
       const int wd = tid * per + q;
       if (wd >= nw) break;
-      uint32_t tb = candb[wd], kept = 0u;
+      uint32_t tb = bm[wd].y, kept = 0u;
       while (tb && keep > 0) {
         const uint32_t low = tb & (0u - tb);
         kept |= low;
         tb ^= low;
         --keep;
       }
-      uint32_t bits = selb[wd] | kept;
+      uint32_t bits = bm[wd].x | kept;
       if (mrow) mrow[wd] = bits;
       while (bits) {
         const int j = __ffs(bits) - 1;
