@@ -213,14 +213,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   uint64_t* q_full = bars;           // 1
   uint64_t* q_empty = bars + 1;      // 1
   uint64_t* k_full = bars + 2;       // [2] K block landed
-  uint64_t* k_empty = bars + 4;      // [2] K block consumed by S = Q K^T
+  // bars + 4, + 5: unused (a K stage is free once s_full of its block completes)
   uint64_t* s_full = bars + 6;       // [2]
   uint64_t* p_full = bars + 10;      // [2]
   uint64_t* pv_done = bars + 12;     // [2] (one phase per block of that parity)
   uint64_t* o_empty = bars + 14;     // 1 (one phase per item)
   uint64_t* mma_done = bars + 16;    // 1
   uint64_t* v_full = bars + 17;      // [2] V block landed
-  uint64_t* v_empty = bars + 19;     // [2] V block consumed by O += P V
+  // bars + 19, + 20: unused (a V stage is free once pv_done of its block completes)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 21);
   uint64_t* ml_full = bars + 22;     // [2] (m, l) of item ni in buffer ni & 1 written
   uint64_t* ml_empty = bars + 24;    // [2] ... and read by the epilogue
@@ -233,8 +233,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1); mbar_init(q_empty, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1);
-      mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1);
+      mbar_init(&k_full[i], 1);
+      mbar_init(&v_full[i], 1);
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 4);
     }
@@ -264,13 +264,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     // ------------------------------------------------------------------ TMA producers
     // warp 0: Q blocks and K blocks; warp 2: V blocks.  K and V have separate rings: a K
     // stage is free as soon as S = Q K^T is done, long before the P V of the same block, so
-    // the next K blocks stream in while the softmax runs.
+    // the next K blocks stream in while the softmax runs.  The MMA thread's commits for the
+    // softmax (s_full) and for the end of P V (pv_done) free the stages as well: block g of
+    // a ring waits for the phase of block g - 2, and neither barrier can run further ahead,
+    // since block g's own product needs the copy this thread is about to start.
     const bool kq = warp == kWarpQK;
     if (lane == 0) {
       uint32_t g = 0, ni = 0;
       bool ok = true;
       uint64_t* full = kq ? k_full : v_full;
-      uint64_t* empty = kq ? k_empty : v_empty;
+      uint64_t* empty = kq ? s_full : pv_done;
       for (int kk_ = 0, i = snake_item(0, blockIdx.x, gridDim.x); ok && i < n_items;
            i = snake_item(++kk_, blockIdx.x, gridDim.x), ++ni) {
         const Item it = item_of(a, i);
@@ -348,7 +351,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                       kd + (uint64_t)(off >> 4), idesc_qk, kk > 0 ? 1u : 0u);
         }
         umma_commit(&s_full[gg & 1]);
-        umma_commit(&k_empty[st]);
         return true;
       };
       for (int kk_ = 0, i = snake_item(0, blockIdx.x, gridDim.x); ok && i < n_items;
@@ -379,7 +381,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             umma_f16_ts(o_tmem, p_tmem + pc, vdesc, idesc_pv, (j >= 2 || kk > 0) ? 1u : 0u);
             umma_f16_ts(o_tmem, p_tmem + pc + 8, vdesc, idesc_pv, 1u);
           }
-          umma_commit(&v_empty[gg & 1]);
           umma_commit(&pv_done[gg & 1]);
         }
         g += nb;
