@@ -27,8 +27,9 @@
 // take alternate key blocks (thread = query row = TMEM lane), each with its own O accumulator
 // and running (max, sum); warp 8 TMA producer of Q and K, warp 10 of V, warp 9 the MMA issuer
 // (one thread); warps 12..15 merge the two groups' O at the end of an item, normalise, gate
-// and store it while the softmax groups start the next item (band items keep that in the
-// softmax groups).  Key blocks come from a per-query-block list of the blocks that hold a
+// and store it while the softmax groups start the next item.  Band items, a few key blocks
+// long, run one softmax group of all eight warps over every block instead -- two threads per
+// row, half of the block's keys each, one O -- and store their output themselves.  Key blocks come from a per-query-block list of the blocks that hold a
 // selected key.  Persistent CTAs take items in snake order, longest first (in bands of query
 // blocks when K/V exceeds the L2).  Every wait is bounded.
 #include <cudaTypedefs.h>
@@ -48,17 +49,15 @@ constexpr int kBlk = 128;     // queries per item = keys per block
 // only completes that warpgroup), 12..15 the output epilogue of each item (one thread per
 // query row): the softmax groups hand over their (m, l) and go on to the next item while
 // the epilogue reads O out.  In band mode (items of a few key blocks, whose epilogue is on
-// the path to the next item's first P V) the two softmax groups write the output themselves,
-// each half of the columns, and warps 12..15 idle.
+// the path to the next item's first P V) the eight softmax warps form one group (warp / 4
+// picks the half of each block's keys) and write the output themselves, each half of the
+// columns, and warps 12..15 idle.
 constexpr int kSoftWarps = 8;
 constexpr int kWarpQK = 8, kWarpMma = 9, kWarpV = 10;
 constexpr int kEpiWarp0 = 12;
-// Register split (setmaxnreg, per warpgroup): the CTA is launched with 512 threads x 128
-// registers = 65536; the two softmax warpgroups raise theirs and the control and epilogue
-// warpgroups lower theirs.
-constexpr int kRegsSoft = 192, kRegsCtl = 64, kRegsEpi = 64;
-static_assert(2 * 128 * kRegsSoft + 128 * kRegsCtl + 128 * kRegsEpi <= 512 * 128,
-              "register split");
+// Register split (setmaxnreg, per warpgroup, FaCfg::REGS_*): the CTA is launched with 512
+// threads x 128 registers = 65536; the two softmax warpgroups raise theirs and the control and
+// epilogue warpgroups lower theirs.
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;
 
@@ -91,12 +90,19 @@ struct FaCfg {
   static constexpr int V_BYTES = VH * SLICE;
   static constexpr int KV_BYTES = K_BYTES + V_BYTES;
   static constexpr int STAGES = 2;
-  static constexpr int BAR_BYTES = 256;
-  static constexpr int ML_BYTES = 2 * 2 * kBlk * 2 * 4;  // [buffer][group][row][m,l] floats
-  static constexpr int SMEM = Q_BYTES + STAGES * KV_BYTES + BAR_BYTES + ML_BYTES + 1024;
+  static constexpr int BAR_BYTES = BAND ? 512 : 256;
+  static constexpr int ML_BYTES = 2 * 2 * kBlk * 2 * 4;  // [buffer][group or half][row][m,l]
+  static constexpr int XCH_BYTES = BAND ? 2 * 2 * kBlk * 4 : 0;  // [block parity][half][row]
+  static constexpr int SMEM =
+      Q_BYTES + STAGES * KV_BYTES + BAR_BYTES + ML_BYTES + XCH_BYTES + 1024;
+  // softmax rows of 128 keys (selection form) need 192 registers, half rows (band form) 160
+  static constexpr int REGS_SOFT = BAND ? 160 : 192, REGS_CTL = BAND ? 96 : 64,
+                       REGS_EPI = BAND ? 96 : 64;
+  static_assert(2 * 128 * REGS_SOFT + 128 * REGS_CTL + 128 * REGS_EPI <= 512 * 128,
+                "register split");
   static constexpr int THREADS = 32 * 16;
   static constexpr int S_COLS = kBlk;              // fp32 columns of one S buffer
-  static constexpr int O_COL = 2 * S_COLS;         // O0, O1 start after S0, S1
+  static constexpr int O_COL = 2 * S_COLS;         // O0, O1 (band: one O) after S0, S1
   static constexpr int TMEM_COLS = 512;
   static_assert(DQK % 64 == 0 && DV % 64 == 0 && DV <= 128, "head dims");
   static_assert(O_COL + 2 * DV <= TMEM_COLS, "TMEM budget");
@@ -224,7 +230,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 21);
   uint64_t* ml_full = bars + 22;     // [2] (m, l) of item ni in buffer ni & 1 written
   uint64_t* ml_empty = bars + 24;    // [2] ... and read by the epilogue
+  // band: [4 quadrants][2 block parities], the two softmax halves of a quadrant meet per block
+  uint64_t* xbar = bars + 32;
   float* ml = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + C::BAR_BYTES);
+  float* xch = ml + C::ML_BYTES / 4;  // band: the two halves' block maxima of each row
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_items = a.B * a.H * a.nqb;
@@ -236,7 +245,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       mbar_init(&k_full[i], 1);
       mbar_init(&v_full[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 4);
+      mbar_init(&p_full[i], C::BAND ? 8 : 4);  // the band's one group has eight warps
     }
     mbar_init(&pv_done[0], 1); mbar_init(&pv_done[1], 1);
     // o_empty: the four epilogue warps, or in band mode the eight softmax warps
@@ -245,6 +254,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       mbar_init(&ml_full[i], 8 * 32);
       mbar_init(&ml_empty[i], 4 * 32);
     }
+    if (C::BAND)
+      for (int i = 0; i < 8; ++i) mbar_init(&xbar[i], 64);
     fence_mbar_init();
     prefetch_tmap(&qmap); prefetch_tmap(&kmap); prefetch_tmap(&vmap);
     if (sink_blocks<C::BAND>(a)) { prefetch_tmap(&skmap); prefetch_tmap(&svmap); }
@@ -259,7 +270,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp >= kSoftWarps && warp < kEpiWarp0) {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl));
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_CTL));
   if (warp == kWarpQK || warp == kWarpV) {
     // ------------------------------------------------------------------ TMA producers
     // warp 0: Q blocks and K blocks; warp 2: V blocks.  K and V have separate rings: a K
@@ -371,14 +382,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           tc_fence_after();
           const uint64_t vd = vdesc0 + (uint64_t)(((gg & 1) * C::KV_BYTES) >> 4);
           const uint32_t p_tmem = tmem + (gg & 1) * C::S_COLS;
-          const uint32_t o_tmem = tmem + C::O_COL + (gg & 1) * C::DV;
+          const uint32_t o_tmem = tmem + C::O_COL + (C::BAND ? 0u : (gg & 1) * C::DV);
 #pragma unroll
           for (int kk = 0; kk < kBlk / 16; ++kk) {
             // keys 16kk..16kk+15: 8 packed columns of P_hi at 16kk, P_lo 8 columns further;
             // V rows 16kk..: 2 swizzle atoms of 8 rows
             const uint32_t pc = 16 * kk;
             const uint64_t vdesc = vd + (uint64_t)((kk * 2048) >> 4);
-            umma_f16_ts(o_tmem, p_tmem + pc, vdesc, idesc_pv, (j >= 2 || kk > 0) ? 1u : 0u);
+            // the first block of each O (of the item's two in the selection form) overwrites it
+            umma_f16_ts(o_tmem, p_tmem + pc, vdesc, idesc_pv,
+                        (j >= (C::BAND ? 1 : 2) || kk > 0) ? 1u : 0u);
             umma_f16_ts(o_tmem, p_tmem + pc + 8, vdesc, idesc_pv, 1u);
           }
           umma_commit(&pv_done[gg & 1]);
@@ -390,7 +403,254 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     }
   }
   } else if (warp < kSoftWarps) {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoft));
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::REGS_SOFT));
+    if constexpr (C::BAND) {
+    // ------------------------------------------------------------------ softmax, band form
+    // Band items are a few key blocks long, so one group of all eight warps takes every key
+    // block (no second group whose pipeline has to fill and drain every item): warp w handles
+    // S columns [64 h, 64 h + 64), h = w >> 2, of the rows of TMEM quadrant w & 3 -- two
+    // threads per query row, each with half of the block's keys, and one O.  The two halves
+    // of a row keep one running max: each block's maxima are exchanged through shared memory
+    // between the two warps of a quadrant (an mbarrier of their 64 threads per block parity,
+    // waited for with the usual bound), so both take the same decisions; each keeps its own
+    // part of the row sum.
+    const int half = warp >> 2;
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
+    const float ninf = __int_as_float(0xff800000);
+    uint32_t g = 0, ni = 0;
+    bool ok = true;
+    for (int kk_ = 0, i = snake_item(0, blockIdx.x, gridDim.x); ok && i < n_items;
+         i = snake_item(++kk_, blockIdx.x, gridDim.x), ++ni) {
+      const Item it = item_of(a, i);
+      int j0, j1;
+      key_range<C::BAND>(a, it, &j0, &j1);
+      const int sb = sink_blocks<C::BAND>(a);
+      const KeyBlocks kb = key_blocks(a, it, j0, j1);
+      const int nb = kb.n + sb;
+      const int s = it.qb * kBlk + row;
+      const int spos = s + a.q_off;
+      const bool row_ok = s < a.S;
+      const uint32_t* mrow =
+          (!C::BAND && row_ok) ? a.mask + ((size_t)it.b * a.S + s) * a.mask_stride : nullptr;
+      float m_used = ninf, l = 0.f;
+      // this half's 2 selection words of key block `blk`
+      auto mask_words = [&](int blk) {
+        return __ldg(reinterpret_cast<const uint2*>(mrow + ((blk * kBlk) >> 5) + 2 * half));
+      };
+      // The words of the next block are fetched one step ahead, and the index of the key
+      // block after it (from the block list) one step before that, so neither load stalls
+      // the chain from S to P.
+      uint2 nw2 = make_uint2(0u, 0u);
+      if (mrow && 0 < nb && 0 >= sb) nw2 = mask_words(kb.at(0));
+      int blk1 = (mrow && 1 < nb && 1 >= sb) ? kb.at(1 - sb) : 0;
+      for (int j = 0; j < nb; ++j) {
+        const uint32_t gg = g + j;
+        const int t0 = (j0 + j - sb) * kBlk + 64 * half;  // this half's first key
+        uint32_t bits[2] = {0u, 0u};
+        if (j < sb) {  // the sink block: its first nsink entries, visible to every query
+#pragma unroll
+          for (int w = 0; w < 2; ++w) {
+            const int n = a.nsink - 64 * half - 32 * w;
+            bits[w] = n >= 32 ? 0xffffffffu : (n > 0 ? (1u << n) - 1u : 0u);
+          }
+        } else if (!C::BAND) {
+          bits[0] = nw2.x; bits[1] = nw2.y;
+        } else if (row_ok) {
+          // band: spos - window < t <= spos, t < T
+          const int lo = max(spos - a.window + 1, 0) - t0, hi = min(spos, a.T - 1) - t0;
+#pragma unroll
+          for (int w = 0; w < 2; ++w) {
+            const int a0 = max(lo - 32 * w, 0), a1 = min(hi - 32 * w, 31);
+            bits[w] = a1 < a0 ? 0u
+                              : ((a1 - a0 == 31) ? 0xffffffffu
+                                                 : (((1u << (a1 - a0 + 1)) - 1u) << a0));
+          }
+        }
+        if (!C::BAND && mrow && j + 1 < nb && j + 1 >= sb) {
+          nw2 = mask_words(blk1);
+          if (j + 2 < nb) blk1 = kb.at(j + 2 - sb);
+        }
+        if (!warp_wait(&s_full[gg & 1], (gg >> 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t s_col = t_lane + (gg & 1) * C::S_COLS + 64 * half;
+        // This half of the row in one TMEM round trip, kept in registers; unselected keys
+        // become -inf there, once.
+        uint32_t r[64];
+        tmem_ld32(s_col + 0, *reinterpret_cast<uint32_t(*)[32]>(r + 0));
+        tmem_ld32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (!(bits[c] & (1u << e))) r[c * 32 + e] = __float_as_uint(ninf);
+        const unsigned long long scale2 = pack2(a.qk_scale, a.qk_scale);
+        unsigned long long rs2 = pack2(0.f, 0.f);  // row sum, two partial sums
+        // 16 keys per chunk: P = exp2(scale*s - m) (0 for unselected keys), split into bf16
+        // P_hi + P_lo (P_lo = bf16(p - P_hi) keeps ~2^-17 relative precision), written over
+        // the chunk's own 16 S columns; mx collects the raw maximum on the way.
+        auto chunk = [&](int kk, unsigned long long nm2, float& mx) {
+          uint32_t ph[8], pl[8];
+#pragma unroll
+          for (int e2 = 0; e2 < 8; ++e2) {
+            const int e = 2 * e2;
+            const float x0 = __uint_as_float(r[16 * kk + e]);
+            const float x1 = __uint_as_float(r[16 * kk + e + 1]);
+            mx = max3(mx, x0, x1);
+            float y0, y1;
+            unpack2(fma2(pack2(x0, x1), scale2, nm2), y0, y1);  // scale*s - m, two keys
+            const float p0 = ex2_ftz(y0), p1 = ex2_ftz(y1);
+            const unsigned long long p2 = pack2(p0, p1);
+            rs2 = add2(rs2, p2);
+            const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+            const uint32_t hb = *reinterpret_cast<const uint32_t*>(&h2);
+            // P_lo = bf16(p - float(P_hi)), the P_hi pair widened by bit moves
+            float d0, d1;
+            unpack2(sub2(p2, pack2(__uint_as_float(hb << 16), __uint_as_float(hb & 0xffff0000u))),
+                    d0, d1);
+            const __nv_bfloat162 l2 = __floats2bfloat162_rn(d0, d1);
+            ph[e2] = hb;
+            pl[e2] = *reinterpret_cast<const uint32_t*>(&l2);
+          }
+          tmem_st8(s_col + kk * 16, ph);
+          tmem_st8(s_col + kk * 16 + 8, pl);
+        };
+        // One pass when every row of the warp already has a running max: P against it at once,
+        // this half's block max taken on the way.  Only a row max above the running one by
+        // more than 2^8 (rare after an item's first block) makes the block run again with the
+        // raised max, as does a first block, whose max is taken first.  Both give the same P
+        // for a row whose max stays.
+        float mloc = ninf;
+        const bool one_pass = __all_sync(0xffffffffu, m_used != ninf);
+        if (one_pass) {
+          const unsigned long long nm2 = pack2(-m_used, -m_used);
+          float mx[2] = {ninf, ninf};  // two chains
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) chunk(kk, nm2, mx[kk & 1]);
+          mloc = fmaxf(mx[0], mx[1]);
+        } else {
+          float mx[4] = {ninf, ninf, ninf, ninf};
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int e = 0; e < 16; e += 2)
+              mx[c] = max3(mx[c], __uint_as_float(r[c * 16 + e]), __uint_as_float(r[c * 16 + e + 1]));
+          mloc = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        }
+        // the row's block max: both halves' maxima, exchanged (double-buffered by block parity)
+        float* xb = xch + (gg & 1) * (2 * kBlk);
+        xb[half * kBlk + row] = mloc;
+        uint64_t* xq = &xbar[quad * 2 + (gg & 1)];
+        mbar_arrive(xq);
+        if (!warp_wait(xq, (gg >> 1) & 1)) { ok = false; break; }
+        const float mraw = fmaxf(mloc, xb[(half ^ 1) * kBlk + row]);
+        bool again = !one_pass || __any_sync(0xffffffffu, mraw * a.qk_scale > m_used + kRescaleLog2);
+        if (again && one_pass) {
+          tmem_wait_st();  // the second pass writes the same columns
+          rs2 = pack2(0.f, 0.f);
+        }
+        // a raised max rescales l now and this half of O (the item's earlier blocks) after P
+        // is written, once their P V landed -- before P_j is published, so P_j V never meets
+        // an unscaled O
+        float alpha = 1.f;
+        bool rescale_o = false, need = false;
+        if (again) {
+          const float mb = mraw * a.qk_scale;
+          need = mb > m_used + kRescaleLog2;
+          if (__any_sync(0xffffffffu, need)) {
+            // whether the row has keys so far is the shared max's business, not this half's
+            // sum: a half without keys yet still scales O, which the other half's keys filled
+            const bool had = m_used != ninf;
+            const float m_new = need ? mb : m_used;
+            alpha = had ? exp2f(m_used - m_new) : 0.f;
+            rescale_o = j >= 1 && __any_sync(0xffffffffu, need && had);
+            if (need) {
+              l *= alpha;
+              m_used = m_new;
+            }
+          }
+          const float msub = m_used == ninf ? 0.f : m_used;
+          const unsigned long long nm2 = pack2(-msub, -msub);
+          float mx = ninf;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) chunk(kk, nm2, mx);
+        }
+        {
+          float r0, r1;
+          unpack2(rs2, r0, r1);
+          l += r0 + r1;
+        }
+        if (rescale_o) {
+          const uint32_t gp = gg - 1;  // the previous block's P V wrote O
+          if (!warp_wait(&pv_done[gp & 1], (gp >> 1) & 1)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < C::DV / 32; ++c) {
+            uint32_t o[16];
+            const uint32_t oc = t_lane + C::O_COL + half * (C::DV / 2) + c * 16;
+            tmem_ld16(oc, o);
+            tmem_wait_ld();
+            if (need) {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            }
+            tmem_st16(oc, o);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[gg & 1]);
+      }
+      if (!ok) break;
+      // Band items are a few key blocks long and their output epilogue is on the path to
+      // the next item's first P V: the two halves normalise and store it themselves, each
+      // half of the columns (the epilogue warps stay idle).
+      const uint32_t gl = g + nb - 1;  // the last block's P V completes O
+      if (!warp_wait(&pv_done[gl & 1], (gl >> 1) & 1)) { ok = false; break; }
+      float* mlb = ml + (ni & 1) * (2 * kBlk * 2);
+      mlb[(half * kBlk + row) * 2 + 1] = l;
+      mbar_arrive(&ml_full[0]);
+      if (!warp_wait(&ml_full[0], ni & 1)) { ok = false; break; }
+      tc_fence_after();
+      const float L = mlb[(0 * kBlk + row) * 2 + 1] + mlb[(1 * kBlk + row) * 2 + 1];
+      float f = L > 0.f ? 1.0f / L : 0.f;
+      if (a.gate && row_ok)
+        f *= gate_act(__bfloat162float(static_cast<const __nv_bfloat16*>(
+                          a.gate)[((size_t)it.b * a.S + s) * a.H + it.h]),
+                      a.gate_mode);
+      __nv_bfloat16* orow = a.out + (((size_t)it.b * a.S + s) * a.H + it.h) * C::DV;
+      // this half writes output columns [half*DV/2, (half+1)*DV/2)
+#pragma unroll 1
+      for (int c = 0; c < C::DV / 64; ++c) {
+        const int col = half * (C::DV / 2) + c * 32;
+        uint32_t r0[32];
+        tmem_ld32(t_lane + C::O_COL + col, r0);
+        tmem_wait_ld();
+        if (row_ok) {
+          uint4 v4[4];
+          uint32_t* vw = reinterpret_cast<uint32_t*>(v4);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            // a row without keys (l = 0) may hold stale values: select, never multiply
+            const float y0 = L > 0.f ? __uint_as_float(r0[2 * e]) * f : 0.f;
+            const float y1 = L > 0.f ? __uint_as_float(r0[2 * e + 1]) * f : 0.f;
+            const __nv_bfloat162 h2 = __floats2bfloat162_rn(y0, y1);
+            vw[e] = *reinterpret_cast<const uint32_t*>(&h2);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(orow + col);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dst[e] = v4[e];
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(o_empty);
+      g += nb;
+    }
+    } else {
     // ------------------------------------------------------------------ softmax
     // Group e (warps 4e..4e+3) owns the key blocks of parity e and accumulator O_e; thread =
     // query row (TMEM lane).  At the end of an item each group leaves its (m, l) in shared
@@ -578,79 +838,21 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         if (lane == 0) mbar_arrive(&p_full[gg & 1]);
       }
       if (!ok) break;
-      if constexpr (!C::BAND) {
-        // hand this group's (m, l) to the epilogue warps; buffer ni & 1 was last read for
-        // item ni - 2 (a group without blocks in an item must not run further ahead)
-        const int mbuf = (int)(ni & 1);
-        if (ni >= 2 && !warp_wait(&ml_empty[mbuf], ((ni >> 1) - 1) & 1)) { ok = false; break; }
-        float* mlb = ml + mbuf * (2 * kBlk * 2);
-        mlb[(grp * kBlk + row) * 2 + 0] = m_used;
-        mlb[(grp * kBlk + row) * 2 + 1] = l;
-        mbar_arrive(&ml_full[mbuf]);
-      } else {
-        // Band items are a few key blocks long and their output epilogue is on the path to
-        // the next item's first P V: the two groups merge and store it themselves, each
-        // half of the columns (the epilogue warps stay idle).
-        const int jlast = ((nb - 1 - jfirst) >= 0) ? jfirst + ((nb - 1 - jfirst) & ~1) : -1;
-        if (jlast >= 0) {
-          const uint32_t gl = g + jlast;
-          if (!warp_wait(&pv_done[gl & 1], (gl >> 1) & 1)) { ok = false; break; }
-        }
-        float* mlb = ml + (ni & 1) * (2 * kBlk * 2);
-        mlb[(grp * kBlk + row) * 2 + 0] = m_used;
-        mlb[(grp * kBlk + row) * 2 + 1] = l;
-        mbar_arrive(&ml_full[0]);
-        if (!warp_wait(&ml_full[0], ni & 1)) { ok = false; break; }
-        tc_fence_after();
-        const float m0 = mlb[(0 * kBlk + row) * 2], l0 = mlb[(0 * kBlk + row) * 2 + 1];
-        const float m1 = mlb[(1 * kBlk + row) * 2], l1 = mlb[(1 * kBlk + row) * 2 + 1];
-        const float M = fmaxf(m0, m1);
-        const float a0 = l0 > 0.f ? exp2f(m0 - M) : 0.f;
-        const float a1 = l1 > 0.f ? exp2f(m1 - M) : 0.f;
-        const float L = l0 * a0 + l1 * a1;
-        float f = L > 0.f ? 1.0f / L : 0.f;
-        if (a.gate && row_ok)
-          f *= gate_act(__bfloat162float(static_cast<const __nv_bfloat16*>(
-                            a.gate)[((size_t)it.b * a.S + s) * a.H + it.h]),
-                        a.gate_mode);
-        const float w0 = a0 * f, w1 = a1 * f;
-        __nv_bfloat16* orow = a.out + (((size_t)it.b * a.S + s) * a.H + it.h) * C::DV;
-        // this group writes output columns [grp*DV/2, (grp+1)*DV/2)
-#pragma unroll 1
-        for (int c = 0; c < C::DV / 64; ++c) {
-          const int col = grp * (C::DV / 2) + c * 32;
-          uint32_t r0[32], r1[32];
-          tmem_ld32(t_lane + C::O_COL + col, r0);
-          tmem_ld32(t_lane + C::O_COL + C::DV + col, r1);
-          tmem_wait_ld();
-          if (row_ok) {
-            uint4 v4[4];
-            uint32_t* vw = reinterpret_cast<uint32_t*>(v4);
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              // an O buffer with no weight (l = 0) may hold stale values: select, never multiply
-              const float y0 = (a0 > 0.f ? __uint_as_float(r0[2 * e]) * w0 : 0.f) +
-                               (a1 > 0.f ? __uint_as_float(r1[2 * e]) * w1 : 0.f);
-              const float y1 = (a0 > 0.f ? __uint_as_float(r0[2 * e + 1]) * w0 : 0.f) +
-                               (a1 > 0.f ? __uint_as_float(r1[2 * e + 1]) * w1 : 0.f);
-              const __nv_bfloat162 h2 = __floats2bfloat162_rn(y0, y1);
-              vw[e] = *reinterpret_cast<const uint32_t*>(&h2);
-            }
-            uint4* dst = reinterpret_cast<uint4*>(orow + col);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) dst[e] = v4[e];
-          }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(o_empty);
-      }
+      // hand this group's (m, l) to the epilogue warps; buffer ni & 1 was last read for
+      // item ni - 2 (a group without blocks in an item must not run further ahead)
+      const int mbuf = (int)(ni & 1);
+      if (ni >= 2 && !warp_wait(&ml_empty[mbuf], ((ni >> 1) - 1) & 1)) { ok = false; break; }
+      float* mlb = ml + mbuf * (2 * kBlk * 2);
+      mlb[(grp * kBlk + row) * 2 + 0] = m_used;
+      mlb[(grp * kBlk + row) * 2 + 1] = l;
+      mbar_arrive(&ml_full[mbuf]);
       g += nb;
+    }
     }
   } else {
     // every warpgroup takes part in the register split (the softmax's setmaxnreg.inc waits
     // for the registers the others give back), in band mode too, where these warps idle
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsEpi));
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_EPI));
     if constexpr (!C::BAND) {
     // ------------------------------------------------------------------ output epilogue
     // Thread = query row (TMEM lane).  Per item: wait for the last P V of each group and for
@@ -895,7 +1097,7 @@ cudaError_t launch_fa(const AttnProblem& p, const uint32_t* mask, int mask_strid
     cudaFuncAttributes fa{};
     return cudaFuncGetAttributes(&fa, kern) == cudaSuccess ? fa.numRegs : 0;
   }();
-  if (launch_regs * C::THREADS < 2 * 128 * kRegsSoft + 128 * kRegsCtl + 128 * kRegsEpi)
+  if (launch_regs * C::THREADS < 2 * 128 * C::REGS_SOFT + 128 * C::REGS_CTL + 128 * C::REGS_EPI)
     return cudaErrorInvalidConfiguration;
   kern<<<grid, C::THREADS, C::SMEM, st>>>(qm, km, vm, skm, svm, a);
   return cudaGetLastError();
