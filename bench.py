@@ -45,10 +45,10 @@ F32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # DRAM traffic per launch from committed ncu captures: (kernel, config) -> (bytes,
 # sha256 of the kernel source when captured).  Reported as null when the source changed.
 NCU_TRAFFIC = {
-    # masked_attn_tc_kernel, c5 full size (the DSA layer): 18.395 GB read + 0.530 GB written
-    ("masked_attn", "c5"): (18925201408, "5066fdaaf91c1115"),
-    # masked_attn_tc_kernel, c2 full size: 64.31 MB read + 3.96 MB written
-    ("masked_attn", "c2"): (68279552, "5066fdaaf91c1115"),
+    # masked_attn_tc_kernel, c5 full size (the DSA layer): 15.426 GB read + 0.532 GB written
+    ("masked_attn", "c5"): (15957929728, "ddd03e9b88d66548"),
+    # masked_attn_tc_kernel, c2 full size: 64.40 MB read + 3.63 MB written
+    ("masked_attn", "c2"): (68023808, "ddd03e9b88d66548"),
     # gather_attn_kernel, c4: captured at B = 32 (same per-row work: 9 splits x 228 keys),
     # 1.3429 GB read + 5.37 MB written, scaled by the rows (x2) to the full B = 64 launch
     ("gather_attn", "c4"): (2696538112, "8652b3612fcab04a"),

@@ -432,19 +432,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       const int s = it.qb * kBlk + row;
       const int spos = s + a.q_off;
       const bool row_ok = s < a.S;
-      const uint32_t* mrow =
-          (!C::BAND && row_ok) ? a.mask + ((size_t)it.b * a.S + s) * a.mask_stride : nullptr;
       float m_used = ninf, l = 0.f;
-      // this half's 2 selection words of key block `blk`
-      auto mask_words = [&](int blk) {
-        return __ldg(reinterpret_cast<const uint2*>(mrow + ((blk * kBlk) >> 5) + 2 * half));
-      };
-      // The words of the next block are fetched one step ahead, and the index of the key
-      // block after it (from the block list) one step before that, so neither load stalls
-      // the chain from S to P.
-      uint2 nw2 = make_uint2(0u, 0u);
-      if (mrow && 0 < nb && 0 >= sb) nw2 = mask_words(kb.at(0));
-      int blk1 = (mrow && 1 < nb && 1 >= sb) ? kb.at(1 - sb) : 0;
       for (int j = 0; j < nb; ++j) {
         const uint32_t gg = g + j;
         const int t0 = (j0 + j - sb) * kBlk + 64 * half;  // this half's first key
@@ -455,8 +443,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             const int n = a.nsink - 64 * half - 32 * w;
             bits[w] = n >= 32 ? 0xffffffffu : (n > 0 ? (1u << n) - 1u : 0u);
           }
-        } else if (!C::BAND) {
-          bits[0] = nw2.x; bits[1] = nw2.y;
         } else if (row_ok) {
           // band: spos - window < t <= spos, t < T
           const int lo = max(spos - a.window + 1, 0) - t0, hi = min(spos, a.T - 1) - t0;
@@ -467,10 +453,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                               : ((a1 - a0 == 31) ? 0xffffffffu
                                                  : (((1u << (a1 - a0 + 1)) - 1u) << a0));
           }
-        }
-        if (!C::BAND && mrow && j + 1 < nb && j + 1 >= sb) {
-          nw2 = mask_words(blk1);
-          if (j + 2 < nb) blk1 = kb.at(j + 2 - sb);
         }
         if (!warp_wait(&s_full[gg & 1], (gg >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
