@@ -440,6 +440,16 @@ const char* dsa_version(void);
  * the device is usable as before.  Returns DSA_OK. */
 dsa_status dsa_test_arm_wait_timeout(void);
 
+/* Testing aid for the top-k (host code, no device needed).  dsa_topk ranks scores by their
+ * order-preserving 32-bit key: the float's bits with the sign bit set for v >= +0.0 (-0.0
+ * counts as +0.0), every bit flipped for v < 0.  This returns the smallest float whose key has
+ * its top 12 bits at or above b, for b in 0..4096 -- the host build of the bound dsa_topk's
+ * second read compares the scores against, so that (key(v) >> 20) >= b exactly when
+ * v >= dsa_test_topk_bucket_floor(b), for every non-NaN v.  Buckets 0..7 hold only NaN images
+ * and -inf, whose bound is -inf; a bucket past the one of +inf gives NaN, which no comparison
+ * passes. */
+float dsa_test_topk_bucket_floor(unsigned b);
+
 #ifdef __cplusplus
 } /* extern "C" */
 #endif

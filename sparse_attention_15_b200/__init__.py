@@ -20,7 +20,7 @@ __all__ = [
     "dsa_sparse_attn_algo", "dsa_forward",
     "dsa_forward_workspace_bytes",
     "dsa_window_attn", "dsa_sparse_attn_noalloc", "dsa_device_status", "dsa_version",
-    "dsa_test_arm_wait_timeout", "LIB_PATH",
+    "dsa_test_arm_wait_timeout", "dsa_test_topk_bucket_floor", "LIB_PATH",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdsa.so")
@@ -100,6 +100,7 @@ _SIGNATURES = {
     "dsa_device_status": (_I, [_I]),
     "dsa_version": (ctypes.c_char_p, []),
     "dsa_test_arm_wait_timeout": (_I, []),
+    "dsa_test_topk_bucket_floor": (ctypes.c_float, [ctypes.c_uint]),
 }
 
 
@@ -163,6 +164,11 @@ def dsa_test_arm_wait_timeout() -> None:
     """Testing aid: the next gather-attention launch runs one bounded wait out on purpose
     (it records DSA_ERR_TIMEOUT; its output is undefined).  One-shot."""
     _check(lib().dsa_test_arm_wait_timeout())
+
+
+def dsa_test_topk_bucket_floor(b: int) -> float:
+    """Testing aid: the top-k's float bound of 12-bit key bucket b (host code)."""
+    return float(lib().dsa_test_topk_bucket_floor(b))
 
 
 def dsa_index_scores(q_idx, k_idx, w, scale, relu="none", scores=None, stream=None):

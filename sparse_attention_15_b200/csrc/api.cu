@@ -337,6 +337,8 @@ const char* dsa_last_error(void) { return g_last_error.c_str(); }
 
 const char* dsa_version(void) { return "dsa-b200 0.2.0 sm_100a"; }
 
+float dsa_test_topk_bucket_floor(unsigned b) { return dsa::topk_bucket_floor(b); }
+
 dsa_status dsa_test_arm_wait_timeout(void) {
   dsa::arm_gather_skip_copy();
   return DSA_OK;

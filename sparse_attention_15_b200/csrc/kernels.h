@@ -64,6 +64,9 @@ cudaError_t launch_hadamard(int dtype, const void* x, void* out, long long rows,
 // Per-row top-k (radix select + ordered compaction).  `mask` (optional) receives the
 // selection bitmask, one bit per key, rows of `mask_stride` 32-bit words
 // (mask_stride >= ceil(T/32); words past the row's keys are zero).
+// The lower bound of bucket b of the top-k's 12-bit key prefix as a float (the host build of
+// the function its second read compares scores against; testing aid).
+float topk_bucket_floor(unsigned b);
 cudaError_t launch_topk(const float* scores, int B, int S, int T, int K, int q_off,
                         int32_t* idx, uint32_t* mask, int mask_stride, cudaStream_t st,
                         const int* run_if = nullptr);

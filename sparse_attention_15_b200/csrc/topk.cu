@@ -15,6 +15,8 @@
 // shared-memory atomics.  The compaction is a block-wide ballot/popc scan in index order, so
 // the output is deterministic and needs no sort.  The same ballots give the selection
 // bitmask (one bit per key) for the masked-tile attention path.
+#include <cstring>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -402,13 +404,18 @@ __device__ __forceinline__ void load_vals(const float* __restrict__ sc, int n, i
 // Buckets 0..7 hold only NaN images and, at the top of bucket 7, -inf; bucket 8 starts at
 // -FLT_MAX; a bucket past the one of +inf has no float (NaN: no comparison passes).  -0.0 and
 // +0.0 share a key and compare equal as floats, so the two tests agree on them as well.
-__device__ __forceinline__ float bucket_floor(uint32_t b) {
-  if (b >= 4096u) return __uint_as_float(0x7fffffffu);
+__host__ __device__ __forceinline__ float float_of_bits(uint32_t u) {
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return f;
+}
+__host__ __device__ __forceinline__ float bucket_floor(uint32_t b) {
+  if (b >= 4096u) return float_of_bits(0x7fffffffu);
   const uint32_t k = b << 20;
-  if (k < 0x00800000u) return __uint_as_float(0xff800000u);       // -inf
-  if (k < 0x80000000u) return __uint_as_float(~k);                // a negative float
+  if (k < 0x00800000u) return float_of_bits(0xff800000u);         // -inf
+  if (k < 0x80000000u) return float_of_bits(~k);                  // a negative float
   const uint32_t u = k ^ 0x80000000u;                             // +0.0 and up
-  return u <= 0x7f800000u ? __uint_as_float(u) : __uint_as_float(0x7fffffffu);
+  return u <= 0x7f800000u ? float_of_bits(u) : float_of_bits(0x7fffffffu);
 }
 
 // Read 2's vote over one batch of U scores per thread (load_vals layout): slot j of the warp
@@ -1105,6 +1112,8 @@ cudaError_t launch_topk_candidates(const uint2* cand, const int* cand_cnt, int c
       cand, cand_cnt, cap, S, T, K, q_off, idx, mask, mask_stride, fail);
   return cudaGetLastError();
 }
+
+float topk_bucket_floor(unsigned b) { return bucket_floor(b); }
 
 cudaError_t launch_topk(const float* scores, int B, int S, int T, int K, int q_off,
                         int32_t* idx, uint32_t* mask, int mask_stride, cudaStream_t st,
