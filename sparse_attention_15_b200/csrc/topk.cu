@@ -265,10 +265,10 @@ __global__ void __launch_bounds__(NT) topk_rows_kernel(const float* __restrict__
 // bounds and one warp vote per 32-key word.  The candidates (a few percent of the keys) are
 // then listed in shared memory as (key, position) from the bitmap, their scores re-read
 // from L2.  On long rows an exact 12-bit histogram of the candidates alone then gives b1;
-// if the sampled window missed the K-th key, read 1 is redone exactly.  Either way b1 and `need` (keys of b1 still to take) are exact.  The low
-// 20 bits are resolved by two 10-bit histogram passes over the candidate list (in shared
-// memory; only a list that overflowed is re-read from L2 through the bitmap), giving the
-// exact threshold key tau.  Candidates above tau join SELECTED; candidates equal to tau are
+// if the sampled window missed the K-th key, read 1 is redone exactly.  Either way b1 and
+// `need` (keys of b1 still to take) are exact.  The low 20 bits are resolved by two 10-bit
+// histogram passes over the candidate list (in shared memory; only a list that overflowed is
+// re-read from L2 through the bitmap), giving the exact threshold key tau.  Candidates above tau join SELECTED; candidates equal to tau are
 // ranked by index with a prefix scan of their bitmap and the first `need` join SELECTED.
 // An ordered scan of SELECTED writes the indices (ascending) and the bitmap itself is the
 // selection mask row.
